@@ -1,0 +1,25 @@
+"""CPU oracle for the MXFP8 grouped expert MLP -- TEST INFRASTRUCTURE ONLY.
+
+A plain, slow, fp64 restatement of what the hot path computes, used to check the
+CUDA library. Only the test-suite, ``__graft_entry__.smoke()`` and the benchmark's
+``cpu_baseline`` / ``--impl reference`` legs may import it; the product package
+never does, and the oracle never imports the product package. Both sides share only
+the seeded input generators in ``moe_workloads``.
+
+Sources (three short web pages on one NVIDIA tutorial; no code, no formulas):
+  * "MoE-Training für biologische Grundmodelle optimieren" (hyper.ai, German)
+  * "NVIDIA apresenta técnicas para tornar mais eficiente o treinamento de modelos
+    biológicos baseados em arquitetura MoE" (conexaotc.com.br, Portuguese)
+  * "NVIDIA optimise l'entraînement MoE des modèles biologiques" (hyper.ai, French)
+They name the steps (grouping tokens by per-expert counts, MXFP8 with one scale per
+32-value block, a fused gate-up + SwiGLU + routing-scale kernel, forward and backward)
+but fix no element format, rounding or layout; every such choice below is a stated
+reading, and each function's docstring says which.
+
+Pins (tests marked ``not gpu``): exhaustive E4M3 round trip, hand-built
+quantisation blocks, brute-force permutation, per-token loop == grouped forward,
+dense-MLP reduction, SwiGLU closed forms, finite differences of the backward.
+Parity unpinned: the end-to-end numeric level against the pages (they print no
+accuracy, loss or worked example).
+"""
+from . import mxfp8, moe  # noqa: F401

@@ -1,0 +1,267 @@
+"""Grouped expert MLP, forward and backward, fp64 (oracle; test infrastructure only).
+
+Follows, in the pages' order, the steps the three pages name:
+  1. tokens are grouped by expert using per-expert token counts ("MoE-Training für
+     biologische Grundmodelle optimieren", hyper.ai/de, GroupedLinear passage);
+  2. activations and weights are quantised to MXFP8 (same page, MXFP8 passage;
+     "NVIDIA optimise l'entraînement MoE des modèles biologiques", hyper.ai/fr);
+  3. the gate-up projection, the ScaledSwiGLU activation and the routing-weight
+     scaling form one fused step, with a matching backward (hyper.ai/de, GroupedMLP
+     passage; "NVIDIA apresenta técnicas ... arquitetura MoE", conexaotc.com.br,
+     third optimisation);
+  4. the down projection and the return to token order (the pages are silent on
+     these; the plain reading: a second expert linear, and a sum over the k routed
+     copies of each token).
+
+Readings where the pages are silent (each is listed in the design notes):
+  * rows are ordered by (expert ascending, token ascending); each expert segment
+    starts at a multiple of ``align`` rows, pad rows are zero and ignored;
+  * W1 is [E, 2F, H] (nn.Linear out x in) with gate rows first, up rows second;
+    W2 is [E, H, F]; no biases;
+  * Z = silu(G) * U * p, p the routed row's probability, applied before the down
+    projection and quantised from its fp64 value;
+  * backward uses the straight-through estimator (every quantiser passes the
+    gradient unchanged) and quantises dY, dGU rowwise and colwise as the consuming
+    GEMMs need; the activations saved for backward are kept in fp64 here.
+Every GEMM is a library matmul over dequantised fp64 operands, one expert at a time.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import mxfp8
+
+ALIGN_ORACLE = 32
+
+
+def _roundup(x, a):
+    return (x + a - 1) // a * a
+
+
+# ----------------------------------------------------------------------------- routing
+
+def route(topk_idx, E, align=ALIGN_ORACLE):
+    """Counting sort of the (token, slot) pairs by expert, stable by token.
+
+    Returns dict with m_splits int64[E], seg_off int64[E+1] (segment e starts at the
+    sum of the earlier segments' counts rounded up to ``align``), row_of_slot
+    int64[T,k], token_of_row int64[Mp] (-1 on pad rows), slot_of_row int64[Mp].
+    Raises ValueError on an expert id out of range or repeated within a token."""
+    idx = np.asarray(topk_idx, dtype=np.int64)
+    T, k = idx.shape
+    if np.any(idx < 0) or np.any(idx >= E):
+        raise ValueError("expert id out of range")
+    for t in range(T):
+        if len(set(idx[t].tolist())) != k:
+            raise ValueError("repeated expert within a token's top-k")
+    tok = np.repeat(np.arange(T), k)
+    slot = np.tile(np.arange(k), T)
+    exp = idx.reshape(-1)
+    order = np.lexsort((tok, exp))            # primary key: expert; secondary: token
+    m_splits = np.bincount(exp, minlength=E).astype(np.int64)
+    seg_off = np.zeros(E + 1, dtype=np.int64)
+    seg_off[1:] = np.cumsum(_roundup(m_splits, align))
+    Mp = int(seg_off[E])
+    row_of_slot = np.zeros((T, k), dtype=np.int64)
+    token_of_row = np.full(Mp, -1, dtype=np.int64)
+    slot_of_row = np.full(Mp, -1, dtype=np.int64)
+    pos = 0
+    for e in range(E):
+        for i in range(m_splits[e]):
+            p = order[pos]
+            pos += 1
+            r = seg_off[e] + i
+            row_of_slot[tok[p], slot[p]] = r
+            token_of_row[r] = tok[p]
+            slot_of_row[r] = slot[p]
+    return dict(m_splits=m_splits, seg_off=seg_off, row_of_slot=row_of_slot,
+                token_of_row=token_of_row, slot_of_row=slot_of_row, Mp=Mp)
+
+
+def permute_rows(x, token_of_row):
+    """Xp[r] = x[token_of_row[r]], zero where token_of_row == -1."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros((len(token_of_row),) + x.shape[1:], dtype=np.float64)
+    live = token_of_row >= 0
+    out[live] = x[token_of_row[live]]
+    return out
+
+
+def unpermute_sum(yp, row_of_slot):
+    """Y[t] = sum over slots j (in order) of Yp[row_of_slot[t, j]]."""
+    yp = np.asarray(yp, dtype=np.float64)
+    T, k = row_of_slot.shape
+    out = np.zeros((T,) + yp.shape[1:], dtype=np.float64)
+    for j in range(k):
+        out += yp[row_of_slot[:, j]]
+    return out
+
+
+# ----------------------------------------------------------------------------- MXFP8 helpers
+
+def quantize_colwise_segments(a, seg_off, m_splits):
+    """Colwise MXFP8 of a permuted [Mp, C] matrix: blocks of 32 rows that start at each
+    expert segment's first row (segments are 32-aligned with zero pad rows), stored
+    transposed -> (codes uint8[C, Mp], scales uint8[C, Mp/32])."""
+    a = np.asarray(a, dtype=np.float64)
+    Mp, C = a.shape
+    codes = np.zeros((C, Mp), dtype=np.uint8)
+    scales = np.zeros((C, Mp // mxfp8.BLOCK), dtype=np.uint8)
+    for e in range(len(m_splits)):
+        s0, s1 = int(seg_off[e]), int(seg_off[e + 1])
+        if s1 == s0:
+            continue
+        assert s0 % mxfp8.BLOCK == 0 and s1 % mxfp8.BLOCK == 0
+        c, s = mxfp8.quantize_colwise_t(a[s0:s1])
+        codes[:, s0:s1] = c
+        scales[:, s0 // mxfp8.BLOCK:s1 // mxfp8.BLOCK] = s
+    return codes, scales
+
+
+def fake_quant_colwise_segments(a, seg_off, m_splits):
+    c, s = quantize_colwise_segments(a, seg_off, m_splits)
+    return mxfp8.dequantize_rowwise(c, s).T
+
+
+def _fq_row(a, quant):
+    return mxfp8.fake_quant_rowwise(a) if quant else np.asarray(a, dtype=np.float64)
+
+
+def _fq_col(a, quant):
+    return mxfp8.fake_quant_colwise(a) if quant else np.asarray(a, dtype=np.float64)
+
+
+def _fq_col_seg(a, r, quant):
+    if not quant:
+        return np.asarray(a, dtype=np.float64)
+    return fake_quant_colwise_segments(a, r["seg_off"], r["m_splits"])
+
+
+# ----------------------------------------------------------------------------- grouped GEMMs
+
+def grouped_gemm(A, B, seg_off):
+    """C[seg_e] = A[seg_e] @ B[e]^T for each expert e (A [Mp, K], B [E, N, K]), fp64;
+    rows outside every segment are zero."""
+    A = np.asarray(A, dtype=np.float64)
+    E, N, _ = B.shape
+    C = np.zeros((A.shape[0], N), dtype=np.float64)
+    for e in range(E):
+        s0, s1 = int(seg_off[e]), int(seg_off[e + 1])
+        if s1 > s0:
+            C[s0:s1] = A[s0:s1] @ np.asarray(B[e], dtype=np.float64).T
+    return C
+
+
+def grouped_gemm_wgrad(At, Bt, seg_off):
+    """C[e] = At[:, seg_e] @ Bt[:, seg_e]^T (At [N, Mp], Bt [K', Mp]) -> [E, N, K'];
+    an expert with no rows gets zeros."""
+    E = len(seg_off) - 1
+    At = np.asarray(At, dtype=np.float64)
+    Bt = np.asarray(Bt, dtype=np.float64)
+    C = np.zeros((E, At.shape[0], Bt.shape[0]), dtype=np.float64)
+    for e in range(E):
+        s0, s1 = int(seg_off[e]), int(seg_off[e + 1])
+        if s1 > s0:
+            C[e] = At[:, s0:s1] @ Bt[:, s0:s1].T
+    return C
+
+
+# ----------------------------------------------------------------------------- SwiGLU
+
+def sigmoid(x):
+    x = np.asarray(x, dtype=np.float64)
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def silu(x):
+    """silu(g) = g / (1 + e^-g)."""
+    x = np.asarray(x, dtype=np.float64)
+    return x * sigmoid(x)
+
+
+def dsilu(x):
+    """d silu / dg = s(g) * (1 + g * (1 - s(g))), s the logistic function."""
+    s = sigmoid(x)
+    return s * (1.0 + x * (1.0 - s))
+
+
+# ----------------------------------------------------------------------------- MLP
+
+def mlp_fwd(x, topk_idx, probs, W1, W2, quant=True, align=ALIGN_ORACLE):
+    """Forward of the grouped expert MLP. Returns (y fp64[T,H], saved dict)."""
+    x = np.asarray(x, dtype=np.float64)
+    probs = np.asarray(probs, dtype=np.float64)
+    E, F2, H = W1.shape
+    F = F2 // 2
+    r = route(topk_idx, E, align)
+    Xp = permute_rows(x, r["token_of_row"])
+    live = r["token_of_row"] >= 0
+    p_row = np.zeros(r["Mp"], dtype=np.float64)
+    p_row[live] = probs[r["token_of_row"][live], r["slot_of_row"][live]]
+    Xq = _fq_row(Xp, quant)                                   # blocks along H
+    W1q = np.stack([_fq_row(W1[e], quant) for e in range(E)])  # blocks along H
+    GU = grouped_gemm(Xq, W1q, r["seg_off"])
+    G, U = GU[:, :F], GU[:, F:]
+    Z = silu(G) * U * p_row[:, None]
+    Zq = _fq_row(Z, quant)                                    # blocks along F
+    W2q = np.stack([_fq_row(W2[e], quant) for e in range(E)])  # blocks along F
+    Yp = grouped_gemm(Zq, W2q, r["seg_off"])
+    y = unpermute_sum(Yp, r["row_of_slot"])
+    saved = dict(route=r, Xp=Xp, p_row=p_row, G=G, U=U, Z=Z, Yp=Yp)
+    return y, saved
+
+
+def mlp_bwd(dy, saved, probs, W1, W2, quant=True):
+    """Backward (straight-through estimator for every quantiser).
+    Returns dict dx fp64[T,H], dW1 fp64[E,2F,H], dW2 fp64[E,H,F], dprobs fp64[T,k]."""
+    r = saved["route"]
+    E, F2, H = W1.shape
+    F = F2 // 2
+    G, U, Z, p_row = saved["G"], saved["U"], saved["Z"], saved["p_row"]
+    dYp = permute_rows(dy, r["token_of_row"])
+    dYq_row = _fq_row(dYp, quant)                         # blocks along H (fc2 dgrad)
+    dYq_col = _fq_col_seg(dYp, r, quant)                  # blocks along M (fc2 wgrad)
+    W2q_col = np.stack([_fq_col(W2[e], quant) for e in range(E)])   # [H, F], blocks along H
+    # fc2 dgrad: dZ = dYp . W2  (contract over H)
+    dZ = grouped_gemm(dYq_row, np.transpose(W2q_col, (0, 2, 1)), r["seg_off"])
+    A = silu(G) * U
+    dprob_row = np.sum(dZ * A, axis=1)
+    dA = dZ * p_row[:, None]
+    dG = dA * U * dsilu(G)
+    dU = dA * silu(G)
+    dGU = np.concatenate([dG, dU], axis=1)
+    dGUq_row = _fq_row(dGU, quant)                        # blocks along 2F (fc1 dgrad)
+    dGUq_col = _fq_col_seg(dGU, r, quant)                 # blocks along M (fc1 wgrad)
+    Zq_col = _fq_col_seg(Z, r, quant)
+    Xq_col = _fq_col_seg(saved["Xp"], r, quant)
+    # fc2 wgrad: dW2[e] = dYp_e^T . Z_e  (contract over the expert's rows)
+    dW2 = grouped_gemm_wgrad(dYq_col.T, Zq_col.T, r["seg_off"])
+    # fc1 dgrad: dXp = dGU . W1  (contract over 2F)
+    W1q_col = np.stack([_fq_col(W1[e], quant) for e in range(E)])   # [2F, H], blocks along 2F
+    dXp = grouped_gemm(dGUq_row, np.transpose(W1q_col, (0, 2, 1)), r["seg_off"])
+    # fc1 wgrad: dW1[e] = dGU_e^T . Xp_e
+    dW1 = grouped_gemm_wgrad(dGUq_col.T, Xq_col.T, r["seg_off"])
+    dx = unpermute_sum(dXp, r["row_of_slot"])
+    dprobs = dprob_row[r["row_of_slot"]]
+    return dict(dx=dx, dW1=dW1, dW2=dW2, dprobs=dprobs, dGU=dGU, dZ=dZ, dXp=dXp)
+
+
+def mlp_per_token(x, topk_idx, probs, W1, W2, quant=True):
+    """Forward written token by token: y[t] = sum_j W2q[e] . q(silu(g) * u * p) with
+    g, u from W1q[e] . q(x[t]), e = topk_idx[t, j]. No grouping, no permutation."""
+    x = np.asarray(x, dtype=np.float64)
+    E, F2, H = W1.shape
+    F = F2 // 2
+    W1q = [_fq_row(W1[e], quant) for e in range(E)]
+    W2q = [_fq_row(W2[e], quant) for e in range(E)]
+    T, k = topk_idx.shape
+    y = np.zeros((T, H), dtype=np.float64)
+    for t in range(T):
+        xq = _fq_row(x[t:t + 1], quant)[0]
+        for j in range(k):
+            e = int(topk_idx[t, j])
+            gu = W1q[e] @ xq
+            z = silu(gu[:F]) * gu[F:] * float(probs[t, j])
+            zq = _fq_row(z[None, :], quant)[0]
+            y[t] += W2q[e] @ zq
+    return y

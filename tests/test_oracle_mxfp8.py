@@ -1,0 +1,136 @@
+"""Pins for the oracle's MXFP8 codec and block quantiser (CPU only).
+
+The pages fix only "8 bits per value, one scale per block of 32 values"
+("MoE-Training für biologische Grundmodelle optimieren", hyper.ai/de, MXFP8
+passage). E4M3/E8M0 and the scale rule are the OCP MX reading; these tests pin the
+oracle against that format's closed-form facts and hand-derived blocks."""
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import mxfp8
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "mxfp8_blocks.txt")
+
+
+def _parse_value(s):
+    s = s.strip()
+    if "*2^" in s:
+        p, q = s.split("*2^")
+        return float(p) * math.ldexp(1.0, int(q))
+    return float(s)
+
+
+def _golden_blocks():
+    out = []
+    for line in open(GOLDEN):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        name, vals, scale, codes = [f.strip() for f in line.split("|")]
+        v = np.zeros(32)
+        for item in vals.split(","):
+            pos, val = item.split(":")
+            v[int(pos)] = _parse_value(val)
+        exp_codes = {int(p): int(c, 16) for p, c in (it.split(":") for it in codes.split(","))}
+        out.append((name, v, int(scale, 16), exp_codes))
+    return out
+
+
+@pytest.mark.parametrize("name,v,scale,codes", _golden_blocks(), ids=lambda x: x if isinstance(x, str) else "")
+def test_hand_built_blocks(name, v, scale, codes):
+    q, s = mxfp8.quantize_blocks(v[None, :])
+    assert int(s[0]) == scale, name
+    for pos, c in codes.items():
+        assert int(q[0, pos]) == c, (name, pos, hex(int(q[0, pos])), hex(c))
+
+
+def test_decode_closed_form_points():
+    assert mxfp8.e4m3_decode(0x7E) == 448.0
+    assert mxfp8.e4m3_decode(0xFE) == -448.0
+    assert mxfp8.e4m3_decode(0x78) == 256.0
+    assert mxfp8.e4m3_decode(0x38) == 1.0
+    assert mxfp8.e4m3_decode(0x08) == 2.0 ** -6        # smallest normal
+    assert mxfp8.e4m3_decode(0x07) == 7 * 2.0 ** -9    # largest subnormal
+    assert mxfp8.e4m3_decode(0x01) == 2.0 ** -9        # smallest subnormal
+    assert mxfp8.e4m3_decode(0x00) == 0.0
+    assert math.copysign(1.0, mxfp8.e4m3_decode(0x80)) == -1.0
+    assert np.isnan(mxfp8.e4m3_decode(0x7F)) and np.isnan(mxfp8.e4m3_decode(0xFF))
+
+
+def test_decode_monotone_and_count():
+    vals = mxfp8.e4m3_decode(np.arange(0x7F))
+    assert np.all(np.diff(vals) > 0)
+    allv = mxfp8.e4m3_decode(np.arange(256))
+    assert np.sum(np.isfinite(allv)) == 254
+
+
+def test_exhaustive_round_trip():
+    """Every finite code, placed in a block whose amax is 448 (scale exponent 0),
+    re-encodes to itself."""
+    for b in range(256):
+        if b in (0x7F, 0xFF):
+            continue
+        v = np.zeros(32)
+        v[0] = 448.0
+        v[1] = mxfp8.e4m3_decode(b)
+        q, s = mxfp8.quantize_blocks(v[None, :])
+        assert s[0] == 127
+        assert q[0, 1] == b, hex(b)
+
+
+def test_encode_midpoints_round_to_even():
+    """Between every pair of neighbouring codes, the midpoint goes to the even code and
+    points just either side go to the nearer one."""
+    vals = mxfp8.e4m3_decode(np.arange(0x7F))
+    for c in range(0x7E):
+        lo, hi = vals[c], vals[c + 1]
+        mid = 0.5 * (lo + hi)
+        want = c if c % 2 == 0 else c + 1
+        assert mxfp8.e4m3_encode(mid) == want
+        eps = (hi - lo) * 1e-3
+        assert mxfp8.e4m3_encode(mid - eps) == c
+        assert mxfp8.e4m3_encode(mid + eps) == c + 1
+
+
+def test_scale_exponent_rule():
+    for a in [1e-30, 2.0 ** -126, 0.3, 1.0, 1.999, 2.0, 447.0, 448.0, 1e30]:
+        want = max(-127, min(127, math.floor(math.log2(a)) - 8))
+        assert mxfp8.scale_exponent(a) == want
+    assert mxfp8.scale_exponent(0.0) == -127
+    assert mxfp8.scale_exponent(2.0 ** 200) == 127
+
+
+def test_quantisation_error_bound():
+    """Relative error of a dequantised element is at most 2^-4 (half an ulp of a 3-bit
+    mantissa) wherever the scaled value lies in E4M3's normal, unsaturated range."""
+    rng = np.random.default_rng(0)
+    v = rng.standard_normal((500, 32)) * np.exp2(rng.integers(-20, 20, (500, 1)))
+    q, s = mxfp8.quantize_blocks(v)
+    d = mxfp8.dequantize_blocks(q, s)
+    X = s.astype(np.int64) - 127
+    lo = np.exp2(X - 6.0)[:, None]
+    hi = 448.0 * np.exp2(X.astype(float))[:, None]
+    normal = (np.abs(v) >= lo) & (np.abs(v) <= hi)      # not subnormal, not saturated
+    rel = np.abs(d - v)[normal] / np.abs(v)[normal]
+    assert rel.max() <= 2.0 ** -4 + 1e-15
+    # and the block max never exceeds 448 * 2^X
+    assert np.all(np.abs(d) <= 448.0 * np.exp2(X.astype(float))[:, None])
+
+
+def test_rowwise_and_colwise_shapes():
+    rng = np.random.default_rng(1)
+    a = rng.standard_normal((64, 96))
+    c, s = mxfp8.quantize_rowwise(a)
+    assert c.shape == (64, 96) and s.shape == (64, 3)
+    ct, st = mxfp8.quantize_colwise_t(a)
+    assert ct.shape == (96, 64) and st.shape == (96, 2)
+    # colwise of a == rowwise of a^T, block by block
+    np.testing.assert_array_equal(ct, mxfp8.quantize_rowwise(a.T)[0])
+    # each colwise block covers 32 consecutive rows of one column
+    blk = a[32:64, 5]
+    qb, sb = mxfp8.quantize_blocks(blk[None, :])
+    np.testing.assert_array_equal(ct[5, 32:64], qb[0])
+    assert st[5, 1] == sb[0]
