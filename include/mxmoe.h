@@ -1,0 +1,270 @@
+/*
+ * mxmoe.h -- C ABI of the B200 (sm_100a) MXFP8 grouped expert-MLP library.
+ *
+ * What the library computes (sources: three short web pages on one NVIDIA tutorial;
+ * they give no formulas, so the exact conventions below are this library's stated
+ * readings):
+ *   - "MoE-Training für biologische Grundmodelle optimieren" (hyper.ai/de): grouping
+ *     of tokens by per-expert token counts so that all expert GEMMs run in one call
+ *     (GroupedLinear passage); MXFP8 with one scale factor per block of 32 values
+ *     (MXFP8 passage); a fused gate-up / ScaledSwiGLU / routing-scale kernel with a
+ *     matching backward (GroupedMLP passage);
+ *   - "NVIDIA apresenta técnicas para tornar mais eficiente o treinamento de modelos
+ *     biológicos baseados em arquitetura MoE" (conexaotc.com.br): the fused kernel
+ *     covers quantisation, SwiGLU and routing-weight scaling (third optimisation);
+ *   - "NVIDIA optimise l'entraînement MoE des modèles biologiques" (hyper.ai/fr):
+ *     expert GEMMs in one GPU call; MXFP8 halves the footprint; SwiGLU and
+ *     quantisation fused, forward and backward.
+ *
+ * Conventions (all entry points):
+ *   - Every pointer argument named *_dev or documented "device" is CUDA device memory
+ *     owned by the caller; the library never allocates, frees or synchronises, and
+ *     enqueues all work asynchronously on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).
+ *   - Device pointers must be 16-byte aligned; byte sizes documented per argument.
+ *   - Host-detectable errors (bad pointer, shape, size) return a non-zero status and
+ *     enqueue nothing. Errors found on the device (an expert id out of range or
+ *     repeated within a token, a wait that timed out) are recorded in a per-device
+ *     status word read with mxmoe_get_device_status(); kernels never trap.
+ *   - bf16 is IEEE bfloat16 stored as uint16; E4M3 is OCP FP8 E4M3 (bias 7, max 448,
+ *     no infinities); E8M0 is an unsigned power-of-two exponent byte (bias 127).
+ *   - MXFP8 rule (OCP Microscaling v1.0): for a block of 32 values with largest
+ *     magnitude amax, X = clamp(floor(log2(amax)) - 8, -127, 127) (amax == 0 gives
+ *     -127), scale byte = X + 127, element = E4M3(v * 2^-X) rounded to nearest-even
+ *     and saturated to +-448.
+ *   - Routed rows are ordered by (expert ascending, token ascending). Expert e's
+ *     segment of rows starts at seg_off[e], a multiple of 128; its first m_splits[e]
+ *     rows are live, the rest up to seg_off[e+1] are zero pad rows. The buffers of
+ *     permuted rows hold mxmoe_rows_capacity(T, k, E) rows.
+ */
+#ifndef MXMOE_H_
+#define MXMOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t mxmoe_status;
+
+#define MXMOE_OK 0
+#define MXMOE_ERR_INVALID_ARG 1          /* null / misaligned pointer, bad enum, negative size */
+#define MXMOE_ERR_UNSUPPORTED_SHAPE 2    /* shape outside what the kernels handle */
+#define MXMOE_ERR_WORKSPACE_TOO_SMALL 3  /* ws_bytes / saved_bytes / wq_bytes below the query */
+#define MXMOE_ERR_CUDA 4                 /* a CUDA runtime call failed (launch, attribute) */
+#define MXMOE_ERR_DEVICE_TIMEOUT 5       /* device: a bounded wait gave up */
+#define MXMOE_ERR_DEVICE_CHECK 6         /* device: invalid routing input */
+
+/* dtypes */
+#define MXMOE_DTYPE_BF16 0
+#define MXMOE_DTYPE_F32 1
+
+/* scale-factor layouts of an mxmoe_mxfp8 matrix */
+#define MXMOE_SCALE_PLAIN 0 /* row-major [rows][cols/32] */
+#define MXMOE_SCALE_MMA 1   /* rows, cols multiples of 128: [rows/128][cols/128] chunks of 512 bytes;
+                               inside a chunk the scale of (row r, block kb) is at byte
+                               (r%32)*16 + ((r/32)%4)*4 + kb%4 -- the tensor cores' scale-factor order */
+
+/*
+ * One MXFP8 matrix: `rows` x `cols` E4M3 codes, row-major (row stride `cols` bytes),
+ * quantised in blocks of 32 consecutive elements along each row, plus rows*cols/32
+ * E8M0 scale bytes laid out as `scale_layout` says. A "colwise" quantisation of a
+ * source matrix S [R, C] (blocks of 32 consecutive rows of S) is stored transposed:
+ * rows = C, cols = R. Both pointers are device memory owned by the caller.
+ */
+typedef struct mxmoe_mxfp8 {
+  uint8_t* data;
+  uint8_t* scale;
+  int64_t rows;
+  int64_t cols;
+  int32_t scale_layout;
+  int32_t reserved; /* must be 0 */
+} mxmoe_mxfp8;
+
+/* ------------------------------------------------------------------ status / sizes */
+
+/* Human-readable name of a status code (static string; never NULL). */
+const char* mxmoe_status_string(mxmoe_status s);
+
+/* Copies the current device's status word (MXMOE_OK or the first device error since
+ * the last clear) to *out_host and the tag of the site that set it to *where_host
+ * (nullable). Synchronises `stream`. */
+mxmoe_status mxmoe_get_device_status(int32_t* out_host, int32_t* where_host, void* stream);
+
+/* Resets the current device's status word to MXMOE_OK (enqueued on `stream`). */
+mxmoe_status mxmoe_clear_device_status(void* stream);
+
+/* Upper bound on the number of permuted rows (live + pad) for T tokens, top-k and E
+ * experts: roundup(T*k + 127*E, 128). Every [Mp, *] buffer below has this many rows. */
+int64_t mxmoe_rows_capacity(int32_t T, int32_t k, int32_t E);
+
+/* ------------------------------------------------------------------ routing (GroupedLinear input) */
+
+/*
+ * moe_permute -- groups the routed (token, slot) pairs by expert: a counting sort,
+ * stable by token ("MoE-Training für biologische Grundmodelle optimieren", GroupedLinear
+ * passage: the per-expert token counts drive the gather of the expert matrices).
+ *   topk_idx_dev  int32 [T, k]  expert id of each token's k choices; distinct within a
+ *                 token and in [0, E). Violations set MXMOE_ERR_DEVICE_CHECK and the
+ *                 offending pair is dropped.
+ *   probs_dev     float [T, k]  routing probabilities (nullable if prob_of_row_dev is).
+ *   Outputs (device, caller-owned):
+ *   m_splits_dev     int32 [E]     tokens per expert
+ *   seg_off_dev      int32 [E+1]   start row of each expert segment (multiples of 128);
+ *                                  seg_off[E] = Mp, the padded row count
+ *   row_of_slot_dev  int32 [T, k]  permuted row of each (token, slot)
+ *   token_of_row_dev int32 [mxmoe_rows_capacity]  token of each row, -1 on pad rows
+ *                                  (rows >= Mp are left untouched)
+ *   prob_of_row_dev  float [mxmoe_rows_capacity]  probability of each row, 0 on pad rows
+ *                                  (nullable)
+ *   ws_dev / ws_bytes  scratch of at least moe_permute_workspace_size(T, k, E) bytes.
+ * Limits: 1 <= k <= 8, 1 <= E <= 256, T >= 0.
+ */
+mxmoe_status moe_permute(const int32_t* topk_idx_dev, const float* probs_dev, int32_t T, int32_t k, int32_t E,
+                         int32_t* m_splits_dev, int32_t* seg_off_dev, int32_t* row_of_slot_dev,
+                         int32_t* token_of_row_dev, float* prob_of_row_dev, void* ws_dev, size_t ws_bytes,
+                         void* stream);
+size_t moe_permute_workspace_size(int32_t T, int32_t k, int32_t E);
+
+/*
+ * moe_unpermute -- returns routed rows to token order and sums the k copies of each
+ * token: y[t] = sum_{j<k} y_perm[row_of_slot[t, j]], accumulated in fp32 in slot order
+ * and rounded once to bf16 (the pages are silent on the combine; this is the plain
+ * reading). y_perm_dev bf16 [rows, H]; y_dev bf16 [T, H]. H % 8 == 0.
+ */
+mxmoe_status moe_unpermute(const void* y_perm_dev, const int32_t* row_of_slot_dev, int32_t T, int32_t k,
+                           int32_t H, void* y_dev, void* stream);
+
+/* ------------------------------------------------------------------ MXFP8 quantisation */
+
+/*
+ * mxfp8_quantize -- MXFP8 quantisation, rowwise and/or colwise, optionally fused with a
+ * row gather ("MoE-Training für biologische Grundmodelle optimieren", MXFP8 passage:
+ * 8-bit values with one scale per 32-value block; GroupedMLP passage: the conversions
+ * between 16-bit and 8-bit are fused instead of run as separate operations).
+ *   src_dev      [batch, rows, cols] of src_dtype (MXMOE_DTYPE_BF16 or _F32), row-major.
+ *   row_gather_dev  nullable int32 [out_rows]: if given (batch must be 1), output row r
+ *                is src row row_gather[r], or zeros where row_gather[r] < 0.
+ *   nrows_dev    nullable int32 (one value, device): only output rows < *nrows_dev are
+ *                written (e.g. &seg_off[E]); must be a multiple of 128 if given.
+ *   out_rows     rows of each output matrix (== rows when there is no gather).
+ *   out_row      nullable: rowwise result, rows = batch*out_rows, cols = cols.
+ *   out_colT     nullable: colwise result (blocks of 32 consecutive output rows within
+ *                each batch matrix), stored transposed: rows = batch*cols, cols = out_rows;
+ *                batch b's matrix occupies rows [b*cols, (b+1)*cols).
+ * Shapes: cols % 32 == 0, out_rows % 32 == 0 (both % 128 == 0 for MXMOE_SCALE_MMA).
+ */
+mxmoe_status mxfp8_quantize(const void* src_dev, int32_t src_dtype, int64_t batch, int64_t rows, int64_t cols,
+                            const int32_t* row_gather_dev, const int32_t* nrows_dev, int64_t out_rows,
+                            const mxmoe_mxfp8* out_row, const mxmoe_mxfp8* out_colT, void* stream);
+
+/* ------------------------------------------------------------------ grouped GEMMs (GroupedLinear) */
+
+/*
+ * grouped_gemm_mxfp8 -- one launch for all experts ("MoE-Training für biologische
+ * Grundmodelle optimieren", GroupedLinear passage; "NVIDIA optimise l'entraînement MoE
+ * des modèles biologiques", first improvement): for every expert e,
+ *     C[seg_e, :] = dequant(A)[seg_e, :] . dequant(B_e)^T,   seg_e = [seg_off[e], seg_off[e+1])
+ * with fp32 accumulation on the tensor cores.
+ *   A   MXFP8 [rows_cap, K], MXMOE_SCALE_MMA; rows_cap % 128 == 0.
+ *   B   MXFP8 [E*N, K], MXMOE_SCALE_MMA (expert e's rows are [e*N, (e+1)*N)).
+ *   seg_off_dev  int32 [E+1], multiples of 128, read on the device (no host sync).
+ *   C_dev [rows_cap, ldc] of c_dtype (MXMOE_DTYPE_BF16 or _F32); rows >= seg_off[E]
+ *         are not written.
+ * Shapes: N % 256 == 0, K % 128 == 0, ldc >= N, ldc % 8 == 0.
+ */
+mxmoe_status grouped_gemm_mxfp8(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, const int32_t* seg_off_dev,
+                                int32_t E, int64_t N, int64_t K, void* C_dev, int32_t c_dtype, int64_t ldc,
+                                void* stream);
+
+/*
+ * grouped_gemm_mxfp8_wgrad -- weight-gradient form, contracting over each expert's
+ * (ragged) rows: C[e] = dequant(At)[:, seg_e] . dequant(Bt)[:, seg_e]^T, fp32, [E, N, K2].
+ * An expert with no rows gets zeros.
+ *   At  MXFP8 [N, rows_cap] (colwise-transposed activations/gradients), MXMOE_SCALE_MMA.
+ *   Bt  MXFP8 [K2, rows_cap], MXMOE_SCALE_MMA.
+ *   C_dev float [E, N, K2].
+ * Shapes: N % 128 == 0, K2 % 256 == 0.
+ */
+mxmoe_status grouped_gemm_mxfp8_wgrad(const mxmoe_mxfp8* At, const mxmoe_mxfp8* Bt, const int32_t* seg_off_dev,
+                                      int32_t E, float* C_dev, void* stream);
+
+/* ------------------------------------------------------------------ fused grouped MLP (GroupedMLP) */
+
+/*
+ * Quantised weights: one opaque device buffer of mxmoe_weights_size(E, H, F) bytes that
+ * holds four MXFP8 copies (MMA scale layout):
+ *   W1 rowwise  [E*2F, H]  (fc1 forward operand; blocks along H)
+ *   W1 colwise  [E*H, 2F]  (fc1 data-gradient operand; blocks along 2F)
+ *   W2 rowwise  [E*H, F]   (fc2 forward operand; blocks along F)
+ *   W2 colwise  [E*F, H]   (fc2 data-gradient operand; blocks along H)
+ * W1_dev bf16 [E, 2F, H] (rows 0..F-1 gate, F..2F-1 up; nn.Linear out x in),
+ * W2_dev bf16 [E, H, F]. Requires H % 256 == 0, F % 256 == 0.
+ */
+size_t mxmoe_weights_size(int32_t E, int32_t H, int32_t F);
+mxmoe_status mxmoe_weights_quantize(const void* W1_dev, const void* W2_dev, int32_t E, int32_t H, int32_t F,
+                                    void* wq_dev, size_t wq_bytes, void* stream);
+/* View of one of the four copies inside a weights buffer (which: 0 W1 row, 1 W1 col,
+ * 2 W2 row, 3 W2 col). Host-only pointer arithmetic. */
+mxmoe_status mxmoe_weights_view(void* wq_dev, int32_t E, int32_t H, int32_t F, int32_t which, mxmoe_mxfp8* out);
+
+/*
+ * Activations saved by the forward for the backward: one opaque device buffer of
+ * grouped_mlp_saved_size(...) bytes (routing maps, colwise MXFP8 copies of the permuted
+ * input and of Z, and the gate/up pre-activations in bf16). Named fields can be located
+ * with grouped_mlp_saved_offset for inspection.
+ */
+#define MXMOE_SAVED_M_SPLITS 0     /* int32 [E] */
+#define MXMOE_SAVED_SEG_OFF 1      /* int32 [E+1] */
+#define MXMOE_SAVED_ROW_OF_SLOT 2  /* int32 [T*k] */
+#define MXMOE_SAVED_TOKEN_OF_ROW 3 /* int32 [cap] */
+#define MXMOE_SAVED_PROB_OF_ROW 4  /* float [cap] */
+#define MXMOE_SAVED_X_COLT 5       /* e4m3 [H, cap] */
+#define MXMOE_SAVED_X_COLT_SF 6    /* e8m0, MMA layout */
+#define MXMOE_SAVED_Z_COLT 7       /* e4m3 [F, cap] */
+#define MXMOE_SAVED_Z_COLT_SF 8    /* e8m0, MMA layout */
+#define MXMOE_SAVED_GU 9           /* bf16 [cap, 2F] (gate | up) */
+size_t grouped_mlp_saved_size(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F);
+int64_t grouped_mlp_saved_offset(int32_t field, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F);
+
+/* Scratch for one forward or backward call (the larger of the two). */
+size_t grouped_mlp_workspace_size(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F);
+
+/*
+ * grouped_mlp_fwd -- forward of the MoE expert MLP as one grouped computation
+ * ("MoE-Training für biologische Grundmodelle optimieren", GroupedLinear, MXFP8 and
+ * GroupedMLP passages; "NVIDIA apresenta técnicas ... arquitetura MoE", third
+ * optimisation):
+ *   route -> permute + quantise x -> fc1 grouped GEMM whose epilogue computes
+ *   Z = silu(G) * U * p (p = the row's routing probability) and quantises Z to MXFP8
+ *   (Z never reaches memory in 16-bit) -> fc2 grouped GEMM -> combine.
+ *   x_dev bf16 [T, H]; topk_idx_dev int32 [T, k]; probs_dev float [T, k];
+ *   wq_dev from mxmoe_weights_quantize; y_dev bf16 [T, H].
+ * Limits: as moe_permute, plus H % 256 == 0, F % 256 == 0.
+ */
+mxmoe_status grouped_mlp_fwd(const void* x_dev, const int32_t* topk_idx_dev, const float* probs_dev,
+                             const void* wq_dev, size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H,
+                             int32_t F, void* y_dev, void* saved_dev, size_t saved_bytes, void* ws_dev,
+                             size_t ws_bytes, void* stream);
+
+/*
+ * grouped_mlp_bwd -- the matching backward (straight-through for every quantiser):
+ *   permute + quantise dy -> fc2 data-gradient GEMM whose epilogue applies the SwiGLU
+ *   and probability-scale backward (dA = dZ*p, dG = dA*U*silu'(G), dU = dA*silu(G),
+ *   dprob = sum_f dZ*A) and quantises dGU rowwise and colwise -> fc2 weight-gradient
+ *   GEMM -> fc1 data-gradient GEMM -> fc1 weight-gradient GEMM -> combine.
+ *   dy_dev bf16 [T, H]; outputs dx_dev bf16 [T, H], dW1_dev float [E, 2F, H],
+ *   dW2_dev float [E, H, F], dprobs_dev float [T, k] (all overwritten; experts with
+ *   no tokens get zero weight gradients).
+ */
+mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t saved_bytes, const void* wq_dev,
+                             size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F, void* dx_dev,
+                             float* dW1_dev, float* dW2_dev, float* dprobs_dev, void* ws_dev, size_t ws_bytes,
+                             void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MXMOE_H_ */

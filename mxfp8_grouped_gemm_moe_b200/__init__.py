@@ -1,0 +1,298 @@
+"""Python binding of libmxmoe.so -- the B200 MXFP8 grouped expert-MLP library.
+
+Argument marshalling only: every function below forwards to the C entry point of the
+same name (declared in include/mxmoe.h) and every step of the computation runs in the
+library's CUDA kernels. PyTorch is used for device memory and the current stream. If
+the shared library is missing or cannot be loaded, every call raises -- there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmxmoe.so")
+
+MXMOE_OK = 0
+STATUS_NAMES = {
+    0: "MXMOE_OK", 1: "MXMOE_ERR_INVALID_ARG", 2: "MXMOE_ERR_UNSUPPORTED_SHAPE",
+    3: "MXMOE_ERR_WORKSPACE_TOO_SMALL", 4: "MXMOE_ERR_CUDA", 5: "MXMOE_ERR_DEVICE_TIMEOUT",
+    6: "MXMOE_ERR_DEVICE_CHECK",
+}
+DTYPE_BF16, DTYPE_F32 = 0, 1
+SCALE_PLAIN, SCALE_MMA = 0, 1
+SAVED_FIELDS = ["m_splits", "seg_off", "row_of_slot", "token_of_row", "prob_of_row",
+                "x_colT", "x_colT_sf", "z_colT", "z_colT_sf", "gu"]
+
+
+class MxmoeError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn} returned {STATUS_NAMES.get(status, status)}")
+
+
+class _MX(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("cols", ctypes.c_int64), ("scale_layout", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+_lib = None
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+_PMX = ctypes.POINTER(_MX)
+
+# name -> (restype, argtypes); the names and order follow include/mxmoe.h
+_SIGNATURES = {
+    "mxmoe_status_string": (ctypes.c_char_p, [_I32]),
+    "mxmoe_get_device_status": (_I32, [ctypes.POINTER(_I32), ctypes.POINTER(_I32), _P]),
+    "mxmoe_clear_device_status": (_I32, [_P]),
+    "mxmoe_rows_capacity": (_I64, [_I32, _I32, _I32]),
+    "moe_permute": (_I32, [_P, _P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_permute_workspace_size": (_SZ, [_I32, _I32, _I32]),
+    "moe_unpermute": (_I32, [_P, _P, _I32, _I32, _I32, _P, _P]),
+    "mxfp8_quantize": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _I64, _PMX, _PMX, _P]),
+    "grouped_gemm_mxfp8": (_I32, [_PMX, _PMX, _P, _I32, _I64, _I64, _P, _I32, _I64, _P]),
+    "grouped_gemm_mxfp8_wgrad": (_I32, [_PMX, _PMX, _P, _I32, _P, _P]),
+    "mxmoe_weights_size": (_SZ, [_I32, _I32, _I32]),
+    "mxmoe_weights_quantize": (_I32, [_P, _P, _I32, _I32, _I32, _P, _SZ, _P]),
+    "mxmoe_weights_view": (_I32, [_P, _I32, _I32, _I32, _I32, _PMX]),
+    "grouped_mlp_saved_size": (_SZ, [_I32, _I32, _I32, _I32, _I32]),
+    "grouped_mlp_saved_offset": (_I64, [_I32, _I32, _I32, _I32, _I32, _I32]),
+    "grouped_mlp_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32]),
+    "grouped_mlp_fwd": (_I32, [_P, _P, _P, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _P, _P, _SZ, _P, _SZ, _P]),
+    "grouped_mlp_bwd": (_I32, [_P, _P, _SZ, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
+}
+
+
+def load(path: str | None = None):
+    """Loads (once) and returns the ctypes handle of libmxmoe.so; raises if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"libmxmoe.so not built ({p}); run __graft_entry__.build() first")
+    lib = ctypes.CDLL(p)
+    for name, (res, args) in _SIGNATURES.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(fn, st):
+    if st != MXMOE_OK:
+        raise MxmoeError(fn, st)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+# ----------------------------------------------------------------------------- MXFP8 tensors
+@dataclass
+class MXFP8:
+    """An MXFP8 matrix: data uint8 [rows, cols] (E4M3 codes), scale uint8 (E8M0), and the
+    scale layout (SCALE_PLAIN = [rows, cols/32]; SCALE_MMA = tensor-core chunk order)."""
+    data: torch.Tensor
+    scale: torch.Tensor
+    layout: int = SCALE_MMA
+
+    @property
+    def rows(self):
+        return self.data.shape[0]
+
+    @property
+    def cols(self):
+        return self.data.shape[1]
+
+    @staticmethod
+    def empty(rows, cols, layout=SCALE_MMA, device="cuda"):
+        return MXFP8(torch.empty((rows, cols), dtype=torch.uint8, device=device),
+                     torch.empty((rows * cols // 32,), dtype=torch.uint8, device=device), layout)
+
+    def as_struct(self):
+        return _MX(self.data.data_ptr(), self.scale.data_ptr(), self.rows, self.cols, self.layout, 0)
+
+    def scale_plain(self):
+        """Scales as a [rows, cols/32] CPU tensor in plain order (index permutation only)."""
+        s = self.scale.cpu()
+        if self.layout == SCALE_PLAIN:
+            return s.view(self.rows, self.cols // 32)
+        return scales_mma_to_plain(s, self.rows, self.cols)
+
+
+def scales_mma_to_plain(s, rows, cols):
+    """Inverse of the MMA scale order: chunk (r//128, kb//4) of 512 bytes, inside it
+    byte (r%32)*16 + ((r//32)%4)*4 + kb%4. Pure index permutation (CPU)."""
+    s = torch.as_tensor(s).reshape(rows // 128, cols // 128, 32, 4, 4)   # [rg, kg, r%32, (r/32)%4, kb%4]
+    s = s.permute(0, 3, 2, 1, 4)                                          # [rg, r/32%4, r%32, kg, kb%4]
+    return s.reshape(rows, cols // 32).contiguous()
+
+
+# ----------------------------------------------------------------------------- entry points
+def status_string(s):
+    return load().mxmoe_status_string(s).decode()
+
+
+def mxmoe_get_device_status():
+    v, w = _I32(0), _I32(0)
+    _check("mxmoe_get_device_status", load().mxmoe_get_device_status(ctypes.byref(v), ctypes.byref(w), _stream()))
+    return v.value, w.value
+
+
+def mxmoe_clear_device_status():
+    _check("mxmoe_clear_device_status", load().mxmoe_clear_device_status(_stream()))
+
+
+def mxmoe_rows_capacity(T, k, E):
+    return int(load().mxmoe_rows_capacity(T, k, E))
+
+
+def moe_permute(topk_idx, probs, E):
+    """-> dict(m_splits, seg_off, row_of_slot, token_of_row, prob_of_row) (device tensors)."""
+    lib = load()
+    T, k = topk_idx.shape
+    cap = mxmoe_rows_capacity(T, k, E)
+    dev = topk_idx.device
+    out = dict(m_splits=torch.empty(E, dtype=torch.int32, device=dev),
+               seg_off=torch.empty(E + 1, dtype=torch.int32, device=dev),
+               row_of_slot=torch.empty((T, k), dtype=torch.int32, device=dev),
+               token_of_row=torch.full((cap,), -2, dtype=torch.int32, device=dev),
+               prob_of_row=torch.full((cap,), -1.0, dtype=torch.float32, device=dev))
+    ws = torch.empty(lib.moe_permute_workspace_size(T, k, E), dtype=torch.uint8, device=dev)
+    st = lib.moe_permute(_ptr(topk_idx), _ptr(probs), T, k, E, _ptr(out["m_splits"]), _ptr(out["seg_off"]),
+                         _ptr(out["row_of_slot"]), _ptr(out["token_of_row"]), _ptr(out["prob_of_row"]),
+                         _ptr(ws), ws.numel(), _stream())
+    _check("moe_permute", st)
+    return out
+
+
+def moe_unpermute(y_perm, row_of_slot, out=None):
+    T, k = row_of_slot.shape
+    H = y_perm.shape[1]
+    y = out if out is not None else torch.empty((T, H), dtype=torch.bfloat16, device=y_perm.device)
+    _check("moe_unpermute", load().moe_unpermute(_ptr(y_perm), _ptr(row_of_slot), T, k, H, _ptr(y), _stream()))
+    return y
+
+
+def mxfp8_quantize(src, rowwise=True, colwise=True, layout=SCALE_MMA, row_gather=None, nrows=None, out_rows=None):
+    """src [rows, cols] or [batch, rows, cols] bf16/fp32 -> (MXFP8 rowwise | None, MXFP8 colT | None)."""
+    lib = load()
+    dt = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}[src.dtype]
+    if src.dim() == 2:
+        batch, (rows, cols) = 1, src.shape
+    else:
+        batch, rows, cols = src.shape
+    orows = rows if out_rows is None else out_rows
+    r = MXFP8.empty(batch * orows, cols, layout, src.device) if rowwise else None
+    c = MXFP8.empty(batch * cols, orows, layout, src.device) if colwise else None
+    rs = ctypes.byref(r.as_struct()) if r is not None else None
+    cs = ctypes.byref(c.as_struct()) if c is not None else None
+    st = lib.mxfp8_quantize(_ptr(src), dt, batch, rows, cols, _ptr(row_gather), _ptr(nrows), orows, rs, cs,
+                            _stream())
+    _check("mxfp8_quantize", st)
+    return r, c
+
+
+def grouped_gemm_mxfp8(A: MXFP8, B: MXFP8, seg_off, E, N, out_dtype=torch.bfloat16, out=None):
+    K = A.cols
+    C = out if out is not None else torch.empty((A.rows, N), dtype=out_dtype, device=A.data.device)
+    dt = DTYPE_BF16 if C.dtype == torch.bfloat16 else DTYPE_F32
+    st = load().grouped_gemm_mxfp8(ctypes.byref(A.as_struct()), ctypes.byref(B.as_struct()), _ptr(seg_off), E, N,
+                                   K, _ptr(C), dt, C.stride(0), _stream())
+    _check("grouped_gemm_mxfp8", st)
+    return C
+
+
+def grouped_gemm_mxfp8_wgrad(At: MXFP8, Bt: MXFP8, seg_off, E, out=None):
+    C = out if out is not None else torch.empty((E, At.rows, Bt.rows), dtype=torch.float32, device=At.data.device)
+    st = load().grouped_gemm_mxfp8_wgrad(ctypes.byref(At.as_struct()), ctypes.byref(Bt.as_struct()), _ptr(seg_off),
+                                         E, _ptr(C), _stream())
+    _check("grouped_gemm_mxfp8_wgrad", st)
+    return C
+
+
+def mxmoe_weights_quantize(W1, W2, out=None):
+    lib = load()
+    E, F2, H = W1.shape
+    F = F2 // 2
+    n = lib.mxmoe_weights_size(E, H, F)
+    wq = out if out is not None else torch.empty(n, dtype=torch.uint8, device=W1.device)
+    _check("mxmoe_weights_quantize",
+           lib.mxmoe_weights_quantize(_ptr(W1), _ptr(W2), E, H, F, _ptr(wq), wq.numel(), _stream()))
+    return wq
+
+
+def mxmoe_weights_view(wq, E, H, F, which):
+    """MXFP8 view (0 W1 row, 1 W1 colT, 2 W2 row, 3 W2 colT) into a weights buffer."""
+    m = _MX()
+    _check("mxmoe_weights_view", load().mxmoe_weights_view(_ptr(wq), E, H, F, which, ctypes.byref(m)))
+    base = wq.data_ptr()
+    d0, s0 = m.data - base, m.scale - base
+    n = m.rows * m.cols
+    return MXFP8(wq[d0:d0 + n].view(m.rows, m.cols), wq[s0:s0 + n // 32], SCALE_MMA)
+
+
+class GroupedMLP:
+    """Buffers for one layer shape; forward/backward call the fused C entry points."""
+
+    def __init__(self, T, k, E, H, F, device="cuda"):
+        lib = load()
+        self.T, self.k, self.E, self.H, self.F = T, k, E, H, F
+        self.cap = mxmoe_rows_capacity(T, k, E)
+        self.saved = torch.empty(lib.grouped_mlp_saved_size(T, k, E, H, F), dtype=torch.uint8, device=device)
+        self.ws = torch.empty(lib.grouped_mlp_workspace_size(T, k, E, H, F), dtype=torch.uint8, device=device)
+        self.wq = torch.empty(lib.mxmoe_weights_size(E, H, F), dtype=torch.uint8, device=device)
+
+    def quantize_weights(self, W1, W2):
+        return mxmoe_weights_quantize(W1, W2, out=self.wq)
+
+    def forward(self, x, topk_idx, probs, y=None):
+        return grouped_mlp_fwd(x, topk_idx, probs, self.wq, self.E, self.F, self.saved, self.ws, y)
+
+    def backward(self, dy, dx=None, dW1=None, dW2=None, dprobs=None):
+        return grouped_mlp_bwd(dy, self.saved, self.wq, self.T, self.k, self.E, self.H, self.F, self.ws,
+                               dx, dW1, dW2, dprobs)
+
+    def saved_field(self, name, dtype=torch.uint8, count=None):
+        """View of a named field of the saved buffer (inspection / tests)."""
+        lib = load()
+        f = SAVED_FIELDS.index(name)
+        off = lib.grouped_mlp_saved_offset(f, self.T, self.k, self.E, self.H, self.F)
+        esz = torch.tensor([], dtype=dtype).element_size()
+        return self.saved[off:off + count * esz].view(dtype)
+
+
+def grouped_mlp_fwd(x, topk_idx, probs, wq, E, F, saved, ws, y=None):
+    T, H = x.shape
+    k = topk_idx.shape[1]
+    y = y if y is not None else torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    st = load().grouped_mlp_fwd(_ptr(x), _ptr(topk_idx), _ptr(probs), _ptr(wq), wq.numel(), T, k, E, H, F, _ptr(y),
+                                _ptr(saved), saved.numel(), _ptr(ws), ws.numel(), _stream())
+    _check("grouped_mlp_fwd", st)
+    return y
+
+
+def grouped_mlp_bwd(dy, saved, wq, T, k, E, H, F, ws, dx=None, dW1=None, dW2=None, dprobs=None):
+    dev = dy.device
+    dx = dx if dx is not None else torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    dW1 = dW1 if dW1 is not None else torch.empty((E, 2 * F, H), dtype=torch.float32, device=dev)
+    dW2 = dW2 if dW2 is not None else torch.empty((E, H, F), dtype=torch.float32, device=dev)
+    dprobs = dprobs if dprobs is not None else torch.empty((T, k), dtype=torch.float32, device=dev)
+    st = load().grouped_mlp_bwd(_ptr(dy), _ptr(saved), saved.numel(), _ptr(wq), wq.numel(), T, k, E, H, F, _ptr(dx),
+                                _ptr(dW1), _ptr(dW2), _ptr(dprobs), _ptr(ws), ws.numel(), _stream())
+    _check("grouped_mlp_bwd", st)
+    return dx, dW1, dW2, dprobs

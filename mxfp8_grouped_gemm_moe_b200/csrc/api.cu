@@ -1,0 +1,473 @@
+// C ABI of the library: argument validation, buffer carving and the orchestration of
+// the fused grouped-MLP forward and backward. Every step of the path runs in this
+// library's kernels; nothing here allocates or synchronises (except the explicit
+// status query).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/mxmoe.h"
+#include "mxmoe_launch.h"
+
+#include "mxmoe_device.cuh"
+
+using namespace mxmoe;
+
+namespace {
+
+inline size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline mxmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MXMOE_OK : MXMOE_ERR_CUDA; }
+
+int64_t rows_cap(int64_t T, int64_t k, int64_t E) { return (T * k + 127 * E + 127) / 128 * 128; }
+
+// Sub-buffers of a caller-provided byte buffer, each 256-byte aligned.
+struct Carver {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    const size_t o = off;
+    off = al256(off + bytes);
+    return o;
+  }
+};
+
+bool valid_moe_shape(int32_t T, int32_t k, int32_t E) { return T >= 0 && k >= 1 && k <= 8 && E >= 1 && E <= 256; }
+bool valid_mlp_shape(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F) {
+  return valid_moe_shape(T, k, E) && H > 0 && F > 0 && H % 256 == 0 && F % 256 == 0;
+}
+
+// ---------------------------------------------------------------- layouts
+struct WeightsLayout {
+  size_t d[4], s[4], total;
+  int64_t rows[4], cols[4];
+};
+WeightsLayout weights_layout(int64_t E, int64_t H, int64_t F) {
+  WeightsLayout L;
+  const int64_t r[4] = {E * 2 * F, E * H, E * H, E * F};
+  const int64_t c[4] = {H, 2 * F, F, H};
+  Carver cv;
+  for (int i = 0; i < 4; ++i) {
+    L.rows[i] = r[i];
+    L.cols[i] = c[i];
+    L.d[i] = cv.take((size_t)(r[i] * c[i]));
+    L.s[i] = cv.take((size_t)(r[i] * c[i] / 32));
+  }
+  L.total = cv.off;
+  return L;
+}
+
+struct SavedLayout {
+  size_t off[10];
+  size_t total;
+};
+SavedLayout saved_layout(int64_t T, int64_t k, int64_t E, int64_t H, int64_t F) {
+  const int64_t cap = rows_cap(T, k, E);
+  SavedLayout L;
+  Carver cv;
+  L.off[MXMOE_SAVED_M_SPLITS] = cv.take(E * 4);
+  L.off[MXMOE_SAVED_SEG_OFF] = cv.take((E + 1) * 4);
+  L.off[MXMOE_SAVED_ROW_OF_SLOT] = cv.take(std::max<int64_t>(T * k, 1) * 4);
+  L.off[MXMOE_SAVED_TOKEN_OF_ROW] = cv.take(cap * 4);
+  L.off[MXMOE_SAVED_PROB_OF_ROW] = cv.take(cap * 4);
+  L.off[MXMOE_SAVED_X_COLT] = cv.take(H * cap);
+  L.off[MXMOE_SAVED_X_COLT_SF] = cv.take(H * cap / 32);
+  L.off[MXMOE_SAVED_Z_COLT] = cv.take(F * cap);
+  L.off[MXMOE_SAVED_Z_COLT_SF] = cv.take(F * cap / 32);
+  L.off[MXMOE_SAVED_GU] = cv.take(cap * 2 * F * 2);
+  L.total = cv.off;
+  return L;
+}
+
+struct FwdWs {
+  size_t route, x_row, x_row_sf, z_row, z_row_sf, y_perm, total;
+};
+FwdWs fwd_ws(int64_t T, int64_t k, int64_t E, int64_t H, int64_t F) {
+  const int64_t cap = rows_cap(T, k, E);
+  FwdWs w;
+  Carver cv;
+  w.route = cv.take(route_workspace_bytes((int)T, (int)k, (int)E));
+  w.x_row = cv.take(cap * H);
+  w.x_row_sf = cv.take(cap * H / 32);
+  w.z_row = cv.take(cap * F);
+  w.z_row_sf = cv.take(cap * F / 32);
+  w.y_perm = cv.take(cap * H * 2);
+  w.total = cv.off;
+  return w;
+}
+
+struct BwdWs {
+  size_t dy_row, dy_row_sf, dy_colT, dy_colT_sf, dgu_row, dgu_row_sf, dgu_colT, dgu_colT_sf, dprob_part, dx_perm,
+      total;
+};
+BwdWs bwd_ws(int64_t T, int64_t k, int64_t E, int64_t H, int64_t F) {
+  const int64_t cap = rows_cap(T, k, E);
+  BwdWs w;
+  Carver cv;
+  w.dy_row = cv.take(cap * H);
+  w.dy_row_sf = cv.take(cap * H / 32);
+  w.dy_colT = cv.take(H * cap);
+  w.dy_colT_sf = cv.take(H * cap / 32);
+  w.dgu_row = cv.take(cap * 2 * F);
+  w.dgu_row_sf = cv.take(cap * 2 * F / 32);
+  w.dgu_colT = cv.take(2 * F * cap);
+  w.dgu_colT_sf = cv.take(2 * F * cap / 32);
+  w.dprob_part = cv.take(cap * (F / 128) * 4);
+  w.dx_perm = cv.take(cap * H * 2);
+  w.total = cv.off;
+  return w;
+}
+
+bool valid_mx(const mxmoe_mxfp8* m) {
+  return m && m->data && m->scale && aligned16(m->data) && aligned16(m->scale) && m->rows >= 0 && m->cols >= 0 &&
+         (m->scale_layout == MXMOE_SCALE_PLAIN || m->scale_layout == MXMOE_SCALE_MMA) && m->reserved == 0;
+}
+bool mma_ready(const mxmoe_mxfp8* m) {
+  return valid_mx(m) && m->scale_layout == MXMOE_SCALE_MMA && m->rows % 128 == 0 && m->cols % 128 == 0;
+}
+
+mxmoe_mxfp8 mk(uint8_t* base, size_t d, size_t s, int64_t rows, int64_t cols) {
+  mxmoe_mxfp8 m;
+  m.data = base + d;
+  m.scale = base + s;
+  m.rows = rows;
+  m.cols = cols;
+  m.scale_layout = MXMOE_SCALE_MMA;
+  m.reserved = 0;
+  return m;
+}
+
+GemmArgs gemm_base(int mode, const mxmoe_mxfp8& A, const mxmoe_mxfp8& B, const int32_t* seg_off, int32_t E) {
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.mode = mode;
+  g.E = E;
+  g.a_data = A.data;
+  g.a_sf = A.scale;
+  g.a_rows = A.rows;
+  g.a_cols = A.cols;
+  g.b_data = B.data;
+  g.b_sf = B.scale;
+  g.b_rows = B.rows;
+  g.b_cols = B.cols;
+  g.seg_off = seg_off;
+  return g;
+}
+
+}  // namespace
+
+// ============================================================================ C ABI
+extern "C" {
+
+const char* mxmoe_status_string(mxmoe_status s) {
+  switch (s) {
+    case MXMOE_OK: return "MXMOE_OK";
+    case MXMOE_ERR_INVALID_ARG: return "MXMOE_ERR_INVALID_ARG";
+    case MXMOE_ERR_UNSUPPORTED_SHAPE: return "MXMOE_ERR_UNSUPPORTED_SHAPE";
+    case MXMOE_ERR_WORKSPACE_TOO_SMALL: return "MXMOE_ERR_WORKSPACE_TOO_SMALL";
+    case MXMOE_ERR_CUDA: return "MXMOE_ERR_CUDA";
+    case MXMOE_ERR_DEVICE_TIMEOUT: return "MXMOE_ERR_DEVICE_TIMEOUT";
+    case MXMOE_ERR_DEVICE_CHECK: return "MXMOE_ERR_DEVICE_CHECK";
+  }
+  return "MXMOE_ERR_UNKNOWN";
+}
+
+mxmoe_status mxmoe_get_device_status(int32_t* out_host, int32_t* where_host, void* stream) {
+  if (!out_host) return MXMOE_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return MXMOE_ERR_CUDA;
+  int32_t v = 0, w = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return MXMOE_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&w, g_device_status_where, sizeof(w)) != cudaSuccess) return MXMOE_ERR_CUDA;
+  *out_host = v;
+  if (where_host) *where_host = w;
+  return MXMOE_OK;
+}
+
+mxmoe_status mxmoe_clear_device_status(void* stream) {
+  static const int32_t zero = 0;
+  cudaError_t e = cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, S(stream));
+  if (e == cudaSuccess)
+    e = cudaMemcpyToSymbolAsync(g_device_status_where, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, S(stream));
+  return cuda_status(e);
+}
+
+int64_t mxmoe_rows_capacity(int32_t T, int32_t k, int32_t E) { return rows_cap(T, k, E); }
+
+size_t moe_permute_workspace_size(int32_t T, int32_t k, int32_t E) {
+  return route_workspace_bytes(T, k, E);
+}
+
+mxmoe_status moe_permute(const int32_t* topk_idx_dev, const float* probs_dev, int32_t T, int32_t k, int32_t E,
+                         int32_t* m_splits_dev, int32_t* seg_off_dev, int32_t* row_of_slot_dev,
+                         int32_t* token_of_row_dev, float* prob_of_row_dev, void* ws_dev, size_t ws_bytes,
+                         void* stream) {
+  if (!valid_moe_shape(T, k, E)) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if ((T > 0 && (!topk_idx_dev || !row_of_slot_dev)) || !m_splits_dev || !seg_off_dev || !token_of_row_dev ||
+      !ws_dev)
+    return MXMOE_ERR_INVALID_ARG;
+  if (prob_of_row_dev && T > 0 && !probs_dev) return MXMOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_permute_workspace_size(T, k, E)) return MXMOE_ERR_WORKSPACE_TOO_SMALL;
+  return cuda_status(launch_route(topk_idx_dev, probs_dev, T, k, E, m_splits_dev, seg_off_dev, row_of_slot_dev,
+                                  token_of_row_dev, prob_of_row_dev, ws_dev, S(stream)));
+}
+
+mxmoe_status moe_unpermute(const void* y_perm_dev, const int32_t* row_of_slot_dev, int32_t T, int32_t k, int32_t H,
+                           void* y_dev, void* stream) {
+  if (T < 0 || k < 1 || k > 8 || H <= 0 || H % 8 != 0) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MXMOE_OK;
+  if (!y_perm_dev || !row_of_slot_dev || !y_dev || !aligned16(y_perm_dev) || !aligned16(y_dev))
+    return MXMOE_ERR_INVALID_ARG;
+  return cuda_status(launch_unpermute(y_perm_dev, row_of_slot_dev, T, k, H, y_dev, S(stream)));
+}
+
+mxmoe_status mxfp8_quantize(const void* src_dev, int32_t src_dtype, int64_t batch, int64_t rows, int64_t cols,
+                            const int32_t* row_gather_dev, const int32_t* nrows_dev, int64_t out_rows,
+                            const mxmoe_mxfp8* out_row, const mxmoe_mxfp8* out_colT, void* stream) {
+  if (src_dtype != MXMOE_DTYPE_BF16 && src_dtype != MXMOE_DTYPE_F32) return MXMOE_ERR_INVALID_ARG;
+  if (!src_dev || !aligned16(src_dev) || (!out_row && !out_colT)) return MXMOE_ERR_INVALID_ARG;
+  if (batch < 1 || rows < 0 || cols <= 0 || out_rows < 0) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if (row_gather_dev && batch != 1) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if (!row_gather_dev && out_rows != rows) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if (cols % 32 != 0 || out_rows % 32 != 0) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if (out_row) {
+    if (!valid_mx(out_row)) return MXMOE_ERR_INVALID_ARG;
+    if (out_row->rows != batch * out_rows || out_row->cols != cols) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+    if (out_row->scale_layout == MXMOE_SCALE_MMA && (out_rows % 128 != 0 || cols % 128 != 0))
+      return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (out_colT) {
+    if (!valid_mx(out_colT)) return MXMOE_ERR_INVALID_ARG;
+    if (out_colT->rows != batch * cols || out_colT->cols != out_rows) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+    if (out_colT->scale_layout == MXMOE_SCALE_MMA && (out_rows % 128 != 0 || cols % 128 != 0))
+      return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (out_rows == 0 || rows == 0) return MXMOE_OK;
+  QuantArgs a;
+  a.src = src_dev;
+  a.src_dtype = src_dtype;
+  a.batch = batch;
+  a.rows = rows;
+  a.cols = cols;
+  a.gather = row_gather_dev;
+  a.nrows = nrows_dev;
+  a.out_rows = out_rows;
+  a.row_data = out_row ? out_row->data : nullptr;
+  a.row_sf = out_row ? out_row->scale : nullptr;
+  a.row_layout = out_row ? out_row->scale_layout : 0;
+  a.col_data = out_colT ? out_colT->data : nullptr;
+  a.col_sf = out_colT ? out_colT->scale : nullptr;
+  a.col_layout = out_colT ? out_colT->scale_layout : 0;
+  return cuda_status(launch_quantize(a, S(stream)));
+}
+
+mxmoe_status grouped_gemm_mxfp8(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, const int32_t* seg_off_dev,
+                                int32_t E, int64_t N, int64_t K, void* C_dev, int32_t c_dtype, int64_t ldc,
+                                void* stream) {
+  if (!A || !B || !seg_off_dev || !C_dev || !aligned16(C_dev)) return MXMOE_ERR_INVALID_ARG;
+  if (c_dtype != MXMOE_DTYPE_BF16 && c_dtype != MXMOE_DTYPE_F32) return MXMOE_ERR_INVALID_ARG;
+  if (!mma_ready(A) || !mma_ready(B)) return MXMOE_ERR_INVALID_ARG;
+  if (E < 1 || E > 256 || N <= 0 || K <= 0 || N % 256 != 0 || K % 128 != 0) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if (A->cols != K || B->cols != K || B->rows != (int64_t)E * N || ldc < N || ldc % 8 != 0)
+    return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if (A->rows == 0) return MXMOE_OK;
+  GemmArgs g = gemm_base(kModeStore, *A, *B, seg_off_dev, E);
+  g.N = N;
+  g.K = K;
+  g.c = C_dev;
+  g.c_dtype = c_dtype;
+  g.ldc = ldc;
+  return cuda_status(launch_gemm(g, S(stream)));
+}
+
+mxmoe_status grouped_gemm_mxfp8_wgrad(const mxmoe_mxfp8* At, const mxmoe_mxfp8* Bt, const int32_t* seg_off_dev,
+                                      int32_t E, float* C_dev, void* stream) {
+  if (!At || !Bt || !seg_off_dev || !C_dev || !aligned16(C_dev)) return MXMOE_ERR_INVALID_ARG;
+  if (!mma_ready(At) || !mma_ready(Bt)) return MXMOE_ERR_INVALID_ARG;
+  if (E < 1 || E > 256 || At->cols != Bt->cols || At->rows <= 0 || Bt->rows % 256 != 0 || Bt->rows <= 0)
+    return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  GemmArgs g = gemm_base(kModeWgrad, *At, *Bt, seg_off_dev, E);
+  g.N = At->rows;
+  g.K2 = Bt->rows;
+  g.c = C_dev;
+  g.c_dtype = MXMOE_DTYPE_F32;
+  g.ldc = Bt->rows;
+  return cuda_status(launch_gemm(g, S(stream)));
+}
+
+size_t mxmoe_weights_size(int32_t E, int32_t H, int32_t F) { return weights_layout(E, H, F).total; }
+
+mxmoe_status mxmoe_weights_view(void* wq_dev, int32_t E, int32_t H, int32_t F, int32_t which, mxmoe_mxfp8* out) {
+  if (!wq_dev || !out || which < 0 || which > 3) return MXMOE_ERR_INVALID_ARG;
+  const WeightsLayout L = weights_layout(E, H, F);
+  *out = mk(reinterpret_cast<uint8_t*>(wq_dev), L.d[which], L.s[which], L.rows[which], L.cols[which]);
+  return MXMOE_OK;
+}
+
+mxmoe_status mxmoe_weights_quantize(const void* W1_dev, const void* W2_dev, int32_t E, int32_t H, int32_t F,
+                                    void* wq_dev, size_t wq_bytes, void* stream) {
+  if (E < 1 || E > 256 || H <= 0 || F <= 0 || H % 256 != 0 || F % 256 != 0) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if (!W1_dev || !W2_dev || !wq_dev || !aligned16(W1_dev) || !aligned16(W2_dev) || !aligned16(wq_dev))
+    return MXMOE_ERR_INVALID_ARG;
+  const WeightsLayout L = weights_layout(E, H, F);
+  if (wq_bytes < L.total) return MXMOE_ERR_WORKSPACE_TOO_SMALL;
+  uint8_t* b = reinterpret_cast<uint8_t*>(wq_dev);
+  mxmoe_mxfp8 w1r = mk(b, L.d[0], L.s[0], L.rows[0], L.cols[0]);
+  mxmoe_mxfp8 w1c = mk(b, L.d[1], L.s[1], L.rows[1], L.cols[1]);
+  mxmoe_mxfp8 w2r = mk(b, L.d[2], L.s[2], L.rows[2], L.cols[2]);
+  mxmoe_mxfp8 w2c = mk(b, L.d[3], L.s[3], L.rows[3], L.cols[3]);
+  mxmoe_status s = mxfp8_quantize(W1_dev, MXMOE_DTYPE_BF16, E, 2 * (int64_t)F, H, nullptr, nullptr, 2 * (int64_t)F,
+                                  &w1r, &w1c, stream);
+  if (s != MXMOE_OK) return s;
+  return mxfp8_quantize(W2_dev, MXMOE_DTYPE_BF16, E, H, F, nullptr, nullptr, H, &w2r, &w2c, stream);
+}
+
+size_t grouped_mlp_saved_size(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F) {
+  return saved_layout(T, k, E, H, F).total;
+}
+
+int64_t grouped_mlp_saved_offset(int32_t field, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F) {
+  if (field < 0 || field > 9) return -1;
+  return (int64_t)saved_layout(T, k, E, H, F).off[field];
+}
+
+size_t grouped_mlp_workspace_size(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F) {
+  return std::max(fwd_ws(T, k, E, H, F).total, bwd_ws(T, k, E, H, F).total);
+}
+
+mxmoe_status grouped_mlp_fwd(const void* x_dev, const int32_t* topk_idx_dev, const float* probs_dev,
+                             const void* wq_dev, size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H,
+                             int32_t F, void* y_dev, void* saved_dev, size_t saved_bytes, void* ws_dev,
+                             size_t ws_bytes, void* stream) {
+  if (!valid_mlp_shape(T, k, E, H, F)) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if (!wq_dev || !saved_dev || !ws_dev || !aligned16(wq_dev) || !aligned16(saved_dev) || !aligned16(ws_dev))
+    return MXMOE_ERR_INVALID_ARG;
+  if (T > 0 && (!x_dev || !topk_idx_dev || !probs_dev || !y_dev || !aligned16(x_dev) || !aligned16(y_dev)))
+    return MXMOE_ERR_INVALID_ARG;
+  if (wq_bytes < mxmoe_weights_size(E, H, F) || saved_bytes < grouped_mlp_saved_size(T, k, E, H, F) ||
+      ws_bytes < grouped_mlp_workspace_size(T, k, E, H, F))
+    return MXMOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = S(stream);
+  const int64_t cap = rows_cap(T, k, E);
+  const SavedLayout SL = saved_layout(T, k, E, H, F);
+  const FwdWs W = fwd_ws(T, k, E, H, F);
+  const WeightsLayout WL = weights_layout(E, H, F);
+  uint8_t* sv = reinterpret_cast<uint8_t*>(saved_dev);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(ws_dev);
+  uint8_t* wq = reinterpret_cast<uint8_t*>(const_cast<void*>(wq_dev));
+  int32_t* m_splits = reinterpret_cast<int32_t*>(sv + SL.off[MXMOE_SAVED_M_SPLITS]);
+  int32_t* seg_off = reinterpret_cast<int32_t*>(sv + SL.off[MXMOE_SAVED_SEG_OFF]);
+  int32_t* ros = reinterpret_cast<int32_t*>(sv + SL.off[MXMOE_SAVED_ROW_OF_SLOT]);
+  int32_t* tor = reinterpret_cast<int32_t*>(sv + SL.off[MXMOE_SAVED_TOKEN_OF_ROW]);
+  float* por = reinterpret_cast<float*>(sv + SL.off[MXMOE_SAVED_PROB_OF_ROW]);
+
+  // 1. route
+  cudaError_t e = launch_route(topk_idx_dev, probs_dev, T, k, E, m_splits, seg_off, ros, tor, por, ws + W.route, st);
+  if (e != cudaSuccess) return MXMOE_ERR_CUDA;
+  if (T == 0) return MXMOE_OK;
+  // 2. permute + quantise x (rowwise for fc1, colwise saved for fc1 wgrad)
+  mxmoe_mxfp8 x_row = mk(ws, W.x_row, W.x_row_sf, cap, H);
+  mxmoe_mxfp8 x_col = mk(sv, SL.off[MXMOE_SAVED_X_COLT], SL.off[MXMOE_SAVED_X_COLT_SF], H, cap);
+  mxmoe_status s = mxfp8_quantize(x_dev, MXMOE_DTYPE_BF16, 1, T, H, tor, seg_off + E, cap, &x_row, &x_col, stream);
+  if (s != MXMOE_OK) return s;
+  // 3. fc1 + SwiGLU x prob -> Z (MXFP8 row + colT), G/U saved
+  mxmoe_mxfp8 w1r = mk(wq, WL.d[0], WL.s[0], WL.rows[0], WL.cols[0]);
+  GemmArgs g = gemm_base(kModeSwigluFwd, x_row, w1r, seg_off, E);
+  g.K = H;
+  g.F = F;
+  g.N = 2 * (int64_t)F;
+  g.rows_cap = cap;
+  g.prob_of_row = por;
+  g.z_row = ws + W.z_row;
+  g.z_row_sf = ws + W.z_row_sf;
+  g.z_colT = sv + SL.off[MXMOE_SAVED_Z_COLT];
+  g.z_colT_sf = sv + SL.off[MXMOE_SAVED_Z_COLT_SF];
+  g.gu = reinterpret_cast<uint16_t*>(sv + SL.off[MXMOE_SAVED_GU]);
+  if (launch_gemm(g, st) != cudaSuccess) return MXMOE_ERR_CUDA;
+  // 4. fc2 -> Yp bf16
+  mxmoe_mxfp8 z_row = mk(ws, W.z_row, W.z_row_sf, cap, F);
+  mxmoe_mxfp8 w2r = mk(wq, WL.d[2], WL.s[2], WL.rows[2], WL.cols[2]);
+  s = grouped_gemm_mxfp8(&z_row, &w2r, seg_off, E, H, F, ws + W.y_perm, MXMOE_DTYPE_BF16, H, stream);
+  if (s != MXMOE_OK) return s;
+  // 5. combine
+  return moe_unpermute(ws + W.y_perm, ros, T, k, H, y_dev, stream);
+}
+
+mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t saved_bytes, const void* wq_dev,
+                             size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F, void* dx_dev,
+                             float* dW1_dev, float* dW2_dev, float* dprobs_dev, void* ws_dev, size_t ws_bytes,
+                             void* stream) {
+  if (!valid_mlp_shape(T, k, E, H, F)) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if (!wq_dev || !saved_dev || !ws_dev || !dW1_dev || !dW2_dev || !aligned16(wq_dev) || !aligned16(saved_dev) ||
+      !aligned16(ws_dev) || !aligned16(dW1_dev) || !aligned16(dW2_dev))
+    return MXMOE_ERR_INVALID_ARG;
+  if (T > 0 && (!dy_dev || !dx_dev || !dprobs_dev || !aligned16(dy_dev) || !aligned16(dx_dev)))
+    return MXMOE_ERR_INVALID_ARG;
+  if (wq_bytes < mxmoe_weights_size(E, H, F) || saved_bytes < grouped_mlp_saved_size(T, k, E, H, F) ||
+      ws_bytes < grouped_mlp_workspace_size(T, k, E, H, F))
+    return MXMOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = S(stream);
+  const int64_t cap = rows_cap(T, k, E);
+  const SavedLayout SL = saved_layout(T, k, E, H, F);
+  const BwdWs W = bwd_ws(T, k, E, H, F);
+  const WeightsLayout WL = weights_layout(E, H, F);
+  uint8_t* sv = reinterpret_cast<uint8_t*>(const_cast<void*>(saved_dev));
+  uint8_t* ws = reinterpret_cast<uint8_t*>(ws_dev);
+  uint8_t* wq = reinterpret_cast<uint8_t*>(const_cast<void*>(wq_dev));
+  const int32_t* seg_off = reinterpret_cast<const int32_t*>(sv + SL.off[MXMOE_SAVED_SEG_OFF]);
+  const int32_t* ros = reinterpret_cast<const int32_t*>(sv + SL.off[MXMOE_SAVED_ROW_OF_SLOT]);
+  const int32_t* tor = reinterpret_cast<const int32_t*>(sv + SL.off[MXMOE_SAVED_TOKEN_OF_ROW]);
+  const float* por = reinterpret_cast<const float*>(sv + SL.off[MXMOE_SAVED_PROB_OF_ROW]);
+
+  // 1. permute + quantise dy: rowwise (fc2 dgrad) and colwise (fc2 wgrad)
+  mxmoe_mxfp8 dy_row = mk(ws, W.dy_row, W.dy_row_sf, cap, H);
+  mxmoe_mxfp8 dy_col = mk(ws, W.dy_colT, W.dy_colT_sf, H, cap);
+  mxmoe_status s;
+  if (T > 0) {
+    s = mxfp8_quantize(dy_dev, MXMOE_DTYPE_BF16, 1, T, H, tor, seg_off + E, cap, &dy_row, &dy_col, stream);
+    if (s != MXMOE_OK) return s;
+  }
+  // 2. fc2 dgrad + SwiGLU/prob backward -> dGU (MXFP8 row + colT), dprob partials
+  mxmoe_mxfp8 w2c = mk(wq, WL.d[3], WL.s[3], WL.rows[3], WL.cols[3]);
+  {
+    GemmArgs g = gemm_base(kModeSwigluBwd, dy_row, w2c, seg_off, E);
+    g.K = H;
+    g.N = F;
+    g.F = F;
+    g.rows_cap = cap;
+    g.prob_of_row = por;
+    g.gu_in = reinterpret_cast<const uint16_t*>(sv + SL.off[MXMOE_SAVED_GU]);
+    g.dgu_row = ws + W.dgu_row;
+    g.dgu_row_sf = ws + W.dgu_row_sf;
+    g.dgu_colT = ws + W.dgu_colT;
+    g.dgu_colT_sf = ws + W.dgu_colT_sf;
+    g.dprob_part = reinterpret_cast<float*>(ws + W.dprob_part);
+    if (T > 0 && launch_gemm(g, st) != cudaSuccess) return MXMOE_ERR_CUDA;
+  }
+  // 3. dprobs
+  if (launch_dprob_reduce(reinterpret_cast<const float*>(ws + W.dprob_part), F / 128, ros, (int64_t)T * k,
+                          dprobs_dev, st) != cudaSuccess)
+    return MXMOE_ERR_CUDA;
+  // 4. fc2 wgrad: dW2[e] = dYp_e^T . Z_e
+  mxmoe_mxfp8 z_col = mk(sv, SL.off[MXMOE_SAVED_Z_COLT], SL.off[MXMOE_SAVED_Z_COLT_SF], F, cap);
+  s = grouped_gemm_mxfp8_wgrad(&dy_col, &z_col, seg_off, E, dW2_dev, stream);
+  if (s != MXMOE_OK) return s;
+  // 5. fc1 dgrad: dXp = dGU . W1 (contract 2F)
+  mxmoe_mxfp8 dgu_row = mk(ws, W.dgu_row, W.dgu_row_sf, cap, 2 * (int64_t)F);
+  mxmoe_mxfp8 w1c = mk(wq, WL.d[1], WL.s[1], WL.rows[1], WL.cols[1]);
+  if (T > 0) {
+    s = grouped_gemm_mxfp8(&dgu_row, &w1c, seg_off, E, H, 2 * (int64_t)F, ws + W.dx_perm, MXMOE_DTYPE_BF16, H,
+                           stream);
+    if (s != MXMOE_OK) return s;
+  }
+  // 6. fc1 wgrad: dW1[e] = dGU_e^T . Xp_e
+  mxmoe_mxfp8 dgu_col = mk(ws, W.dgu_colT, W.dgu_colT_sf, 2 * (int64_t)F, cap);
+  mxmoe_mxfp8 x_col = mk(sv, SL.off[MXMOE_SAVED_X_COLT], SL.off[MXMOE_SAVED_X_COLT_SF], H, cap);
+  s = grouped_gemm_mxfp8_wgrad(&dgu_col, &x_col, seg_off, E, dW1_dev, stream);
+  if (s != MXMOE_OK) return s;
+  // 7. combine dX
+  return moe_unpermute(ws + W.dx_perm, ros, T, k, H, dx_dev, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,88 @@
+// Internal host-side launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/mxmoe.h"
+
+namespace mxmoe {
+
+// ---------------------------------------------------------------- routing / combine
+size_t route_workspace_bytes(int T, int k, int E);
+cudaError_t launch_route(const int32_t* idx, const float* probs, int T, int k, int E, int32_t* m_splits,
+                         int32_t* seg_off, int32_t* row_of_slot, int32_t* token_of_row, float* prob_of_row,
+                         void* ws, cudaStream_t st);
+cudaError_t launch_unpermute(const void* yp, const int32_t* ros, int T, int k, int H, void* y, cudaStream_t st);
+cudaError_t launch_dprob_reduce(const float* part, int nparts, const int32_t* ros, int64_t n, float* dprobs,
+                                cudaStream_t st);
+
+// ---------------------------------------------------------------- quantisation
+struct QuantArgs {
+  const void* src;
+  int32_t src_dtype;
+  int64_t batch, rows, cols;
+  const int32_t* gather;  // nullable
+  const int32_t* nrows;   // nullable (device)
+  int64_t out_rows;
+  uint8_t* row_data;  // nullable
+  uint8_t* row_sf;
+  int32_t row_layout;
+  uint8_t* col_data;  // nullable
+  uint8_t* col_sf;
+  int32_t col_layout;
+};
+cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- grouped GEMM
+enum GemmMode : int32_t {
+  kModeStore = 0,       // C = A . B_e^T, bf16 or fp32 out (M grouped by expert segments)
+  kModeSwigluFwd = 1,   // fc1 + SwiGLU x prob -> MXFP8 Z (row + colT), GU bf16 saved
+  kModeSwigluBwd = 2,   // fc2 dgrad + SwiGLU/prob backward -> MXFP8 dGU (row + colT), dprob partials
+  kModeWgrad = 3,       // C[e] = At_e . Bt_e^T, fp32, contraction over the expert's rows
+};
+
+struct GemmArgs {
+  int32_t mode;
+  int32_t E;
+  // operands (MMA scale layout)
+  const uint8_t* a_data;
+  const uint8_t* a_sf;
+  int64_t a_rows, a_cols;
+  const uint8_t* b_data;
+  const uint8_t* b_sf;
+  int64_t b_rows, b_cols;
+  const int32_t* seg_off;  // device [E+1]
+  int64_t N;               // per-expert B rows (store/bwd), F (fwd), output rows per expert (wgrad)
+  int64_t K;               // contraction length (not used by wgrad)
+  // plain output
+  void* c;
+  int32_t c_dtype;
+  int64_t ldc;
+  int64_t K2;  // wgrad: output columns per expert
+  // SwiGLU forward epilogue
+  const float* prob_of_row;
+  int64_t F;
+  int64_t rows_cap;
+  uint8_t* z_row;
+  uint8_t* z_row_sf;
+  uint8_t* z_colT;
+  uint8_t* z_colT_sf;
+  uint16_t* gu;  // bf16 [rows_cap, 2F]
+  // SwiGLU backward epilogue
+  const uint16_t* gu_in;
+  uint8_t* dgu_row;
+  uint8_t* dgu_row_sf;
+  uint8_t* dgu_colT;
+  uint8_t* dgu_colT_sf;
+  float* dprob_part;  // [rows_cap, F/128]
+  // debug: if non-zero, the MMA warp withholds its first accumulator-ready signal so
+  // that the epilogue's bounded wait expires (tests the timeout path; never set in
+  // normal use)
+  int32_t debug_drop_commit;
+};
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st);
+int gemm_num_sms();
+
+}  // namespace mxmoe

@@ -1,0 +1,136 @@
+// MXFP8 quantisation of activations and weights, rowwise and colwise from one read,
+// optionally fused with the expert permutation (row gather).
+//
+// "MoE-Training für biologische Grundmodelle optimieren" (hyper.ai/de), MXFP8 passage:
+// 8-bit values with one scale per block of 32; GroupedMLP passage: the 16-bit -> 8-bit
+// conversions are fused rather than run as separate operations. Element / scale rule:
+// OCP MX (E4M3 elements, E8M0 scale, X = clamp(floor(log2 amax) - 8, -127, 127),
+// round-to-nearest-even with saturation).
+//
+// One CTA quantises a 128 x 128 tile staged in shared memory: rowwise blocks (32
+// consecutive columns of a row) and colwise blocks (32 consecutive rows of a column,
+// written transposed) come from the same HBM read. Loads and stores are 16-byte
+// vectors; a warp's rowwise / colwise stores cover whole 32-byte sectors.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "mxmoe_device.cuh"
+#include "mxmoe_launch.h"
+
+namespace mxmoe {
+
+constexpr int kQTile = 128;
+constexpr int kQThreads = 256;
+
+template <typename T>
+struct SrcTraits;
+template <>
+struct SrcTraits<__nv_bfloat16> {
+  static constexpr int kPad = 8;  // elements of row padding in shared memory (16 bytes)
+  static constexpr int kVec = 8;  // elements per 16-byte vector
+};
+template <>
+struct SrcTraits<float> {
+  static constexpr int kPad = 4;
+  static constexpr int kVec = 4;
+};
+
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float to_f32(float v) { return v; }
+
+template <typename T>
+__global__ void __launch_bounds__(kQThreads) mxfp8_quantize_kernel(QuantArgs a) {
+  using Tr = SrcTraits<T>;
+  constexpr int LD = kQTile + Tr::kPad;
+  extern __shared__ __align__(16) uint8_t q_smem_raw[];
+  T* tile = reinterpret_cast<T*>(q_smem_raw);
+
+  const int64_t c0 = (int64_t)blockIdx.x * kQTile;
+  const int64_t r0 = (int64_t)blockIdx.y * kQTile;
+  const int64_t b = blockIdx.z;
+  int64_t nvalid = a.out_rows;
+  if (a.nrows) {
+    const int64_t nv = *a.nrows;
+    nvalid = nv < nvalid ? nv : nvalid;
+  }
+  if (r0 >= nvalid) return;
+  const T* src = reinterpret_cast<const T*>(a.src);
+
+  // ---- load the tile (gathered rows, zero outside the matrix / for pad rows)
+  constexpr int VPR = kQTile / Tr::kVec;  // vectors per tile row
+  for (int i = threadIdx.x; i < kQTile * VPR; i += kQThreads) {
+    const int row = i / VPR, cv = i % VPR;
+    const int64_t orow = r0 + row;
+    const int64_t col = c0 + (int64_t)cv * Tr::kVec;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (orow < nvalid && col < a.cols) {
+      int64_t srow;
+      if (a.gather) srow = a.gather[orow];
+      else srow = b * a.rows + orow;
+      if (srow >= 0) v = __ldg(reinterpret_cast<const uint4*>(src + srow * a.cols + col));
+    }
+    *reinterpret_cast<uint4*>(tile + row * LD + cv * Tr::kVec) = v;
+  }
+  __syncthreads();
+
+  // ---- rowwise: 128 rows x 4 blocks
+  if (a.row_data) {
+    for (int it = threadIdx.x; it < kQTile * 4; it += kQThreads) {
+      const int row = it >> 2, blk = it & 3;
+      const int64_t orow = r0 + row;
+      const int64_t col = c0 + 32 * blk;
+      if (orow >= nvalid || col >= a.cols) continue;
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = to_f32(tile[row * LD + 32 * blk + i]);
+      uint32_t q[8];
+      const uint8_t sb = quant_block32(v, q);
+      const int64_t grow = b * a.out_rows + orow;
+      uint4* dst = reinterpret_cast<uint4*>(a.row_data + grow * a.cols + col);
+      dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
+      dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
+      a.row_sf[sf_offset(a.row_layout, a.batch * a.out_rows, a.cols, grow, col / 32)] = sb;
+    }
+  }
+  // ---- colwise: 128 columns x 4 row blocks, stored transposed
+  if (a.col_data) {
+    for (int it = threadIdx.x; it < kQTile * 4; it += kQThreads) {
+      const int cc = it & (kQTile - 1), rb = it >> 7;
+      const int64_t col = c0 + cc;
+      const int64_t orow = r0 + 32 * rb;
+      if (orow >= nvalid || col >= a.cols) continue;
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = to_f32(tile[(32 * rb + i) * LD + cc]);
+      uint32_t q[8];
+      const uint8_t sb = quant_block32(v, q);
+      const int64_t grow = b * a.cols + col;  // row of the transposed matrix
+      uint4* dst = reinterpret_cast<uint4*>(a.col_data + grow * a.out_rows + orow);
+      dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
+      dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
+      a.col_sf[sf_offset(a.col_layout, a.batch * a.cols, a.out_rows, grow, orow / 32)] = sb;
+    }
+  }
+}
+
+template <typename T>
+static cudaError_t launch_q(const QuantArgs& a, cudaStream_t st) {
+  using Tr = SrcTraits<T>;
+  const size_t smem = (size_t)kQTile * (kQTile + Tr::kPad) * sizeof(T);
+  cudaError_t e =
+      cudaFuncSetAttribute(mxfp8_quantize_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((a.cols + kQTile - 1) / kQTile), (unsigned)((a.out_rows + kQTile - 1) / kQTile),
+            (unsigned)a.batch);
+  if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
+  mxfp8_quantize_kernel<T><<<grid, kQThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st) {
+  if (a.src_dtype == MXMOE_DTYPE_BF16) return launch_q<__nv_bfloat16>(a, st);
+  return launch_q<float>(a, st);
+}
+
+}  // namespace mxmoe

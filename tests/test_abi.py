@@ -1,0 +1,106 @@
+"""The C-ABI library loads without a GPU, exports every entry point that
+include/mxmoe.h declares, and rejects bad arguments on the host before touching the
+device (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mxmoe.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    pat = re.compile(r"^\s*(?:const\s+)?(?:mxmoe_status|size_t|int64_t|char\s*\*)\s*\*?\s*(\w+)\s*\(", re.M)
+    return sorted(set(pat.findall(text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import __graft_entry__
+    __graft_entry__.build()
+    import mxfp8_grouped_gemm_moe_b200 as mx
+    return mx.load()
+
+
+def test_header_declares_the_north_star_entry_points():
+    names = _declared_functions()
+    for n in ["moe_permute", "moe_unpermute", "mxfp8_quantize", "grouped_gemm_mxfp8", "grouped_gemm_mxfp8_wgrad",
+              "grouped_mlp_fwd", "grouped_mlp_bwd", "mxmoe_weights_quantize"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_binding_signatures_cover_header(lib):
+    import mxfp8_grouped_gemm_moe_b200 as mx
+    assert set(_declared_functions()) == set(mx._SIGNATURES)
+
+
+def test_status_strings(lib):
+    import mxfp8_grouped_gemm_moe_b200 as mx
+    for code, name in mx.STATUS_NAMES.items():
+        assert lib.mxmoe_status_string(code).decode() == name
+
+
+def test_sizes_are_host_only(lib):
+    assert lib.mxmoe_rows_capacity(8192, 2, 8) == (8192 * 2 + 127 * 8 + 127) // 128 * 128
+    assert lib.mxmoe_rows_capacity(0, 1, 1) == 128
+    # weights: 4 copies of E*2F*H-ish bytes plus scales
+    E, H, F = 8, 4096, 14336
+    w = lib.mxmoe_weights_size(E, H, F)
+    assert w >= 2 * (3 * E * H * F) * (1 + 1 / 32)
+    s = lib.grouped_mlp_saved_size(8192, 2, 8, 4096, 14336)
+    cap = lib.mxmoe_rows_capacity(8192, 2, 8)
+    assert s >= cap * (4096 + 14336) * (1 + 1 / 32) + cap * 2 * 14336 * 2
+    offs = [lib.grouped_mlp_saved_offset(f, 8192, 2, 8, 4096, 14336) for f in range(10)]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert lib.grouped_mlp_saved_offset(10, 1, 1, 1, 256, 256) == -1
+
+
+def test_host_argument_errors_enqueue_nothing(lib):
+    """Every one of these is rejected before any CUDA call (so it runs without a GPU)."""
+    import mxfp8_grouped_gemm_moe_b200 as mx
+    P = ctypes.c_void_p
+    bad = P(0)
+    fake = P(1 << 20)             # never dereferenced: validation fails first
+    S = P(0)
+    # shapes
+    assert lib.moe_permute(fake, fake, 10, 9, 4, fake, fake, fake, fake, fake, fake, 1 << 20, S) == 2
+    assert lib.moe_permute(fake, fake, 10, 2, 300, fake, fake, fake, fake, fake, fake, 1 << 20, S) == 2
+    assert lib.moe_permute(fake, fake, -1, 2, 4, fake, fake, fake, fake, fake, fake, 1 << 20, S) == 2
+    # null pointers
+    assert lib.moe_permute(bad, fake, 10, 2, 4, fake, fake, fake, fake, fake, fake, 1 << 20, S) == 1
+    # workspace too small
+    assert lib.moe_permute(fake, fake, 10, 2, 4, fake, fake, fake, fake, fake, fake, 4, S) == 3
+    assert lib.moe_unpermute(fake, fake, 4, 2, 12, fake, S) == 2            # H % 8
+    assert lib.moe_unpermute(bad, fake, 4, 2, 16, fake, S) == 1
+    # quantize: bad dtype, bad shape, no outputs
+    m = mx._MX(1 << 20, 1 << 20, 64, 64, 0, 0)
+    assert lib.mxfp8_quantize(fake, 7, 1, 64, 64, None, None, 64, ctypes.byref(m), None, S) == 1
+    assert lib.mxfp8_quantize(fake, 0, 1, 64, 48, None, None, 64, ctypes.byref(m), None, S) == 2
+    assert lib.mxfp8_quantize(fake, 0, 1, 64, 64, None, None, 64, None, None, S) == 1
+    m_bad_layout = mx._MX(1 << 20, 1 << 20, 64, 64, 1, 0)   # MMA layout needs multiples of 128
+    assert lib.mxfp8_quantize(fake, 0, 1, 64, 64, None, None, 64, ctypes.byref(m_bad_layout), None, S) == 2
+    # grouped GEMM: N not a multiple of 256; A not in MMA layout
+    A = mx._MX(1 << 20, 1 << 20, 256, 256, 1, 0)
+    B = mx._MX(1 << 20, 1 << 20, 2 * 384, 256, 1, 0)
+    assert lib.grouped_gemm_mxfp8(ctypes.byref(A), ctypes.byref(B), fake, 2, 384, 256, fake, 0, 384, S) == 2
+    Ap = mx._MX(1 << 20, 1 << 20, 256, 256, 0, 0)
+    B2 = mx._MX(1 << 20, 1 << 20, 512, 256, 1, 0)
+    assert lib.grouped_gemm_mxfp8(ctypes.byref(Ap), ctypes.byref(B2), fake, 2, 256, 256, fake, 0, 256, S) == 1
+    # fused MLP: F not a multiple of 256, workspace too small
+    assert lib.grouped_mlp_fwd(fake, fake, fake, fake, 1 << 40, 16, 2, 4, 256, 384, fake, fake, 1 << 40, fake,
+                               1 << 40, S) == 2
+    assert lib.grouped_mlp_fwd(fake, fake, fake, fake, 1 << 40, 16, 2, 4, 256, 512, fake, fake, 1 << 40, fake,
+                               16, S) == 3
+    assert lib.grouped_mlp_bwd(fake, fake, 1 << 40, fake, 1 << 40, 16, 2, 4, 256, 512, fake, bad, fake, fake,
+                               fake, 1 << 40, S) == 1

@@ -1,0 +1,114 @@
+"""GPU parity of mxfp8_quantize with the oracle's quantiser: bytes and scales bit-exact."""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import moe_workloads as wl
+from oracle import moe as omoe
+from oracle import mxfp8 as omx
+from tests.util import f64, u8
+
+pytestmark = pytest.mark.gpu
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "mxfp8_blocks.txt")
+
+
+def _golden():
+    rows = []
+    for line in open(GOLDEN):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        name, vals, scale, codes = [f.strip() for f in line.split("|")]
+        v = np.zeros(32)
+        for it in vals.split(","):
+            p, x = it.split(":")
+            x = x.strip()
+            v[int(p)] = float(x.split("*2^")[0]) * math.ldexp(1.0, int(x.split("*2^")[1])) if "*2^" in x else float(x)
+        rows.append((name, v, int(scale, 16), {int(p): int(c, 16) for p, c in (i.split(":") for i in codes.split(","))}))
+    return rows
+
+
+def test_golden_blocks_on_gpu(gpu_lib):
+    """The hand-built blocks, quantised by the GPU (fp32 input), rowwise and colwise."""
+    blocks = _golden()
+    n = len(blocks)
+    src = np.zeros((max(32, n), 32), dtype=np.float32)
+    for i, (_, v, _, _) in enumerate(blocks):
+        src[i] = v
+    t = torch.from_numpy(src).cuda()
+    r, c = gpu_lib.mxfp8_quantize(t, layout=gpu_lib.SCALE_PLAIN)
+    codes = u8(r.data)
+    sc = u8(r.scale_plain())
+    for i, (name, v, scale, exp) in enumerate(blocks):
+        assert sc[i, 0] == scale, name
+        for p, cc in exp.items():
+            assert codes[i, p] == cc, (name, p, hex(codes[i, p]), hex(cc))
+    # colwise of the transposed input gives the same bytes
+    r2, c2 = gpu_lib.mxfp8_quantize(torch.from_numpy(np.ascontiguousarray(src.T)).cuda(), rowwise=False,
+                                    layout=gpu_lib.SCALE_PLAIN)
+    np.testing.assert_array_equal(u8(c2.data), codes)
+    np.testing.assert_array_equal(u8(c2.scale_plain()), sc)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("layout", [0, 1])
+@pytest.mark.parametrize("shape", [(256, 384), (384, 128), (128, 4096)])
+def test_quantize_matches_oracle(gpu_lib, dtype, layout, shape):
+    R, C = shape
+    x = wl.random_matrix(R, C, seed=R + C, dtype=torch.float32)
+    # widen the dynamic range: per-row powers of two from 2^-40 to 2^40
+    g = torch.Generator().manual_seed(1)
+    x = x * torch.exp2(torch.randint(-40, 40, (R, 1), generator=g).float())
+    x[3, :40] = 0.0                      # an all-zero block
+    x[5, 7] = -1e-30                     # tiny negative next to normal values
+    x = x.to(dtype)
+    r, c = gpu_lib.mxfp8_quantize(x.cuda(), layout=layout)
+    torch.cuda.synchronize()
+    qr, sr = omx.quantize_rowwise(f64(x))
+    qc, sc = omx.quantize_colwise_t(f64(x))
+    np.testing.assert_array_equal(u8(r.data), qr)
+    np.testing.assert_array_equal(u8(r.scale_plain()), sr)
+    np.testing.assert_array_equal(u8(c.data), qc)
+    np.testing.assert_array_equal(u8(c.scale_plain()), sc)
+
+
+def test_quantize_batched_weights(gpu_lib):
+    E, N, K = 3, 256, 384
+    W = wl.random_matrix(N, K, seed=9, std=0.02, batch=E)
+    r, c = gpu_lib.mxfp8_quantize(W.cuda())
+    torch.cuda.synchronize()
+    rd, rs = u8(r.data), u8(r.scale_plain())
+    cd, cs = u8(c.data), u8(c.scale_plain())
+    for e in range(E):
+        qr, sr = omx.quantize_rowwise(f64(W[e]))
+        qc, sc = omx.quantize_colwise_t(f64(W[e]))
+        np.testing.assert_array_equal(rd[e * N:(e + 1) * N], qr)
+        np.testing.assert_array_equal(rs[e * N:(e + 1) * N], sr)
+        np.testing.assert_array_equal(cd[e * K:(e + 1) * K], qc)
+        np.testing.assert_array_equal(cs[e * K:(e + 1) * K], sc)
+
+
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_permute_quantize_matches_oracle(gpu_lib, name):
+    """Fused gather + quantise of the routed activations: rowwise along H, colwise in
+    32-row blocks of each 128-aligned expert segment."""
+    cfg = wl.CONFIGS[name]
+    idx, probs = wl.make_routing(cfg)
+    x = wl.make_activations(cfg)
+    out = gpu_lib.moe_permute(idx.cuda(), probs.cuda(), cfg.E)
+    cap = gpu_lib.mxmoe_rows_capacity(cfg.T, cfg.k, cfg.E)
+    r, c = gpu_lib.mxfp8_quantize(x.cuda(), row_gather=out["token_of_row"], nrows=out["seg_off"][cfg.E:],
+                                  out_rows=cap)
+    torch.cuda.synchronize()
+    ro = omoe.route(idx.numpy(), cfg.E, align=128)
+    Mp = ro["Mp"]
+    Xp = omoe.permute_rows(f64(x), ro["token_of_row"])
+    qr, sr = omx.quantize_rowwise(Xp)
+    qc, sc = omoe.quantize_colwise_segments(Xp, ro["seg_off"], ro["m_splits"])
+    np.testing.assert_array_equal(u8(r.data)[:Mp], qr)
+    np.testing.assert_array_equal(u8(r.scale_plain())[:Mp], sr)
+    np.testing.assert_array_equal(u8(c.data)[:, :Mp], qc)
+    np.testing.assert_array_equal(u8(c.scale_plain())[:, :Mp // 32], sc)
