@@ -100,4 +100,4 @@ def test_unpermute_matches_oracle(gpu_lib, k, H):
     assert np.all(np.abs(got - want) <= ulp + 1e-30)
     # and bit-exact where the fp32 sum is exact (k <= 2 of bf16 values)
     if k <= 2:
-        np.testing.assert_array_equal(y.cpu(), torch.from_numpy(want).to(torch.bfloat16))
+        np.testing.assert_array_equal(got, f64(torch.from_numpy(want).to(torch.bfloat16)))
