@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""Benchmark of the MXFP8 grouped expert MLP (forward + backward) on B200.
+
+One step = one pass of the whole hot path over one batch: MXFP8 quantisation of W1
+and W2, routing, permute + quantise of x, fc1 grouped GEMM with the fused
+SwiGLU x prob -> MXFP8 epilogue, fc2 grouped GEMM, combine, then the backward
+(permute + quantise of dy, fc2 data-gradient GEMM with the fused SwiGLU backward,
+dprob reduction, fc2 and fc1 weight-gradient GEMMs, fc1 data-gradient GEMM, combine).
+
+Default workload: the Mixtral-8x7B-shaped layer (8192 tokens, hidden 4096, FFN 14336,
+8 experts, top-2). Prints one JSON line (rank 0). `--impl reference` times the fp64
+CPU oracle on a bounded sample of the same workload instead.
+
+Multi-GPU (`torchrun ... bench.py --gpus N`): independent replicas, one per GPU (the
+path has no exchange step on one node without expert parallelism): weak scaling,
+timing = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "grouped-MLP fwd+bwd TFLOP/s & tokens/s on 1 B200; % of MXFP8 peak / HBM BW"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 4.5 / 2.25     # nominal dense ratio (MXFP8 / bf16) on B200
+SPEC_FP8_TFLOPS = 4500.0
+GEMM_FLOP_FACTOR = {"fc1_swiglu": 4, "fc2": 2, "fc2_dgrad_swiglu_bwd": 2, "fc2_wgrad": 2, "fc1_dgrad": 4,
+                    "fc1_wgrad": 4}     # x M*H*F
+GEMM_KERNEL_SOURCES = ["mxfp8_grouped_gemm_moe_b200/csrc/gemm.cu", "mxfp8_grouped_gemm_moe_b200/csrc/ptx_sm100.cuh",
+                       "mxfp8_grouped_gemm_moe_b200/csrc/mxmoe_device.cuh"]
+QUANT_KERNEL_SOURCES = ["mxfp8_grouped_gemm_moe_b200/csrc/quantize.cu",
+                        "mxfp8_grouped_gemm_moe_b200/csrc/mxmoe_device.cuh"]
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["mxmoe", "reference"], default="mxmoe")
+    p.add_argument("--config", default="mixtral", help="tiny | small | mixtral | mixtral_zipf | genomics")
+    p.add_argument("--tokens", type=int, default=0, help="override the token count (profiling runs)")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-rows", type=int, default=512, help="routed rows in the CPU oracle sample")
+    p.add_argument("--cpu-fslice", type=int, default=1024, help="FFN columns in the CPU oracle sample")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel_key, paths, units):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel source (else None). The summary stores bytes per unit of work."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    ent = d.get(kernel_key)
+    if not ent or ent.get("source_hash") != source_hash(paths):
+        return None
+    return float(ent["bytes_per_unit"]) * units
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"mxmoe_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]), power=float(f[3]), hw=f[5], hwt=f[6], swt=f[7],
+                                 pcap=f[8]))
+            except ValueError:
+                continue
+        os.remove(self.path)
+        if not rows:
+            return None
+        pmax = max(r["power"] for r in rows)
+        load = [r for r in rows if r["power"] >= 0.5 * pmax] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(load), "power_w_max": pmax}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1:
+        import torch
+        import torch.distributed as dist
+        lr = int(os.environ.get("LOCAL_RANK", "0"))
+        if args.impl == "mxmoe":
+            torch.cuda.set_device(lr)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", lr))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=600))
+        return dist, dist.get_rank(), ws, lr
+    return None, 0, 1, 0
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks(dist, v):
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- CPU oracle sample
+def _keep_freed_memory():
+    """glibc: serve large numpy temporaries from the heap and keep freed memory, so the
+    CPU baseline is not dominated by page faults on fresh mmap'd buffers."""
+    try:
+        import ctypes
+        libc = ctypes.CDLL("libc.so.6")
+        libc.mallopt(-3, 1 << 30)        # M_MMAP_THRESHOLD
+        libc.mallopt(-1, 2 ** 31 - 1)    # M_TRIM_THRESHOLD
+    except OSError:
+        pass
+
+
+def oracle_sample(cfg, rows, f_slice):
+    """The fp64 oracle (as it stands) on a bounded sample of the workload: the first
+    `rows` tokens routed to expert 0 and the first `f_slice` FFN columns of that
+    expert (gate rows [0, f), up rows [F, F+f), W2 columns [0, f)), forward + backward.
+    Every step of the path scales linearly in rows and in f, so the sample's
+    throughput stands for the workload's. Returns (seconds, flops, description, rows)."""
+    import numpy as np
+
+    import moe_workloads as wl
+    from oracle import moe as omoe
+
+    _keep_freed_memory()
+    idx, probs = wl.make_routing(cfg)
+    sel = (idx == 0).nonzero()[:rows]
+    toks, slots = sel[:, 0], sel[:, 1]
+    M = len(toks)
+    fs = min(f_slice, cfg.F)
+    x = wl.make_activations(cfg)[toks]
+    dy = wl.make_grad_output(cfg)[toks]
+    p = probs[toks, slots].reshape(M, 1)
+    W1, W2 = wl.make_expert_weights(cfg, 0)
+    W1s = np.concatenate([W1[:fs].float().numpy(), W1[cfg.F:cfg.F + fs].float().numpy()]).astype(np.float64)
+    W2s = W2[:, :fs].float().numpy().astype(np.float64)
+    f = lambda t: t.float().numpy().astype(np.float64)  # noqa: E731
+    xs, dys, ps = f(x), f(dy), f(p)
+    one = np.zeros((M, 1), dtype=np.int64)
+    t0 = time.perf_counter()
+    _, saved = omoe.mlp_fwd(xs, one, ps, W1s[None], W2s[None])
+    omoe.mlp_bwd(dys, saved, ps, W1s[None], W2s[None])
+    dt = time.perf_counter() - t0
+    desc = (f"expert 0 of the {cfg.name} workload: its first {M} routed rows x H={cfg.H} x the first {fs} of "
+            f"F={cfg.F} FFN columns (weights sliced accordingly); fp64 numpy oracle forward+backward incl. "
+            f"MXFP8 quantisation of weights and activations")
+    return dt, 18.0 * M * cfg.H * fs, desc, M
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args, cfg, dist, rank, world):
+    if rank != 0:
+        return
+    times, flops, desc, M = [], 0.0, "", 0
+    for i in range(args.warmup + args.steps):
+        dt, flops, desc, M = oracle_sample(cfg, args.cpu_rows, args.cpu_fslice)
+        if i >= args.warmup:
+            times.append(dt)
+    sec = sum(times) / len(times)
+    tflops = flops / sec / 1e12
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_json(cfg, world),
+            "tokens_per_s": tflops * 1e12 / (18.0 * cfg.k * cfg.H * cfg.F),
+            "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_json(cfg, world):
+    return {"workload": f"{cfg.name}: MoE expert MLP layer, {cfg.T} tokens, hidden {cfg.H}, FFN {cfg.F}, "
+                        f"{cfg.E} experts, top-{cfg.k}, fwd+bwd",
+            "tokens": cfg.T, "hidden": cfg.H, "ffn": cfg.F, "experts": cfg.E, "top_k": cfg.k,
+            "routing": cfg.routing, "seed": cfg.seed, "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+            "l2": "inputs larger than L2 (weights alone are several GB); no flush needed",
+            "flops_per_step": cfg.fwdbwd_flops}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_gpu(args, cfg, dist, rank, world, local_rank):
+    import torch
+
+    import moe_workloads as wl
+    import mxfp8_grouped_gemm_moe_b200 as mx
+
+    mx.load()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    # inputs: routing from the workload recipe (CPU, seeded); dense tensors drawn with a
+    # seeded CUDA generator (same distributions as the recipe; resident in HBM)
+    idx_h, probs_h = wl.make_routing(cfg)
+    g = torch.Generator(device=dev)
+    g.manual_seed(cfg.seed)
+    W1 = (torch.randn((cfg.E, 2 * cfg.F, cfg.H), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    W2 = (torch.randn((cfg.E, cfg.H, cfg.F), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    x = torch.randn((cfg.T, cfg.H), generator=g, device=dev).to(torch.bfloat16)
+    dy = torch.randn((cfg.T, cfg.H), generator=g, device=dev).to(torch.bfloat16)
+    idx, probs = idx_h.to(dev), probs_h.to(dev)
+    layer = mx.GroupedMLP(cfg.T, cfg.k, cfg.E, cfg.H, cfg.F, device=dev)
+    y = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
+    dx = torch.empty_like(y)
+    dW1 = torch.empty((cfg.E, 2 * cfg.F, cfg.H), dtype=torch.float32, device=dev)
+    dW2 = torch.empty((cfg.E, cfg.H, cfg.F), dtype=torch.float32, device=dev)
+    dprobs = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        layer.quantize_weights(W1, W2)
+        layer.forward(x, idx, probs, y)
+        layer.backward(dy, dx, dW1, dW2, dprobs)
+
+    mx.mxmoe_clear_device_status()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- device-resident timed region (stage events on, clocks sampled)
+    clocks = ClockSampler(local_rank)
+    mx.mxmoe_profile_enable(64 * (args.steps + 1))
+    mx.mxmoe_profile_read()
+    clocks.start()
+    barrier(dist)
+    torch.cuda.synchronize()
+    n0 = mx.mxmoe_launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(dist)
+    launches = mx.mxmoe_launch_count() - n0
+    ms = ev0.elapsed_time(ev1) / args.steps
+    stages = mx.mxmoe_profile_read()
+    mx.mxmoe_profile_disable()
+    ms = max_over_ranks(dist, ms)
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+        x_h, dy_h, idx_p, probs_p = pin(x), pin(dy), pin(idx), pin(probs)
+        y_h, dx_h, dp_h = pin(y), pin(dx), pin(dprobs)
+        h2d = sum(t.numel() * t.element_size() for t in (x_h, dy_h, idx_p, probs_p))
+        d2h = sum(t.numel() * t.element_size() for t in (y_h, dx_h, dp_h))
+
+        def e2e_step():
+            x.copy_(x_h, non_blocking=True)
+            idx.copy_(idx_p, non_blocking=True)
+            probs.copy_(probs_p, non_blocking=True)
+            dy.copy_(dy_h, non_blocking=True)
+            step()
+            y_h.copy_(y, non_blocking=True)
+            dx_h.copy_(dx, non_blocking=True)
+            dp_h.copy_(dprobs, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(dist)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(dist)
+        ems = max_over_ranks(dist, e0.elapsed_time(e1) / args.steps)
+        e2e = {"value": world * cfg.fwdbwd_flops / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems,
+               "tokens_per_s": world * cfg.T / (ems * 1e-3)}
+    clk = clocks.stop()
+
+    st, where = mx.mxmoe_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} (site {where}) after the benchmark")
+
+    # ---- per-stage times and rooflines
+    peaks, peak_kind = load_peaks()
+    MHF = float(cfg.M) * cfg.H * cfg.F
+    per = {}
+    for name, t in stages:
+        per.setdefault(name, []).append(t)
+    stage_json = {}
+    hbm_bytes = {
+        "quant_x": cfg.T * cfg.H * 2 + 2 * (cfg.M * cfg.H + cfg.M * cfg.H / 32),
+        "quant_dy": cfg.T * cfg.H * 2 + 2 * (cfg.M * cfg.H + cfg.M * cfg.H / 32),
+        "combine": cfg.M * cfg.H * 2 + cfg.T * cfg.H * 2,
+        "combine_dx": cfg.M * cfg.H * 2 + cfg.T * cfg.H * 2,
+        "quant_w1": cfg.E * 2 * cfg.F * cfg.H * (2 + 2 * (1 + 1 / 32)),
+        "quant_w2": cfg.E * cfg.F * cfg.H * (2 + 2 * (1 + 1 / 32)),
+    }
+    fp8_peak = peaks["bf16_tflops_sustained"] * FP8_OVER_BF16
+    for name, ts in per.items():
+        a = sum(ts) / len(ts)
+        ent = {"ms": a, "launches": len(ts)}
+        if name in GEMM_FLOP_FACTOR:
+            tf = GEMM_FLOP_FACTOR[name] * MHF / (a * 1e-3) / 1e12
+            ent.update(tflops=tf, frac_of_measured=tf / fp8_peak, frac_of_spec=tf / SPEC_FP8_TFLOPS)
+        elif name in hbm_bytes:
+            gbs = hbm_bytes[name] / (a * 1e-3) / 1e9
+            ent.update(gbs=gbs, frac_of_measured=gbs / peaks["hbm_gbs"])
+        stage_json[name] = ent
+    gemm_names = [n for n in stage_json if n in GEMM_FLOP_FACTOR]
+    dom = max(gemm_names, key=lambda n: stage_json[n]["ms"])
+    dom_units = GEMM_FLOP_FACTOR[dom] * MHF
+    roofline = {"bound": "tensor", "kernel": f"mxgemm_kernel ({dom})", "achieved": stage_json[dom]["tflops"],
+                "peak": fp8_peak, "unit": "TFLOP/s", "frac": stage_json[dom]["tflops"] / fp8_peak,
+                "peak_source": f"{peak_kind} bf16 sustained x {FP8_OVER_BF16:g} (nominal MXFP8/bf16 ratio)",
+                "frac_of_spec_4500": stage_json[dom]["tflops"] / SPEC_FP8_TFLOPS,
+                "traffic": load_traffic(f"{dom}:{cfg.name}", GEMM_KERNEL_SOURCES, 1.0)}
+    q = stage_json.get("quant_x", {})
+    roofline_hbm = {"bound": "hbm", "kernel": "mxfp8_quantize_kernel (permute + quantise x)",
+                    "achieved": q.get("gbs"), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": (q.get("gbs") or 0) / peaks["hbm_gbs"], "peak_source": peak_kind,
+                    "traffic": load_traffic(f"quant_x:{cfg.name}", QUANT_KERNEL_SOURCES, 1.0)}
+    gemm_ms = sum(stage_json[n]["ms"] for n in gemm_names)
+    value = world * cfg.fwdbwd_flops / (ms * 1e-3) / 1e12
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "mxfp8-e4m3 (fp32 accumulate)", "data": "synthetic",
+            "config": config_json(cfg, world),
+            "tokens_per_s": world * cfg.T / (ms * 1e-3),
+            "gemm_tflops": (18.0 * MHF) / (gemm_ms * 1e-3) / 1e12,
+            "gemm_frac_of_measured_fp8": (18.0 * MHF) / (gemm_ms * 1e-3) / 1e12 / fp8_peak,
+            "roofline": roofline, "roofline_hbm": roofline_hbm, "stages": stage_json,
+            "gpu_launches": launches, "e2e": e2e, "clocks": clk}
+    return line
+
+
+def main():
+    args = parse_args()
+    dist, rank, world, local_rank = dist_setup(args)
+    import dataclasses
+
+    import moe_workloads as wl
+    cfg = wl.CONFIGS[args.config]
+    if args.tokens:
+        cfg = dataclasses.replace(cfg, T=args.tokens)
+    try:
+        if args.impl == "reference":
+            run_reference(args, cfg, dist, rank, world)
+            return
+        line = run_gpu(args, cfg, dist, rank, world, local_rank)
+        if rank == 0:
+            if not args.no_cpu_baseline and world == 1:
+                dt, flops, desc, M = oracle_sample(cfg, args.cpu_rows, args.cpu_fslice)
+                line["cpu_baseline"] = {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+                                        "kind": "oracle", "sample": desc, "seconds": dt,
+                                        "tokens_per_s": flops / dt / (18.0 * cfg.k * cfg.H * cfg.F)}
+            print(json.dumps(line), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -264,6 +264,39 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
                              float* dW1_dev, float* dW2_dev, float* dprobs_dev, void* ws_dev, size_t ws_bytes,
                              void* stream);
 
+/* ------------------------------------------------------------------ instrumentation */
+
+/* Stage tags reported by mxmoe_profile_read (one per enqueued stage). */
+#define MXMOE_STAGE_ROUTE 1          /* moe_permute (3 small kernels) */
+#define MXMOE_STAGE_QUANT_X 2        /* permute + quantise x (rowwise + colwise) */
+#define MXMOE_STAGE_FC1_SWIGLU 3     /* fc1 grouped GEMM + SwiGLU x prob -> MXFP8 epilogue */
+#define MXMOE_STAGE_FC2 4            /* fc2 grouped GEMM */
+#define MXMOE_STAGE_COMBINE 5        /* moe_unpermute of y */
+#define MXMOE_STAGE_QUANT_W1 6       /* W1 rowwise + colwise */
+#define MXMOE_STAGE_QUANT_W2 7       /* W2 rowwise + colwise */
+#define MXMOE_STAGE_QUANT_DY 8       /* permute + quantise dy */
+#define MXMOE_STAGE_FC2_DGRAD 9      /* fc2 data-gradient GEMM + SwiGLU backward epilogue */
+#define MXMOE_STAGE_DPROB 10         /* dprob reduction */
+#define MXMOE_STAGE_FC2_WGRAD 11     /* fc2 weight-gradient GEMM */
+#define MXMOE_STAGE_FC1_DGRAD 12     /* fc1 data-gradient GEMM */
+#define MXMOE_STAGE_FC1_WGRAD 13     /* fc1 weight-gradient GEMM */
+#define MXMOE_STAGE_COMBINE_DX 14    /* moe_unpermute of dx */
+#define MXMOE_STAGE_GEMM 15          /* standalone grouped_gemm_mxfp8 */
+#define MXMOE_STAGE_WGRAD 16         /* standalone grouped_gemm_mxfp8_wgrad */
+#define MXMOE_STAGE_QUANT 17         /* standalone mxfp8_quantize */
+
+/* Host-side stage timing, off by default: while enabled, every stage the library
+ * enqueues is bracketed by two CUDA events recorded on that stage's stream (up to
+ * max_stages stages; later ones are not recorded). Creates 2*max_stages events on the
+ * current device. Not thread-safe; for benchmarks. */
+mxmoe_status mxmoe_profile_enable(int32_t max_stages);
+mxmoe_status mxmoe_profile_disable(void);
+/* Waits for the recorded events, writes up to `cap` (tag, milliseconds) pairs, returns
+ * how many stages were recorded (and clears the record). */
+int32_t mxmoe_profile_read(int32_t* tags_host, float* ms_host, int32_t cap);
+/* Number of CUDA kernels this library has launched since it was loaded. */
+int64_t mxmoe_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -168,3 +168,14 @@ def random_matrix(rows, cols, seed, std=1.0, dtype=torch.bfloat16, batch=None):
     g = _gen(seed, 9)
     shape = (rows, cols) if batch is None else (batch, rows, cols)
     return _randn(shape, std, g, dtype=dtype)
+
+
+def make_expert_weights(cfg: MoEConfig, e: int):
+    """Expert e's (W1[e], W2[e]), identical to the slices of make_weights(cfg), drawn
+    without materialising the other experts (earlier experts are drawn and dropped)."""
+    g1, g2 = _gen(cfg.seed, 3), _gen(cfg.seed, 4)
+    w1 = w2 = None
+    for i in range(e + 1):
+        w1 = (torch.randn((1, 2 * cfg.F, cfg.H), generator=g1) * 0.02).to(torch.bfloat16)
+        w2 = (torch.randn((1, cfg.H, cfg.F), generator=g2) * 0.02).to(torch.bfloat16)
+    return w1[0], w2[0]

@@ -68,7 +68,15 @@ _SIGNATURES = {
     "grouped_mlp_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32]),
     "grouped_mlp_fwd": (_I32, [_P, _P, _P, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _P, _P, _SZ, _P, _SZ, _P]),
     "grouped_mlp_bwd": (_I32, [_P, _P, _SZ, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
+    "mxmoe_profile_enable": (_I32, [_I32]),
+    "mxmoe_profile_disable": (_I32, []),
+    "mxmoe_profile_read": (_I32, [ctypes.POINTER(_I32), ctypes.POINTER(ctypes.c_float), _I32]),
+    "mxmoe_launch_count": (_I64, []),
 }
+
+STAGE_NAMES = {1: "route", 2: "quant_x", 3: "fc1_swiglu", 4: "fc2", 5: "combine", 6: "quant_w1", 7: "quant_w2",
+               8: "quant_dy", 9: "fc2_dgrad_swiglu_bwd", 10: "dprob", 11: "fc2_wgrad", 12: "fc1_dgrad",
+               13: "fc1_wgrad", 14: "combine_dx", 15: "gemm", 16: "wgrad", 17: "quant"}
 
 
 def load(path: str | None = None):
@@ -296,3 +304,24 @@ def grouped_mlp_bwd(dy, saved, wq, T, k, E, H, F, ws, dx=None, dW1=None, dW2=Non
                                 _ptr(dW1), _ptr(dW2), _ptr(dprobs), _ptr(ws), ws.numel(), _stream())
     _check("grouped_mlp_bwd", st)
     return dx, dW1, dW2, dprobs
+
+
+# ----------------------------------------------------------------------------- instrumentation
+def mxmoe_profile_enable(max_stages=4096):
+    _check("mxmoe_profile_enable", load().mxmoe_profile_enable(max_stages))
+
+
+def mxmoe_profile_disable():
+    _check("mxmoe_profile_disable", load().mxmoe_profile_disable())
+
+
+def mxmoe_profile_read(cap=4096):
+    """-> list of (stage name, milliseconds) for the stages recorded since the last read."""
+    tags = (_I32 * cap)()
+    ms = (ctypes.c_float * cap)()
+    n = load().mxmoe_profile_read(tags, ms, cap)
+    return [(STAGE_NAMES.get(tags[i], str(tags[i])), ms[i]) for i in range(min(n, cap))]
+
+
+def mxmoe_launch_count():
+    return int(load().mxmoe_launch_count())

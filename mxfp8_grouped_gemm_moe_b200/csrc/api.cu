@@ -156,6 +156,38 @@ GemmArgs gemm_base(int mode, const mxmoe_mxfp8& A, const mxmoe_mxfp8& B, const i
   return g;
 }
 
+
+// ---------------------------------------------------------------- stage timing
+// Host-side only: CUDA events around each stage, when enabled. Only the outermost
+// stage scope records (a fused call's inner entry points are attributed to it).
+struct Profiler {
+  bool on = false;
+  int cap = 0, n = 0, depth = 0;
+  cudaEvent_t* ev = nullptr;
+  int32_t* tags = nullptr;
+};
+Profiler g_prof;
+
+struct StageScope {
+  cudaStream_t st;
+  bool rec = false;
+  StageScope(int32_t tag, cudaStream_t s) : st(s) {
+    if (g_prof.on && g_prof.depth == 0 && g_prof.n < g_prof.cap) {
+      cudaEventRecord(g_prof.ev[2 * g_prof.n], st);
+      g_prof.tags[g_prof.n] = tag;
+      rec = true;
+    }
+    ++g_prof.depth;
+  }
+  ~StageScope() {
+    --g_prof.depth;
+    if (rec) {
+      cudaEventRecord(g_prof.ev[2 * g_prof.n + 1], st);
+      ++g_prof.n;
+    }
+  }
+};
+
 }  // namespace
 
 // ============================================================================ C ABI
@@ -209,6 +241,7 @@ mxmoe_status moe_permute(const int32_t* topk_idx_dev, const float* probs_dev, in
     return MXMOE_ERR_INVALID_ARG;
   if (prob_of_row_dev && T > 0 && !probs_dev) return MXMOE_ERR_INVALID_ARG;
   if (ws_bytes < moe_permute_workspace_size(T, k, E)) return MXMOE_ERR_WORKSPACE_TOO_SMALL;
+  StageScope sc(MXMOE_STAGE_ROUTE, S(stream));
   return cuda_status(launch_route(topk_idx_dev, probs_dev, T, k, E, m_splits_dev, seg_off_dev, row_of_slot_dev,
                                   token_of_row_dev, prob_of_row_dev, ws_dev, S(stream)));
 }
@@ -219,6 +252,7 @@ mxmoe_status moe_unpermute(const void* y_perm_dev, const int32_t* row_of_slot_de
   if (T == 0) return MXMOE_OK;
   if (!y_perm_dev || !row_of_slot_dev || !y_dev || !aligned16(y_perm_dev) || !aligned16(y_dev))
     return MXMOE_ERR_INVALID_ARG;
+  StageScope sc(MXMOE_STAGE_COMBINE, S(stream));
   return cuda_status(launch_unpermute(y_perm_dev, row_of_slot_dev, T, k, H, y_dev, S(stream)));
 }
 
@@ -259,6 +293,7 @@ mxmoe_status mxfp8_quantize(const void* src_dev, int32_t src_dtype, int64_t batc
   a.col_data = out_colT ? out_colT->data : nullptr;
   a.col_sf = out_colT ? out_colT->scale : nullptr;
   a.col_layout = out_colT ? out_colT->scale_layout : 0;
+  StageScope sc(MXMOE_STAGE_QUANT, S(stream));
   return cuda_status(launch_quantize(a, S(stream)));
 }
 
@@ -278,6 +313,7 @@ mxmoe_status grouped_gemm_mxfp8(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, cons
   g.c = C_dev;
   g.c_dtype = c_dtype;
   g.ldc = ldc;
+  StageScope sc(MXMOE_STAGE_GEMM, S(stream));
   return cuda_status(launch_gemm(g, S(stream)));
 }
 
@@ -293,6 +329,7 @@ mxmoe_status grouped_gemm_mxfp8_wgrad(const mxmoe_mxfp8* At, const mxmoe_mxfp8* 
   g.c = C_dev;
   g.c_dtype = MXMOE_DTYPE_F32;
   g.ldc = Bt->rows;
+  StageScope sc(MXMOE_STAGE_WGRAD, S(stream));
   return cuda_status(launch_gemm(g, S(stream)));
 }
 
@@ -317,9 +354,14 @@ mxmoe_status mxmoe_weights_quantize(const void* W1_dev, const void* W2_dev, int3
   mxmoe_mxfp8 w1c = mk(b, L.d[1], L.s[1], L.rows[1], L.cols[1]);
   mxmoe_mxfp8 w2r = mk(b, L.d[2], L.s[2], L.rows[2], L.cols[2]);
   mxmoe_mxfp8 w2c = mk(b, L.d[3], L.s[3], L.rows[3], L.cols[3]);
-  mxmoe_status s = mxfp8_quantize(W1_dev, MXMOE_DTYPE_BF16, E, 2 * (int64_t)F, H, nullptr, nullptr, 2 * (int64_t)F,
-                                  &w1r, &w1c, stream);
+  mxmoe_status s;
+  {
+    StageScope sc(MXMOE_STAGE_QUANT_W1, S(stream));
+    s = mxfp8_quantize(W1_dev, MXMOE_DTYPE_BF16, E, 2 * (int64_t)F, H, nullptr, nullptr, 2 * (int64_t)F, &w1r,
+                       &w1c, stream);
+  }
   if (s != MXMOE_OK) return s;
+  StageScope sc(MXMOE_STAGE_QUANT_W2, S(stream));
   return mxfp8_quantize(W2_dev, MXMOE_DTYPE_BF16, E, H, F, nullptr, nullptr, H, &w2r, &w2c, stream);
 }
 
@@ -363,13 +405,21 @@ mxmoe_status grouped_mlp_fwd(const void* x_dev, const int32_t* topk_idx_dev, con
   float* por = reinterpret_cast<float*>(sv + SL.off[MXMOE_SAVED_PROB_OF_ROW]);
 
   // 1. route
-  cudaError_t e = launch_route(topk_idx_dev, probs_dev, T, k, E, m_splits, seg_off, ros, tor, por, ws + W.route, st);
+  cudaError_t e;
+  {
+    StageScope sc(MXMOE_STAGE_ROUTE, st);
+    e = launch_route(topk_idx_dev, probs_dev, T, k, E, m_splits, seg_off, ros, tor, por, ws + W.route, st);
+  }
   if (e != cudaSuccess) return MXMOE_ERR_CUDA;
   if (T == 0) return MXMOE_OK;
   // 2. permute + quantise x (rowwise for fc1, colwise saved for fc1 wgrad)
   mxmoe_mxfp8 x_row = mk(ws, W.x_row, W.x_row_sf, cap, H);
   mxmoe_mxfp8 x_col = mk(sv, SL.off[MXMOE_SAVED_X_COLT], SL.off[MXMOE_SAVED_X_COLT_SF], H, cap);
-  mxmoe_status s = mxfp8_quantize(x_dev, MXMOE_DTYPE_BF16, 1, T, H, tor, seg_off + E, cap, &x_row, &x_col, stream);
+  mxmoe_status s;
+  {
+    StageScope sc(MXMOE_STAGE_QUANT_X, st);
+    s = mxfp8_quantize(x_dev, MXMOE_DTYPE_BF16, 1, T, H, tor, seg_off + E, cap, &x_row, &x_col, stream);
+  }
   if (s != MXMOE_OK) return s;
   // 3. fc1 + SwiGLU x prob -> Z (MXFP8 row + colT), G/U saved
   mxmoe_mxfp8 w1r = mk(wq, WL.d[0], WL.s[0], WL.rows[0], WL.cols[0]);
@@ -384,13 +434,21 @@ mxmoe_status grouped_mlp_fwd(const void* x_dev, const int32_t* topk_idx_dev, con
   g.z_colT = sv + SL.off[MXMOE_SAVED_Z_COLT];
   g.z_colT_sf = sv + SL.off[MXMOE_SAVED_Z_COLT_SF];
   g.gu = reinterpret_cast<uint16_t*>(sv + SL.off[MXMOE_SAVED_GU]);
-  if (launch_gemm(g, st) != cudaSuccess) return MXMOE_ERR_CUDA;
+  {
+    StageScope sc(MXMOE_STAGE_FC1_SWIGLU, st);
+    e = launch_gemm(g, st);
+  }
+  if (e != cudaSuccess) return MXMOE_ERR_CUDA;
   // 4. fc2 -> Yp bf16
   mxmoe_mxfp8 z_row = mk(ws, W.z_row, W.z_row_sf, cap, F);
   mxmoe_mxfp8 w2r = mk(wq, WL.d[2], WL.s[2], WL.rows[2], WL.cols[2]);
-  s = grouped_gemm_mxfp8(&z_row, &w2r, seg_off, E, H, F, ws + W.y_perm, MXMOE_DTYPE_BF16, H, stream);
+  {
+    StageScope sc(MXMOE_STAGE_FC2, st);
+    s = grouped_gemm_mxfp8(&z_row, &w2r, seg_off, E, H, F, ws + W.y_perm, MXMOE_DTYPE_BF16, H, stream);
+  }
   if (s != MXMOE_OK) return s;
   // 5. combine
+  StageScope sc(MXMOE_STAGE_COMBINE, st);
   return moe_unpermute(ws + W.y_perm, ros, T, k, H, y_dev, stream);
 }
 
@@ -425,6 +483,7 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
   mxmoe_mxfp8 dy_col = mk(ws, W.dy_colT, W.dy_colT_sf, H, cap);
   mxmoe_status s;
   if (T > 0) {
+    StageScope sc(MXMOE_STAGE_QUANT_DY, st);
     s = mxfp8_quantize(dy_dev, MXMOE_DTYPE_BF16, 1, T, H, tor, seg_off + E, cap, &dy_row, &dy_col, stream);
     if (s != MXMOE_OK) return s;
   }
@@ -443,20 +502,28 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
     g.dgu_colT = ws + W.dgu_colT;
     g.dgu_colT_sf = ws + W.dgu_colT_sf;
     g.dprob_part = reinterpret_cast<float*>(ws + W.dprob_part);
+    StageScope sc(MXMOE_STAGE_FC2_DGRAD, st);
     if (T > 0 && launch_gemm(g, st) != cudaSuccess) return MXMOE_ERR_CUDA;
   }
   // 3. dprobs
-  if (launch_dprob_reduce(reinterpret_cast<const float*>(ws + W.dprob_part), F / 128, ros, (int64_t)T * k,
-                          dprobs_dev, st) != cudaSuccess)
-    return MXMOE_ERR_CUDA;
+  {
+    StageScope sc(MXMOE_STAGE_DPROB, st);
+    if (launch_dprob_reduce(reinterpret_cast<const float*>(ws + W.dprob_part), F / 128, ros, (int64_t)T * k,
+                            dprobs_dev, st) != cudaSuccess)
+      return MXMOE_ERR_CUDA;
+  }
   // 4. fc2 wgrad: dW2[e] = dYp_e^T . Z_e
   mxmoe_mxfp8 z_col = mk(sv, SL.off[MXMOE_SAVED_Z_COLT], SL.off[MXMOE_SAVED_Z_COLT_SF], F, cap);
-  s = grouped_gemm_mxfp8_wgrad(&dy_col, &z_col, seg_off, E, dW2_dev, stream);
+  {
+    StageScope sc(MXMOE_STAGE_FC2_WGRAD, st);
+    s = grouped_gemm_mxfp8_wgrad(&dy_col, &z_col, seg_off, E, dW2_dev, stream);
+  }
   if (s != MXMOE_OK) return s;
   // 5. fc1 dgrad: dXp = dGU . W1 (contract 2F)
   mxmoe_mxfp8 dgu_row = mk(ws, W.dgu_row, W.dgu_row_sf, cap, 2 * (int64_t)F);
   mxmoe_mxfp8 w1c = mk(wq, WL.d[1], WL.s[1], WL.rows[1], WL.cols[1]);
   if (T > 0) {
+    StageScope sc(MXMOE_STAGE_FC1_DGRAD, st);
     s = grouped_gemm_mxfp8(&dgu_row, &w1c, seg_off, E, H, 2 * (int64_t)F, ws + W.dx_perm, MXMOE_DTYPE_BF16, H,
                            stream);
     if (s != MXMOE_OK) return s;
@@ -464,10 +531,52 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
   // 6. fc1 wgrad: dW1[e] = dGU_e^T . Xp_e
   mxmoe_mxfp8 dgu_col = mk(ws, W.dgu_colT, W.dgu_colT_sf, 2 * (int64_t)F, cap);
   mxmoe_mxfp8 x_col = mk(sv, SL.off[MXMOE_SAVED_X_COLT], SL.off[MXMOE_SAVED_X_COLT_SF], H, cap);
-  s = grouped_gemm_mxfp8_wgrad(&dgu_col, &x_col, seg_off, E, dW1_dev, stream);
+  {
+    StageScope sc(MXMOE_STAGE_FC1_WGRAD, st);
+    s = grouped_gemm_mxfp8_wgrad(&dgu_col, &x_col, seg_off, E, dW1_dev, stream);
+  }
   if (s != MXMOE_OK) return s;
   // 7. combine dX
+  StageScope sc(MXMOE_STAGE_COMBINE_DX, st);
   return moe_unpermute(ws + W.dx_perm, ros, T, k, H, dx_dev, stream);
 }
+
+mxmoe_status mxmoe_profile_enable(int32_t max_stages) {
+  if (max_stages <= 0 || g_prof.on) return MXMOE_ERR_INVALID_ARG;
+  g_prof.ev = new cudaEvent_t[2 * (size_t)max_stages];
+  g_prof.tags = new int32_t[max_stages];
+  for (int i = 0; i < 2 * max_stages; ++i)
+    if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) return MXMOE_ERR_CUDA;
+  g_prof.cap = max_stages;
+  g_prof.n = 0;
+  g_prof.depth = 0;
+  g_prof.on = true;
+  return MXMOE_OK;
+}
+
+mxmoe_status mxmoe_profile_disable(void) {
+  if (!g_prof.ev) return MXMOE_OK;
+  for (int i = 0; i < 2 * g_prof.cap; ++i) cudaEventDestroy(g_prof.ev[i]);
+  delete[] g_prof.ev;
+  delete[] g_prof.tags;
+  g_prof = Profiler();
+  return MXMOE_OK;
+}
+
+int32_t mxmoe_profile_read(int32_t* tags_host, float* ms_host, int32_t cap) {
+  if (!g_prof.on) return 0;
+  const int n = g_prof.n;
+  for (int i = 0; i < n && i < cap; ++i) {
+    cudaEventSynchronize(g_prof.ev[2 * i + 1]);
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]);
+    if (tags_host) tags_host[i] = g_prof.tags[i];
+    if (ms_host) ms_host[i] = ms;
+  }
+  g_prof.n = 0;
+  return n;
+}
+
+int64_t mxmoe_launch_count(void) { return g_launch_count.load(); }
 
 }  // extern "C"

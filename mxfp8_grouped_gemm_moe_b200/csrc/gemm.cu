@@ -570,6 +570,7 @@ static cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb, con
   const int nsm = gemm_num_sms();
   const int grid = (int)(tiles_ub < nsm ? (tiles_ub > 0 ? tiles_ub : 1) : nsm);
   mxgemm_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(ma, mb, g);
+  ++g_launch_count;
   return cudaGetLastError();
 }
 

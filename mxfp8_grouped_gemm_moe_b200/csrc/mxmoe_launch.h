@@ -2,12 +2,16 @@
 #pragma once
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 
 #include "../../include/mxmoe.h"
 
 namespace mxmoe {
+
+// Kernels launched by this library since load (reported by mxmoe_launch_count).
+inline std::atomic<int64_t> g_launch_count{0};
 
 // ---------------------------------------------------------------- routing / combine
 size_t route_workspace_bytes(int T, int k, int E);

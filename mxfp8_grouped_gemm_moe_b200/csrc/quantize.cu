@@ -125,6 +125,7 @@ static cudaError_t launch_q(const QuantArgs& a, cudaStream_t st) {
             (unsigned)a.batch);
   if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
   mxfp8_quantize_kernel<T><<<grid, kQThreads, smem, st>>>(a);
+  ++g_launch_count;
   return cudaGetLastError();
 }
 

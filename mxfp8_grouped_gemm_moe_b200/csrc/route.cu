@@ -191,6 +191,7 @@ cudaError_t launch_route(const int32_t* idx, const float* probs, int T, int k, i
   if (nb > 0)
     route_scatter_kernel<<<nb, kRouteTokensPerBlock, 0, st>>>(idx, probs, T, k, E, base, row_of_slot, token_of_row,
                                                               prob_of_row);
+  g_launch_count += (nb > 0) ? 3 : 1;
   return cudaGetLastError();
 }
 
@@ -199,6 +200,7 @@ cudaError_t launch_unpermute(const void* yp, const int32_t* ros, int T, int k, i
   const int threads = std::min(256, std::max(32, (H / 8 + 31) / 32 * 32));
   unpermute_kernel<<<T, threads, 0, st>>>(reinterpret_cast<const uint4*>(yp), ros, T, k, H,
                                           reinterpret_cast<uint4*>(y));
+  ++g_launch_count;
   return cudaGetLastError();
 }
 
@@ -206,6 +208,7 @@ cudaError_t launch_dprob_reduce(const float* part, int nparts, const int32_t* ro
                                 cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   dprob_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(part, nparts, ros, n, dprobs);
+  ++g_launch_count;
   return cudaGetLastError();
 }
 

@@ -14,7 +14,7 @@ HEADER = os.path.join(ROOT, "include", "mxmoe.h")
 def _declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    pat = re.compile(r"^\s*(?:const\s+)?(?:mxmoe_status|size_t|int64_t|char\s*\*)\s*\*?\s*(\w+)\s*\(", re.M)
+    pat = re.compile(r"^\s*(?:const\s+)?(?:mxmoe_status|size_t|int64_t|int32_t|char\s*\*)\s*\*?\s*(\w+)\s*\(", re.M)
     return sorted(set(pat.findall(text)))
 
 
