@@ -50,6 +50,7 @@ def parse_args():
     p.add_argument("--impl", choices=["mxmoe", "reference"], default="mxmoe")
     p.add_argument("--config", default="mixtral", help="tiny | small | mixtral | mixtral_zipf | genomics")
     p.add_argument("--tokens", type=int, default=0, help="override the token count (profiling runs)")
+    p.add_argument("--experts", type=int, default=0, help="override the expert count (profiling runs)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=512, help="routed rows in the CPU oracle sample")
@@ -423,6 +424,8 @@ def main():
     cfg = wl.CONFIGS[args.config]
     if args.tokens:
         cfg = dataclasses.replace(cfg, T=args.tokens)
+    if args.experts:
+        cfg = dataclasses.replace(cfg, E=args.experts, k=min(cfg.k, args.experts))
     try:
         if args.impl == "reference":
             run_reference(args, cfg, dist, rank, world)

@@ -146,34 +146,52 @@ __device__ __forceinline__ TileInfo get_tile(const GemmArgs& g, int64_t idx, con
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
 
-// Warp-wide colwise MXFP8 of 32 columns: lane = row of a 32-row block, v[i] = column i.
-// Writes the codes transposed (column i -> 32 consecutive bytes at dst + i*ld) through
-// the warp's staging buffer, and the 32 scale bytes (lane i writes column i's).
-__device__ __forceinline__ void colwise_quant_store(const float (&v)[32], uint8_t* stg, int lane, uint8_t* dst,
+// Warp-wide colwise MXFP8 of a 32 x 32 fp32 block held one row per lane (lane = row,
+// v[i] = column i): blocks of 32 rows of one column, written transposed (column i ->
+// 32 consecutive bytes at dst + i*ld) with one scale byte per column.
+// The block is transposed through the warp's 2 KB staging buffer in two rounds of 16
+// columns. Staging layout (fp32 words): row r = 16*h + i (i < 16) lives in line i (32
+// words), half h; its four 16-byte chunks are XOR-swizzled by (i & 7), so both the
+// row-wise 16-byte stores and the column-wise 4-byte loads are bank-conflict free.
+// After the transpose, lane (c = lane % 16, h = lane / 16) holds rows [16h, 16h+16) of
+// column c; the two halves combine their amax with one shuffle.
+__device__ __forceinline__ void colwise_quant_store(const float (&v)[32], float* stg, int lane, uint8_t* dst,
                                                     int64_t ld, uint8_t* sf_base, int64_t sf_rows, int64_t sf_cols,
                                                     int64_t col_row0, int64_t kb) {
-  uint32_t my_sb = 0;
+  const int wi = lane & 15, wh = lane >> 4;  // this lane's row as (line, half) when writing
+  const int c = lane & 15, rh = lane >> 4;   // column and row half this lane reads
 #pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    const uint32_t am0 = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[i])));
-    const uint32_t am1 = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[i + 1])));
-    const int32_t X0 = mx_scale_exp_from_amax_bits(am0);
-    const int32_t X1 = mx_scale_exp_from_amax_bits(am1);
-    if (lane == i) my_sb = (uint32_t)(X0 + 127);
-    if (lane == i + 1) my_sb = (uint32_t)(X1 + 127);
-    const uint16_t q = e4m3x2(v[i] * mx_inv_scale(X0), v[i + 1] * mx_inv_scale(X1));
-    stg[i * 32 + lane] = (uint8_t)(q & 0xFF);
-    stg[(i + 1) * 32 + lane] = (uint8_t)(q >> 8);
+  for (int r = 0; r < 2; ++r) {
+#pragma unroll
+    for (int qd = 0; qd < 4; ++qd) {
+      const int phys = ((wh << 2) | qd) ^ (wi & 7);
+      *reinterpret_cast<float4*>(stg + wi * 32 + phys * 4) =
+          make_float4(v[16 * r + 4 * qd], v[16 * r + 4 * qd + 1], v[16 * r + 4 * qd + 2], v[16 * r + 4 * qd + 3]);
+    }
+    __syncwarp();
+    float w[16];
+    uint32_t amax = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int phys = ((rh << 2) | (c >> 2)) ^ (j & 7);
+      w[j] = stg[j * 32 + phys * 4 + (c & 3)];
+      amax = max(amax, __float_as_uint(fabsf(w[j])));
+    }
+    __syncwarp();
+    amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
+    const int32_t X = mx_scale_exp_from_amax_bits(amax);
+    const float sc = mx_inv_scale(X);
+    uint32_t q[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t lo = e4m3x2(w[4 * i] * sc, w[4 * i + 1] * sc);
+      const uint32_t hi = e4m3x2(w[4 * i + 2] * sc, w[4 * i + 3] * sc);
+      q[i] = lo | (hi << 16);
+    }
+    const int col = 16 * r + c;
+    *reinterpret_cast<uint4*>(dst + (int64_t)col * ld + 16 * rh) = make_uint4(q[0], q[1], q[2], q[3]);
+    if (rh == 0) sf_base[sf_offset(MXMOE_SCALE_MMA, sf_rows, sf_cols, col_row0 + col, kb)] = (uint8_t)(X + 127);
   }
-  __syncwarp();
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(stg + lane * 32);
-    uint4* d = reinterpret_cast<uint4*>(dst + (int64_t)lane * ld);
-    d[0] = src[0];
-    d[1] = src[1];
-  }
-  sf_base[sf_offset(MXMOE_SCALE_MMA, sf_rows, sf_cols, col_row0 + lane, kb)] = (uint8_t)my_sb;
-  __syncwarp();
 }
 
 __device__ __forceinline__ void rowwise_quant_store(const float (&v)[32], uint8_t* dst, uint8_t* sf, int64_t rows,
@@ -191,7 +209,7 @@ __device__ __forceinline__ void rowwise_quant_store(const float (&v)[32], uint8_
 // rowwise (32 columns of this row) and colwise (32 rows of each column); accumulates
 // dprob += dZ * silu(G) * U. dz holds 32 bf16 values of dZ packed in pairs.
 __device__ __forceinline__ void swiglu_bwd_chunk(const uint32_t (&dz)[16], const GemmArgs& g, int64_t row,
-                                                 int64_t f0, float p, float& dprob, uint8_t* stg, int lane,
+                                                 int64_t f0, float p, float& dprob, float* stg, int lane,
                                                  int64_t mrow0) {
   const int64_t F = g.F, F2 = 2 * g.F;
   const uint4* gs = reinterpret_cast<const uint4*>(g.gu_in + row * F2 + f0);
@@ -237,7 +255,7 @@ __device__ __forceinline__ void swiglu_bwd_chunk(const uint32_t (&dz)[16], const
 
 template <int C>
 __device__ __forceinline__ void swiglu_bwd_chunks(const uint32_t (&acc)[128], const GemmArgs& g, int64_t row,
-                                                  int64_t f0, float p, float& dprob, uint8_t* stg, int lane,
+                                                  int64_t f0, float p, float& dprob, float* stg, int lane,
                                                   int64_t mrow0) {
   if constexpr (C < 4) {
     uint32_t d[16];
@@ -397,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ew = warp - 2;
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int h = ew >> 2;   // column half
-    uint8_t* stg = smem + kOffStaging + ew * kStagingPerWarp;
+    float* stg = reinterpret_cast<float*>(smem + kOffStaging + ew * kStagingPerWarp);
     uint32_t acc_ph = 0;
     const uint32_t t_lane = tmem_base + ((uint32_t)(32 * q) << 16);
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {

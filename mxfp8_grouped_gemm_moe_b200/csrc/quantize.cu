@@ -57,21 +57,27 @@ __global__ void __launch_bounds__(kQThreads) mxfp8_quantize_kernel(QuantArgs a) 
   if (r0 >= nvalid) return;
   const T* src = reinterpret_cast<const T*>(a.src);
 
-  // ---- load the tile (gathered rows, zero outside the matrix / for pad rows)
-  constexpr int VPR = kQTile / Tr::kVec;  // vectors per tile row
-  for (int i = threadIdx.x; i < kQTile * VPR; i += kQThreads) {
-    const int row = i / VPR, cv = i % VPR;
-    const int64_t orow = r0 + row;
-    const int64_t col = c0 + (int64_t)cv * Tr::kVec;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (orow < nvalid && col < a.cols) {
-      int64_t srow;
-      if (a.gather) srow = a.gather[orow];
-      else srow = b * a.rows + orow;
-      if (srow >= 0) v = __ldg(reinterpret_cast<const uint4*>(src + srow * a.cols + col));
-    }
-    *reinterpret_cast<uint4*>(tile + row * LD + cv * Tr::kVec) = v;
+  // ---- load the tile (gathered rows, zero outside the matrix / for pad rows); all of a
+  // thread's row indices, then all of its 16-byte loads, are issued before any use
+  constexpr int VPR = kQTile / Tr::kVec;              // vectors per tile row
+  constexpr int NL = kQTile * VPR / kQThreads;        // vectors per thread
+  constexpr int RSTEP = kQThreads / VPR;              // tile rows between a thread's vectors
+  const int row_t = threadIdx.x / VPR, cv = threadIdx.x % VPR;
+  const int64_t col = c0 + (int64_t)cv * Tr::kVec;
+  int64_t srow[NL];
+#pragma unroll
+  for (int k = 0; k < NL; ++k) {
+    const int64_t orow = r0 + row_t + k * RSTEP;
+    srow[k] = -1;
+    if (orow < nvalid && col < a.cols) srow[k] = a.gather ? (int64_t)__ldg(a.gather + orow) : b * a.rows + orow;
   }
+  uint4 buf[NL];
+#pragma unroll
+  for (int k = 0; k < NL; ++k)
+    buf[k] = srow[k] >= 0 ? __ldg(reinterpret_cast<const uint4*>(src + srow[k] * a.cols + col)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int k = 0; k < NL; ++k)
+    *reinterpret_cast<uint4*>(tile + (row_t + k * RSTEP) * LD + cv * Tr::kVec) = buf[k];
   __syncthreads();
 
   // ---- rowwise: 128 rows x 4 blocks
