@@ -59,6 +59,7 @@ constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack for 1 KB alignment
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemSfa = 256;  // two buffers of 4 columns
 constexpr uint32_t kTmemSfb = 264;  // two buffers of 8 columns
+constexpr uint32_t kTmemStash = 384;  // epilogue scratch: 64 columns per (lane quadrant, half)
 constexpr int GROUP_M = 16;         // m tiles per raster group (L2 reuse of B)
 
 static_assert(kStageBytes >= kTxBytes && kStageBytes % 1024 == 0, "stage layout");
@@ -204,66 +205,23 @@ __device__ __forceinline__ void rowwise_quant_store(const float (&v)[32], uint8_
   sf[sf_offset(MXMOE_SCALE_MMA, rows, cols, row, kb)] = sb;
 }
 
-// SwiGLU / probability-scale backward for 32 columns of one row (one thread = one row,
-// the warp = 32 rows): dG = dZ*p*U*silu'(G) and dU = dZ*p*silu(G), each quantised
-// rowwise (32 columns of this row) and colwise (32 rows of each column); accumulates
-// dprob += dZ * silu(G) * U. dz holds 32 bf16 values of dZ packed in pairs.
-__device__ __forceinline__ void swiglu_bwd_chunk(const uint32_t (&dz)[16], const GemmArgs& g, int64_t row,
-                                                 int64_t f0, float p, float& dprob, float* stg, int lane,
-                                                 int64_t mrow0) {
-  const int64_t F = g.F, F2 = 2 * g.F;
-  const uint4* gs = reinterpret_cast<const uint4*>(g.gu_in + row * F2 + f0);
-  const uint4* us = reinterpret_cast<const uint4*>(g.gu_in + row * F2 + F + f0);
-  float v[32];
-  // dG (8 columns per 16-byte load of G and U keeps the live set small)
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint4 a = gs[j], b = us[j];
-    const uint32_t gw[4] = {a.x, a.y, a.z, a.w};
-    const uint32_t uw[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int c = 8 * j + i;
-      const float gg = (i & 1) ? bf16_hi(gw[i >> 1]) : bf16_lo(gw[i >> 1]);
-      const float uu = (i & 1) ? bf16_hi(uw[i >> 1]) : bf16_lo(uw[i >> 1]);
-      const float d = (c & 1) ? bf16_hi(dz[c >> 1]) : bf16_lo(dz[c >> 1]);
-      const float sg = 1.0f / (1.0f + __expf(-gg));
-      dprob += d * (gg * sg * uu);
-      v[c] = d * p * uu * (sg * (1.0f + gg * (1.0f - sg)));
-    }
-  }
-  rowwise_quant_store(v, g.dgu_row + row * F2 + f0, g.dgu_row_sf, g.rows_cap, F2, row, f0 / 32);
-  colwise_quant_store(v, stg, lane, g.dgu_colT + f0 * g.rows_cap + mrow0, g.rows_cap, g.dgu_colT_sf, F2,
-                      g.rows_cap, f0, mrow0 / 32);
-  // dU (G reloaded; it is in L1)
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint4 a = gs[j];
-    const uint32_t gw[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int c = 8 * j + i;
-      const float gg = (i & 1) ? bf16_hi(gw[i >> 1]) : bf16_lo(gw[i >> 1]);
-      const float d = (c & 1) ? bf16_hi(dz[c >> 1]) : bf16_lo(dz[c >> 1]);
-      v[c] = d * p * silu_f(gg);
-    }
-  }
-  rowwise_quant_store(v, g.dgu_row + row * F2 + F + f0, g.dgu_row_sf, g.rows_cap, F2, row, (F + f0) / 32);
-  colwise_quant_store(v, stg, lane, g.dgu_colT + (F + f0) * g.rows_cap + mrow0, g.rows_cap, g.dgu_colT_sf, F2,
-                      g.rows_cap, F + f0, mrow0 / 32);
+// Hands the accumulator back to the MMA warp once this warp's TMEM reads (and writes
+// to its spare columns) have completed.
+__device__ __forceinline__ void release_accumulator(uint64_t* bar_acc_empty, int lane) {
+  ptx::tc_fence_before();
+  __syncwarp();
+  if (lane == 0) ptx::mbar_arrive(bar_acc_empty);
 }
 
-template <int C>
-__device__ __forceinline__ void swiglu_bwd_chunks(const uint32_t (&acc)[128], const GemmArgs& g, int64_t row,
-                                                  int64_t f0, float p, float& dprob, float* stg, int lane,
-                                                  int64_t mrow0) {
-  if constexpr (C < 4) {
-    uint32_t d[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) d[i] = acc[16 * C + i];
-    swiglu_bwd_chunk(d, g, row, f0 + 32 * C, p, dprob, stg, lane, mrow0);
-    swiglu_bwd_chunks<C + 1>(acc, g, row, f0, p, dprob, stg, lane, mrow0);
-  }
+// 8 fp32 (bit patterns) starting at v[i0] -> 8 bf16 in one 16-byte vector.
+template <int N>
+__device__ __forceinline__ uint4 pack8_bf16(const uint32_t (&v)[N], int i0) {
+  uint4 o;
+  o.x = pack_bf16x2(__uint_as_float(v[i0 + 0]), __uint_as_float(v[i0 + 1]));
+  o.y = pack_bf16x2(__uint_as_float(v[i0 + 2]), __uint_as_float(v[i0 + 3]));
+  o.z = pack_bf16x2(__uint_as_float(v[i0 + 4]), __uint_as_float(v[i0 + 5]));
+  o.w = pack_bf16x2(__uint_as_float(v[i0 + 6]), __uint_as_float(v[i0 + 7]));
+  return o;
 }
 
 template <int MODE>
@@ -418,14 +376,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* stg = reinterpret_cast<float*>(smem + kOffStaging + ew * kStagingPerWarp);
     uint32_t acc_ph = 0;
     const uint32_t t_lane = tmem_base + ((uint32_t)(32 * q) << 16);
+    const uint32_t t_stash = t_lane + kTmemStash + 64 * h;  // this warp's 64 spare TMEM columns
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
       // warp-uniform abort check (the TMEM loads below are warp-collective)
       if (__any_sync(0xffffffffu, *s_abort != 0)) break;
       const TileInfo t = get_tile<MODE>(g, tile, s_seg, s_order);
-      const int rr = 32 * q + lane;
-      const int64_t row = t.row0 + rr;
-      uint32_t acc[128];
-      if (t.k_iters > 0) {
+      const int64_t mrow0 = t.row0 + 32 * q;  // first row of this warp's 32-row block
+      const int64_t row = mrow0 + lane;
+      const bool have_acc = t.k_iters > 0;
+      if (have_acc) {
         const bool ok = ptx::mbar_wait(bar_acc_full, acc_ph, 4);
         if (!__all_sync(0xffffffffu, ok)) {
           *s_abort = 1;
@@ -434,40 +393,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         acc_ph ^= 1u;
         ptx::tc_fence_after();
-        if (MODE == kModeSwigluBwd) {
-          // drain 32 columns at a time and keep dZ as packed bf16 pairs (64 registers for
-          // 128 columns): the E4M3 rounding that follows dominates that rounding by 2^5
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t tmp[32];
-            ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 32 * c, tmp);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              acc[16 * c + i] = pack_bf16x2(__uint_as_float(tmp[2 * i]), __uint_as_float(tmp[2 * i + 1]));
-          }
-        } else if (MODE == kModeSwigluFwd) {
-          // gate columns [64h, 64h+64), up columns [128 + 64h, +64)
-          ptx::tmem_ld_32x32b_x32(t_lane + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&acc[0]));
-          ptx::tmem_ld_32x32b_x32(t_lane + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&acc[32]));
-          ptx::tmem_ld_32x32b_x32(t_lane + 128 + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&acc[64]));
-          ptx::tmem_ld_32x32b_x32(t_lane + 128 + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&acc[96]));
-        } else {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&acc[32 * c]));
-        }
-        ptx::tmem_wait_ld();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar_acc_empty);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) acc[i] = 0u;
       }
 
       if (MODE == kModeStore || MODE == kModeWgrad) {
-        const int64_t col0 = (MODE == kModeWgrad ? (int64_t)t.n_tile * BN : (int64_t)t.n_tile * BN) + 128 * h;
+        uint32_t acc[128];
+        if (have_acc) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&acc[32 * c]));
+          ptx::tmem_wait_ld();
+          release_accumulator(bar_acc_empty, lane);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 128; ++i) acc[i] = 0u;
+        }
+        const int64_t col0 = (int64_t)t.n_tile * BN + 128 * h;
         if (MODE == kModeWgrad || g.c_dtype == MXMOE_DTYPE_F32) {
           float* c = reinterpret_cast<float*>(g.c) + row * g.ldc + col0;
 #pragma unroll
@@ -476,59 +416,115 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           uint16_t* c = reinterpret_cast<uint16_t*>(g.c) + row * g.ldc + col0;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            uint4 o;
-            o.x = pack_bf16x2(__uint_as_float(acc[8 * i + 0]), __uint_as_float(acc[8 * i + 1]));
-            o.y = pack_bf16x2(__uint_as_float(acc[8 * i + 2]), __uint_as_float(acc[8 * i + 3]));
-            o.z = pack_bf16x2(__uint_as_float(acc[8 * i + 4]), __uint_as_float(acc[8 * i + 5]));
-            o.w = pack_bf16x2(__uint_as_float(acc[8 * i + 6]), __uint_as_float(acc[8 * i + 7]));
-            reinterpret_cast<uint4*>(c)[i] = o;
-          }
+          for (int i = 0; i < 16; ++i) reinterpret_cast<uint4*>(c)[i] = pack8_bf16(acc, 8 * i);
         }
       } else if (MODE == kModeSwigluFwd) {
         const int64_t F = g.F, F2 = 2 * g.F;
         const float p = g.prob_of_row[row];
-        const int64_t f0 = (int64_t)t.n_tile * 128 + 64 * h;
-        // save G and U (bf16) for the backward
-        {
-          uint16_t* gd = g.gu + row * F2 + f0;
-          uint16_t* ud = gd + F;
+        const int64_t f0 = (int64_t)t.n_tile * 128 + 64 * h;  // this warp's 64 Z columns
+        // phase 1: drain gate / up (TMEM columns [64h, +64) and [128 + 64h, +64)), save them
+        // in bf16 for the backward, form Z = silu(G) * U * p in fp32 and park it in TMEM
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            uint4 o;
-            o.x = pack_bf16x2(__uint_as_float(acc[8 * i + 0]), __uint_as_float(acc[8 * i + 1]));
-            o.y = pack_bf16x2(__uint_as_float(acc[8 * i + 2]), __uint_as_float(acc[8 * i + 3]));
-            o.z = pack_bf16x2(__uint_as_float(acc[8 * i + 4]), __uint_as_float(acc[8 * i + 5]));
-            o.w = pack_bf16x2(__uint_as_float(acc[8 * i + 6]), __uint_as_float(acc[8 * i + 7]));
-            reinterpret_cast<uint4*>(gd)[i] = o;
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(acc[64 + 8 * i + 0]), __uint_as_float(acc[64 + 8 * i + 1]));
-            u.y = pack_bf16x2(__uint_as_float(acc[64 + 8 * i + 2]), __uint_as_float(acc[64 + 8 * i + 3]));
-            u.z = pack_bf16x2(__uint_as_float(acc[64 + 8 * i + 4]), __uint_as_float(acc[64 + 8 * i + 5]));
-            u.w = pack_bf16x2(__uint_as_float(acc[64 + 8 * i + 6]), __uint_as_float(acc[64 + 8 * i + 7]));
-            reinterpret_cast<uint4*>(ud)[i] = u;
+        for (int c = 0; c < 2; ++c) {
+          uint32_t gr[32], ur[32];
+          ptx::tmem_ld_32x32b_x32(t_lane + 64 * h + 32 * c, gr);
+          ptx::tmem_ld_32x32b_x32(t_lane + 128 + 64 * h + 32 * c, ur);
+          ptx::tmem_wait_ld();
+          uint4* gd = reinterpret_cast<uint4*>(g.gu + row * F2 + f0 + 32 * c);
+          uint4* ud = reinterpret_cast<uint4*>(g.gu + row * F2 + F + f0 + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            gd[i] = pack8_bf16(gr, 8 * i);
+            ud[i] = pack8_bf16(ur, 8 * i);
           }
-        }
 #pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
+          for (int i = 0; i < 32; ++i)
+            gr[i] = __float_as_uint(silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]) * p);
+          ptx::tmem_st_32x32b_x16(t_stash + 32 * c, *reinterpret_cast<uint32_t(*)[16]>(&gr[0]));
+          ptx::tmem_st_32x32b_x16(t_stash + 32 * c + 16, *reinterpret_cast<uint32_t(*)[16]>(&gr[16]));
+        }
+        ptx::tmem_wait_st();
+        release_accumulator(bar_acc_empty, lane);
+        // phase 2: MXFP8 of Z, rowwise (fc2 operand) and colwise (fc2 weight-gradient operand)
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t zr[32];
+          ptx::tmem_ld_32x32b_x32(t_stash + 32 * c, zr);
+          ptx::tmem_wait_ld();
           float z[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float gg = __uint_as_float(acc[32 * blk + i]);
-            const float uu = __uint_as_float(acc[64 + 32 * blk + i]);
-            z[i] = silu_f(gg) * uu * p;
-          }
-          const int64_t fc = f0 + 32 * blk;
+          for (int i = 0; i < 32; ++i) z[i] = __uint_as_float(zr[i]);
+          const int64_t fc = f0 + 32 * c;
           rowwise_quant_store(z, g.z_row + row * F + fc, g.z_row_sf, g.rows_cap, F, row, fc / 32);
-          colwise_quant_store(z, stg, lane, g.z_colT + fc * g.rows_cap + (t.row0 + 32 * q), g.rows_cap, g.z_colT_sf, F,
-                              g.rows_cap, fc, (t.row0 + 32 * q) / 32);
+          colwise_quant_store(z, stg, lane, g.z_colT + fc * g.rows_cap + mrow0, g.rows_cap, g.z_colT_sf, F,
+                              g.rows_cap, fc, mrow0 / 32);
         }
       } else if (MODE == kModeSwigluBwd) {
+        const int64_t F = g.F, F2 = 2 * g.F;
         const float p = g.prob_of_row[row];
+        const int64_t f0 = (int64_t)t.n_tile * BN + 128 * h;  // this warp's 128 dZ columns
+        // phase 1: drain dZ, park it in TMEM as packed bf16 pairs (the E4M3 rounding that
+        // follows is 2^5 coarser than that rounding)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t tmp[32], pk[16];
+          ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 32 * c, tmp);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(tmp[2 * i]), __uint_as_float(tmp[2 * i + 1]));
+          ptx::tmem_st_32x32b_x16(t_stash + 16 * c, pk);
+        }
+        ptx::tmem_wait_st();
+        release_accumulator(bar_acc_empty, lane);
+        // phase 2: SwiGLU / probability backward, 32 columns at a time; G and U of the next
+        // chunk are fetched while this one is processed
+        const uint4* gsrc = reinterpret_cast<const uint4*>(g.gu_in + row * F2 + f0);
+        const uint4* usrc = reinterpret_cast<const uint4*>(g.gu_in + row * F2 + F + f0);
+        uint4 gq[4], uq[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          gq[i] = gsrc[i];
+          uq[i] = usrc[i];
+        }
         float dprob = 0.f;
-        const int64_t f0 = (int64_t)t.n_tile * BN + 128 * h;
-        swiglu_bwd_chunks<0>(acc, g, row, f0, p, dprob, stg, lane, t.row0 + 32 * q);
-        g.dprob_part[row * (g.F / 128) + t.n_tile * 2 + h] = dprob;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t dzw[16];
+          ptx::tmem_ld_32x32b_x16(t_stash + 16 * c, dzw);
+          const uint32_t gw[16] = {gq[0].x, gq[0].y, gq[0].z, gq[0].w, gq[1].x, gq[1].y, gq[1].z, gq[1].w,
+                                   gq[2].x, gq[2].y, gq[2].z, gq[2].w, gq[3].x, gq[3].y, gq[3].z, gq[3].w};
+          const uint32_t uw[16] = {uq[0].x, uq[0].y, uq[0].z, uq[0].w, uq[1].x, uq[1].y, uq[1].z, uq[1].w,
+                                   uq[2].x, uq[2].y, uq[2].z, uq[2].w, uq[3].x, uq[3].y, uq[3].z, uq[3].w};
+          if (c < 3) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              gq[i] = gsrc[4 * (c + 1) + i];
+              uq[i] = usrc[4 * (c + 1) + i];
+            }
+          }
+          ptx::tmem_wait_ld();
+          float vg[32], vu[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float gg = (i & 1) ? bf16_hi(gw[i >> 1]) : bf16_lo(gw[i >> 1]);
+            const float uu = (i & 1) ? bf16_hi(uw[i >> 1]) : bf16_lo(uw[i >> 1]);
+            const float dz = (i & 1) ? bf16_hi(dzw[i >> 1]) : bf16_lo(dzw[i >> 1]);
+            const float sg = 1.0f / (1.0f + __expf(-gg));  // sigmoid(G)
+            const float sl = gg * sg;                        // silu(G)
+            const float da = dz * p;                         // dA = dZ * p
+            dprob += dz * sl * uu;                           // dprob += dZ * A
+            vg[i] = da * uu * (sg * (1.0f + gg * (1.0f - sg)));
+            vu[i] = da * sl;
+          }
+          const int64_t fg = f0 + 32 * c;
+          rowwise_quant_store(vg, g.dgu_row + row * F2 + fg, g.dgu_row_sf, g.rows_cap, F2, row, fg / 32);
+          colwise_quant_store(vg, stg, lane, g.dgu_colT + fg * g.rows_cap + mrow0, g.rows_cap, g.dgu_colT_sf, F2,
+                              g.rows_cap, fg, mrow0 / 32);
+          rowwise_quant_store(vu, g.dgu_row + row * F2 + F + fg, g.dgu_row_sf, g.rows_cap, F2, row, (F + fg) / 32);
+          colwise_quant_store(vu, stg, lane, g.dgu_colT + (F + fg) * g.rows_cap + mrow0, g.rows_cap,
+                              g.dgu_colT_sf, F2, g.rows_cap, F + fg, mrow0 / 32);
+        }
+        g.dprob_part[row * (F / 128) + t.n_tile * 2 + h] = dprob;
       }
     }
   }
