@@ -38,7 +38,10 @@ namespace mxmoe {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;
-constexpr int STAGES = 4;
+#ifndef MXMOE_STAGES
+#define MXMOE_STAGES 4
+#endif
+constexpr int STAGES = MXMOE_STAGES;
 constexpr int kThreads = 320;  // 10 warps
 constexpr int kEpiWarps = 8;
 
@@ -422,20 +425,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t F = g.F, F2 = 2 * g.F;
         const float p = g.prob_of_row[row];
         const int64_t f0 = (int64_t)t.n_tile * 128 + 64 * h;  // this warp's 64 Z columns
-        // phase 1: drain gate / up (TMEM columns [64h, +64) and [128 + 64h, +64)), save them
-        // in bf16 for the backward, form Z = silu(G) * U * p in fp32 and park it in TMEM
+        // phase 1 (the MMA warp waits for it): drain gate / up (TMEM columns [64h, +64) and
+        // [128 + 64h, +64)), keep them as packed bf16 for the backward's saved copy, form
+        // Z = silu(G) * U * p in fp32 and park Z in this warp's spare TMEM columns
+        uint4 gsave[8], usave[8];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t gr[32], ur[32];
           ptx::tmem_ld_32x32b_x32(t_lane + 64 * h + 32 * c, gr);
           ptx::tmem_ld_32x32b_x32(t_lane + 128 + 64 * h + 32 * c, ur);
           ptx::tmem_wait_ld();
-          uint4* gd = reinterpret_cast<uint4*>(g.gu + row * F2 + f0 + 32 * c);
-          uint4* ud = reinterpret_cast<uint4*>(g.gu + row * F2 + F + f0 + 32 * c);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            gd[i] = pack8_bf16(gr, 8 * i);
-            ud[i] = pack8_bf16(ur, 8 * i);
+            gsave[4 * c + i] = pack8_bf16(gr, 8 * i);
+            usave[4 * c + i] = pack8_bf16(ur, 8 * i);
           }
 #pragma unroll
           for (int i = 0; i < 32; ++i)
@@ -445,6 +448,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::tmem_wait_st();
         release_accumulator(bar_acc_empty, lane);
+        {
+          uint4* gd = reinterpret_cast<uint4*>(g.gu + row * F2 + f0);
+          uint4* ud = reinterpret_cast<uint4*>(g.gu + row * F2 + F + f0);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            gd[i] = gsave[i];
+            ud[i] = usave[i];
+          }
+        }
         // phase 2: MXFP8 of Z, rowwise (fc2 operand) and colwise (fc2 weight-gradient operand)
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
