@@ -39,6 +39,36 @@ struct SrcTraits<float> {
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 __device__ __forceinline__ float to_f32(float v) { return v; }
 
+// 32 consecutive elements of a shared-memory row -> fp32 (16-byte loads).
+__device__ __forceinline__ void load32_row(const __nv_bfloat16* p, float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 w = reinterpret_cast<const uint4*>(p)[i];
+    v[8 * i + 0] = bf16_lo(w.x); v[8 * i + 1] = bf16_hi(w.x);
+    v[8 * i + 2] = bf16_lo(w.y); v[8 * i + 3] = bf16_hi(w.y);
+    v[8 * i + 4] = bf16_lo(w.z); v[8 * i + 5] = bf16_hi(w.z);
+    v[8 * i + 6] = bf16_lo(w.w); v[8 * i + 7] = bf16_hi(w.w);
+  }
+}
+__device__ __forceinline__ void load32_row(const float* p, float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 w = reinterpret_cast<const float4*>(p)[i];
+    v[4 * i + 0] = w.x; v[4 * i + 1] = w.y; v[4 * i + 2] = w.z; v[4 * i + 3] = w.w;
+  }
+}
+// Two adjacent elements of a shared-memory row -> fp32.
+__device__ __forceinline__ void load_pair(const __nv_bfloat16* p, float& a, float& b) {
+  const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+  a = bf16_lo(w);
+  b = bf16_hi(w);
+}
+__device__ __forceinline__ void load_pair(const float* p, float& a, float& b) {
+  const float2 w = *reinterpret_cast<const float2*>(p);
+  a = w.x;
+  b = w.y;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kQThreads) mxfp8_quantize_kernel(QuantArgs a) {
   using Tr = SrcTraits<T>;
@@ -80,16 +110,17 @@ __global__ void __launch_bounds__(kQThreads) mxfp8_quantize_kernel(QuantArgs a) 
     *reinterpret_cast<uint4*>(tile + (row_t + k * RSTEP) * LD + cv * Tr::kVec) = buf[k];
   __syncthreads();
 
-  // ---- rowwise: 128 rows x 4 blocks
+  // ---- rowwise: item = (32-column block, row); a warp takes 32 consecutive rows of one
+  // block, so its 16-byte shared loads hit distinct banks (row stride = 4 banks mod 32)
   if (a.row_data) {
+#pragma unroll 1
     for (int it = threadIdx.x; it < kQTile * 4; it += kQThreads) {
-      const int row = it >> 2, blk = it & 3;
+      const int row = it & (kQTile - 1), blk = it >> 7;
       const int64_t orow = r0 + row;
       const int64_t col = c0 + 32 * blk;
       if (orow >= nvalid || col >= a.cols) continue;
       float v[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = to_f32(tile[row * LD + 32 * blk + i]);
+      load32_row(tile + row * LD + 32 * blk, v);
       uint32_t q[8];
       const uint8_t sb = quant_block32(v, q);
       const int64_t grow = b * a.out_rows + orow;
@@ -99,23 +130,28 @@ __global__ void __launch_bounds__(kQThreads) mxfp8_quantize_kernel(QuantArgs a) 
       a.row_sf[sf_offset(a.row_layout, a.batch * a.out_rows, a.cols, grow, col / 32)] = sb;
     }
   }
-  // ---- colwise: 128 columns x 4 row blocks, stored transposed
+  // ---- colwise: item = (pair of adjacent columns, 32-row block), one per thread; a warp
+  // reads 32 consecutive column pairs of a row per load (conflict free)
   if (a.col_data) {
-    for (int it = threadIdx.x; it < kQTile * 4; it += kQThreads) {
-      const int cc = it & (kQTile - 1), rb = it >> 7;
-      const int64_t col = c0 + cc;
-      const int64_t orow = r0 + 32 * rb;
-      if (orow >= nvalid || col >= a.cols) continue;
-      float v[32];
+    const int pcol = threadIdx.x & 63, rb = threadIdx.x >> 6;
+    const int64_t col = c0 + 2 * pcol;
+    const int64_t orow = r0 + 32 * rb;
+    if (orow < nvalid && col < a.cols) {
+      float v0[32], v1[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = to_f32(tile[(32 * rb + i) * LD + cc]);
+      for (int i = 0; i < 32; ++i) load_pair(tile + (32 * rb + i) * LD + 2 * pcol, v0[i], v1[i]);
       uint32_t q[8];
-      const uint8_t sb = quant_block32(v, q);
       const int64_t grow = b * a.cols + col;  // row of the transposed matrix
+      uint8_t sb = quant_block32(v0, q);
       uint4* dst = reinterpret_cast<uint4*>(a.col_data + grow * a.out_rows + orow);
       dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
       dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
       a.col_sf[sf_offset(a.col_layout, a.batch * a.cols, a.out_rows, grow, orow / 32)] = sb;
+      sb = quant_block32(v1, q);
+      dst = reinterpret_cast<uint4*>(a.col_data + (grow + 1) * a.out_rows + orow);
+      dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
+      dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
+      a.col_sf[sf_offset(a.col_layout, a.batch * a.cols, a.out_rows, grow + 1, orow / 32)] = sb;
     }
   }
 }
