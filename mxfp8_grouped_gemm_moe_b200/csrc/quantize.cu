@@ -70,123 +70,185 @@ __device__ __forceinline__ void load_pair(const float* p, float& a, float& b) {
   b = w.y;
 }
 
-// 16-byte asynchronous global -> shared copy (zero-filled when src_bytes == 0).
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
-               "l"(gmem), "r"(src_bytes)
-               : "memory");
+// MXFP8 of 32 bf16 values given as 16 packed words (element 2k in the low half of w[k],
+// 2k+1 in the high half). |bf16| bit patterns order like unsigned 16-bit integers, so
+// the block amax is a SIMD max over the masked words; the result equals the amax of the
+// values widened to fp32 (widening is exact), hence the same scale as quant_block32.
+__device__ __forceinline__ uint8_t quant_block32_bf16(const uint32_t (&w)[16], uint32_t (&out)[8]) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+  const uint32_t amax = max(m << 16, m & 0xFFFF0000u);
+  const int32_t X = mx_scale_exp_from_amax_bits(amax);
+  const float s = mx_inv_scale(X);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t lo = e4m3x2(bf16_lo(w[2 * i]) * s, bf16_hi(w[2 * i]) * s);
+    const uint32_t hi = e4m3x2(bf16_lo(w[2 * i + 1]) * s, bf16_hi(w[2 * i + 1]) * s);
+    out[i] = lo | (hi << 16);
+  }
+  return (uint8_t)(X + 127);
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
-// Persistent over 128 x 128 tiles (tile t: batch, row tile, column tile), two shared
-// buffers: tile t+1 is in flight while tile t is quantised.
+// Colwise MXFP8 of two adjacent columns over 32 rows: w[r] holds (column c, row r) in
+// its low half and (column c+1, row r) in its high half.
+__device__ __forceinline__ void quant_colpair_bf16(const uint32_t (&w)[32], uint32_t (&o0)[8], uint32_t (&o1)[8],
+                                                   uint8_t& sb0, uint8_t& sb1) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+  const int32_t X0 = mx_scale_exp_from_amax_bits(m << 16);
+  const int32_t X1 = mx_scale_exp_from_amax_bits(m & 0xFFFF0000u);
+  const float s0 = mx_inv_scale(X0), s1 = mx_inv_scale(X1);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    o0[i] = (uint32_t)e4m3x2(bf16_lo(w[4 * i]) * s0, bf16_lo(w[4 * i + 1]) * s0) |
+            ((uint32_t)e4m3x2(bf16_lo(w[4 * i + 2]) * s0, bf16_lo(w[4 * i + 3]) * s0) << 16);
+    o1[i] = (uint32_t)e4m3x2(bf16_hi(w[4 * i]) * s1, bf16_hi(w[4 * i + 1]) * s1) |
+            ((uint32_t)e4m3x2(bf16_hi(w[4 * i + 2]) * s1, bf16_hi(w[4 * i + 3]) * s1) << 16);
+  }
+  sb0 = (uint8_t)(X0 + 127);
+  sb1 = (uint8_t)(X1 + 127);
+}
+
 template <typename T>
-__global__ void __launch_bounds__(kQThreads) mxfp8_quantize_kernel(QuantArgs a) {
+__device__ __forceinline__ uint8_t quant_row_block(const T* p, uint32_t (&q)[8]);
+template <>
+__device__ __forceinline__ uint8_t quant_row_block<__nv_bfloat16>(const __nv_bfloat16* p, uint32_t (&q)[8]) {
+  uint32_t w[16];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 v = reinterpret_cast<const uint4*>(p)[i];
+    w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+  }
+  return quant_block32_bf16(w, q);
+}
+template <>
+__device__ __forceinline__ uint8_t quant_row_block<float>(const float* p, uint32_t (&q)[8]) {
+  float v[32];
+  load32_row(p, v);
+  return quant_block32(v, q);
+}
+
+template <typename T>
+__device__ __forceinline__ void quant_col_pair(const T* p, int ld, uint32_t (&q0)[8], uint32_t (&q1)[8], uint8_t& s0,
+                                               uint8_t& s1);
+template <>
+__device__ __forceinline__ void quant_col_pair<__nv_bfloat16>(const __nv_bfloat16* p, int ld, uint32_t (&q0)[8],
+                                                              uint32_t (&q1)[8], uint8_t& s0, uint8_t& s1) {
+  uint32_t w[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) w[i] = *reinterpret_cast<const uint32_t*>(p + i * ld);
+  quant_colpair_bf16(w, q0, q1, s0, s1);
+}
+template <>
+__device__ __forceinline__ void quant_col_pair<float>(const float* p, int ld, uint32_t (&q0)[8], uint32_t (&q1)[8],
+                                                      uint8_t& s0, uint8_t& s1) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = p[i * ld];
+  s0 = quant_block32(v, q0);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = p[i * ld + 1];
+  s1 = quant_block32(v, q1);
+}
+
+// One CTA per 128 x 128 tile (many resident per SM to overlap load latency).
+template <typename T>
+__global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quantize_kernel(QuantArgs a) {
   using Tr = SrcTraits<T>;
   constexpr int LD = kQTile + Tr::kPad;
-  constexpr int VPR = kQTile / Tr::kVec;        // 16-byte vectors per tile row
-  constexpr int NL = kQTile * VPR / kQThreads;  // vectors per thread
-  constexpr int RSTEP = kQThreads / VPR;        // tile rows between a thread's vectors
   extern __shared__ __align__(16) uint8_t q_smem_raw[];
-  T* bufs[2] = {reinterpret_cast<T*>(q_smem_raw), reinterpret_cast<T*>(q_smem_raw) + kQTile * LD};
+  T* tile = reinterpret_cast<T*>(q_smem_raw);
 
+  const int64_t c0 = (int64_t)blockIdx.x * kQTile;
+  const int64_t r0 = (int64_t)blockIdx.y * kQTile;
+  const int64_t b = blockIdx.z;
   int64_t nvalid = a.out_rows;
   if (a.nrows) {
     const int64_t nv = *a.nrows;
     nvalid = nv < nvalid ? nv : nvalid;
   }
-  const int64_t ct = (a.cols + kQTile - 1) / kQTile;
-  const int64_t rt = (nvalid + kQTile - 1) / kQTile;   // row tiles that hold valid rows
-  const int64_t ntiles = a.batch * rt * ct;
+  if (r0 >= nvalid) return;
   const T* src = reinterpret_cast<const T*>(a.src);
-  const int row_t = threadIdx.x / VPR, cv = threadIdx.x % VPR;
 
-  auto issue = [&](int64_t tile, T* dst) {
-    const int64_t b = tile / (rt * ct), rem = tile % (rt * ct);
-    const int64_t r0 = (rem / ct) * kQTile, c0 = (rem % ct) * kQTile;
+  // ---- load the tile (gathered rows, zero outside the matrix / for pad rows); all of a
+  // thread's row indices, then all of its 16-byte loads, are issued before any use
+  constexpr int VPR = kQTile / Tr::kVec;        // vectors per tile row
+  constexpr int NL = kQTile * VPR / kQThreads;  // vectors per thread
+  constexpr int RSTEP = kQThreads / VPR;        // tile rows between a thread's vectors
+  const int row_t = threadIdx.x / VPR, cv = threadIdx.x % VPR;
+  {
     const int64_t col = c0 + (int64_t)cv * Tr::kVec;
+    int64_t srow[NL];
 #pragma unroll
     for (int k = 0; k < NL; ++k) {
       const int64_t orow = r0 + row_t + k * RSTEP;
-      int64_t srow = -1;
-      if (orow < nvalid && col < a.cols) srow = a.gather ? (int64_t)__ldg(a.gather + orow) : b * a.rows + orow;
-      const T* g = srow >= 0 ? src + srow * a.cols + col : src;
-      cp_async16(dst + (row_t + k * RSTEP) * LD + cv * Tr::kVec, g, srow >= 0 ? 16u : 0u);
+      srow[k] = -1;
+      if (orow < nvalid && col < a.cols) srow[k] = a.gather ? (int64_t)__ldg(a.gather + orow) : b * a.rows + orow;
     }
-  };
-
-  int64_t tile = blockIdx.x;
-  if (tile < ntiles) issue(tile, bufs[0]);
-  cp_async_commit();
-  for (int it = 0; tile < ntiles; ++it, tile += gridDim.x) {
-    T* cur = bufs[it & 1];
-    if (tile + gridDim.x < ntiles) issue(tile + gridDim.x, bufs[(it + 1) & 1]);
-    cp_async_commit();
-    cp_async_wait_1();
-    __syncthreads();
-
-    const int64_t b = tile / (rt * ct), rem = tile % (rt * ct);
-    const int64_t r0 = (rem / ct) * kQTile, c0 = (rem % ct) * kQTile;
-    // ---- rowwise: item = (32-column block, row); a warp takes 32 consecutive rows of one
-    // block, so its 16-byte shared loads hit distinct banks (row stride = 4 banks mod 32)
-    if (a.row_data) {
-#pragma unroll 1
-      for (int i2 = threadIdx.x; i2 < kQTile * 4; i2 += kQThreads) {
-        const int row = i2 & (kQTile - 1), blk = i2 >> 7;
-        const int64_t orow = r0 + row;
-        const int64_t col = c0 + 32 * blk;
-        if (orow >= nvalid || col >= a.cols) continue;
-        float v[32];
-        load32_row(cur + row * LD + 32 * blk, v);
-        uint32_t q[8];
-        const uint8_t sb = quant_block32(v, q);
-        const int64_t grow = b * a.out_rows + orow;
-        uint4* dst = reinterpret_cast<uint4*>(a.row_data + grow * a.cols + col);
-        dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
-        dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
-        a.row_sf[sf_offset(a.row_layout, a.batch * a.out_rows, a.cols, grow, col / 32)] = sb;
-      }
-    }
-    // ---- colwise: item = (column, 32-row block); a warp reads 32 consecutive columns of
-    // a row per load (conflict free); stored transposed
-    if (a.col_data) {
-#pragma unroll 1
-      for (int i2 = threadIdx.x; i2 < kQTile * 4; i2 += kQThreads) {
-        const int cc = i2 & (kQTile - 1), rb = i2 >> 7;
-        const int64_t col = c0 + cc;
-        const int64_t orow = r0 + 32 * rb;
-        if (orow >= nvalid || col >= a.cols) continue;
-        float v[32];
+    uint4 buf[NL];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = to_f32(cur[(32 * rb + i) * LD + cc]);
-        uint32_t q[8];
-        const uint8_t sb = quant_block32(v, q);
-        const int64_t grow = b * a.cols + col;  // row of the transposed matrix
-        uint4* dst = reinterpret_cast<uint4*>(a.col_data + grow * a.out_rows + orow);
-        dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
-        dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
-        a.col_sf[sf_offset(a.col_layout, a.batch * a.cols, a.out_rows, grow, orow / 32)] = sb;
-      }
+    for (int k = 0; k < NL; ++k)
+      buf[k] = srow[k] >= 0 ? __ldg(reinterpret_cast<const uint4*>(src + srow[k] * a.cols + col))
+                            : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int k = 0; k < NL; ++k) *reinterpret_cast<uint4*>(tile + (row_t + k * RSTEP) * LD + cv * Tr::kVec) = buf[k];
+  }
+  __syncthreads();
+
+  // ---- rowwise: item = (32-column block, row); a warp takes 32 consecutive rows of one
+  // block, so its 16-byte shared loads hit distinct banks (row stride = 4 banks mod 32)
+  if (a.row_data) {
+#pragma unroll 1
+    for (int it = threadIdx.x; it < kQTile * 4; it += kQThreads) {
+      const int row = it & (kQTile - 1), blk = it >> 7;
+      const int64_t orow = r0 + row;
+      const int64_t col = c0 + 32 * blk;
+      if (orow >= nvalid || col >= a.cols) continue;
+      uint32_t q[8];
+      const uint8_t sb = quant_row_block<T>(tile + row * LD + 32 * blk, q);
+      const int64_t grow = b * a.out_rows + orow;
+      uint4* dst = reinterpret_cast<uint4*>(a.row_data + grow * a.cols + col);
+      dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
+      dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
+      a.row_sf[sf_offset(a.row_layout, a.batch * a.out_rows, a.cols, grow, col / 32)] = sb;
     }
-    __syncthreads();  // `cur` is refilled two tiles from now
+  }
+  // ---- colwise: item = (pair of adjacent columns, 32-row block), one per thread; a warp
+  // reads 32 consecutive column pairs of a row per load (conflict free); stored transposed
+  if (a.col_data) {
+    const int pcol = threadIdx.x & 63, rb = threadIdx.x >> 6;
+    const int64_t col = c0 + 2 * pcol;
+    const int64_t orow = r0 + 32 * rb;
+    if (orow < nvalid && col < a.cols) {
+      uint32_t q0[8], q1[8];
+      uint8_t s0, s1;
+      quant_col_pair<T>(tile + (32 * rb) * LD + 2 * pcol, LD, q0, q1, s0, s1);
+      const int64_t grow = b * a.cols + col;  // row of the transposed matrix
+      uint4* d0 = reinterpret_cast<uint4*>(a.col_data + grow * a.out_rows + orow);
+      uint4* d1 = reinterpret_cast<uint4*>(a.col_data + (grow + 1) * a.out_rows + orow);
+      d0[0] = make_uint4(q0[0], q0[1], q0[2], q0[3]);
+      d0[1] = make_uint4(q0[4], q0[5], q0[6], q0[7]);
+      d1[0] = make_uint4(q1[0], q1[1], q1[2], q1[3]);
+      d1[1] = make_uint4(q1[4], q1[5], q1[6], q1[7]);
+      a.col_sf[sf_offset(a.col_layout, a.batch * a.cols, a.out_rows, grow, orow / 32)] = s0;
+      a.col_sf[sf_offset(a.col_layout, a.batch * a.cols, a.out_rows, grow + 1, orow / 32)] = s1;
+    }
   }
 }
 
 template <typename T>
 static cudaError_t launch_q(const QuantArgs& a, cudaStream_t st) {
   using Tr = SrcTraits<T>;
-  const size_t smem = 2 * (size_t)kQTile * (kQTile + Tr::kPad) * sizeof(T);
+  const size_t smem = (size_t)kQTile * (kQTile + Tr::kPad) * sizeof(T);
   cudaError_t e =
       cudaFuncSetAttribute(mxfp8_quantize_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int64_t tiles = a.batch * ((a.out_rows + kQTile - 1) / kQTile) * ((a.cols + kQTile - 1) / kQTile);
-  if (tiles == 0) return cudaSuccess;
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mxfp8_quantize_kernel<T>, kQThreads, smem);
-  if (e != cudaSuccess) return e;
-  const int64_t grid = std::min<int64_t>(tiles, (int64_t)gemm_num_sms() * std::max(per_sm, 1));
-  mxfp8_quantize_kernel<T><<<(unsigned)grid, kQThreads, smem, st>>>(a);
+  dim3 grid((unsigned)((a.cols + kQTile - 1) / kQTile), (unsigned)((a.out_rows + kQTile - 1) / kQTile),
+            (unsigned)a.batch);
+  if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
+  mxfp8_quantize_kernel<T><<<grid, kQThreads, smem, st>>>(a);
   ++g_launch_count;
   return cudaGetLastError();
 }
