@@ -26,16 +26,25 @@ constexpr int kQThreads = 256;
 
 template <typename T>
 struct SrcTraits;
+// Shared tile layout: each 32-element block of a row is followed by 16 bytes of padding
+// (block stride kBS elements, row stride 4 * kBS). With 4 lanes per row (one per block)
+// the rowwise 16-byte loads, and with consecutive column pairs per warp the colwise
+// 4-/8-byte loads, hit distinct banks.
 template <>
 struct SrcTraits<__nv_bfloat16> {
-  static constexpr int kPad = 8;  // elements of row padding in shared memory (16 bytes)
-  static constexpr int kVec = 8;  // elements per 16-byte vector
+  static constexpr int kVec = 8;   // elements per 16-byte vector
+  static constexpr int kBS = 40;   // 32 elements + 16 bytes
 };
 template <>
 struct SrcTraits<float> {
-  static constexpr int kPad = 4;
   static constexpr int kVec = 4;
+  static constexpr int kBS = 36;
 };
+template <typename T>
+__device__ __forceinline__ int tile_off(int row, int col) {
+  using Tr = SrcTraits<T>;
+  return row * (4 * Tr::kBS) + (col >> 5) * Tr::kBS + (col & 31);
+}
 
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 __device__ __forceinline__ float to_f32(float v) { return v; }
@@ -157,7 +166,6 @@ __device__ __forceinline__ void quant_col_pair<float>(const float* p, int ld, ui
 template <typename T>
 __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quantize_kernel(QuantArgs a) {
   using Tr = SrcTraits<T>;
-  constexpr int LD = kQTile + Tr::kPad;
   extern __shared__ __align__(16) uint8_t q_smem_raw[];
   T* tile = reinterpret_cast<T*>(q_smem_raw);
 
@@ -193,21 +201,22 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
       buf[k] = srow[k] >= 0 ? __ldg(reinterpret_cast<const uint4*>(src + srow[k] * a.cols + col))
                             : make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int k = 0; k < NL; ++k) *reinterpret_cast<uint4*>(tile + (row_t + k * RSTEP) * LD + cv * Tr::kVec) = buf[k];
+    for (int k = 0; k < NL; ++k)
+      *reinterpret_cast<uint4*>(tile + tile_off<T>(row_t + k * RSTEP, cv * Tr::kVec)) = buf[k];
   }
   __syncthreads();
 
-  // ---- rowwise: item = (32-column block, row); a warp takes 32 consecutive rows of one
-  // block, so its 16-byte shared loads hit distinct banks (row stride = 4 banks mod 32)
+  // ---- rowwise: item = (row, 32-column block); 4 lanes cover a row, so a warp stores 8
+  // whole 128-byte lines
   if (a.row_data) {
 #pragma unroll 1
     for (int it = threadIdx.x; it < kQTile * 4; it += kQThreads) {
-      const int row = it & (kQTile - 1), blk = it >> 7;
+      const int row = it >> 2, blk = it & 3;
       const int64_t orow = r0 + row;
       const int64_t col = c0 + 32 * blk;
       if (orow >= nvalid || col >= a.cols) continue;
       uint32_t q[8];
-      const uint8_t sb = quant_row_block<T>(tile + row * LD + 32 * blk, q);
+      const uint8_t sb = quant_row_block<T>(tile + tile_off<T>(row, 32 * blk), q);
       const int64_t grow = b * a.out_rows + orow;
       uint4* dst = reinterpret_cast<uint4*>(a.row_data + grow * a.cols + col);
       dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
@@ -224,7 +233,7 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
     if (orow < nvalid && col < a.cols) {
       uint32_t q0[8], q1[8];
       uint8_t s0, s1;
-      quant_col_pair<T>(tile + (32 * rb) * LD + 2 * pcol, LD, q0, q1, s0, s1);
+      quant_col_pair<T>(tile + tile_off<T>(32 * rb, 2 * pcol), 4 * Tr::kBS, q0, q1, s0, s1);
       const int64_t grow = b * a.cols + col;  // row of the transposed matrix
       uint4* d0 = reinterpret_cast<uint4*>(a.col_data + grow * a.out_rows + orow);
       uint4* d1 = reinterpret_cast<uint4*>(a.col_data + (grow + 1) * a.out_rows + orow);
@@ -241,7 +250,7 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
 template <typename T>
 static cudaError_t launch_q(const QuantArgs& a, cudaStream_t st) {
   using Tr = SrcTraits<T>;
-  const size_t smem = (size_t)kQTile * (kQTile + Tr::kPad) * sizeof(T);
+  const size_t smem = (size_t)kQTile * 4 * Tr::kBS * sizeof(T);
   cudaError_t e =
       cudaFuncSetAttribute(mxfp8_quantize_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
