@@ -129,6 +129,29 @@ mxmoe_status moe_permute(const int32_t* topk_idx_dev, const float* probs_dev, in
 size_t moe_permute_workspace_size(int32_t T, int32_t k, int32_t E);
 
 /*
+ * moe_permute_noalloc -- the same routing index as moe_permute, for callers that cannot
+ * provide a scratch buffer (no counterpart in the pages: it is a calling convenience).
+ * Such callers include serving runtimes that plan all device memory ahead of time and
+ * have no free buffer to lend per call, and plain C callers without a device allocator.
+ * It allocates nothing and takes no workspace: its scratch is a fixed 256 KiB array in
+ * the library's own device memory, present on every GPU that loads the library until
+ * the process exits.
+ *   Arguments and outputs: as moe_permute.
+ *   Limit: 8 * ceil(T / 256) * E + 256 bytes of scratch must fit in 256 KiB (e.g.
+ *   T = 65536 with E = 128, or T = 32768 with E = 256); larger problems return
+ *   MXMOE_ERR_WORKSPACE_TOO_SMALL and enqueue nothing.
+ *   The first call on a device looks up the array's device address (once per device,
+ *   with that device current); make that first call before any stream capture.
+ *   All calls on a device share the one array: calls that may overlap on the GPU (for
+ *   example on two streams without ordering between them) race and must be serialised
+ *   by the caller. Nothing in the array needs clearing between calls: every word a call
+ *   reads, it has written first.
+ */
+mxmoe_status moe_permute_noalloc(const int32_t* topk_idx_dev, const float* probs_dev, int32_t T, int32_t k,
+                                 int32_t E, int32_t* m_splits_dev, int32_t* seg_off_dev, int32_t* row_of_slot_dev,
+                                 int32_t* token_of_row_dev, float* prob_of_row_dev, void* stream);
+
+/*
  * moe_unpermute -- returns routed rows to token order and sums the k copies of each
  * token: y[t] = sum_{j<k} y_perm[row_of_slot[t, j]], accumulated in fp32 in slot order
  * and rounded once to bf16 (the pages are silent on the combine; this is the plain

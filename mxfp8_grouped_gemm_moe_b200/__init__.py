@@ -56,6 +56,7 @@ _SIGNATURES = {
     "mxmoe_rows_capacity": (_I64, [_I32, _I32, _I32]),
     "moe_permute": (_I32, [_P, _P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_permute_workspace_size": (_SZ, [_I32, _I32, _I32]),
+    "moe_permute_noalloc": (_I32, [_P, _P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P]),
     "moe_unpermute": (_I32, [_P, _P, _I32, _I32, _I32, _P, _P]),
     "mxfp8_quantize": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _I64, _PMX, _PMX, _P]),
     "grouped_gemm_mxfp8": (_I32, [_PMX, _PMX, _P, _I32, _I64, _I64, _P, _I32, _I64, _P]),
