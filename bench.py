@@ -468,9 +468,9 @@ def main():
     import moe_workloads as wl
     cfg = wl.CONFIGS[args.config]
     if args.tokens:
-        cfg = dataclasses.replace(cfg, T=args.tokens)
+        cfg = dataclasses.replace(cfg, T=args.tokens, name=f"{cfg.name}_T{args.tokens}")
     if args.experts:
-        cfg = dataclasses.replace(cfg, E=args.experts, k=min(cfg.k, args.experts))
+        cfg = dataclasses.replace(cfg, E=args.experts, k=min(cfg.k, args.experts), name=f"{cfg.name}_E{args.experts}")
     try:
         if args.impl == "reference":
             run_reference(args, cfg, dist, rank, world)
