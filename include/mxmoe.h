@@ -33,7 +33,7 @@
  *     -127), scale byte = X + 127, element = E4M3(v * 2^-X) rounded to nearest-even
  *     and saturated to +-448.
  *   - Routed rows are ordered by (expert ascending, token ascending). Expert e's
- *     segment of rows starts at seg_off[e], a multiple of 128; its first m_splits[e]
+ *     segment of rows starts at seg_off[e], a multiple of 256; its first m_splits[e]
  *     rows are live, the rest up to seg_off[e+1] are zero pad rows. The buffers of
  *     permuted rows hold mxmoe_rows_capacity(T, k, E) rows.
  */
@@ -97,7 +97,7 @@ mxmoe_status mxmoe_get_device_status(int32_t* out_host, int32_t* where_host, voi
 mxmoe_status mxmoe_clear_device_status(void* stream);
 
 /* Upper bound on the number of permuted rows (live + pad) for T tokens, top-k and E
- * experts: roundup(T*k + 127*E, 128). Every [Mp, *] buffer below has this many rows. */
+ * experts: roundup(T*k + 255*E, 256). Every [Mp, *] buffer below has this many rows. */
 int64_t mxmoe_rows_capacity(int32_t T, int32_t k, int32_t E);
 
 /* ------------------------------------------------------------------ routing (GroupedLinear input) */
@@ -112,7 +112,7 @@ int64_t mxmoe_rows_capacity(int32_t T, int32_t k, int32_t E);
  *   probs_dev     float [T, k]  routing probabilities (nullable if prob_of_row_dev is).
  *   Outputs (device, caller-owned):
  *   m_splits_dev     int32 [E]     tokens per expert
- *   seg_off_dev      int32 [E+1]   start row of each expert segment (multiples of 128);
+ *   seg_off_dev      int32 [E+1]   start row of each expert segment (multiples of 256);
  *                                  seg_off[E] = Mp, the padded row count
  *   row_of_slot_dev  int32 [T, k]  permuted row of each (token, slot)
  *   token_of_row_dev int32 [mxmoe_rows_capacity]  token of each row, -1 on pad rows
@@ -191,12 +191,16 @@ mxmoe_status mxfp8_quantize(const void* src_dev, int32_t src_dtype, int64_t batc
  * des modèles biologiques", first improvement): for every expert e,
  *     C[seg_e, :] = dequant(A)[seg_e, :] . dequant(B_e)^T,   seg_e = [seg_off[e], seg_off[e+1])
  * with fp32 accumulation on the tensor cores.
- *   A   MXFP8 [rows_cap, K], MXMOE_SCALE_MMA; rows_cap % 128 == 0.
+ *   A   MXFP8 [rows_cap, K], MXMOE_SCALE_MMA; rows_cap % 256 == 0.
  *   B   MXFP8 [E*N, K], MXMOE_SCALE_MMA (expert e's rows are [e*N, (e+1)*N)).
- *   seg_off_dev  int32 [E+1], multiples of 128, read on the device (no host sync).
+ *   seg_off_dev  int32 [E+1], multiples of 256, read on the device (no host sync).
  *   C_dev [rows_cap, ldc] of c_dtype (MXMOE_DTYPE_BF16 or _F32); rows >= seg_off[E]
  *         are not written.
  * Shapes: N % 256 == 0, K % 128 == 0, ldc >= N, ldc % 8 == 0.
+ * Errors: host-checkable argument and shape errors are returned; segment offsets that
+ * are not non-decreasing multiples of 256 starting at 0 and ending at most at rows_cap
+ * are caught on the device (nothing is computed; mxmoe_get_device_status then reports
+ * MXMOE_ERR_DEVICE_CHECK).
  */
 mxmoe_status grouped_gemm_mxfp8(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, const int32_t* seg_off_dev,
                                 int32_t E, int64_t N, int64_t K, void* C_dev, int32_t c_dtype, int64_t ldc,
@@ -209,7 +213,8 @@ mxmoe_status grouped_gemm_mxfp8(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, cons
  *   At  MXFP8 [N, rows_cap] (colwise-transposed activations/gradients), MXMOE_SCALE_MMA.
  *   Bt  MXFP8 [K2, rows_cap], MXMOE_SCALE_MMA.
  *   C_dev float [E, N, K2].
- * Shapes: N % 128 == 0, K2 % 256 == 0.
+ * Shapes: N % 256 == 0, K2 % 256 == 0, rows_cap % 256 == 0. Segment offsets are
+ * checked on the device as for grouped_gemm_mxfp8.
  */
 mxmoe_status grouped_gemm_mxfp8_wgrad(const mxmoe_mxfp8* At, const mxmoe_mxfp8* Bt, const int32_t* seg_off_dev,
                                       int32_t E, float* C_dev, void* stream);
@@ -223,6 +228,9 @@ mxmoe_status grouped_gemm_mxfp8_wgrad(const mxmoe_mxfp8* At, const mxmoe_mxfp8* 
  *   W1 colwise  [E*H, 2F]  (fc1 data-gradient operand; blocks along 2F)
  *   W2 rowwise  [E*H, F]   (fc2 forward operand; blocks along F)
  *   W2 colwise  [E*F, H]   (fc2 data-gradient operand; blocks along H)
+ * The W1 rowwise copy keeps each expert's rows in 64-row blocks interleaved gate / up
+ * (gate 0..63, up 0..63, gate 64..127, ...), so that one 128-row operand tile holds
+ * matching gate and up columns; the other three copies keep the natural row order.
  * W1_dev bf16 [E, 2F, H] (rows 0..F-1 gate, F..2F-1 up; nn.Linear out x in),
  * W2_dev bf16 [E, H, F]. Requires H % 256 == 0, F % 256 == 0.
  */

@@ -22,7 +22,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 inline mxmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MXMOE_OK : MXMOE_ERR_CUDA; }
 
-int64_t rows_cap(int64_t T, int64_t k, int64_t E) { return (T * k + 127 * E + 127) / 128 * 128; }
+int64_t rows_cap(int64_t T, int64_t k, int64_t E) { return (T * k + 255 * E + 255) / 256 * 256; }
 
 // Sub-buffers of a caller-provided byte buffer, each 256-byte aligned.
 struct Carver {
@@ -256,9 +256,12 @@ mxmoe_status moe_unpermute(const void* y_perm_dev, const int32_t* row_of_slot_de
   return cuda_status(launch_unpermute(y_perm_dev, row_of_slot_dev, T, k, H, y_dev, S(stream)));
 }
 
-mxmoe_status mxfp8_quantize(const void* src_dev, int32_t src_dtype, int64_t batch, int64_t rows, int64_t cols,
-                            const int32_t* row_gather_dev, const int32_t* nrows_dev, int64_t out_rows,
-                            const mxmoe_mxfp8* out_row, const mxmoe_mxfp8* out_colT, void* stream) {
+// mxfp8_quantize with an optional gate/up row interleave of the rowwise copy (row_ilv =
+// half the rows of each batch matrix; the library uses it for the fc1 weight operand).
+static mxmoe_status quantize_impl(const void* src_dev, int32_t src_dtype, int64_t batch, int64_t rows, int64_t cols,
+                                  const int32_t* row_gather_dev, const int32_t* nrows_dev, int64_t out_rows,
+                                  const mxmoe_mxfp8* out_row, const mxmoe_mxfp8* out_colT, int64_t row_ilv,
+                                  void* stream) {
   if (src_dtype != MXMOE_DTYPE_BF16 && src_dtype != MXMOE_DTYPE_F32) return MXMOE_ERR_INVALID_ARG;
   if (!src_dev || !aligned16(src_dev) || (!out_row && !out_colT)) return MXMOE_ERR_INVALID_ARG;
   if (batch < 1 || rows < 0 || cols <= 0 || out_rows < 0) return MXMOE_ERR_UNSUPPORTED_SHAPE;
@@ -293,8 +296,16 @@ mxmoe_status mxfp8_quantize(const void* src_dev, int32_t src_dtype, int64_t batc
   a.col_data = out_colT ? out_colT->data : nullptr;
   a.col_sf = out_colT ? out_colT->scale : nullptr;
   a.col_layout = out_colT ? out_colT->scale_layout : 0;
+  a.row_ilv = row_ilv;
   StageScope sc(MXMOE_STAGE_QUANT, S(stream));
   return cuda_status(launch_quantize(a, S(stream)));
+}
+
+mxmoe_status mxfp8_quantize(const void* src_dev, int32_t src_dtype, int64_t batch, int64_t rows, int64_t cols,
+                            const int32_t* row_gather_dev, const int32_t* nrows_dev, int64_t out_rows,
+                            const mxmoe_mxfp8* out_row, const mxmoe_mxfp8* out_colT, void* stream) {
+  return quantize_impl(src_dev, src_dtype, batch, rows, cols, row_gather_dev, nrows_dev, out_rows, out_row, out_colT, 0,
+                       stream);
 }
 
 mxmoe_status grouped_gemm_mxfp8(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, const int32_t* seg_off_dev,
@@ -304,7 +315,7 @@ mxmoe_status grouped_gemm_mxfp8(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, cons
   if (c_dtype != MXMOE_DTYPE_BF16 && c_dtype != MXMOE_DTYPE_F32) return MXMOE_ERR_INVALID_ARG;
   if (!mma_ready(A) || !mma_ready(B)) return MXMOE_ERR_INVALID_ARG;
   if (E < 1 || E > 256 || N <= 0 || K <= 0 || N % 256 != 0 || K % 128 != 0) return MXMOE_ERR_UNSUPPORTED_SHAPE;
-  if (A->cols != K || B->cols != K || B->rows != (int64_t)E * N || ldc < N || ldc % 8 != 0)
+  if (A->rows % 256 != 0 || A->cols != K || B->cols != K || B->rows != (int64_t)E * N || ldc < N || ldc % 8 != 0)
     return MXMOE_ERR_UNSUPPORTED_SHAPE;
   if (A->rows == 0) return MXMOE_OK;
   GemmArgs g = gemm_base(kModeStore, *A, *B, seg_off_dev, E);
@@ -321,7 +332,8 @@ mxmoe_status grouped_gemm_mxfp8_wgrad(const mxmoe_mxfp8* At, const mxmoe_mxfp8* 
                                       int32_t E, float* C_dev, void* stream) {
   if (!At || !Bt || !seg_off_dev || !C_dev || !aligned16(C_dev)) return MXMOE_ERR_INVALID_ARG;
   if (!mma_ready(At) || !mma_ready(Bt)) return MXMOE_ERR_INVALID_ARG;
-  if (E < 1 || E > 256 || At->cols != Bt->cols || At->rows <= 0 || Bt->rows % 256 != 0 || Bt->rows <= 0)
+  if (E < 1 || E > 256 || At->cols != Bt->cols || At->rows <= 0 || At->rows % 256 != 0 || Bt->rows % 256 != 0 ||
+      Bt->rows <= 0 || At->cols % 256 != 0)
     return MXMOE_ERR_UNSUPPORTED_SHAPE;
   GemmArgs g = gemm_base(kModeWgrad, *At, *Bt, seg_off_dev, E);
   g.N = At->rows;
@@ -357,8 +369,8 @@ mxmoe_status mxmoe_weights_quantize(const void* W1_dev, const void* W2_dev, int3
   mxmoe_status s;
   {
     StageScope sc(MXMOE_STAGE_QUANT_W1, S(stream));
-    s = mxfp8_quantize(W1_dev, MXMOE_DTYPE_BF16, E, 2 * (int64_t)F, H, nullptr, nullptr, 2 * (int64_t)F, &w1r,
-                       &w1c, stream);
+    s = quantize_impl(W1_dev, MXMOE_DTYPE_BF16, E, 2 * (int64_t)F, H, nullptr, nullptr, 2 * (int64_t)F, &w1r, &w1c,
+                      F, stream);
   }
   if (s != MXMOE_OK) return s;
   StageScope sc(MXMOE_STAGE_QUANT_W2, S(stream));

@@ -9,23 +9,34 @@
 // arquitetura MoE" (conexaotc.com.br) adds that quantisation is part of that fusion.
 //
 // Design (B200):
-//  * one CTA per SM, persistent over a linear tile list; expert segments are 128-row
-//    aligned, so an M tile never straddles two experts and its expert is found from
-//    the device-side segment offsets (no host synchronisation on m_splits);
-//  * tile 128 x 256 x 128 (M x N x K), 4-stage TMA -> shared-memory ring; operand
-//    tiles use the 128-byte swizzle; the E8M0 scales arrive with plain bulk copies in
-//    the tensor cores' scale order and are moved to TMEM with tcgen05.cp;
+//  * persistent over a linear tile list; expert segments are 256-row aligned, so an M
+//    tile never straddles two experts and its expert is found from the device-side
+//    segment offsets (no host synchronisation on m_splits);
+//  * two variants of one kernel template (PAIR):
+//      PAIR = 2 (default): a cluster of two CTAs on neighbouring SMs computes a 256 x 256
+//        output tile with one tcgen05 instruction stream (cta_group::2, M = 256). Each
+//        CTA stages its own 128 rows of A and its half (128 rows) of B per K step, so
+//        a B tile crosses L2 -> SM once per pair instead of once per CTA; every TMA of
+//        both CTAs completes on the leader's stage barrier and the leader's commits
+//        release the stage in both CTAs (multicast commit; the loads themselves are
+//        never multicast). 6-stage ring of 34 KB.
+//      PAIR = 1: one CTA per SM, tile 128 x 256, 4-stage ring of 50 KB.
+//    Each CTA ends a tile with the same 128 x 256 fp32 accumulator in its own TMEM, so
+//    the epilogues are shared by both variants;
+//  * K step 128; operand tiles use the 128-byte swizzle; the E8M0 scales arrive in the
+//    tensor cores' scale order and are moved to TMEM with tcgen05.cp;
 //  * warp 0 issues the copies, warp 1 issues tcgen05.mma (kind::mxf8f6f4, block32
-//    scales), warps 2..9 are the epilogue: they drain the 128 x 256 fp32 accumulator
-//    from TMEM into registers, hand TMEM back to the MMA warp at once, then run the
-//    epilogue math and stores while the next tile's MMAs proceed;
+//    scales), warps 2..9 are the epilogue: they drain the accumulator from TMEM into
+//    registers (or spare TMEM columns), hand it back to the MMA warp at once, then run
+//    the epilogue math and stores while the next tile's MMAs proceed;
 //  * every wait is bounded (1 s) and reports MXMOE_ERR_DEVICE_TIMEOUT instead of
-//    hanging; no cluster, no multicast.
+//    hanging; the segment offsets are checked on the device before any tile is issued.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -35,93 +46,95 @@
 
 namespace mxmoe {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 128;
-#ifndef MXMOE_STAGES
-#define MXMOE_STAGES 4
-#endif
-constexpr int STAGES = MXMOE_STAGES;
+constexpr int BN = 256;  // output tile columns (both variants)
+constexpr int BK = 128;  // K per pipeline stage
 constexpr int kThreads = 320;  // 10 warps
 constexpr int kEpiWarps = 8;
 
-constexpr uint32_t kABytes = BM * BK;       // 16 KB
-constexpr uint32_t kBBytes = BN * BK;       // 32 KB
-constexpr uint32_t kSfaBytes = 512;         // 128 rows x 4 scale bytes
-constexpr uint32_t kSfbBytes = 1024;        // 256 rows x 4 scale bytes
-constexpr uint32_t kStageBytes = 51200;     // A + B + SFA + SFB, padded to 1 KB
-constexpr uint32_t kTxBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+constexpr uint32_t kABytes = 128 * BK;  // this CTA's 128 rows of A per stage
+constexpr uint32_t kSfaBytes = 512;     // 128 rows x 4 scale bytes
+constexpr uint32_t kSfbBytes = 1024;    // 256 rows x 4 scale bytes
 constexpr uint32_t kStagingPerWarp = 2048;  // colwise transpose staging
-constexpr uint32_t kOffStaging = STAGES * kStageBytes;
-constexpr uint32_t kOffBars = kOffStaging + kEpiWarps * kStagingPerWarp;
 constexpr int kMaxE = 256;
-constexpr uint32_t kOffSeg = kOffBars + 256;
-constexpr uint32_t kOffOrder = kOffSeg + (kMaxE + 1) * 4 + 12;
-constexpr uint32_t kSmemUsed = kOffOrder + kMaxE * 4;
-constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack for 1 KB alignment
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemSfa = 256;  // two buffers of 4 columns
-constexpr uint32_t kTmemSfb = 264;  // two buffers of 8 columns
+constexpr uint32_t kTmemSfa = 256;    // two buffers of 4 columns
+constexpr uint32_t kTmemSfb = 264;    // two buffers of 8 columns
 constexpr uint32_t kTmemStash = 384;  // epilogue scratch: 64 columns per (lane quadrant, half)
-constexpr int GROUP_M = 16;         // m tiles per raster group (L2 reuse of B)
 
-static_assert(kStageBytes >= kTxBytes && kStageBytes % 1024 == 0, "stage layout");
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+template <int PAIR>
+struct Cfg {
+  static constexpr int TM = 128 * PAIR;                        // output tile rows
+  static constexpr int STAGES = PAIR == 2 ? 6 : 4;
+  static constexpr uint32_t kBBytes = (BN / PAIR) * BK;        // this CTA's B rows per stage
+  static constexpr uint32_t kStageBytes = PAIR == 2 ? 34816 : 51200;
+  static constexpr uint32_t kTxBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // per CTA
+  static constexpr uint32_t kOffStaging = STAGES * kStageBytes;
+  static constexpr uint32_t kOffBars = kOffStaging + kEpiWarps * kStagingPerWarp;
+  static constexpr uint32_t kOffSeg = kOffBars + 256;
+  static constexpr uint32_t kOffOrder = kOffSeg + (kMaxE + 1) * 4 + 12;
+  static constexpr uint32_t kSmemBytes = kOffOrder + kMaxE * 4 + 1024;  // + slack for 1 KB alignment
+  static constexpr int GROUP_M = 16 / PAIR;                    // M tiles per raster group (2048 rows)
+  static_assert(kStageBytes >= kTxBytes && kStageBytes % 1024 == 0, "stage layout");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
 
 struct TileInfo {
   int32_t e;
   int32_t k_iters;
-  int32_t a_y, a_x0;
-  int32_t b_y0, b_y1, b_x0;
+  int32_t a_y, a_x0;      // this CTA's A rows start, K start
+  int32_t b_y0, b_y1, b_x0;  // the tile's two 128-row B halves, K start
   int32_t n_tile;
-  int64_t row0;  // output row base
+  int64_t row0;  // this CTA's output row base
 };
 
-template <int MODE>
+template <int MODE, int PAIR>
 __device__ __forceinline__ int32_t n_tiles_of(const GemmArgs& g) {
   if (MODE == kModeStore) return (int32_t)(g.N / BN);
   if (MODE == kModeSwigluFwd) return (int32_t)(g.F / 128);
   if (MODE == kModeSwigluBwd) return (int32_t)(g.F / BN);
-  return (int32_t)((g.N / BM) * (g.K2 / BN));  // per expert, wgrad
+  return (int32_t)((g.N / Cfg<PAIR>::TM) * (g.K2 / BN));  // per expert, wgrad
 }
 
-template <int MODE>
+template <int MODE, int PAIR>
 __device__ __forceinline__ int64_t total_tiles(const GemmArgs& g, const int32_t* s_seg) {
-  if (MODE == kModeWgrad) return (int64_t)g.E * n_tiles_of<MODE>(g);
-  return (int64_t)(s_seg[g.E] / BM) * n_tiles_of<MODE>(g);
+  if (MODE == kModeWgrad) return (int64_t)g.E * n_tiles_of<MODE, PAIR>(g);
+  return (int64_t)(s_seg[g.E] / Cfg<PAIR>::TM) * n_tiles_of<MODE, PAIR>(g);
 }
 
-template <int MODE>
-__device__ __forceinline__ TileInfo get_tile(const GemmArgs& g, int64_t idx, const int32_t* s_seg,
-                                             const int32_t* s_order) {
+// Tile `idx` of the launch as seen by CTA `rank` of its pair (rank 0 when PAIR == 1).
+template <int MODE, int PAIR>
+__device__ __forceinline__ TileInfo get_tile(const GemmArgs& g, int32_t idx, const int32_t* s_seg,
+                                             const int32_t* s_order, uint32_t rank) {
+  constexpr int TM = Cfg<PAIR>::TM;
+  constexpr int GROUP_M = Cfg<PAIR>::GROUP_M;
   TileInfo t;
   if (MODE == kModeWgrad) {
-    const int32_t per = n_tiles_of<MODE>(g);
+    const int32_t per = n_tiles_of<MODE, PAIR>(g);
     const int32_t nk2 = (int32_t)(g.K2 / BN);
-    const int32_t pos = (int32_t)(idx / per), r = (int32_t)(idx % per);
+    const int32_t pos = idx / per, r = idx % per;
     const int32_t e = s_order[pos];
     const int32_t n_t = r / nk2, k2_t = r % nk2;
     t.e = e;
     t.k_iters = (s_seg[e + 1] - s_seg[e]) / BK;
-    t.a_y = n_t * BM;
+    t.a_y = n_t * TM + 128 * (int32_t)rank;
     t.a_x0 = s_seg[e];
     t.b_y0 = k2_t * BN;
     t.b_y1 = t.b_y0 + 128;
     t.b_x0 = s_seg[e];
     t.n_tile = k2_t;
-    t.row0 = (int64_t)e * g.N + (int64_t)n_t * BM;
+    t.row0 = (int64_t)e * g.N + t.a_y;
     return t;
   }
-  const int32_t ntn = n_tiles_of<MODE>(g);
-  const int32_t num_m = s_seg[g.E] / BM;
-  const int64_t group_size = (int64_t)GROUP_M * ntn;
-  const int32_t grp = (int32_t)(idx / group_size);
-  const int32_t r = (int32_t)(idx % group_size);
+  const int32_t ntn = n_tiles_of<MODE, PAIR>(g);
+  const int32_t num_m = s_seg[g.E] / TM;
+  const int32_t group_size = GROUP_M * ntn;
+  const int32_t grp = idx / group_size;
+  const int32_t r = idx % group_size;
   const int32_t m0 = grp * GROUP_M;
   const int32_t gm = min(GROUP_M, num_m - m0);
   const int32_t m_t = m0 + r % gm;
   const int32_t n_t = r / gm;
-  const int32_t row = m_t * BM;
+  const int32_t row = m_t * TM;
   // expert = the e with s_seg[e] <= row < s_seg[e+1] (segments of empty experts have
   // zero length and are skipped by the search)
   int32_t lo = 0, hi = g.E - 1;
@@ -133,18 +146,19 @@ __device__ __forceinline__ TileInfo get_tile(const GemmArgs& g, int64_t idx, con
   const int32_t e = lo;
   t.e = e;
   t.k_iters = (int32_t)(g.K / BK);
-  t.a_y = row;
+  t.a_y = row + 128 * (int32_t)rank;
   t.a_x0 = 0;
   t.b_x0 = 0;
   t.n_tile = n_t;
-  t.row0 = row;
+  t.row0 = t.a_y;
   if (MODE == kModeSwigluFwd) {
-    t.b_y0 = (int32_t)(e * 2 * g.F + (int64_t)n_t * 128);
-    t.b_y1 = (int32_t)(e * 2 * g.F + g.F + (int64_t)n_t * 128);
+    // the rowwise W1 copy interleaves gate / up rows in 64-row blocks: FFN columns
+    // [128 n_t, 128 n_t + 128) are rows [256 n_t, 256 n_t + 256) = gate 64 | up 64 | gate 64 | up 64
+    t.b_y0 = (int32_t)(e * 2 * g.F + (int64_t)n_t * 256);
   } else {
     t.b_y0 = (int32_t)((int64_t)e * g.N + (int64_t)n_t * BN);
-    t.b_y1 = t.b_y0 + 128;
   }
+  t.b_y1 = t.b_y0 + 128;
   return t;
 }
 
@@ -218,11 +232,16 @@ __device__ __forceinline__ void rowwise_quant_store(const float (&v)[32], uint8_
 }
 
 // Hands the accumulator back to the MMA warp once this warp's TMEM reads (and writes
-// to its spare columns) have completed.
-__device__ __forceinline__ void release_accumulator(uint64_t* bar_acc_empty, int lane) {
+// to its spare columns) have completed. `acc_empty` is the leader CTA's barrier (a
+// cluster address when PAIR == 2).
+template <int PAIR>
+__device__ __forceinline__ void release_accumulator(uint64_t* bar_local, uint32_t acc_empty_cluster, int lane) {
   ptx::tc_fence_before();
   __syncwarp();
-  if (lane == 0) ptx::mbar_arrive(bar_acc_empty);
+  if (lane == 0) {
+    if (PAIR == 1) ptx::mbar_arrive(bar_local);
+    else ptx::mbar_arrive_cluster(acc_empty_cluster);
+  }
 }
 
 // 8 fp32 (bit patterns) starting at v[i0] -> 8 bf16 in one 16-byte vector.
@@ -236,87 +255,132 @@ __device__ __forceinline__ uint4 pack8_bf16(const uint32_t (&v)[N], int i0) {
   return o;
 }
 
-template <int MODE>
+template <int MODE, int PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     mxgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                   const __grid_constant__ GemmArgs g) {
+  using C = Cfg<PAIR>;
+  constexpr int STAGES = C::STAGES;
+  constexpr uint32_t kStageBytes = C::kStageBytes;
+  constexpr uint32_t kBBytes = C::kBBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + kOffBars);
+  uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
   uint64_t* bar_empty = bar_full + STAGES;
   uint64_t* bar_acc_full = bar_empty + STAGES;
-  uint64_t* bar_acc_empty = bar_acc_full + 1;
+  uint64_t* bar_acc_empty = bar_acc_full + 1;  // used in the leader CTA only
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_acc_empty + 1);
   volatile int32_t* s_abort = reinterpret_cast<volatile int32_t*>(s_tmem + 1);
-  int32_t* s_seg = reinterpret_cast<int32_t*>(smem + kOffSeg);
-  int32_t* s_order = reinterpret_cast<int32_t*>(smem + kOffOrder);
+  int32_t* s_bad = const_cast<int32_t*>(s_abort + 1);
+  int32_t* s_seg = reinterpret_cast<int32_t*>(smem + C::kOffSeg);
+  int32_t* s_order = reinterpret_cast<int32_t*>(smem + C::kOffOrder);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR == 2 ? ptx::cluster_rank() : 0u;
+  const int32_t first = (int32_t)(blockIdx.x / PAIR), stride = (int32_t)(gridDim.x / PAIR);
 
   // ---- setup
-  for (int i = threadIdx.x; i <= g.E; i += blockDim.x) s_seg[i] = g.seg_off[i];
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(&bar_full[s], 1);
       ptx::mbar_init(&bar_empty[s], 1);
     }
     ptx::mbar_init(bar_acc_full, 1);
-    ptx::mbar_init(bar_acc_empty, kEpiWarps);
+    ptx::mbar_init(bar_acc_empty, kEpiWarps * PAIR);
     *s_abort = 0;
+    *s_bad = 0;
     ptx::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tensormap(&tmA);
     ptx::prefetch_tensormap(&tmB);
+    if (PAIR == 2) {
+      ptx::prefetch_tensormap(&tmSFA);
+      ptx::prefetch_tensormap(&tmSFB);
+    }
   }
   if (warp == 1) {
-    ptx::tmem_alloc(s_tmem, kTmemCols);
-    ptx::tmem_relinquish();
+    if (PAIR == 2) {
+      ptx::tmem_alloc_pair(s_tmem, kTmemCols);
+      ptx::tmem_relinquish_pair();
+    } else {
+      ptx::tmem_alloc(s_tmem, kTmemCols);
+      ptx::tmem_relinquish();
+    }
   }
   __syncthreads();
+  // segment offsets: non-decreasing, tile aligned, inside the token dimension of the
+  // operands; anything else is reported and no tile is issued
+  {
+    const int64_t tok_extent = MODE == kModeWgrad ? g.a_cols : g.a_rows;
+    for (int i = threadIdx.x; i <= g.E; i += blockDim.x) {
+      const int32_t v = g.seg_off[i];
+      s_seg[i] = v;
+      const bool bad = v < 0 || (v % C::TM) != 0 || v > tok_extent || (i == 0 && v != 0) ||
+                       (i > 0 && g.seg_off[i - 1] > v);
+      if (bad) *s_bad = 1;
+    }
+  }
+  __syncthreads();
+  if (*s_bad && blockIdx.x == 0 && threadIdx.x == 0) record_error(MXMOE_ERR_DEVICE_CHECK, 20);
   if (MODE == kModeWgrad) {
     // experts in decreasing size (largest first), ties by index
     for (int e = threadIdx.x; e < g.E; e += blockDim.x) {
       const int32_t me = s_seg[e + 1] - s_seg[e];
-      int32_t rank = 0;
+      int32_t rk = 0;
       for (int f = 0; f < g.E; ++f) {
         const int32_t mf = s_seg[f + 1] - s_seg[f];
-        rank += (mf > me) || (mf == me && f < e);
+        rk += (mf > me) || (mf == me && f < e);
       }
-      s_order[rank] = e;
+      s_order[rk] = e;
     }
   }
   ptx::tc_fence_before();
-  __syncthreads();
+  if (PAIR == 2) ptx::cluster_sync();  // barriers of both CTAs initialised, TMEM allocated in both
+  else __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
-  const int64_t ntiles = total_tiles<MODE>(g, s_seg);
+  const int32_t ntiles = *s_bad ? 0 : (int32_t)total_tiles<MODE, PAIR>(g, s_seg);
 
   if (warp == 0) {
-    // ===================================================== TMA producer
+    // ===================================================== TMA producer (every CTA)
     if (lane == 0) {
       int stage = 0;
       uint32_t ph = 0;
       const int64_t a_kchunks = g.a_cols / 128, b_kchunks = g.b_cols / 128;
-      for (int64_t tile = blockIdx.x; tile < ntiles && !*s_abort; tile += gridDim.x) {
-        const TileInfo t = get_tile<MODE>(g, tile, s_seg, s_order);
+      for (int32_t tile = first; tile < ntiles && !*s_abort; tile += stride) {
+        const TileInfo t = get_tile<MODE, PAIR>(g, tile, s_seg, s_order, rank);
         for (int kb = 0; kb < t.k_iters; ++kb) {
           if (!ptx::mbar_wait(&bar_empty[stage], ph ^ 1u, 1)) {
             *s_abort = 1;
             break;
           }
           uint8_t* sb = smem + stage * kStageBytes;
-          ptx::mbar_arrive_expect_tx(&bar_full[stage], kTxBytes);
           const int32_t kx_a = t.a_x0 + kb * BK, kx_b = t.b_x0 + kb * BK;
-          ptx::tma_load_2d(sb, &tmA, kx_a, t.a_y, &bar_full[stage]);
-          ptx::tma_load_2d(sb + kABytes, &tmB, kx_b, t.b_y0, &bar_full[stage]);
-          ptx::tma_load_2d(sb + kABytes + kBBytes / 2, &tmB, kx_b, t.b_y1, &bar_full[stage]);
+          // scale chunks: index of the 128 x 128 block in the MMA-order scale arrays
           const int64_t ca = (int64_t)(t.a_y / 128) * a_kchunks + kx_a / 128;
           const int64_t cb0 = (int64_t)(t.b_y0 / 128) * b_kchunks + kx_b / 128;
-          const int64_t cb1 = (int64_t)(t.b_y1 / 128) * b_kchunks + kx_b / 128;
-          ptx::bulk_load(sb + kABytes + kBBytes, g.a_sf + ca * 512, 512, &bar_full[stage]);
-          ptx::bulk_load(sb + kABytes + kBBytes + kSfaBytes, g.b_sf + cb0 * 512, 512, &bar_full[stage]);
-          ptx::bulk_load(sb + kABytes + kBBytes + kSfaBytes + 512, g.b_sf + cb1 * 512, 512, &bar_full[stage]);
+          const int64_t cb1 = cb0 + b_kchunks;
+          uint8_t* s_sfa = sb + kABytes + kBBytes;
+          if (PAIR == 1) {
+            ptx::mbar_arrive_expect_tx(&bar_full[stage], C::kTxBytes);
+            ptx::tma_load_2d(sb, &tmA, kx_a, t.a_y, &bar_full[stage]);
+            ptx::tma_load_2d(sb + kABytes, &tmB, kx_b, t.b_y0, &bar_full[stage]);
+            ptx::tma_load_2d(sb + kABytes + kBBytes / 2, &tmB, kx_b, t.b_y1, &bar_full[stage]);
+            ptx::bulk_load(s_sfa, g.a_sf + ca * 512, 512, &bar_full[stage]);
+            ptx::bulk_load(s_sfa + kSfaBytes, g.b_sf + cb0 * 512, 512, &bar_full[stage]);
+            ptx::bulk_load(s_sfa + kSfaBytes + 512, g.b_sf + cb1 * 512, 512, &bar_full[stage]);
+          } else {
+            // both CTAs' copies complete on the leader's barrier, which expects the pair's bytes
+            const uint32_t full_leader = ptx::map_to_rank(ptx::smem_u32(&bar_full[stage]), 0);
+            if (rank == 0) ptx::mbar_arrive_expect_tx(&bar_full[stage], 2 * C::kTxBytes);
+            ptx::tma_load_2d_pair(sb, &tmA, kx_a, t.a_y, full_leader);
+            ptx::tma_load_2d_pair(sb + kABytes, &tmB, kx_b, rank ? t.b_y1 : t.b_y0, full_leader);
+            ptx::tma_load_2d_pair(s_sfa, &tmSFA, 0, (int32_t)ca, full_leader);
+            ptx::tma_load_2d_pair(s_sfa + kSfaBytes, &tmSFB, 0, (int32_t)cb0, full_leader);
+            ptx::tma_load_2d_pair(s_sfa + kSfaBytes + 512, &tmSFB, 0, (int32_t)cb1, full_leader);
+          }
           if (++stage == STAGES) {
             stage = 0;
             ph ^= 1u;
@@ -325,13 +389,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ===================================================== MMA issuer
-    if (lane == 0) {
+    // ===================================================== MMA issuer (leader CTA)
+    if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t ph = 0, acc_ph = 0;
       bool dropped = false;
-      for (int64_t tile = blockIdx.x; tile < ntiles && !*s_abort; tile += gridDim.x) {
-        const TileInfo t = get_tile<MODE>(g, tile, s_seg, s_order);
+      for (int32_t tile = first; tile < ntiles && !*s_abort; tile += stride) {
+        const TileInfo t = get_tile<MODE, PAIR>(g, tile, s_seg, s_order, 0);
         if (t.k_iters == 0) continue;
         if (!ptx::mbar_wait(bar_acc_empty, acc_ph ^ 1u, 2)) {
           *s_abort = 1;
@@ -350,19 +414,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t t_sfa = tmem_base + kTmemSfa + buf * 4;
           const uint32_t t_sfb = tmem_base + kTmemSfb + buf * 8;
           const uint32_t sfa_s = sbase + kABytes + kBBytes;
-          ptx::tmem_cp_32x128b_warpx4(t_sfa, ptx::make_smem_desc(sfa_s, 0, 128, ptx::kLayoutSwizzleNone));
-          ptx::tmem_cp_32x128b_warpx4(t_sfb, ptx::make_smem_desc(sfa_s + kSfaBytes, 0, 128, ptx::kLayoutSwizzleNone));
-          ptx::tmem_cp_32x128b_warpx4(t_sfb + 4,
-                                      ptx::make_smem_desc(sfa_s + kSfaBytes + 512, 0, 128, ptx::kLayoutSwizzleNone));
+          const uint64_t dsa = ptx::make_smem_desc(sfa_s, 0, 128, ptx::kLayoutSwizzleNone);
+          const uint64_t dsb0 = ptx::make_smem_desc(sfa_s + kSfaBytes, 0, 128, ptx::kLayoutSwizzleNone);
+          const uint64_t dsb1 = ptx::make_smem_desc(sfa_s + kSfaBytes + 512, 0, 128, ptx::kLayoutSwizzleNone);
+          if (PAIR == 1) {
+            ptx::tmem_cp_32x128b_warpx4(t_sfa, dsa);
+            ptx::tmem_cp_32x128b_warpx4(t_sfb, dsb0);
+            ptx::tmem_cp_32x128b_warpx4(t_sfb + 4, dsb1);
+          } else {
+            ptx::tmem_cp_pair_32x128b_warpx4(t_sfa, dsa);
+            ptx::tmem_cp_pair_32x128b_warpx4(t_sfb, dsb0);
+            ptx::tmem_cp_pair_32x128b_warpx4(t_sfb + 4, dsb1);
+          }
           const uint64_t adesc = ptx::make_smem_desc(sbase, 16, 1024, ptx::kLayoutSwizzle128B);
           const uint64_t bdesc = ptx::make_smem_desc(sbase + kABytes, 16, 1024, ptx::kLayoutSwizzle128B);
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
-            const uint32_t idesc = ptx::make_idesc_mxf8(BM, BN, (uint32_t)kk, (uint32_t)kk);
-            ptx::mma_mxf8(tmem_base, adesc + (uint64_t)(2 * kk), bdesc + (uint64_t)(2 * kk), idesc, t_sfa, t_sfb,
-                          (kb | kk) != 0 ? 1u : 0u);
+            const uint32_t idesc = ptx::make_idesc_mxf8(C::TM, BN, (uint32_t)kk, (uint32_t)kk);
+            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            if (PAIR == 1)
+              ptx::mma_mxf8(tmem_base, adesc + (uint64_t)(2 * kk), bdesc + (uint64_t)(2 * kk), idesc, t_sfa, t_sfb,
+                            acc);
+            else
+              ptx::mma_mxf8_pair(tmem_base, adesc + (uint64_t)(2 * kk), bdesc + (uint64_t)(2 * kk), idesc, t_sfa,
+                                 t_sfb, acc);
           }
-          ptx::tc_commit(&bar_empty[stage]);
+          if (PAIR == 1) ptx::tc_commit(&bar_empty[stage]);
+          else ptx::tc_commit_pair(&bar_empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             ph ^= 1u;
@@ -374,25 +452,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (g.debug_drop_commit && !dropped && blockIdx.x == 0) {
           dropped = true;  // withhold the signal (timeout-path test)
-        } else {
+        } else if (PAIR == 1) {
           ptx::tc_commit(bar_acc_full);
+        } else {
+          ptx::tc_commit_pair(bar_acc_full);
         }
         acc_ph ^= 1u;
       }
     }
   } else {
-    // ===================================================== epilogue warps 2..9
+    // ===================================================== epilogue warps 2..9 (every CTA)
     const int ew = warp - 2;
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int h = ew >> 2;   // column half
-    float* stg = reinterpret_cast<float*>(smem + kOffStaging + ew * kStagingPerWarp);
+    float* stg = reinterpret_cast<float*>(smem + C::kOffStaging + ew * kStagingPerWarp);
     uint32_t acc_ph = 0;
     const uint32_t t_lane = tmem_base + ((uint32_t)(32 * q) << 16);
     const uint32_t t_stash = t_lane + kTmemStash + 64 * h;  // this warp's 64 spare TMEM columns
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const uint32_t acc_empty_leader = PAIR == 2 ? ptx::map_to_rank(ptx::smem_u32(bar_acc_empty), 0) : 0u;
+    for (int32_t tile = first; tile < ntiles; tile += stride) {
       // warp-uniform abort check (the TMEM loads below are warp-collective)
       if (__any_sync(0xffffffffu, *s_abort != 0)) break;
-      const TileInfo t = get_tile<MODE>(g, tile, s_seg, s_order);
+      const TileInfo t = get_tile<MODE, PAIR>(g, tile, s_seg, s_order, rank);
       const int64_t mrow0 = t.row0 + 32 * q;  // first row of this warp's 32-row block
       const int64_t row = mrow0 + lane;
       const bool have_acc = t.k_iters > 0;
@@ -414,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 4; ++c)
             ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&acc[32 * c]));
           ptx::tmem_wait_ld();
-          release_accumulator(bar_acc_empty, lane);
+          release_accumulator<PAIR>(bar_acc_empty, acc_empty_leader, lane);
         } else {
 #pragma unroll
           for (int i = 0; i < 128; ++i) acc[i] = 0u;
@@ -434,15 +515,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t F = g.F, F2 = 2 * g.F;
         const float p = g.prob_of_row[row];
         const int64_t f0 = (int64_t)t.n_tile * 128 + 64 * h;  // this warp's 64 Z columns
-        // phase 1 (the MMA warp waits for it): drain gate / up (TMEM columns [64h, +64) and
-        // [128 + 64h, +64)), keep them as packed bf16 for the backward's saved copy, form
-        // Z = silu(G) * U * p in fp32 and park Z in this warp's spare TMEM columns
+        // phase 1 (the MMA warp waits for it): drain gate / up (TMEM columns [128h, +64) and
+        // [128h + 64, +64), the interleaved operand order), keep them as packed bf16 for the
+        // backward's saved copy, form Z = silu(G) * U * p in fp32 and park Z in this warp's
+        // spare TMEM columns
         uint4 gsave[8], usave[8];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t gr[32], ur[32];
-          ptx::tmem_ld_32x32b_x32(t_lane + 64 * h + 32 * c, gr);
-          ptx::tmem_ld_32x32b_x32(t_lane + 128 + 64 * h + 32 * c, ur);
+          ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 32 * c, gr);
+          ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 64 + 32 * c, ur);
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -456,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tmem_st_32x32b_x16(t_stash + 32 * c + 16, *reinterpret_cast<uint32_t(*)[16]>(&gr[16]));
         }
         ptx::tmem_wait_st();
-        release_accumulator(bar_acc_empty, lane);
+        release_accumulator<PAIR>(bar_acc_empty, acc_empty_leader, lane);
         {
           uint4* gd = reinterpret_cast<uint4*>(g.gu + row * F2 + f0);
           uint4* ud = reinterpret_cast<uint4*>(g.gu + row * F2 + F + f0);
@@ -496,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tmem_st_32x32b_x16(t_stash + 16 * c, pk);
         }
         ptx::tmem_wait_st();
-        release_accumulator(bar_acc_empty, lane);
+        release_accumulator<PAIR>(bar_acc_empty, acc_empty_leader, lane);
         // phase 2: SwiGLU / probability backward, 32 columns at a time; G and U of the next
         // chunk are fetched while this one is processed
         const uint4* gsrc = reinterpret_cast<const uint4*>(g.gu_in + row * F2 + f0);
@@ -551,13 +633,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---- teardown: every role has finished issuing; the epilogue has drained the last
-  // accumulator, so every MMA has completed before TMEM is released.
+  // accumulator, so every MMA has completed before TMEM is released. With CTA pairs the
+  // cluster barrier also keeps each CTA (and the barriers its peer signals) alive until
+  // the peer is done.
   ptx::tc_fence_before();
   __syncthreads();
+  if (PAIR == 2) ptx::cluster_sync();
   if (warp == 1) {
     __syncwarp();
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, kTmemCols);
+    if (PAIR == 2) ptx::tmem_dealloc_pair(tmem_base, kTmemCols);
+    else ptx::tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -589,6 +675,20 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t col
   return r == CUDA_SUCCESS;
 }
 
+// [chunks, 512 B] view of an MMA-order scale array (one row per 128 x 128 block) as
+// 32-bit elements; box = one block's 512 scale bytes.
+static bool make_sf_map(CUtensorMap* m, const void* base, int64_t chunks) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {128, (cuuint64_t)chunks};
+  cuuint64_t strides[1] = {512};
+  cuuint32_t box[2] = {128, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int gemm_num_sms() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -596,39 +696,67 @@ int gemm_num_sms() {
   return n > 0 ? n : 148;
 }
 
-template <int MODE>
-static cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, int64_t tiles_ub,
-                               cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(mxgemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
+int gemm_tile_rows() {
+  // MXMOE_GEMM_PAIR=1 selects the single-CTA variant (128-row tiles); the default is
+  // CTA pairs (256-row tiles)
+  const char* v = std::getenv("MXMOE_GEMM_PAIR");
+  return (v && v[0] == '1' && v[1] == '\0') ? 128 : 256;
+}
+
+template <int MODE, int PAIR>
+static cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msa,
+                               const CUtensorMap& msb, const GemmArgs& g, int64_t tiles_ub, cudaStream_t st) {
+  constexpr uint32_t smem = Cfg<PAIR>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(mxgemm_kernel<MODE, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
   if (e != cudaSuccess) return e;
-  const int nsm = gemm_num_sms();
-  const int grid = (int)(tiles_ub < nsm ? (tiles_ub > 0 ? tiles_ub : 1) : nsm);
-  mxgemm_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(ma, mb, g);
+  const int units = gemm_num_sms() / PAIR;  // SMs, or SM pairs
+  const int n = (int)(tiles_ub < units ? (tiles_ub > 0 ? tiles_ub : 1) : units);
+  if (PAIR == 1) {
+    mxgemm_kernel<MODE, 1><<<n, kThreads, smem, st>>>(ma, mb, msa, msb, g);
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * n, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, mxgemm_kernel<MODE, PAIR>, ma, mb, msa, msb, g);
+    if (e != cudaSuccess) return e;
+  }
   ++g_launch_count;
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
-  CUtensorMap ma, mb;
-  if (!make_map(&ma, g.a_data, g.a_rows, g.a_cols) || !make_map(&mb, g.b_data, g.b_rows, g.b_cols))
+template <int PAIR>
+static cudaError_t launch_variant(const GemmArgs& g, cudaStream_t st) {
+  CUtensorMap ma, mb, msa, msb;
+  if (!make_map(&ma, g.a_data, g.a_rows, g.a_cols) || !make_map(&mb, g.b_data, g.b_rows, g.b_cols) ||
+      !make_sf_map(&msa, g.a_sf, (g.a_rows / 128) * (g.a_cols / 128)) ||
+      !make_sf_map(&msb, g.b_sf, (g.b_rows / 128) * (g.b_cols / 128)))
     return cudaErrorInvalidValue;
-  int64_t tiles_ub;
+  constexpr int TM = Cfg<PAIR>::TM;
   switch (g.mode) {
     case kModeStore:
-      tiles_ub = (g.a_rows / BM) * (g.N / BN);
-      return launch_mode<kModeStore>(ma, mb, g, tiles_ub, st);
+      return launch_mode<kModeStore, PAIR>(ma, mb, msa, msb, g, (g.a_rows / TM) * (g.N / BN), st);
     case kModeSwigluFwd:
-      tiles_ub = (g.a_rows / BM) * (g.F / 128);
-      return launch_mode<kModeSwigluFwd>(ma, mb, g, tiles_ub, st);
+      return launch_mode<kModeSwigluFwd, PAIR>(ma, mb, msa, msb, g, (g.a_rows / TM) * (g.F / 128), st);
     case kModeSwigluBwd:
-      tiles_ub = (g.a_rows / BM) * (g.F / BN);
-      return launch_mode<kModeSwigluBwd>(ma, mb, g, tiles_ub, st);
+      return launch_mode<kModeSwigluBwd, PAIR>(ma, mb, msa, msb, g, (g.a_rows / TM) * (g.F / BN), st);
     case kModeWgrad:
-      tiles_ub = (int64_t)g.E * (g.N / BM) * (g.K2 / BN);
-      return launch_mode<kModeWgrad>(ma, mb, g, tiles_ub, st);
+      return launch_mode<kModeWgrad, PAIR>(ma, mb, msa, msb, g, (int64_t)g.E * (g.N / TM) * (g.K2 / BN), st);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
+  return gemm_tile_rows() == 128 ? launch_variant<1>(g, st) : launch_variant<2>(g, st);
 }
 
 }  // namespace mxmoe

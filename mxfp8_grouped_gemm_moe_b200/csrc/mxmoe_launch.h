@@ -36,6 +36,9 @@ struct QuantArgs {
   uint8_t* col_data;  // nullable
   uint8_t* col_sf;
   int32_t col_layout;
+  // > 0: the rowwise copy of each [2*row_ilv, cols] batch matrix stores its rows in
+  // 64-row blocks interleaved [first half 0..63, second half 0..63, first 64..127, ...]
+  int64_t row_ilv;
 };
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
 

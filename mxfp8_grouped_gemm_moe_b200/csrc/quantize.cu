@@ -217,7 +217,12 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
       if (orow >= nvalid || col >= a.cols) continue;
       uint32_t q[8];
       const uint8_t sb = quant_row_block<T>(tile + tile_off<T>(row, 32 * blk), q);
-      const int64_t grow = b * a.out_rows + orow;
+      int64_t drow = orow;
+      if (a.row_ilv > 0) {  // gate / up interleave of the fc1 operand
+        const int64_t hf = orow >= a.row_ilv, rr = orow - hf * a.row_ilv;
+        drow = (rr >> 6) * 128 + hf * 64 + (rr & 63);
+      }
+      const int64_t grow = b * a.out_rows + drow;
       uint4* dst = reinterpret_cast<uint4*>(a.row_data + grow * a.cols + col);
       dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
       dst[1] = make_uint4(q[4], q[5], q[6], q[7]);

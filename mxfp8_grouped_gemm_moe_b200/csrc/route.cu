@@ -4,7 +4,7 @@
 //
 // "MoE-Training für biologische Grundmodelle optimieren" (hyper.ai/de), GroupedLinear
 // passage: the expert matrices are gathered from per-expert token counts. Order of rows
-// within an expert and the 128-row segment alignment are this library's reading.
+// within an expert and the 256-row segment alignment are this library's reading.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -18,6 +18,7 @@ namespace mxmoe {
 constexpr int kRouteTokensPerBlock = 256;
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 8;
+constexpr int kSegAlign = 256;  // expert segments start at multiples of the GEMM's 256-row tile
 
 // Pass 1: per-block expert histogram; validates ids (out of range or repeated within a
 // token -> device check error, pair dropped).
@@ -46,7 +47,7 @@ __global__ void __launch_bounds__(kRouteTokensPerBlock) route_count_kernel(const
   for (int e = threadIdx.x; e < E; e += blockDim.x) block_counts[(int64_t)blockIdx.x * E + e] = cnt[e];
 }
 
-// Pass 2 (one block): m_splits, 128-aligned segment offsets, per-(block, expert) base
+// Pass 2 (one block): m_splits, 256-aligned segment offsets, per-(block, expert) base
 // rows; marks pad rows (token -1, prob 0).
 __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restrict__ block_counts, int nblocks,
                                                           int E, int32_t* __restrict__ block_base,
@@ -66,7 +67,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
     int32_t o = 0;
     for (int e = 0; e < E; ++e) {
       s_off[e] = o;
-      o += (s_m[e] + 127) / 128 * 128;
+      o += (s_m[e] + kSegAlign - 1) / kSegAlign * kSegAlign;
     }
     s_off[E] = o;
   }

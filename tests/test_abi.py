@@ -52,8 +52,8 @@ def test_status_strings(lib):
 
 
 def test_sizes_are_host_only(lib):
-    assert lib.mxmoe_rows_capacity(8192, 2, 8) == (8192 * 2 + 127 * 8 + 127) // 128 * 128
-    assert lib.mxmoe_rows_capacity(0, 1, 1) == 128
+    assert lib.mxmoe_rows_capacity(8192, 2, 8) == (8192 * 2 + 255 * 8 + 255) // 256 * 256
+    assert lib.mxmoe_rows_capacity(0, 1, 1) == 256
     # weights: 4 copies of E*2F*H-ish bytes plus scales
     E, H, F = 8, 4096, 14336
     w = lib.mxmoe_weights_size(E, H, F)
@@ -90,10 +90,14 @@ def test_host_argument_errors_enqueue_nothing(lib):
     assert lib.mxfp8_quantize(fake, 0, 1, 64, 64, None, None, 64, None, None, S) == 1
     m_bad_layout = mx._MX(1 << 20, 1 << 20, 64, 64, 1, 0)   # MMA layout needs multiples of 128
     assert lib.mxfp8_quantize(fake, 0, 1, 64, 64, None, None, 64, ctypes.byref(m_bad_layout), None, S) == 2
-    # grouped GEMM: N not a multiple of 256; A not in MMA layout
+    # grouped GEMM: N not a multiple of 128; A not in MMA layout
     A = mx._MX(1 << 20, 1 << 20, 256, 256, 1, 0)
-    B = mx._MX(1 << 20, 1 << 20, 2 * 384, 256, 1, 0)
-    assert lib.grouped_gemm_mxfp8(ctypes.byref(A), ctypes.byref(B), fake, 2, 384, 256, fake, 0, 384, S) == 2
+    B = mx._MX(1 << 20, 1 << 20, 2 * 192, 256, 1, 0)
+    assert lib.grouped_gemm_mxfp8(ctypes.byref(A), ctypes.byref(B), fake, 2, 192, 256, fake, 0, 192, S) == 2
+    # weight-gradient GEMM: output rows must be a multiple of 256
+    At = mx._MX(1 << 20, 1 << 20, 128, 256, 1, 0)
+    Bt = mx._MX(1 << 20, 1 << 20, 128, 256, 1, 0)
+    assert lib.grouped_gemm_mxfp8_wgrad(ctypes.byref(At), ctypes.byref(Bt), fake, 2, fake, S) == 2
     Ap = mx._MX(1 << 20, 1 << 20, 256, 256, 0, 0)
     B2 = mx._MX(1 << 20, 1 << 20, 512, 256, 1, 0)
     assert lib.grouped_gemm_mxfp8(ctypes.byref(Ap), ctypes.byref(B2), fake, 2, 256, 256, fake, 0, 256, S) == 1

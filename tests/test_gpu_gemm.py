@@ -10,11 +10,18 @@ import torch
 import moe_workloads as wl
 from oracle import moe as omoe
 from oracle import mxfp8 as omx
-from tests.util import f64, rel_l2
+from tests.util import f64, rel_l2, SEG_ALIGN
 
 pytestmark = pytest.mark.gpu
 TOL_GEMM = 5e-3   # bf16 output: the spec bar per GEMM stage
 TOL_F32 = 5e-4    # fp32 output: fp32 accumulation over K <= 4096 terms stays well inside K * 2^-24
+
+
+@pytest.fixture(params=["pair", "single"])
+def variant(request, monkeypatch):
+    """Both kernel variants: CTA pairs (256-row tiles, default) and one CTA per tile."""
+    monkeypatch.setenv("MXMOE_GEMM_PAIR", "2" if request.param == "pair" else "1")
+    return request.param
 
 
 def _segments(counts):
@@ -34,16 +41,16 @@ def _dense_perm_input(gpu_lib, counts, K, seed):
     out = gpu_lib.moe_permute(idx.cuda(), probs.cuda(), E)
     x = wl.random_matrix(T, K, seed=seed)
     cap = gpu_lib.mxmoe_rows_capacity(T, 1, E)
-    r = omoe.route(idx.numpy(), E, align=128)
+    r = omoe.route(idx.numpy(), E, align=SEG_ALIGN)
     return x, out, cap, r, E
 
 
 @pytest.mark.parametrize("N,K", [(256, 128), (256, 512), (512, 384)])
-def test_single_tile_and_small(gpu_lib, N, K):
-    """One expert, one or a few 128 x 256 tiles: the tcgen05 path in isolation."""
-    A = wl.random_matrix(128, K, seed=11)
+def test_single_tile_and_small(gpu_lib, variant, N, K):
+    """One expert, one or two 256-column tiles: the tcgen05 path in isolation."""
+    A = wl.random_matrix(256, K, seed=11)
     B = wl.random_matrix(N, K, seed=12, std=0.05)
-    seg = torch.tensor([0, 128], dtype=torch.int32, device="cuda")
+    seg = torch.tensor([0, 256], dtype=torch.int32, device="cuda")
     ar, _ = gpu_lib.mxfp8_quantize(A.cuda(), colwise=False)
     br, _ = gpu_lib.mxfp8_quantize(B.cuda(), colwise=False)
     for dt in (torch.float32, torch.bfloat16):
@@ -59,7 +66,7 @@ def test_single_tile_and_small(gpu_lib, N, K):
     ([1000, 500, 31, 33], 512, 1024),
     ([127, 129, 40, 700, 0, 0, 1, 255], 768, 384),
 ])
-def test_grouped_gemm_ragged(gpu_lib, counts, N, K):
+def test_grouped_gemm_ragged(gpu_lib, variant, counts, N, K):
     x, out, cap, r, E = _dense_perm_input(gpu_lib, counts, K, seed=sum(counts))
     xr, _ = gpu_lib.mxfp8_quantize(x.cuda(), colwise=False, row_gather=out["token_of_row"],
                                    nrows=out["seg_off"][E:], out_rows=cap)
@@ -81,10 +88,10 @@ def test_grouped_gemm_ragged(gpu_lib, counts, N, K):
 
 
 @pytest.mark.parametrize("counts,N,K2", [
-    ([300, 0, 129, 1, 640], 128, 256),
-    ([1000, 500, 31, 33], 384, 512),
+    ([300, 0, 129, 1, 640], 256, 256),
+    ([1000, 500, 31, 33], 512, 768),
 ])
-def test_grouped_wgrad_ragged(gpu_lib, counts, N, K2):
+def test_grouped_wgrad_ragged(gpu_lib, variant, counts, N, K2):
     idx, E = _segments(counts)
     T = idx.shape[0]
     out = gpu_lib.moe_permute(idx.cuda(), torch.ones((T, 1)).cuda(), E)
@@ -98,7 +105,7 @@ def test_grouped_wgrad_ragged(gpu_lib, counts, N, K2):
     C = torch.full((E, N, K2), float("nan"), device="cuda")
     gpu_lib.grouped_gemm_mxfp8_wgrad(ac, bc, out["seg_off"], E, out=C)
     torch.cuda.synchronize()
-    r = omoe.route(idx.numpy(), E, align=128)
+    r = omoe.route(idx.numpy(), E, align=SEG_ALIGN)
     Ap = omoe.permute_rows(f64(a), r["token_of_row"])
     Bp = omoe.permute_rows(f64(b), r["token_of_row"])
     Aq = omoe.fake_quant_colwise_segments(Ap, r["seg_off"], r["m_splits"])
@@ -110,3 +117,23 @@ def test_grouped_wgrad_ragged(gpu_lib, counts, N, K2):
             assert np.all(got[e] == 0), e
         else:
             assert rel_l2(got[e], want[e]) <= TOL_F32, e
+
+
+@pytest.mark.parametrize("seg", [[0, 128, 256], [0, 512, 256], [0, 256, 4096]])
+def test_bad_segments_reported(gpu_lib, variant, seg):
+    """Segment offsets that are misaligned, decreasing or past the operand rows are
+    caught on the device: nothing is written and the device status says so."""
+    if variant == "single" and seg == [0, 128, 256]:
+        pytest.skip("128-row segments are valid for single-CTA tiles")
+    A = wl.random_matrix(512, 256, seed=31)
+    B = wl.random_matrix(2 * 256, 256, seed=32, std=0.05)
+    ar, _ = gpu_lib.mxfp8_quantize(A.cuda(), colwise=False)
+    br, _ = gpu_lib.mxfp8_quantize(B.cuda(), colwise=False)
+    gpu_lib.mxmoe_clear_device_status()
+    C = torch.full((512, 256), 7.0, device="cuda")
+    gpu_lib.grouped_gemm_mxfp8(ar, br, torch.tensor(seg, dtype=torch.int32, device="cuda"), 2, 256, out=C)
+    torch.cuda.synchronize()
+    st, _ = gpu_lib.mxmoe_get_device_status()
+    gpu_lib.mxmoe_clear_device_status()
+    assert st == 6  # MXMOE_ERR_DEVICE_CHECK
+    assert torch.all(C == 7.0)

@@ -9,7 +9,7 @@ import torch
 
 import moe_workloads as wl
 from oracle import moe as omoe
-from tests.util import f64, rel_l2
+from tests.util import f64, rel_l2, SEG_ALIGN
 
 pytestmark = pytest.mark.gpu
 TOL_E2E = 2e-2
@@ -43,7 +43,7 @@ def test_fused_mlp_matches_oracle(gpu_lib, name):
     torch.cuda.synchronize()
     yo, saved, go = _oracle(d)
     # saved routing maps: bit-exact with the oracle's (128-aligned segments)
-    r = omoe.route(d["topk_idx"].numpy(), cfg.E, align=128)
+    r = omoe.route(d["topk_idx"].numpy(), cfg.E, align=SEG_ALIGN)
     np.testing.assert_array_equal(layer.saved_field("m_splits", torch.int32, cfg.E).cpu().numpy(), r["m_splits"])
     np.testing.assert_array_equal(layer.saved_field("seg_off", torch.int32, cfg.E + 1).cpu().numpy(), r["seg_off"])
     errs = dict(y=rel_l2(f64(y), yo), dx=rel_l2(f64(dx), go["dx"]), dW1=rel_l2(f64(dW1), go["dW1"]),

@@ -9,7 +9,7 @@ import torch
 import moe_workloads as wl
 from oracle import moe as omoe
 from oracle import mxfp8 as omx
-from tests.util import f64, u8
+from tests.util import f64, u8, SEG_ALIGN
 
 pytestmark = pytest.mark.gpu
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "mxfp8_blocks.txt")
@@ -103,7 +103,7 @@ def test_permute_quantize_matches_oracle(gpu_lib, name):
     r, c = gpu_lib.mxfp8_quantize(x.cuda(), row_gather=out["token_of_row"], nrows=out["seg_off"][cfg.E:],
                                   out_rows=cap)
     torch.cuda.synchronize()
-    ro = omoe.route(idx.numpy(), cfg.E, align=128)
+    ro = omoe.route(idx.numpy(), cfg.E, align=SEG_ALIGN)
     Mp = ro["Mp"]
     Xp = omoe.permute_rows(f64(x), ro["token_of_row"])
     qr, sr = omx.quantize_rowwise(Xp)

@@ -5,7 +5,7 @@ import torch
 
 import moe_workloads as wl
 from oracle import moe as omoe
-from tests.util import f64
+from tests.util import f64, SEG_ALIGN
 
 pytestmark = pytest.mark.gpu
 
@@ -13,7 +13,7 @@ pytestmark = pytest.mark.gpu
 def _check_route(mx, idx, probs, E):
     out = mx.moe_permute(idx.cuda(), probs.cuda(), E)
     torch.cuda.synchronize()
-    r = omoe.route(idx.numpy(), E, align=128)
+    r = omoe.route(idx.numpy(), E, align=SEG_ALIGN)
     np.testing.assert_array_equal(out["m_splits"].cpu().numpy(), r["m_splits"])
     np.testing.assert_array_equal(out["seg_off"].cpu().numpy(), r["seg_off"])
     np.testing.assert_array_equal(out["row_of_slot"].cpu().numpy(), r["row_of_slot"])
@@ -92,7 +92,7 @@ def test_unpermute_matches_oracle(gpu_lib, k, H):
     yp = wl.random_matrix(cap, H, seed=3)
     y = gpu_lib.moe_unpermute(yp.cuda(), out["row_of_slot"])
     torch.cuda.synchronize()
-    r = omoe.route(idx.numpy(), E, align=128)
+    r = omoe.route(idx.numpy(), E, align=SEG_ALIGN)
     want = omoe.unpermute_sum(f64(yp), r["row_of_slot"])
     got = f64(y)
     # one rounding to bf16 of an fp32 sum: within one bf16 ulp of the exact sum

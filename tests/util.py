@@ -22,3 +22,7 @@ def u8(t):
 
 def to_cuda(d):
     return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+# Expert segments of the CUDA path start at multiples of 256 rows (its GEMM tile); the
+# oracle's results do not depend on the alignment (pinned in test_oracle_moe.py).
+SEG_ALIGN = 256
