@@ -54,26 +54,32 @@ constexpr int kEpiWarps = 8;
 constexpr uint32_t kABytes = 128 * BK;  // this CTA's 128 rows of A per stage
 constexpr uint32_t kSfaBytes = 512;     // 128 rows x 4 scale bytes
 constexpr uint32_t kSfbBytes = 1024;    // 256 rows x 4 scale bytes
-constexpr uint32_t kStagingPerWarp = 2048;  // colwise transpose staging
 constexpr int kMaxE = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemSfa = 256;    // two buffers of 4 columns
 constexpr uint32_t kTmemSfb = 264;    // two buffers of 8 columns
 constexpr uint32_t kTmemStash = 384;  // epilogue scratch: 64 columns per (lane quadrant, half)
 
-template <int PAIR>
+// Per-variant layout. The plain-store and weight-gradient modes write their output
+// through shared memory with TMA stores (two 4 KB boxes per epilogue warp); the fused
+// modes keep 4 KB per warp for the colwise-quantisation transpose. Ring depths beyond 4
+// stages measured no faster on long-K tiles.
+template <int PAIR, int MODE>
 struct Cfg {
+  static constexpr bool kTmaStore = MODE == kModeStore || MODE == kModeWgrad;
   static constexpr int TM = 128 * PAIR;                        // output tile rows
-  static constexpr int STAGES = PAIR == 2 ? 6 : 4;
+  static constexpr int STAGES = kTmaStore ? (PAIR == 2 ? 4 : 3) : (PAIR == 2 ? 5 : 3);
   static constexpr uint32_t kBBytes = (BN / PAIR) * BK;        // this CTA's B rows per stage
   static constexpr uint32_t kStageBytes = PAIR == 2 ? 34816 : 51200;
   static constexpr uint32_t kTxBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // per CTA
+  static constexpr uint32_t kStagingPerWarp = kTmaStore ? 8192 : 4096;
   static constexpr uint32_t kOffStaging = STAGES * kStageBytes;
   static constexpr uint32_t kOffBars = kOffStaging + kEpiWarps * kStagingPerWarp;
   static constexpr uint32_t kOffSeg = kOffBars + 256;
   static constexpr uint32_t kOffOrder = kOffSeg + (kMaxE + 1) * 4 + 12;
   static constexpr uint32_t kSmemBytes = kOffOrder + kMaxE * 4 + 1024;  // + slack for 1 KB alignment
   static constexpr int GROUP_M = 16 / PAIR;                    // M tiles per raster group (2048 rows)
+  static constexpr int GROUP_W = 16 / PAIR;                    // wgrad N tiles per raster group
   static_assert(kStageBytes >= kTxBytes && kStageBytes % 1024 == 0, "stage layout");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -92,28 +98,34 @@ __device__ __forceinline__ int32_t n_tiles_of(const GemmArgs& g) {
   if (MODE == kModeStore) return (int32_t)(g.N / BN);
   if (MODE == kModeSwigluFwd) return (int32_t)(g.F / 128);
   if (MODE == kModeSwigluBwd) return (int32_t)(g.F / BN);
-  return (int32_t)((g.N / Cfg<PAIR>::TM) * (g.K2 / BN));  // per expert, wgrad
+  return (int32_t)((g.N / Cfg<PAIR, MODE>::TM) * (g.K2 / BN));  // per expert, wgrad
 }
 
 template <int MODE, int PAIR>
 __device__ __forceinline__ int64_t total_tiles(const GemmArgs& g, const int32_t* s_seg) {
   if (MODE == kModeWgrad) return (int64_t)g.E * n_tiles_of<MODE, PAIR>(g);
-  return (int64_t)(s_seg[g.E] / Cfg<PAIR>::TM) * n_tiles_of<MODE, PAIR>(g);
+  return (int64_t)(s_seg[g.E] / Cfg<PAIR, MODE>::TM) * n_tiles_of<MODE, PAIR>(g);
 }
 
 // Tile `idx` of the launch as seen by CTA `rank` of its pair (rank 0 when PAIR == 1).
 template <int MODE, int PAIR>
 __device__ __forceinline__ TileInfo get_tile(const GemmArgs& g, int32_t idx, const int32_t* s_seg,
                                              const int32_t* s_order, uint32_t rank) {
-  constexpr int TM = Cfg<PAIR>::TM;
-  constexpr int GROUP_M = Cfg<PAIR>::GROUP_M;
+  constexpr int TM = Cfg<PAIR, MODE>::TM;
+  constexpr int GROUP_M = Cfg<PAIR, MODE>::GROUP_M;
   TileInfo t;
   if (MODE == kModeWgrad) {
+    // per expert, groups of GROUP_W row tiles; inside a group the row tile varies fastest,
+    // so the tiles in flight share a few A and B slices in L2
     const int32_t per = n_tiles_of<MODE, PAIR>(g);
     const int32_t nk2 = (int32_t)(g.K2 / BN);
+    const int32_t nn = (int32_t)(g.N / TM);
     const int32_t pos = idx / per, r = idx % per;
     const int32_t e = s_order[pos];
-    const int32_t n_t = r / nk2, k2_t = r % nk2;
+    constexpr int32_t GW = Cfg<PAIR, MODE>::GROUP_W;
+    const int32_t grp = r / (GW * nk2), rr = r % (GW * nk2);
+    const int32_t n0 = grp * GW, gn = min(GW, nn - n0);
+    const int32_t n_t = n0 + rr % gn, k2_t = rr / gn;
     t.e = e;
     t.k_iters = (s_seg[e + 1] - s_seg[e]) / BK;
     t.a_y = n_t * TM + 128 * (int32_t)rank;
@@ -173,62 +185,68 @@ __device__ __forceinline__ float tanh_approx(float x) {
 __device__ __forceinline__ float sigmoid_f(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
 __device__ __forceinline__ float silu_f(float x) { return x * sigmoid_f(x); }
 
+// Largest |v[i]| as an fp32 bit pattern (integer max of the magnitude bits; a pairwise
+// tree so the 32 comparisons are 5 dependent steps deep).
+__device__ __forceinline__ uint32_t amax_bits32(const float (&v)[32]) {
+  uint32_t m[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) m[i] = max(__float_as_uint(v[2 * i]) & 0x7FFFFFFFu, __float_as_uint(v[2 * i + 1]) & 0x7FFFFFFFu);
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) m[i] = max(m[i], m[i + w]);
+  return m[0];
+}
+
+// 32 fp32 -> 32 E4M3 codes (8 words) under the block's scale; returns the E8M0 byte.
+__device__ __forceinline__ uint8_t quant32(const float (&v)[32], uint32_t (&q)[8]) {
+  const int32_t X = mx_scale_exp_from_amax_bits(amax_bits32(v));
+  const float sc = mx_inv_scale(X);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t lo = e4m3x2(v[4 * i] * sc, v[4 * i + 1] * sc);
+    const uint32_t hi = e4m3x2(v[4 * i + 2] * sc, v[4 * i + 3] * sc);
+    q[i] = lo | (hi << 16);
+  }
+  return (uint8_t)(X + 127);
+}
+
 // Warp-wide colwise MXFP8 of a 32 x 32 fp32 block held one row per lane (lane = row,
-// v[i] = column i): blocks of 32 rows of one column, written transposed (column i ->
-// 32 consecutive bytes at dst + i*ld) with one scale byte per column.
-// The block is transposed through the warp's 2 KB staging buffer in two rounds of 16
-// columns. Staging layout (fp32 words): row r = 16*h + i (i < 16) lives in line i (32
-// words), half h; its four 16-byte chunks are XOR-swizzled by (i & 7), so both the
-// row-wise 16-byte stores and the column-wise 4-byte loads are bank-conflict free.
-// After the transpose, lane (c = lane % 16, h = lane / 16) holds rows [16h, 16h+16) of
-// column c; the two halves combine their amax with one shuffle.
+// v[i] = column i): each column's 32 values are one block, written transposed (column i
+// -> 32 consecutive bytes at dst + i*ld) with one scale byte per column. The block is
+// transposed through the warp's 4 KB staging buffer in one round: row r occupies words
+// [32r, 32r + 32) with its 16-byte chunk j stored at chunk j ^ (r % 8), so the row-wise
+// 16-byte writes and the column-wise 4-byte reads are both bank-conflict free; lane c
+// then holds column c whole.
 __device__ __forceinline__ void colwise_quant_store(const float (&v)[32], float* stg, int lane, uint8_t* dst,
                                                     int64_t ld, uint8_t* sf_base, int64_t sf_rows, int64_t sf_cols,
                                                     int64_t col_row0, int64_t kb) {
-  const int wi = lane & 15, wh = lane >> 4;  // this lane's row as (line, half) when writing
-  const int c = lane & 15, rh = lane >> 4;   // column and row half this lane reads
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<float4*>(stg + lane * 32 + ((j ^ (lane & 7)) << 2)) =
+        make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  __syncwarp();
+  float w[32];
 #pragma unroll
-    for (int qd = 0; qd < 4; ++qd) {
-      const int phys = ((wh << 2) | qd) ^ (wi & 7);
-      *reinterpret_cast<float4*>(stg + wi * 32 + phys * 4) =
-          make_float4(v[16 * r + 4 * qd], v[16 * r + 4 * qd + 1], v[16 * r + 4 * qd + 2], v[16 * r + 4 * qd + 3]);
-    }
-    __syncwarp();
-    float w[16];
-    uint32_t amax = 0;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int phys = ((rh << 2) | (c >> 2)) ^ (j & 7);
-      w[j] = stg[j * 32 + phys * 4 + (c & 3)];
-      amax = max(amax, __float_as_uint(fabsf(w[j])));
-    }
-    __syncwarp();
-    amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
-    const int32_t X = mx_scale_exp_from_amax_bits(amax);
-    const float sc = mx_inv_scale(X);
-    uint32_t q[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t lo = e4m3x2(w[4 * i] * sc, w[4 * i + 1] * sc);
-      const uint32_t hi = e4m3x2(w[4 * i + 2] * sc, w[4 * i + 3] * sc);
-      q[i] = lo | (hi << 16);
-    }
-    const int col = 16 * r + c;
-    *reinterpret_cast<uint4*>(dst + (int64_t)col * ld + 16 * rh) = make_uint4(q[0], q[1], q[2], q[3]);
-    if (rh == 0) sf_base[sf_offset(MXMOE_SCALE_MMA, sf_rows, sf_cols, col_row0 + col, kb)] = (uint8_t)(X + 127);
-  }
+  for (int r = 0; r < 32; ++r) w[r] = stg[r * 32 + ((((lane >> 2) ^ (r & 7)) << 2) | (lane & 3))];
+  __syncwarp();  // the buffer may be refilled once every lane has read its column
+  uint32_t q[8];
+  const uint8_t sb = quant32(w, q);
+  uint4* d = reinterpret_cast<uint4*>(dst + (int64_t)lane * ld);
+  d[0] = make_uint4(q[0], q[1], q[2], q[3]);
+  d[1] = make_uint4(q[4], q[5], q[6], q[7]);
+  sf_base[sf_offset(MXMOE_SCALE_MMA, sf_rows, sf_cols, col_row0 + lane, kb)] = sb;
 }
 
-__device__ __forceinline__ void rowwise_quant_store(const float (&v)[32], uint8_t* dst, uint8_t* sf, int64_t rows,
-                                                    int64_t cols, int64_t row, int64_t kb) {
+// Rowwise MXFP8 of the 32 values one thread holds: 32 codes to dst (32-byte aligned);
+// returns the scale byte (the caller stores the scales of several blocks together).
+__device__ __forceinline__ uint32_t rowwise_quant_codes(const float (&v)[32], uint8_t* dst) {
   uint32_t q[8];
-  const uint8_t sb = quant_block32(v, q);
+  const uint8_t sb = quant32(v, q);
   uint4* d = reinterpret_cast<uint4*>(dst);
   d[0] = make_uint4(q[0], q[1], q[2], q[3]);
   d[1] = make_uint4(q[4], q[5], q[6], q[7]);
-  sf[sf_offset(MXMOE_SCALE_MMA, rows, cols, row, kb)] = sb;
+  return sb;
 }
 
 // Hands the accumulator back to the MMA warp once this warp's TMEM reads (and writes
@@ -242,6 +260,32 @@ __device__ __forceinline__ void release_accumulator(uint64_t* bar_local, uint32_
     if (PAIR == 1) ptx::mbar_arrive(bar_local);
     else ptx::mbar_arrive_cluster(acc_empty_cluster);
   }
+}
+
+// Plain-store epilogue output path: each epilogue warp owns two 4 KB staging boxes of
+// 32 rows x 128 bytes in the TMA 128-byte-swizzle layout (16-byte chunk j of row r at
+// chunk j ^ (r % 8), which also makes the row-per-lane writes bank-conflict free). A box
+// is filled by the warp and written out by one TMA store; the two boxes alternate, so a
+// box is reused only after the store issued two boxes earlier has read it.
+__device__ __forceinline__ uint8_t* out_box_acquire(uint8_t* stg8, uint32_t n_out, int lane) {
+  if (n_out >= 2) {
+    if (lane == 0) ptx::bulk_wait_group_read<1>();
+    __syncwarp();
+  }
+  return stg8 + (n_out & 1u) * 4096;
+}
+__device__ __forceinline__ void out_box_put(uint8_t* box, int lane, int j, uint4 v) {
+  *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
+}
+__device__ __forceinline__ void out_box_issue(const CUtensorMap* map, uint8_t* box, int32_t x, int32_t y, int lane,
+                                              uint32_t& n_out, uint64_t policy) {
+  ptx::fence_proxy_async_shared();
+  __syncwarp();
+  if (lane == 0) {
+    ptx::tma_store_2d_hint(map, box, x, y, policy);
+    ptx::bulk_commit_group();
+  }
+  ++n_out;
 }
 
 // 8 fp32 (bit patterns) starting at v[i0] -> 8 bf16 in one 16-byte vector.
@@ -259,8 +303,8 @@ template <int MODE, int PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     mxgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
-                  const __grid_constant__ GemmArgs g) {
-  using C = Cfg<PAIR>;
+                  const __grid_constant__ CUtensorMap tmC, const __grid_constant__ GemmArgs g) {
+  using C = Cfg<PAIR, MODE>;
   constexpr int STAGES = C::STAGES;
   constexpr uint32_t kStageBytes = C::kStageBytes;
   constexpr uint32_t kBBytes = C::kBBytes;
@@ -299,6 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::prefetch_tensormap(&tmSFA);
       ptx::prefetch_tensormap(&tmSFB);
     }
+    if (C::kTmaStore) ptx::prefetch_tensormap(&tmC);
   }
   if (warp == 1) {
     if (PAIR == 2) {
@@ -465,7 +510,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ew = warp - 2;
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int h = ew >> 2;   // column half
-    float* stg = reinterpret_cast<float*>(smem + C::kOffStaging + ew * kStagingPerWarp);
+    float* stg = reinterpret_cast<float*>(smem + C::kOffStaging + ew * C::kStagingPerWarp);
+    uint32_t n_out = 0;  // output boxes this warp has handed to TMA (plain-store modes)
+    const uint64_t out_policy = ptx::make_policy_evict_first();
     uint32_t acc_ph = 0;
     const uint32_t t_lane = tmem_base + ((uint32_t)(32 * q) << 16);
     const uint32_t t_stash = t_lane + kTmemStash + 64 * h;  // this warp's 64 spare TMEM columns
@@ -477,6 +524,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t mrow0 = t.row0 + 32 * q;  // first row of this warp's 32-row block
       const int64_t row = mrow0 + lane;
       const bool have_acc = t.k_iters > 0;
+      if (MODE == kModeSwigluBwd) {
+        // pull this row's G and U slices (2 x 256 B) into L2 while the MMAs run
+        const uint16_t* gp = g.gu_in + row * (2 * g.F) + (int64_t)t.n_tile * BN + 128 * h;
+        ptx::prefetch_l2(gp);
+        ptx::prefetch_l2(gp + 64);
+        ptx::prefetch_l2(gp + g.F);
+        ptx::prefetch_l2(gp + g.F + 64);
+      }
       if (have_acc) {
         const bool ok = ptx::mbar_wait(bar_acc_full, acc_ph, 4);
         if (!__all_sync(0xffffffffu, ok)) {
@@ -500,16 +555,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 128; ++i) acc[i] = 0u;
         }
-        const int64_t col0 = (int64_t)t.n_tile * BN + 128 * h;
+        const int32_t col0 = t.n_tile * BN + 128 * h;
+        uint8_t* stg8 = reinterpret_cast<uint8_t*>(stg);
         if (MODE == kModeWgrad || g.c_dtype == MXMOE_DTYPE_F32) {
-          float* c = reinterpret_cast<float*>(g.c) + row * g.ldc + col0;
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            reinterpret_cast<uint4*>(c)[i] = make_uint4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+          for (int b = 0; b < 4; ++b) {
+            uint8_t* box = out_box_acquire(stg8, n_out, lane);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              out_box_put(box, lane, j,
+                          make_uint4(acc[32 * b + 4 * j], acc[32 * b + 4 * j + 1], acc[32 * b + 4 * j + 2],
+                                     acc[32 * b + 4 * j + 3]));
+            out_box_issue(&tmC, box, col0 + 32 * b, (int32_t)mrow0, lane, n_out, out_policy);
+          }
         } else {
-          uint16_t* c = reinterpret_cast<uint16_t*>(g.c) + row * g.ldc + col0;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) reinterpret_cast<uint4*>(c)[i] = pack8_bf16(acc, 8 * i);
+          for (int b = 0; b < 2; ++b) {
+            uint8_t* box = out_box_acquire(stg8, n_out, lane);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) out_box_put(box, lane, j, pack8_bf16(acc, 64 * b + 8 * j));
+            out_box_issue(&tmC, box, col0 + 64 * b, (int32_t)mrow0, lane, n_out, out_policy);
+          }
         }
       } else if (MODE == kModeSwigluFwd) {
         const int64_t F = g.F, F2 = 2 * g.F;
@@ -549,6 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // phase 2: MXFP8 of Z, rowwise (fc2 operand) and colwise (fc2 weight-gradient operand)
+        uint32_t zsf = 0;
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
           uint32_t zr[32];
@@ -558,10 +625,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) z[i] = __uint_as_float(zr[i]);
           const int64_t fc = f0 + 32 * c;
-          rowwise_quant_store(z, g.z_row + row * F + fc, g.z_row_sf, g.rows_cap, F, row, fc / 32);
+          zsf |= rowwise_quant_codes(z, g.z_row + row * F + fc) << (8 * c);
           colwise_quant_store(z, stg, lane, g.z_colT + fc * g.rows_cap + mrow0, g.rows_cap, g.z_colT_sf, F,
                               g.rows_cap, fc, mrow0 / 32);
         }
+        // row scales of the blocks [f0, f0 + 64): adjacent bytes (block index 2h, 2h + 1 mod 4)
+        *reinterpret_cast<uint16_t*>(g.z_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F, row, f0 / 32)) =
+            (uint16_t)zsf;
       } else if (MODE == kModeSwigluBwd) {
         const int64_t F = g.F, F2 = 2 * g.F;
         const float p = g.prob_of_row[row];
@@ -579,32 +649,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::tmem_wait_st();
         release_accumulator<PAIR>(bar_acc_empty, acc_empty_leader, lane);
-        // phase 2: SwiGLU / probability backward, 32 columns at a time; G and U of the next
-        // chunk are fetched while this one is processed
+        // phase 2: SwiGLU / probability backward, 32 columns at a time (G and U were pulled
+        // into L2 when the tile started)
         const uint4* gsrc = reinterpret_cast<const uint4*>(g.gu_in + row * F2 + f0);
         const uint4* usrc = reinterpret_cast<const uint4*>(g.gu_in + row * F2 + F + f0);
-        uint4 gq[4], uq[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          gq[i] = gsrc[i];
-          uq[i] = usrc[i];
-        }
         float dprob = 0.f;
+        uint32_t sfg = 0, sfu = 0;  // row scales of the four dG / dU blocks
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t dzw[16];
           ptx::tmem_ld_32x32b_x16(t_stash + 16 * c, dzw);
+          uint4 gq[4], uq[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            gq[i] = gsrc[4 * c + i];
+            uq[i] = usrc[4 * c + i];
+          }
           const uint32_t gw[16] = {gq[0].x, gq[0].y, gq[0].z, gq[0].w, gq[1].x, gq[1].y, gq[1].z, gq[1].w,
                                    gq[2].x, gq[2].y, gq[2].z, gq[2].w, gq[3].x, gq[3].y, gq[3].z, gq[3].w};
           const uint32_t uw[16] = {uq[0].x, uq[0].y, uq[0].z, uq[0].w, uq[1].x, uq[1].y, uq[1].z, uq[1].w,
                                    uq[2].x, uq[2].y, uq[2].z, uq[2].w, uq[3].x, uq[3].y, uq[3].z, uq[3].w};
-          if (c < 3) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              gq[i] = gsrc[4 * (c + 1) + i];
-              uq[i] = usrc[4 * (c + 1) + i];
-            }
-          }
           ptx::tmem_wait_ld();
           float vg[32], vu[32];
 #pragma unroll
@@ -620,16 +684,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             vu[i] = da * sl;
           }
           const int64_t fg = f0 + 32 * c;
-          rowwise_quant_store(vg, g.dgu_row + row * F2 + fg, g.dgu_row_sf, g.rows_cap, F2, row, fg / 32);
+          sfg |= rowwise_quant_codes(vg, g.dgu_row + row * F2 + fg) << (8 * c);
           colwise_quant_store(vg, stg, lane, g.dgu_colT + fg * g.rows_cap + mrow0, g.rows_cap, g.dgu_colT_sf, F2,
                               g.rows_cap, fg, mrow0 / 32);
-          rowwise_quant_store(vu, g.dgu_row + row * F2 + F + fg, g.dgu_row_sf, g.rows_cap, F2, row, (F + fg) / 32);
+          sfu |= rowwise_quant_codes(vu, g.dgu_row + row * F2 + F + fg) << (8 * c);
           colwise_quant_store(vu, stg, lane, g.dgu_colT + (F + fg) * g.rows_cap + mrow0, g.rows_cap,
                               g.dgu_colT_sf, F2, g.rows_cap, F + fg, mrow0 / 32);
         }
+        // row scales: blocks f0/32 .. +3 (and their up-half twins) are one aligned word each
+        *reinterpret_cast<uint32_t*>(g.dgu_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F2, row, f0 / 32)) = sfg;
+        *reinterpret_cast<uint32_t*>(g.dgu_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F2, row, (F + f0) / 32)) =
+            sfu;
         g.dprob_part[row * (F / 128) + t.n_tile * 2 + h] = dprob;
       }
     }
+    // output boxes fully written before the CTA retires
+    if (C::kTmaStore && lane == 0) ptx::bulk_wait_group<0>();
   }
 
   // ---- teardown: every role has finished issuing; the epilogue has drained the last
@@ -703,17 +773,35 @@ int gemm_tile_rows() {
   return (v && v[0] == '1' && v[1] == '\0') ? 128 : 256;
 }
 
+// Output map of the plain-store modes: [rows, cols] row-major with row pitch `ld`
+// elements, box 32 rows x 128 bytes, 128-byte swizzle (the staging layout).
+static bool make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_t ld, bool f32) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  const int64_t esz = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * esz)};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / esz), 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct GemmMaps {
+  CUtensorMap a, b, sfa, sfb, c;
+};
+
 template <int MODE, int PAIR>
-static cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msa,
-                               const CUtensorMap& msb, const GemmArgs& g, int64_t tiles_ub, cudaStream_t st) {
-  constexpr uint32_t smem = Cfg<PAIR>::kSmemBytes;
+static cudaError_t launch_mode(const GemmMaps& m, const GemmArgs& g, int64_t tiles_ub, cudaStream_t st) {
+  constexpr uint32_t smem = Cfg<PAIR, MODE>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(mxgemm_kernel<MODE, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   const int units = gemm_num_sms() / PAIR;  // SMs, or SM pairs
   const int n = (int)(tiles_ub < units ? (tiles_ub > 0 ? tiles_ub : 1) : units);
   if (PAIR == 1) {
-    mxgemm_kernel<MODE, 1><<<n, kThreads, smem, st>>>(ma, mb, msa, msb, g);
+    mxgemm_kernel<MODE, 1><<<n, kThreads, smem, st>>>(m.a, m.b, m.sfa, m.sfb, m.c, g);
   } else {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * n, 1, 1);
@@ -727,7 +815,7 @@ static cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb, con
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, mxgemm_kernel<MODE, PAIR>, ma, mb, msa, msb, g);
+    e = cudaLaunchKernelEx(&cfg, mxgemm_kernel<MODE, PAIR>, m.a, m.b, m.sfa, m.sfb, m.c, g);
     if (e != cudaSuccess) return e;
   }
   ++g_launch_count;
@@ -736,21 +824,24 @@ static cudaError_t launch_mode(const CUtensorMap& ma, const CUtensorMap& mb, con
 
 template <int PAIR>
 static cudaError_t launch_variant(const GemmArgs& g, cudaStream_t st) {
-  CUtensorMap ma, mb, msa, msb;
-  if (!make_map(&ma, g.a_data, g.a_rows, g.a_cols) || !make_map(&mb, g.b_data, g.b_rows, g.b_cols) ||
-      !make_sf_map(&msa, g.a_sf, (g.a_rows / 128) * (g.a_cols / 128)) ||
-      !make_sf_map(&msb, g.b_sf, (g.b_rows / 128) * (g.b_cols / 128)))
+  GemmMaps m;
+  std::memset(&m.c, 0, sizeof(m.c));
+  if (!make_map(&m.a, g.a_data, g.a_rows, g.a_cols) || !make_map(&m.b, g.b_data, g.b_rows, g.b_cols) ||
+      !make_sf_map(&m.sfa, g.a_sf, (g.a_rows / 128) * (g.a_cols / 128)) ||
+      !make_sf_map(&m.sfb, g.b_sf, (g.b_rows / 128) * (g.b_cols / 128)))
     return cudaErrorInvalidValue;
-  constexpr int TM = Cfg<PAIR>::TM;
+  constexpr int TM = 128 * PAIR;
   switch (g.mode) {
     case kModeStore:
-      return launch_mode<kModeStore, PAIR>(ma, mb, msa, msb, g, (g.a_rows / TM) * (g.N / BN), st);
+      if (!make_out_map(&m.c, g.c, g.a_rows, g.N, g.ldc, g.c_dtype == MXMOE_DTYPE_F32)) return cudaErrorInvalidValue;
+      return launch_mode<kModeStore, PAIR>(m, g, (g.a_rows / TM) * (g.N / BN), st);
     case kModeSwigluFwd:
-      return launch_mode<kModeSwigluFwd, PAIR>(ma, mb, msa, msb, g, (g.a_rows / TM) * (g.F / 128), st);
+      return launch_mode<kModeSwigluFwd, PAIR>(m, g, (g.a_rows / TM) * (g.F / 128), st);
     case kModeSwigluBwd:
-      return launch_mode<kModeSwigluBwd, PAIR>(ma, mb, msa, msb, g, (g.a_rows / TM) * (g.F / BN), st);
+      return launch_mode<kModeSwigluBwd, PAIR>(m, g, (g.a_rows / TM) * (g.F / BN), st);
     case kModeWgrad:
-      return launch_mode<kModeWgrad, PAIR>(ma, mb, msa, msb, g, (int64_t)g.E * (g.N / TM) * (g.K2 / BN), st);
+      if (!make_out_map(&m.c, g.c, (int64_t)g.E * g.N, g.K2, g.K2, true)) return cudaErrorInvalidValue;
+      return launch_mode<kModeWgrad, PAIR>(m, g, (int64_t)g.E * (g.N / TM) * (g.K2 / BN), st);
   }
   return cudaErrorInvalidValue;
 }
