@@ -37,9 +37,11 @@ SPEC_FP8_TFLOPS = 4500.0
 GEMM_FLOP_FACTOR = {"fc1_swiglu": 4, "fc2": 2, "fc2_dgrad_swiglu_bwd": 2, "fc2_wgrad": 2, "fc1_dgrad": 4,
                     "fc1_wgrad": 4}     # x M*H*F
 GEMM_KERNEL_SOURCES = ["mxfp8_grouped_gemm_moe_b200/csrc/gemm.cu", "mxfp8_grouped_gemm_moe_b200/csrc/ptx_sm100.cuh",
-                       "mxfp8_grouped_gemm_moe_b200/csrc/mxmoe_device.cuh"]
+                       "mxfp8_grouped_gemm_moe_b200/csrc/mxmoe_device.cuh",
+                       "mxfp8_grouped_gemm_moe_b200/csrc/tensor_map.h"]
 QUANT_KERNEL_SOURCES = ["mxfp8_grouped_gemm_moe_b200/csrc/quantize.cu",
-                        "mxfp8_grouped_gemm_moe_b200/csrc/mxmoe_device.cuh"]
+                        "mxfp8_grouped_gemm_moe_b200/csrc/mxmoe_device.cuh",
+                        "mxfp8_grouped_gemm_moe_b200/csrc/ptx_sm100.cuh"]
 
 
 def parse_args():
@@ -441,11 +443,13 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
                 "peak_source": f"{peak_kind} bf16 sustained x {FP8_OVER_BF16:g} (nominal MXFP8/bf16 ratio)",
                 "frac_of_spec_4500": stage_json[dom]["tflops"] / SPEC_FP8_TFLOPS,
                 "traffic": load_traffic(f"{dom}:{cfg.name}", GEMM_KERNEL_SOURCES, 1.0)}
-    q = stage_json.get("quant_x", {})
-    roofline_hbm = {"bound": "hbm", "kernel": "mxfp8_quantize_kernel (permute + quantise x)",
+    # the largest HBM-bound kernel of the step: the W1 quantiser (rowwise + colwise copies)
+    q = stage_json.get("quant_w1", {})
+    roofline_hbm = {"bound": "hbm", "kernel": "mxfp8_quantize_tma_kernel (W1 rowwise + colwise)",
                     "achieved": q.get("gbs"), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": (q.get("gbs") or 0) / peaks["hbm_gbs"], "peak_source": peak_kind,
-                    "traffic": load_traffic(f"quant_x:{cfg.name}", QUANT_KERNEL_SOURCES, 1.0)}
+                    "algorithmic_bytes": hbm_bytes["quant_w1"],
+                    "traffic": load_traffic(f"quant_w1:{cfg.name}", QUANT_KERNEL_SOURCES, 1.0)}
     gemm_ms = sum(stage_json[n]["ms"] for n in gemm_names)
     value = world * cfg.fwdbwd_flops / (ms * 1e-3) / 1e12
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,

@@ -26,7 +26,7 @@
 //  * K step 128; operand tiles use the 128-byte swizzle; the E8M0 scales arrive in the
 //    tensor cores' scale order and are moved to TMEM with tcgen05.cp;
 //  * warp 0 issues the copies, warp 1 issues tcgen05.mma (kind::mxf8f6f4, block32
-//    scales), warps 2..9 are the epilogue: they drain the accumulator from TMEM into
+//    scales), warps 4..11 are the epilogue: they drain the accumulator from TMEM into
 //    registers (or spare TMEM columns), hand it back to the MMA warp at once, then run
 //    the epilogue math and stores while the next tile's MMAs proceed;
 //  * every wait is bounded (1 s) and reports MXMOE_ERR_DEVICE_TIMEOUT instead of
@@ -43,13 +43,24 @@
 #include "mxmoe_device.cuh"
 #include "mxmoe_launch.h"
 #include "ptx_sm100.cuh"
+#include "tensor_map.h"
 
 namespace mxmoe {
 
 constexpr int BN = 256;  // output tile columns (both variants)
 constexpr int BK = 128;  // K per pipeline stage
-constexpr int kThreads = 320;  // 10 warps
+// Warp roles: warp 0 TMA producer, warp 1 MMA issuer, then 8 epilogue warps.
+//  * plain-store / weight-gradient modes: 10 warps, epilogue warps 2..9, 168 registers
+//    per thread (the ptxas limit once three warps share a scheduler);
+//  * fused SwiGLU modes: 12 warps = 3 warpgroups, epilogue warps 4..11 (warps 2-3 idle).
+//    The block launches with 168 registers per thread; warpgroup 0 then drops to
+//    kRegsCtl and the epilogue warpgroups rise to kRegsEpi, which together use exactly
+//    the launch allocation: 128 * kRegsCtl + 256 * kRegsEpi == 384 * kRegsLaunch.
 constexpr int kEpiWarps = 8;
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsCtl = 88;
+constexpr int kRegsEpi = 208;
+static_assert(128 * kRegsCtl + 256 * kRegsEpi == 384 * kRegsLaunch, "register split");
 
 constexpr uint32_t kABytes = 128 * BK;  // this CTA's 128 rows of A per stage
 constexpr uint32_t kSfaBytes = 512;     // 128 rows x 4 scale bytes
@@ -59,6 +70,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemSfa = 256;    // two buffers of 4 columns
 constexpr uint32_t kTmemSfb = 264;    // two buffers of 8 columns
 constexpr uint32_t kTmemStash = 384;  // epilogue scratch: 64 columns per (lane quadrant, half)
+constexpr int kPrefetchSteps = 8;     // K steps of the next tile pulled into L2 at a tile start
 
 // Per-variant layout. The plain-store and weight-gradient modes write their output
 // through shared memory with TMA stores (two 4 KB boxes per epilogue warp); the fused
@@ -67,6 +79,9 @@ constexpr uint32_t kTmemStash = 384;  // epilogue scratch: 64 columns per (lane 
 template <int PAIR, int MODE>
 struct Cfg {
   static constexpr bool kTmaStore = MODE == kModeStore || MODE == kModeWgrad;
+  static constexpr bool kSplitRegs = !kTmaStore;            // 12 warps with the register split
+  static constexpr int kThreads = kSplitRegs ? 384 : 320;
+  static constexpr int kEpiWarp0 = kSplitRegs ? 4 : 2;      // first epilogue warp
   static constexpr int TM = 128 * PAIR;                        // output tile rows
   static constexpr int STAGES = kTmaStore ? (PAIR == 2 ? 4 : 3) : (PAIR == 2 ? 5 : 3);
   static constexpr uint32_t kBBytes = (BN / PAIR) * BK;        // this CTA's B rows per stage
@@ -300,7 +315,7 @@ __device__ __forceinline__ uint4 pack8_bf16(const uint32_t (&v)[N], int i0) {
 }
 
 template <int MODE, int PAIR>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
     mxgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ GemmArgs g) {
@@ -388,7 +403,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *s_tmem;
   const int32_t ntiles = *s_bad ? 0 : (int32_t)total_tiles<MODE, PAIR>(g, s_seg);
 
-  if (warp == 0) {
+  if (warp < C::kEpiWarp0) {
+   if (C::kSplitRegs) ptx::setmaxnreg_dec<kRegsCtl>();
+   if (warp == 0) {
     // ===================================================== TMA producer (every CTA)
     if (lane == 0) {
       int stage = 0;
@@ -396,6 +413,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t a_kchunks = g.a_cols / 128, b_kchunks = g.b_cols / 128;
       for (int32_t tile = first; tile < ntiles && !*s_abort; tile += stride) {
         const TileInfo t = get_tile<MODE, PAIR>(g, tile, s_seg, s_order, rank);
+        if (tile + stride < ntiles) {
+          // warm L2 with the first K steps of this CTA's next tile (its operands usually
+          // come from HBM; the ring alone is too short to hide that at a tile change)
+          const TileInfo nt = get_tile<MODE, PAIR>(g, tile + stride, s_seg, s_order, rank);
+          const int npf = min(nt.k_iters, kPrefetchSteps);
+          for (int kb = 0; kb < npf; ++kb) {
+            ptx::tma_prefetch_2d(&tmA, nt.a_x0 + kb * BK, nt.a_y);
+            ptx::tma_prefetch_2d(&tmB, nt.b_x0 + kb * BK, PAIR == 2 && rank ? nt.b_y1 : nt.b_y0);
+            if (PAIR == 1) ptx::tma_prefetch_2d(&tmB, nt.b_x0 + kb * BK, nt.b_y1);
+          }
+        }
         for (int kb = 0; kb < t.k_iters; ++kb) {
           if (!ptx::mbar_wait(&bar_empty[stage], ph ^ 1u, 1)) {
             *s_abort = 1;
@@ -433,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
+   } else if (warp == 1) {
     // ===================================================== MMA issuer (leader CTA)
     if (lane == 0 && rank == 0) {
       int stage = 0;
@@ -505,9 +533,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc_ph ^= 1u;
       }
     }
+   }
   } else {
-    // ===================================================== epilogue warps 2..9 (every CTA)
-    const int ew = warp - 2;
+    if (C::kSplitRegs) ptx::setmaxnreg_inc<kRegsEpi>();
+    // ===================================================== epilogue warps (every CTA)
+    const int ew = warp - C::kEpiWarp0;
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int h = ew >> 2;   // column half
     float* stg = reinterpret_cast<float*>(smem + C::kOffStaging + ew * C::kStagingPerWarp);
@@ -581,49 +611,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t F = g.F, F2 = 2 * g.F;
         const float p = g.prob_of_row[row];
         const int64_t f0 = (int64_t)t.n_tile * 128 + 64 * h;  // this warp's 64 Z columns
-        // phase 1 (the MMA warp waits for it): drain gate / up (TMEM columns [128h, +64) and
-        // [128h + 64, +64), the interleaved operand order), keep them as packed bf16 for the
-        // backward's saved copy, form Z = silu(G) * U * p in fp32 and park Z in this warp's
-        // spare TMEM columns
-        uint4 gsave[8], usave[8];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t gr[32], ur[32];
-          ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 32 * c, gr);
-          ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 64 + 32 * c, ur);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            gsave[4 * c + i] = pack8_bf16(gr, 8 * i);
-            usave[4 * c + i] = pack8_bf16(ur, 8 * i);
-          }
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            gr[i] = __float_as_uint(silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]) * p);
-          ptx::tmem_st_32x32b_x16(t_stash + 32 * c, *reinterpret_cast<uint32_t(*)[16]>(&gr[0]));
-          ptx::tmem_st_32x32b_x16(t_stash + 32 * c + 16, *reinterpret_cast<uint32_t(*)[16]>(&gr[16]));
-        }
-        ptx::tmem_wait_st();
+        // drain gate / up (TMEM columns [128h, +64) and [128h + 64, +64), the interleaved
+        // operand order) into registers and hand the accumulator back at once; then save G
+        // and U as bf16 for the backward and form Z = silu(G) * U * p in fp32
+        uint32_t gr[64], ur[64];
+        ptx::tmem_ld_32x32b_x32(t_lane + 128 * h, *reinterpret_cast<uint32_t(*)[32]>(&gr[0]));
+        ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&gr[32]));
+        ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 64, *reinterpret_cast<uint32_t(*)[32]>(&ur[0]));
+        ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 96, *reinterpret_cast<uint32_t(*)[32]>(&ur[32]));
+        ptx::tmem_wait_ld();
         release_accumulator<PAIR>(bar_acc_empty, acc_empty_leader, lane);
         {
           uint4* gd = reinterpret_cast<uint4*>(g.gu + row * F2 + f0);
           uint4* ud = reinterpret_cast<uint4*>(g.gu + row * F2 + F + f0);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            gd[i] = gsave[i];
-            ud[i] = usave[i];
+            gd[i] = pack8_bf16(gr, 8 * i);
+            ud[i] = pack8_bf16(ur, 8 * i);
           }
         }
+        float zf[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) zf[i] = silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]) * p;
         // phase 2: MXFP8 of Z, rowwise (fc2 operand) and colwise (fc2 weight-gradient operand)
         uint32_t zsf = 0;
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          uint32_t zr[32];
-          ptx::tmem_ld_32x32b_x32(t_stash + 32 * c, zr);
-          ptx::tmem_wait_ld();
-          float z[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) z[i] = __uint_as_float(zr[i]);
+        for (int c = 0; c < 2; ++c) {
+          const float(&z)[32] = *reinterpret_cast<const float(*)[32]>(&zf[32 * c]);
           const int64_t fc = f0 + 32 * c;
           zsf |= rowwise_quant_codes(z, g.z_row + row * F + fc) << (8 * c);
           colwise_quant_store(z, stg, lane, g.z_colT + fc * g.rows_cap + mrow0, g.rows_cap, g.z_colT_sf, F,
@@ -636,39 +650,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t F = g.F, F2 = 2 * g.F;
         const float p = g.prob_of_row[row];
         const int64_t f0 = (int64_t)t.n_tile * BN + 128 * h;  // this warp's 128 dZ columns
-        // phase 1: drain dZ, park it in TMEM as packed bf16 pairs (the E4M3 rounding that
+        // phase 1: drain dZ into registers and hand the accumulator back at once, then park
+        // dZ in this warp's spare TMEM columns as packed bf16 pairs (the E4M3 rounding that
         // follows is 2^5 coarser than that rounding)
+        {
+          uint32_t dzr[128];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t tmp[32], pk[16];
-          ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 32 * c, tmp);
+          for (int c = 0; c < 4; ++c)
+            ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&dzr[32 * c]));
           ptx::tmem_wait_ld();
+          release_accumulator<PAIR>(bar_acc_empty, acc_empty_leader, lane);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(tmp[2 * i]), __uint_as_float(tmp[2 * i + 1]));
-          ptx::tmem_st_32x32b_x16(t_stash + 16 * c, pk);
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(__uint_as_float(dzr[32 * c + 2 * i]), __uint_as_float(dzr[32 * c + 2 * i + 1]));
+            ptx::tmem_st_32x32b_x16(t_stash + 16 * c, pk);
+          }
+          ptx::tmem_wait_st();
         }
-        ptx::tmem_wait_st();
-        release_accumulator<PAIR>(bar_acc_empty, acc_empty_leader, lane);
-        // phase 2: SwiGLU / probability backward, 32 columns at a time (G and U were pulled
-        // into L2 when the tile started)
+        // phase 2: SwiGLU / probability backward, 32 columns at a time; G and U (pulled into
+        // L2 when the tile started) of the next chunk are fetched while this one is processed
         const uint4* gsrc = reinterpret_cast<const uint4*>(g.gu_in + row * F2 + f0);
         const uint4* usrc = reinterpret_cast<const uint4*>(g.gu_in + row * F2 + F + f0);
+        uint4 gq[4], uq[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          gq[i] = gsrc[i];
+          uq[i] = usrc[i];
+        }
         float dprob = 0.f;
         uint32_t sfg = 0, sfu = 0;  // row scales of the four dG / dU blocks
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t dzw[16];
           ptx::tmem_ld_32x32b_x16(t_stash + 16 * c, dzw);
-          uint4 gq[4], uq[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            gq[i] = gsrc[4 * c + i];
-            uq[i] = usrc[4 * c + i];
-          }
           const uint32_t gw[16] = {gq[0].x, gq[0].y, gq[0].z, gq[0].w, gq[1].x, gq[1].y, gq[1].z, gq[1].w,
                                    gq[2].x, gq[2].y, gq[2].z, gq[2].w, gq[3].x, gq[3].y, gq[3].z, gq[3].w};
           const uint32_t uw[16] = {uq[0].x, uq[0].y, uq[0].z, uq[0].w, uq[1].x, uq[1].y, uq[1].z, uq[1].w,
                                    uq[2].x, uq[2].y, uq[2].z, uq[2].w, uq[3].x, uq[3].y, uq[3].z, uq[3].w};
+          if (c < 3) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              gq[i] = gsrc[4 * (c + 1) + i];
+              uq[i] = usrc[4 * (c + 1) + i];
+            }
+          }
           ptx::tmem_wait_ld();
           float vg[32], vu[32];
 #pragma unroll
@@ -718,19 +746,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ----------------------------------------------------------------------------- host side
-static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 // 2-D uint8 tensor map over a row-major [rows, cols] matrix, box 128 x 128, 128-byte swizzle.
 static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
   auto fn = get_encode_fn();
@@ -798,14 +813,19 @@ static cudaError_t launch_mode(const GemmMaps& m, const GemmArgs& g, int64_t til
   cudaError_t e = cudaFuncSetAttribute(mxgemm_kernel<MODE, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
+  // the warpgroup register split assumes the launch allocation it was sized for
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, mxgemm_kernel<MODE, PAIR>);
+  if (e != cudaSuccess) return e;
+  if (Cfg<PAIR, MODE>::kSplitRegs && fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
   const int units = gemm_num_sms() / PAIR;  // SMs, or SM pairs
   const int n = (int)(tiles_ub < units ? (tiles_ub > 0 ? tiles_ub : 1) : units);
   if (PAIR == 1) {
-    mxgemm_kernel<MODE, 1><<<n, kThreads, smem, st>>>(m.a, m.b, m.sfa, m.sfb, m.c, g);
+    mxgemm_kernel<MODE, 1><<<n, Cfg<PAIR, MODE>::kThreads, smem, st>>>(m.a, m.b, m.sfa, m.sfb, m.c, g);
   } else {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * n, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(Cfg<PAIR, MODE>::kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];

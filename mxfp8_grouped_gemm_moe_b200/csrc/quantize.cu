@@ -18,6 +18,8 @@
 
 #include "mxmoe_device.cuh"
 #include "mxmoe_launch.h"
+#include "ptx_sm100.cuh"
+#include "tensor_map.h"
 
 namespace mxmoe {
 
@@ -252,6 +254,204 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
   }
 }
 
+// ----------------------------------------------------------------------------- dense bf16 path
+// Persistent variant for dense (ungathered) bf16 matrices whose rows and columns are
+// multiples of 128 -- the expert weights. Each CTA walks a strided list of 128 x 128
+// tiles. Tiles arrive by TMA into a 2-stage ring (the next tile is read while this one is
+// quantised); a stage holds the tile as two 64-column halves of [128 rows][128 bytes] in
+// the TMA 128-byte swizzle (16-byte chunk j of row r at chunk j ^ (r % 8)). The E4M3
+// codes of both copies are assembled in shared memory in the same swizzled layout and
+// leave by TMA stores of whole 128-byte lines; only the scale bytes are stored directly.
+constexpr int kQtStages = 2;
+constexpr uint32_t kQtStageBytes = 2 * 128 * 128;   // 32 KB of bf16
+constexpr uint32_t kQtOutBytes = 128 * 128;         // 16 KB of codes per copy
+constexpr uint32_t kQtOffOut = kQtStages * kQtStageBytes;
+constexpr uint32_t kQtOffBar = kQtOffOut + 2 * kQtOutBytes;
+constexpr uint32_t kQtSmem = kQtOffBar + 64 + 1024;
+
+// Byte offset of (row, 16-byte chunk j) in a [rows][128 bytes] 128-byte-swizzled region.
+__device__ __forceinline__ uint32_t sw128(int row, int j) {
+  return (uint32_t)row * 128u + ((uint32_t)(j ^ (row & 7)) << 4);
+}
+// Byte offset of (row, col) of a bf16 tile inside its stage.
+__device__ __forceinline__ uint32_t qt_off(int row, int col) {
+  const uint32_t half = (uint32_t)col >> 6, byte = ((uint32_t)col & 63) * 2;
+  return half * 16384u + sw128(row, (int)(byte >> 4)) + (byte & 15);
+}
+
+__global__ void __launch_bounds__(kQThreads, 2)
+    mxfp8_quantize_tma_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tm_row,
+                              const __grid_constant__ CUtensorMap tm_col, const __grid_constant__ QuantArgs a,
+                              int32_t tiles_c, int32_t tiles_per_batch, int32_t ntiles) {
+  extern __shared__ uint8_t qt_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qt_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* out_row = smem + kQtOffOut;
+  uint8_t* out_col = out_row + kQtOutBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQtOffBar);
+  volatile int32_t* s_abort = reinterpret_cast<volatile int32_t*>(full + kQtStages);
+
+  const int32_t first = (int32_t)blockIdx.x, stride = (int32_t)gridDim.x;
+  const int32_t mine = first < ntiles ? (ntiles - 1 - first) / stride + 1 : 0;
+  auto tile_of = [&](int32_t i, int64_t& b, int64_t& r0, int64_t& c0) {
+    const int32_t t = first + i * stride;
+    b = t / tiles_per_batch;
+    const int32_t rem = t % tiles_per_batch;
+    r0 = (int64_t)(rem / tiles_c) * kQTile;
+    c0 = (int64_t)(rem % tiles_c) * kQTile;
+  };
+  auto issue = [&](int32_t i) {  // thread 0: TMA loads of my i-th tile into stage i % S
+    int64_t b, r0, c0;
+    tile_of(i, b, r0, c0);
+    uint8_t* st = smem + (i % kQtStages) * kQtStageBytes;
+    uint64_t* bar = &full[i % kQtStages];
+    ptx::mbar_arrive_expect_tx(bar, kQtStageBytes);
+    const int32_t y = (int32_t)(b * a.rows + r0);
+    ptx::tma_load_2d(st, &tm, (int32_t)c0, y, bar);
+    ptx::tma_load_2d(st + 16384, &tm, (int32_t)c0 + 64, y, bar);
+  };
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQtStages; ++s) ptx::mbar_init(&full[s], 1);
+    *s_abort = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tensormap(&tm);
+    ptx::prefetch_tensormap(&tm_row);
+    ptx::prefetch_tensormap(&tm_col);
+    for (int32_t i = 0; i < kQtStages && i < mine; ++i) issue(i);
+  }
+  __syncthreads();
+
+  for (int32_t i = 0; i < mine; ++i) {
+    const bool ok = ptx::mbar_wait(&full[i % kQtStages], (uint32_t)(i / kQtStages) & 1u, 30);
+    if (!ok) *s_abort = 1;
+    // the previous tile's output stores have read the staging buffers
+    if (threadIdx.x == 0) ptx::bulk_wait_group_read<0>();
+    __syncthreads();
+    if (*s_abort) break;
+    const uint8_t* st = smem + (i % kQtStages) * kQtStageBytes;
+    int64_t b, r0, c0;
+    tile_of(i, b, r0, c0);
+
+    // rowwise: 512 items (row, 32-column block), 2 per thread; a warp takes 8 rows and
+    // lanes l, l + 8, l + 16, l + 24 share a row, so each 8-lane phase of a 16-byte shared
+    // access touches 8 distinct chunk positions (conflict free)
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int it = threadIdx.x + k * kQThreads;
+      const int l = it & 31;
+      const int row = 8 * (it >> 5) + (l & 7), blk = l >> 3;
+      uint32_t w[16];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const uint4 v = *reinterpret_cast<const uint4*>(st + qt_off(row, 32 * blk + 8 * t));
+        w[4 * t] = v.x; w[4 * t + 1] = v.y; w[4 * t + 2] = v.z; w[4 * t + 3] = v.w;
+      }
+      uint32_t q[8];
+      const uint8_t sb = quant_block32_bf16(w, q);
+      *reinterpret_cast<uint4*>(out_row + sw128(row, 2 * blk)) = make_uint4(q[0], q[1], q[2], q[3]);
+      *reinterpret_cast<uint4*>(out_row + sw128(row, 2 * blk + 1)) = make_uint4(q[4], q[5], q[6], q[7]);
+      const int64_t orow = r0 + row;
+      int64_t drow = orow;
+      if (a.row_ilv > 0) {  // gate / up interleave of the fc1 operand
+        const int64_t hf = orow >= a.row_ilv, rr = orow - hf * a.row_ilv;
+        drow = (rr >> 6) * 128 + hf * 64 + (rr & 63);
+      }
+      a.row_sf[sf_offset(a.row_layout, a.batch * a.out_rows, a.cols, b * a.out_rows + drow, (c0 >> 5) + blk)] = sb;
+    }
+    // colwise: item = (pair of adjacent columns, 32-row block), one per thread; a warp
+    // reads 32 consecutive column pairs (one 128-byte half-row) per load, conflict free.
+    // Codes go to rows 2p, 2p + 1 of the transposed [128 columns][128 rows] output tile.
+    {
+      const int pcol = threadIdx.x & 63, rb = threadIdx.x >> 6;
+      uint32_t w[32];
+#pragma unroll
+      for (int r = 0; r < 32; ++r) w[r] = *reinterpret_cast<const uint32_t*>(st + qt_off(32 * rb + r, 2 * pcol));
+      uint32_t q0[8], q1[8];
+      uint8_t s0, s1;
+      quant_colpair_bf16(w, q0, q1, s0, s1);
+      *reinterpret_cast<uint4*>(out_col + sw128(2 * pcol, 2 * rb)) = make_uint4(q0[0], q0[1], q0[2], q0[3]);
+      *reinterpret_cast<uint4*>(out_col + sw128(2 * pcol, 2 * rb + 1)) = make_uint4(q0[4], q0[5], q0[6], q0[7]);
+      *reinterpret_cast<uint4*>(out_col + sw128(2 * pcol + 1, 2 * rb)) = make_uint4(q1[0], q1[1], q1[2], q1[3]);
+      *reinterpret_cast<uint4*>(out_col + sw128(2 * pcol + 1, 2 * rb + 1)) = make_uint4(q1[4], q1[5], q1[6], q1[7]);
+      const int64_t grow = b * a.cols + c0 + 2 * pcol;  // row of the transposed matrix
+      const int64_t kb = (r0 >> 5) + rb;
+      a.col_sf[sf_offset(a.col_layout, a.batch * a.cols, a.out_rows, grow, kb)] = s0;
+      a.col_sf[sf_offset(a.col_layout, a.batch * a.cols, a.out_rows, grow + 1, kb)] = s1;
+    }
+    ptx::fence_proxy_async_shared();  // this thread's staging writes before the TMA stores
+    __syncthreads();                  // stage i fully read, staging fully written
+    if (threadIdx.x == 0) {
+      // rowwise copy: two 64-row boxes (the fc1 interleave moves 64-row blocks)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        int64_t drow = r0 + 64 * hh;
+        if (a.row_ilv > 0) {
+          const int64_t hf = drow >= a.row_ilv, rr = drow - hf * a.row_ilv;
+          drow = (rr >> 6) * 128 + hf * 64;
+        }
+        ptx::tma_store_2d(&tm_row, out_row + hh * 8192, (int32_t)c0, (int32_t)(b * a.out_rows + drow));
+      }
+      // colwise copy: the transposed tile, [128 columns][128 rows]
+      ptx::tma_store_2d(&tm_col, out_col, (int32_t)r0, (int32_t)(b * a.cols + c0));
+      ptx::bulk_commit_group();
+      if (i + kQtStages < mine) issue(i + kQtStages);
+    }
+  }
+  if (threadIdx.x == 0) ptx::bulk_wait_group<0>();
+}
+
+static bool qt_applies(const QuantArgs& a) {
+  return a.src_dtype == MXMOE_DTYPE_BF16 && !a.gather && !a.nrows && a.out_rows == a.rows && a.rows % kQTile == 0 &&
+         a.cols % kQTile == 0 && a.batch * a.rows < (int64_t)1 << 31 && a.batch * a.cols < (int64_t)1 << 31 &&
+         a.row_data && a.col_data && (reinterpret_cast<uintptr_t>(a.row_data) & 15) == 0 &&
+         (reinterpret_cast<uintptr_t>(a.col_data) & 15) == 0;
+}
+
+// 2-D uint8 map over [rows, 128 * k] codes for the TMA stores: box `box_rows` x 128 bytes,
+// 128-byte swizzle (the staging layout).
+static bool make_code_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols, uint32_t box_rows) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static cudaError_t launch_qt(const QuantArgs& a, cudaStream_t st) {
+  auto fn = get_encode_fn();
+  if (!fn) return cudaErrorInvalidValue;
+  CUtensorMap tm, tm_row, tm_col;
+  cuuint64_t dims[2] = {(cuuint64_t)a.cols, (cuuint64_t)(a.batch * a.rows)};
+  cuuint64_t strides[1] = {(cuuint64_t)(a.cols * 2)};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.src), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  if (!make_code_map(&tm_row, a.row_data, a.batch * a.out_rows, a.cols, 64) ||
+      !make_code_map(&tm_col, a.col_data, a.batch * a.cols, a.out_rows, 128))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(mxfp8_quantize_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kQtSmem);
+  if (e != cudaSuccess) return e;
+  const int32_t tiles_c = (int32_t)(a.cols / kQTile);
+  const int32_t tiles_per_batch = (int32_t)(a.rows / kQTile) * tiles_c;
+  const int32_t ntiles = tiles_per_batch * (int32_t)a.batch;
+  if (ntiles == 0) return cudaSuccess;
+  int dev = 0, nsm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = std::min<int64_t>(ntiles, (int64_t)(nsm > 0 ? nsm : 148) * 2);
+  mxfp8_quantize_tma_kernel<<<grid, kQThreads, kQtSmem, st>>>(tm, tm_row, tm_col, a, tiles_c, tiles_per_batch,
+                                                               ntiles);
+  ++g_launch_count;
+  return cudaGetLastError();
+}
+
 template <typename T>
 static cudaError_t launch_q(const QuantArgs& a, cudaStream_t st) {
   using Tr = SrcTraits<T>;
@@ -268,6 +468,7 @@ static cudaError_t launch_q(const QuantArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st) {
+  if (qt_applies(a)) return launch_qt(a, st);
   if (a.src_dtype == MXMOE_DTYPE_BF16) return launch_q<__nv_bfloat16>(a, st);
   return launch_q<float>(a, st);
 }

@@ -75,6 +75,22 @@ def test_quantize_matches_oracle(gpu_lib, dtype, layout, shape):
     np.testing.assert_array_equal(u8(c.scale_plain()), sc)
 
 
+@pytest.mark.parametrize("shape", [(96, 160), (224, 32)])
+def test_quantize_untiled_shapes(gpu_lib, shape):
+    """bf16 shapes that are not multiples of 128 take the per-tile kernel (the dense
+    persistent kernel needs whole 128 x 128 tiles); same bytes as the oracle."""
+    R, C = shape
+    x = wl.random_matrix(R, C, seed=R * C, dtype=torch.float32).to(torch.bfloat16)
+    r, c = gpu_lib.mxfp8_quantize(x.cuda(), layout=gpu_lib.SCALE_PLAIN)
+    torch.cuda.synchronize()
+    qr, sr = omx.quantize_rowwise(f64(x))
+    qc, sc = omx.quantize_colwise_t(f64(x))
+    np.testing.assert_array_equal(u8(r.data), qr)
+    np.testing.assert_array_equal(u8(r.scale_plain()), sr)
+    np.testing.assert_array_equal(u8(c.data), qc)
+    np.testing.assert_array_equal(u8(c.scale_plain()), sc)
+
+
 def test_quantize_batched_weights(gpu_lib):
     E, N, K = 3, 256, 384
     W = wl.random_matrix(N, K, seed=9, std=0.02, batch=E)
@@ -112,3 +128,32 @@ def test_permute_quantize_matches_oracle(gpu_lib, name):
     np.testing.assert_array_equal(u8(r.scale_plain())[:Mp], sr)
     np.testing.assert_array_equal(u8(c.data)[:, :Mp], qc)
     np.testing.assert_array_equal(u8(c.scale_plain())[:, :Mp // 32], sc)
+
+
+def test_weights_buffer_layout(gpu_lib):
+    """mxmoe_weights_quantize: the four copies match the oracle byte for byte, the W1
+    rowwise copy with each expert's gate and up rows interleaved in 64-row blocks."""
+    E, H, F = 2, 256, 512
+    W1 = wl.random_matrix(2 * F, H, seed=41, std=0.02, batch=E)
+    W2 = wl.random_matrix(H, F, seed=42, std=0.02, batch=E)
+    wq = gpu_lib.mxmoe_weights_quantize(W1.cuda(), W2.cuda())
+    torch.cuda.synchronize()
+    views = [gpu_lib.mxmoe_weights_view(wq, E, H, F, w) for w in range(4)]
+    # destination row of W1 row r of one expert (gate rows 0..F-1, up rows F..2F-1)
+    r = np.arange(2 * F)
+    hf, rr = (r >= F).astype(int), r - (r >= F) * F
+    dst = (rr // 64) * 128 + hf * 64 + rr % 64
+    for e in range(E):
+        qr, sr = omx.quantize_rowwise(f64(W1[e]))
+        got, gsc = u8(views[0].data)[e * 2 * F:(e + 1) * 2 * F], u8(views[0].scale_plain())[e * 2 * F:(e + 1) * 2 * F]
+        np.testing.assert_array_equal(got[dst], qr)
+        np.testing.assert_array_equal(gsc[dst], sr)
+        qc, sc = omx.quantize_colwise_t(f64(W1[e]))
+        np.testing.assert_array_equal(u8(views[1].data)[e * H:(e + 1) * H], qc)
+        np.testing.assert_array_equal(u8(views[1].scale_plain())[e * H:(e + 1) * H], sc)
+        qr2, sr2 = omx.quantize_rowwise(f64(W2[e]))
+        np.testing.assert_array_equal(u8(views[2].data)[e * H:(e + 1) * H], qr2)
+        np.testing.assert_array_equal(u8(views[2].scale_plain())[e * H:(e + 1) * H], sr2)
+        qc2, sc2 = omx.quantize_colwise_t(f64(W2[e]))
+        np.testing.assert_array_equal(u8(views[3].data)[e * F:(e + 1) * F], qc2)
+        np.testing.assert_array_equal(u8(views[3].scale_plain())[e * F:(e + 1) * F], sc2)
