@@ -72,10 +72,10 @@ constexpr uint32_t kTmemSfb = 264;    // two buffers of 8 columns
 constexpr uint32_t kTmemStash = 384;  // epilogue scratch: 64 columns per (lane quadrant, half)
 constexpr int kPrefetchSteps = 8;     // K steps of the next tile pulled into L2 at a tile start
 
-// Per-variant layout. The plain-store and weight-gradient modes write their output
-// through shared memory with TMA stores (two 4 KB boxes per epilogue warp); the fused
-// modes keep 4 KB per warp for the colwise-quantisation transpose. Ring depths beyond 4
-// stages measured no faster on long-K tiles.
+// Per-variant layout. Every epilogue warp owns 8 KB of staging: two 4 KB output boxes for
+// the TMA stores of the plain-store and weight-gradient modes, two 4 KB transpose tiles
+// for the colwise quantisation of the fused modes. Ring depths beyond 4 stages measured
+// no faster.
 template <int PAIR, int MODE>
 struct Cfg {
   static constexpr bool kTmaStore = MODE == kModeStore || MODE == kModeWgrad;
@@ -83,11 +83,11 @@ struct Cfg {
   static constexpr int kThreads = kSplitRegs ? 384 : 320;
   static constexpr int kEpiWarp0 = kSplitRegs ? 4 : 2;      // first epilogue warp
   static constexpr int TM = 128 * PAIR;                        // output tile rows
-  static constexpr int STAGES = kTmaStore ? (PAIR == 2 ? 4 : 3) : (PAIR == 2 ? 5 : 3);
+  static constexpr int STAGES = PAIR == 2 ? 4 : 3;
   static constexpr uint32_t kBBytes = (BN / PAIR) * BK;        // this CTA's B rows per stage
   static constexpr uint32_t kStageBytes = PAIR == 2 ? 34816 : 51200;
   static constexpr uint32_t kTxBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // per CTA
-  static constexpr uint32_t kStagingPerWarp = kTmaStore ? 8192 : 4096;
+  static constexpr uint32_t kStagingPerWarp = 8192;
   static constexpr uint32_t kOffStaging = STAGES * kStageBytes;
   static constexpr uint32_t kOffBars = kOffStaging + kEpiWarps * kStagingPerWarp;
   static constexpr uint32_t kOffSeg = kOffBars + 256;
@@ -226,31 +226,46 @@ __device__ __forceinline__ uint8_t quant32(const float (&v)[32], uint32_t (&q)[8
   return (uint8_t)(X + 127);
 }
 
-// Warp-wide colwise MXFP8 of a 32 x 32 fp32 block held one row per lane (lane = row,
+// Warp-wide colwise MXFP8 of 32 x 32 fp32 blocks held one row per lane (lane = row,
 // v[i] = column i): each column's 32 values are one block, written transposed (column i
-// -> 32 consecutive bytes at dst + i*ld) with one scale byte per column. The block is
-// transposed through the warp's 4 KB staging buffer in one round: row r occupies words
+// -> 32 consecutive bytes at dst + i*ld) with one scale byte per column. A block is
+// transposed through 4 KB of the warp's staging buffer in one round: row r occupies words
 // [32r, 32r + 32) with its 16-byte chunk j stored at chunk j ^ (r % 8), so the row-wise
 // 16-byte writes and the column-wise 4-byte reads are both bank-conflict free; lane c
 // then holds column c whole.
-__device__ __forceinline__ void colwise_quant_store(const float (&v)[32], float* stg, int lane, uint8_t* dst,
-                                                    int64_t ld, uint8_t* sf_base, int64_t sf_rows, int64_t sf_cols,
-                                                    int64_t col_row0, int64_t kb) {
+// Two blocks go through the two 4 KB halves of the staging buffer together, with one
+// pair of warp syncs, so the two transposes and reductions interleave.
+__device__ __forceinline__ void colwise_quant_store2(const float (&v0)[32], const float (&v1)[32], float* stg, int lane,
+                                                     uint8_t* dst0, uint8_t* dst1, int64_t ld, uint8_t* sf_base,
+                                                     int64_t sf_rows, int64_t sf_cols, int64_t col_row0_0,
+                                                     int64_t col_row0_1, int64_t kb) {
+  float* stg1 = stg + 1024;
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    *reinterpret_cast<float4*>(stg + lane * 32 + ((j ^ (lane & 7)) << 2)) =
-        make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  for (int j = 0; j < 8; ++j) {
+    const int o = lane * 32 + ((j ^ (lane & 7)) << 2);
+    *reinterpret_cast<float4*>(stg + o) = make_float4(v0[4 * j], v0[4 * j + 1], v0[4 * j + 2], v0[4 * j + 3]);
+    *reinterpret_cast<float4*>(stg1 + o) = make_float4(v1[4 * j], v1[4 * j + 1], v1[4 * j + 2], v1[4 * j + 3]);
+  }
   __syncwarp();
-  float w[32];
+  float w0[32], w1[32];
 #pragma unroll
-  for (int r = 0; r < 32; ++r) w[r] = stg[r * 32 + ((((lane >> 2) ^ (r & 7)) << 2) | (lane & 3))];
-  __syncwarp();  // the buffer may be refilled once every lane has read its column
-  uint32_t q[8];
-  const uint8_t sb = quant32(w, q);
-  uint4* d = reinterpret_cast<uint4*>(dst + (int64_t)lane * ld);
-  d[0] = make_uint4(q[0], q[1], q[2], q[3]);
-  d[1] = make_uint4(q[4], q[5], q[6], q[7]);
-  sf_base[sf_offset(MXMOE_SCALE_MMA, sf_rows, sf_cols, col_row0 + lane, kb)] = sb;
+  for (int r = 0; r < 32; ++r) {
+    const int o = r * 32 + ((((lane >> 2) ^ (r & 7)) << 2) | (lane & 3));
+    w0[r] = stg[o];
+    w1[r] = stg1[o];
+  }
+  __syncwarp();  // the buffer may be refilled once every lane has read its columns
+  uint32_t q0[8], q1[8];
+  const uint8_t sb0 = quant32(w0, q0);
+  const uint8_t sb1 = quant32(w1, q1);
+  uint4* d0 = reinterpret_cast<uint4*>(dst0 + (int64_t)lane * ld);
+  uint4* d1 = reinterpret_cast<uint4*>(dst1 + (int64_t)lane * ld);
+  d0[0] = make_uint4(q0[0], q0[1], q0[2], q0[3]);
+  d0[1] = make_uint4(q0[4], q0[5], q0[6], q0[7]);
+  d1[0] = make_uint4(q1[0], q1[1], q1[2], q1[3]);
+  d1[1] = make_uint4(q1[4], q1[5], q1[6], q1[7]);
+  sf_base[sf_offset(MXMOE_SCALE_MMA, sf_rows, sf_cols, col_row0_0 + lane, kb)] = sb0;
+  sf_base[sf_offset(MXMOE_SCALE_MMA, sf_rows, sf_cols, col_row0_1 + lane, kb)] = sb1;
 }
 
 // Rowwise MXFP8 of the 32 values one thread holds: 32 codes to dst (32-byte aligned);
@@ -634,15 +649,13 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 64; ++i) zf[i] = silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]) * p;
         // phase 2: MXFP8 of Z, rowwise (fc2 operand) and colwise (fc2 weight-gradient operand)
-        uint32_t zsf = 0;
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const float(&z)[32] = *reinterpret_cast<const float(*)[32]>(&zf[32 * c]);
-          const int64_t fc = f0 + 32 * c;
-          zsf |= rowwise_quant_codes(z, g.z_row + row * F + fc) << (8 * c);
-          colwise_quant_store(z, stg, lane, g.z_colT + fc * g.rows_cap + mrow0, g.rows_cap, g.z_colT_sf, F,
-                              g.rows_cap, fc, mrow0 / 32);
-        }
+        const float(&z0)[32] = *reinterpret_cast<const float(*)[32]>(&zf[0]);
+        const float(&z1)[32] = *reinterpret_cast<const float(*)[32]>(&zf[32]);
+        const uint32_t zsf = rowwise_quant_codes(z0, g.z_row + row * F + f0) |
+                             (rowwise_quant_codes(z1, g.z_row + row * F + f0 + 32) << 8);
+        colwise_quant_store2(z0, z1, stg, lane, g.z_colT + f0 * g.rows_cap + mrow0,
+                             g.z_colT + (f0 + 32) * g.rows_cap + mrow0, g.rows_cap, g.z_colT_sf, F, g.rows_cap, f0,
+                             f0 + 32, mrow0 / 32);
         // row scales of the blocks [f0, f0 + 64): adjacent bytes (block index 2h, 2h + 1 mod 4)
         *reinterpret_cast<uint16_t*>(g.z_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F, row, f0 / 32)) =
             (uint16_t)zsf;
@@ -713,11 +726,10 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           }
           const int64_t fg = f0 + 32 * c;
           sfg |= rowwise_quant_codes(vg, g.dgu_row + row * F2 + fg) << (8 * c);
-          colwise_quant_store(vg, stg, lane, g.dgu_colT + fg * g.rows_cap + mrow0, g.rows_cap, g.dgu_colT_sf, F2,
-                              g.rows_cap, fg, mrow0 / 32);
           sfu |= rowwise_quant_codes(vu, g.dgu_row + row * F2 + F + fg) << (8 * c);
-          colwise_quant_store(vu, stg, lane, g.dgu_colT + (F + fg) * g.rows_cap + mrow0, g.rows_cap,
-                              g.dgu_colT_sf, F2, g.rows_cap, F + fg, mrow0 / 32);
+          colwise_quant_store2(vg, vu, stg, lane, g.dgu_colT + fg * g.rows_cap + mrow0,
+                               g.dgu_colT + (F + fg) * g.rows_cap + mrow0, g.rows_cap, g.dgu_colT_sf, F2, g.rows_cap,
+                               fg, F + fg, mrow0 / 32);
         }
         // row scales: blocks f0/32 .. +3 (and their up-half twins) are one aligned word each
         *reinterpret_cast<uint32_t*>(g.dgu_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F2, row, f0 / 32)) = sfg;
