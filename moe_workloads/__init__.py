@@ -179,3 +179,18 @@ def make_expert_weights(cfg: MoEConfig, e: int):
         w1 = (torch.randn((1, 2 * cfg.F, cfg.H), generator=g1) * 0.02).to(torch.bfloat16)
         w2 = (torch.randn((1, cfg.H, cfg.F), generator=g2) * 0.02).to(torch.bfloat16)
     return w1[0], w2[0]
+
+
+def make_weights_on(cfg: MoEConfig, device):
+    """W1 bf16[E,2F,H] and W2 bf16[E,H,F] ~N(0,0.02) drawn on ``device`` with a seeded
+    generator of that device, one expert at a time: the full-size workloads hold billions
+    of weights, which take minutes to draw on the CPU. Same shapes and distributions as
+    make_weights, different values."""
+    g = torch.Generator(device=device)
+    g.manual_seed(cfg.seed * 1000 + 6)
+    W1 = torch.empty((cfg.E, 2 * cfg.F, cfg.H), dtype=torch.bfloat16, device=device)
+    W2 = torch.empty((cfg.E, cfg.H, cfg.F), dtype=torch.bfloat16, device=device)
+    for e in range(cfg.E):
+        W1[e] = (torch.randn((2 * cfg.F, cfg.H), generator=g, device=device) * 0.02).to(torch.bfloat16)
+        W2[e] = (torch.randn((cfg.H, cfg.F), generator=g, device=device) * 0.02).to(torch.bfloat16)
+    return W1, W2
