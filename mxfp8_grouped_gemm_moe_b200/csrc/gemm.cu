@@ -234,11 +234,10 @@ __device__ __forceinline__ uint8_t quant32(const float (&v)[32], uint32_t (&q)[8
 // 16-byte writes and the column-wise 4-byte reads are both bank-conflict free; lane c
 // then holds column c whole.
 // Two blocks go through the two 4 KB halves of the staging buffer together, with one
-// pair of warp syncs, so the two transposes and reductions interleave.
-__device__ __forceinline__ void colwise_quant_store2(const float (&v0)[32], const float (&v1)[32], float* stg, int lane,
-                                                     uint8_t* dst0, uint8_t* dst1, int64_t ld, uint8_t* sf_base,
-                                                     int64_t sf_rows, int64_t sf_cols, int64_t col_row0_0,
-                                                     int64_t col_row0_1, int64_t kb) {
+// pair of warp syncs, so the two transposes and reductions interleave. Lane c gets the
+// 32 codes (and the scale byte) of column c of each block.
+__device__ __forceinline__ void colwise_codes2(const float (&v0)[32], const float (&v1)[32], float* stg, int lane,
+                                               uint32_t (&q0)[8], uint32_t (&q1)[8], uint8_t& sb0, uint8_t& sb1) {
   float* stg1 = stg + 1024;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
@@ -255,28 +254,26 @@ __device__ __forceinline__ void colwise_quant_store2(const float (&v0)[32], cons
     w1[r] = stg1[o];
   }
   __syncwarp();  // the buffer may be refilled once every lane has read its columns
-  uint32_t q0[8], q1[8];
-  const uint8_t sb0 = quant32(w0, q0);
-  const uint8_t sb1 = quant32(w1, q1);
-  uint4* d0 = reinterpret_cast<uint4*>(dst0 + (int64_t)lane * ld);
-  uint4* d1 = reinterpret_cast<uint4*>(dst1 + (int64_t)lane * ld);
-  d0[0] = make_uint4(q0[0], q0[1], q0[2], q0[3]);
-  d0[1] = make_uint4(q0[4], q0[5], q0[6], q0[7]);
-  d1[0] = make_uint4(q1[0], q1[1], q1[2], q1[3]);
-  d1[1] = make_uint4(q1[4], q1[5], q1[6], q1[7]);
-  sf_base[sf_offset(MXMOE_SCALE_MMA, sf_rows, sf_cols, col_row0_0 + lane, kb)] = sb0;
-  sf_base[sf_offset(MXMOE_SCALE_MMA, sf_rows, sf_cols, col_row0_1 + lane, kb)] = sb1;
+  sb0 = quant32(w0, q0);
+  sb1 = quant32(w1, q1);
 }
 
-// Rowwise MXFP8 of the 32 values one thread holds: 32 codes to dst (32-byte aligned);
-// returns the scale byte (the caller stores the scales of several blocks together).
-__device__ __forceinline__ uint32_t rowwise_quant_codes(const float (&v)[32], uint8_t* dst) {
-  uint32_t q[8];
-  const uint8_t sb = quant32(v, q);
-  uint4* d = reinterpret_cast<uint4*>(dst);
+// Fused-epilogue output path: a warp's 32 x 32 block of E4M3 codes (lane r's 32 bytes at
+// r * 32) is assembled in its staging buffer and written by one TMA store; the codes of
+// a chunk (up to four blocks) leave together. A block is written into the staging
+// buffer only after the warp's previous stores have read it.
+__device__ __forceinline__ void staging_acquire(int lane) {
+  if (lane == 0) ptx::bulk_wait_group_read<0>();
+  __syncwarp();
+}
+__device__ __forceinline__ void put_codes32(uint8_t* box, int lane, const uint32_t (&q)[8]) {
+  uint4* d = reinterpret_cast<uint4*>(box + lane * 32);
   d[0] = make_uint4(q[0], q[1], q[2], q[3]);
   d[1] = make_uint4(q[4], q[5], q[6], q[7]);
-  return sb;
+}
+__device__ __forceinline__ void staging_publish() {
+  ptx::fence_proxy_async_shared();
+  __syncwarp();
 }
 
 // Hands the accumulator back to the MMA warp once this warp's TMEM reads (and writes
@@ -333,7 +330,8 @@ template <int MODE, int PAIR>
 __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
     mxgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
-                  const __grid_constant__ CUtensorMap tmC, const __grid_constant__ GemmArgs g) {
+                  const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
+                  const __grid_constant__ CUtensorMap tmE, const __grid_constant__ GemmArgs g) {
   using C = Cfg<PAIR, MODE>;
   constexpr int STAGES = C::STAGES;
   constexpr uint32_t kStageBytes = C::kStageBytes;
@@ -373,7 +371,11 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
       ptx::prefetch_tensormap(&tmSFA);
       ptx::prefetch_tensormap(&tmSFB);
     }
-    if (C::kTmaStore) ptx::prefetch_tensormap(&tmC);
+    ptx::prefetch_tensormap(&tmC);
+    if (!C::kTmaStore) {
+      ptx::prefetch_tensormap(&tmD);
+      if (MODE == kModeSwigluFwd) ptx::prefetch_tensormap(&tmE);
+    }
   }
   if (warp == 1) {
     if (PAIR == 2) {
@@ -636,26 +638,45 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
         ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 96, *reinterpret_cast<uint32_t(*)[32]>(&ur[32]));
         ptx::tmem_wait_ld();
         release_accumulator<PAIR>(bar_acc_empty, acc_empty_leader, lane);
-        {
-          uint4* gd = reinterpret_cast<uint4*>(g.gu + row * F2 + f0);
-          uint4* ud = reinterpret_cast<uint4*>(g.gu + row * F2 + F + f0);
+        uint8_t* stg8 = reinterpret_cast<uint8_t*>(stg);
+        // G and U as bf16 for the backward: two 32-row x 128-byte boxes (128-byte swizzle)
+        staging_acquire(lane);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            gd[i] = pack8_bf16(gr, 8 * i);
-            ud[i] = pack8_bf16(ur, 8 * i);
-          }
+        for (int j = 0; j < 8; ++j) {
+          out_box_put(stg8, lane, j, pack8_bf16(gr, 8 * j));
+          out_box_put(stg8 + 4096, lane, j, pack8_bf16(ur, 8 * j));
+        }
+        staging_publish();
+        if (lane == 0) {
+          ptx::tma_store_2d(&tmE, stg8, (int32_t)f0, (int32_t)mrow0);
+          ptx::tma_store_2d(&tmE, stg8 + 4096, (int32_t)(F + f0), (int32_t)mrow0);
+          ptx::bulk_commit_group();
         }
         float zf[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i) zf[i] = silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]) * p;
-        // phase 2: MXFP8 of Z, rowwise (fc2 operand) and colwise (fc2 weight-gradient operand)
+        // MXFP8 of Z, rowwise (fc2 operand) and colwise (fc2 weight-gradient operand)
         const float(&z0)[32] = *reinterpret_cast<const float(*)[32]>(&zf[0]);
         const float(&z1)[32] = *reinterpret_cast<const float(*)[32]>(&zf[32]);
-        const uint32_t zsf = rowwise_quant_codes(z0, g.z_row + row * F + f0) |
-                             (rowwise_quant_codes(z1, g.z_row + row * F + f0 + 32) << 8);
-        colwise_quant_store2(z0, z1, stg, lane, g.z_colT + f0 * g.rows_cap + mrow0,
-                             g.z_colT + (f0 + 32) * g.rows_cap + mrow0, g.rows_cap, g.z_colT_sf, F, g.rows_cap, f0,
-                             f0 + 32, mrow0 / 32);
+        uint32_t r0[8], r1[8], c0[8], c1[8];
+        uint8_t cs0, cs1;
+        const uint32_t zsf = (uint32_t)quant32(z0, r0) | ((uint32_t)quant32(z1, r1) << 8);
+        staging_acquire(lane);
+        colwise_codes2(z0, z1, stg, lane, c0, c1, cs0, cs1);
+        put_codes32(stg8, lane, r0);
+        put_codes32(stg8 + 1024, lane, r1);
+        put_codes32(stg8 + 2048, lane, c0);
+        put_codes32(stg8 + 3072, lane, c1);
+        staging_publish();
+        if (lane == 0) {
+          ptx::tma_store_2d(&tmC, stg8, (int32_t)f0, (int32_t)mrow0);
+          ptx::tma_store_2d(&tmC, stg8 + 1024, (int32_t)(f0 + 32), (int32_t)mrow0);
+          ptx::tma_store_2d(&tmD, stg8 + 2048, (int32_t)mrow0, (int32_t)f0);
+          ptx::tma_store_2d(&tmD, stg8 + 3072, (int32_t)mrow0, (int32_t)(f0 + 32));
+          ptx::bulk_commit_group();
+        }
+        g.z_colT_sf[sf_offset(MXMOE_SCALE_MMA, F, g.rows_cap, f0 + lane, mrow0 / 32)] = cs0;
+        g.z_colT_sf[sf_offset(MXMOE_SCALE_MMA, F, g.rows_cap, f0 + 32 + lane, mrow0 / 32)] = cs1;
         // row scales of the blocks [f0, f0 + 64): adjacent bytes (block index 2h, 2h + 1 mod 4)
         *reinterpret_cast<uint16_t*>(g.z_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F, row, f0 / 32)) =
             (uint16_t)zsf;
@@ -725,11 +746,27 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
             vu[i] = da * sl;
           }
           const int64_t fg = f0 + 32 * c;
-          sfg |= rowwise_quant_codes(vg, g.dgu_row + row * F2 + fg) << (8 * c);
-          sfu |= rowwise_quant_codes(vu, g.dgu_row + row * F2 + F + fg) << (8 * c);
-          colwise_quant_store2(vg, vu, stg, lane, g.dgu_colT + fg * g.rows_cap + mrow0,
-                               g.dgu_colT + (F + fg) * g.rows_cap + mrow0, g.rows_cap, g.dgu_colT_sf, F2, g.rows_cap,
-                               fg, F + fg, mrow0 / 32);
+          uint32_t rg[8], ru[8], cg[8], cu[8];
+          uint8_t csg, csu;
+          sfg |= (uint32_t)quant32(vg, rg) << (8 * c);
+          sfu |= (uint32_t)quant32(vu, ru) << (8 * c);
+          staging_acquire(lane);
+          colwise_codes2(vg, vu, stg, lane, cg, cu, csg, csu);
+          uint8_t* stg8 = reinterpret_cast<uint8_t*>(stg);
+          put_codes32(stg8, lane, rg);
+          put_codes32(stg8 + 1024, lane, ru);
+          put_codes32(stg8 + 2048, lane, cg);
+          put_codes32(stg8 + 3072, lane, cu);
+          staging_publish();
+          if (lane == 0) {
+            ptx::tma_store_2d(&tmC, stg8, (int32_t)fg, (int32_t)mrow0);
+            ptx::tma_store_2d(&tmC, stg8 + 1024, (int32_t)(F + fg), (int32_t)mrow0);
+            ptx::tma_store_2d(&tmD, stg8 + 2048, (int32_t)mrow0, (int32_t)fg);
+            ptx::tma_store_2d(&tmD, stg8 + 3072, (int32_t)mrow0, (int32_t)(F + fg));
+            ptx::bulk_commit_group();
+          }
+          g.dgu_colT_sf[sf_offset(MXMOE_SCALE_MMA, F2, g.rows_cap, fg + lane, mrow0 / 32)] = csg;
+          g.dgu_colT_sf[sf_offset(MXMOE_SCALE_MMA, F2, g.rows_cap, F + fg + lane, mrow0 / 32)] = csu;
         }
         // row scales: blocks f0/32 .. +3 (and their up-half twins) are one aligned word each
         *reinterpret_cast<uint32_t*>(g.dgu_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F2, row, f0 / 32)) = sfg;
@@ -739,7 +776,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
       }
     }
     // output boxes fully written before the CTA retires
-    if (C::kTmaStore && lane == 0) ptx::bulk_wait_group<0>();
+    if (lane == 0) ptx::bulk_wait_group<0>();
   }
 
   // ---- teardown: every role has finished issuing; the epilogue has drained the last
@@ -815,8 +852,23 @@ static bool make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Map over a [rows, cols] uint8 code matrix for the fused epilogues' TMA stores: box 32 x
+// 32 bytes, no swizzle (one warp's block of codes).
+static bool make_codes32_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct GemmMaps {
-  CUtensorMap a, b, sfa, sfb, c;
+  CUtensorMap a, b, sfa, sfb;
+  CUtensorMap c, d, e;  // epilogue outputs (unused ones zeroed)
 };
 
 template <int MODE, int PAIR>
@@ -833,7 +885,7 @@ static cudaError_t launch_mode(const GemmMaps& m, const GemmArgs& g, int64_t til
   const int units = gemm_num_sms() / PAIR;  // SMs, or SM pairs
   const int n = (int)(tiles_ub < units ? (tiles_ub > 0 ? tiles_ub : 1) : units);
   if (PAIR == 1) {
-    mxgemm_kernel<MODE, 1><<<n, Cfg<PAIR, MODE>::kThreads, smem, st>>>(m.a, m.b, m.sfa, m.sfb, m.c, g);
+    mxgemm_kernel<MODE, 1><<<n, Cfg<PAIR, MODE>::kThreads, smem, st>>>(m.a, m.b, m.sfa, m.sfb, m.c, m.d, m.e, g);
   } else {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * n, 1, 1);
@@ -847,7 +899,7 @@ static cudaError_t launch_mode(const GemmMaps& m, const GemmArgs& g, int64_t til
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, mxgemm_kernel<MODE, PAIR>, m.a, m.b, m.sfa, m.sfb, m.c, g);
+    e = cudaLaunchKernelEx(&cfg, mxgemm_kernel<MODE, PAIR>, m.a, m.b, m.sfa, m.sfb, m.c, m.d, m.e, g);
     if (e != cudaSuccess) return e;
   }
   ++g_launch_count;
@@ -858,6 +910,8 @@ template <int PAIR>
 static cudaError_t launch_variant(const GemmArgs& g, cudaStream_t st) {
   GemmMaps m;
   std::memset(&m.c, 0, sizeof(m.c));
+  std::memset(&m.d, 0, sizeof(m.d));
+  std::memset(&m.e, 0, sizeof(m.e));
   if (!make_map(&m.a, g.a_data, g.a_rows, g.a_cols) || !make_map(&m.b, g.b_data, g.b_rows, g.b_cols) ||
       !make_sf_map(&m.sfa, g.a_sf, (g.a_rows / 128) * (g.a_cols / 128)) ||
       !make_sf_map(&m.sfb, g.b_sf, (g.b_rows / 128) * (g.b_cols / 128)))
@@ -868,8 +922,14 @@ static cudaError_t launch_variant(const GemmArgs& g, cudaStream_t st) {
       if (!make_out_map(&m.c, g.c, g.a_rows, g.N, g.ldc, g.c_dtype == MXMOE_DTYPE_F32)) return cudaErrorInvalidValue;
       return launch_mode<kModeStore, PAIR>(m, g, (g.a_rows / TM) * (g.N / BN), st);
     case kModeSwigluFwd:
+      if (!make_codes32_map(&m.c, g.z_row, g.rows_cap, g.F) || !make_codes32_map(&m.d, g.z_colT, g.F, g.rows_cap) ||
+          !make_out_map(&m.e, g.gu, g.rows_cap, 2 * g.F, 2 * g.F, false))
+        return cudaErrorInvalidValue;
       return launch_mode<kModeSwigluFwd, PAIR>(m, g, (g.a_rows / TM) * (g.F / 128), st);
     case kModeSwigluBwd:
+      if (!make_codes32_map(&m.c, g.dgu_row, g.rows_cap, 2 * g.F) ||
+          !make_codes32_map(&m.d, g.dgu_colT, 2 * g.F, g.rows_cap))
+        return cudaErrorInvalidValue;
       return launch_mode<kModeSwigluBwd, PAIR>(m, g, (g.a_rows / TM) * (g.F / BN), st);
     case kModeWgrad:
       if (!make_out_map(&m.c, g.c, (int64_t)g.E * g.N, g.K2, g.K2, true)) return cudaErrorInvalidValue;
