@@ -625,7 +625,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           }
         }
       } else if (MODE == kModeSwigluFwd) {
-        const int64_t F = g.F, F2 = 2 * g.F;
+        const int64_t F = g.F;
         const float p = g.prob_of_row[row];
         const int64_t f0 = (int64_t)t.n_tile * 128 + 64 * h;  // this warp's 64 Z columns
         // drain gate / up (TMEM columns [128h, +64) and [128h + 64, +64), the interleaved
