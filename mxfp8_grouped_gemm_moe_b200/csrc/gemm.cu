@@ -72,10 +72,11 @@ constexpr uint32_t kTmemSfb = 264;    // two buffers of 8 columns
 constexpr uint32_t kTmemStash = 384;  // epilogue scratch: 64 columns per (lane quadrant, half)
 constexpr int kPrefetchSteps = 8;     // K steps of the next tile pulled into L2 at a tile start
 
-// Per-variant layout. Every epilogue warp owns 8 KB of staging: two 4 KB output boxes for
-// the TMA stores of the plain-store and weight-gradient modes, two 4 KB transpose tiles
-// for the colwise quantisation of the fused modes. Ring depths beyond 4 stages measured
-// no faster.
+// Per-variant layout. Plain-store and weight-gradient modes: 5-stage operand ring, one
+// 4 KB output box per epilogue warp for the TMA stores (the deeper ring measured faster
+// for the short-K weight-gradient tiles than a second box). Fused modes: 4 stages and
+// 8 KB per warp (two 4 KB transpose tiles, then the code blocks); 3 stages measured
+// clearly slower there.
 template <int PAIR, int MODE>
 struct Cfg {
   static constexpr bool kTmaStore = MODE == kModeStore || MODE == kModeWgrad;
@@ -83,11 +84,11 @@ struct Cfg {
   static constexpr int kThreads = kSplitRegs ? 384 : 320;
   static constexpr int kEpiWarp0 = kSplitRegs ? 4 : 2;      // first epilogue warp
   static constexpr int TM = 128 * PAIR;                        // output tile rows
-  static constexpr int STAGES = PAIR == 2 ? 4 : 3;
+  static constexpr int STAGES = PAIR == 2 ? (kTmaStore ? 5 : 4) : 3;
   static constexpr uint32_t kBBytes = (BN / PAIR) * BK;        // this CTA's B rows per stage
   static constexpr uint32_t kStageBytes = PAIR == 2 ? 34816 : 51200;
   static constexpr uint32_t kTxBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // per CTA
-  static constexpr uint32_t kStagingPerWarp = 8192;
+  static constexpr uint32_t kStagingPerWarp = kTmaStore ? 4096 : 8192;
   static constexpr uint32_t kOffStaging = STAGES * kStageBytes;
   static constexpr uint32_t kOffBars = kOffStaging + kEpiWarps * kStagingPerWarp;
   static constexpr uint32_t kOffSeg = kOffBars + 256;
@@ -289,17 +290,17 @@ __device__ __forceinline__ void release_accumulator(uint64_t* bar_local, uint32_
   }
 }
 
-// Plain-store epilogue output path: each epilogue warp owns two 4 KB staging boxes of
-// 32 rows x 128 bytes in the TMA 128-byte-swizzle layout (16-byte chunk j of row r at
-// chunk j ^ (r % 8), which also makes the row-per-lane writes bank-conflict free). A box
-// is filled by the warp and written out by one TMA store; the two boxes alternate, so a
-// box is reused only after the store issued two boxes earlier has read it.
+// Plain-store epilogue output path: each epilogue warp owns a 4 KB staging box of 32 rows
+// x 128 bytes in the TMA 128-byte-swizzle layout (16-byte chunk j of row r at chunk
+// j ^ (r % 8), which also makes the row-per-lane writes bank-conflict free). The box is
+// filled by the warp and written out by one TMA store, and refilled only after that
+// store has read it.
 __device__ __forceinline__ uint8_t* out_box_acquire(uint8_t* stg8, uint32_t n_out, int lane) {
-  if (n_out >= 2) {
-    if (lane == 0) ptx::bulk_wait_group_read<1>();
+  if (n_out >= 1) {
+    if (lane == 0) ptx::bulk_wait_group_read<0>();
     __syncwarp();
   }
-  return stg8 + (n_out & 1u) * 4096;
+  return stg8;
 }
 __device__ __forceinline__ void out_box_put(uint8_t* box, int lane, int j, uint4 v) {
   *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
