@@ -18,8 +18,10 @@ reading, and each function's docstring says which.
 
 Pins (tests marked ``not gpu``): exhaustive E4M3 round trip, hand-built
 quantisation blocks, brute-force permutation, per-token loop == grouped forward,
-dense-MLP reduction, SwiGLU closed forms, finite differences of the backward.
+dense-MLP reduction, SwiGLU closed forms, finite differences of the backward; for the
+router (``router``): softmax closed forms, brute-force top-k with ties, -inf experts,
+finite differences of the top-k backward.
 Parity unpinned: the end-to-end numeric level against the pages (they print no
 accuracy, loss or worked example).
 """
-from . import mxfp8, moe  # noqa: F401
+from . import mxfp8, moe, router  # noqa: F401
