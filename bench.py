@@ -324,6 +324,33 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
     mx.mxmoe_profile_disable()
     ms = max_over_ranks(dist, ms)
 
+    # ---- router (the step upstream of the layer; timed on its own, not part of `value`)
+    router = None
+    if rank == 0:
+        lg = torch.randn((cfg.T, cfg.E), generator=g, device=dev)
+        ridx, rp = mx.moe_router_topk(lg, cfg.k)
+        rdp = torch.randn_like(rp)
+        rdl = mx.moe_router_topk_bwd(lg, ridx, rdp)
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        times = []
+        for fn in (lambda: mx.moe_router_topk(lg, cfg.k), lambda: mx.moe_router_topk_bwd(lg, ridx, rdp)):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            r0.record(stream)
+            for _ in range(20):
+                fn()
+            r1.record(stream)
+            torch.cuda.synchronize()
+            times.append(r0.elapsed_time(r1) / 20)
+        fb = cfg.T * cfg.E * 4 + cfg.T * cfg.k * 8
+        bb = 2 * cfg.T * cfg.E * 4 + cfg.T * cfg.k * 8
+        router = {"fwd_ms": times[0], "bwd_ms": times[1], "fwd_gbs": fb / (times[0] * 1e-3) / 1e9,
+                  "bwd_gbs": bb / (times[1] * 1e-3) / 1e9,
+                  "note": "softmax over all experts + top-k, and its backward, on [T, E] fp32 logits; "
+                          "timed separately (the layer's input routing is given)"}
+        del lg, ridx, rp, rdp, rdl
+
     # ---- end to end through the public API with host buffers: every step copies its
     # inputs (x, top-k ids, probabilities, dY) from pinned host memory and reads its
     # results (y, dX, dprobs) back. The copies run on a side stream, double-buffered, so
@@ -460,7 +487,7 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
             "gemm_tflops": (18.0 * MHF) / (gemm_ms * 1e-3) / 1e12,
             "gemm_frac_of_measured_fp8": (18.0 * MHF) / (gemm_ms * 1e-3) / 1e12 / fp8_peak,
             "roofline": roofline, "roofline_hbm": roofline_hbm, "stages": stage_json,
-            "gpu_launches": launches, "e2e": e2e, "clocks": clk}
+            "gpu_launches": launches, "e2e": e2e, "clocks": clk, "router": router}
     return line
 
 

@@ -100,6 +100,37 @@ mxmoe_status mxmoe_clear_device_status(void* stream);
  * experts: roundup(T*k + 255*E, 256). Every [Mp, *] buffer below has this many rows. */
 int64_t mxmoe_rows_capacity(int32_t T, int32_t k, int32_t E);
 
+/* ------------------------------------------------------------------ router (upstream of the path) */
+
+/*
+ * moe_router_topk -- the router step ahead of the expert MLP ("MoE-Training für
+ * biologische Grundmodelle optimieren", routing passage: a router assigns every token to
+ * its experts). The pages give no formula; readings: probabilities are a softmax over all
+ * E experts (not renormalised over the k selected), the k largest are selected in
+ * descending order, equal logits keep the lower expert index first, and a logit of -inf
+ * marks an expert the token may not use (probability 0; selected last).
+ *   logits_dev    float [T, E]  row-major, finite or -inf, at least one finite per row.
+ *   topk_idx_dev  int32 [T, k]  out: selected experts, descending probability.
+ *   probs_dev     float [T, k]  out: their softmax probabilities (fp32).
+ * A row with NaN or no finite logit sets MXMOE_ERR_DEVICE_CHECK and gets ids -1 and
+ * probabilities 0 (moe_permute then rejects those pairs).
+ * Limits: 1 <= E <= 256, 1 <= k <= min(E, 8), T >= 0.
+ */
+mxmoe_status moe_router_topk(const float* logits_dev, int32_t T, int32_t E, int32_t k, int32_t* topk_idx_dev,
+                             float* probs_dev, void* stream);
+
+/*
+ * moe_router_topk_bwd -- gradient of a loss that depends on the selected probabilities:
+ *   dlogits[t, e] = P[t, e] * (g[t, e] - sum_j dprobs[t, j] * P[t, idx[t, j]]),
+ * P the softmax of the row, g[t, e] = dprobs[t, j] for e = idx[t, j] (0 otherwise).
+ * The softmax is recomputed from the logits (nothing is saved by the forward).
+ *   logits_dev [T, E], topk_idx_dev [T, k] (as returned by moe_router_topk),
+ *   dprobs_dev float [T, k], dlogits_dev float [T, E] (out).
+ * Same limits and device checks as the forward.
+ */
+mxmoe_status moe_router_topk_bwd(const float* logits_dev, const int32_t* topk_idx_dev, const float* dprobs_dev,
+                                 int32_t T, int32_t E, int32_t k, float* dlogits_dev, void* stream);
+
 /* ------------------------------------------------------------------ routing (GroupedLinear input) */
 
 /*
@@ -315,6 +346,8 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
 #define MXMOE_STAGE_GEMM 15          /* standalone grouped_gemm_mxfp8 */
 #define MXMOE_STAGE_WGRAD 16         /* standalone grouped_gemm_mxfp8_wgrad */
 #define MXMOE_STAGE_QUANT 17         /* standalone mxfp8_quantize */
+#define MXMOE_STAGE_ROUTER 18        /* moe_router_topk */
+#define MXMOE_STAGE_ROUTER_BWD 19    /* moe_router_topk_bwd */
 
 /* Host-side stage timing, off by default: while enabled, every stage the library
  * enqueues is bracketed by two CUDA events recorded on that stage's stream (up to

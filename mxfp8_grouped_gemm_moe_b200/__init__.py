@@ -58,6 +58,8 @@ _SIGNATURES = {
     "moe_permute_workspace_size": (_SZ, [_I32, _I32, _I32]),
     "moe_permute_noalloc": (_I32, [_P, _P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P]),
     "moe_unpermute": (_I32, [_P, _P, _I32, _I32, _I32, _P, _P]),
+    "moe_router_topk": (_I32, [_P, _I32, _I32, _I32, _P, _P, _P]),
+    "moe_router_topk_bwd": (_I32, [_P, _P, _P, _I32, _I32, _I32, _P, _P]),
     "mxfp8_quantize": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _I64, _PMX, _PMX, _P]),
     "grouped_gemm_mxfp8": (_I32, [_PMX, _PMX, _P, _I32, _I64, _I64, _P, _I32, _I64, _P]),
     "grouped_gemm_mxfp8_wgrad": (_I32, [_PMX, _PMX, _P, _I32, _P, _P]),
@@ -77,7 +79,8 @@ _SIGNATURES = {
 
 STAGE_NAMES = {1: "route", 2: "quant_x", 3: "fc1_swiglu", 4: "fc2", 5: "combine", 6: "quant_w1", 7: "quant_w2",
                8: "quant_dy", 9: "fc2_dgrad_swiglu_bwd", 10: "dprob", 11: "fc2_wgrad", 12: "fc1_dgrad",
-               13: "fc1_wgrad", 14: "combine_dx", 15: "gemm", 16: "wgrad", 17: "quant"}
+               13: "fc1_wgrad", 14: "combine_dx", 15: "gemm", 16: "wgrad", 17: "quant", 18: "router",
+               19: "router_bwd"}
 
 
 def load(path: str | None = None):
@@ -195,6 +198,26 @@ def moe_unpermute(y_perm, row_of_slot, out=None):
     y = out if out is not None else torch.empty((T, H), dtype=torch.bfloat16, device=y_perm.device)
     _check("moe_unpermute", load().moe_unpermute(_ptr(y_perm), _ptr(row_of_slot), T, k, H, _ptr(y), _stream()))
     return y
+
+
+
+def moe_router_topk(logits, k):
+    """logits float32 [T, E] (cuda) -> (topk_idx int32 [T, k], probs float32 [T, k])."""
+    T, E = logits.shape
+    idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    probs = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    _check("moe_router_topk", load().moe_router_topk(_ptr(logits), T, E, k, _ptr(idx), _ptr(probs), _stream()))
+    return idx, probs
+
+
+def moe_router_topk_bwd(logits, topk_idx, dprobs):
+    """-> dlogits float32 [T, E]."""
+    T, E = logits.shape
+    k = topk_idx.shape[1]
+    dl = torch.empty((T, E), dtype=torch.float32, device=logits.device)
+    _check("moe_router_topk_bwd", load().moe_router_topk_bwd(_ptr(logits), _ptr(topk_idx), _ptr(dprobs), T, E, k,
+                                                                 _ptr(dl), _stream()))
+    return dl
 
 
 def mxfp8_quantize(src, rowwise=True, colwise=True, layout=SCALE_MMA, row_gather=None, nrows=None, out_rows=None):

@@ -246,6 +246,24 @@ mxmoe_status moe_permute(const int32_t* topk_idx_dev, const float* probs_dev, in
                                   token_of_row_dev, prob_of_row_dev, ws_dev, S(stream)));
 }
 
+mxmoe_status moe_router_topk(const float* logits_dev, int32_t T, int32_t E, int32_t k, int32_t* topk_idx_dev,
+                             float* probs_dev, void* stream) {
+  if (T < 0 || E < 1 || E > 256 || k < 1 || k > 8 || k > E) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MXMOE_OK;
+  if (!logits_dev || !topk_idx_dev || !probs_dev) return MXMOE_ERR_INVALID_ARG;
+  StageScope sc(MXMOE_STAGE_ROUTER, S(stream));
+  return cuda_status(launch_router_topk(logits_dev, T, E, k, topk_idx_dev, probs_dev, S(stream)));
+}
+
+mxmoe_status moe_router_topk_bwd(const float* logits_dev, const int32_t* topk_idx_dev, const float* dprobs_dev,
+                                 int32_t T, int32_t E, int32_t k, float* dlogits_dev, void* stream) {
+  if (T < 0 || E < 1 || E > 256 || k < 1 || k > 8 || k > E) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MXMOE_OK;
+  if (!logits_dev || !topk_idx_dev || !dprobs_dev || !dlogits_dev) return MXMOE_ERR_INVALID_ARG;
+  StageScope sc(MXMOE_STAGE_ROUTER_BWD, S(stream));
+  return cuda_status(launch_router_topk_bwd(logits_dev, topk_idx_dev, dprobs_dev, T, E, k, dlogits_dev, S(stream)));
+}
+
 mxmoe_status moe_unpermute(const void* y_perm_dev, const int32_t* row_of_slot_dev, int32_t T, int32_t k, int32_t H,
                            void* y_dev, void* stream) {
   if (T < 0 || k < 1 || k > 8 || H <= 0 || H % 8 != 0) return MXMOE_ERR_UNSUPPORTED_SHAPE;

@@ -22,6 +22,12 @@ cudaError_t launch_unpermute(const void* yp, const int32_t* ros, int T, int k, i
 cudaError_t launch_dprob_reduce(const float* part, int nparts, const int32_t* ros, int64_t n, float* dprobs,
                                 cudaStream_t st);
 
+// ---------------------------------------------------------------- router
+cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* probs,
+                               cudaStream_t st);
+cudaError_t launch_router_topk_bwd(const float* logits, const int32_t* idx, const float* dprobs, int T, int E, int k,
+                                   float* dlogits, cudaStream_t st);
+
 // ---------------------------------------------------------------- quantisation
 struct QuantArgs {
   const void* src;

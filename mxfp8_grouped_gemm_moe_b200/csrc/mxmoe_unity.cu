@@ -2,6 +2,7 @@
 // kernels without relocatable device code).
 #include "route.cu"
 #include "route_noalloc.cu"
+#include "router.cu"
 #include "quantize.cu"
 #include "gemm.cu"
 #include "api.cu"

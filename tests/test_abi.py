@@ -83,6 +83,14 @@ def test_host_argument_errors_enqueue_nothing(lib):
     assert lib.moe_permute(fake, fake, 10, 2, 4, fake, fake, fake, fake, fake, fake, 4, S) == 3
     assert lib.moe_unpermute(fake, fake, 4, 2, 12, fake, S) == 2            # H % 8
     assert lib.moe_unpermute(bad, fake, 4, 2, 16, fake, S) == 1
+    # router: k above E or 8, E out of range, missing outputs; T = 0 is a no-op
+    assert lib.moe_router_topk(fake, 16, 4, 5, fake, fake, S) == 2
+    assert lib.moe_router_topk(fake, 16, 300, 2, fake, fake, S) == 2
+    assert lib.moe_router_topk(fake, 16, 64, 9, fake, fake, S) == 2
+    assert lib.moe_router_topk(fake, 16, 8, 2, None, fake, S) == 1
+    assert lib.moe_router_topk(None, 0, 8, 2, None, None, S) == 0
+    assert lib.moe_router_topk_bwd(fake, fake, None, 16, 8, 2, fake, S) == 1
+    assert lib.moe_router_topk_bwd(fake, fake, fake, 16, 0, 1, fake, S) == 2
     # quantize: bad dtype, bad shape, no outputs
     m = mx._MX(1 << 20, 1 << 20, 64, 64, 0, 0)
     assert lib.mxfp8_quantize(fake, 7, 1, 64, 64, None, None, 64, ctypes.byref(m), None, S) == 1
