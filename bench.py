@@ -57,6 +57,8 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=512, help="routed rows in the CPU oracle sample")
     p.add_argument("--cpu-fslice", type=int, default=1024, help="FFN columns in the CPU oracle sample")
+    p.add_argument("--no-bf16-compare", action="store_true",
+                   help="skip timing the six GEMM stages on bf16 operands (same scheduler) for comparison")
     return p.parse_args()
 
 
@@ -266,6 +268,63 @@ def config_json(cfg, world):
 
 
 # ----------------------------------------------------------------------------- GPU arm
+def time_bf16_gemms(cfg, layer, stream, g, dev, stage_json_ms=None, iters=5):
+    """Each GEMM stage of the layer on bf16 operands with the layer's own routing (expert
+    segments of the saved forward): fc1 / fc2 / fc2 dgrad / fc1 dgrad as plain grouped
+    GEMMs (bf16 out), the two weight gradients as grouped wgrad GEMMs (fp32 out)."""
+    import torch
+
+    import mxfp8_grouped_gemm_moe_b200 as mx
+    E, H, F, cap = cfg.E, cfg.H, cfg.F, layer.cap
+    seg = layer.saved_field("seg_off", torch.int32, E + 1)
+    r = lambda *sh: (torch.randn(sh, generator=g, device=dev) * 0.05).to(torch.bfloat16)  # noqa: E731
+    ms = {}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timeit(name, fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(iters):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms[name] = e0.elapsed_time(e1) / iters
+
+    xa, w1 = r(cap, H), r(E * 2 * F, H)
+    out = torch.empty((cap, 2 * F), dtype=torch.bfloat16, device=dev)
+    timeit("fc1_swiglu", lambda: mx.grouped_gemm_bf16(xa, w1, seg, E, 2 * F, out=out))
+    del out
+    za, w2 = r(cap, F), r(E * H, F)
+    out = torch.empty((cap, H), dtype=torch.bfloat16, device=dev)
+    timeit("fc2", lambda: mx.grouped_gemm_bf16(za, w2, seg, E, H, out=out))
+    del w2
+    dya, w2t = r(cap, H), r(E * F, H)
+    out2 = torch.empty((cap, F), dtype=torch.bfloat16, device=dev)
+    timeit("fc2_dgrad_swiglu_bwd", lambda: mx.grouped_gemm_bf16(dya, w2t, seg, E, F, out=out2))
+    del w2t, out2
+    dyt, zt = dya.t().contiguous(), za.t().contiguous()
+    del dya, za
+    dw2 = torch.empty((E, H, F), dtype=torch.float32, device=dev)
+    timeit("fc2_wgrad", lambda: mx.grouped_gemm_bf16_wgrad(dyt, zt, seg, E, out=dw2))
+    del dyt, zt, dw2, w1
+    dgu, w1t = r(cap, 2 * F), r(E * H, 2 * F)
+    timeit("fc1_dgrad", lambda: mx.grouped_gemm_bf16(dgu, w1t, seg, E, H, out=out))
+    del w1t, out
+    dgut, xt = dgu.t().contiguous(), xa.t().contiguous()
+    del dgu, xa
+    dw1 = torch.empty((E, 2 * F, H), dtype=torch.float32, device=dev)
+    timeit("fc1_wgrad", lambda: mx.grouped_gemm_bf16_wgrad(dgut, xt, seg, E, out=dw1))
+    del dgut, xt, dw1
+    torch.cuda.empty_cache()
+    MHF = float(cfg.M) * H * F
+    return {"ms": ms, "total_ms": sum(ms.values()),
+            "tflops": {n: GEMM_FLOP_FACTOR[n] * MHF / (t * 1e-3) / 1e12 for n, t in ms.items()},
+            "note": "bf16 operands on the same grouped scheduler (kind::f16, CTA pairs), plain outputs; compare "
+                    "with the MXFP8 stage times of the same run"}
+
+
 def run_gpu(args, cfg, dist, rank, world, local_rank):
     import torch
 
@@ -323,6 +382,12 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
     stages = mx.mxmoe_profile_read()
     mx.mxmoe_profile_disable()
     ms = max_over_ranks(dist, ms)
+
+    # ---- the six GEMM stages on bf16 operands (same scheduler, CTA-pair tiles, kind::f16):
+    # the 16-bit comparison point, timed on its own (plain outputs, no fused epilogues)
+    bf16_gemms = None
+    if rank == 0 and world == 1 and not args.no_bf16_compare:
+        bf16_gemms = time_bf16_gemms(cfg, layer, stream, g, dev, stage_json_ms=None)
 
     # ---- router (the step upstream of the layer; timed on its own, not part of `value`)
     router = None
@@ -488,6 +553,12 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
             "gemm_frac_of_measured_fp8": (18.0 * MHF) / (gemm_ms * 1e-3) / 1e12 / fp8_peak,
             "roofline": roofline, "roofline_hbm": roofline_hbm, "stages": stage_json,
             "gpu_launches": launches, "e2e": e2e, "clocks": clk, "router": router}
+    if bf16_gemms is not None:
+        mx_ms = {n: stage_json[n]["ms"] for n in GEMM_FLOP_FACTOR}
+        bf16_gemms["mxfp8_ms"] = mx_ms
+        bf16_gemms["mxfp8_total_ms"] = sum(mx_ms.values())
+        bf16_gemms["speedup_mxfp8_over_bf16"] = bf16_gemms["total_ms"] / bf16_gemms["mxfp8_total_ms"]
+        line["bf16_gemms"] = bf16_gemms
     return line
 
 

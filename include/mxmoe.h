@@ -250,6 +250,26 @@ mxmoe_status grouped_gemm_mxfp8(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, cons
 mxmoe_status grouped_gemm_mxfp8_wgrad(const mxmoe_mxfp8* At, const mxmoe_mxfp8* Bt, const int32_t* seg_off_dev,
                                       int32_t E, float* C_dev, void* stream);
 
+/*
+ * grouped_gemm_bf16 / grouped_gemm_bf16_wgrad -- the same grouped GEMMs on bf16 operands
+ * (no quantisation; the 16-bit comparison point the pages set MXFP8 against: "MoE-Training
+ * für biologische Grundmodelle optimieren", MXFP8 passage), on the same persistent
+ * scheduler and CTA-pair tiles, fp32 accumulation (tcgen05 kind::f16).
+ *   grouped_gemm_bf16: C[seg_e, :] = A[seg_e, :] . B_e^T
+ *     A_dev  bf16 [rows_cap, K] row-major; B_dev bf16 [E*N, K]; seg_off_dev as above;
+ *     C_dev  [rows_cap, ldc] of c_dtype (MXMOE_DTYPE_BF16 or _F32).
+ *     Shapes: rows_cap % 256 == 0, N % 256 == 0, K % 64 == 0, ldc >= N, ldc % 8 == 0.
+ *   grouped_gemm_bf16_wgrad: C[e] = At[:, seg_e] . Bt[:, seg_e]^T, fp32 [E, N, K2]
+ *     At_dev bf16 [N, rows_cap]; Bt_dev bf16 [K2, rows_cap] (transposed activations /
+ *     gradients). Shapes: N % 256 == 0, K2 % 256 == 0, rows_cap % 256 == 0.
+ * All pointers 16-byte aligned; segment offsets are checked on the device as above.
+ */
+mxmoe_status grouped_gemm_bf16(const void* A_dev, int64_t rows_cap, const void* B_dev, const int32_t* seg_off_dev,
+                               int32_t E, int64_t N, int64_t K, void* C_dev, int32_t c_dtype, int64_t ldc,
+                               void* stream);
+mxmoe_status grouped_gemm_bf16_wgrad(const void* At_dev, const void* Bt_dev, int64_t N, int64_t K2, int64_t rows_cap,
+                                     const int32_t* seg_off_dev, int32_t E, float* C_dev, void* stream);
+
 /* ------------------------------------------------------------------ fused grouped MLP (GroupedMLP) */
 
 /*

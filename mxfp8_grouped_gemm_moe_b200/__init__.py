@@ -59,6 +59,8 @@ _SIGNATURES = {
     "moe_permute_noalloc": (_I32, [_P, _P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P]),
     "moe_unpermute": (_I32, [_P, _P, _I32, _I32, _I32, _P, _P]),
     "moe_router_topk": (_I32, [_P, _I32, _I32, _I32, _P, _P, _P]),
+    "grouped_gemm_bf16": (_I32, [_P, _I64, _P, _P, _I32, _I64, _I64, _P, _I32, _I64, _P]),
+    "grouped_gemm_bf16_wgrad": (_I32, [_P, _P, _I64, _I64, _I64, _P, _I32, _P, _P]),
     "moe_router_topk_bwd": (_I32, [_P, _P, _P, _I32, _I32, _I32, _P, _P]),
     "mxfp8_quantize": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _I64, _PMX, _PMX, _P]),
     "grouped_gemm_mxfp8": (_I32, [_PMX, _PMX, _P, _I32, _I64, _I64, _P, _I32, _I64, _P]),
@@ -254,6 +256,26 @@ def grouped_gemm_mxfp8_wgrad(At: MXFP8, Bt: MXFP8, seg_off, E, out=None):
     st = load().grouped_gemm_mxfp8_wgrad(ctypes.byref(At.as_struct()), ctypes.byref(Bt.as_struct()), _ptr(seg_off),
                                          E, _ptr(C), _stream())
     _check("grouped_gemm_mxfp8_wgrad", st)
+    return C
+
+
+def grouped_gemm_bf16(A, B, seg_off, E, N, out_dtype=torch.bfloat16, out=None):
+    """A bf16 [rows_cap, K], B bf16 [E*N, K] (or [E, N, K]) -> C [rows_cap, N]."""
+    rows, K = A.shape
+    C = out if out is not None else torch.empty((rows, N), dtype=out_dtype, device=A.device)
+    dt = DTYPE_BF16 if C.dtype == torch.bfloat16 else DTYPE_F32
+    _check("grouped_gemm_bf16", load().grouped_gemm_bf16(_ptr(A), rows, _ptr(B), _ptr(seg_off), E, N, K, _ptr(C), dt,
+                                                         C.stride(0), _stream()))
+    return C
+
+
+def grouped_gemm_bf16_wgrad(At, Bt, seg_off, E, out=None):
+    """At bf16 [N, rows_cap], Bt bf16 [K2, rows_cap] -> C fp32 [E, N, K2]."""
+    N, rows = At.shape
+    K2 = Bt.shape[0]
+    C = out if out is not None else torch.empty((E, N, K2), dtype=torch.float32, device=At.device)
+    _check("grouped_gemm_bf16_wgrad", load().grouped_gemm_bf16_wgrad(_ptr(At), _ptr(Bt), N, K2, rows, _ptr(seg_off), E,
+                                                                     _ptr(C), _stream()))
     return C
 
 

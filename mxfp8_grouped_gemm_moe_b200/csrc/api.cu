@@ -363,6 +363,64 @@ mxmoe_status grouped_gemm_mxfp8_wgrad(const mxmoe_mxfp8* At, const mxmoe_mxfp8* 
   return cuda_status(launch_gemm(g, S(stream)));
 }
 
+mxmoe_status grouped_gemm_bf16(const void* A_dev, int64_t rows_cap, const void* B_dev, const int32_t* seg_off_dev,
+                               int32_t E, int64_t N, int64_t K, void* C_dev, int32_t c_dtype, int64_t ldc,
+                               void* stream) {
+  if (!A_dev || !B_dev || !seg_off_dev || !C_dev || !aligned16(A_dev) || !aligned16(B_dev) || !aligned16(C_dev))
+    return MXMOE_ERR_INVALID_ARG;
+  if (c_dtype != MXMOE_DTYPE_BF16 && c_dtype != MXMOE_DTYPE_F32) return MXMOE_ERR_INVALID_ARG;
+  if (E < 1 || E > 256 || N <= 0 || K <= 0 || rows_cap < 0 || N % 256 != 0 || K % 64 != 0 || rows_cap % 256 != 0 ||
+      ldc < N || ldc % 8 != 0)
+    return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if (rows_cap == 0) return MXMOE_OK;
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.mode = kModeStore;
+  g.bf16_operands = 1;
+  g.E = E;
+  g.a_data = static_cast<const uint8_t*>(A_dev);
+  g.a_rows = rows_cap;
+  g.a_cols = K;
+  g.b_data = static_cast<const uint8_t*>(B_dev);
+  g.b_rows = (int64_t)E * N;
+  g.b_cols = K;
+  g.seg_off = seg_off_dev;
+  g.N = N;
+  g.K = K;
+  g.c = C_dev;
+  g.c_dtype = c_dtype;
+  g.ldc = ldc;
+  StageScope sc(MXMOE_STAGE_GEMM, S(stream));
+  return cuda_status(launch_gemm(g, S(stream)));
+}
+
+mxmoe_status grouped_gemm_bf16_wgrad(const void* At_dev, const void* Bt_dev, int64_t N, int64_t K2, int64_t rows_cap,
+                                     const int32_t* seg_off_dev, int32_t E, float* C_dev, void* stream) {
+  if (!At_dev || !Bt_dev || !seg_off_dev || !C_dev || !aligned16(At_dev) || !aligned16(Bt_dev) || !aligned16(C_dev))
+    return MXMOE_ERR_INVALID_ARG;
+  if (E < 1 || E > 256 || N <= 0 || K2 <= 0 || rows_cap <= 0 || N % 256 != 0 || K2 % 256 != 0 || rows_cap % 256 != 0)
+    return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.mode = kModeWgrad;
+  g.bf16_operands = 1;
+  g.E = E;
+  g.a_data = static_cast<const uint8_t*>(At_dev);
+  g.a_rows = N;
+  g.a_cols = rows_cap;
+  g.b_data = static_cast<const uint8_t*>(Bt_dev);
+  g.b_rows = K2;
+  g.b_cols = rows_cap;
+  g.seg_off = seg_off_dev;
+  g.N = N;
+  g.K2 = K2;
+  g.c = C_dev;
+  g.c_dtype = MXMOE_DTYPE_F32;
+  g.ldc = K2;
+  StageScope sc(MXMOE_STAGE_WGRAD, S(stream));
+  return cuda_status(launch_gemm(g, S(stream)));
+}
+
 size_t mxmoe_weights_size(int32_t E, int32_t H, int32_t F) { return weights_layout(E, H, F).total; }
 
 mxmoe_status mxmoe_weights_view(void* wq_dev, int32_t E, int32_t H, int32_t F, int32_t which, mxmoe_mxfp8* out) {

@@ -124,7 +124,9 @@ __device__ __forceinline__ int64_t total_tiles(const GemmArgs& g, const int32_t*
 }
 
 // Tile `idx` of the launch as seen by CTA `rank` of its pair (rank 0 when PAIR == 1).
-template <int MODE, int PAIR>
+// K coordinates of the tile (a_x0, b_x0, k_iters) are in bytes of the operand rows: ESZ
+// bytes per element (1 for E4M3, 2 for bf16), BK = 128 bytes per pipeline stage.
+template <int MODE, int PAIR, int ESZ = 1>
 __device__ __forceinline__ TileInfo get_tile(const GemmArgs& g, int32_t idx, const int32_t* s_seg,
                                              const int32_t* s_order, uint32_t rank) {
   constexpr int TM = Cfg<PAIR, MODE>::TM;
@@ -143,12 +145,12 @@ __device__ __forceinline__ TileInfo get_tile(const GemmArgs& g, int32_t idx, con
     const int32_t n0 = grp * GW, gn = min(GW, nn - n0);
     const int32_t n_t = n0 + rr % gn, k2_t = rr / gn;
     t.e = e;
-    t.k_iters = (s_seg[e + 1] - s_seg[e]) / BK;
+    t.k_iters = (s_seg[e + 1] - s_seg[e]) * ESZ / BK;
     t.a_y = n_t * TM + 128 * (int32_t)rank;
-    t.a_x0 = s_seg[e];
+    t.a_x0 = s_seg[e] * ESZ;
     t.b_y0 = k2_t * BN;
     t.b_y1 = t.b_y0 + 128;
-    t.b_x0 = s_seg[e];
+    t.b_x0 = s_seg[e] * ESZ;
     t.n_tile = k2_t;
     t.row0 = (int64_t)e * g.N + t.a_y;
     return t;
@@ -173,7 +175,7 @@ __device__ __forceinline__ TileInfo get_tile(const GemmArgs& g, int32_t idx, con
   }
   const int32_t e = lo;
   t.e = e;
-  t.k_iters = (int32_t)(g.K / BK);
+  t.k_iters = (int32_t)(g.K * ESZ / BK);
   t.a_y = row + 128 * (int32_t)rank;
   t.a_x0 = 0;
   t.b_x0 = 0;
@@ -327,14 +329,18 @@ __device__ __forceinline__ uint4 pack8_bf16(const uint32_t (&v)[N], int i0) {
   return o;
 }
 
-template <int MODE, int PAIR>
+// ESZ: operand element bytes -- 1: MXFP8 (E4M3 + E8M0 scales, kind::mxf8f6f4.block_scale),
+// 2: bf16 (kind::f16, no scales; plain-store and weight-gradient modes, CTA pairs only).
+template <int MODE, int PAIR, int ESZ>
 __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
     mxgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
                   const __grid_constant__ CUtensorMap tmE, const __grid_constant__ GemmArgs g) {
   using C = Cfg<PAIR, MODE>;
+  static_assert(ESZ == 1 || (PAIR == 2 && C::kTmaStore), "bf16 operands: CTA pairs, plain-store / wgrad modes");
   constexpr int STAGES = C::STAGES;
+  constexpr uint32_t kTx = ESZ == 1 ? C::kTxBytes : kABytes + C::kBBytes;  // bytes per CTA per stage
   constexpr uint32_t kStageBytes = C::kStageBytes;
   constexpr uint32_t kBBytes = C::kBBytes;
   extern __shared__ uint8_t smem_raw[];
@@ -368,7 +374,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tensormap(&tmA);
     ptx::prefetch_tensormap(&tmB);
-    if (PAIR == 2) {
+    if (PAIR == 2 && ESZ == 1) {
       ptx::prefetch_tensormap(&tmSFA);
       ptx::prefetch_tensormap(&tmSFB);
     }
@@ -430,11 +436,11 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
       uint32_t ph = 0;
       const int64_t a_kchunks = g.a_cols / 128, b_kchunks = g.b_cols / 128;
       for (int32_t tile = first; tile < ntiles && !*s_abort; tile += stride) {
-        const TileInfo t = get_tile<MODE, PAIR>(g, tile, s_seg, s_order, rank);
+        const TileInfo t = get_tile<MODE, PAIR, ESZ>(g, tile, s_seg, s_order, rank);
         if (tile + stride < ntiles) {
           // warm L2 with the first K steps of this CTA's next tile (its operands usually
           // come from HBM; the ring alone is too short to hide that at a tile change)
-          const TileInfo nt = get_tile<MODE, PAIR>(g, tile + stride, s_seg, s_order, rank);
+          const TileInfo nt = get_tile<MODE, PAIR, ESZ>(g, tile + stride, s_seg, s_order, rank);
           const int npf = min(nt.k_iters, kPrefetchSteps);
           for (int kb = 0; kb < npf; ++kb) {
             ptx::tma_prefetch_2d(&tmA, nt.a_x0 + kb * BK, nt.a_y);
@@ -465,12 +471,14 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           } else {
             // both CTAs' copies complete on the leader's barrier, which expects the pair's bytes
             const uint32_t full_leader = ptx::map_to_rank(ptx::smem_u32(&bar_full[stage]), 0);
-            if (rank == 0) ptx::mbar_arrive_expect_tx(&bar_full[stage], 2 * C::kTxBytes);
+            if (rank == 0) ptx::mbar_arrive_expect_tx(&bar_full[stage], 2 * kTx);
             ptx::tma_load_2d_pair(sb, &tmA, kx_a, t.a_y, full_leader);
             ptx::tma_load_2d_pair(sb + kABytes, &tmB, kx_b, rank ? t.b_y1 : t.b_y0, full_leader);
-            ptx::tma_load_2d_pair(s_sfa, &tmSFA, 0, (int32_t)ca, full_leader);
-            ptx::tma_load_2d_pair(s_sfa + kSfaBytes, &tmSFB, 0, (int32_t)cb0, full_leader);
-            ptx::tma_load_2d_pair(s_sfa + kSfaBytes + 512, &tmSFB, 0, (int32_t)cb1, full_leader);
+            if (ESZ == 1) {
+              ptx::tma_load_2d_pair(s_sfa, &tmSFA, 0, (int32_t)ca, full_leader);
+              ptx::tma_load_2d_pair(s_sfa + kSfaBytes, &tmSFB, 0, (int32_t)cb0, full_leader);
+              ptx::tma_load_2d_pair(s_sfa + kSfaBytes + 512, &tmSFB, 0, (int32_t)cb1, full_leader);
+            }
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -486,7 +494,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
       uint32_t ph = 0, acc_ph = 0;
       bool dropped = false;
       for (int32_t tile = first; tile < ntiles && !*s_abort; tile += stride) {
-        const TileInfo t = get_tile<MODE, PAIR>(g, tile, s_seg, s_order, 0);
+        const TileInfo t = get_tile<MODE, PAIR, ESZ>(g, tile, s_seg, s_order, 0);
         if (t.k_iters == 0) continue;
         if (!ptx::mbar_wait(bar_acc_empty, acc_ph ^ 1u, 2)) {
           *s_abort = 1;
@@ -508,21 +516,28 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           const uint64_t dsa = ptx::make_smem_desc(sfa_s, 0, 128, ptx::kLayoutSwizzleNone);
           const uint64_t dsb0 = ptx::make_smem_desc(sfa_s + kSfaBytes, 0, 128, ptx::kLayoutSwizzleNone);
           const uint64_t dsb1 = ptx::make_smem_desc(sfa_s + kSfaBytes + 512, 0, 128, ptx::kLayoutSwizzleNone);
-          if (PAIR == 1) {
-            ptx::tmem_cp_32x128b_warpx4(t_sfa, dsa);
-            ptx::tmem_cp_32x128b_warpx4(t_sfb, dsb0);
-            ptx::tmem_cp_32x128b_warpx4(t_sfb + 4, dsb1);
-          } else {
-            ptx::tmem_cp_pair_32x128b_warpx4(t_sfa, dsa);
-            ptx::tmem_cp_pair_32x128b_warpx4(t_sfb, dsb0);
-            ptx::tmem_cp_pair_32x128b_warpx4(t_sfb + 4, dsb1);
+          if (ESZ == 1) {
+            if (PAIR == 1) {
+              ptx::tmem_cp_32x128b_warpx4(t_sfa, dsa);
+              ptx::tmem_cp_32x128b_warpx4(t_sfb, dsb0);
+              ptx::tmem_cp_32x128b_warpx4(t_sfb + 4, dsb1);
+            } else {
+              ptx::tmem_cp_pair_32x128b_warpx4(t_sfa, dsa);
+              ptx::tmem_cp_pair_32x128b_warpx4(t_sfb, dsb0);
+              ptx::tmem_cp_pair_32x128b_warpx4(t_sfb + 4, dsb1);
+            }
           }
           const uint64_t adesc = ptx::make_smem_desc(sbase, 16, 1024, ptx::kLayoutSwizzle128B);
           const uint64_t bdesc = ptx::make_smem_desc(sbase + kABytes, 16, 1024, ptx::kLayoutSwizzle128B);
 #pragma unroll
-          for (int kk = 0; kk < BK / 32; ++kk) {
-            const uint32_t idesc = ptx::make_idesc_mxf8(C::TM, BN, (uint32_t)kk, (uint32_t)kk);
+          for (int kk = 0; kk < BK / 32; ++kk) {  // 32 bytes of K per MMA (32 E4M3 or 16 bf16)
             const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            if (ESZ == 2) {
+              ptx::mma_bf16_pair(tmem_base, adesc + (uint64_t)(2 * kk), bdesc + (uint64_t)(2 * kk),
+                                 ptx::make_idesc_bf16(C::TM, BN), acc);
+              continue;
+            }
+            const uint32_t idesc = ptx::make_idesc_mxf8(C::TM, BN, (uint32_t)kk, (uint32_t)kk);
             if (PAIR == 1)
               ptx::mma_mxf8(tmem_base, adesc + (uint64_t)(2 * kk), bdesc + (uint64_t)(2 * kk), idesc, t_sfa, t_sfb,
                             acc);
@@ -568,7 +583,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
     for (int32_t tile = first; tile < ntiles; tile += stride) {
       // warp-uniform abort check (the TMEM loads below are warp-collective)
       if (__any_sync(0xffffffffu, *s_abort != 0)) break;
-      const TileInfo t = get_tile<MODE, PAIR>(g, tile, s_seg, s_order, rank);
+      const TileInfo t = get_tile<MODE, PAIR, ESZ>(g, tile, s_seg, s_order, rank);
       const int64_t mrow0 = t.row0 + 32 * q;  // first row of this warp's 32-row block
       const int64_t row = mrow0 + lane;
       const bool have_acc = t.k_iters > 0;
@@ -872,21 +887,21 @@ struct GemmMaps {
   CUtensorMap c, d, e;  // epilogue outputs (unused ones zeroed)
 };
 
-template <int MODE, int PAIR>
+template <int MODE, int PAIR, int ESZ = 1>
 static cudaError_t launch_mode(const GemmMaps& m, const GemmArgs& g, int64_t tiles_ub, cudaStream_t st) {
   constexpr uint32_t smem = Cfg<PAIR, MODE>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(mxgemm_kernel<MODE, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(mxgemm_kernel<MODE, PAIR, ESZ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   // the warpgroup register split assumes the launch allocation it was sized for
   cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, mxgemm_kernel<MODE, PAIR>);
+  e = cudaFuncGetAttributes(&fa, mxgemm_kernel<MODE, PAIR, ESZ>);
   if (e != cudaSuccess) return e;
   if (Cfg<PAIR, MODE>::kSplitRegs && fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
   const int units = gemm_num_sms() / PAIR;  // SMs, or SM pairs
   const int n = (int)(tiles_ub < units ? (tiles_ub > 0 ? tiles_ub : 1) : units);
-  if (PAIR == 1) {
-    mxgemm_kernel<MODE, 1><<<n, Cfg<PAIR, MODE>::kThreads, smem, st>>>(m.a, m.b, m.sfa, m.sfb, m.c, m.d, m.e, g);
+  if constexpr (PAIR == 1) {
+    mxgemm_kernel<MODE, 1, ESZ><<<n, Cfg<PAIR, MODE>::kThreads, smem, st>>>(m.a, m.b, m.sfa, m.sfb, m.c, m.d, m.e, g);
   } else {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * n, 1, 1);
@@ -900,7 +915,7 @@ static cudaError_t launch_mode(const GemmMaps& m, const GemmArgs& g, int64_t til
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, mxgemm_kernel<MODE, PAIR>, m.a, m.b, m.sfa, m.sfb, m.c, m.d, m.e, g);
+    e = cudaLaunchKernelEx(&cfg, mxgemm_kernel<MODE, PAIR, ESZ>, m.a, m.b, m.sfa, m.sfb, m.c, m.d, m.e, g);
     if (e != cudaSuccess) return e;
   }
   ++g_launch_count;
@@ -939,7 +954,26 @@ static cudaError_t launch_variant(const GemmArgs& g, cudaStream_t st) {
   return cudaErrorInvalidValue;
 }
 
+// bf16 operands (plain-store and weight-gradient modes, CTA pairs): no scale arrays; the
+// operand maps cover the rows' bytes.
+static cudaError_t launch_bf16(const GemmArgs& g, cudaStream_t st) {
+  GemmMaps m;
+  std::memset(&m, 0, sizeof(m));
+  if (!make_map(&m.a, g.a_data, g.a_rows, g.a_cols * 2) || !make_map(&m.b, g.b_data, g.b_rows, g.b_cols * 2))
+    return cudaErrorInvalidValue;
+  switch (g.mode) {
+    case kModeStore:
+      if (!make_out_map(&m.c, g.c, g.a_rows, g.N, g.ldc, g.c_dtype == MXMOE_DTYPE_F32)) return cudaErrorInvalidValue;
+      return launch_mode<kModeStore, 2, 2>(m, g, (g.a_rows / 256) * (g.N / BN), st);
+    case kModeWgrad:
+      if (!make_out_map(&m.c, g.c, (int64_t)g.E * g.N, g.K2, g.K2, true)) return cudaErrorInvalidValue;
+      return launch_mode<kModeWgrad, 2, 2>(m, g, (int64_t)g.E * (g.N / 256) * (g.K2 / BN), st);
+  }
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
+  if (g.bf16_operands) return launch_bf16(g, st);
   return gemm_tile_rows() == 128 ? launch_variant<1>(g, st) : launch_variant<2>(g, st);
 }
 

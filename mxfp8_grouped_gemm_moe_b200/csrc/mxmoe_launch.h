@@ -59,7 +59,8 @@ enum GemmMode : int32_t {
 struct GemmArgs {
   int32_t mode;
   int32_t E;
-  // operands (MMA scale layout)
+  int32_t bf16_operands;  // 0: MXFP8 E4M3 operands with E8M0 scales; 1: bf16 operands, no scales
+  // operands (MMA scale layout); a_cols / b_cols count elements
   const uint8_t* a_data;
   const uint8_t* a_sf;
   int64_t a_rows, a_cols;

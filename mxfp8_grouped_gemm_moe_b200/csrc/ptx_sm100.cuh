@@ -294,6 +294,16 @@ __device__ __forceinline__ void mma_mxf8_pair(uint32_t d_tmem, uint64_t a_desc, 
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
+// Dense MMA with bf16 A and B (kind::f16), fp32 accumulate, no scale factors.
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Each CTA of the pair copies its own shared-memory matrix into its own TMEM.
 __device__ __forceinline__ void tmem_cp_pair_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
@@ -331,6 +341,13 @@ constexpr uint32_t kLayoutSwizzle128B = 2;
 __host__ __device__ constexpr uint32_t make_idesc_mxf8(uint32_t M, uint32_t N, uint32_t sfa_id, uint32_t sfb_id) {
   return ((sfb_id & 3u) << 4) | (0u << 7) /*A E4M3*/ | (0u << 10) /*B E4M3*/ | ((N >> 3) << 17) |
          (1u << 23) /*E8M0 scales*/ | ((M >> 4) << 24) | ((sfa_id & 3u) << 29);
+}
+
+// Instruction descriptor for kind::f16: A and B bf16 (both the same type), K-major,
+// fp32 accumulate.
+__host__ __device__ constexpr uint32_t make_idesc_bf16(uint32_t M, uint32_t N) {
+  return (1u << 4) /*F32 accumulate*/ | (1u << 7) /*A BF16*/ | (1u << 10) /*B BF16*/ | ((N >> 3) << 17) |
+         ((M >> 4) << 24);
 }
 
 }  // namespace ptx
