@@ -58,7 +58,7 @@ def parse_args():
     p.add_argument("--cpu-rows", type=int, default=512, help="routed rows in the CPU oracle sample")
     p.add_argument("--cpu-fslice", type=int, default=1024, help="FFN columns in the CPU oracle sample")
     p.add_argument("--no-bf16-compare", action="store_true",
-                   help="skip timing the six GEMM stages on bf16 operands (same scheduler) for comparison")
+                   help="skip timing the same step on the bf16 layer for comparison")
     return p.parse_args()
 
 
@@ -268,61 +268,65 @@ def config_json(cfg, world):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def time_bf16_gemms(cfg, layer, stream, g, dev, stage_json_ms=None, iters=5):
-    """Each GEMM stage of the layer on bf16 operands with the layer's own routing (expert
-    segments of the saved forward): fc1 / fc2 / fc2 dgrad / fc1 dgrad as plain grouped
-    GEMMs (bf16 out), the two weight gradients as grouped wgrad GEMMs (fp32 out)."""
+def layer_memory(cfg):
+    """Device bytes of the layer's buffers, MXFP8 vs bf16: prepared weights, activations
+    saved by the forward for the backward, and scratch."""
+    import mxfp8_grouped_gemm_moe_b200 as mx
+    lib = mx.load()
+    a = (cfg.T, cfg.k, cfg.E, cfg.H, cfg.F)
+    return {"mxfp8": {"weights": lib.mxmoe_weights_size(cfg.E, cfg.H, cfg.F),
+                      "saved": lib.grouped_mlp_saved_size(*a), "workspace": lib.grouped_mlp_workspace_size(*a)},
+            "bf16": {"weights": lib.mxmoe_weights_bf16_size(cfg.E, cfg.H, cfg.F),
+                     "saved": lib.grouped_mlp_bf16_saved_size(*a),
+                     "workspace": lib.grouped_mlp_bf16_workspace_size(*a)}}
+
+
+def time_bf16_layer(cfg, W1, W2, x, idx, probs, dy, stream, dev, steps):
+    """The same fused forward + backward on the bf16 layer (grouped_mlp_bf16_*: bf16 copies
+    instead of quantisers, kind::f16 GEMMs, bf16 Z / dGU from the fused epilogues), weights
+    prepared every step as in the MXFP8 step: the 16-bit comparison point."""
     import torch
 
     import mxfp8_grouped_gemm_moe_b200 as mx
-    E, H, F, cap = cfg.E, cfg.H, cfg.F, layer.cap
-    seg = layer.saved_field("seg_off", torch.int32, E + 1)
-    r = lambda *sh: (torch.randn(sh, generator=g, device=dev) * 0.05).to(torch.bfloat16)  # noqa: E731
-    ms = {}
+    layer = mx.GroupedMLP(cfg.T, cfg.k, cfg.E, cfg.H, cfg.F, device=dev, precision="bf16")
+    y = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
+    dx = torch.empty_like(y)
+    dW1 = torch.empty((cfg.E, 2 * cfg.F, cfg.H), dtype=torch.float32, device=dev)
+    dW2 = torch.empty((cfg.E, cfg.H, cfg.F), dtype=torch.float32, device=dev)
+    dprobs = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=dev)
+
+    def step():
+        layer.quantize_weights(W1, W2)
+        layer.forward(x, idx, probs, y)
+        layer.backward(dy, dx, dW1, dW2, dprobs)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    mx.mxmoe_profile_enable(64 * (steps + 1))
+    mx.mxmoe_profile_read()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-
-    def timeit(name, fn):
-        for _ in range(2):
-            fn()
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(iters):
-            fn()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        ms[name] = e0.elapsed_time(e1) / iters
-
-    xa, w1 = r(cap, H), r(E * 2 * F, H)
-    out = torch.empty((cap, 2 * F), dtype=torch.bfloat16, device=dev)
-    timeit("fc1_swiglu", lambda: mx.grouped_gemm_bf16(xa, w1, seg, E, 2 * F, out=out))
-    del out
-    za, w2 = r(cap, F), r(E * H, F)
-    out = torch.empty((cap, H), dtype=torch.bfloat16, device=dev)
-    timeit("fc2", lambda: mx.grouped_gemm_bf16(za, w2, seg, E, H, out=out))
-    del w2
-    dya, w2t = r(cap, H), r(E * F, H)
-    out2 = torch.empty((cap, F), dtype=torch.bfloat16, device=dev)
-    timeit("fc2_dgrad_swiglu_bwd", lambda: mx.grouped_gemm_bf16(dya, w2t, seg, E, F, out=out2))
-    del w2t, out2
-    dyt, zt = dya.t().contiguous(), za.t().contiguous()
-    del dya, za
-    dw2 = torch.empty((E, H, F), dtype=torch.float32, device=dev)
-    timeit("fc2_wgrad", lambda: mx.grouped_gemm_bf16_wgrad(dyt, zt, seg, E, out=dw2))
-    del dyt, zt, dw2, w1
-    dgu, w1t = r(cap, 2 * F), r(E * H, 2 * F)
-    timeit("fc1_dgrad", lambda: mx.grouped_gemm_bf16(dgu, w1t, seg, E, H, out=out))
-    del w1t, out
-    dgut, xt = dgu.t().contiguous(), xa.t().contiguous()
-    del dgu, xa
-    dw1 = torch.empty((E, 2 * F, H), dtype=torch.float32, device=dev)
-    timeit("fc1_wgrad", lambda: mx.grouped_gemm_bf16_wgrad(dgut, xt, seg, E, out=dw1))
-    del dgut, xt, dw1
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    stages = mx.mxmoe_profile_read()
+    mx.mxmoe_profile_disable()
+    ms = e0.elapsed_time(e1) / steps
+    per = {}
+    for name, t in stages:
+        per.setdefault(name, []).append(t)
+    MHF = float(cfg.M) * cfg.H * cfg.F
+    st_ms = {n: sum(v) / len(v) for n, v in per.items()}
+    out = {"ms_per_step": ms, "tflops": cfg.fwdbwd_flops / (ms * 1e-3) / 1e12, "stages_ms": st_ms,
+           "gemm_tflops": {n: GEMM_FLOP_FACTOR[n] * MHF / (t * 1e-3) / 1e12
+                           for n, t in st_ms.items() if n in GEMM_FLOP_FACTOR},
+           "note": "bf16 layer (grouped_mlp_bf16_fwd/bwd), same step as the headline; quant_* stages are "
+                   "bf16 row + transposed copies here"}
+    del layer, y, dx, dW1, dW2, dprobs
     torch.cuda.empty_cache()
-    MHF = float(cfg.M) * H * F
-    return {"ms": ms, "total_ms": sum(ms.values()),
-            "tflops": {n: GEMM_FLOP_FACTOR[n] * MHF / (t * 1e-3) / 1e12 for n, t in ms.items()},
-            "note": "bf16 operands on the same grouped scheduler (kind::f16, CTA pairs), plain outputs; compare "
-                    "with the MXFP8 stage times of the same run"}
+    return out
 
 
 def run_gpu(args, cfg, dist, rank, world, local_rank):
@@ -383,11 +387,10 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
     mx.mxmoe_profile_disable()
     ms = max_over_ranks(dist, ms)
 
-    # ---- the six GEMM stages on bf16 operands (same scheduler, CTA-pair tiles, kind::f16):
-    # the 16-bit comparison point, timed on its own (plain outputs, no fused epilogues)
-    bf16_gemms = None
+    # ---- the same step on the bf16 layer: the 16-bit comparison point, timed on its own
+    bf16_layer = None
     if rank == 0 and world == 1 and not args.no_bf16_compare:
-        bf16_gemms = time_bf16_gemms(cfg, layer, stream, g, dev, stage_json_ms=None)
+        bf16_layer = time_bf16_layer(cfg, W1, W2, x, idx, probs, dy, stream, dev, min(args.steps, 5))
 
     # ---- router (the step upstream of the layer; timed on its own, not part of `value`)
     router = None
@@ -553,12 +556,10 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
             "gemm_frac_of_measured_fp8": (18.0 * MHF) / (gemm_ms * 1e-3) / 1e12 / fp8_peak,
             "roofline": roofline, "roofline_hbm": roofline_hbm, "stages": stage_json,
             "gpu_launches": launches, "e2e": e2e, "clocks": clk, "router": router}
-    if bf16_gemms is not None:
-        mx_ms = {n: stage_json[n]["ms"] for n in GEMM_FLOP_FACTOR}
-        bf16_gemms["mxfp8_ms"] = mx_ms
-        bf16_gemms["mxfp8_total_ms"] = sum(mx_ms.values())
-        bf16_gemms["speedup_mxfp8_over_bf16"] = bf16_gemms["total_ms"] / bf16_gemms["mxfp8_total_ms"]
-        line["bf16_gemms"] = bf16_gemms
+    if bf16_layer is not None:
+        bf16_layer["speedup_mxfp8_over_bf16"] = bf16_layer["ms_per_step"] / ms
+        bf16_layer["memory_bytes"] = layer_memory(cfg)
+        line["bf16_layer"] = bf16_layer
     return line
 
 

@@ -346,6 +346,38 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
                              float* dW1_dev, float* dW2_dev, float* dprobs_dev, void* ws_dev, size_t ws_bytes,
                              void* stream);
 
+/* ------------------------------------------------------------------ bf16 grouped MLP */
+
+/*
+ * The same expert MLP in bf16: the 16-bit comparison point the pages set MXFP8 against
+ * ("MoE-Training für biologische Grundmodelle optimieren", MXFP8 passage: MXFP8 halves the
+ * bits of the 16-bit operands). Every step of grouped_mlp_fwd / grouped_mlp_bwd runs with
+ * the quantisers replaced by bf16 copies (the permuted rows and their transposes) and the
+ * GEMMs on tcgen05 kind::f16 with fp32 accumulation; the fused epilogues write Z and dGU
+ * in bf16. Same argument meaning, limits and error behaviour as the MXFP8 layer.
+ *
+ * Weights: one opaque device buffer of mxmoe_weights_bf16_size(E, H, F) bytes holding
+ *   W1 rows [E*2F, H] (gate / up interleaved in 64-row blocks, as the MXFP8 copy),
+ *   W1^T [E*H, 2F], W2 rows [E*H, F], W2^T [E*F, H], all bf16,
+ * written by mxmoe_weights_bf16_prepare from W1_dev bf16 [E, 2F, H], W2_dev bf16 [E, H, F].
+ * Saved activations: grouped_mlp_bf16_saved_size bytes (routing maps, the transposed
+ * permuted input [H, cap] and Z^T [F, cap], gate/up pre-activations [cap, 2F], bf16).
+ * Scratch: grouped_mlp_bf16_workspace_size bytes for either call.
+ */
+size_t mxmoe_weights_bf16_size(int32_t E, int32_t H, int32_t F);
+mxmoe_status mxmoe_weights_bf16_prepare(const void* W1_dev, const void* W2_dev, int32_t E, int32_t H, int32_t F,
+                                        void* wb_dev, size_t wb_bytes, void* stream);
+size_t grouped_mlp_bf16_saved_size(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F);
+size_t grouped_mlp_bf16_workspace_size(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F);
+mxmoe_status grouped_mlp_bf16_fwd(const void* x_dev, const int32_t* topk_idx_dev, const float* probs_dev,
+                                  const void* wb_dev, size_t wb_bytes, int32_t T, int32_t k, int32_t E, int32_t H,
+                                  int32_t F, void* y_dev, void* saved_dev, size_t saved_bytes, void* ws_dev,
+                                  size_t ws_bytes, void* stream);
+mxmoe_status grouped_mlp_bf16_bwd(const void* dy_dev, const void* saved_dev, size_t saved_bytes, const void* wb_dev,
+                                  size_t wb_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
+                                  void* dx_dev, float* dW1_dev, float* dW2_dev, float* dprobs_dev, void* ws_dev,
+                                  size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------ instrumentation */
 
 /* Stage tags reported by mxmoe_profile_read (one per enqueued stage). */

@@ -73,6 +73,13 @@ _SIGNATURES = {
     "grouped_mlp_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32]),
     "grouped_mlp_fwd": (_I32, [_P, _P, _P, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _P, _P, _SZ, _P, _SZ, _P]),
     "grouped_mlp_bwd": (_I32, [_P, _P, _SZ, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
+    "mxmoe_weights_bf16_size": (_SZ, [_I32, _I32, _I32]),
+    "mxmoe_weights_bf16_prepare": (_I32, [_P, _P, _I32, _I32, _I32, _P, _SZ, _P]),
+    "grouped_mlp_bf16_saved_size": (_SZ, [_I32, _I32, _I32, _I32, _I32]),
+    "grouped_mlp_bf16_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32]),
+    "grouped_mlp_bf16_fwd": (_I32, [_P, _P, _P, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _P, _P, _SZ, _P, _SZ, _P]),
+    "grouped_mlp_bf16_bwd": (_I32, [_P, _P, _SZ, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ,
+                                    _P]),
     "mxmoe_profile_enable": (_I32, [_I32]),
     "mxmoe_profile_disable": (_I32, []),
     "mxmoe_profile_read": (_I32, [ctypes.POINTER(_I32), ctypes.POINTER(ctypes.c_float), _I32]),
@@ -301,33 +308,63 @@ def mxmoe_weights_view(wq, E, H, F, which):
 
 
 class GroupedMLP:
-    """Buffers for one layer shape; forward/backward call the fused C entry points."""
+    """Buffers for one layer shape; forward/backward call the fused C entry points.
 
-    def __init__(self, T, k, E, H, F, device="cuda"):
+    precision "mxfp8" (default) runs the MXFP8 layer (grouped_mlp_fwd / _bwd); "bf16" runs
+    the same steps on bf16 operands (grouped_mlp_bf16_fwd / _bwd)."""
+
+    def __init__(self, T, k, E, H, F, device="cuda", precision="mxfp8"):
+        if precision not in ("mxfp8", "bf16"):
+            raise ValueError(f"unknown precision {precision!r}")
         lib = load()
         self.T, self.k, self.E, self.H, self.F = T, k, E, H, F
+        self.precision = precision
         self.cap = mxmoe_rows_capacity(T, k, E)
-        self.saved = torch.empty(lib.grouped_mlp_saved_size(T, k, E, H, F), dtype=torch.uint8, device=device)
-        self.ws = torch.empty(lib.grouped_mlp_workspace_size(T, k, E, H, F), dtype=torch.uint8, device=device)
-        self.wq = torch.empty(lib.mxmoe_weights_size(E, H, F), dtype=torch.uint8, device=device)
+        b16 = precision == "bf16"
+        saved = (lib.grouped_mlp_bf16_saved_size if b16 else lib.grouped_mlp_saved_size)(T, k, E, H, F)
+        ws = (lib.grouped_mlp_bf16_workspace_size if b16 else lib.grouped_mlp_workspace_size)(T, k, E, H, F)
+        wsz = (lib.mxmoe_weights_bf16_size if b16 else lib.mxmoe_weights_size)(E, H, F)
+        if saved == 0 or ws == 0:
+            raise MxmoeError("grouped_mlp sizes", 2)
+        self.saved = torch.empty(saved, dtype=torch.uint8, device=device)
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
+        self.wq = torch.empty(wsz, dtype=torch.uint8, device=device)
 
     def quantize_weights(self, W1, W2):
+        """Prepares the weights buffer: MXFP8 copies, or bf16 row / transposed copies."""
+        if self.precision == "bf16":
+            return mxmoe_weights_bf16_prepare(W1, W2, out=self.wq)
         return mxmoe_weights_quantize(W1, W2, out=self.wq)
 
     def forward(self, x, topk_idx, probs, y=None):
-        return grouped_mlp_fwd(x, topk_idx, probs, self.wq, self.E, self.F, self.saved, self.ws, y)
+        fn = grouped_mlp_bf16_fwd if self.precision == "bf16" else grouped_mlp_fwd
+        return fn(x, topk_idx, probs, self.wq, self.E, self.F, self.saved, self.ws, y)
 
     def backward(self, dy, dx=None, dW1=None, dW2=None, dprobs=None):
-        return grouped_mlp_bwd(dy, self.saved, self.wq, self.T, self.k, self.E, self.H, self.F, self.ws,
-                               dx, dW1, dW2, dprobs)
+        fn = grouped_mlp_bf16_bwd if self.precision == "bf16" else grouped_mlp_bwd
+        return fn(dy, self.saved, self.wq, self.T, self.k, self.E, self.H, self.F, self.ws, dx, dW1, dW2, dprobs)
 
     def saved_field(self, name, dtype=torch.uint8, count=None):
-        """View of a named field of the saved buffer (inspection / tests)."""
+        """View of a named field of the saved buffer of the MXFP8 layer (inspection / tests)."""
+        if self.precision != "mxfp8":
+            raise ValueError("saved_field describes the MXFP8 layer's saved buffer")
         lib = load()
         f = SAVED_FIELDS.index(name)
         off = lib.grouped_mlp_saved_offset(f, self.T, self.k, self.E, self.H, self.F)
         esz = torch.tensor([], dtype=dtype).element_size()
         return self.saved[off:off + count * esz].view(dtype)
+
+
+def mxmoe_weights_bf16_prepare(W1, W2, out=None):
+    """bf16 W1 [E, 2F, H], W2 [E, H, F] -> the bf16 layer's weights buffer (uint8)."""
+    E, F2, H = W1.shape
+    F = F2 // 2
+    lib = load()
+    n = lib.mxmoe_weights_bf16_size(E, H, F)
+    wb = out if out is not None else torch.empty(n, dtype=torch.uint8, device=W1.device)
+    _check("mxmoe_weights_bf16_prepare",
+           lib.mxmoe_weights_bf16_prepare(_ptr(W1), _ptr(W2), E, H, F, _ptr(wb), wb.numel(), _stream()))
+    return wb
 
 
 def grouped_mlp_fwd(x, topk_idx, probs, wq, E, F, saved, ws, y=None):
@@ -349,6 +386,28 @@ def grouped_mlp_bwd(dy, saved, wq, T, k, E, H, F, ws, dx=None, dW1=None, dW2=Non
     st = load().grouped_mlp_bwd(_ptr(dy), _ptr(saved), saved.numel(), _ptr(wq), wq.numel(), T, k, E, H, F, _ptr(dx),
                                 _ptr(dW1), _ptr(dW2), _ptr(dprobs), _ptr(ws), ws.numel(), _stream())
     _check("grouped_mlp_bwd", st)
+    return dx, dW1, dW2, dprobs
+
+
+def grouped_mlp_bf16_fwd(x, topk_idx, probs, wb, E, F, saved, ws, y=None):
+    T, H = x.shape
+    k = topk_idx.shape[1]
+    y = y if y is not None else torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    st = load().grouped_mlp_bf16_fwd(_ptr(x), _ptr(topk_idx), _ptr(probs), _ptr(wb), wb.numel(), T, k, E, H, F,
+                                     _ptr(y), _ptr(saved), saved.numel(), _ptr(ws), ws.numel(), _stream())
+    _check("grouped_mlp_bf16_fwd", st)
+    return y
+
+
+def grouped_mlp_bf16_bwd(dy, saved, wb, T, k, E, H, F, ws, dx=None, dW1=None, dW2=None, dprobs=None):
+    dev = dy.device
+    dx = dx if dx is not None else torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    dW1 = dW1 if dW1 is not None else torch.empty((E, 2 * F, H), dtype=torch.float32, device=dev)
+    dW2 = dW2 if dW2 is not None else torch.empty((E, H, F), dtype=torch.float32, device=dev)
+    dprobs = dprobs if dprobs is not None else torch.empty((T, k), dtype=torch.float32, device=dev)
+    st = load().grouped_mlp_bf16_bwd(_ptr(dy), _ptr(saved), saved.numel(), _ptr(wb), wb.numel(), T, k, E, H, F,
+                                     _ptr(dx), _ptr(dW1), _ptr(dW2), _ptr(dprobs), _ptr(ws), ws.numel(), _stream())
+    _check("grouped_mlp_bf16_bwd", st)
     return dx, dW1, dW2, dprobs
 
 

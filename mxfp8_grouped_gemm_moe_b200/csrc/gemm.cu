@@ -239,8 +239,8 @@ __device__ __forceinline__ uint8_t quant32(const float (&v)[32], uint32_t (&q)[8
 // Two blocks go through the two 4 KB halves of the staging buffer together, with one
 // pair of warp syncs, so the two transposes and reductions interleave. Lane c gets the
 // 32 codes (and the scale byte) of column c of each block.
-__device__ __forceinline__ void colwise_codes2(const float (&v0)[32], const float (&v1)[32], float* stg, int lane,
-                                               uint32_t (&q0)[8], uint32_t (&q1)[8], uint8_t& sb0, uint8_t& sb1) {
+__device__ __forceinline__ void colwise_transpose2(const float (&v0)[32], const float (&v1)[32], float* stg, int lane,
+                                                   float (&w0)[32], float (&w1)[32]) {
   float* stg1 = stg + 1024;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
@@ -249,7 +249,6 @@ __device__ __forceinline__ void colwise_codes2(const float (&v0)[32], const floa
     *reinterpret_cast<float4*>(stg1 + o) = make_float4(v1[4 * j], v1[4 * j + 1], v1[4 * j + 2], v1[4 * j + 3]);
   }
   __syncwarp();
-  float w0[32], w1[32];
 #pragma unroll
   for (int r = 0; r < 32; ++r) {
     const int o = r * 32 + ((((lane >> 2) ^ (r & 7)) << 2) | (lane & 3));
@@ -257,8 +256,22 @@ __device__ __forceinline__ void colwise_codes2(const float (&v0)[32], const floa
     w1[r] = stg1[o];
   }
   __syncwarp();  // the buffer may be refilled once every lane has read its columns
+}
+__device__ __forceinline__ void colwise_codes2(const float (&v0)[32], const float (&v1)[32], float* stg, int lane,
+                                               uint32_t (&q0)[8], uint32_t (&q1)[8], uint8_t& sb0, uint8_t& sb1) {
+  float w0[32], w1[32];
+  colwise_transpose2(v0, v1, stg, lane, w0, w1);
   sb0 = quant32(w0, q0);
   sb1 = quant32(w1, q1);
+}
+// bf16 output mode: lane r's 32 values as 64 bytes of bf16 at box + r * 64 (one row of a
+// 32 x 32 bf16 box).
+__device__ __forceinline__ void put_bf16_row64(uint8_t* box, int lane, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(box + lane * 64);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    d[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                      pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
 }
 
 // Fused-epilogue output path: a warp's 32 x 32 block of E4M3 codes (lane r's 32 bytes at
@@ -338,7 +351,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
                   const __grid_constant__ CUtensorMap tmE, const __grid_constant__ GemmArgs g) {
   using C = Cfg<PAIR, MODE>;
-  static_assert(ESZ == 1 || (PAIR == 2 && C::kTmaStore), "bf16 operands: CTA pairs, plain-store / wgrad modes");
+  static_assert(ESZ == 1 || PAIR == 2, "bf16 operands run on CTA pairs");
   constexpr int STAGES = C::STAGES;
   constexpr uint32_t kTx = ESZ == 1 ? C::kTxBytes : kABytes + C::kBBytes;  // bytes per CTA per stage
   constexpr uint32_t kStageBytes = C::kStageBytes;
@@ -674,6 +687,24 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
         // MXFP8 of Z, rowwise (fc2 operand) and colwise (fc2 weight-gradient operand)
         const float(&z0)[32] = *reinterpret_cast<const float(*)[32]>(&zf[0]);
         const float(&z1)[32] = *reinterpret_cast<const float(*)[32]>(&zf[32]);
+        if (ESZ == 2) {  // bf16 Z: rows and transposed rows, no quantisation
+          float w0[32], w1[32];
+          staging_acquire(lane);
+          colwise_transpose2(z0, z1, stg, lane, w0, w1);
+          put_bf16_row64(stg8, lane, z0);
+          put_bf16_row64(stg8 + 2048, lane, z1);
+          put_bf16_row64(stg8 + 4096, lane, w0);
+          put_bf16_row64(stg8 + 6144, lane, w1);
+          staging_publish();
+          if (lane == 0) {
+            ptx::tma_store_2d(&tmC, stg8, (int32_t)f0, (int32_t)mrow0);
+            ptx::tma_store_2d(&tmC, stg8 + 2048, (int32_t)(f0 + 32), (int32_t)mrow0);
+            ptx::tma_store_2d(&tmD, stg8 + 4096, (int32_t)mrow0, (int32_t)f0);
+            ptx::tma_store_2d(&tmD, stg8 + 6144, (int32_t)mrow0, (int32_t)(f0 + 32));
+            ptx::bulk_commit_group();
+          }
+          continue;
+        }
         uint32_t r0[8], r1[8], c0[8], c1[8];
         uint8_t cs0, cs1;
         const uint32_t zsf = (uint32_t)quant32(z0, r0) | ((uint32_t)quant32(z1, r1) << 8);
@@ -762,6 +793,25 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
             vu[i] = da * sl;
           }
           const int64_t fg = f0 + 32 * c;
+          if (ESZ == 2) {  // bf16 dG / dU: rows and transposed rows, no quantisation
+            float wg[32], wu[32];
+            staging_acquire(lane);
+            colwise_transpose2(vg, vu, stg, lane, wg, wu);
+            uint8_t* stg8 = reinterpret_cast<uint8_t*>(stg);
+            put_bf16_row64(stg8, lane, vg);
+            put_bf16_row64(stg8 + 2048, lane, vu);
+            put_bf16_row64(stg8 + 4096, lane, wg);
+            put_bf16_row64(stg8 + 6144, lane, wu);
+            staging_publish();
+            if (lane == 0) {
+              ptx::tma_store_2d(&tmC, stg8, (int32_t)fg, (int32_t)mrow0);
+              ptx::tma_store_2d(&tmC, stg8 + 2048, (int32_t)(F + fg), (int32_t)mrow0);
+              ptx::tma_store_2d(&tmD, stg8 + 4096, (int32_t)mrow0, (int32_t)fg);
+              ptx::tma_store_2d(&tmD, stg8 + 6144, (int32_t)mrow0, (int32_t)(F + fg));
+              ptx::bulk_commit_group();
+            }
+            continue;
+          }
           uint32_t rg[8], ru[8], cg[8], cu[8];
           uint8_t csg, csu;
           sfg |= (uint32_t)quant32(vg, rg) << (8 * c);
@@ -785,9 +835,11 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           g.dgu_colT_sf[sf_offset(MXMOE_SCALE_MMA, F2, g.rows_cap, F + fg + lane, mrow0 / 32)] = csu;
         }
         // row scales: blocks f0/32 .. +3 (and their up-half twins) are one aligned word each
-        *reinterpret_cast<uint32_t*>(g.dgu_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F2, row, f0 / 32)) = sfg;
-        *reinterpret_cast<uint32_t*>(g.dgu_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F2, row, (F + f0) / 32)) =
-            sfu;
+        if (ESZ == 1) {
+          *reinterpret_cast<uint32_t*>(g.dgu_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F2, row, f0 / 32)) = sfg;
+          *reinterpret_cast<uint32_t*>(g.dgu_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F2, row, (F + f0) / 32)) =
+              sfu;
+        }
         g.dprob_part[row * (F / 128) + t.n_tile * 2 + h] = dprob;
       }
     }
@@ -882,6 +934,20 @@ static bool make_codes32_map(CUtensorMap* m, void* base, int64_t rows, int64_t c
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Map over a [rows, cols] bf16 matrix for the bf16 fused epilogues: box 32 x 32 elements
+// (64-byte rows), no swizzle.
+static bool make_bf16_box_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct GemmMaps {
   CUtensorMap a, b, sfa, sfb;
   CUtensorMap c, d, e;  // epilogue outputs (unused ones zeroed)
@@ -954,8 +1020,8 @@ static cudaError_t launch_variant(const GemmArgs& g, cudaStream_t st) {
   return cudaErrorInvalidValue;
 }
 
-// bf16 operands (plain-store and weight-gradient modes, CTA pairs): no scale arrays; the
-// operand maps cover the rows' bytes.
+// bf16 operands (CTA pairs): no scale arrays; the operand maps cover the rows' bytes; the
+// fused modes write bf16 rows and transposed rows instead of MXFP8 codes.
 static cudaError_t launch_bf16(const GemmArgs& g, cudaStream_t st) {
   GemmMaps m;
   std::memset(&m, 0, sizeof(m));
@@ -968,6 +1034,16 @@ static cudaError_t launch_bf16(const GemmArgs& g, cudaStream_t st) {
     case kModeWgrad:
       if (!make_out_map(&m.c, g.c, (int64_t)g.E * g.N, g.K2, g.K2, true)) return cudaErrorInvalidValue;
       return launch_mode<kModeWgrad, 2, 2>(m, g, (int64_t)g.E * (g.N / 256) * (g.K2 / BN), st);
+    case kModeSwigluFwd:
+      if (!make_bf16_box_map(&m.c, g.z_row, g.rows_cap, g.F) || !make_bf16_box_map(&m.d, g.z_colT, g.F, g.rows_cap) ||
+          !make_out_map(&m.e, g.gu, g.rows_cap, 2 * g.F, 2 * g.F, false))
+        return cudaErrorInvalidValue;
+      return launch_mode<kModeSwigluFwd, 2, 2>(m, g, (g.a_rows / 256) * (g.F / 128), st);
+    case kModeSwigluBwd:
+      if (!make_bf16_box_map(&m.c, g.dgu_row, g.rows_cap, 2 * g.F) ||
+          !make_bf16_box_map(&m.d, g.dgu_colT, 2 * g.F, g.rows_cap))
+        return cudaErrorInvalidValue;
+      return launch_mode<kModeSwigluBwd, 2, 2>(m, g, (g.a_rows / 256) * (g.F / BN), st);
   }
   return cudaErrorInvalidValue;
 }

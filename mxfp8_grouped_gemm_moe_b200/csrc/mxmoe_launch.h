@@ -47,6 +47,10 @@ struct QuantArgs {
   int64_t row_ilv;
 };
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
+// bf16 -> bf16 copies with the same row gather / valid-row count / gate-up interleave as
+// launch_quantize: row_data receives the (permuted) rows, col_data the transposed matrix
+// [batch*cols, out_rows]; the scale fields are ignored. bf16 sources only.
+cudaError_t launch_bf16_copy(const QuantArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------- grouped GEMM
 enum GemmMode : int32_t {

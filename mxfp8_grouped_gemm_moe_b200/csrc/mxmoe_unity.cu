@@ -6,3 +6,4 @@
 #include "quantize.cu"
 #include "gemm.cu"
 #include "api.cu"
+#include "api_bf16.cu"

@@ -399,6 +399,102 @@ __global__ void __launch_bounds__(kQThreads, 2)
   if (threadIdx.x == 0) ptx::bulk_wait_group<0>();
 }
 
+// ----------------------------------------------------------------------------- bf16 operand copies
+// Operands of the bf16 grouped MLP: the same tiles, gather and interleave as the
+// quantiser, but the outputs are plain bf16 -- the (permuted) rows and the transposed
+// matrix (K-major operand of the weight-gradient GEMMs).
+__global__ void __launch_bounds__(kQThreads, 4) bf16_copy_kernel(QuantArgs a) {
+  using T = __nv_bfloat16;
+  using Tr = SrcTraits<T>;
+  extern __shared__ __align__(16) uint8_t q_smem_raw[];
+  T* tile = reinterpret_cast<T*>(q_smem_raw);
+  const int64_t c0 = (int64_t)blockIdx.x * kQTile;
+  const int64_t r0 = (int64_t)blockIdx.y * kQTile;
+  const int64_t b = blockIdx.z;
+  int64_t nvalid = a.out_rows;
+  if (a.nrows) {
+    const int64_t nv = *a.nrows;
+    nvalid = nv < nvalid ? nv : nvalid;
+  }
+  if (r0 >= nvalid) return;
+  const T* src = reinterpret_cast<const T*>(a.src);
+  constexpr int VPR = kQTile / Tr::kVec;
+  constexpr int NL = kQTile * VPR / kQThreads;
+  constexpr int RSTEP = kQThreads / VPR;
+  const int row_t = threadIdx.x / VPR, cv = threadIdx.x % VPR;
+  {
+    const int64_t col = c0 + (int64_t)cv * Tr::kVec;
+    uint4 buf[NL];
+#pragma unroll
+    for (int k = 0; k < NL; ++k) {
+      const int64_t orow = r0 + row_t + k * RSTEP;
+      int64_t srow = -1;
+      if (orow < nvalid && col < a.cols) srow = a.gather ? (int64_t)__ldg(a.gather + orow) : b * a.rows + orow;
+      buf[k] = srow >= 0 ? __ldg(reinterpret_cast<const uint4*>(src + srow * a.cols + col)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int k = 0; k < NL; ++k)
+      *reinterpret_cast<uint4*>(tile + tile_off<T>(row_t + k * RSTEP, cv * Tr::kVec)) = buf[k];
+  }
+  __syncthreads();
+  uint16_t* rout = reinterpret_cast<uint16_t*>(a.row_data);
+  uint16_t* cout = reinterpret_cast<uint16_t*>(a.col_data);
+  if (rout) {
+#pragma unroll 1
+    for (int it = threadIdx.x; it < kQTile * 4; it += kQThreads) {
+      const int row = it >> 2, blk = it & 3;
+      const int64_t orow = r0 + row, col = c0 + 32 * blk;
+      if (orow >= nvalid || col >= a.cols) continue;
+      int64_t drow = orow;
+      if (a.row_ilv > 0) {
+        const int64_t hf = orow >= a.row_ilv, rr = orow - hf * a.row_ilv;
+        drow = (rr >> 6) * 128 + hf * 64 + (rr & 63);
+      }
+      const uint4* sp = reinterpret_cast<const uint4*>(tile + tile_off<T>(row, 32 * blk));
+      uint4* dp = reinterpret_cast<uint4*>(rout + (b * a.out_rows + drow) * a.cols + col);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dp[i] = sp[i];
+    }
+  }
+  if (cout) {
+    // a thread transposes a pair of adjacent columns over 32 rows
+    const int pcol = threadIdx.x & 63, rb = threadIdx.x >> 6;
+    const int64_t col = c0 + 2 * pcol, orow = r0 + 32 * rb;
+    if (orow < nvalid && col < a.cols) {
+      uint32_t w[32];
+      const T* p = tile + tile_off<T>(32 * rb, 2 * pcol);
+#pragma unroll
+      for (int r = 0; r < 32; ++r) w[r] = *reinterpret_cast<const uint32_t*>(p + r * 4 * Tr::kBS);
+      uint32_t lo[16], hi[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        lo[j] = __byte_perm(w[2 * j], w[2 * j + 1], 0x5410);  // column col, rows 2j, 2j+1
+        hi[j] = __byte_perm(w[2 * j], w[2 * j + 1], 0x7632);  // column col + 1
+      }
+      uint4* d0 = reinterpret_cast<uint4*>(cout + (b * a.cols + col) * a.out_rows + orow);
+      uint4* d1 = reinterpret_cast<uint4*>(cout + (b * a.cols + col + 1) * a.out_rows + orow);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        d0[i] = make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]);
+        d1[i] = make_uint4(hi[4 * i], hi[4 * i + 1], hi[4 * i + 2], hi[4 * i + 3]);
+      }
+    }
+  }
+}
+
+cudaError_t launch_bf16_copy(const QuantArgs& a, cudaStream_t st) {
+  if (a.src_dtype != MXMOE_DTYPE_BF16) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)kQTile * 4 * SrcTraits<__nv_bfloat16>::kBS * sizeof(__nv_bfloat16);
+  cudaError_t e = cudaFuncSetAttribute(bf16_copy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((a.cols + kQTile - 1) / kQTile), (unsigned)((a.out_rows + kQTile - 1) / kQTile),
+            (unsigned)a.batch);
+  if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
+  bf16_copy_kernel<<<grid, kQThreads, smem, st>>>(a);
+  ++g_launch_count;
+  return cudaGetLastError();
+}
+
 static bool qt_applies(const QuantArgs& a) {
   return a.src_dtype == MXMOE_DTYPE_BF16 && !a.gather && !a.nrows && a.out_rows == a.rows && a.rows % kQTile == 0 &&
          a.cols % kQTile == 0 && a.batch * a.rows < (int64_t)1 << 31 && a.batch * a.cols < (int64_t)1 << 31 &&
