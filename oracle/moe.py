@@ -22,7 +22,9 @@ Readings where the pages are silent (each is listed in the design notes):
     projection and quantised from its fp64 value;
   * backward uses the straight-through estimator (every quantiser passes the
     gradient unchanged) and quantises dY, dGU rowwise and colwise as the consuming
-    GEMMs need; the activations saved for backward are kept in fp64 here.
+    GEMMs need; the activations saved for backward are kept in fp64 here;
+  * gradients are E4M3 like everything else; ``grad_fmt="e5m2"`` is the variant that
+    quantises dY and dGU to MXFP8 E5M2 instead (weights and activations stay E4M3).
 Every GEMM is a library matmul over dequantised fp64 operands, one expert at a time.
 """
 from __future__ import annotations
@@ -99,7 +101,7 @@ def unpermute_sum(yp, row_of_slot):
 
 # ----------------------------------------------------------------------------- MXFP8 helpers
 
-def quantize_colwise_segments(a, seg_off, m_splits):
+def quantize_colwise_segments(a, seg_off, m_splits, fmt="e4m3"):
     """Colwise MXFP8 of a permuted [Mp, C] matrix: blocks of 32 rows that start at each
     expert segment's first row (segments are 32-aligned with zero pad rows), stored
     transposed -> (codes uint8[C, Mp], scales uint8[C, Mp/32])."""
@@ -112,29 +114,29 @@ def quantize_colwise_segments(a, seg_off, m_splits):
         if s1 == s0:
             continue
         assert s0 % mxfp8.BLOCK == 0 and s1 % mxfp8.BLOCK == 0
-        c, s = mxfp8.quantize_colwise_t(a[s0:s1])
+        c, s = mxfp8.quantize_colwise_t(a[s0:s1], fmt)
         codes[:, s0:s1] = c
         scales[:, s0 // mxfp8.BLOCK:s1 // mxfp8.BLOCK] = s
     return codes, scales
 
 
-def fake_quant_colwise_segments(a, seg_off, m_splits):
-    c, s = quantize_colwise_segments(a, seg_off, m_splits)
-    return mxfp8.dequantize_rowwise(c, s).T
+def fake_quant_colwise_segments(a, seg_off, m_splits, fmt="e4m3"):
+    c, s = quantize_colwise_segments(a, seg_off, m_splits, fmt)
+    return mxfp8.dequantize_rowwise(c, s, fmt).T
 
 
-def _fq_row(a, quant):
-    return mxfp8.fake_quant_rowwise(a) if quant else np.asarray(a, dtype=np.float64)
+def _fq_row(a, quant, fmt="e4m3"):
+    return mxfp8.fake_quant_rowwise(a, fmt) if quant else np.asarray(a, dtype=np.float64)
 
 
 def _fq_col(a, quant):
     return mxfp8.fake_quant_colwise(a) if quant else np.asarray(a, dtype=np.float64)
 
 
-def _fq_col_seg(a, r, quant):
+def _fq_col_seg(a, r, quant, fmt="e4m3"):
     if not quant:
         return np.asarray(a, dtype=np.float64)
-    return fake_quant_colwise_segments(a, r["seg_off"], r["m_splits"])
+    return fake_quant_colwise_segments(a, r["seg_off"], r["m_splits"], fmt)
 
 
 # ----------------------------------------------------------------------------- grouped GEMMs
@@ -211,16 +213,17 @@ def mlp_fwd(x, topk_idx, probs, W1, W2, quant=True, align=ALIGN_ORACLE):
     return y, saved
 
 
-def mlp_bwd(dy, saved, probs, W1, W2, quant=True):
-    """Backward (straight-through estimator for every quantiser).
+def mlp_bwd(dy, saved, probs, W1, W2, quant=True, grad_fmt="e4m3"):
+    """Backward (straight-through estimator for every quantiser). grad_fmt is the MXFP8
+    element format of the gradients dY and dGU ("e4m3" or "e5m2").
     Returns dict dx fp64[T,H], dW1 fp64[E,2F,H], dW2 fp64[E,H,F], dprobs fp64[T,k]."""
     r = saved["route"]
     E, F2, H = W1.shape
     F = F2 // 2
     G, U, Z, p_row = saved["G"], saved["U"], saved["Z"], saved["p_row"]
     dYp = permute_rows(dy, r["token_of_row"])
-    dYq_row = _fq_row(dYp, quant)                         # blocks along H (fc2 dgrad)
-    dYq_col = _fq_col_seg(dYp, r, quant)                  # blocks along M (fc2 wgrad)
+    dYq_row = _fq_row(dYp, quant, grad_fmt)               # blocks along H (fc2 dgrad)
+    dYq_col = _fq_col_seg(dYp, r, quant, grad_fmt)        # blocks along M (fc2 wgrad)
     W2q_col = np.stack([_fq_col(W2[e], quant) for e in range(E)])   # [H, F], blocks along H
     # fc2 dgrad: dZ = dYp . W2  (contract over H)
     dZ = grouped_gemm(dYq_row, np.transpose(W2q_col, (0, 2, 1)), r["seg_off"])
@@ -230,8 +233,8 @@ def mlp_bwd(dy, saved, probs, W1, W2, quant=True):
     dG = dA * U * dsilu(G)
     dU = dA * silu(G)
     dGU = np.concatenate([dG, dU], axis=1)
-    dGUq_row = _fq_row(dGU, quant)                        # blocks along 2F (fc1 dgrad)
-    dGUq_col = _fq_col_seg(dGU, r, quant)                 # blocks along M (fc1 wgrad)
+    dGUq_row = _fq_row(dGU, quant, grad_fmt)              # blocks along 2F (fc1 dgrad)
+    dGUq_col = _fq_col_seg(dGU, r, quant, grad_fmt)       # blocks along M (fc1 wgrad)
     Zq_col = _fq_col_seg(Z, r, quant)
     Xq_col = _fq_col_seg(saved["Xp"], r, quant)
     # fc2 wgrad: dW2[e] = dYp_e^T . Z_e  (contract over the expert's rows)

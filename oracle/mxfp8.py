@@ -16,6 +16,12 @@ is a reading, stated where it is used:
   GEMM that consumes the tensor ("rowwise" = along columns; "colwise" = 32 rows of
   one expert segment, stored transposed).
 
+The E5M2 element format is the variant for gradients (the pages name FP8 beside MXFP8
+and fix neither element format; OCP FP8 E5M2: bias 15, 2 mantissa bits, subnormals,
+max 57344, S.11111.00 infinite, S.11111.xx with xx != 0 NaN). Its scale rule is the same
+with the format's largest exponent: X = clamp(floor(log2(amax)) - 15, -127, 127); its
+elements saturate to +-57344.
+
 The encoder is a nearest-value search over the table of finite codes; it never uses
 bit manipulation, so that it is independent of the decoder's closed form.
 """
@@ -25,6 +31,8 @@ import numpy as np
 
 E4M3_MAX = 448.0
 E4M3_EMAX = 8          # floor(log2(448))
+E5M2_MAX = 57344.0
+E5M2_EMAX = 15         # floor(log2(57344))
 SCALE_BIAS = 127
 SCALE_MIN_EXP = -127
 SCALE_MAX_EXP = 127
@@ -48,83 +56,120 @@ _POS_CODES = np.arange(0x7F, dtype=np.int64)
 _POS_VALUES = e4m3_decode(_POS_CODES)
 
 
-def e4m3_encode(x):
-    """Nearest E4M3 code to each fp64 value; ties go to the even code (mantissa LSB 0);
-    magnitudes beyond 448 saturate to 448; the sign bit follows the input's sign."""
+def _nearest_code(x, pos_codes, pos_values, vmax):
+    """Nearest code of a table of non-negative finite values (ascending) to each fp64
+    value; ties go to the even code (mantissa LSB 0); magnitudes beyond vmax saturate to
+    the largest code; the sign bit (0x80) follows the input's sign."""
     x = np.asarray(x, dtype=np.float64)
     if not np.all(np.isfinite(x)):
-        raise ValueError("e4m3_encode: non-finite input")
+        raise ValueError("fp8 encode: non-finite input")
     a = np.abs(x)
-    hi = np.searchsorted(_POS_VALUES, a, side="left")       # first value >= a
-    hi = np.minimum(hi, len(_POS_VALUES) - 1)
+    hi = np.searchsorted(pos_values, a, side="left")        # first value >= a
+    hi = np.minimum(hi, len(pos_values) - 1)
     lo = np.maximum(hi - 1, 0)
-    vlo, vhi = _POS_VALUES[lo], _POS_VALUES[hi]
+    vlo, vhi = pos_values[lo], pos_values[hi]
     dlo, dhi = a - vlo, vhi - a
-    pick_hi = (dhi < dlo) | ((dhi == dlo) & ((_POS_CODES[hi] & 1) == 0))
-    code = np.where(pick_hi, _POS_CODES[hi], _POS_CODES[lo])
-    code = np.where(a >= vhi, _POS_CODES[hi], code)          # exact hit / above table top
-    code = np.where(a >= E4M3_MAX, 0x7E, code)               # saturate
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & ((pos_codes[hi] & 1) == 0))
+    code = np.where(pick_hi, pos_codes[hi], pos_codes[lo])
+    code = np.where(a >= vhi, pos_codes[hi], code)           # exact hit / above table top
+    code = np.where(a >= vmax, pos_codes[-1], code)          # saturate
     neg = np.signbit(x)
     return (code | np.where(neg, 0x80, 0)).astype(np.uint8)
 
 
-def scale_exponent(amax):
-    """X = clamp(floor(log2(amax)) - 8, -127, 127); amax == 0 -> -127 (byte 0x00)."""
+def e4m3_encode(x):
+    """Nearest E4M3 code to each fp64 value; ties go to the even code (mantissa LSB 0);
+    magnitudes beyond 448 saturate to 448; the sign bit follows the input's sign."""
+    return _nearest_code(x, _POS_CODES, _POS_VALUES, E4M3_MAX)
+
+
+def e5m2_decode(code):
+    """Closed form of OCP E5M2: (-1)^s * 2^(e-15) * (1 + m/4), subnormal 2^-14 * m/4;
+    exponent field 31 is infinity (m == 0) or NaN."""
+    c = np.asarray(code, dtype=np.int64)
+    s = (c >> 7) & 1
+    e = (c >> 2) & 0x1F
+    m = c & 0x3
+    mag = np.where(e == 0, (m / 4.0) * 2.0 ** -14, (1.0 + m / 4.0) * np.exp2(e.astype(np.float64) - 15.0))
+    mag = np.where(e == 31, np.where(m == 0, np.inf, np.nan), mag)
+    return np.where(s == 1, -mag, mag)
+
+
+# Non-negative finite E5M2 codes 0x00..0x7B and their values, ascending.
+_POS_CODES_E5M2 = np.arange(0x7C, dtype=np.int64)
+_POS_VALUES_E5M2 = e5m2_decode(_POS_CODES_E5M2)
+
+
+def e5m2_encode(x):
+    """Nearest E5M2 code to each fp64 value; ties to the even code; magnitudes beyond
+    57344 saturate to 57344 (never infinity); the sign bit follows the input's sign."""
+    return _nearest_code(x, _POS_CODES_E5M2, _POS_VALUES_E5M2, E5M2_MAX)
+
+
+# element formats: name -> (encode, decode, largest exponent)
+FORMATS = {"e4m3": (e4m3_encode, e4m3_decode, E4M3_EMAX), "e5m2": (e5m2_encode, e5m2_decode, E5M2_EMAX)}
+
+
+def scale_exponent(amax, emax=E4M3_EMAX):
+    """X = clamp(floor(log2(amax)) - emax, -127, 127); amax == 0 -> -127 (byte 0x00).
+    emax = the element format's largest exponent (8 for E4M3, 15 for E5M2)."""
     amax = np.asarray(amax, dtype=np.float64)
     mant, ex = np.frexp(amax)            # amax = mant * 2^ex, mant in [0.5, 1)
     fl = ex.astype(np.int64) - 1         # floor(log2(amax)) for amax > 0
-    X = np.clip(fl - E4M3_EMAX, SCALE_MIN_EXP, SCALE_MAX_EXP)
+    X = np.clip(fl - emax, SCALE_MIN_EXP, SCALE_MAX_EXP)
     return np.where(amax == 0, SCALE_MIN_EXP, X).astype(np.int64)
 
 
-def quantize_blocks(v):
+def quantize_blocks(v, fmt="e4m3"):
     """Quantise ``v[..., 32]`` block by block -> (codes uint8[..., 32], scale bytes uint8[...])."""
+    encode, _, emax = FORMATS[fmt]
     v = np.asarray(v, dtype=np.float64)
     assert v.shape[-1] == BLOCK
     amax = np.max(np.abs(v), axis=-1)
-    X = scale_exponent(amax)
+    X = scale_exponent(amax, emax)
     scaled = v * np.exp2(-X.astype(np.float64))[..., None]   # exact power-of-two scaling in fp64
-    codes = e4m3_encode(scaled)
+    codes = encode(scaled)
     return codes, (X + SCALE_BIAS).astype(np.uint8)
 
 
-def dequantize_blocks(codes, scale_bytes):
+def dequantize_blocks(codes, scale_bytes, fmt="e4m3"):
     """decode(code) * 2^(scale byte - 127), exact in fp64."""
+    decode = FORMATS[fmt][1]
     X = scale_bytes.astype(np.int64) - SCALE_BIAS
-    return e4m3_decode(codes) * np.exp2(X.astype(np.float64))[..., None]
+    return decode(codes) * np.exp2(X.astype(np.float64))[..., None]
 
 
-def quantize_rowwise(a):
+def quantize_rowwise(a, fmt="e4m3"):
     """Blocks of 32 along the last axis of a 2-D matrix [R, C] (C % 32 == 0).
     Returns (codes uint8[R, C], scales uint8[R, C/32])."""
     a = np.asarray(a, dtype=np.float64)
     R, C = a.shape
     assert C % BLOCK == 0
-    codes, sc = quantize_blocks(a.reshape(R, C // BLOCK, BLOCK))
+    codes, sc = quantize_blocks(a.reshape(R, C // BLOCK, BLOCK), fmt)
     return codes.reshape(R, C), sc
 
 
-def dequantize_rowwise(codes, scales):
+def dequantize_rowwise(codes, scales, fmt="e4m3"):
     R, C = codes.shape
-    return dequantize_blocks(codes.reshape(R, C // BLOCK, BLOCK), scales).reshape(R, C)
+    return dequantize_blocks(codes.reshape(R, C // BLOCK, BLOCK), scales, fmt).reshape(R, C)
 
 
-def quantize_colwise_t(a):
+def quantize_colwise_t(a, fmt="e4m3"):
     """Blocks of 32 consecutive rows in each column of [R, C] (R % 32 == 0), stored
     transposed: (codes uint8[C, R], scales uint8[C, R/32]). The caller lays segments
     out so that no block crosses an expert boundary."""
     a = np.asarray(a, dtype=np.float64)
-    return quantize_rowwise(a.T)
+    return quantize_rowwise(a.T, fmt)
 
 
-def fake_quant_rowwise(a):
+def fake_quant_rowwise(a, fmt="e4m3"):
     """Quantise then dequantise along rows (used where the oracle needs the value a
     quantised operand stands for)."""
-    c, s = quantize_rowwise(a)
-    return dequantize_rowwise(c, s)
+    c, s = quantize_rowwise(a, fmt)
+    return dequantize_rowwise(c, s, fmt)
 
 
-def fake_quant_colwise(a):
+def fake_quant_colwise(a, fmt="e4m3"):
     """Colwise quantise/dequantise, returned in the original [R, C] orientation."""
-    c, s = quantize_colwise_t(a)
-    return dequantize_rowwise(c, s).T
+    c, s = quantize_colwise_t(a, fmt)
+    return dequantize_rowwise(c, s, fmt).T

@@ -264,3 +264,24 @@ def test_colwise_blocks_restart_at_segments():
     np.testing.assert_array_equal(s1[:, :2], s2[:, :2])
     np.testing.assert_array_equal(c1[:, :64], c2[:, :64])
     assert np.any(s1[:, 2] != s2[:, 2])
+
+
+def test_e5m2_gradients_variant():
+    """Gradients in E5M2 (one mantissa bit fewer than E4M3): the backward stays close to the
+    unquantised one, further from it than the all-E4M3 backward; the forward is unchanged
+    and only the gradient outputs move."""
+    cfg = wl.custom("e5", T=96, H=64, F=64, E=3, k=2, seed=9)
+    d = wl.make_all(cfg)
+    x, W1, W2, p = (d[n].double().numpy() for n in ("x", "W1", "W2", "probs"))
+    idx, dy = d["topk_idx"].numpy(), d["dy"].double().numpy()
+    _, sq = moe.mlp_fwd(x, idx, p, W1, W2)
+    _, su = moe.mlp_fwd(x, idx, p, W1, W2, quant=False)
+    g4 = moe.mlp_bwd(dy, sq, p, W1, W2)
+    g5 = moe.mlp_bwd(dy, sq, p, W1, W2, grad_fmt="e5m2")
+    gu = moe.mlp_bwd(dy, su, p, W1, W2, quant=False)
+    rel = lambda a, b: np.linalg.norm(a - b) / np.linalg.norm(b)  # noqa: E731
+    for n in ("dx", "dW1", "dW2"):
+        assert rel(g5[n], gu[n]) < 0.15, n
+        assert rel(g5[n], gu[n]) > rel(g4[n], gu[n]), n
+    # dZ = dYq . W2q: only dY's format changed between the two
+    assert not np.array_equal(g5["dZ"], g4["dZ"])

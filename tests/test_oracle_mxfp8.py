@@ -134,3 +134,64 @@ def test_rowwise_and_colwise_shapes():
     qb, sb = mxfp8.quantize_blocks(blk[None, :])
     np.testing.assert_array_equal(ct[5, 32:64], qb[0])
     assert st[5, 1] == sb[0]
+
+
+# ----------------------------------------------------------------------------- E5M2 (gradient variant)
+
+def _fp16_of_e5m2_code(c):
+    """E5M2 is the high byte of IEEE binary16 (same sign, 5-bit exponent with bias 15,
+    top 2 mantissa bits): an independent decoder through numpy's float16."""
+    return np.array([c << 8], dtype=np.uint16).view(np.float16).astype(np.float64)[0]
+
+
+def test_e5m2_decode_is_fp16_high_byte():
+    for c in range(256):
+        want = _fp16_of_e5m2_code(c)
+        got = float(mxfp8.e5m2_decode(c))
+        if np.isnan(want):
+            assert np.isnan(got), hex(c)
+        else:
+            assert got == want and math.copysign(1.0, got) == math.copysign(1.0, want), hex(c)
+    assert mxfp8.e5m2_decode(0x7B) == 57344.0 == mxfp8.E5M2_MAX
+    assert mxfp8.e5m2_decode(0x04) == 2.0 ** -14         # smallest normal
+    assert mxfp8.e5m2_decode(0x01) == 2.0 ** -16         # smallest subnormal
+    assert mxfp8.e5m2_decode(0x3C) == 1.0
+
+
+def test_e5m2_encode_matches_fp16_integer_rounding():
+    """For every value representable in binary16 with |v| <= 57344, the nearest-even E5M2
+    code is the fp16 bit pattern rounded to its high byte with round-half-to-even on the
+    integer bits (IEEE rounding carries across the subnormal/normal boundary)."""
+    bits = np.arange(0, 0x7C00, dtype=np.uint32)            # all finite non-negative fp16
+    v = bits.astype(np.uint16).view(np.float16).astype(np.float64)
+    keep = v <= 57344.0
+    bits, v = bits[keep], v[keep]
+    want = ((bits + 0x7F + ((bits >> 8) & 1)) >> 8).astype(np.uint8)
+    got = mxfp8.e5m2_encode(v)
+    assert np.array_equal(got, want)
+    assert np.array_equal(mxfp8.e5m2_encode(-v[1:]), want[1:] | 0x80)
+
+
+def test_e5m2_saturates_instead_of_infinity():
+    v = np.zeros(32)
+    v[0] = 65535.0                                         # amax < 2^16: X = 0
+    v[1] = 61440.0                                         # IEEE would round to infinity
+    q, s = mxfp8.quantize_blocks(v[None, :], "e5m2")
+    assert s[0] == 127 and q[0, 0] == 0x7B and q[0, 1] == 0x7B
+
+
+def test_e5m2_scale_rule_and_error_bound():
+    for a in [1e-30, 0.3, 1.0, 2.0, 57344.0, 65535.0, 1e30]:
+        want = max(-127, min(127, math.floor(math.log2(a)) - 15))
+        assert mxfp8.scale_exponent(a, mxfp8.E5M2_EMAX) == want
+    rng = np.random.default_rng(3)
+    v = rng.standard_normal((500, 32)) * np.exp2(rng.integers(-20, 20, (500, 1)))
+    q, s = mxfp8.quantize_blocks(v, "e5m2")
+    d = mxfp8.dequantize_blocks(q, s, "e5m2")
+    X = (s.astype(np.int64) - 127).astype(float)[:, None]
+    normal = (np.abs(v) >= np.exp2(X - 14.0)) & (np.abs(v) <= 57344.0 * np.exp2(X))
+    rel = np.abs(d - v)[normal] / np.abs(v)[normal]
+    assert rel.max() <= 2.0 ** -3 + 1e-15                   # half an ulp of a 2-bit mantissa
+    assert rel.max() > 2.0 ** -4                            # coarser than E4M3
+    # a block quantised to E5M2 keeps 6 more binades below its max than E4M3
+    assert np.all(np.abs(d) <= 57344.0 * np.exp2(X))
