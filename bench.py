@@ -58,7 +58,7 @@ def parse_args():
     p.add_argument("--cpu-rows", type=int, default=512, help="routed rows in the CPU oracle sample")
     p.add_argument("--cpu-fslice", type=int, default=1024, help="FFN columns in the CPU oracle sample")
     p.add_argument("--no-bf16-compare", action="store_true",
-                   help="skip timing the same step on the bf16 layer for comparison")
+                   help="skip the comparison timings (the bf16 layer's step, the E5M2-gradient backward)")
     return p.parse_args()
 
 
@@ -268,6 +268,31 @@ def config_json(cfg, world):
 
 
 # ----------------------------------------------------------------------------- GPU arm
+def time_grad_formats(cfg, layer, dy, dx, dW1, dW2, dprobs, stream, iters=5):
+    """The backward alone with E4M3 gradients (the headline) and with E5M2 gradients (the
+    variant), on the layer's saved forward; CUDA events, after two warm-up calls each."""
+    import torch
+
+    import mxfp8_grouped_gemm_moe_b200 as mx
+    out = {}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for name, fmt in (("e4m3", mx.FMT_E4M3), ("e5m2", mx.FMT_E5M2)):
+        def bwd():
+            mx.grouped_mlp_bwd(dy, layer.saved, layer.wq, cfg.T, cfg.k, cfg.E, cfg.H, cfg.F, layer.ws, dx, dW1, dW2,
+                               dprobs, grad_format=fmt)
+        for _ in range(2):
+            bwd()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(iters):
+            bwd()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out[name + "_bwd_ms"] = e0.elapsed_time(e1) / iters
+    out["note"] = "backward only (permute+quantise dY, four GEMMs, combine); gradients dY and dGU in the named format"
+    return out
+
+
 def layer_memory(cfg):
     """Device bytes of the layer's buffers, MXFP8 vs bf16: prepared weights, activations
     saved by the forward for the backward, and scratch."""
@@ -386,6 +411,11 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
     stages = mx.mxmoe_profile_read()
     mx.mxmoe_profile_disable()
     ms = max_over_ranks(dist, ms)
+
+    # ---- the backward with E5M2 gradients (the precision variant) beside the E4M3 one
+    grad_formats = None
+    if rank == 0 and world == 1 and not args.no_bf16_compare:
+        grad_formats = time_grad_formats(cfg, layer, dy, dx, dW1, dW2, dprobs, stream)
 
     # ---- the same step on the bf16 layer: the 16-bit comparison point, timed on its own
     bf16_layer = None
@@ -556,6 +586,8 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
             "gemm_frac_of_measured_fp8": (18.0 * MHF) / (gemm_ms * 1e-3) / 1e12 / fp8_peak,
             "roofline": roofline, "roofline_hbm": roofline_hbm, "stages": stage_json,
             "gpu_launches": launches, "e2e": e2e, "clocks": clk, "router": router}
+    if grad_formats is not None:
+        line["grad_formats"] = grad_formats
     if bf16_layer is not None:
         bf16_layer["speedup_mxfp8_over_bf16"] = bf16_layer["ms_per_step"] / ms
         bf16_layer["memory_bytes"] = layer_memory(cfg)

@@ -61,6 +61,10 @@ typedef int32_t mxmoe_status;
 #define MXMOE_DTYPE_BF16 0
 #define MXMOE_DTYPE_F32 1
 
+/* element formats of an mxmoe_mxfp8 matrix */
+#define MXMOE_FMT_E4M3 0 /* OCP FP8 E4M3: bias 7, max 448 (activations, weights; gradients by default) */
+#define MXMOE_FMT_E5M2 1 /* OCP FP8 E5M2: bias 15, max 57344, saturating (the gradient variant) */
+
 /* scale-factor layouts of an mxmoe_mxfp8 matrix */
 #define MXMOE_SCALE_PLAIN 0 /* row-major [rows][cols/32] */
 #define MXMOE_SCALE_MMA 1   /* rows, cols multiples of 128: [rows/128][cols/128] chunks of 512 bytes;
@@ -68,11 +72,13 @@ typedef int32_t mxmoe_status;
                                (r%32)*16 + ((r/32)%4)*4 + kb%4 -- the tensor cores' scale-factor order */
 
 /*
- * One MXFP8 matrix: `rows` x `cols` E4M3 codes, row-major (row stride `cols` bytes),
- * quantised in blocks of 32 consecutive elements along each row, plus rows*cols/32
- * E8M0 scale bytes laid out as `scale_layout` says. A "colwise" quantisation of a
- * source matrix S [R, C] (blocks of 32 consecutive rows of S) is stored transposed:
- * rows = C, cols = R. Both pointers are device memory owned by the caller.
+ * One MXFP8 matrix: `rows` x `cols` FP8 codes of `elem_format`, row-major (row stride
+ * `cols` bytes), quantised in blocks of 32 consecutive elements along each row, plus
+ * rows*cols/32 E8M0 scale bytes laid out as `scale_layout` says. A "colwise"
+ * quantisation of a source matrix S [R, C] (blocks of 32 consecutive rows of S) is
+ * stored transposed: rows = C, cols = R. Both pointers are device memory owned by the
+ * caller. The scale rule of an E5M2 matrix is the MXFP8 rule below with 15 (the largest
+ * exponent of E5M2) in place of 8.
  */
 typedef struct mxmoe_mxfp8 {
   uint8_t* data;
@@ -80,7 +86,7 @@ typedef struct mxmoe_mxfp8 {
   int64_t rows;
   int64_t cols;
   int32_t scale_layout;
-  int32_t reserved; /* must be 0 */
+  int32_t elem_format; /* MXMOE_FMT_E4M3 (0) or MXMOE_FMT_E5M2 */
 } mxmoe_mxfp8;
 
 /* ------------------------------------------------------------------ status / sizes */
@@ -209,6 +215,8 @@ mxmoe_status moe_unpermute(const void* y_perm_dev, const int32_t* row_of_slot_de
  *                each batch matrix), stored transposed: rows = batch*cols, cols = out_rows;
  *                batch b's matrix occupies rows [b*cols, (b+1)*cols).
  * Shapes: cols % 32 == 0, out_rows % 32 == 0 (both % 128 == 0 for MXMOE_SCALE_MMA).
+ * Element format: each output's elem_format (E4M3 or E5M2); when both outputs are given
+ * their formats must agree (else MXMOE_ERR_INVALID_ARG).
  */
 mxmoe_status mxfp8_quantize(const void* src_dev, int32_t src_dtype, int64_t batch, int64_t rows, int64_t cols,
                             const int32_t* row_gather_dev, const int32_t* nrows_dev, int64_t out_rows,
@@ -221,7 +229,8 @@ mxmoe_status mxfp8_quantize(const void* src_dev, int32_t src_dtype, int64_t batc
  * Grundmodelle optimieren", GroupedLinear passage; "NVIDIA optimise l'entraînement MoE
  * des modèles biologiques", first improvement): for every expert e,
  *     C[seg_e, :] = dequant(A)[seg_e, :] . dequant(B_e)^T,   seg_e = [seg_off[e], seg_off[e+1])
- * with fp32 accumulation on the tensor cores.
+ * with fp32 accumulation on the tensor cores. A and B may each be E4M3 or E5M2 (their
+ * elem_format; e.g. an E5M2 gradient times an E4M3 weight).
  *   A   MXFP8 [rows_cap, K], MXMOE_SCALE_MMA; rows_cap % 256 == 0.
  *   B   MXFP8 [E*N, K], MXMOE_SCALE_MMA (expert e's rows are [e*N, (e+1)*N)).
  *   seg_off_dev  int32 [E+1], multiples of 256, read on the device (no host sync).
@@ -345,6 +354,19 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
                              size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F, void* dx_dev,
                              float* dW1_dev, float* dW2_dev, float* dprobs_dev, void* ws_dev, size_t ws_bytes,
                              void* stream);
+
+/*
+ * grouped_mlp_bwd_fmt -- grouped_mlp_bwd with the MXFP8 element format of the gradients
+ * chosen: grad_format MXMOE_FMT_E4M3 (identical to grouped_mlp_bwd) or MXMOE_FMT_E5M2, the
+ * gradient variant: dY and dGU are quantised to E5M2 (wider range, one mantissa bit fewer;
+ * the pages name FP8 beside MXFP8 and fix no element format), every data- and
+ * weight-gradient GEMM multiplies an E5M2 gradient by an E4M3 weight or activation.
+ * Any other grad_format returns MXMOE_ERR_INVALID_ARG. Same buffers and sizes.
+ */
+mxmoe_status grouped_mlp_bwd_fmt(const void* dy_dev, const void* saved_dev, size_t saved_bytes, const void* wq_dev,
+                                 size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
+                                 int32_t grad_format, void* dx_dev, float* dW1_dev, float* dW2_dev, float* dprobs_dev,
+                                 void* ws_dev, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------ bf16 grouped MLP */
 

@@ -25,6 +25,8 @@ STATUS_NAMES = {
 }
 DTYPE_BF16, DTYPE_F32 = 0, 1
 SCALE_PLAIN, SCALE_MMA = 0, 1
+FMT_E4M3, FMT_E5M2 = 0, 1
+_FMT = {"e4m3": FMT_E4M3, "e5m2": FMT_E5M2}
 SAVED_FIELDS = ["m_splits", "seg_off", "row_of_slot", "token_of_row", "prob_of_row",
                 "x_colT", "x_colT_sf", "z_colT", "z_colT_sf", "gu"]
 
@@ -37,7 +39,7 @@ class MxmoeError(RuntimeError):
 
 class _MX(ctypes.Structure):
     _fields_ = [("data", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("rows", ctypes.c_int64),
-                ("cols", ctypes.c_int64), ("scale_layout", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("cols", ctypes.c_int64), ("scale_layout", ctypes.c_int32), ("elem_format", ctypes.c_int32)]
 
 
 _lib = None
@@ -73,6 +75,8 @@ _SIGNATURES = {
     "grouped_mlp_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32]),
     "grouped_mlp_fwd": (_I32, [_P, _P, _P, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _P, _P, _SZ, _P, _SZ, _P]),
     "grouped_mlp_bwd": (_I32, [_P, _P, _SZ, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
+    "grouped_mlp_bwd_fmt": (_I32, [_P, _P, _SZ, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ,
+                                   _P]),
     "mxmoe_weights_bf16_size": (_SZ, [_I32, _I32, _I32]),
     "mxmoe_weights_bf16_prepare": (_I32, [_P, _P, _I32, _I32, _I32, _P, _SZ, _P]),
     "grouped_mlp_bf16_saved_size": (_SZ, [_I32, _I32, _I32, _I32, _I32]),
@@ -125,11 +129,13 @@ def _ptr(t):
 # ----------------------------------------------------------------------------- MXFP8 tensors
 @dataclass
 class MXFP8:
-    """An MXFP8 matrix: data uint8 [rows, cols] (E4M3 codes), scale uint8 (E8M0), and the
-    scale layout (SCALE_PLAIN = [rows, cols/32]; SCALE_MMA = tensor-core chunk order)."""
+    """An MXFP8 matrix: data uint8 [rows, cols] (FP8 codes of `fmt`: FMT_E4M3 or FMT_E5M2),
+    scale uint8 (E8M0), and the scale layout (SCALE_PLAIN = [rows, cols/32]; SCALE_MMA =
+    tensor-core chunk order)."""
     data: torch.Tensor
     scale: torch.Tensor
     layout: int = SCALE_MMA
+    fmt: int = FMT_E4M3
 
     @property
     def rows(self):
@@ -140,12 +146,12 @@ class MXFP8:
         return self.data.shape[1]
 
     @staticmethod
-    def empty(rows, cols, layout=SCALE_MMA, device="cuda"):
+    def empty(rows, cols, layout=SCALE_MMA, device="cuda", fmt=FMT_E4M3):
         return MXFP8(torch.empty((rows, cols), dtype=torch.uint8, device=device),
-                     torch.empty((rows * cols // 32,), dtype=torch.uint8, device=device), layout)
+                     torch.empty((rows * cols // 32,), dtype=torch.uint8, device=device), layout, fmt)
 
     def as_struct(self):
-        return _MX(self.data.data_ptr(), self.scale.data_ptr(), self.rows, self.cols, self.layout, 0)
+        return _MX(self.data.data_ptr(), self.scale.data_ptr(), self.rows, self.cols, self.layout, self.fmt)
 
     def scale_plain(self):
         """Scales as a [rows, cols/32] CPU tensor in plain order (index permutation only)."""
@@ -229,8 +235,10 @@ def moe_router_topk_bwd(logits, topk_idx, dprobs):
     return dl
 
 
-def mxfp8_quantize(src, rowwise=True, colwise=True, layout=SCALE_MMA, row_gather=None, nrows=None, out_rows=None):
-    """src [rows, cols] or [batch, rows, cols] bf16/fp32 -> (MXFP8 rowwise | None, MXFP8 colT | None)."""
+def mxfp8_quantize(src, rowwise=True, colwise=True, layout=SCALE_MMA, row_gather=None, nrows=None, out_rows=None,
+                   fmt=FMT_E4M3):
+    """src [rows, cols] or [batch, rows, cols] bf16/fp32 -> (MXFP8 rowwise | None, MXFP8 colT | None);
+    fmt FMT_E4M3 or FMT_E5M2 (element format of both outputs)."""
     lib = load()
     dt = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}[src.dtype]
     if src.dim() == 2:
@@ -238,8 +246,8 @@ def mxfp8_quantize(src, rowwise=True, colwise=True, layout=SCALE_MMA, row_gather
     else:
         batch, rows, cols = src.shape
     orows = rows if out_rows is None else out_rows
-    r = MXFP8.empty(batch * orows, cols, layout, src.device) if rowwise else None
-    c = MXFP8.empty(batch * cols, orows, layout, src.device) if colwise else None
+    r = MXFP8.empty(batch * orows, cols, layout, src.device, fmt) if rowwise else None
+    c = MXFP8.empty(batch * cols, orows, layout, src.device, fmt) if colwise else None
     rs = ctypes.byref(r.as_struct()) if r is not None else None
     cs = ctypes.byref(c.as_struct()) if c is not None else None
     st = lib.mxfp8_quantize(_ptr(src), dt, batch, rows, cols, _ptr(row_gather), _ptr(nrows), orows, rs, cs,
@@ -311,11 +319,16 @@ class GroupedMLP:
     """Buffers for one layer shape; forward/backward call the fused C entry points.
 
     precision "mxfp8" (default) runs the MXFP8 layer (grouped_mlp_fwd / _bwd); "bf16" runs
-    the same steps on bf16 operands (grouped_mlp_bf16_fwd / _bwd)."""
+    the same steps on bf16 operands (grouped_mlp_bf16_fwd / _bwd). grad_format "e4m3"
+    (default) or "e5m2" picks the MXFP8 element format of the gradients (dY, dGU) of the
+    MXFP8 layer's backward."""
 
-    def __init__(self, T, k, E, H, F, device="cuda", precision="mxfp8"):
+    def __init__(self, T, k, E, H, F, device="cuda", precision="mxfp8", grad_format="e4m3"):
         if precision not in ("mxfp8", "bf16"):
             raise ValueError(f"unknown precision {precision!r}")
+        if grad_format not in _FMT or (precision == "bf16" and grad_format != "e4m3"):
+            raise ValueError(f"unsupported grad_format {grad_format!r} for precision {precision!r}")
+        self.grad_format = _FMT[grad_format]
         lib = load()
         self.T, self.k, self.E, self.H, self.F = T, k, E, H, F
         self.precision = precision
@@ -341,8 +354,11 @@ class GroupedMLP:
         return fn(x, topk_idx, probs, self.wq, self.E, self.F, self.saved, self.ws, y)
 
     def backward(self, dy, dx=None, dW1=None, dW2=None, dprobs=None):
-        fn = grouped_mlp_bf16_bwd if self.precision == "bf16" else grouped_mlp_bwd
-        return fn(dy, self.saved, self.wq, self.T, self.k, self.E, self.H, self.F, self.ws, dx, dW1, dW2, dprobs)
+        if self.precision == "bf16":
+            return grouped_mlp_bf16_bwd(dy, self.saved, self.wq, self.T, self.k, self.E, self.H, self.F, self.ws,
+                                        dx, dW1, dW2, dprobs)
+        return grouped_mlp_bwd(dy, self.saved, self.wq, self.T, self.k, self.E, self.H, self.F, self.ws, dx, dW1,
+                               dW2, dprobs, grad_format=self.grad_format)
 
     def saved_field(self, name, dtype=torch.uint8, count=None):
         """View of a named field of the saved buffer of the MXFP8 layer (inspection / tests)."""
@@ -377,15 +393,22 @@ def grouped_mlp_fwd(x, topk_idx, probs, wq, E, F, saved, ws, y=None):
     return y
 
 
-def grouped_mlp_bwd(dy, saved, wq, T, k, E, H, F, ws, dx=None, dW1=None, dW2=None, dprobs=None):
+def grouped_mlp_bwd(dy, saved, wq, T, k, E, H, F, ws, dx=None, dW1=None, dW2=None, dprobs=None,
+                    grad_format=FMT_E4M3):
     dev = dy.device
     dx = dx if dx is not None else torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     dW1 = dW1 if dW1 is not None else torch.empty((E, 2 * F, H), dtype=torch.float32, device=dev)
     dW2 = dW2 if dW2 is not None else torch.empty((E, H, F), dtype=torch.float32, device=dev)
     dprobs = dprobs if dprobs is not None else torch.empty((T, k), dtype=torch.float32, device=dev)
-    st = load().grouped_mlp_bwd(_ptr(dy), _ptr(saved), saved.numel(), _ptr(wq), wq.numel(), T, k, E, H, F, _ptr(dx),
-                                _ptr(dW1), _ptr(dW2), _ptr(dprobs), _ptr(ws), ws.numel(), _stream())
-    _check("grouped_mlp_bwd", st)
+    if grad_format == FMT_E4M3:
+        st = load().grouped_mlp_bwd(_ptr(dy), _ptr(saved), saved.numel(), _ptr(wq), wq.numel(), T, k, E, H, F,
+                                    _ptr(dx), _ptr(dW1), _ptr(dW2), _ptr(dprobs), _ptr(ws), ws.numel(), _stream())
+        _check("grouped_mlp_bwd", st)
+    else:
+        st = load().grouped_mlp_bwd_fmt(_ptr(dy), _ptr(saved), saved.numel(), _ptr(wq), wq.numel(), T, k, E, H, F,
+                                        grad_format, _ptr(dx), _ptr(dW1), _ptr(dW2), _ptr(dprobs), _ptr(ws),
+                                        ws.numel(), _stream())
+        _check("grouped_mlp_bwd_fmt", st)
     return dx, dW1, dW2, dprobs
 
 

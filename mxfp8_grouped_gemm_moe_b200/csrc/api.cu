@@ -122,20 +122,21 @@ BwdWs bwd_ws(int64_t T, int64_t k, int64_t E, int64_t H, int64_t F) {
 
 bool valid_mx(const mxmoe_mxfp8* m) {
   return m && m->data && m->scale && aligned16(m->data) && aligned16(m->scale) && m->rows >= 0 && m->cols >= 0 &&
-         (m->scale_layout == MXMOE_SCALE_PLAIN || m->scale_layout == MXMOE_SCALE_MMA) && m->reserved == 0;
+         (m->scale_layout == MXMOE_SCALE_PLAIN || m->scale_layout == MXMOE_SCALE_MMA) &&
+         (m->elem_format == MXMOE_FMT_E4M3 || m->elem_format == MXMOE_FMT_E5M2);
 }
 bool mma_ready(const mxmoe_mxfp8* m) {
   return valid_mx(m) && m->scale_layout == MXMOE_SCALE_MMA && m->rows % 128 == 0 && m->cols % 128 == 0;
 }
 
-mxmoe_mxfp8 mk(uint8_t* base, size_t d, size_t s, int64_t rows, int64_t cols) {
+mxmoe_mxfp8 mk(uint8_t* base, size_t d, size_t s, int64_t rows, int64_t cols, int32_t fmt = MXMOE_FMT_E4M3) {
   mxmoe_mxfp8 m;
   m.data = base + d;
   m.scale = base + s;
   m.rows = rows;
   m.cols = cols;
   m.scale_layout = MXMOE_SCALE_MMA;
-  m.reserved = 0;
+  m.elem_format = fmt;
   return m;
 }
 
@@ -152,6 +153,8 @@ GemmArgs gemm_base(int mode, const mxmoe_mxfp8& A, const mxmoe_mxfp8& B, const i
   g.b_sf = B.scale;
   g.b_rows = B.rows;
   g.b_cols = B.cols;
+  g.a_fmt = A.elem_format;
+  g.b_fmt = B.elem_format;
   g.seg_off = seg_off;
   return g;
 }
@@ -298,8 +301,10 @@ static mxmoe_status quantize_impl(const void* src_dev, int32_t src_dtype, int64_
     if (out_colT->scale_layout == MXMOE_SCALE_MMA && (out_rows % 128 != 0 || cols % 128 != 0))
       return MXMOE_ERR_UNSUPPORTED_SHAPE;
   }
+  if (out_row && out_colT && out_row->elem_format != out_colT->elem_format) return MXMOE_ERR_INVALID_ARG;
   if (out_rows == 0 || rows == 0) return MXMOE_OK;
   QuantArgs a;
+  a.fmt = out_row ? out_row->elem_format : out_colT->elem_format;
   a.src = src_dev;
   a.src_dtype = src_dtype;
   a.batch = batch;
@@ -544,6 +549,15 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
                              size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F, void* dx_dev,
                              float* dW1_dev, float* dW2_dev, float* dprobs_dev, void* ws_dev, size_t ws_bytes,
                              void* stream) {
+  return grouped_mlp_bwd_fmt(dy_dev, saved_dev, saved_bytes, wq_dev, wq_bytes, T, k, E, H, F, MXMOE_FMT_E4M3, dx_dev,
+                             dW1_dev, dW2_dev, dprobs_dev, ws_dev, ws_bytes, stream);
+}
+
+mxmoe_status grouped_mlp_bwd_fmt(const void* dy_dev, const void* saved_dev, size_t saved_bytes, const void* wq_dev,
+                                 size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
+                                 int32_t grad_format, void* dx_dev, float* dW1_dev, float* dW2_dev, float* dprobs_dev,
+                                 void* ws_dev, size_t ws_bytes, void* stream) {
+  if (grad_format != MXMOE_FMT_E4M3 && grad_format != MXMOE_FMT_E5M2) return MXMOE_ERR_INVALID_ARG;
   if (!valid_mlp_shape(T, k, E, H, F)) return MXMOE_ERR_UNSUPPORTED_SHAPE;
   if (!wq_dev || !saved_dev || !ws_dev || !dW1_dev || !dW2_dev || !aligned16(wq_dev) || !aligned16(saved_dev) ||
       !aligned16(ws_dev) || !aligned16(dW1_dev) || !aligned16(dW2_dev))
@@ -567,8 +581,8 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
   const float* por = reinterpret_cast<const float*>(sv + SL.off[MXMOE_SAVED_PROB_OF_ROW]);
 
   // 1. permute + quantise dy: rowwise (fc2 dgrad) and colwise (fc2 wgrad)
-  mxmoe_mxfp8 dy_row = mk(ws, W.dy_row, W.dy_row_sf, cap, H);
-  mxmoe_mxfp8 dy_col = mk(ws, W.dy_colT, W.dy_colT_sf, H, cap);
+  mxmoe_mxfp8 dy_row = mk(ws, W.dy_row, W.dy_row_sf, cap, H, grad_format);
+  mxmoe_mxfp8 dy_col = mk(ws, W.dy_colT, W.dy_colT_sf, H, cap, grad_format);
   mxmoe_status s;
   if (T > 0) {
     StageScope sc(MXMOE_STAGE_QUANT_DY, st);
@@ -590,6 +604,7 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
     g.dgu_colT = ws + W.dgu_colT;
     g.dgu_colT_sf = ws + W.dgu_colT_sf;
     g.dprob_part = reinterpret_cast<float*>(ws + W.dprob_part);
+    g.out_fmt = grad_format;
     StageScope sc(MXMOE_STAGE_FC2_DGRAD, st);
     if (T > 0 && launch_gemm(g, st) != cudaSuccess) return MXMOE_ERR_CUDA;
   }
@@ -608,7 +623,7 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
   }
   if (s != MXMOE_OK) return s;
   // 5. fc1 dgrad: dXp = dGU . W1 (contract 2F)
-  mxmoe_mxfp8 dgu_row = mk(ws, W.dgu_row, W.dgu_row_sf, cap, 2 * (int64_t)F);
+  mxmoe_mxfp8 dgu_row = mk(ws, W.dgu_row, W.dgu_row_sf, cap, 2 * (int64_t)F, grad_format);
   mxmoe_mxfp8 w1c = mk(wq, WL.d[1], WL.s[1], WL.rows[1], WL.cols[1]);
   if (T > 0) {
     StageScope sc(MXMOE_STAGE_FC1_DGRAD, st);
@@ -617,7 +632,7 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
     if (s != MXMOE_OK) return s;
   }
   // 6. fc1 wgrad: dW1[e] = dGU_e^T . Xp_e
-  mxmoe_mxfp8 dgu_col = mk(ws, W.dgu_colT, W.dgu_colT_sf, 2 * (int64_t)F, cap);
+  mxmoe_mxfp8 dgu_col = mk(ws, W.dgu_colT, W.dgu_colT_sf, 2 * (int64_t)F, cap, grad_format);
   mxmoe_mxfp8 x_col = mk(sv, SL.off[MXMOE_SAVED_X_COLT], SL.off[MXMOE_SAVED_X_COLT_SF], H, cap);
   {
     StageScope sc(MXMOE_STAGE_FC1_WGRAD, st);

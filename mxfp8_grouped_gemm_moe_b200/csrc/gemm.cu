@@ -216,14 +216,16 @@ __device__ __forceinline__ uint32_t amax_bits32(const float (&v)[32]) {
   return m[0];
 }
 
-// 32 fp32 -> 32 E4M3 codes (8 words) under the block's scale; returns the E8M0 byte.
+// 32 fp32 -> 32 FP8 codes of format FMT (8 words) under the block's scale; returns the
+// E8M0 byte.
+template <int FMT = MXMOE_FMT_E4M3>
 __device__ __forceinline__ uint8_t quant32(const float (&v)[32], uint32_t (&q)[8]) {
-  const int32_t X = mx_scale_exp_from_amax_bits(amax_bits32(v));
+  const int32_t X = mx_scale_exp_from_amax_bits<FMT>(amax_bits32(v));
   const float sc = mx_inv_scale(X);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t lo = e4m3x2(v[4 * i] * sc, v[4 * i + 1] * sc);
-    const uint32_t hi = e4m3x2(v[4 * i + 2] * sc, v[4 * i + 3] * sc);
+    const uint32_t lo = fp8x2<FMT>(v[4 * i] * sc, v[4 * i + 1] * sc);
+    const uint32_t hi = fp8x2<FMT>(v[4 * i + 2] * sc, v[4 * i + 3] * sc);
     q[i] = lo | (hi << 16);
   }
   return (uint8_t)(X + 127);
@@ -257,12 +259,13 @@ __device__ __forceinline__ void colwise_transpose2(const float (&v0)[32], const 
   }
   __syncwarp();  // the buffer may be refilled once every lane has read its columns
 }
+template <int FMT = MXMOE_FMT_E4M3>
 __device__ __forceinline__ void colwise_codes2(const float (&v0)[32], const float (&v1)[32], float* stg, int lane,
                                                uint32_t (&q0)[8], uint32_t (&q1)[8], uint8_t& sb0, uint8_t& sb1) {
   float w0[32], w1[32];
   colwise_transpose2(v0, v1, stg, lane, w0, w1);
-  sb0 = quant32(w0, q0);
-  sb1 = quant32(w1, q1);
+  sb0 = quant32<FMT>(w0, q0);
+  sb1 = quant32<FMT>(w1, q1);
 }
 // bf16 output mode: lane r's 32 values as 64 bytes of bf16 at box + r * 64 (one row of a
 // 32 x 32 bf16 box).
@@ -342,9 +345,12 @@ __device__ __forceinline__ uint4 pack8_bf16(const uint32_t (&v)[N], int i0) {
   return o;
 }
 
-// ESZ: operand element bytes -- 1: MXFP8 (E4M3 + E8M0 scales, kind::mxf8f6f4.block_scale),
-// 2: bf16 (kind::f16, no scales; plain-store and weight-gradient modes, CTA pairs only).
-template <int MODE, int PAIR, int ESZ>
+// ESZ: operand element bytes -- 1: MXFP8 (E4M3 or E5M2 codes + E8M0 scales,
+// kind::mxf8f6f4.block_scale; the operand formats come from GemmArgs), 2: bf16 (kind::f16,
+// no scales; CTA pairs only).
+// OF: element format of the MXFP8 outputs of the backward fused epilogue (dGU): E4M3, or
+// E5M2 for the gradient variant.
+template <int MODE, int PAIR, int ESZ, int OF = MXMOE_FMT_E4M3>
 __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
     mxgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
@@ -506,6 +512,9 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
       int stage = 0;
       uint32_t ph = 0, acc_ph = 0;
       bool dropped = false;
+      // operand element formats (E4M3 = 0, E5M2 = 1) in the instruction descriptor's A / B
+      // format fields, bits [7, 10) and [10, 13)
+      const uint32_t fmt_bits = ((uint32_t)(g.a_fmt & 1) << 7) | ((uint32_t)(g.b_fmt & 1) << 10);
       for (int32_t tile = first; tile < ntiles && !*s_abort; tile += stride) {
         const TileInfo t = get_tile<MODE, PAIR, ESZ>(g, tile, s_seg, s_order, 0);
         if (t.k_iters == 0) continue;
@@ -550,7 +559,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
                                  ptx::make_idesc_bf16(C::TM, BN), acc);
               continue;
             }
-            const uint32_t idesc = ptx::make_idesc_mxf8(C::TM, BN, (uint32_t)kk, (uint32_t)kk);
+            const uint32_t idesc = ptx::make_idesc_mxf8(C::TM, BN, (uint32_t)kk, (uint32_t)kk) | fmt_bits;
             if (PAIR == 1)
               ptx::mma_mxf8(tmem_base, adesc + (uint64_t)(2 * kk), bdesc + (uint64_t)(2 * kk), idesc, t_sfa, t_sfb,
                             acc);
@@ -814,10 +823,10 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           }
           uint32_t rg[8], ru[8], cg[8], cu[8];
           uint8_t csg, csu;
-          sfg |= (uint32_t)quant32(vg, rg) << (8 * c);
-          sfu |= (uint32_t)quant32(vu, ru) << (8 * c);
+          sfg |= (uint32_t)quant32<OF>(vg, rg) << (8 * c);
+          sfu |= (uint32_t)quant32<OF>(vu, ru) << (8 * c);
           staging_acquire(lane);
-          colwise_codes2(vg, vu, stg, lane, cg, cu, csg, csu);
+          colwise_codes2<OF>(vg, vu, stg, lane, cg, cu, csg, csu);
           uint8_t* stg8 = reinterpret_cast<uint8_t*>(stg);
           put_codes32(stg8, lane, rg);
           put_codes32(stg8 + 1024, lane, ru);
@@ -953,21 +962,21 @@ struct GemmMaps {
   CUtensorMap c, d, e;  // epilogue outputs (unused ones zeroed)
 };
 
-template <int MODE, int PAIR, int ESZ = 1>
+template <int MODE, int PAIR, int ESZ = 1, int OF = MXMOE_FMT_E4M3>
 static cudaError_t launch_mode(const GemmMaps& m, const GemmArgs& g, int64_t tiles_ub, cudaStream_t st) {
   constexpr uint32_t smem = Cfg<PAIR, MODE>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(mxgemm_kernel<MODE, PAIR, ESZ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(mxgemm_kernel<MODE, PAIR, ESZ, OF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   // the warpgroup register split assumes the launch allocation it was sized for
   cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, mxgemm_kernel<MODE, PAIR, ESZ>);
+  e = cudaFuncGetAttributes(&fa, mxgemm_kernel<MODE, PAIR, ESZ, OF>);
   if (e != cudaSuccess) return e;
   if (Cfg<PAIR, MODE>::kSplitRegs && fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
   const int units = gemm_num_sms() / PAIR;  // SMs, or SM pairs
   const int n = (int)(tiles_ub < units ? (tiles_ub > 0 ? tiles_ub : 1) : units);
   if constexpr (PAIR == 1) {
-    mxgemm_kernel<MODE, 1, ESZ><<<n, Cfg<PAIR, MODE>::kThreads, smem, st>>>(m.a, m.b, m.sfa, m.sfb, m.c, m.d, m.e, g);
+    mxgemm_kernel<MODE, 1, ESZ, OF><<<n, Cfg<PAIR, MODE>::kThreads, smem, st>>>(m.a, m.b, m.sfa, m.sfb, m.c, m.d, m.e, g);
   } else {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * n, 1, 1);
@@ -981,7 +990,7 @@ static cudaError_t launch_mode(const GemmMaps& m, const GemmArgs& g, int64_t til
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, mxgemm_kernel<MODE, PAIR, ESZ>, m.a, m.b, m.sfa, m.sfb, m.c, m.d, m.e, g);
+    e = cudaLaunchKernelEx(&cfg, mxgemm_kernel<MODE, PAIR, ESZ, OF>, m.a, m.b, m.sfa, m.sfb, m.c, m.d, m.e, g);
     if (e != cudaSuccess) return e;
   }
   ++g_launch_count;
@@ -999,6 +1008,8 @@ static cudaError_t launch_variant(const GemmArgs& g, cudaStream_t st) {
       !make_sf_map(&m.sfb, g.b_sf, (g.b_rows / 128) * (g.b_cols / 128)))
     return cudaErrorInvalidValue;
   constexpr int TM = 128 * PAIR;
+  if (g.out_fmt != MXMOE_FMT_E4M3 && (g.mode != kModeSwigluBwd || g.out_fmt != MXMOE_FMT_E5M2))
+    return cudaErrorInvalidValue;  // Z stays E4M3; only the backward epilogue writes E5M2
   switch (g.mode) {
     case kModeStore:
       if (!make_out_map(&m.c, g.c, g.a_rows, g.N, g.ldc, g.c_dtype == MXMOE_DTYPE_F32)) return cudaErrorInvalidValue;
@@ -1012,6 +1023,8 @@ static cudaError_t launch_variant(const GemmArgs& g, cudaStream_t st) {
       if (!make_codes32_map(&m.c, g.dgu_row, g.rows_cap, 2 * g.F) ||
           !make_codes32_map(&m.d, g.dgu_colT, 2 * g.F, g.rows_cap))
         return cudaErrorInvalidValue;
+      if (g.out_fmt == MXMOE_FMT_E5M2)
+        return launch_mode<kModeSwigluBwd, PAIR, 1, MXMOE_FMT_E5M2>(m, g, (g.a_rows / TM) * (g.F / BN), st);
       return launch_mode<kModeSwigluBwd, PAIR>(m, g, (g.a_rows / TM) * (g.F / BN), st);
     case kModeWgrad:
       if (!make_out_map(&m.c, g.c, (int64_t)g.E * g.N, g.K2, g.K2, true)) return cudaErrorInvalidValue;

@@ -1,5 +1,5 @@
 // Device-side helpers shared by the library's kernels: the device status word, the
-// MXFP8 block quantiser (OCP MX: E4M3 elements, E8M0 power-of-two scale per 32
+// MXFP8 block quantiser (OCP MX: E4M3 or E5M2 elements, E8M0 power-of-two scale per 32
 // values) and the scale-factor layouts.
 #pragma once
 #include <cstdint>
@@ -25,12 +25,15 @@ __device__ __forceinline__ void record_error(int32_t code, int32_t where) {
 __device__ __forceinline__ void record_timeout(int32_t where) { record_error(MXMOE_ERR_DEVICE_TIMEOUT, where); }
 
 // ----------------------------------------------------------------------------- quantiser
-// Scale exponent X = clamp(floor(log2(amax)) - 8, -127, 127) from the bit pattern of a
-// non-negative fp32 amax; zero or subnormal amax gives the lower clamp (-127).
+// Scale exponent X = clamp(floor(log2(amax)) - emax, -127, 127) from the bit pattern of a
+// non-negative fp32 amax (emax = 8 for E4M3 elements, 15 for E5M2); zero or subnormal
+// amax gives the lower clamp (-127).
+template <int FMT = MXMOE_FMT_E4M3>
 __device__ __forceinline__ int32_t mx_scale_exp_from_amax_bits(uint32_t amax_bits) {
+  constexpr int32_t kEmax = FMT == MXMOE_FMT_E4M3 ? 8 : 15;  // largest exponent of the element format
   const int32_t ef = (int32_t)((amax_bits >> 23) & 0xFFu);
   if (ef == 0) return -127;
-  int32_t X = ef - 127 - 8;
+  int32_t X = ef - 127 - kEmax;
   return X < -127 ? -127 : (X > 127 ? 127 : X);
 }
 
@@ -39,23 +42,28 @@ __device__ __forceinline__ float mx_inv_scale(int32_t X) {
   return __uint_as_float((uint32_t)(127 - X) << 23);
 }
 
-// Two fp32 -> two E4M3 (round to nearest even, saturate to +-448), low byte = a.
-__device__ __forceinline__ uint16_t e4m3x2(float a, float b) {
-  return (uint16_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+// Two fp32 -> two FP8 codes of the element format (round to nearest even, saturate to
+// the largest finite value: +-448 for E4M3, +-57344 for E5M2), low byte = a.
+template <int FMT = MXMOE_FMT_E4M3>
+__device__ __forceinline__ uint16_t fp8x2(float a, float b) {
+  return (uint16_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE,
+                                            FMT == MXMOE_FMT_E4M3 ? __NV_E4M3 : __NV_E5M2);
 }
+__device__ __forceinline__ uint16_t e4m3x2(float a, float b) { return fp8x2<MXMOE_FMT_E4M3>(a, b); }
 
 // Quantise 32 fp32 values held by one thread -> 32 codes packed in 8 words; returns the
 // E8M0 scale byte.
+template <int FMT = MXMOE_FMT_E4M3>
 __device__ __forceinline__ uint8_t quant_block32(const float (&v)[32], uint32_t (&out)[8]) {
   uint32_t amax = 0;
 #pragma unroll
   for (int i = 0; i < 32; ++i) amax = max(amax, __float_as_uint(fabsf(v[i])));
-  const int32_t X = mx_scale_exp_from_amax_bits(amax);
+  const int32_t X = mx_scale_exp_from_amax_bits<FMT>(amax);
   const float s = mx_inv_scale(X);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t lo = e4m3x2(v[4 * i + 0] * s, v[4 * i + 1] * s);
-    const uint32_t hi = e4m3x2(v[4 * i + 2] * s, v[4 * i + 3] * s);
+    const uint32_t lo = fp8x2<FMT>(v[4 * i + 0] * s, v[4 * i + 1] * s);
+    const uint32_t hi = fp8x2<FMT>(v[4 * i + 2] * s, v[4 * i + 3] * s);
     out[i] = lo | (hi << 16);
   }
   return (uint8_t)(X + 127);

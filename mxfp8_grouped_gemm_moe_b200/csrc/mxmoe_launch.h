@@ -45,6 +45,7 @@ struct QuantArgs {
   // > 0: the rowwise copy of each [2*row_ilv, cols] batch matrix stores its rows in
   // 64-row blocks interleaved [first half 0..63, second half 0..63, first 64..127, ...]
   int64_t row_ilv;
+  int32_t fmt;  // element format of both outputs: MXMOE_FMT_E4M3 or MXMOE_FMT_E5M2
 };
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
 // bf16 -> bf16 copies with the same row gather / valid-row count / gate-up interleave as
@@ -71,6 +72,7 @@ struct GemmArgs {
   const uint8_t* b_data;
   const uint8_t* b_sf;
   int64_t b_rows, b_cols;
+  int32_t a_fmt, b_fmt;    // element formats of the MXFP8 operands (MXMOE_FMT_*)
   const int32_t* seg_off;  // device [E+1]
   int64_t N;               // per-expert B rows (store/bwd), F (fwd), output rows per expert (wgrad)
   int64_t K;               // contraction length (not used by wgrad)
@@ -95,6 +97,7 @@ struct GemmArgs {
   uint8_t* dgu_colT;
   uint8_t* dgu_colT_sf;
   float* dprob_part;  // [rows_cap, F/128]
+  int32_t out_fmt;    // element format of the fused epilogues' MXFP8 outputs (Z / dGU)
   // debug: if non-zero, the MMA warp withholds its first accumulator-ready signal so
   // that the epilogue's bounded wait expires (tests the timeout path; never set in
   // normal use)

@@ -5,7 +5,8 @@
 // 8-bit values with one scale per block of 32; GroupedMLP passage: the 16-bit -> 8-bit
 // conversions are fused rather than run as separate operations. Element / scale rule:
 // OCP MX (E4M3 elements, E8M0 scale, X = clamp(floor(log2 amax) - 8, -127, 127),
-// round-to-nearest-even with saturation).
+// round-to-nearest-even with saturation); E5M2 elements (largest exponent 15 in place of
+// 8) for the gradient variant, on the gathered per-tile path.
 //
 // One CTA quantises a 128 x 128 tile staged in shared memory: rowwise blocks (32
 // consecutive columns of a row) and colwise blocks (32 consecutive rows of a column,
@@ -85,17 +86,18 @@ __device__ __forceinline__ void load_pair(const float* p, float& a, float& b) {
 // 2k+1 in the high half). |bf16| bit patterns order like unsigned 16-bit integers, so
 // the block amax is a SIMD max over the masked words; the result equals the amax of the
 // values widened to fp32 (widening is exact), hence the same scale as quant_block32.
+template <int FMT = MXMOE_FMT_E4M3>
 __device__ __forceinline__ uint8_t quant_block32_bf16(const uint32_t (&w)[16], uint32_t (&out)[8]) {
   uint32_t m = 0;
 #pragma unroll
   for (int i = 0; i < 16; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
   const uint32_t amax = max(m << 16, m & 0xFFFF0000u);
-  const int32_t X = mx_scale_exp_from_amax_bits(amax);
+  const int32_t X = mx_scale_exp_from_amax_bits<FMT>(amax);
   const float s = mx_inv_scale(X);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t lo = e4m3x2(bf16_lo(w[2 * i]) * s, bf16_hi(w[2 * i]) * s);
-    const uint32_t hi = e4m3x2(bf16_lo(w[2 * i + 1]) * s, bf16_hi(w[2 * i + 1]) * s);
+    const uint32_t lo = fp8x2<FMT>(bf16_lo(w[2 * i]) * s, bf16_hi(w[2 * i]) * s);
+    const uint32_t hi = fp8x2<FMT>(bf16_lo(w[2 * i + 1]) * s, bf16_hi(w[2 * i + 1]) * s);
     out[i] = lo | (hi << 16);
   }
   return (uint8_t)(X + 127);
@@ -103,69 +105,65 @@ __device__ __forceinline__ uint8_t quant_block32_bf16(const uint32_t (&w)[16], u
 
 // Colwise MXFP8 of two adjacent columns over 32 rows: w[r] holds (column c, row r) in
 // its low half and (column c+1, row r) in its high half.
+template <int FMT = MXMOE_FMT_E4M3>
 __device__ __forceinline__ void quant_colpair_bf16(const uint32_t (&w)[32], uint32_t (&o0)[8], uint32_t (&o1)[8],
                                                    uint8_t& sb0, uint8_t& sb1) {
   uint32_t m = 0;
 #pragma unroll
   for (int i = 0; i < 32; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
-  const int32_t X0 = mx_scale_exp_from_amax_bits(m << 16);
-  const int32_t X1 = mx_scale_exp_from_amax_bits(m & 0xFFFF0000u);
+  const int32_t X0 = mx_scale_exp_from_amax_bits<FMT>(m << 16);
+  const int32_t X1 = mx_scale_exp_from_amax_bits<FMT>(m & 0xFFFF0000u);
   const float s0 = mx_inv_scale(X0), s1 = mx_inv_scale(X1);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    o0[i] = (uint32_t)e4m3x2(bf16_lo(w[4 * i]) * s0, bf16_lo(w[4 * i + 1]) * s0) |
-            ((uint32_t)e4m3x2(bf16_lo(w[4 * i + 2]) * s0, bf16_lo(w[4 * i + 3]) * s0) << 16);
-    o1[i] = (uint32_t)e4m3x2(bf16_hi(w[4 * i]) * s1, bf16_hi(w[4 * i + 1]) * s1) |
-            ((uint32_t)e4m3x2(bf16_hi(w[4 * i + 2]) * s1, bf16_hi(w[4 * i + 3]) * s1) << 16);
+    o0[i] = (uint32_t)fp8x2<FMT>(bf16_lo(w[4 * i]) * s0, bf16_lo(w[4 * i + 1]) * s0) |
+            ((uint32_t)fp8x2<FMT>(bf16_lo(w[4 * i + 2]) * s0, bf16_lo(w[4 * i + 3]) * s0) << 16);
+    o1[i] = (uint32_t)fp8x2<FMT>(bf16_hi(w[4 * i]) * s1, bf16_hi(w[4 * i + 1]) * s1) |
+            ((uint32_t)fp8x2<FMT>(bf16_hi(w[4 * i + 2]) * s1, bf16_hi(w[4 * i + 3]) * s1) << 16);
   }
   sb0 = (uint8_t)(X0 + 127);
   sb1 = (uint8_t)(X1 + 127);
 }
 
-template <typename T>
-__device__ __forceinline__ uint8_t quant_row_block(const T* p, uint32_t (&q)[8]);
-template <>
-__device__ __forceinline__ uint8_t quant_row_block<__nv_bfloat16>(const __nv_bfloat16* p, uint32_t (&q)[8]) {
+template <int FMT>
+__device__ __forceinline__ uint8_t quant_row_block(const __nv_bfloat16* p, uint32_t (&q)[8]) {
   uint32_t w[16];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint4 v = reinterpret_cast<const uint4*>(p)[i];
     w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
   }
-  return quant_block32_bf16(w, q);
+  return quant_block32_bf16<FMT>(w, q);
 }
-template <>
-__device__ __forceinline__ uint8_t quant_row_block<float>(const float* p, uint32_t (&q)[8]) {
+template <int FMT>
+__device__ __forceinline__ uint8_t quant_row_block(const float* p, uint32_t (&q)[8]) {
   float v[32];
   load32_row(p, v);
-  return quant_block32(v, q);
+  return quant_block32<FMT>(v, q);
 }
 
-template <typename T>
-__device__ __forceinline__ void quant_col_pair(const T* p, int ld, uint32_t (&q0)[8], uint32_t (&q1)[8], uint8_t& s0,
-                                               uint8_t& s1);
-template <>
-__device__ __forceinline__ void quant_col_pair<__nv_bfloat16>(const __nv_bfloat16* p, int ld, uint32_t (&q0)[8],
-                                                              uint32_t (&q1)[8], uint8_t& s0, uint8_t& s1) {
+template <int FMT>
+__device__ __forceinline__ void quant_col_pair(const __nv_bfloat16* p, int ld, uint32_t (&q0)[8], uint32_t (&q1)[8],
+                                               uint8_t& s0, uint8_t& s1) {
   uint32_t w[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) w[i] = *reinterpret_cast<const uint32_t*>(p + i * ld);
-  quant_colpair_bf16(w, q0, q1, s0, s1);
+  quant_colpair_bf16<FMT>(w, q0, q1, s0, s1);
 }
-template <>
-__device__ __forceinline__ void quant_col_pair<float>(const float* p, int ld, uint32_t (&q0)[8], uint32_t (&q1)[8],
-                                                      uint8_t& s0, uint8_t& s1) {
+template <int FMT>
+__device__ __forceinline__ void quant_col_pair(const float* p, int ld, uint32_t (&q0)[8], uint32_t (&q1)[8],
+                                               uint8_t& s0, uint8_t& s1) {
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = p[i * ld];
-  s0 = quant_block32(v, q0);
+  s0 = quant_block32<FMT>(v, q0);
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = p[i * ld + 1];
-  s1 = quant_block32(v, q1);
+  s1 = quant_block32<FMT>(v, q1);
 }
 
 // One CTA per 128 x 128 tile (many resident per SM to overlap load latency).
-template <typename T>
+template <typename T, int FMT>
 __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quantize_kernel(QuantArgs a) {
   using Tr = SrcTraits<T>;
   extern __shared__ __align__(16) uint8_t q_smem_raw[];
@@ -218,7 +216,7 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
       const int64_t col = c0 + 32 * blk;
       if (orow >= nvalid || col >= a.cols) continue;
       uint32_t q[8];
-      const uint8_t sb = quant_row_block<T>(tile + tile_off<T>(row, 32 * blk), q);
+      const uint8_t sb = quant_row_block<FMT>(tile + tile_off<T>(row, 32 * blk), q);
       int64_t drow = orow;
       if (a.row_ilv > 0) {  // gate / up interleave of the fc1 operand
         const int64_t hf = orow >= a.row_ilv, rr = orow - hf * a.row_ilv;
@@ -240,7 +238,7 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
     if (orow < nvalid && col < a.cols) {
       uint32_t q0[8], q1[8];
       uint8_t s0, s1;
-      quant_col_pair<T>(tile + tile_off<T>(32 * rb, 2 * pcol), 4 * Tr::kBS, q0, q1, s0, s1);
+      quant_col_pair<FMT>(tile + tile_off<T>(32 * rb, 2 * pcol), 4 * Tr::kBS, q0, q1, s0, s1);
       const int64_t grow = b * a.cols + col;  // row of the transposed matrix
       uint4* d0 = reinterpret_cast<uint4*>(a.col_data + grow * a.out_rows + orow);
       uint4* d1 = reinterpret_cast<uint4*>(a.col_data + (grow + 1) * a.out_rows + orow);
@@ -496,7 +494,7 @@ cudaError_t launch_bf16_copy(const QuantArgs& a, cudaStream_t st) {
 }
 
 static bool qt_applies(const QuantArgs& a) {
-  return a.src_dtype == MXMOE_DTYPE_BF16 && !a.gather && !a.nrows && a.out_rows == a.rows && a.rows % kQTile == 0 &&
+  return a.src_dtype == MXMOE_DTYPE_BF16 && a.fmt == MXMOE_FMT_E4M3 && !a.gather && !a.nrows && a.out_rows == a.rows && a.rows % kQTile == 0 &&
          a.cols % kQTile == 0 && a.batch * a.rows < (int64_t)1 << 31 && a.batch * a.cols < (int64_t)1 << 31 &&
          a.row_data && a.col_data && (reinterpret_cast<uintptr_t>(a.row_data) & 15) == 0 &&
          (reinterpret_cast<uintptr_t>(a.col_data) & 15) == 0;
@@ -548,25 +546,29 @@ static cudaError_t launch_qt(const QuantArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <typename T>
+template <typename T, int FMT>
 static cudaError_t launch_q(const QuantArgs& a, cudaStream_t st) {
   using Tr = SrcTraits<T>;
   const size_t smem = (size_t)kQTile * 4 * Tr::kBS * sizeof(T);
   cudaError_t e =
-      cudaFuncSetAttribute(mxfp8_quantize_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cudaFuncSetAttribute(mxfp8_quantize_kernel<T, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((a.cols + kQTile - 1) / kQTile), (unsigned)((a.out_rows + kQTile - 1) / kQTile),
             (unsigned)a.batch);
   if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
-  mxfp8_quantize_kernel<T><<<grid, kQThreads, smem, st>>>(a);
+  mxfp8_quantize_kernel<T, FMT><<<grid, kQThreads, smem, st>>>(a);
   ++g_launch_count;
   return cudaGetLastError();
 }
 
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st) {
+  if (a.fmt != MXMOE_FMT_E4M3 && a.fmt != MXMOE_FMT_E5M2) return cudaErrorInvalidValue;
   if (qt_applies(a)) return launch_qt(a, st);
-  if (a.src_dtype == MXMOE_DTYPE_BF16) return launch_q<__nv_bfloat16>(a, st);
-  return launch_q<float>(a, st);
+  if (a.fmt == MXMOE_FMT_E5M2)
+    return a.src_dtype == MXMOE_DTYPE_BF16 ? launch_q<__nv_bfloat16, MXMOE_FMT_E5M2>(a, st)
+                                           : launch_q<float, MXMOE_FMT_E5M2>(a, st);
+  return a.src_dtype == MXMOE_DTYPE_BF16 ? launch_q<__nv_bfloat16, MXMOE_FMT_E4M3>(a, st)
+                                         : launch_q<float, MXMOE_FMT_E4M3>(a, st);
 }
 
 }  // namespace mxmoe

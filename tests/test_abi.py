@@ -116,3 +116,18 @@ def test_host_argument_errors_enqueue_nothing(lib):
                                16, S) == 3
     assert lib.grouped_mlp_bwd(fake, fake, 1 << 40, fake, 1 << 40, 16, 2, 4, 256, 512, fake, bad, fake, fake,
                                fake, 1 << 40, S) == 1
+    # gradient element format: only E4M3 (0) and E5M2 (1)
+    assert lib.grouped_mlp_bwd_fmt(fake, fake, 1 << 40, fake, 1 << 40, 16, 2, 4, 256, 512, 2, fake, fake, fake, fake,
+                                   fake, 1 << 40, S) == 1
+    # an MXFP8 descriptor with an unknown element format; row / colT formats that disagree
+    m_bad_fmt = mx._MX(1 << 20, 1 << 20, 64, 64, 0, 3)
+    assert lib.mxfp8_quantize(fake, 0, 1, 64, 64, None, None, 64, ctypes.byref(m_bad_fmt), None, S) == 1
+    r4 = mx._MX(1 << 20, 1 << 20, 64, 64, 0, 0)
+    c5 = mx._MX(1 << 20, 1 << 20, 64, 64, 0, 1)
+    assert lib.mxfp8_quantize(fake, 0, 1, 64, 64, None, None, 64, ctypes.byref(r4), ctypes.byref(c5), S) == 1
+    # bf16 layer: same shape and size checks
+    assert lib.grouped_mlp_bf16_fwd(fake, fake, fake, fake, 1 << 40, 16, 2, 4, 256, 384, fake, fake, 1 << 40, fake,
+                                    1 << 40, S) == 2
+    assert lib.grouped_mlp_bf16_bwd(fake, fake, 1 << 40, fake, 16, 16, 2, 4, 256, 512, fake, fake, fake, fake,
+                                    fake, 1 << 40, S) == 3
+    assert lib.mxmoe_weights_bf16_prepare(fake, fake, 2, 256, 384, fake, 1 << 40, S) == 2

@@ -1,0 +1,148 @@
+"""GPU parity of the E5M2-gradient variant with the oracle: the E5M2 quantiser (bytes and
+scales bit-exact), grouped GEMMs that multiply an E5M2 operand by an E4M3 one (both
+kernel variants), and the fused backward with E5M2 gradients (rel-L2 <= 2e-2)."""
+import numpy as np
+import pytest
+import torch
+
+import moe_workloads as wl
+from oracle import moe as omoe
+from oracle import mxfp8 as omx
+from tests.util import f64, rel_l2, u8, SEG_ALIGN
+
+pytestmark = pytest.mark.gpu
+TOL_F32 = 5e-4
+TOL_E2E = 2e-2
+
+
+@pytest.fixture(params=["pair", "single"])
+def variant(request, monkeypatch):
+    monkeypatch.setenv("MXMOE_GEMM_PAIR", "2" if request.param == "pair" else "1")
+    return request.param
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("layout", [0, 1])
+def test_quantize_e5m2_matches_oracle(gpu_lib, dtype, layout):
+    R, C = 256, 384
+    x = wl.random_matrix(R, C, seed=77, dtype=torch.float32)
+    g = torch.Generator().manual_seed(2)
+    x = x * torch.exp2(torch.randint(-40, 40, (R, 1), generator=g).float())
+    x[3, :40] = 0.0
+    x[6, 5] = 65000.0 * 2.0 ** 10          # saturating block (amax just below 2^16 * 2^X)
+    x = x.to(dtype)
+    r, c = gpu_lib.mxfp8_quantize(x.cuda(), layout=layout, fmt=gpu_lib.FMT_E5M2)
+    torch.cuda.synchronize()
+    qr, sr = omx.quantize_rowwise(f64(x), "e5m2")
+    qc, sc = omx.quantize_colwise_t(f64(x), "e5m2")
+    np.testing.assert_array_equal(u8(r.data), qr)
+    np.testing.assert_array_equal(u8(r.scale_plain()), sr)
+    np.testing.assert_array_equal(u8(c.data), qc)
+    np.testing.assert_array_equal(u8(c.scale_plain()), sc)
+
+
+def test_permute_quantize_e5m2(gpu_lib):
+    """The gathered path (dY of the backward): rowwise along H, colwise per segment."""
+    cfg = wl.CONFIGS["tiny"]
+    idx, probs = wl.make_routing(cfg)
+    x = wl.make_activations(cfg)
+    out = gpu_lib.moe_permute(idx.cuda(), probs.cuda(), cfg.E)
+    cap = gpu_lib.mxmoe_rows_capacity(cfg.T, cfg.k, cfg.E)
+    r, c = gpu_lib.mxfp8_quantize(x.cuda(), row_gather=out["token_of_row"], nrows=out["seg_off"][cfg.E:],
+                                  out_rows=cap, fmt=gpu_lib.FMT_E5M2)
+    torch.cuda.synchronize()
+    ro = omoe.route(idx.numpy(), cfg.E, align=SEG_ALIGN)
+    Mp = ro["Mp"]
+    Xp = omoe.permute_rows(f64(x), ro["token_of_row"])
+    qr, sr = omx.quantize_rowwise(Xp, "e5m2")
+    qc, sc = omoe.quantize_colwise_segments(Xp, ro["seg_off"], ro["m_splits"], "e5m2")
+    np.testing.assert_array_equal(u8(r.data)[:Mp], qr)
+    np.testing.assert_array_equal(u8(r.scale_plain())[:Mp], sr)
+    np.testing.assert_array_equal(u8(c.data)[:, :Mp], qc)
+    np.testing.assert_array_equal(u8(c.scale_plain())[:, :Mp // 32], sc)
+
+
+def test_mixed_format_grouped_gemm(gpu_lib, variant):
+    """C = dequant_E5M2(A) . dequant_E4M3(B_e)^T over ragged expert segments (fp32 out)."""
+    counts = [300, 0, 129, 640]
+    E, N, K = len(counts), 512, 384
+    idx = torch.tensor(sum(([e] * c for e, c in enumerate(counts)), []), dtype=torch.int32).reshape(-1, 1)
+    T = idx.shape[0]
+    out = gpu_lib.moe_permute(idx.cuda(), torch.ones((T, 1)).cuda(), E)
+    cap = gpu_lib.mxmoe_rows_capacity(T, 1, E)
+    x = wl.random_matrix(T, K, seed=5)
+    xr, _ = gpu_lib.mxfp8_quantize(x.cuda(), colwise=False, row_gather=out["token_of_row"],
+                                   nrows=out["seg_off"][E:], out_rows=cap, fmt=gpu_lib.FMT_E5M2)
+    W = wl.random_matrix(N, K, seed=6, std=0.05, batch=E)
+    wr, _ = gpu_lib.mxfp8_quantize(W.cuda(), colwise=False)
+    C = gpu_lib.grouped_gemm_mxfp8(xr, wr, out["seg_off"], E, N, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    r = omoe.route(idx.numpy(), E, align=SEG_ALIGN)
+    Xp = omoe.permute_rows(f64(x), r["token_of_row"])
+    Bq = np.stack([omx.fake_quant_rowwise(f64(W[e])) for e in range(E)])
+    want = omoe.grouped_gemm(omx.fake_quant_rowwise(Xp, "e5m2"), Bq, r["seg_off"])
+    got = f64(C)[:r["Mp"]]
+    for e in range(E):
+        s0, s1 = r["seg_off"][e], r["seg_off"][e] + r["m_splits"][e]
+        if s1 > s0:
+            assert rel_l2(got[s0:s1], want[s0:s1]) <= TOL_F32, e
+    # the E4M3-quantised product is much further away: the E5M2 codes and format bits were used
+    wrong = omoe.grouped_gemm(omx.fake_quant_rowwise(Xp), Bq, r["seg_off"])
+    assert rel_l2(got, wrong) > 10 * rel_l2(got, want)
+
+
+def test_mixed_format_wgrad(gpu_lib, variant):
+    """C[e] = dequant_E5M2(At)[:, seg_e] . dequant_E4M3(Bt)[:, seg_e]^T."""
+    counts = [300, 0, 129, 1, 640]
+    E, N, K2 = len(counts), 256, 512
+    idx = torch.tensor(sum(([e] * c for e, c in enumerate(counts)), []), dtype=torch.int32).reshape(-1, 1)
+    T = idx.shape[0]
+    out = gpu_lib.moe_permute(idx.cuda(), torch.ones((T, 1)).cuda(), E)
+    cap = gpu_lib.mxmoe_rows_capacity(T, 1, E)
+    a = wl.random_matrix(T, N, seed=31)
+    b = wl.random_matrix(T, K2, seed=32)
+    kw = dict(rowwise=False, row_gather=out["token_of_row"], nrows=out["seg_off"][E:], out_rows=cap)
+    _, ac = gpu_lib.mxfp8_quantize(a.cuda(), fmt=gpu_lib.FMT_E5M2, **kw)
+    _, bc = gpu_lib.mxfp8_quantize(b.cuda(), **kw)
+    C = torch.full((E, N, K2), float("nan"), device="cuda")
+    gpu_lib.grouped_gemm_mxfp8_wgrad(ac, bc, out["seg_off"], E, out=C)
+    torch.cuda.synchronize()
+    r = omoe.route(idx.numpy(), E, align=SEG_ALIGN)
+    Ap = omoe.permute_rows(f64(a), r["token_of_row"])
+    Bp = omoe.permute_rows(f64(b), r["token_of_row"])
+    Aq = omoe.fake_quant_colwise_segments(Ap, r["seg_off"], r["m_splits"], "e5m2")
+    Bq = omoe.fake_quant_colwise_segments(Bp, r["seg_off"], r["m_splits"])
+    want = omoe.grouped_gemm_wgrad(Aq.T, Bq.T, r["seg_off"])
+    got = f64(C)
+    for e in range(E):
+        if counts[e] == 0:
+            assert np.all(got[e] == 0), e
+        else:
+            assert rel_l2(got[e], want[e]) <= TOL_F32, e
+
+
+@pytest.mark.parametrize("name", ["tiny_fb", "small"])
+def test_fused_backward_e5m2_matches_oracle(gpu_lib, name):
+    cfg = wl.CONFIGS["small"] if name == "small" else wl.custom(
+        "tiny_fb", T=1024, H=256, F=512, E=4, k=2, seed=1)
+    d = wl.make_all(cfg)
+    dev = {k: (v.cuda() if v is not None else None) for k, v in d.items()}
+    layer = gpu_lib.GroupedMLP(cfg.T, cfg.k, cfg.E, cfg.H, cfg.F, grad_format="e5m2")
+    gpu_lib.mxmoe_clear_device_status()
+    layer.quantize_weights(dev["W1"], dev["W2"])
+    layer.forward(dev["x"], dev["topk_idx"], dev["probs"])
+    dx, dW1, dW2, dprobs = layer.backward(dev["dy"])
+    torch.cuda.synchronize()
+    st, where = gpu_lib.mxmoe_get_device_status()
+    assert st == 0, (st, where)
+    x, W1, W2, probs = f64(d["x"]), f64(d["W1"]), f64(d["W2"]), f64(d["probs"])
+    _, saved = omoe.mlp_fwd(x, d["topk_idx"].numpy(), probs, W1, W2)
+    g5 = omoe.mlp_bwd(f64(d["dy"]), saved, probs, W1, W2, grad_fmt="e5m2")
+    g4 = omoe.mlp_bwd(f64(d["dy"]), saved, probs, W1, W2)
+    got = dict(dx=f64(dx), dW1=f64(dW1), dW2=f64(dW2), dprobs=f64(dprobs))
+    errs = {k: rel_l2(v, g5[k]) for k, v in got.items()}
+    print(name, {k: f"{v:.2e}" for k, v in errs.items()})
+    for k, v in errs.items():
+        assert v <= TOL_E2E, (k, v)
+    # the E5M2 result is the E5M2 oracle's, not the E4M3 one's
+    assert rel_l2(got["dW2"], g5["dW2"]) < rel_l2(got["dW2"], g4["dW2"])
