@@ -58,7 +58,7 @@ def parse_args():
     p.add_argument("--cpu-rows", type=int, default=512, help="routed rows in the CPU oracle sample")
     p.add_argument("--cpu-fslice", type=int, default=1024, help="FFN columns in the CPU oracle sample")
     p.add_argument("--no-bf16-compare", action="store_true",
-                   help="skip the comparison timings (the bf16 layer's step, the E5M2-gradient backward)")
+                   help="skip the comparison timings (the bf16 layer's step, the alternative recipes)")
     return p.parse_args()
 
 
@@ -268,28 +268,46 @@ def config_json(cfg, world):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def time_grad_formats(cfg, layer, dy, dx, dW1, dW2, dprobs, stream, iters=5):
-    """The backward alone with E4M3 gradients (the headline) and with E5M2 gradients (the
-    variant), on the layer's saved forward; CUDA events, after two warm-up calls each."""
+def time_recipes(cfg, layer, W1, W2, x, idx, probs, dy, y, dx, dW1, dW2, dprobs, stream, steps):
+    """The same full step (weights quantised, forward, backward) under the layer's two
+    alternative recipes, beside the headline: E5M2 gradients (the backward's dY and dGU in
+    E5M2) and G / U recomputed in the backward instead of saved. CUDA events over `steps`
+    steps after two warm-up steps; the saved-activation bytes of each recipe."""
     import torch
 
     import mxfp8_grouped_gemm_moe_b200 as mx
+    lib = mx.load()
+    a = (cfg.T, cfg.k, cfg.E, cfg.H, cfg.F)
     out = {}
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for name, fmt in (("e4m3", mx.FMT_E4M3), ("e5m2", mx.FMT_E5M2)):
-        def bwd():
-            mx.grouped_mlp_bwd(dy, layer.saved, layer.wq, cfg.T, cfg.k, cfg.E, cfg.H, cfg.F, layer.ws, dx, dW1, dW2,
-                               dprobs, grad_format=fmt)
+    for name, recipe in (("grad_e5m2", mx.RECIPE_GRAD_E5M2), ("recompute_gu", mx.RECIPE_RECOMPUTE_GU)):
+        if recipe & mx.RECIPE_RECOMPUTE_GU:
+            saved = torch.empty(lib.grouped_mlp_saved_size_ex(*a, recipe), dtype=torch.uint8, device=x.device)
+            ws = torch.empty(lib.grouped_mlp_workspace_size_ex(*a, recipe), dtype=torch.uint8, device=x.device)
+        else:
+            saved, ws = layer.saved, layer.ws
+
+        def step():
+            mx.mxmoe_weights_quantize(W1, W2, out=layer.wq)
+            mx.grouped_mlp_fwd(x, idx, probs, layer.wq, cfg.E, cfg.F, saved, ws, y, recipe=recipe)
+            mx.grouped_mlp_bwd(dy, saved, layer.wq, *a, ws, dx, dW1, dW2, dprobs, recipe=recipe)
         for _ in range(2):
-            bwd()
+            step()
         torch.cuda.synchronize()
         e0.record(stream)
-        for _ in range(iters):
-            bwd()
+        for _ in range(steps):
+            step()
         e1.record(stream)
         torch.cuda.synchronize()
-        out[name + "_bwd_ms"] = e0.elapsed_time(e1) / iters
-    out["note"] = "backward only (permute+quantise dY, four GEMMs, combine); gradients dY and dGU in the named format"
+        ms = e0.elapsed_time(e1) / steps
+        out[name] = {"ms_per_step": ms, "tflops": cfg.fwdbwd_flops / (ms * 1e-3) / 1e12,
+                     "saved_bytes": lib.grouped_mlp_saved_size_ex(*a, recipe),
+                     "workspace_bytes": lib.grouped_mlp_workspace_size_ex(*a, recipe)}
+        del saved, ws
+    torch.cuda.empty_cache()
+    out["default_saved_bytes"] = lib.grouped_mlp_saved_size(*a)
+    out["note"] = ("same step as the headline under each recipe; tflops counts the headline's algorithmic FLOPs "
+                   "(the recompute's extra fc1 GEMM is not credited)")
     return out
 
 
@@ -412,10 +430,11 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
     mx.mxmoe_profile_disable()
     ms = max_over_ranks(dist, ms)
 
-    # ---- the backward with E5M2 gradients (the precision variant) beside the E4M3 one
-    grad_formats = None
+    # ---- the same step under the alternative recipes (E5M2 gradients; G / U recomputed)
+    recipes = None
     if rank == 0 and world == 1 and not args.no_bf16_compare:
-        grad_formats = time_grad_formats(cfg, layer, dy, dx, dW1, dW2, dprobs, stream)
+        recipes = time_recipes(cfg, layer, W1, W2, x, idx, probs, dy, y, dx, dW1, dW2, dprobs, stream,
+                               min(args.steps, 5))
 
     # ---- the same step on the bf16 layer: the 16-bit comparison point, timed on its own
     bf16_layer = None
@@ -586,8 +605,8 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
             "gemm_frac_of_measured_fp8": (18.0 * MHF) / (gemm_ms * 1e-3) / 1e12 / fp8_peak,
             "roofline": roofline, "roofline_hbm": roofline_hbm, "stages": stage_json,
             "gpu_launches": launches, "e2e": e2e, "clocks": clk, "router": router}
-    if grad_formats is not None:
-        line["grad_formats"] = grad_formats
+    if recipes is not None:
+        line["recipes"] = recipes
     if bf16_layer is not None:
         bf16_layer["speedup_mxfp8_over_bf16"] = bf16_layer["ms_per_step"] / ms
         bf16_layer["memory_bytes"] = layer_memory(cfg)

@@ -316,7 +316,9 @@ mxmoe_status mxmoe_weights_view(void* wq_dev, int32_t E, int32_t H, int32_t F, i
 #define MXMOE_SAVED_X_COLT_SF 6    /* e8m0, MMA layout */
 #define MXMOE_SAVED_Z_COLT 7       /* e4m3 [F, cap] */
 #define MXMOE_SAVED_Z_COLT_SF 8    /* e8m0, MMA layout */
-#define MXMOE_SAVED_GU 9           /* bf16 [cap, 2F] (gate | up) */
+#define MXMOE_SAVED_GU 9           /* bf16 [cap, 2F] (gate | up); 0 bytes with MXMOE_RECIPE_RECOMPUTE_GU */
+#define MXMOE_SAVED_X_ROW 10       /* e4m3 [cap, H], only with MXMOE_RECIPE_RECOMPUTE_GU (else 0 bytes) */
+#define MXMOE_SAVED_X_ROW_SF 11    /* e8m0, MMA layout, likewise */
 size_t grouped_mlp_saved_size(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F);
 int64_t grouped_mlp_saved_offset(int32_t field, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F);
 
@@ -356,17 +358,37 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
                              void* stream);
 
 /*
- * grouped_mlp_bwd_fmt -- grouped_mlp_bwd with the MXFP8 element format of the gradients
- * chosen: grad_format MXMOE_FMT_E4M3 (identical to grouped_mlp_bwd) or MXMOE_FMT_E5M2, the
- * gradient variant: dY and dGU are quantised to E5M2 (wider range, one mantissa bit fewer;
- * the pages name FP8 beside MXFP8 and fix no element format), every data- and
- * weight-gradient GEMM multiplies an E5M2 gradient by an E4M3 weight or activation.
- * Any other grad_format returns MXMOE_ERR_INVALID_ARG. Same buffers and sizes.
+ * Recipes of the fused layer (bit flags; 0 = the default above). The forward and the
+ * backward of one step take the same recipe; the saved-buffer and workspace sizes depend
+ * on it (query them with the _ex size functions).
+ *   MXMOE_RECIPE_GRAD_E5M2      the gradients dY and dGU are quantised to MXFP8 E5M2
+ *                               (wider range, one mantissa bit fewer; the pages name FP8
+ *                               beside MXFP8 and fix no element format): every backward
+ *                               GEMM multiplies an E5M2 gradient by an E4M3 weight or
+ *                               activation. Backward only.
+ *   MXMOE_RECIPE_RECOMPUTE_GU   the forward saves the rowwise MXFP8 copy of the permuted
+ *                               input (cap*H*(1+1/32) bytes) instead of the bf16 gate/up
+ *                               pre-activations (cap*2F*2 bytes), and the backward first
+ *                               recomputes G / U with the fc1 GEMM ("MoE-Training für
+ *                               biologische Grundmodelle optimieren": activation memory
+ *                               is the pressure MXFP8 and the fused kernel relieve). The
+ *                               recomputed G / U live in the workspace for the call.
+ * A recipe with any other bit set returns MXMOE_ERR_INVALID_ARG (sizes: 0 / -1).
  */
-mxmoe_status grouped_mlp_bwd_fmt(const void* dy_dev, const void* saved_dev, size_t saved_bytes, const void* wq_dev,
-                                 size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
-                                 int32_t grad_format, void* dx_dev, float* dW1_dev, float* dW2_dev, float* dprobs_dev,
-                                 void* ws_dev, size_t ws_bytes, void* stream);
+#define MXMOE_RECIPE_GRAD_E5M2 1
+#define MXMOE_RECIPE_RECOMPUTE_GU 2
+size_t grouped_mlp_saved_size_ex(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F, int32_t recipe);
+int64_t grouped_mlp_saved_offset_ex(int32_t field, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
+                                    int32_t recipe);
+size_t grouped_mlp_workspace_size_ex(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F, int32_t recipe);
+mxmoe_status grouped_mlp_fwd_ex(const void* x_dev, const int32_t* topk_idx_dev, const float* probs_dev,
+                                const void* wq_dev, size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H,
+                                int32_t F, int32_t recipe, void* y_dev, void* saved_dev, size_t saved_bytes,
+                                void* ws_dev, size_t ws_bytes, void* stream);
+mxmoe_status grouped_mlp_bwd_ex(const void* dy_dev, const void* saved_dev, size_t saved_bytes, const void* wq_dev,
+                                size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
+                                int32_t recipe, void* dx_dev, float* dW1_dev, float* dW2_dev, float* dprobs_dev,
+                                void* ws_dev, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------ bf16 grouped MLP */
 
@@ -422,6 +444,7 @@ mxmoe_status grouped_mlp_bf16_bwd(const void* dy_dev, const void* saved_dev, siz
 #define MXMOE_STAGE_QUANT 17         /* standalone mxfp8_quantize */
 #define MXMOE_STAGE_ROUTER 18        /* moe_router_topk */
 #define MXMOE_STAGE_ROUTER_BWD 19    /* moe_router_topk_bwd */
+#define MXMOE_STAGE_FC1_RECOMPUTE 20 /* backward: fc1 GEMM recomputing G / U (MXMOE_RECIPE_RECOMPUTE_GU) */
 
 /* Host-side stage timing, off by default: while enabled, every stage the library
  * enqueues is bracketed by two CUDA events recorded on that stage's stream (up to

@@ -26,9 +26,10 @@ STATUS_NAMES = {
 DTYPE_BF16, DTYPE_F32 = 0, 1
 SCALE_PLAIN, SCALE_MMA = 0, 1
 FMT_E4M3, FMT_E5M2 = 0, 1
+RECIPE_GRAD_E5M2, RECIPE_RECOMPUTE_GU = 1, 2
 _FMT = {"e4m3": FMT_E4M3, "e5m2": FMT_E5M2}
 SAVED_FIELDS = ["m_splits", "seg_off", "row_of_slot", "token_of_row", "prob_of_row",
-                "x_colT", "x_colT_sf", "z_colT", "z_colT_sf", "gu"]
+                "x_colT", "x_colT_sf", "z_colT", "z_colT_sf", "gu", "x_row", "x_row_sf"]
 
 
 class MxmoeError(RuntimeError):
@@ -75,8 +76,12 @@ _SIGNATURES = {
     "grouped_mlp_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32]),
     "grouped_mlp_fwd": (_I32, [_P, _P, _P, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _P, _P, _SZ, _P, _SZ, _P]),
     "grouped_mlp_bwd": (_I32, [_P, _P, _SZ, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
-    "grouped_mlp_bwd_fmt": (_I32, [_P, _P, _SZ, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ,
-                                   _P]),
+    "grouped_mlp_saved_size_ex": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32]),
+    "grouped_mlp_saved_offset_ex": (_I64, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
+    "grouped_mlp_workspace_size_ex": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32]),
+    "grouped_mlp_fwd_ex": (_I32, [_P, _P, _P, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P, _SZ, _P, _SZ, _P]),
+    "grouped_mlp_bwd_ex": (_I32, [_P, _P, _SZ, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ,
+                                  _P]),
     "mxmoe_weights_bf16_size": (_SZ, [_I32, _I32, _I32]),
     "mxmoe_weights_bf16_prepare": (_I32, [_P, _P, _I32, _I32, _I32, _P, _SZ, _P]),
     "grouped_mlp_bf16_saved_size": (_SZ, [_I32, _I32, _I32, _I32, _I32]),
@@ -93,7 +98,7 @@ _SIGNATURES = {
 STAGE_NAMES = {1: "route", 2: "quant_x", 3: "fc1_swiglu", 4: "fc2", 5: "combine", 6: "quant_w1", 7: "quant_w2",
                8: "quant_dy", 9: "fc2_dgrad_swiglu_bwd", 10: "dprob", 11: "fc2_wgrad", 12: "fc1_dgrad",
                13: "fc1_wgrad", 14: "combine_dx", 15: "gemm", 16: "wgrad", 17: "quant", 18: "router",
-               19: "router_bwd"}
+               19: "router_bwd", 20: "fc1_recompute"}
 
 
 def load(path: str | None = None):
@@ -319,24 +324,32 @@ class GroupedMLP:
     """Buffers for one layer shape; forward/backward call the fused C entry points.
 
     precision "mxfp8" (default) runs the MXFP8 layer (grouped_mlp_fwd / _bwd); "bf16" runs
-    the same steps on bf16 operands (grouped_mlp_bf16_fwd / _bwd). grad_format "e4m3"
-    (default) or "e5m2" picks the MXFP8 element format of the gradients (dY, dGU) of the
-    MXFP8 layer's backward."""
+    the same steps on bf16 operands (grouped_mlp_bf16_fwd / _bwd). For the MXFP8 layer,
+    grad_format "e4m3" (default) or "e5m2" picks the element format of the gradients (dY,
+    dGU), and recompute_gu=True saves the rowwise MXFP8 input instead of the bf16 gate/up
+    pre-activations and recomputes those in the backward (the recipe flags of
+    grouped_mlp_fwd_ex / _bwd_ex)."""
 
-    def __init__(self, T, k, E, H, F, device="cuda", precision="mxfp8", grad_format="e4m3"):
+    def __init__(self, T, k, E, H, F, device="cuda", precision="mxfp8", grad_format="e4m3", recompute_gu=False):
         if precision not in ("mxfp8", "bf16"):
             raise ValueError(f"unknown precision {precision!r}")
-        if grad_format not in _FMT or (precision == "bf16" and grad_format != "e4m3"):
-            raise ValueError(f"unsupported grad_format {grad_format!r} for precision {precision!r}")
-        self.grad_format = _FMT[grad_format]
+        if grad_format not in _FMT:
+            raise ValueError(f"unknown grad_format {grad_format!r}")
+        self.recipe = (RECIPE_GRAD_E5M2 if grad_format == "e5m2" else 0) | (RECIPE_RECOMPUTE_GU if recompute_gu else 0)
+        if precision == "bf16" and self.recipe:
+            raise ValueError("grad_format / recompute_gu apply to the MXFP8 layer")
         lib = load()
         self.T, self.k, self.E, self.H, self.F = T, k, E, H, F
         self.precision = precision
         self.cap = mxmoe_rows_capacity(T, k, E)
-        b16 = precision == "bf16"
-        saved = (lib.grouped_mlp_bf16_saved_size if b16 else lib.grouped_mlp_saved_size)(T, k, E, H, F)
-        ws = (lib.grouped_mlp_bf16_workspace_size if b16 else lib.grouped_mlp_workspace_size)(T, k, E, H, F)
-        wsz = (lib.mxmoe_weights_bf16_size if b16 else lib.mxmoe_weights_size)(E, H, F)
+        if precision == "bf16":
+            saved = lib.grouped_mlp_bf16_saved_size(T, k, E, H, F)
+            ws = lib.grouped_mlp_bf16_workspace_size(T, k, E, H, F)
+            wsz = lib.mxmoe_weights_bf16_size(E, H, F)
+        else:
+            saved = lib.grouped_mlp_saved_size_ex(T, k, E, H, F, self.recipe)
+            ws = lib.grouped_mlp_workspace_size_ex(T, k, E, H, F, self.recipe)
+            wsz = lib.mxmoe_weights_size(E, H, F)
         if saved == 0 or ws == 0:
             raise MxmoeError("grouped_mlp sizes", 2)
         self.saved = torch.empty(saved, dtype=torch.uint8, device=device)
@@ -350,15 +363,17 @@ class GroupedMLP:
         return mxmoe_weights_quantize(W1, W2, out=self.wq)
 
     def forward(self, x, topk_idx, probs, y=None):
-        fn = grouped_mlp_bf16_fwd if self.precision == "bf16" else grouped_mlp_fwd
-        return fn(x, topk_idx, probs, self.wq, self.E, self.F, self.saved, self.ws, y)
+        if self.precision == "bf16":
+            return grouped_mlp_bf16_fwd(x, topk_idx, probs, self.wq, self.E, self.F, self.saved, self.ws, y)
+        return grouped_mlp_fwd(x, topk_idx, probs, self.wq, self.E, self.F, self.saved, self.ws, y,
+                               recipe=self.recipe)
 
     def backward(self, dy, dx=None, dW1=None, dW2=None, dprobs=None):
         if self.precision == "bf16":
             return grouped_mlp_bf16_bwd(dy, self.saved, self.wq, self.T, self.k, self.E, self.H, self.F, self.ws,
                                         dx, dW1, dW2, dprobs)
         return grouped_mlp_bwd(dy, self.saved, self.wq, self.T, self.k, self.E, self.H, self.F, self.ws, dx, dW1,
-                               dW2, dprobs, grad_format=self.grad_format)
+                               dW2, dprobs, recipe=self.recipe)
 
     def saved_field(self, name, dtype=torch.uint8, count=None):
         """View of a named field of the saved buffer of the MXFP8 layer (inspection / tests)."""
@@ -366,7 +381,7 @@ class GroupedMLP:
             raise ValueError("saved_field describes the MXFP8 layer's saved buffer")
         lib = load()
         f = SAVED_FIELDS.index(name)
-        off = lib.grouped_mlp_saved_offset(f, self.T, self.k, self.E, self.H, self.F)
+        off = lib.grouped_mlp_saved_offset_ex(f, self.T, self.k, self.E, self.H, self.F, self.recipe)
         esz = torch.tensor([], dtype=dtype).element_size()
         return self.saved[off:off + count * esz].view(dtype)
 
@@ -383,32 +398,36 @@ def mxmoe_weights_bf16_prepare(W1, W2, out=None):
     return wb
 
 
-def grouped_mlp_fwd(x, topk_idx, probs, wq, E, F, saved, ws, y=None):
+def grouped_mlp_fwd(x, topk_idx, probs, wq, E, F, saved, ws, y=None, recipe=0):
     T, H = x.shape
     k = topk_idx.shape[1]
     y = y if y is not None else torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
-    st = load().grouped_mlp_fwd(_ptr(x), _ptr(topk_idx), _ptr(probs), _ptr(wq), wq.numel(), T, k, E, H, F, _ptr(y),
-                                _ptr(saved), saved.numel(), _ptr(ws), ws.numel(), _stream())
-    _check("grouped_mlp_fwd", st)
+    if recipe == 0:
+        st = load().grouped_mlp_fwd(_ptr(x), _ptr(topk_idx), _ptr(probs), _ptr(wq), wq.numel(), T, k, E, H, F,
+                                    _ptr(y), _ptr(saved), saved.numel(), _ptr(ws), ws.numel(), _stream())
+        _check("grouped_mlp_fwd", st)
+    else:
+        st = load().grouped_mlp_fwd_ex(_ptr(x), _ptr(topk_idx), _ptr(probs), _ptr(wq), wq.numel(), T, k, E, H, F,
+                                       recipe, _ptr(y), _ptr(saved), saved.numel(), _ptr(ws), ws.numel(), _stream())
+        _check("grouped_mlp_fwd_ex", st)
     return y
 
 
-def grouped_mlp_bwd(dy, saved, wq, T, k, E, H, F, ws, dx=None, dW1=None, dW2=None, dprobs=None,
-                    grad_format=FMT_E4M3):
+def grouped_mlp_bwd(dy, saved, wq, T, k, E, H, F, ws, dx=None, dW1=None, dW2=None, dprobs=None, recipe=0):
     dev = dy.device
     dx = dx if dx is not None else torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     dW1 = dW1 if dW1 is not None else torch.empty((E, 2 * F, H), dtype=torch.float32, device=dev)
     dW2 = dW2 if dW2 is not None else torch.empty((E, H, F), dtype=torch.float32, device=dev)
     dprobs = dprobs if dprobs is not None else torch.empty((T, k), dtype=torch.float32, device=dev)
-    if grad_format == FMT_E4M3:
+    if recipe == 0:
         st = load().grouped_mlp_bwd(_ptr(dy), _ptr(saved), saved.numel(), _ptr(wq), wq.numel(), T, k, E, H, F,
                                     _ptr(dx), _ptr(dW1), _ptr(dW2), _ptr(dprobs), _ptr(ws), ws.numel(), _stream())
         _check("grouped_mlp_bwd", st)
     else:
-        st = load().grouped_mlp_bwd_fmt(_ptr(dy), _ptr(saved), saved.numel(), _ptr(wq), wq.numel(), T, k, E, H, F,
-                                        grad_format, _ptr(dx), _ptr(dW1), _ptr(dW2), _ptr(dprobs), _ptr(ws),
-                                        ws.numel(), _stream())
-        _check("grouped_mlp_bwd_fmt", st)
+        st = load().grouped_mlp_bwd_ex(_ptr(dy), _ptr(saved), saved.numel(), _ptr(wq), wq.numel(), T, k, E, H, F,
+                                       recipe, _ptr(dx), _ptr(dW1), _ptr(dW2), _ptr(dprobs), _ptr(ws), ws.numel(),
+                                       _stream())
+        _check("grouped_mlp_bwd_ex", st)
     return dx, dW1, dW2, dprobs
 
 

@@ -59,12 +59,18 @@ WeightsLayout weights_layout(int64_t E, int64_t H, int64_t F) {
   return L;
 }
 
+bool valid_recipe(int32_t recipe) { return (recipe & ~(MXMOE_RECIPE_GRAD_E5M2 | MXMOE_RECIPE_RECOMPUTE_GU)) == 0; }
+bool recomputes_gu(int32_t recipe) { return (recipe & MXMOE_RECIPE_RECOMPUTE_GU) != 0; }
+
 struct SavedLayout {
-  size_t off[10];
+  size_t off[12];
   size_t total;
 };
-SavedLayout saved_layout(int64_t T, int64_t k, int64_t E, int64_t H, int64_t F) {
+// With MXMOE_RECIPE_RECOMPUTE_GU the gate/up pre-activations are not saved (zero bytes)
+// and the rowwise MXFP8 copy of the permuted input is, for the backward's recompute.
+SavedLayout saved_layout(int64_t T, int64_t k, int64_t E, int64_t H, int64_t F, int32_t recipe = 0) {
   const int64_t cap = rows_cap(T, k, E);
+  const bool rc = recomputes_gu(recipe);
   SavedLayout L;
   Carver cv;
   L.off[MXMOE_SAVED_M_SPLITS] = cv.take(E * 4);
@@ -76,7 +82,9 @@ SavedLayout saved_layout(int64_t T, int64_t k, int64_t E, int64_t H, int64_t F) 
   L.off[MXMOE_SAVED_X_COLT_SF] = cv.take(H * cap / 32);
   L.off[MXMOE_SAVED_Z_COLT] = cv.take(F * cap);
   L.off[MXMOE_SAVED_Z_COLT_SF] = cv.take(F * cap / 32);
-  L.off[MXMOE_SAVED_GU] = cv.take(cap * 2 * F * 2);
+  L.off[MXMOE_SAVED_GU] = cv.take(rc ? 0 : cap * 2 * F * 2);
+  L.off[MXMOE_SAVED_X_ROW] = cv.take(rc ? cap * H : 0);
+  L.off[MXMOE_SAVED_X_ROW_SF] = cv.take(rc ? cap * H / 32 : 0);
   L.total = cv.off;
   return L;
 }
@@ -99,10 +107,10 @@ FwdWs fwd_ws(int64_t T, int64_t k, int64_t E, int64_t H, int64_t F) {
 }
 
 struct BwdWs {
-  size_t dy_row, dy_row_sf, dy_colT, dy_colT_sf, dgu_row, dgu_row_sf, dgu_colT, dgu_colT_sf, dprob_part, dx_perm,
+  size_t dy_row, dy_row_sf, dy_colT, dy_colT_sf, dgu_row, dgu_row_sf, dgu_colT, dgu_colT_sf, dprob_part, dx_perm, gu,
       total;
 };
-BwdWs bwd_ws(int64_t T, int64_t k, int64_t E, int64_t H, int64_t F) {
+BwdWs bwd_ws(int64_t T, int64_t k, int64_t E, int64_t H, int64_t F, int32_t recipe = 0) {
   const int64_t cap = rows_cap(T, k, E);
   BwdWs w;
   Carver cv;
@@ -116,6 +124,7 @@ BwdWs bwd_ws(int64_t T, int64_t k, int64_t E, int64_t H, int64_t F) {
   w.dgu_colT_sf = cv.take(2 * F * cap / 32);
   w.dprob_part = cv.take(cap * (F / 128) * 4);
   w.dx_perm = cv.take(cap * H * 2);
+  w.gu = cv.take(recomputes_gu(recipe) ? cap * 2 * F * 2 : 0);  // recomputed G / U (bf16)
   w.total = cv.off;
   return w;
 }
@@ -459,33 +468,55 @@ mxmoe_status mxmoe_weights_quantize(const void* W1_dev, const void* W2_dev, int3
 }
 
 size_t grouped_mlp_saved_size(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F) {
-  return saved_layout(T, k, E, H, F).total;
+  return grouped_mlp_saved_size_ex(T, k, E, H, F, 0);
+}
+size_t grouped_mlp_saved_size_ex(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F, int32_t recipe) {
+  if (!valid_recipe(recipe)) return 0;
+  return saved_layout(T, k, E, H, F, recipe).total;
 }
 
 int64_t grouped_mlp_saved_offset(int32_t field, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F) {
-  if (field < 0 || field > 9) return -1;
-  return (int64_t)saved_layout(T, k, E, H, F).off[field];
+  return grouped_mlp_saved_offset_ex(field, T, k, E, H, F, 0);
+}
+int64_t grouped_mlp_saved_offset_ex(int32_t field, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
+                                    int32_t recipe) {
+  if (field < 0 || field > 11 || !valid_recipe(recipe)) return -1;
+  return (int64_t)saved_layout(T, k, E, H, F, recipe).off[field];
 }
 
 size_t grouped_mlp_workspace_size(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F) {
-  return std::max(fwd_ws(T, k, E, H, F).total, bwd_ws(T, k, E, H, F).total);
+  return grouped_mlp_workspace_size_ex(T, k, E, H, F, 0);
+}
+size_t grouped_mlp_workspace_size_ex(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F, int32_t recipe) {
+  if (!valid_recipe(recipe)) return 0;
+  return std::max(fwd_ws(T, k, E, H, F).total, bwd_ws(T, k, E, H, F, recipe).total);
 }
 
 mxmoe_status grouped_mlp_fwd(const void* x_dev, const int32_t* topk_idx_dev, const float* probs_dev,
                              const void* wq_dev, size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H,
                              int32_t F, void* y_dev, void* saved_dev, size_t saved_bytes, void* ws_dev,
                              size_t ws_bytes, void* stream) {
+  return grouped_mlp_fwd_ex(x_dev, topk_idx_dev, probs_dev, wq_dev, wq_bytes, T, k, E, H, F, 0, y_dev, saved_dev,
+                            saved_bytes, ws_dev, ws_bytes, stream);
+}
+
+mxmoe_status grouped_mlp_fwd_ex(const void* x_dev, const int32_t* topk_idx_dev, const float* probs_dev,
+                                const void* wq_dev, size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H,
+                                int32_t F, int32_t recipe, void* y_dev, void* saved_dev, size_t saved_bytes,
+                                void* ws_dev, size_t ws_bytes, void* stream) {
+  if (!valid_recipe(recipe)) return MXMOE_ERR_INVALID_ARG;
   if (!valid_mlp_shape(T, k, E, H, F)) return MXMOE_ERR_UNSUPPORTED_SHAPE;
   if (!wq_dev || !saved_dev || !ws_dev || !aligned16(wq_dev) || !aligned16(saved_dev) || !aligned16(ws_dev))
     return MXMOE_ERR_INVALID_ARG;
   if (T > 0 && (!x_dev || !topk_idx_dev || !probs_dev || !y_dev || !aligned16(x_dev) || !aligned16(y_dev)))
     return MXMOE_ERR_INVALID_ARG;
-  if (wq_bytes < mxmoe_weights_size(E, H, F) || saved_bytes < grouped_mlp_saved_size(T, k, E, H, F) ||
-      ws_bytes < grouped_mlp_workspace_size(T, k, E, H, F))
+  if (wq_bytes < mxmoe_weights_size(E, H, F) || saved_bytes < grouped_mlp_saved_size_ex(T, k, E, H, F, recipe) ||
+      ws_bytes < grouped_mlp_workspace_size_ex(T, k, E, H, F, recipe))
     return MXMOE_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = S(stream);
   const int64_t cap = rows_cap(T, k, E);
-  const SavedLayout SL = saved_layout(T, k, E, H, F);
+  const bool rc = recomputes_gu(recipe);
+  const SavedLayout SL = saved_layout(T, k, E, H, F, recipe);
   const FwdWs W = fwd_ws(T, k, E, H, F);
   const WeightsLayout WL = weights_layout(E, H, F);
   uint8_t* sv = reinterpret_cast<uint8_t*>(saved_dev);
@@ -505,8 +536,10 @@ mxmoe_status grouped_mlp_fwd(const void* x_dev, const int32_t* topk_idx_dev, con
   }
   if (e != cudaSuccess) return MXMOE_ERR_CUDA;
   if (T == 0) return MXMOE_OK;
-  // 2. permute + quantise x (rowwise for fc1, colwise saved for fc1 wgrad)
-  mxmoe_mxfp8 x_row = mk(ws, W.x_row, W.x_row_sf, cap, H);
+  // 2. permute + quantise x (rowwise for fc1 -- saved when the backward recomputes G / U --
+  // and colwise, saved for fc1 wgrad)
+  mxmoe_mxfp8 x_row = rc ? mk(sv, SL.off[MXMOE_SAVED_X_ROW], SL.off[MXMOE_SAVED_X_ROW_SF], cap, H)
+                         : mk(ws, W.x_row, W.x_row_sf, cap, H);
   mxmoe_mxfp8 x_col = mk(sv, SL.off[MXMOE_SAVED_X_COLT], SL.off[MXMOE_SAVED_X_COLT_SF], H, cap);
   mxmoe_status s;
   {
@@ -514,7 +547,7 @@ mxmoe_status grouped_mlp_fwd(const void* x_dev, const int32_t* topk_idx_dev, con
     s = mxfp8_quantize(x_dev, MXMOE_DTYPE_BF16, 1, T, H, tor, seg_off + E, cap, &x_row, &x_col, stream);
   }
   if (s != MXMOE_OK) return s;
-  // 3. fc1 + SwiGLU x prob -> Z (MXFP8 row + colT), G/U saved
+  // 3. fc1 + SwiGLU x prob -> Z (MXFP8 row + colT), G/U saved unless recomputed
   mxmoe_mxfp8 w1r = mk(wq, WL.d[0], WL.s[0], WL.rows[0], WL.cols[0]);
   GemmArgs g = gemm_base(kModeSwigluFwd, x_row, w1r, seg_off, E);
   g.K = H;
@@ -526,7 +559,7 @@ mxmoe_status grouped_mlp_fwd(const void* x_dev, const int32_t* topk_idx_dev, con
   g.z_row_sf = ws + W.z_row_sf;
   g.z_colT = sv + SL.off[MXMOE_SAVED_Z_COLT];
   g.z_colT_sf = sv + SL.off[MXMOE_SAVED_Z_COLT_SF];
-  g.gu = reinterpret_cast<uint16_t*>(sv + SL.off[MXMOE_SAVED_GU]);
+  g.gu = rc ? nullptr : reinterpret_cast<uint16_t*>(sv + SL.off[MXMOE_SAVED_GU]);
   {
     StageScope sc(MXMOE_STAGE_FC1_SWIGLU, st);
     e = launch_gemm(g, st);
@@ -549,28 +582,30 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
                              size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F, void* dx_dev,
                              float* dW1_dev, float* dW2_dev, float* dprobs_dev, void* ws_dev, size_t ws_bytes,
                              void* stream) {
-  return grouped_mlp_bwd_fmt(dy_dev, saved_dev, saved_bytes, wq_dev, wq_bytes, T, k, E, H, F, MXMOE_FMT_E4M3, dx_dev,
-                             dW1_dev, dW2_dev, dprobs_dev, ws_dev, ws_bytes, stream);
+  return grouped_mlp_bwd_ex(dy_dev, saved_dev, saved_bytes, wq_dev, wq_bytes, T, k, E, H, F, 0, dx_dev, dW1_dev,
+                            dW2_dev, dprobs_dev, ws_dev, ws_bytes, stream);
 }
 
-mxmoe_status grouped_mlp_bwd_fmt(const void* dy_dev, const void* saved_dev, size_t saved_bytes, const void* wq_dev,
-                                 size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
-                                 int32_t grad_format, void* dx_dev, float* dW1_dev, float* dW2_dev, float* dprobs_dev,
-                                 void* ws_dev, size_t ws_bytes, void* stream) {
-  if (grad_format != MXMOE_FMT_E4M3 && grad_format != MXMOE_FMT_E5M2) return MXMOE_ERR_INVALID_ARG;
+mxmoe_status grouped_mlp_bwd_ex(const void* dy_dev, const void* saved_dev, size_t saved_bytes, const void* wq_dev,
+                                size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
+                                int32_t recipe, void* dx_dev, float* dW1_dev, float* dW2_dev, float* dprobs_dev,
+                                void* ws_dev, size_t ws_bytes, void* stream) {
+  if (!valid_recipe(recipe)) return MXMOE_ERR_INVALID_ARG;
+  const int32_t grad_format = (recipe & MXMOE_RECIPE_GRAD_E5M2) ? MXMOE_FMT_E5M2 : MXMOE_FMT_E4M3;
   if (!valid_mlp_shape(T, k, E, H, F)) return MXMOE_ERR_UNSUPPORTED_SHAPE;
   if (!wq_dev || !saved_dev || !ws_dev || !dW1_dev || !dW2_dev || !aligned16(wq_dev) || !aligned16(saved_dev) ||
       !aligned16(ws_dev) || !aligned16(dW1_dev) || !aligned16(dW2_dev))
     return MXMOE_ERR_INVALID_ARG;
   if (T > 0 && (!dy_dev || !dx_dev || !dprobs_dev || !aligned16(dy_dev) || !aligned16(dx_dev)))
     return MXMOE_ERR_INVALID_ARG;
-  if (wq_bytes < mxmoe_weights_size(E, H, F) || saved_bytes < grouped_mlp_saved_size(T, k, E, H, F) ||
-      ws_bytes < grouped_mlp_workspace_size(T, k, E, H, F))
+  if (wq_bytes < mxmoe_weights_size(E, H, F) || saved_bytes < grouped_mlp_saved_size_ex(T, k, E, H, F, recipe) ||
+      ws_bytes < grouped_mlp_workspace_size_ex(T, k, E, H, F, recipe))
     return MXMOE_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = S(stream);
   const int64_t cap = rows_cap(T, k, E);
-  const SavedLayout SL = saved_layout(T, k, E, H, F);
-  const BwdWs W = bwd_ws(T, k, E, H, F);
+  const bool rc = recomputes_gu(recipe);
+  const SavedLayout SL = saved_layout(T, k, E, H, F, recipe);
+  const BwdWs W = bwd_ws(T, k, E, H, F, recipe);
   const WeightsLayout WL = weights_layout(E, H, F);
   uint8_t* sv = reinterpret_cast<uint8_t*>(const_cast<void*>(saved_dev));
   uint8_t* ws = reinterpret_cast<uint8_t*>(ws_dev);
@@ -589,6 +624,22 @@ mxmoe_status grouped_mlp_bwd_fmt(const void* dy_dev, const void* saved_dev, size
     s = mxfp8_quantize(dy_dev, MXMOE_DTYPE_BF16, 1, T, H, tor, seg_off + E, cap, &dy_row, &dy_col, stream);
     if (s != MXMOE_OK) return s;
   }
+  // 1b. G / U recomputed from the saved rowwise x (the fc1 GEMM again, epilogue writing
+  // only G / U) when the forward did not save them
+  if (rc && T > 0) {
+    mxmoe_mxfp8 x_row = mk(sv, SL.off[MXMOE_SAVED_X_ROW], SL.off[MXMOE_SAVED_X_ROW_SF], cap, H);
+    mxmoe_mxfp8 w1r = mk(wq, WL.d[0], WL.s[0], WL.rows[0], WL.cols[0]);
+    GemmArgs g = gemm_base(kModeSwigluFwd, x_row, w1r, seg_off, E);
+    g.K = H;
+    g.F = F;
+    g.N = 2 * (int64_t)F;
+    g.rows_cap = cap;
+    g.prob_of_row = por;
+    g.gu = reinterpret_cast<uint16_t*>(ws + W.gu);
+    StageScope sc(MXMOE_STAGE_FC1_RECOMPUTE, st);
+    if (launch_gemm(g, st) != cudaSuccess) return MXMOE_ERR_CUDA;
+  }
+  const uint16_t* gu = reinterpret_cast<const uint16_t*>(rc ? ws + W.gu : sv + SL.off[MXMOE_SAVED_GU]);
   // 2. fc2 dgrad + SwiGLU/prob backward -> dGU (MXFP8 row + colT), dprob partials
   mxmoe_mxfp8 w2c = mk(wq, WL.d[3], WL.s[3], WL.rows[3], WL.cols[3]);
   {
@@ -598,7 +649,7 @@ mxmoe_status grouped_mlp_bwd_fmt(const void* dy_dev, const void* saved_dev, size
     g.F = F;
     g.rows_cap = cap;
     g.prob_of_row = por;
-    g.gu_in = reinterpret_cast<const uint16_t*>(sv + SL.off[MXMOE_SAVED_GU]);
+    g.gu_in = gu;
     g.dgu_row = ws + W.dgu_row;
     g.dgu_row_sf = ws + W.dgu_row_sf;
     g.dgu_colT = ws + W.dgu_colT;

@@ -677,19 +677,23 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
         ptx::tmem_wait_ld();
         release_accumulator<PAIR>(bar_acc_empty, acc_empty_leader, lane);
         uint8_t* stg8 = reinterpret_cast<uint8_t*>(stg);
-        // G and U as bf16 for the backward: two 32-row x 128-byte boxes (128-byte swizzle)
-        staging_acquire(lane);
+        // G and U as bf16 for the backward: two 32-row x 128-byte boxes (128-byte swizzle);
+        // skipped when the forward does not save them (the backward recomputes them)
+        if (g.gu != nullptr) {
+          staging_acquire(lane);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          out_box_put(stg8, lane, j, pack8_bf16(gr, 8 * j));
-          out_box_put(stg8 + 4096, lane, j, pack8_bf16(ur, 8 * j));
+          for (int j = 0; j < 8; ++j) {
+            out_box_put(stg8, lane, j, pack8_bf16(gr, 8 * j));
+            out_box_put(stg8 + 4096, lane, j, pack8_bf16(ur, 8 * j));
+          }
+          staging_publish();
+          if (lane == 0) {
+            ptx::tma_store_2d(&tmE, stg8, (int32_t)f0, (int32_t)mrow0);
+            ptx::tma_store_2d(&tmE, stg8 + 4096, (int32_t)(F + f0), (int32_t)mrow0);
+            ptx::bulk_commit_group();
+          }
         }
-        staging_publish();
-        if (lane == 0) {
-          ptx::tma_store_2d(&tmE, stg8, (int32_t)f0, (int32_t)mrow0);
-          ptx::tma_store_2d(&tmE, stg8 + 4096, (int32_t)(F + f0), (int32_t)mrow0);
-          ptx::bulk_commit_group();
-        }
+        if (g.z_row == nullptr) continue;  // recompute of G / U for the backward: no Z
         float zf[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i) zf[i] = silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]) * p;
@@ -1015,9 +1019,13 @@ static cudaError_t launch_variant(const GemmArgs& g, cudaStream_t st) {
       if (!make_out_map(&m.c, g.c, g.a_rows, g.N, g.ldc, g.c_dtype == MXMOE_DTYPE_F32)) return cudaErrorInvalidValue;
       return launch_mode<kModeStore, PAIR>(m, g, (g.a_rows / TM) * (g.N / BN), st);
     case kModeSwigluFwd:
-      if (!make_codes32_map(&m.c, g.z_row, g.rows_cap, g.F) || !make_codes32_map(&m.d, g.z_colT, g.F, g.rows_cap) ||
-          !make_out_map(&m.e, g.gu, g.rows_cap, 2 * g.F, 2 * g.F, false))
+      // Z (rows + colT) and the saved G / U are each optional, not both absent
+      if ((g.z_row == nullptr) != (g.z_colT == nullptr) || (g.z_row == nullptr && g.gu == nullptr))
         return cudaErrorInvalidValue;
+      if (g.z_row && (!make_codes32_map(&m.c, g.z_row, g.rows_cap, g.F) ||
+                      !make_codes32_map(&m.d, g.z_colT, g.F, g.rows_cap)))
+        return cudaErrorInvalidValue;
+      if (g.gu && !make_out_map(&m.e, g.gu, g.rows_cap, 2 * g.F, 2 * g.F, false)) return cudaErrorInvalidValue;
       return launch_mode<kModeSwigluFwd, PAIR>(m, g, (g.a_rows / TM) * (g.F / 128), st);
     case kModeSwigluBwd:
       if (!make_codes32_map(&m.c, g.dgu_row, g.rows_cap, 2 * g.F) ||

@@ -63,7 +63,7 @@ def test_sizes_are_host_only(lib):
     assert s >= cap * (4096 + 14336) * (1 + 1 / 32) + cap * 2 * 14336 * 2
     offs = [lib.grouped_mlp_saved_offset(f, 8192, 2, 8, 4096, 14336) for f in range(10)]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
-    assert lib.grouped_mlp_saved_offset(10, 1, 1, 1, 256, 256) == -1
+    assert lib.grouped_mlp_saved_offset(12, 1, 1, 1, 256, 256) == -1
 
 
 def test_host_argument_errors_enqueue_nothing(lib):
@@ -116,9 +116,19 @@ def test_host_argument_errors_enqueue_nothing(lib):
                                16, S) == 3
     assert lib.grouped_mlp_bwd(fake, fake, 1 << 40, fake, 1 << 40, 16, 2, 4, 256, 512, fake, bad, fake, fake,
                                fake, 1 << 40, S) == 1
-    # gradient element format: only E4M3 (0) and E5M2 (1)
-    assert lib.grouped_mlp_bwd_fmt(fake, fake, 1 << 40, fake, 1 << 40, 16, 2, 4, 256, 512, 2, fake, fake, fake, fake,
-                                   fake, 1 << 40, S) == 1
+    # recipe flags: only MXMOE_RECIPE_GRAD_E5M2 | MXMOE_RECIPE_RECOMPUTE_GU
+    assert lib.grouped_mlp_bwd_ex(fake, fake, 1 << 40, fake, 1 << 40, 16, 2, 4, 256, 512, 4, fake, fake, fake, fake,
+                                  fake, 1 << 40, S) == 1
+    assert lib.grouped_mlp_fwd_ex(fake, fake, fake, fake, 1 << 40, 16, 2, 4, 256, 512, 8, fake, fake, 1 << 40, fake,
+                                  1 << 40, S) == 1
+    assert lib.grouped_mlp_saved_size_ex(16, 2, 4, 256, 512, 4) == 0
+    # the recompute recipe saves the rowwise input instead of G / U: smaller saved buffer,
+    # larger workspace (G / U recomputed there)
+    a = (4096, 2, 8, 1024, 2816)
+    assert lib.grouped_mlp_saved_size_ex(*a, 2) < lib.grouped_mlp_saved_size(*a)
+    assert lib.grouped_mlp_workspace_size_ex(*a, 2) > lib.grouped_mlp_workspace_size(*a)
+    assert lib.grouped_mlp_saved_size_ex(*a, 1) == lib.grouped_mlp_saved_size(*a)
+    assert lib.grouped_mlp_saved_offset_ex(10, *a, 0) == lib.grouped_mlp_saved_offset_ex(11, *a, 0)  # empty x_row
     # an MXFP8 descriptor with an unknown element format; row / colT formats that disagree
     m_bad_fmt = mx._MX(1 << 20, 1 << 20, 64, 64, 0, 3)
     assert lib.mxfp8_quantize(fake, 0, 1, 64, 64, None, None, 64, ctypes.byref(m_bad_fmt), None, S) == 1

@@ -1,6 +1,7 @@
-"""GPU parity of the E5M2-gradient variant with the oracle: the E5M2 quantiser (bytes and
-scales bit-exact), grouped GEMMs that multiply an E5M2 operand by an E4M3 one (both
-kernel variants), and the fused backward with E5M2 gradients (rel-L2 <= 2e-2)."""
+"""GPU parity of the layer's alternative recipes with the oracle: E5M2 gradients (the E5M2
+quantiser, bytes and scales bit-exact; grouped GEMMs that multiply an E5M2 operand by an
+E4M3 one, both kernel variants; the fused backward, rel-L2 <= 2e-2) and G / U recomputed in
+the backward instead of saved (bit-identical to the saving recipe)."""
 import numpy as np
 import pytest
 import torch
@@ -146,3 +147,38 @@ def test_fused_backward_e5m2_matches_oracle(gpu_lib, name):
         assert v <= TOL_E2E, (k, v)
     # the E5M2 result is the E5M2 oracle's, not the E4M3 one's
     assert rel_l2(got["dW2"], g5["dW2"]) < rel_l2(got["dW2"], g4["dW2"])
+
+
+def _layer_run(gpu_lib, cfg, dev, **kw):
+    layer = gpu_lib.GroupedMLP(cfg.T, cfg.k, cfg.E, cfg.H, cfg.F, **kw)
+    layer.quantize_weights(dev["W1"], dev["W2"])
+    y = layer.forward(dev["x"], dev["topk_idx"], dev["probs"])
+    g = layer.backward(dev["dy"])
+    torch.cuda.synchronize()
+    return layer, y, g
+
+
+@pytest.mark.parametrize("grad_format", ["e4m3", "e5m2"])
+def test_recompute_gu_is_bit_identical(gpu_lib, grad_format):
+    """Recomputing G / U in the backward (instead of saving them) runs the same fc1 GEMM on
+    the same operands: every output equals the saving recipe's byte for byte, while the
+    saved buffer shrinks by the bf16 G / U it no longer holds."""
+    cfg = wl.CONFIGS["small"]
+    d = wl.make_all(cfg)
+    dev = {k: (v.cuda() if v is not None else None) for k, v in d.items()}
+    gpu_lib.mxmoe_clear_device_status()
+    base, y0, g0 = _layer_run(gpu_lib, cfg, dev, grad_format=grad_format)
+    rc, y1, g1 = _layer_run(gpu_lib, cfg, dev, grad_format=grad_format, recompute_gu=True)
+    st, where = gpu_lib.mxmoe_get_device_status()
+    assert st == 0, (st, where)
+    assert torch.equal(y0, y1)
+    for a, b in zip(g0, g1):
+        assert torch.equal(a, b)
+    # the saved rowwise input equals the forward's fc1 operand: the oracle's rowwise codes
+    cap = rc.cap
+    Mp = omoe.route(d["topk_idx"].numpy(), cfg.E, align=SEG_ALIGN)
+    Xp = omoe.permute_rows(f64(d["x"]), Mp["token_of_row"])
+    qr, _ = omx.quantize_rowwise(Xp)
+    codes = rc.saved_field("x_row", torch.uint8, cap * cfg.H).view(cap, cfg.H)
+    np.testing.assert_array_equal(u8(codes)[:Mp["Mp"]], qr)
+    assert rc.saved.numel() < base.saved.numel() - cap * 2 * cfg.F * 2 + cap * cfg.H * 1.04
