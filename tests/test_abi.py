@@ -26,7 +26,7 @@ def lib():
     return mx.load()
 
 
-def test_header_declares_the_north_star_entry_points():
+def test_header_declares_the_layer_entry_points():
     names = _declared_functions()
     for n in ["moe_permute", "moe_unpermute", "mxfp8_quantize", "grouped_gemm_mxfp8", "grouped_gemm_mxfp8_wgrad",
               "grouped_mlp_fwd", "grouped_mlp_bwd", "mxmoe_weights_quantize"]:
@@ -141,3 +141,21 @@ def test_host_argument_errors_enqueue_nothing(lib):
     assert lib.grouped_mlp_bf16_bwd(fake, fake, 1 << 40, fake, 16, 16, 2, 4, 256, 512, fake, fake, fake, fake,
                                     fake, 1 << 40, S) == 3
     assert lib.mxmoe_weights_bf16_prepare(fake, fake, 2, 256, 384, fake, 1 << 40, S) == 2
+
+
+def test_layer_arguments_checked_before_allocation(lib):
+    """GroupedMLP rejects an unknown precision or a recipe the bf16 layer does not have,
+    before any device memory is touched."""
+    import mxfp8_grouped_gemm_moe_b200 as mx
+    with pytest.raises(ValueError):
+        mx.GroupedMLP(16, 2, 4, 256, 512, device="cpu", precision="fp4")
+    with pytest.raises(ValueError):
+        mx.GroupedMLP(16, 2, 4, 256, 512, device="cpu", precision="bf16", grad_format="e5m2")
+    with pytest.raises(ValueError):
+        mx.GroupedMLP(16, 2, 4, 256, 512, device="cpu", grad_format="e3m4")
+    # sizes of a valid layer on the host (no kernel runs): the recompute recipe's saved
+    # buffer holds the rowwise input instead of G / U
+    a = mx.GroupedMLP(64, 2, 4, 256, 512, device="cpu")
+    b = mx.GroupedMLP(64, 2, 4, 256, 512, device="cpu", recompute_gu=True)
+    assert a.recipe == 0 and b.recipe == mx.RECIPE_RECOMPUTE_GU
+    assert b.saved.numel() < a.saved.numel()

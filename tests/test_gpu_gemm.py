@@ -13,7 +13,7 @@ from oracle import mxfp8 as omx
 from tests.util import f64, rel_l2, SEG_ALIGN
 
 pytestmark = pytest.mark.gpu
-TOL_GEMM = 5e-3   # bf16 output: the spec bar per GEMM stage
+TOL_GEMM = 5e-3   # bf16 output: the stated bar per GEMM stage
 TOL_F32 = 5e-4    # fp32 output: fp32 accumulation over K <= 4096 terms stays well inside K * 2^-24
 
 

@@ -1,6 +1,6 @@
 """GPU parity of the fused grouped-MLP forward and backward with the oracle.
 
-Bar (the benchmark spec): relative L2 <= 2e-2 for y, dx, dW1, dW2, dprobs against the
+Bar (the stated end-to-end tolerance): relative L2 <= 2e-2 for y, dx, dW1, dW2, dprobs against the
 quantisation-emulating fp64 oracle; the routing maps saved by the forward are
 bit-exact."""
 import numpy as np
