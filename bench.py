@@ -56,7 +56,7 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=512, help="routed rows in the CPU oracle sample")
-    p.add_argument("--cpu-fslice", type=int, default=1024, help="FFN columns in the CPU oracle sample")
+    p.add_argument("--cpu-fslice", type=int, default=2048, help="FFN columns in the CPU oracle sample")
     p.add_argument("--no-bf16-compare", action="store_true",
                    help="skip the comparison timings (the bf16 layer's step, the alternative recipes)")
     return p.parse_args()
