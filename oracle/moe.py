@@ -24,7 +24,9 @@ Readings where the pages are silent (each is listed in the design notes):
     gradient unchanged) and quantises dY, dGU rowwise and colwise as the consuming
     GEMMs need; the activations saved for backward are kept in fp64 here;
   * gradients are E4M3 like everything else; ``grad_fmt="e5m2"`` is the variant that
-    quantises dY and dGU to MXFP8 E5M2 instead (weights and activations stay E4M3).
+    quantises dY and dGU to MXFP8 E5M2 instead (weights and activations stay E4M3);
+  * every quantiser uses the OCP scale rule; ``scale_rule="ceil"`` is the variant whose
+    scale is rounded up so that no element saturates (all quantisers of the layer).
 Every GEMM is a library matmul over dequantised fp64 operands, one expert at a time.
 """
 from __future__ import annotations
@@ -101,7 +103,7 @@ def unpermute_sum(yp, row_of_slot):
 
 # ----------------------------------------------------------------------------- MXFP8 helpers
 
-def quantize_colwise_segments(a, seg_off, m_splits, fmt="e4m3"):
+def quantize_colwise_segments(a, seg_off, m_splits, fmt="e4m3", rule="ocp"):
     """Colwise MXFP8 of a permuted [Mp, C] matrix: blocks of 32 rows that start at each
     expert segment's first row (segments are 32-aligned with zero pad rows), stored
     transposed -> (codes uint8[C, Mp], scales uint8[C, Mp/32])."""
@@ -114,29 +116,29 @@ def quantize_colwise_segments(a, seg_off, m_splits, fmt="e4m3"):
         if s1 == s0:
             continue
         assert s0 % mxfp8.BLOCK == 0 and s1 % mxfp8.BLOCK == 0
-        c, s = mxfp8.quantize_colwise_t(a[s0:s1], fmt)
+        c, s = mxfp8.quantize_colwise_t(a[s0:s1], fmt, rule)
         codes[:, s0:s1] = c
         scales[:, s0 // mxfp8.BLOCK:s1 // mxfp8.BLOCK] = s
     return codes, scales
 
 
-def fake_quant_colwise_segments(a, seg_off, m_splits, fmt="e4m3"):
-    c, s = quantize_colwise_segments(a, seg_off, m_splits, fmt)
+def fake_quant_colwise_segments(a, seg_off, m_splits, fmt="e4m3", rule="ocp"):
+    c, s = quantize_colwise_segments(a, seg_off, m_splits, fmt, rule)
     return mxfp8.dequantize_rowwise(c, s, fmt).T
 
 
-def _fq_row(a, quant, fmt="e4m3"):
-    return mxfp8.fake_quant_rowwise(a, fmt) if quant else np.asarray(a, dtype=np.float64)
+def _fq_row(a, quant, fmt="e4m3", rule="ocp"):
+    return mxfp8.fake_quant_rowwise(a, fmt, rule) if quant else np.asarray(a, dtype=np.float64)
 
 
-def _fq_col(a, quant):
-    return mxfp8.fake_quant_colwise(a) if quant else np.asarray(a, dtype=np.float64)
+def _fq_col(a, quant, rule="ocp"):
+    return mxfp8.fake_quant_colwise(a, "e4m3", rule) if quant else np.asarray(a, dtype=np.float64)
 
 
-def _fq_col_seg(a, r, quant, fmt="e4m3"):
+def _fq_col_seg(a, r, quant, fmt="e4m3", rule="ocp"):
     if not quant:
         return np.asarray(a, dtype=np.float64)
-    return fake_quant_colwise_segments(a, r["seg_off"], r["m_splits"], fmt)
+    return fake_quant_colwise_segments(a, r["seg_off"], r["m_splits"], fmt, rule)
 
 
 # ----------------------------------------------------------------------------- grouped GEMMs
@@ -189,8 +191,10 @@ def dsilu(x):
 
 # ----------------------------------------------------------------------------- MLP
 
-def mlp_fwd(x, topk_idx, probs, W1, W2, quant=True, align=ALIGN_ORACLE):
-    """Forward of the grouped expert MLP. Returns (y fp64[T,H], saved dict)."""
+def mlp_fwd(x, topk_idx, probs, W1, W2, quant=True, align=ALIGN_ORACLE, scale_rule="ocp"):
+    """Forward of the grouped expert MLP. Returns (y fp64[T,H], saved dict). scale_rule
+    ("ocp" or "ceil") is the scale choice of every quantiser of the layer; the backward
+    takes it from the saved dict."""
     x = np.asarray(x, dtype=np.float64)
     probs = np.asarray(probs, dtype=np.float64)
     E, F2, H = W1.shape
@@ -200,16 +204,17 @@ def mlp_fwd(x, topk_idx, probs, W1, W2, quant=True, align=ALIGN_ORACLE):
     live = r["token_of_row"] >= 0
     p_row = np.zeros(r["Mp"], dtype=np.float64)
     p_row[live] = probs[r["token_of_row"][live], r["slot_of_row"][live]]
-    Xq = _fq_row(Xp, quant)                                   # blocks along H
-    W1q = np.stack([_fq_row(W1[e], quant) for e in range(E)])  # blocks along H
+    sr = scale_rule
+    Xq = _fq_row(Xp, quant, rule=sr)                                   # blocks along H
+    W1q = np.stack([_fq_row(W1[e], quant, rule=sr) for e in range(E)])  # blocks along H
     GU = grouped_gemm(Xq, W1q, r["seg_off"])
     G, U = GU[:, :F], GU[:, F:]
     Z = silu(G) * U * p_row[:, None]
-    Zq = _fq_row(Z, quant)                                    # blocks along F
-    W2q = np.stack([_fq_row(W2[e], quant) for e in range(E)])  # blocks along F
+    Zq = _fq_row(Z, quant, rule=sr)                                    # blocks along F
+    W2q = np.stack([_fq_row(W2[e], quant, rule=sr) for e in range(E)])  # blocks along F
     Yp = grouped_gemm(Zq, W2q, r["seg_off"])
     y = unpermute_sum(Yp, r["row_of_slot"])
-    saved = dict(route=r, Xp=Xp, p_row=p_row, G=G, U=U, Z=Z, Yp=Yp)
+    saved = dict(route=r, Xp=Xp, p_row=p_row, G=G, U=U, Z=Z, Yp=Yp, scale_rule=sr)
     return y, saved
 
 
@@ -221,10 +226,11 @@ def mlp_bwd(dy, saved, probs, W1, W2, quant=True, grad_fmt="e4m3"):
     E, F2, H = W1.shape
     F = F2 // 2
     G, U, Z, p_row = saved["G"], saved["U"], saved["Z"], saved["p_row"]
+    sr = saved.get("scale_rule", "ocp")
     dYp = permute_rows(dy, r["token_of_row"])
-    dYq_row = _fq_row(dYp, quant, grad_fmt)               # blocks along H (fc2 dgrad)
-    dYq_col = _fq_col_seg(dYp, r, quant, grad_fmt)        # blocks along M (fc2 wgrad)
-    W2q_col = np.stack([_fq_col(W2[e], quant) for e in range(E)])   # [H, F], blocks along H
+    dYq_row = _fq_row(dYp, quant, grad_fmt, sr)           # blocks along H (fc2 dgrad)
+    dYq_col = _fq_col_seg(dYp, r, quant, grad_fmt, sr)    # blocks along M (fc2 wgrad)
+    W2q_col = np.stack([_fq_col(W2[e], quant, sr) for e in range(E)])   # [H, F], blocks along H
     # fc2 dgrad: dZ = dYp . W2  (contract over H)
     dZ = grouped_gemm(dYq_row, np.transpose(W2q_col, (0, 2, 1)), r["seg_off"])
     A = silu(G) * U
@@ -233,14 +239,14 @@ def mlp_bwd(dy, saved, probs, W1, W2, quant=True, grad_fmt="e4m3"):
     dG = dA * U * dsilu(G)
     dU = dA * silu(G)
     dGU = np.concatenate([dG, dU], axis=1)
-    dGUq_row = _fq_row(dGU, quant, grad_fmt)              # blocks along 2F (fc1 dgrad)
-    dGUq_col = _fq_col_seg(dGU, r, quant, grad_fmt)       # blocks along M (fc1 wgrad)
-    Zq_col = _fq_col_seg(Z, r, quant)
-    Xq_col = _fq_col_seg(saved["Xp"], r, quant)
+    dGUq_row = _fq_row(dGU, quant, grad_fmt, sr)          # blocks along 2F (fc1 dgrad)
+    dGUq_col = _fq_col_seg(dGU, r, quant, grad_fmt, sr)   # blocks along M (fc1 wgrad)
+    Zq_col = _fq_col_seg(Z, r, quant, rule=sr)
+    Xq_col = _fq_col_seg(saved["Xp"], r, quant, rule=sr)
     # fc2 wgrad: dW2[e] = dYp_e^T . Z_e  (contract over the expert's rows)
     dW2 = grouped_gemm_wgrad(dYq_col.T, Zq_col.T, r["seg_off"])
     # fc1 dgrad: dXp = dGU . W1  (contract over 2F)
-    W1q_col = np.stack([_fq_col(W1[e], quant) for e in range(E)])   # [2F, H], blocks along 2F
+    W1q_col = np.stack([_fq_col(W1[e], quant, sr) for e in range(E)])   # [2F, H], blocks along 2F
     dXp = grouped_gemm(dGUq_row, np.transpose(W1q_col, (0, 2, 1)), r["seg_off"])
     # fc1 wgrad: dW1[e] = dGU_e^T . Xp_e
     dW1 = grouped_gemm_wgrad(dGUq_col.T, Xq_col.T, r["seg_off"])

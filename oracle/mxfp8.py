@@ -22,6 +22,11 @@ max 57344, S.11111.00 infinite, S.11111.xx with xx != 0 NaN). Its scale rule is 
 with the format's largest exponent: X = clamp(floor(log2(amax)) - 15, -127, 127); its
 elements saturate to +-57344.
 
+The "ceil" scale rule is a variant of the scale choice (the pages give none): the
+smallest power of two for which no element of the block exceeds the format's largest
+value, so nothing saturates (the OCP exponent, plus one when the block's amax lies
+above that value times the OCP scale).
+
 The encoder is a nearest-value search over the table of finite codes; it never uses
 bit manipulation, so that it is independent of the decoder's closed form.
 """
@@ -106,27 +111,39 @@ def e5m2_encode(x):
     return _nearest_code(x, _POS_CODES_E5M2, _POS_VALUES_E5M2, E5M2_MAX)
 
 
-# element formats: name -> (encode, decode, largest exponent)
-FORMATS = {"e4m3": (e4m3_encode, e4m3_decode, E4M3_EMAX), "e5m2": (e5m2_encode, e5m2_decode, E5M2_EMAX)}
+# element formats: name -> (encode, decode, largest exponent, largest finite value)
+FORMATS = {"e4m3": (e4m3_encode, e4m3_decode, E4M3_EMAX, E4M3_MAX),
+           "e5m2": (e5m2_encode, e5m2_decode, E5M2_EMAX, E5M2_MAX)}
 
 
-def scale_exponent(amax, emax=E4M3_EMAX):
-    """X = clamp(floor(log2(amax)) - emax, -127, 127); amax == 0 -> -127 (byte 0x00).
-    emax = the element format's largest exponent (8 for E4M3, 15 for E5M2)."""
+def scale_exponent(amax, emax=E4M3_EMAX, rule="ocp", vmax=None):
+    """Scale exponent of a block with largest magnitude amax (amax == 0 -> -127, byte 0x00).
+    rule "ocp": X = clamp(floor(log2(amax)) - emax, -127, 127), emax = the element
+      format's largest exponent (8 for E4M3, 15 for E5M2); elements above vmax * 2^X
+      saturate.
+    rule "ceil": the smallest X with amax <= vmax * 2^X (vmax = the format's largest
+      finite value), clamped likewise: the power-of-two scale rounded up so that no
+      element saturates. It is the "ocp" exponent, or one more when amax lies above
+      vmax * 2^X_ocp."""
     amax = np.asarray(amax, dtype=np.float64)
     mant, ex = np.frexp(amax)            # amax = mant * 2^ex, mant in [0.5, 1)
     fl = ex.astype(np.int64) - 1         # floor(log2(amax)) for amax > 0
-    X = np.clip(fl - emax, SCALE_MIN_EXP, SCALE_MAX_EXP)
+    X = fl - emax
+    if rule == "ceil":
+        X = X + (amax > vmax * np.exp2(X.astype(np.float64))).astype(np.int64)
+    elif rule != "ocp":
+        raise ValueError(f"unknown scale rule {rule!r}")
+    X = np.clip(X, SCALE_MIN_EXP, SCALE_MAX_EXP)
     return np.where(amax == 0, SCALE_MIN_EXP, X).astype(np.int64)
 
 
-def quantize_blocks(v, fmt="e4m3"):
+def quantize_blocks(v, fmt="e4m3", rule="ocp"):
     """Quantise ``v[..., 32]`` block by block -> (codes uint8[..., 32], scale bytes uint8[...])."""
-    encode, _, emax = FORMATS[fmt]
+    encode, _, emax, vmax = FORMATS[fmt]
     v = np.asarray(v, dtype=np.float64)
     assert v.shape[-1] == BLOCK
     amax = np.max(np.abs(v), axis=-1)
-    X = scale_exponent(amax, emax)
+    X = scale_exponent(amax, emax, rule, vmax)
     scaled = v * np.exp2(-X.astype(np.float64))[..., None]   # exact power-of-two scaling in fp64
     codes = encode(scaled)
     return codes, (X + SCALE_BIAS).astype(np.uint8)
@@ -139,13 +156,13 @@ def dequantize_blocks(codes, scale_bytes, fmt="e4m3"):
     return decode(codes) * np.exp2(X.astype(np.float64))[..., None]
 
 
-def quantize_rowwise(a, fmt="e4m3"):
+def quantize_rowwise(a, fmt="e4m3", rule="ocp"):
     """Blocks of 32 along the last axis of a 2-D matrix [R, C] (C % 32 == 0).
     Returns (codes uint8[R, C], scales uint8[R, C/32])."""
     a = np.asarray(a, dtype=np.float64)
     R, C = a.shape
     assert C % BLOCK == 0
-    codes, sc = quantize_blocks(a.reshape(R, C // BLOCK, BLOCK), fmt)
+    codes, sc = quantize_blocks(a.reshape(R, C // BLOCK, BLOCK), fmt, rule)
     return codes.reshape(R, C), sc
 
 
@@ -154,22 +171,22 @@ def dequantize_rowwise(codes, scales, fmt="e4m3"):
     return dequantize_blocks(codes.reshape(R, C // BLOCK, BLOCK), scales, fmt).reshape(R, C)
 
 
-def quantize_colwise_t(a, fmt="e4m3"):
+def quantize_colwise_t(a, fmt="e4m3", rule="ocp"):
     """Blocks of 32 consecutive rows in each column of [R, C] (R % 32 == 0), stored
     transposed: (codes uint8[C, R], scales uint8[C, R/32]). The caller lays segments
     out so that no block crosses an expert boundary."""
     a = np.asarray(a, dtype=np.float64)
-    return quantize_rowwise(a.T, fmt)
+    return quantize_rowwise(a.T, fmt, rule)
 
 
-def fake_quant_rowwise(a, fmt="e4m3"):
+def fake_quant_rowwise(a, fmt="e4m3", rule="ocp"):
     """Quantise then dequantise along rows (used where the oracle needs the value a
     quantised operand stands for)."""
-    c, s = quantize_rowwise(a, fmt)
+    c, s = quantize_rowwise(a, fmt, rule)
     return dequantize_rowwise(c, s, fmt)
 
 
-def fake_quant_colwise(a, fmt="e4m3"):
+def fake_quant_colwise(a, fmt="e4m3", rule="ocp"):
     """Colwise quantise/dequantise, returned in the original [R, C] orientation."""
-    c, s = quantize_colwise_t(a, fmt)
+    c, s = quantize_colwise_t(a, fmt, rule)
     return dequantize_rowwise(c, s, fmt).T

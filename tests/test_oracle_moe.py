@@ -285,3 +285,28 @@ def test_e5m2_gradients_variant():
         assert rel(g5[n], gu[n]) > rel(g4[n], gu[n]), n
     # dZ = dYq . W2q: only dY's format changed between the two
     assert not np.array_equal(g5["dZ"], g4["dZ"])
+
+
+def test_ceil_scale_rule_variant():
+    """The round-up scale rule changes only the blocks whose amax the OCP rule would
+    saturate: the layer stays close to the unquantised one, and a block-wise comparison of
+    the two rules' quantised inputs differs exactly where the OCP exponent is one lower."""
+    cfg = wl.custom("ce", T=96, H=64, F=64, E=3, k=2, seed=10)
+    d = wl.make_all(cfg)
+    x, W1, W2, p = (d[n].double().numpy() for n in ("x", "W1", "W2", "probs"))
+    idx, dy = d["topk_idx"].numpy(), d["dy"].double().numpy()
+    yc, sc = moe.mlp_fwd(x, idx, p, W1, W2, scale_rule="ceil")
+    yu, su = moe.mlp_fwd(x, idx, p, W1, W2, quant=False)
+    gc = moe.mlp_bwd(dy, sc, p, W1, W2)
+    gu = moe.mlp_bwd(dy, su, p, W1, W2, quant=False)
+    rel = lambda a, b: np.linalg.norm(a - b) / np.linalg.norm(b)  # noqa: E731
+    assert rel(yc, yu) < 0.1
+    for n in ("dx", "dW1", "dW2", "dprobs"):
+        assert rel(gc[n], gu[n]) < 0.15, n
+    blocks = x.reshape(-1, 32)
+    _, s_ocp = mxfp8.quantize_blocks(blocks)
+    _, s_ceil = mxfp8.quantize_blocks(blocks, "e4m3", "ceil")
+    amax = np.abs(blocks).max(axis=1)
+    saturating = amax > 448.0 * np.exp2(s_ocp.astype(float) - 127)
+    assert np.array_equal(s_ceil.astype(int) - s_ocp.astype(int), saturating.astype(int))
+    assert saturating.any() and not saturating.all()

@@ -195,3 +195,48 @@ def test_e5m2_scale_rule_and_error_bound():
     assert rel.max() > 2.0 ** -4                            # coarser than E4M3
     # a block quantised to E5M2 keeps 6 more binades below its max than E4M3
     assert np.all(np.abs(d) <= 57344.0 * np.exp2(X))
+
+
+# ----------------------------------------------------------------------------- "ceil" scale rule (variant)
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+def test_ceil_rule_is_the_smallest_non_saturating_power_of_two(fmt):
+    """Brute force over candidate exponents: the ceil rule picks the smallest X for which
+    amax * 2^-X does not exceed the format's largest value; the OCP rule picks X or X - 1."""
+    _, decode, emax, vmax = mxfp8.FORMATS[fmt]
+    rng = np.random.default_rng(7)
+    amax = np.abs(rng.standard_normal(2000)) * np.exp2(rng.integers(-60, 60, 2000))
+    amax = np.concatenate([amax, vmax * np.exp2(np.arange(-20.0, 20.0)),          # exactly at the top: no +1
+                           np.nextafter(vmax, np.inf) * np.exp2(np.arange(-20.0, 20.0))])  # just above: +1
+    Xc = mxfp8.scale_exponent(amax, emax, "ceil", vmax)
+    Xo = mxfp8.scale_exponent(amax, emax)
+    for a, xc, xo in zip(amax, Xc, Xo):
+        cands = [x for x in range(-127, 128) if a <= vmax * 2.0 ** x]
+        assert xc == min(cands), (a, xc)
+        assert xc - xo in (0, 1)
+    assert np.all(Xc[-40:] == Xo[-40:] + 1) and np.all(Xc[-80:-40] == Xo[-80:-40])
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+def test_ceil_rule_never_saturates(fmt):
+    """Under the ceil rule no element of a block reaches beyond the format's top value, and
+    a block whose amax the OCP rule would saturate gets the next scale up."""
+    _, decode, _, vmax = mxfp8.FORMATS[fmt]
+    rng = np.random.default_rng(8)
+    v = rng.standard_normal((400, 32)) * np.exp2(rng.integers(-30, 30, (400, 1)))
+    q, s = mxfp8.quantize_blocks(v, fmt, "ceil")
+    X = (s.astype(np.int64) - 127).astype(float)[:, None]
+    assert np.all(np.abs(v) * np.exp2(-X) <= vmax)
+    d = mxfp8.dequantize_blocks(q, s, fmt)
+    rel = np.abs(d - v)[np.abs(v) * np.exp2(-X) >= 1.0] / np.abs(v)[np.abs(v) * np.exp2(-X) >= 1.0]
+    assert rel.max() <= (2.0 ** -4 if fmt == "e4m3" else 2.0 ** -3) + 1e-15
+    blk = np.zeros(32)
+    blk[0] = 480.0 if fmt == "e4m3" else 60000.0        # saturates under the OCP rule
+    q4, s4 = mxfp8.quantize_blocks(blk[None, :], fmt)
+    qc, sc = mxfp8.quantize_blocks(blk[None, :], fmt, "ceil")
+    assert decode(q4[0, 0]) == vmax and sc[0] == s4[0] + 1
+    back = decode(qc[0, 0]) * 2.0 ** (int(sc[0]) - 127)
+    if fmt == "e4m3":
+        assert back == blk[0]                 # 480 = 240 * 2, and 240 is an E4M3 value
+    else:
+        assert abs(back - blk[0]) <= 2.0 ** -3 * blk[0]   # rounded, not clipped to 57344
