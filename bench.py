@@ -269,9 +269,9 @@ def config_json(cfg, world):
 
 # ----------------------------------------------------------------------------- GPU arm
 def time_recipes(cfg, layer, W1, W2, x, idx, probs, dy, y, dx, dW1, dW2, dprobs, stream, steps):
-    """The same full step (weights quantised, forward, backward) under the layer's two
+    """The same full step (weights quantised, forward, backward) under the layer's
     alternative recipes, beside the headline: E5M2 gradients (the backward's dY and dGU in
-    E5M2) and G / U recomputed in the backward instead of saved. CUDA events over `steps`
+    E5M2), G / U recomputed in the backward instead of saved, and the round-up scale rule. CUDA events over `steps`
     steps after two warm-up steps; the saved-activation bytes of each recipe."""
     import torch
 
@@ -280,7 +280,9 @@ def time_recipes(cfg, layer, W1, W2, x, idx, probs, dy, y, dx, dW1, dW2, dprobs,
     a = (cfg.T, cfg.k, cfg.E, cfg.H, cfg.F)
     out = {}
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for name, recipe in (("grad_e5m2", mx.RECIPE_GRAD_E5M2), ("recompute_gu", mx.RECIPE_RECOMPUTE_GU)):
+    for name, recipe in (("grad_e5m2", mx.RECIPE_GRAD_E5M2), ("recompute_gu", mx.RECIPE_RECOMPUTE_GU),
+                         ("scale_ceil", mx.RECIPE_SCALE_CEIL)):
+        rule = mx.SCALE_RULE_CEIL if recipe & mx.RECIPE_SCALE_CEIL else mx.SCALE_RULE_OCP
         if recipe & mx.RECIPE_RECOMPUTE_GU:
             saved = torch.empty(lib.grouped_mlp_saved_size_ex(*a, recipe), dtype=torch.uint8, device=x.device)
             ws = torch.empty(lib.grouped_mlp_workspace_size_ex(*a, recipe), dtype=torch.uint8, device=x.device)
@@ -288,7 +290,7 @@ def time_recipes(cfg, layer, W1, W2, x, idx, probs, dy, y, dx, dW1, dW2, dprobs,
             saved, ws = layer.saved, layer.ws
 
         def step():
-            mx.mxmoe_weights_quantize(W1, W2, out=layer.wq)
+            mx.mxmoe_weights_quantize(W1, W2, out=layer.wq, scale_rule=rule)
             mx.grouped_mlp_fwd(x, idx, probs, layer.wq, cfg.E, cfg.F, saved, ws, y, recipe=recipe)
             mx.grouped_mlp_bwd(dy, saved, layer.wq, *a, ws, dx, dW1, dW2, dprobs, recipe=recipe)
         for _ in range(2):

@@ -61,6 +61,11 @@ typedef int32_t mxmoe_status;
 #define MXMOE_DTYPE_BF16 0
 #define MXMOE_DTYPE_F32 1
 
+/* scale rules of a quantisation (mxfp8_quantize_ex, mxmoe_weights_quantize_ex) */
+#define MXMOE_SCALE_RULE_OCP 0  /* X = clamp(floor(log2(amax)) - emax, -127, 127); elements saturate */
+#define MXMOE_SCALE_RULE_CEIL 1 /* smallest X with amax <= max * 2^X (the OCP X, or one more): nothing
+                                   saturates (a variant; the pages give no rule) */
+
 /* element formats of an mxmoe_mxfp8 matrix */
 #define MXMOE_FMT_E4M3 0 /* OCP FP8 E4M3: bias 7, max 448 (activations, weights; gradients by default) */
 #define MXMOE_FMT_E5M2 1 /* OCP FP8 E5M2: bias 15, max 57344, saturating (the gradient variant) */
@@ -221,6 +226,14 @@ mxmoe_status moe_unpermute(const void* y_perm_dev, const int32_t* row_of_slot_de
 mxmoe_status mxfp8_quantize(const void* src_dev, int32_t src_dtype, int64_t batch, int64_t rows, int64_t cols,
                             const int32_t* row_gather_dev, const int32_t* nrows_dev, int64_t out_rows,
                             const mxmoe_mxfp8* out_row, const mxmoe_mxfp8* out_colT, void* stream);
+/* mxfp8_quantize with the scale rule chosen (MXMOE_SCALE_RULE_OCP, the rule above, or
+ * MXMOE_SCALE_RULE_CEIL: the OCP exponent plus one for the blocks whose amax lies above
+ * the format's largest value times the OCP scale, so that no element saturates). Any
+ * other rule returns MXMOE_ERR_INVALID_ARG. */
+mxmoe_status mxfp8_quantize_ex(const void* src_dev, int32_t src_dtype, int64_t batch, int64_t rows, int64_t cols,
+                               const int32_t* row_gather_dev, const int32_t* nrows_dev, int64_t out_rows,
+                               const mxmoe_mxfp8* out_row, const mxmoe_mxfp8* out_colT, int32_t scale_rule,
+                               void* stream);
 
 /* ------------------------------------------------------------------ grouped GEMMs (GroupedLinear) */
 
@@ -297,6 +310,10 @@ mxmoe_status grouped_gemm_bf16_wgrad(const void* At_dev, const void* Bt_dev, int
 size_t mxmoe_weights_size(int32_t E, int32_t H, int32_t F);
 mxmoe_status mxmoe_weights_quantize(const void* W1_dev, const void* W2_dev, int32_t E, int32_t H, int32_t F,
                                     void* wq_dev, size_t wq_bytes, void* stream);
+/* The same with the scale rule chosen (MXMOE_SCALE_RULE_*); a layer run with
+ * MXMOE_RECIPE_SCALE_CEIL takes weights quantised with MXMOE_SCALE_RULE_CEIL. */
+mxmoe_status mxmoe_weights_quantize_ex(const void* W1_dev, const void* W2_dev, int32_t E, int32_t H, int32_t F,
+                                       int32_t scale_rule, void* wq_dev, size_t wq_bytes, void* stream);
 /* View of one of the four copies inside a weights buffer (which: 0 W1 row, 1 W1 col,
  * 2 W2 row, 3 W2 col). Host-only pointer arithmetic. */
 mxmoe_status mxmoe_weights_view(void* wq_dev, int32_t E, int32_t H, int32_t F, int32_t which, mxmoe_mxfp8* out);
@@ -373,10 +390,14 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
  *                               biologische Grundmodelle optimieren": activation memory
  *                               is the pressure MXFP8 and the fused kernel relieve). The
  *                               recomputed G / U live in the workspace for the call.
+ *   MXMOE_RECIPE_SCALE_CEIL     every quantiser of the call (x, Z; dY, dGU) uses
+ *                               MXMOE_SCALE_RULE_CEIL; quantise the weights with
+ *                               mxmoe_weights_quantize_ex(..., MXMOE_SCALE_RULE_CEIL, ...).
  * A recipe with any other bit set returns MXMOE_ERR_INVALID_ARG (sizes: 0 / -1).
  */
 #define MXMOE_RECIPE_GRAD_E5M2 1
 #define MXMOE_RECIPE_RECOMPUTE_GU 2
+#define MXMOE_RECIPE_SCALE_CEIL 4
 size_t grouped_mlp_saved_size_ex(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F, int32_t recipe);
 int64_t grouped_mlp_saved_offset_ex(int32_t field, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
                                     int32_t recipe);

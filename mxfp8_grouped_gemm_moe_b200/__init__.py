@@ -26,7 +26,9 @@ STATUS_NAMES = {
 DTYPE_BF16, DTYPE_F32 = 0, 1
 SCALE_PLAIN, SCALE_MMA = 0, 1
 FMT_E4M3, FMT_E5M2 = 0, 1
-RECIPE_GRAD_E5M2, RECIPE_RECOMPUTE_GU = 1, 2
+RECIPE_GRAD_E5M2, RECIPE_RECOMPUTE_GU, RECIPE_SCALE_CEIL = 1, 2, 4
+SCALE_RULE_OCP, SCALE_RULE_CEIL = 0, 1
+_RULE = {"ocp": SCALE_RULE_OCP, "ceil": SCALE_RULE_CEIL}
 _FMT = {"e4m3": FMT_E4M3, "e5m2": FMT_E5M2}
 SAVED_FIELDS = ["m_splits", "seg_off", "row_of_slot", "token_of_row", "prob_of_row",
                 "x_colT", "x_colT_sf", "z_colT", "z_colT_sf", "gu", "x_row", "x_row_sf"]
@@ -66,10 +68,12 @@ _SIGNATURES = {
     "grouped_gemm_bf16_wgrad": (_I32, [_P, _P, _I64, _I64, _I64, _P, _I32, _P, _P]),
     "moe_router_topk_bwd": (_I32, [_P, _P, _P, _I32, _I32, _I32, _P, _P]),
     "mxfp8_quantize": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _I64, _PMX, _PMX, _P]),
+    "mxfp8_quantize_ex": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _I64, _PMX, _PMX, _I32, _P]),
     "grouped_gemm_mxfp8": (_I32, [_PMX, _PMX, _P, _I32, _I64, _I64, _P, _I32, _I64, _P]),
     "grouped_gemm_mxfp8_wgrad": (_I32, [_PMX, _PMX, _P, _I32, _P, _P]),
     "mxmoe_weights_size": (_SZ, [_I32, _I32, _I32]),
     "mxmoe_weights_quantize": (_I32, [_P, _P, _I32, _I32, _I32, _P, _SZ, _P]),
+    "mxmoe_weights_quantize_ex": (_I32, [_P, _P, _I32, _I32, _I32, _I32, _P, _SZ, _P]),
     "mxmoe_weights_view": (_I32, [_P, _I32, _I32, _I32, _I32, _PMX]),
     "grouped_mlp_saved_size": (_SZ, [_I32, _I32, _I32, _I32, _I32]),
     "grouped_mlp_saved_offset": (_I64, [_I32, _I32, _I32, _I32, _I32, _I32]),
@@ -241,9 +245,10 @@ def moe_router_topk_bwd(logits, topk_idx, dprobs):
 
 
 def mxfp8_quantize(src, rowwise=True, colwise=True, layout=SCALE_MMA, row_gather=None, nrows=None, out_rows=None,
-                   fmt=FMT_E4M3):
+                   fmt=FMT_E4M3, scale_rule=SCALE_RULE_OCP):
     """src [rows, cols] or [batch, rows, cols] bf16/fp32 -> (MXFP8 rowwise | None, MXFP8 colT | None);
-    fmt FMT_E4M3 or FMT_E5M2 (element format of both outputs)."""
+    fmt FMT_E4M3 or FMT_E5M2 (element format of both outputs); scale_rule SCALE_RULE_OCP or
+    SCALE_RULE_CEIL."""
     lib = load()
     dt = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}[src.dtype]
     if src.dim() == 2:
@@ -255,9 +260,14 @@ def mxfp8_quantize(src, rowwise=True, colwise=True, layout=SCALE_MMA, row_gather
     c = MXFP8.empty(batch * cols, orows, layout, src.device, fmt) if colwise else None
     rs = ctypes.byref(r.as_struct()) if r is not None else None
     cs = ctypes.byref(c.as_struct()) if c is not None else None
-    st = lib.mxfp8_quantize(_ptr(src), dt, batch, rows, cols, _ptr(row_gather), _ptr(nrows), orows, rs, cs,
-                            _stream())
-    _check("mxfp8_quantize", st)
+    if scale_rule == SCALE_RULE_OCP:
+        st = lib.mxfp8_quantize(_ptr(src), dt, batch, rows, cols, _ptr(row_gather), _ptr(nrows), orows, rs, cs,
+                                _stream())
+        _check("mxfp8_quantize", st)
+    else:
+        st = lib.mxfp8_quantize_ex(_ptr(src), dt, batch, rows, cols, _ptr(row_gather), _ptr(nrows), orows, rs, cs,
+                                   scale_rule, _stream())
+        _check("mxfp8_quantize_ex", st)
     return r, c
 
 
@@ -299,14 +309,19 @@ def grouped_gemm_bf16_wgrad(At, Bt, seg_off, E, out=None):
     return C
 
 
-def mxmoe_weights_quantize(W1, W2, out=None):
+def mxmoe_weights_quantize(W1, W2, out=None, scale_rule=SCALE_RULE_OCP):
     lib = load()
     E, F2, H = W1.shape
     F = F2 // 2
     n = lib.mxmoe_weights_size(E, H, F)
     wq = out if out is not None else torch.empty(n, dtype=torch.uint8, device=W1.device)
-    _check("mxmoe_weights_quantize",
-           lib.mxmoe_weights_quantize(_ptr(W1), _ptr(W2), E, H, F, _ptr(wq), wq.numel(), _stream()))
+    if scale_rule == SCALE_RULE_OCP:
+        _check("mxmoe_weights_quantize",
+               lib.mxmoe_weights_quantize(_ptr(W1), _ptr(W2), E, H, F, _ptr(wq), wq.numel(), _stream()))
+    else:
+        _check("mxmoe_weights_quantize_ex",
+               lib.mxmoe_weights_quantize_ex(_ptr(W1), _ptr(W2), E, H, F, scale_rule, _ptr(wq), wq.numel(),
+                                             _stream()))
     return wq
 
 
@@ -326,18 +341,25 @@ class GroupedMLP:
     precision "mxfp8" (default) runs the MXFP8 layer (grouped_mlp_fwd / _bwd); "bf16" runs
     the same steps on bf16 operands (grouped_mlp_bf16_fwd / _bwd). For the MXFP8 layer,
     grad_format "e4m3" (default) or "e5m2" picks the element format of the gradients (dY,
-    dGU), and recompute_gu=True saves the rowwise MXFP8 input instead of the bf16 gate/up
-    pre-activations and recomputes those in the backward (the recipe flags of
-    grouped_mlp_fwd_ex / _bwd_ex)."""
+    dGU), recompute_gu=True saves the rowwise MXFP8 input instead of the bf16 gate/up
+    pre-activations and recomputes those in the backward, and scale_rule "ocp" (default) or
+    "ceil" picks the scale rule of every quantiser, the weights' included (the recipe flags
+    of grouped_mlp_fwd_ex / _bwd_ex)."""
 
-    def __init__(self, T, k, E, H, F, device="cuda", precision="mxfp8", grad_format="e4m3", recompute_gu=False):
+    def __init__(self, T, k, E, H, F, device="cuda", precision="mxfp8", grad_format="e4m3", recompute_gu=False,
+                 scale_rule="ocp"):
         if precision not in ("mxfp8", "bf16"):
             raise ValueError(f"unknown precision {precision!r}")
         if grad_format not in _FMT:
             raise ValueError(f"unknown grad_format {grad_format!r}")
-        self.recipe = (RECIPE_GRAD_E5M2 if grad_format == "e5m2" else 0) | (RECIPE_RECOMPUTE_GU if recompute_gu else 0)
+        if scale_rule not in _RULE:
+            raise ValueError(f"unknown scale_rule {scale_rule!r}")
+        self.scale_rule = _RULE[scale_rule]
+        self.recipe = ((RECIPE_GRAD_E5M2 if grad_format == "e5m2" else 0) |
+                       (RECIPE_RECOMPUTE_GU if recompute_gu else 0) |
+                       (RECIPE_SCALE_CEIL if scale_rule == "ceil" else 0))
         if precision == "bf16" and self.recipe:
-            raise ValueError("grad_format / recompute_gu apply to the MXFP8 layer")
+            raise ValueError("grad_format / recompute_gu / scale_rule apply to the MXFP8 layer")
         lib = load()
         self.T, self.k, self.E, self.H, self.F = T, k, E, H, F
         self.precision = precision
@@ -360,7 +382,7 @@ class GroupedMLP:
         """Prepares the weights buffer: MXFP8 copies, or bf16 row / transposed copies."""
         if self.precision == "bf16":
             return mxmoe_weights_bf16_prepare(W1, W2, out=self.wq)
-        return mxmoe_weights_quantize(W1, W2, out=self.wq)
+        return mxmoe_weights_quantize(W1, W2, out=self.wq, scale_rule=self.scale_rule)
 
     def forward(self, x, topk_idx, probs, y=None):
         if self.precision == "bf16":

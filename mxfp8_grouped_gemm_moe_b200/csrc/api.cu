@@ -59,7 +59,12 @@ WeightsLayout weights_layout(int64_t E, int64_t H, int64_t F) {
   return L;
 }
 
-bool valid_recipe(int32_t recipe) { return (recipe & ~(MXMOE_RECIPE_GRAD_E5M2 | MXMOE_RECIPE_RECOMPUTE_GU)) == 0; }
+bool valid_recipe(int32_t recipe) {
+  return (recipe & ~(MXMOE_RECIPE_GRAD_E5M2 | MXMOE_RECIPE_RECOMPUTE_GU | MXMOE_RECIPE_SCALE_CEIL)) == 0;
+}
+int32_t recipe_scale_rule(int32_t recipe) {
+  return (recipe & MXMOE_RECIPE_SCALE_CEIL) ? MXMOE_SCALE_RULE_CEIL : MXMOE_SCALE_RULE_OCP;
+}
 bool recomputes_gu(int32_t recipe) { return (recipe & MXMOE_RECIPE_RECOMPUTE_GU) != 0; }
 
 struct SavedLayout {
@@ -291,8 +296,9 @@ mxmoe_status moe_unpermute(const void* y_perm_dev, const int32_t* row_of_slot_de
 static mxmoe_status quantize_impl(const void* src_dev, int32_t src_dtype, int64_t batch, int64_t rows, int64_t cols,
                                   const int32_t* row_gather_dev, const int32_t* nrows_dev, int64_t out_rows,
                                   const mxmoe_mxfp8* out_row, const mxmoe_mxfp8* out_colT, int64_t row_ilv,
-                                  void* stream) {
+                                  int32_t scale_rule, void* stream) {
   if (src_dtype != MXMOE_DTYPE_BF16 && src_dtype != MXMOE_DTYPE_F32) return MXMOE_ERR_INVALID_ARG;
+  if (scale_rule != MXMOE_SCALE_RULE_OCP && scale_rule != MXMOE_SCALE_RULE_CEIL) return MXMOE_ERR_INVALID_ARG;
   if (!src_dev || !aligned16(src_dev) || (!out_row && !out_colT)) return MXMOE_ERR_INVALID_ARG;
   if (batch < 1 || rows < 0 || cols <= 0 || out_rows < 0) return MXMOE_ERR_UNSUPPORTED_SHAPE;
   if (row_gather_dev && batch != 1) return MXMOE_ERR_UNSUPPORTED_SHAPE;
@@ -314,6 +320,7 @@ static mxmoe_status quantize_impl(const void* src_dev, int32_t src_dtype, int64_
   if (out_rows == 0 || rows == 0) return MXMOE_OK;
   QuantArgs a;
   a.fmt = out_row ? out_row->elem_format : out_colT->elem_format;
+  a.scale_rule = scale_rule;
   a.src = src_dev;
   a.src_dtype = src_dtype;
   a.batch = batch;
@@ -337,7 +344,15 @@ mxmoe_status mxfp8_quantize(const void* src_dev, int32_t src_dtype, int64_t batc
                             const int32_t* row_gather_dev, const int32_t* nrows_dev, int64_t out_rows,
                             const mxmoe_mxfp8* out_row, const mxmoe_mxfp8* out_colT, void* stream) {
   return quantize_impl(src_dev, src_dtype, batch, rows, cols, row_gather_dev, nrows_dev, out_rows, out_row, out_colT, 0,
-                       stream);
+                       MXMOE_SCALE_RULE_OCP, stream);
+}
+
+mxmoe_status mxfp8_quantize_ex(const void* src_dev, int32_t src_dtype, int64_t batch, int64_t rows, int64_t cols,
+                               const int32_t* row_gather_dev, const int32_t* nrows_dev, int64_t out_rows,
+                               const mxmoe_mxfp8* out_row, const mxmoe_mxfp8* out_colT, int32_t scale_rule,
+                               void* stream) {
+  return quantize_impl(src_dev, src_dtype, batch, rows, cols, row_gather_dev, nrows_dev, out_rows, out_row, out_colT, 0,
+                       scale_rule, stream);
 }
 
 mxmoe_status grouped_gemm_mxfp8(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, const int32_t* seg_off_dev,
@@ -446,6 +461,12 @@ mxmoe_status mxmoe_weights_view(void* wq_dev, int32_t E, int32_t H, int32_t F, i
 
 mxmoe_status mxmoe_weights_quantize(const void* W1_dev, const void* W2_dev, int32_t E, int32_t H, int32_t F,
                                     void* wq_dev, size_t wq_bytes, void* stream) {
+  return mxmoe_weights_quantize_ex(W1_dev, W2_dev, E, H, F, MXMOE_SCALE_RULE_OCP, wq_dev, wq_bytes, stream);
+}
+
+mxmoe_status mxmoe_weights_quantize_ex(const void* W1_dev, const void* W2_dev, int32_t E, int32_t H, int32_t F,
+                                       int32_t scale_rule, void* wq_dev, size_t wq_bytes, void* stream) {
+  if (scale_rule != MXMOE_SCALE_RULE_OCP && scale_rule != MXMOE_SCALE_RULE_CEIL) return MXMOE_ERR_INVALID_ARG;
   if (E < 1 || E > 256 || H <= 0 || F <= 0 || H % 256 != 0 || F % 256 != 0) return MXMOE_ERR_UNSUPPORTED_SHAPE;
   if (!W1_dev || !W2_dev || !wq_dev || !aligned16(W1_dev) || !aligned16(W2_dev) || !aligned16(wq_dev))
     return MXMOE_ERR_INVALID_ARG;
@@ -460,11 +481,11 @@ mxmoe_status mxmoe_weights_quantize(const void* W1_dev, const void* W2_dev, int3
   {
     StageScope sc(MXMOE_STAGE_QUANT_W1, S(stream));
     s = quantize_impl(W1_dev, MXMOE_DTYPE_BF16, E, 2 * (int64_t)F, H, nullptr, nullptr, 2 * (int64_t)F, &w1r, &w1c,
-                      F, stream);
+                      F, scale_rule, stream);
   }
   if (s != MXMOE_OK) return s;
   StageScope sc(MXMOE_STAGE_QUANT_W2, S(stream));
-  return mxfp8_quantize(W2_dev, MXMOE_DTYPE_BF16, E, H, F, nullptr, nullptr, H, &w2r, &w2c, stream);
+  return mxfp8_quantize_ex(W2_dev, MXMOE_DTYPE_BF16, E, H, F, nullptr, nullptr, H, &w2r, &w2c, scale_rule, stream);
 }
 
 size_t grouped_mlp_saved_size(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F) {
@@ -544,7 +565,8 @@ mxmoe_status grouped_mlp_fwd_ex(const void* x_dev, const int32_t* topk_idx_dev, 
   mxmoe_status s;
   {
     StageScope sc(MXMOE_STAGE_QUANT_X, st);
-    s = mxfp8_quantize(x_dev, MXMOE_DTYPE_BF16, 1, T, H, tor, seg_off + E, cap, &x_row, &x_col, stream);
+    s = mxfp8_quantize_ex(x_dev, MXMOE_DTYPE_BF16, 1, T, H, tor, seg_off + E, cap, &x_row, &x_col,
+                          recipe_scale_rule(recipe), stream);
   }
   if (s != MXMOE_OK) return s;
   // 3. fc1 + SwiGLU x prob -> Z (MXFP8 row + colT), G/U saved unless recomputed
@@ -559,6 +581,7 @@ mxmoe_status grouped_mlp_fwd_ex(const void* x_dev, const int32_t* topk_idx_dev, 
   g.z_row_sf = ws + W.z_row_sf;
   g.z_colT = sv + SL.off[MXMOE_SAVED_Z_COLT];
   g.z_colT_sf = sv + SL.off[MXMOE_SAVED_Z_COLT_SF];
+  g.scale_rule = recipe_scale_rule(recipe);
   g.gu = rc ? nullptr : reinterpret_cast<uint16_t*>(sv + SL.off[MXMOE_SAVED_GU]);
   {
     StageScope sc(MXMOE_STAGE_FC1_SWIGLU, st);
@@ -621,7 +644,8 @@ mxmoe_status grouped_mlp_bwd_ex(const void* dy_dev, const void* saved_dev, size_
   mxmoe_status s;
   if (T > 0) {
     StageScope sc(MXMOE_STAGE_QUANT_DY, st);
-    s = mxfp8_quantize(dy_dev, MXMOE_DTYPE_BF16, 1, T, H, tor, seg_off + E, cap, &dy_row, &dy_col, stream);
+    s = mxfp8_quantize_ex(dy_dev, MXMOE_DTYPE_BF16, 1, T, H, tor, seg_off + E, cap, &dy_row, &dy_col,
+                          recipe_scale_rule(recipe), stream);
     if (s != MXMOE_OK) return s;
   }
   // 1b. G / U recomputed from the saved rowwise x (the fc1 GEMM again, epilogue writing
@@ -656,6 +680,7 @@ mxmoe_status grouped_mlp_bwd_ex(const void* dy_dev, const void* saved_dev, size_
     g.dgu_colT_sf = ws + W.dgu_colT_sf;
     g.dprob_part = reinterpret_cast<float*>(ws + W.dprob_part);
     g.out_fmt = grad_format;
+    g.scale_rule = recipe_scale_rule(recipe);
     StageScope sc(MXMOE_STAGE_FC2_DGRAD, st);
     if (T > 0 && launch_gemm(g, st) != cudaSuccess) return MXMOE_ERR_CUDA;
   }

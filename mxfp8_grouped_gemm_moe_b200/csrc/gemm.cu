@@ -219,8 +219,8 @@ __device__ __forceinline__ uint32_t amax_bits32(const float (&v)[32]) {
 // 32 fp32 -> 32 FP8 codes of format FMT (8 words) under the block's scale; returns the
 // E8M0 byte.
 template <int FMT = MXMOE_FMT_E4M3>
-__device__ __forceinline__ uint8_t quant32(const float (&v)[32], uint32_t (&q)[8]) {
-  const int32_t X = mx_scale_exp_from_amax_bits<FMT>(amax_bits32(v));
+__device__ __forceinline__ uint8_t quant32(const float (&v)[32], uint32_t (&q)[8], bool ceil_rule = false) {
+  const int32_t X = mx_scale_exp_from_amax_bits<FMT>(amax_bits32(v), ceil_rule);
   const float sc = mx_inv_scale(X);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -261,11 +261,12 @@ __device__ __forceinline__ void colwise_transpose2(const float (&v0)[32], const 
 }
 template <int FMT = MXMOE_FMT_E4M3>
 __device__ __forceinline__ void colwise_codes2(const float (&v0)[32], const float (&v1)[32], float* stg, int lane,
-                                               uint32_t (&q0)[8], uint32_t (&q1)[8], uint8_t& sb0, uint8_t& sb1) {
+                                               uint32_t (&q0)[8], uint32_t (&q1)[8], uint8_t& sb0, uint8_t& sb1,
+                                               bool ceil_rule = false) {
   float w0[32], w1[32];
   colwise_transpose2(v0, v1, stg, lane, w0, w1);
-  sb0 = quant32<FMT>(w0, q0);
-  sb1 = quant32<FMT>(w1, q1);
+  sb0 = quant32<FMT>(w0, q0, ceil_rule);
+  sb1 = quant32<FMT>(w1, q1, ceil_rule);
 }
 // bf16 output mode: lane r's 32 values as 64 bytes of bf16 at box + r * 64 (one row of a
 // 32 x 32 bf16 box).
@@ -720,9 +721,10 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
         }
         uint32_t r0[8], r1[8], c0[8], c1[8];
         uint8_t cs0, cs1;
-        const uint32_t zsf = (uint32_t)quant32(z0, r0) | ((uint32_t)quant32(z1, r1) << 8);
+        const bool cr = g.scale_rule != 0;
+        const uint32_t zsf = (uint32_t)quant32(z0, r0, cr) | ((uint32_t)quant32(z1, r1, cr) << 8);
         staging_acquire(lane);
-        colwise_codes2(z0, z1, stg, lane, c0, c1, cs0, cs1);
+        colwise_codes2(z0, z1, stg, lane, c0, c1, cs0, cs1, cr);
         put_codes32(stg8, lane, r0);
         put_codes32(stg8 + 1024, lane, r1);
         put_codes32(stg8 + 2048, lane, c0);
@@ -827,10 +829,11 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           }
           uint32_t rg[8], ru[8], cg[8], cu[8];
           uint8_t csg, csu;
-          sfg |= (uint32_t)quant32<OF>(vg, rg) << (8 * c);
-          sfu |= (uint32_t)quant32<OF>(vu, ru) << (8 * c);
+          const bool cr = g.scale_rule != 0;
+          sfg |= (uint32_t)quant32<OF>(vg, rg, cr) << (8 * c);
+          sfu |= (uint32_t)quant32<OF>(vu, ru, cr) << (8 * c);
           staging_acquire(lane);
-          colwise_codes2<OF>(vg, vu, stg, lane, cg, cu, csg, csu);
+          colwise_codes2<OF>(vg, vu, stg, lane, cg, cu, csg, csu, cr);
           uint8_t* stg8 = reinterpret_cast<uint8_t*>(stg);
           put_codes32(stg8, lane, rg);
           put_codes32(stg8 + 1024, lane, ru);

@@ -28,12 +28,16 @@ __device__ __forceinline__ void record_timeout(int32_t where) { record_error(MXM
 // Scale exponent X = clamp(floor(log2(amax)) - emax, -127, 127) from the bit pattern of a
 // non-negative fp32 amax (emax = 8 for E4M3 elements, 15 for E5M2); zero or subnormal
 // amax gives the lower clamp (-127).
+// With ceil_rule the exponent is one higher when amax's significand exceeds 1.75 (both
+// formats' largest value is 1.75 * 2^emax): the smallest power-of-two scale under which no
+// element saturates.
 template <int FMT = MXMOE_FMT_E4M3>
-__device__ __forceinline__ int32_t mx_scale_exp_from_amax_bits(uint32_t amax_bits) {
+__device__ __forceinline__ int32_t mx_scale_exp_from_amax_bits(uint32_t amax_bits, bool ceil_rule = false) {
   constexpr int32_t kEmax = FMT == MXMOE_FMT_E4M3 ? 8 : 15;  // largest exponent of the element format
   const int32_t ef = (int32_t)((amax_bits >> 23) & 0xFFu);
   if (ef == 0) return -127;
   int32_t X = ef - 127 - kEmax;
+  if (ceil_rule && (amax_bits & 0x7FFFFFu) > 0x600000u) ++X;
   return X < -127 ? -127 : (X > 127 ? 127 : X);
 }
 
@@ -54,11 +58,11 @@ __device__ __forceinline__ uint16_t e4m3x2(float a, float b) { return fp8x2<MXMO
 // Quantise 32 fp32 values held by one thread -> 32 codes packed in 8 words; returns the
 // E8M0 scale byte.
 template <int FMT = MXMOE_FMT_E4M3>
-__device__ __forceinline__ uint8_t quant_block32(const float (&v)[32], uint32_t (&out)[8]) {
+__device__ __forceinline__ uint8_t quant_block32(const float (&v)[32], uint32_t (&out)[8], bool ceil_rule = false) {
   uint32_t amax = 0;
 #pragma unroll
   for (int i = 0; i < 32; ++i) amax = max(amax, __float_as_uint(fabsf(v[i])));
-  const int32_t X = mx_scale_exp_from_amax_bits<FMT>(amax);
+  const int32_t X = mx_scale_exp_from_amax_bits<FMT>(amax, ceil_rule);
   const float s = mx_inv_scale(X);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {

@@ -45,7 +45,8 @@ struct QuantArgs {
   // > 0: the rowwise copy of each [2*row_ilv, cols] batch matrix stores its rows in
   // 64-row blocks interleaved [first half 0..63, second half 0..63, first 64..127, ...]
   int64_t row_ilv;
-  int32_t fmt;  // element format of both outputs: MXMOE_FMT_E4M3 or MXMOE_FMT_E5M2
+  int32_t fmt;         // element format of both outputs: MXMOE_FMT_E4M3 or MXMOE_FMT_E5M2
+  int32_t scale_rule;  // MXMOE_SCALE_RULE_OCP or MXMOE_SCALE_RULE_CEIL
 };
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
 // bf16 -> bf16 copies with the same row gather / valid-row count / gate-up interleave as
@@ -98,6 +99,7 @@ struct GemmArgs {
   uint8_t* dgu_colT_sf;
   float* dprob_part;  // [rows_cap, F/128]
   int32_t out_fmt;    // element format of the fused epilogues' MXFP8 outputs (Z / dGU)
+  int32_t scale_rule; // scale rule of the fused epilogues' quantisers (MXMOE_SCALE_RULE_*)
   // debug: if non-zero, the MMA warp withholds its first accumulator-ready signal so
   // that the epilogue's bounded wait expires (tests the timeout path; never set in
   // normal use)

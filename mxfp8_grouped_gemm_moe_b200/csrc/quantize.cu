@@ -87,12 +87,13 @@ __device__ __forceinline__ void load_pair(const float* p, float& a, float& b) {
 // the block amax is a SIMD max over the masked words; the result equals the amax of the
 // values widened to fp32 (widening is exact), hence the same scale as quant_block32.
 template <int FMT = MXMOE_FMT_E4M3>
-__device__ __forceinline__ uint8_t quant_block32_bf16(const uint32_t (&w)[16], uint32_t (&out)[8]) {
+__device__ __forceinline__ uint8_t quant_block32_bf16(const uint32_t (&w)[16], uint32_t (&out)[8],
+                                                      bool ceil_rule = false) {
   uint32_t m = 0;
 #pragma unroll
   for (int i = 0; i < 16; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
   const uint32_t amax = max(m << 16, m & 0xFFFF0000u);
-  const int32_t X = mx_scale_exp_from_amax_bits<FMT>(amax);
+  const int32_t X = mx_scale_exp_from_amax_bits<FMT>(amax, ceil_rule);
   const float s = mx_inv_scale(X);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -107,12 +108,12 @@ __device__ __forceinline__ uint8_t quant_block32_bf16(const uint32_t (&w)[16], u
 // its low half and (column c+1, row r) in its high half.
 template <int FMT = MXMOE_FMT_E4M3>
 __device__ __forceinline__ void quant_colpair_bf16(const uint32_t (&w)[32], uint32_t (&o0)[8], uint32_t (&o1)[8],
-                                                   uint8_t& sb0, uint8_t& sb1) {
+                                                   uint8_t& sb0, uint8_t& sb1, bool ceil_rule = false) {
   uint32_t m = 0;
 #pragma unroll
   for (int i = 0; i < 32; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
-  const int32_t X0 = mx_scale_exp_from_amax_bits<FMT>(m << 16);
-  const int32_t X1 = mx_scale_exp_from_amax_bits<FMT>(m & 0xFFFF0000u);
+  const int32_t X0 = mx_scale_exp_from_amax_bits<FMT>(m << 16, ceil_rule);
+  const int32_t X1 = mx_scale_exp_from_amax_bits<FMT>(m & 0xFFFF0000u, ceil_rule);
   const float s0 = mx_inv_scale(X0), s1 = mx_inv_scale(X1);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -126,40 +127,40 @@ __device__ __forceinline__ void quant_colpair_bf16(const uint32_t (&w)[32], uint
 }
 
 template <int FMT>
-__device__ __forceinline__ uint8_t quant_row_block(const __nv_bfloat16* p, uint32_t (&q)[8]) {
+__device__ __forceinline__ uint8_t quant_row_block(const __nv_bfloat16* p, uint32_t (&q)[8], bool ceil_rule) {
   uint32_t w[16];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint4 v = reinterpret_cast<const uint4*>(p)[i];
     w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
   }
-  return quant_block32_bf16<FMT>(w, q);
+  return quant_block32_bf16<FMT>(w, q, ceil_rule);
 }
 template <int FMT>
-__device__ __forceinline__ uint8_t quant_row_block(const float* p, uint32_t (&q)[8]) {
+__device__ __forceinline__ uint8_t quant_row_block(const float* p, uint32_t (&q)[8], bool ceil_rule) {
   float v[32];
   load32_row(p, v);
-  return quant_block32<FMT>(v, q);
+  return quant_block32<FMT>(v, q, ceil_rule);
 }
 
 template <int FMT>
 __device__ __forceinline__ void quant_col_pair(const __nv_bfloat16* p, int ld, uint32_t (&q0)[8], uint32_t (&q1)[8],
-                                               uint8_t& s0, uint8_t& s1) {
+                                               uint8_t& s0, uint8_t& s1, bool ceil_rule) {
   uint32_t w[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) w[i] = *reinterpret_cast<const uint32_t*>(p + i * ld);
-  quant_colpair_bf16<FMT>(w, q0, q1, s0, s1);
+  quant_colpair_bf16<FMT>(w, q0, q1, s0, s1, ceil_rule);
 }
 template <int FMT>
 __device__ __forceinline__ void quant_col_pair(const float* p, int ld, uint32_t (&q0)[8], uint32_t (&q1)[8],
-                                               uint8_t& s0, uint8_t& s1) {
+                                               uint8_t& s0, uint8_t& s1, bool ceil_rule) {
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = p[i * ld];
-  s0 = quant_block32<FMT>(v, q0);
+  s0 = quant_block32<FMT>(v, q0, ceil_rule);
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = p[i * ld + 1];
-  s1 = quant_block32<FMT>(v, q1);
+  s1 = quant_block32<FMT>(v, q1, ceil_rule);
 }
 
 // One CTA per 128 x 128 tile (many resident per SM to overlap load latency).
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
       const int64_t col = c0 + 32 * blk;
       if (orow >= nvalid || col >= a.cols) continue;
       uint32_t q[8];
-      const uint8_t sb = quant_row_block<FMT>(tile + tile_off<T>(row, 32 * blk), q);
+      const uint8_t sb = quant_row_block<FMT>(tile + tile_off<T>(row, 32 * blk), q, a.scale_rule != 0);
       int64_t drow = orow;
       if (a.row_ilv > 0) {  // gate / up interleave of the fc1 operand
         const int64_t hf = orow >= a.row_ilv, rr = orow - hf * a.row_ilv;
@@ -238,7 +239,7 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
     if (orow < nvalid && col < a.cols) {
       uint32_t q0[8], q1[8];
       uint8_t s0, s1;
-      quant_col_pair<FMT>(tile + tile_off<T>(32 * rb, 2 * pcol), 4 * Tr::kBS, q0, q1, s0, s1);
+      quant_col_pair<FMT>(tile + tile_off<T>(32 * rb, 2 * pcol), 4 * Tr::kBS, q0, q1, s0, s1, a.scale_rule != 0);
       const int64_t grow = b * a.cols + col;  // row of the transposed matrix
       uint4* d0 = reinterpret_cast<uint4*>(a.col_data + grow * a.out_rows + orow);
       uint4* d1 = reinterpret_cast<uint4*>(a.col_data + (grow + 1) * a.out_rows + orow);
@@ -344,7 +345,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
         w[4 * t] = v.x; w[4 * t + 1] = v.y; w[4 * t + 2] = v.z; w[4 * t + 3] = v.w;
       }
       uint32_t q[8];
-      const uint8_t sb = quant_block32_bf16(w, q);
+      const uint8_t sb = quant_block32_bf16(w, q, a.scale_rule != 0);
       *reinterpret_cast<uint4*>(out_row + sw128(row, 2 * blk)) = make_uint4(q[0], q[1], q[2], q[3]);
       *reinterpret_cast<uint4*>(out_row + sw128(row, 2 * blk + 1)) = make_uint4(q[4], q[5], q[6], q[7]);
       const int64_t orow = r0 + row;
@@ -365,7 +366,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
       for (int r = 0; r < 32; ++r) w[r] = *reinterpret_cast<const uint32_t*>(st + qt_off(32 * rb + r, 2 * pcol));
       uint32_t q0[8], q1[8];
       uint8_t s0, s1;
-      quant_colpair_bf16(w, q0, q1, s0, s1);
+      quant_colpair_bf16(w, q0, q1, s0, s1, a.scale_rule != 0);
       *reinterpret_cast<uint4*>(out_col + sw128(2 * pcol, 2 * rb)) = make_uint4(q0[0], q0[1], q0[2], q0[3]);
       *reinterpret_cast<uint4*>(out_col + sw128(2 * pcol, 2 * rb + 1)) = make_uint4(q0[4], q0[5], q0[6], q0[7]);
       *reinterpret_cast<uint4*>(out_col + sw128(2 * pcol + 1, 2 * rb)) = make_uint4(q1[0], q1[1], q1[2], q1[3]);

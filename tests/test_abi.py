@@ -67,7 +67,12 @@ def test_sizes_are_host_only(lib):
 
 
 def test_host_argument_errors_enqueue_nothing(lib):
-    """Every one of these is rejected before any CUDA call (so it runs without a GPU)."""
+    """Every one of these is rejected before any CUDA call (so it runs without a GPU).
+    The calls pass fake device addresses: should a check ever let one through, the call
+    would reach a kernel launch, so the test refuses to run where a GPU is visible."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("passes fake device pointers; host-only test")
     import mxfp8_grouped_gemm_moe_b200 as mx
     P = ctypes.c_void_p
     bad = P(0)
@@ -116,12 +121,17 @@ def test_host_argument_errors_enqueue_nothing(lib):
                                16, S) == 3
     assert lib.grouped_mlp_bwd(fake, fake, 1 << 40, fake, 1 << 40, 16, 2, 4, 256, 512, fake, bad, fake, fake,
                                fake, 1 << 40, S) == 1
-    # recipe flags: only MXMOE_RECIPE_GRAD_E5M2 | MXMOE_RECIPE_RECOMPUTE_GU
-    assert lib.grouped_mlp_bwd_ex(fake, fake, 1 << 40, fake, 1 << 40, 16, 2, 4, 256, 512, 4, fake, fake, fake, fake,
+    # recipe flags: only MXMOE_RECIPE_GRAD_E5M2 | _RECOMPUTE_GU | _SCALE_CEIL (1 | 2 | 4)
+    assert lib.grouped_mlp_bwd_ex(fake, fake, 1 << 40, fake, 1 << 40, 16, 2, 4, 256, 512, 8, fake, fake, fake, fake,
                                   fake, 1 << 40, S) == 1
-    assert lib.grouped_mlp_fwd_ex(fake, fake, fake, fake, 1 << 40, 16, 2, 4, 256, 512, 8, fake, fake, 1 << 40, fake,
+    assert lib.grouped_mlp_fwd_ex(fake, fake, fake, fake, 1 << 40, 16, 2, 4, 256, 512, 16, fake, fake, 1 << 40, fake,
                                   1 << 40, S) == 1
-    assert lib.grouped_mlp_saved_size_ex(16, 2, 4, 256, 512, 4) == 0
+    assert lib.grouped_mlp_saved_size_ex(16, 2, 4, 256, 512, 8) == 0
+    assert lib.grouped_mlp_saved_size_ex(16, 2, 4, 256, 512, 7) > 0
+    # scale rules: only OCP (0) and CEIL (1)
+    m_ok = mx._MX(1 << 20, 1 << 20, 64, 64, 0, 0)
+    assert lib.mxfp8_quantize_ex(fake, 0, 1, 64, 64, None, None, 64, ctypes.byref(m_ok), None, 2, S) == 1
+    assert lib.mxmoe_weights_quantize_ex(fake, fake, 2, 256, 512, -1, fake, 1 << 40, S) == 1
     # the recompute recipe saves the rowwise input instead of G / U: smaller saved buffer,
     # larger workspace (G / U recomputed there)
     a = (4096, 2, 8, 1024, 2816)

@@ -182,3 +182,75 @@ def test_recompute_gu_is_bit_identical(gpu_lib, grad_format):
     codes = rc.saved_field("x_row", torch.uint8, cap * cfg.H).view(cap, cfg.H)
     np.testing.assert_array_equal(u8(codes)[:Mp["Mp"]], qr)
     assert rc.saved.numel() < base.saved.numel() - cap * 2 * cfg.F * 2 + cap * cfg.H * 1.04
+
+
+# ----------------------------------------------------------------------------- "ceil" scale rule
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("layout", [0, 1])
+def test_quantize_ceil_rule_matches_oracle(gpu_lib, dtype, fmt, layout):
+    """Bytes and scales bit-exact under the round-up scale rule, incl. blocks the OCP rule
+    would saturate (bf16 E4M3 with 128-multiple shapes runs the dense TMA kernel)."""
+    R, C = 256, 384
+    x = wl.random_matrix(R, C, seed=91, dtype=torch.float32)
+    g = torch.Generator().manual_seed(3)
+    x = x * torch.exp2(torch.randint(-30, 30, (R, 1), generator=g).float())
+    x[7, 3] = 480.0 * 2.0 ** 5                  # E4M3: saturates under the OCP rule
+    x[9, 40] = 61440.0 * 2.0 ** -3              # E5M2: saturates under the OCP rule
+    x[3, :40] = 0.0
+    x = x.to(dtype)
+    f = gpu_lib.FMT_E5M2 if fmt == "e5m2" else gpu_lib.FMT_E4M3
+    r, c = gpu_lib.mxfp8_quantize(x.cuda(), layout=layout, fmt=f, scale_rule=gpu_lib.SCALE_RULE_CEIL)
+    torch.cuda.synchronize()
+    qr, sr = omx.quantize_rowwise(f64(x), fmt, "ceil")
+    qc, sc = omx.quantize_colwise_t(f64(x), fmt, "ceil")
+    np.testing.assert_array_equal(u8(r.data), qr)
+    np.testing.assert_array_equal(u8(r.scale_plain()), sr)
+    np.testing.assert_array_equal(u8(c.data), qc)
+    np.testing.assert_array_equal(u8(c.scale_plain()), sc)
+    assert not np.array_equal(sr, omx.quantize_rowwise(f64(x), fmt)[1])   # the rule made a difference
+
+
+def test_weights_quantize_ceil_rule(gpu_lib):
+    E, H, F = 2, 256, 512
+    W1 = wl.random_matrix(2 * F, H, seed=43, std=0.02, batch=E)
+    W2 = wl.random_matrix(H, F, seed=44, std=0.02, batch=E)
+    wq = gpu_lib.mxmoe_weights_quantize(W1.cuda(), W2.cuda(), scale_rule=gpu_lib.SCALE_RULE_CEIL)
+    torch.cuda.synchronize()
+    v = [gpu_lib.mxmoe_weights_view(wq, E, H, F, w) for w in range(4)]
+    r = np.arange(2 * F)
+    hf, rr = (r >= F).astype(int), r - (r >= F) * F
+    dst = (rr // 64) * 128 + hf * 64 + rr % 64
+    for e in range(E):
+        qr, sr = omx.quantize_rowwise(f64(W1[e]), "e4m3", "ceil")
+        np.testing.assert_array_equal(u8(v[0].data)[e * 2 * F:(e + 1) * 2 * F][dst], qr)
+        np.testing.assert_array_equal(u8(v[0].scale_plain())[e * 2 * F:(e + 1) * 2 * F][dst], sr)
+        qc, sc = omx.quantize_colwise_t(f64(W2[e]), "e4m3", "ceil")
+        np.testing.assert_array_equal(u8(v[3].data)[e * F:(e + 1) * F], qc)
+        np.testing.assert_array_equal(u8(v[3].scale_plain())[e * F:(e + 1) * F], sc)
+
+
+@pytest.mark.parametrize("grad_format", ["e4m3", "e5m2"])
+def test_fused_layer_ceil_rule_matches_oracle(gpu_lib, grad_format):
+    """Forward and backward with every quantiser on the round-up rule (the weights too)."""
+    cfg = wl.custom("tiny_fb", T=1024, H=256, F=512, E=4, k=2, seed=1)
+    d = wl.make_all(cfg)
+    dev = {k: (v.cuda() if v is not None else None) for k, v in d.items()}
+    gpu_lib.mxmoe_clear_device_status()
+    layer, y, (dx, dW1, dW2, dprobs) = _layer_run(gpu_lib, cfg, dev, grad_format=grad_format, scale_rule="ceil")
+    st, where = gpu_lib.mxmoe_get_device_status()
+    assert st == 0, (st, where)
+    x, W1, W2, probs = f64(d["x"]), f64(d["W1"]), f64(d["W2"]), f64(d["probs"])
+    yo, saved = omoe.mlp_fwd(x, d["topk_idx"].numpy(), probs, W1, W2, scale_rule="ceil")
+    go = omoe.mlp_bwd(f64(d["dy"]), saved, probs, W1, W2, grad_fmt=grad_format)
+    errs = dict(y=rel_l2(f64(y), yo), dx=rel_l2(f64(dx), go["dx"]), dW1=rel_l2(f64(dW1), go["dW1"]),
+                dW2=rel_l2(f64(dW2), go["dW2"]), dprobs=rel_l2(f64(dprobs), go["dprobs"]))
+    print(grad_format, {k: f"{v:.2e}" for k, v in errs.items()})
+    # The GPU computes dGU in fp32 from a bf16 dZ, the oracle in fp64: near rounding
+    # midpoints the two pick neighbouring codes. Such flips are rarer and larger as the code
+    # step grows, so the relative L2 error grows as the square root of the step: E5M2
+    # gradients (one mantissa bit fewer) get sqrt(2) times the E4M3 bar.
+    tol = TOL_E2E * (np.sqrt(2.0) if grad_format == "e5m2" else 1.0)
+    for k, v in errs.items():
+        assert v <= tol, (k, v)
