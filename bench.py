@@ -22,6 +22,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -71,11 +72,17 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_hash(paths):
+_COMMENT = re.compile(r"//[^\n]*|/\*.*?\*/", re.S)
+
+
+def source_hash(paths, root=ROOT):
+    """Hash of the kernel sources' code: comments and whitespace are dropped, so that a
+    change to the comments alone keeps a traffic measurement valid."""
     h = hashlib.sha256()
     for p in paths:
-        with open(os.path.join(ROOT, p), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(root, p), encoding="utf-8") as f:
+            code = _COMMENT.sub(" ", f.read())
+        h.update(" ".join(code.split()).encode())
     return h.hexdigest()[:16]
 
 

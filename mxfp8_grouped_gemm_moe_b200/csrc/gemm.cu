@@ -19,16 +19,23 @@
 //        a B tile crosses L2 -> SM once per pair instead of once per CTA; every TMA of
 //        both CTAs completes on the leader's stage barrier and the leader's commits
 //        release the stage in both CTAs (multicast commit; the loads themselves are
-//        never multicast). 6-stage ring of 34 KB.
-//      PAIR = 1: one CTA per SM, tile 128 x 256, 4-stage ring of 50 KB.
+//        never multicast). Ring of 34 KB stages: 5 for the plain-store and weight-
+//        gradient modes, 4 for the fused modes.
+//      PAIR = 1: one CTA per SM, tile 128 x 256, 3-stage ring of 50 KB.
 //    Each CTA ends a tile with the same 128 x 256 fp32 accumulator in its own TMEM, so
 //    the epilogues are shared by both variants;
-//  * K step 128; operand tiles use the 128-byte swizzle; the E8M0 scales arrive in the
-//    tensor cores' scale order and are moved to TMEM with tcgen05.cp;
-//  * warp 0 issues the copies, warp 1 issues tcgen05.mma (kind::mxf8f6f4, block32
-//    scales), warps 4..11 are the epilogue: they drain the accumulator from TMEM into
-//    registers (or spare TMEM columns), hand it back to the MMA warp at once, then run
-//    the epilogue math and stores while the next tile's MMAs proceed;
+//  * K step 128 bytes; operand tiles use the 128-byte swizzle. MXFP8 operands (ESZ = 1;
+//    E4M3 or E5M2, per operand, in the instruction descriptor): the E8M0 scales arrive in
+//    the tensor cores' scale order and are moved to TMEM with tcgen05.cp, and the MMA is
+//    kind::mxf8f6f4 with block-32 scales. bf16 operands (ESZ = 2, CTA pairs): kind::f16,
+//    no scales; the fused epilogues then write bf16 instead of MXFP8;
+//  * warp 0 issues the copies, warp 1 issues tcgen05.mma; the epilogue warps (2..9 for
+//    plain stores and weight gradients, 4..11 for the fused modes, which run 12 warps
+//    with a register split) drain the accumulator from TMEM into registers (or spare
+//    TMEM columns), hand it back to the MMA warp at once, then run the epilogue math and
+//    stores while the next tile's MMAs proceed. The fused epilogues' quantisers take a
+//    scale rule (OCP, or rounded up so nothing saturates) and the backward's an element
+//    format (E4M3, or E5M2 for gradients);
 //  * every wait is bounded (1 s) and reports MXMOE_ERR_DEVICE_TIMEOUT instead of
 //    hanging; the segment offsets are checked on the device before any tile is issued.
 #include <cuda.h>

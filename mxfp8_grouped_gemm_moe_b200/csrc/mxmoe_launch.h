@@ -57,7 +57,7 @@ cudaError_t launch_bf16_copy(const QuantArgs& a, cudaStream_t st);
 // ---------------------------------------------------------------- grouped GEMM
 enum GemmMode : int32_t {
   kModeStore = 0,       // C = A . B_e^T, bf16 or fp32 out (M grouped by expert segments)
-  kModeSwigluFwd = 1,   // fc1 + SwiGLU x prob -> MXFP8 Z (row + colT), GU bf16 saved
+  kModeSwigluFwd = 1,   // fc1 + SwiGLU x prob -> MXFP8 Z (row + colT) and / or G, U bf16 (each optional)
   kModeSwigluBwd = 2,   // fc2 dgrad + SwiGLU/prob backward -> MXFP8 dGU (row + colT), dprob partials
   kModeWgrad = 3,       // C[e] = At_e . Bt_e^T, fp32, contraction over the expert's rows
 };

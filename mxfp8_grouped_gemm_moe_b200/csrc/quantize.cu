@@ -6,7 +6,8 @@
 // conversions are fused rather than run as separate operations. Element / scale rule:
 // OCP MX (E4M3 elements, E8M0 scale, X = clamp(floor(log2 amax) - 8, -127, 127),
 // round-to-nearest-even with saturation); E5M2 elements (largest exponent 15 in place of
-// 8) for the gradient variant, on the gathered per-tile path.
+// 8) for the gradient variant, on the per-tile path; either scale rule (OCP, or the
+// exponent rounded up so that nothing saturates) on both paths.
 //
 // One CTA quantises a 128 x 128 tile staged in shared memory: rowwise blocks (32
 // consecutive columns of a row) and colwise blocks (32 consecutive rows of a column,
