@@ -169,3 +169,8 @@ def test_layer_arguments_checked_before_allocation(lib):
     b = mx.GroupedMLP(64, 2, 4, 256, 512, device="cpu", recompute_gu=True)
     assert a.recipe == 0 and b.recipe == mx.RECIPE_RECOMPUTE_GU
     assert b.saved.numel() < a.saved.numel()
+    c = mx.GroupedMLP(64, 2, 4, 256, 512, device="cpu", grad_format="e5m2", scale_rule="ceil")
+    assert c.recipe == mx.RECIPE_GRAD_E5M2 | mx.RECIPE_SCALE_CEIL and c.scale_rule == mx.SCALE_RULE_CEIL
+    assert c.saved.numel() == a.saved.numel()
+    with pytest.raises(ValueError):
+        mx.GroupedMLP(16, 2, 4, 256, 512, device="cpu", scale_rule="floor")
