@@ -18,7 +18,11 @@ reading, and each function's docstring says which.
 
 Pins (tests marked ``not gpu``): exhaustive E4M3 round trip, hand-built
 quantisation blocks, brute-force permutation, per-token loop == grouped forward,
-dense-MLP reduction, SwiGLU closed forms, finite differences of the backward; for the
+dense-MLP reduction, SwiGLU closed forms, finite differences of the backward (quantisation
+off); the quantised backward equals ``moe.mlp_bwd_per_expert``, an expert-by-expert
+restatement that quantises each backward GEMM's operands along that GEMM's contraction
+index in an explicit block loop (a planted swap of any operand's block direction fails
+it); for the
 router (``router``): softmax closed forms, brute-force top-k with ties, -inf experts,
 finite differences of the top-k backward.
 Parity unpinned: the end-to-end numeric level against the pages (they print no

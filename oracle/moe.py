@@ -274,3 +274,90 @@ def mlp_per_token(x, topk_idx, probs, W1, W2, quant=True):
             zq = _fq_row(z[None, :], quant)[0]
             y[t] += W2q[e] @ zq
     return y
+
+
+# ----------------------------------------------------------------------------- independent restatement
+
+def _fake_quant_along(a, axis, fmt="e4m3", rule="ocp"):
+    """Quantise then dequantise a 2-D fp64 matrix in blocks of 32 consecutive entries
+    along ``axis`` (1: along each row; 0: down each column). When the axis length is not a
+    multiple of 32 the last block is short: its scale is taken over the entries it has (as
+    if zero-padded to 32) and only those entries are returned. Written as a plain loop over
+    the blocks, each gathered into a [.., 32] array for ``mxfp8.quantize_blocks``."""
+    a = np.asarray(a, dtype=np.float64)
+    out = np.empty_like(a)
+    n = a.shape[axis]
+    for b0 in range(0, n, mxfp8.BLOCK):
+        b1 = min(n, b0 + mxfp8.BLOCK)
+        part = a[:, b0:b1] if axis == 1 else a[b0:b1, :].T        # [other, b1 - b0]
+        blk = np.zeros((part.shape[0], mxfp8.BLOCK), dtype=np.float64)
+        blk[:, :b1 - b0] = part
+        codes, sb = mxfp8.quantize_blocks(blk, fmt, rule)
+        deq = mxfp8.dequantize_blocks(codes, sb, fmt)[:, :b1 - b0]
+        if axis == 1:
+            out[:, b0:b1] = deq
+        else:
+            out[b0:b1, :] = deq.T
+    return out
+
+
+def mlp_bwd_per_expert(x, dy, topk_idx, probs, W1, W2, grad_fmt="e4m3", scale_rule="ocp"):
+    """The quantised backward restated one expert at a time, without the routing tables,
+    the padded permuted layout or any of the rowwise / colwise helpers above.
+
+    For each expert e its rows are the (token, slot) pairs routed to it, in token order.
+    The forward's fc1 is recomputed for those rows (x and W1 with blocks along H), then
+    each of the four backward GEMMs quantises its two operands with 32-value blocks along
+    THAT GEMM's contraction index -- the rule that lets a block's scale factor out of
+    every partial dot product ("MoE-Training für biologische Grundmodelle optimieren",
+    hyper.ai/de, MXFP8 passage: one scale per block of 32 values):
+      fc2 data gradient   dZ    = dY_e . W2_e        contracts H:   dY along H, W2_e down H;
+      fc2 weight gradient dW2_e = dY_e^T . Z_e       contracts rows: both down the rows;
+      fc1 data gradient   dX_e  = dGU_e . W1_e       contracts 2F:  dGU along 2F, W1_e down 2F;
+      fc1 weight gradient dW1_e = dGU_e^T . X_e      contracts rows: both down the rows.
+    The expert's row blocks start at its first row and its last block may be short (the
+    padded layout's zero rows change no scale). Gradients dY, dGU take ``grad_fmt``;
+    weights, x and Z stay E4M3; every quantiser takes ``scale_rule``.
+    Returns dict dx [T,H], dW1 [E,2F,H], dW2 [E,H,F], dprobs [T,k] (fp64)."""
+    x = np.asarray(x, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    probs = np.asarray(probs, dtype=np.float64)
+    idx = np.asarray(topk_idx, dtype=np.int64)
+    E, F2, H = W1.shape
+    F = F2 // 2
+    T, k = idx.shape
+    sr = scale_rule
+
+    def q(a, axis, fmt="e4m3"):
+        return _fake_quant_along(a, axis, fmt, sr)
+
+    dx = np.zeros((T, H))
+    dW1 = np.zeros((E, F2, H))
+    dW2 = np.zeros((E, H, F))
+    dprobs = np.zeros((T, k))
+    for e in range(E):
+        pairs = [(t, j) for t in range(T) for j in range(k) if idx[t, j] == e]
+        if not pairs:
+            continue                                   # no rows: zero weight gradients
+        tok = np.array([t for t, _ in pairs])
+        slot = np.array([j for _, j in pairs])
+        p = probs[tok, slot]
+        W1e = np.asarray(W1[e], dtype=np.float64)      # [2F, H]
+        W2e = np.asarray(W2[e], dtype=np.float64)      # [H, F]
+        Xe = x[tok]                                    # [m, H]
+        GU = q(Xe, 1) @ q(W1e, 1).T                    # forward fc1, contracts H
+        G, U = GU[:, :F], GU[:, F:]
+        A = silu(G) * U
+        Ze = A * p[:, None]
+        dYe = dy[tok]                                  # [m, H]
+        dZ = q(dYe, 1, grad_fmt) @ q(W2e, 0)           # contracts H
+        dprob = np.sum(dZ * A, axis=1)
+        dA = dZ * p[:, None]
+        dGU = np.concatenate([dA * U * dsilu(G), dA * silu(G)], axis=1)   # [m, 2F]
+        dW2[e] = q(dYe, 0, grad_fmt).T @ q(Ze, 0)      # contracts the expert's rows
+        dXe = q(dGU, 1, grad_fmt) @ q(W1e, 0)          # contracts 2F
+        dW1[e] = q(dGU, 0, grad_fmt).T @ q(Xe, 0)      # contracts the expert's rows
+        for i, (t, j) in enumerate(pairs):
+            dx[t] += dXe[i]
+            dprobs[t, j] = dprob[i]
+    return dict(dx=dx, dW1=dW1, dW2=dW2, dprobs=dprobs)

@@ -310,3 +310,110 @@ def test_ceil_scale_rule_variant():
     saturating = amax > 448.0 * np.exp2(s_ocp.astype(float) - 127)
     assert np.array_equal(s_ceil.astype(int) - s_ocp.astype(int), saturating.astype(int))
     assert saturating.any() and not saturating.all()
+
+
+# ----------------------------------------------------------------------------- quantised backward pin
+
+def _pin_problem():
+    # H != F and 2F != H, so a transposed operand cannot pass for the right one; ragged
+    # experts (about 47 rows each: a short last block of rows) and one expert with no tokens
+    cfg = wl.custom("pin", T=70, H=64, F=96, E=4, k=2, seed=21, routing="dead_last")
+    d = wl.make_all(cfg)
+    x, W1, W2, p = (d[n].double().numpy() for n in ("x", "W1", "W2", "probs"))
+    return cfg, x, W1, W2, p, d["topk_idx"].numpy(), d["dy"].double().numpy()
+
+
+def _assert_same_grads(got, want, rtol=1e-11):
+    for n in ("dx", "dW1", "dW2", "dprobs"):
+        scale = np.max(np.abs(want[n]))
+        np.testing.assert_allclose(got[n], want[n], rtol=rtol, atol=rtol * scale, err_msg=n)
+
+
+@pytest.mark.parametrize("grad_fmt", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("rule", ["ocp", "ceil"])
+def test_quantised_backward_equals_per_expert_restatement(grad_fmt, rule):
+    """The grouped, padded backward equals the expert-by-expert restatement in which each
+    backward GEMM quantises its two operands along its own contraction index (up to the
+    order of fp64 sums)."""
+    cfg, x, W1, W2, p, idx, dy = _pin_problem()
+    m = moe.route(idx, cfg.E)["m_splits"]
+    assert m[cfg.E - 1] == 0 and np.any(m % 32 != 0) and np.all(m[:-1] > 32)
+    _, saved = moe.mlp_fwd(x, idx, p, W1, W2, scale_rule=rule)
+    g = moe.mlp_bwd(dy, saved, p, W1, W2, grad_fmt=grad_fmt)
+    ge = moe.mlp_bwd_per_expert(x, dy, idx, p, W1, W2, grad_fmt=grad_fmt, scale_rule=rule)
+    _assert_same_grads(g, ge)
+    assert np.all(ge["dW1"][cfg.E - 1] == 0) and np.all(ge["dW2"][cfg.E - 1] == 0)
+
+
+def test_fake_quant_along_matches_blockwise_definition():
+    """The restatement's block loop against the hand-built definition on one column: a
+    short last block takes its scale over its own entries only."""
+    a = np.zeros((40, 1))
+    a[:32, 0] = 1.0
+    a[5, 0] = 3.0           # first block: amax 3 -> scale 2^(1-8)
+    a[32:, 0] = 0.0
+    a[35, 0] = 0.75         # short block of 8: amax 0.75 -> its own scale, value exact
+    a[36, 0] = 0.3          # 0.3 * 2^9 = 153.6; E4M3 steps by 16 in [128, 256) -> 160
+    out = moe._fake_quant_along(a, 0)
+    assert out[5, 0] == 3.0 and out[0, 0] == 1.0
+    assert out[35, 0] == 0.75
+    assert out[36, 0] == 160.0 * 2.0 ** -9
+    np.testing.assert_array_equal(moe._fake_quant_along(a.T, 1), out.T)
+
+
+def _mutated(monkeypatch, helper, call, replacement):
+    """Replace call number ``call`` (0-based) of oracle helper ``helper`` inside the
+    backward by ``replacement``; all other calls pass through."""
+    orig = getattr(moe, helper)
+    n = {"i": 0}
+
+    def patched(*a, **kw):
+        i = n["i"]
+        n["i"] += 1
+        return replacement(*a, **kw) if i in call else orig(*a, **kw)
+
+    monkeypatch.setattr(moe, helper, patched)
+
+
+def _rowwise(a, quant, fmt="e4m3", rule="ocp"):
+    return mxfp8.fake_quant_rowwise(a, fmt, rule)
+
+
+def _rowwise_seg(a, r, quant, fmt="e4m3", rule="ocp"):
+    return mxfp8.fake_quant_rowwise(a, fmt, rule)
+
+
+def _colwise(a, quant, fmt="e4m3", rule="ocp"):
+    return mxfp8.fake_quant_colwise(a, fmt, rule)
+
+
+# (helper, calls to replace, replacement): every operand of the four backward GEMMs given
+# the other block direction. In the backward, _fq_row is called for dY then dGU;
+# _fq_col_seg for dY, dGU, Z, Xp; _fq_col for W2[0..E) then W1[0..E).
+_E_PIN = 4
+MUTATIONS = {
+    "fc2_dgrad_dY_colwise": ("_fq_row", {0}, _colwise),
+    "fc1_dgrad_dGU_colwise": ("_fq_row", {1}, _colwise),
+    "fc2_wgrad_dY_rowwise": ("_fq_col_seg", {0}, _rowwise_seg),
+    "fc1_wgrad_dGU_rowwise": ("_fq_col_seg", {1}, _rowwise_seg),
+    "fc2_wgrad_Z_rowwise": ("_fq_col_seg", {2}, _rowwise_seg),
+    "fc1_wgrad_Xp_rowwise": ("_fq_col_seg", {3}, _rowwise_seg),
+    "fc2_dgrad_W2_rowwise": ("_fq_col", set(range(_E_PIN)), lambda a, quant, rule="ocp": _rowwise(a, quant, "e4m3", rule)),
+    "fc1_dgrad_W1_rowwise": ("_fq_col", set(range(_E_PIN, 2 * _E_PIN)),
+                             lambda a, quant, rule="ocp": _rowwise(a, quant, "e4m3", rule)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_per_expert_pin_catches_swapped_block_direction(monkeypatch, name):
+    """A mistake planted in the oracle's backward -- one operand quantised with blocks
+    along the wrong index -- makes it disagree with the restatement."""
+    cfg, x, W1, W2, p, idx, dy = _pin_problem()
+    assert cfg.E == _E_PIN
+    _, saved = moe.mlp_fwd(x, idx, p, W1, W2)
+    ge = moe.mlp_bwd_per_expert(x, dy, idx, p, W1, W2)
+    helper, calls, repl = MUTATIONS[name]
+    _mutated(monkeypatch, helper, calls, repl)
+    g = moe.mlp_bwd(dy, saved, p, W1, W2)
+    with pytest.raises(AssertionError):
+        _assert_same_grads(g, ge)
