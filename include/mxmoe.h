@@ -183,7 +183,9 @@ size_t moe_permute_workspace_size(int32_t T, int32_t k, int32_t E);
  *   T = 65536 with E = 128, or T = 32768 with E = 256); larger problems return
  *   MXMOE_ERR_WORKSPACE_TOO_SMALL and enqueue nothing.
  *   The first call on a device looks up the array's device address (once per device,
- *   with that device current); make that first call before any stream capture.
+ *   with that device current); make that first call before any stream capture. The
+ *   address is kept for the life of the process: calls after cudaDeviceReset (which
+ *   reloads the library's device code and may move the array) are not supported.
  *   All calls on a device share the one array: calls that may overlap on the GPU (for
  *   example on two streams without ordering between them) race and must be serialised
  *   by the caller. Nothing in the array needs clearing between calls: every word a call

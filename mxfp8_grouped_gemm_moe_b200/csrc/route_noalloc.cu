@@ -38,7 +38,10 @@ cudaError_t noalloc_scratch(void** out) {
   if (!g_noalloc_ptr[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+      cudaGetLastError();  // clear the runtime's error slot: later calls must not report it
+      return e;
+    }
     g_noalloc_ptr[dev] = p;
   }
   *out = g_noalloc_ptr[dev];

@@ -3,14 +3,18 @@
 For callers that cannot lend the library device memory per call (runtimes with a fixed
 memory plan, plain C callers without an allocator). Checked through the C ABI against
 moe_permute (which takes a workspace) on two calls in a row with different problems:
-the outputs are indices and routing probabilities, so they must match exactly.
-Kept in its own file, collected last."""
+the outputs are indices and routing probabilities, so they must match exactly. The maps
+are also compared with the oracle's routing directly. Kept in its own file, collected
+last."""
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
 import moe_workloads as wl
+from oracle import moe as omoe
+from tests.util import SEG_ALIGN
 
 pytestmark = pytest.mark.gpu
 
@@ -58,11 +62,30 @@ def test_noalloc_matches_workspace_entry_point_twice(gpu_lib):
         assert torch.equal(got["token_of_row"][:Mp], want["token_of_row"][:Mp])
         assert torch.equal(got["prob_of_row"][:Mp], want["prob_of_row"][:Mp])
         assert int(got["m_splits"].sum()) == cfg.T * cfg.k
+        # the oracle's counting sort (same 256-row segment alignment), bit for bit
+        r = omoe.route(idx.cpu().numpy(), cfg.E, align=SEG_ALIGN)
+        np.testing.assert_array_equal(got["m_splits"].cpu().numpy(), r["m_splits"])
+        np.testing.assert_array_equal(got["seg_off"].cpu().numpy(), r["seg_off"])
+        np.testing.assert_array_equal(got["row_of_slot"].cpu().numpy(), r["row_of_slot"])
+        np.testing.assert_array_equal(got["token_of_row"][:Mp].cpu().numpy(), r["token_of_row"])
+        live = r["token_of_row"] >= 0
+        want_p = probs.cpu().numpy()[r["token_of_row"][live], r["slot_of_row"][live]]
+        np.testing.assert_array_equal(got["prob_of_row"][:Mp].cpu().numpy()[live], want_p)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(gpu_lib):
+    """A problem whose scratch exceeds the fixed array is refused before anything is
+    enqueued: real device buffers are passed and stay untouched."""
     lib = gpu_lib.load()
     T, k, E = 70000, 2, 256            # needs 8 * 274 * 256 + 256 bytes > 256 KiB
-    fake = ctypes.c_void_p(1 << 20)    # never touched: the size check comes first
-    st = lib.moe_permute_noalloc(fake, fake, T, k, E, fake, fake, fake, fake, fake, ctypes.c_void_p(0))
+    idx = torch.zeros((T, k), dtype=torch.int32, device="cuda")
+    idx[:, 1] = 1
+    probs = torch.full((T, k), 0.5, dtype=torch.float32, device="cuda")
+    o = _outputs(T, k, E, lib.mxmoe_rows_capacity(T, k, E), "cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    st = lib.moe_permute_noalloc(_ptr(idx), _ptr(probs), T, k, E, _ptr(o["m_splits"]), _ptr(o["seg_off"]),
+                                 _ptr(o["row_of_slot"]), _ptr(o["token_of_row"]), _ptr(o["prob_of_row"]), stream)
     assert st == 3                      # MXMOE_ERR_WORKSPACE_TOO_SMALL
+    torch.cuda.synchronize()
+    for name in ("m_splits", "seg_off", "row_of_slot", "token_of_row"):
+        assert bool((o[name] == -7).all()), name
