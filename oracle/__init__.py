@@ -24,7 +24,11 @@ restatement that quantises each backward GEMM's operands along that GEMM's contr
 index in an explicit block loop (a planted swap of any operand's block direction fails
 it); for the
 router (``router``): softmax closed forms, brute-force top-k with ties, -inf experts,
-finite differences of the top-k backward.
+finite differences of the top-k backward; for the per-tensor FP8 recipe
+(``moe.mlp_fwd_fp8_tensor`` / ``mlp_bwd_fp8_tensor``): the fp32 multiplier against exact
+rational arithmetic, the largest magnitude onto 448, the fp32 rounding of the product, the
+2^-4 error bound, reduction to the unquantised layer under an identity quantiser, and a
+token-by-token restatement (with and without saturation of the delayed Z / dGU scales).
 Parity unpinned: the end-to-end numeric level against the pages (they print no
 accuracy, loss or worked example).
 """

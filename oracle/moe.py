@@ -361,3 +361,75 @@ def mlp_bwd_per_expert(x, dy, topk_idx, probs, W1, W2, grad_fmt="e4m3", scale_ru
             dx[t] += dXe[i]
             dprobs[t, j] = dprob[i]
     return dict(dx=dx, dW1=dW1, dW2=dW2, dprobs=dprobs)
+
+
+# ----------------------------------------------------------------------------- per-tensor FP8 recipe
+
+def mlp_fwd_fp8_tensor(x, topk_idx, probs, W1, W2, z_amax_in, align=ALIGN_ORACLE):
+    """Forward with per-tensor FP8 in place of MXFP8 (the pages' "FP8" beside "MXFP8":
+    "MoE-Training für biologische Grundmodelle optimieren", hyper.ai/de, precision passage).
+
+    Every operand is E4M3 under one fp32 multiplier per tensor (mxfp8.tensor_multiplier):
+    x (all tokens), W1[e] and W2[e] (one per expert), from their own largest magnitude
+    (current scaling). Z is produced tile by tile inside the fused step, so its multiplier
+    comes from ``z_amax_in`` -- a largest magnitude known before the step (delayed scaling,
+    e.g. the previous step's); values beyond it saturate. Returns (y, saved) where saved
+    also holds ``z_amax`` (the largest |Z| over live rows, for the next step) and the
+    multipliers."""
+    x = np.asarray(x, dtype=np.float64)
+    probs = np.asarray(probs, dtype=np.float64)
+    E, F2, H = W1.shape
+    F = F2 // 2
+    r = route(topk_idx, E, align)
+    live = r["token_of_row"] >= 0
+    p_row = np.zeros(r["Mp"], dtype=np.float64)
+    p_row[live] = probs[r["token_of_row"][live], r["slot_of_row"][live]]
+    m_x = mxfp8.tensor_multiplier(np.max(np.abs(x)))
+    m_w1 = [mxfp8.tensor_multiplier(np.max(np.abs(W1[e]))) for e in range(E)]
+    m_w2 = [mxfp8.tensor_multiplier(np.max(np.abs(W2[e]))) for e in range(E)]
+    m_z = mxfp8.tensor_multiplier(z_amax_in)
+    Xq = permute_rows(mxfp8.fake_quant_tensor(x, m_x), r["token_of_row"])
+    W1q = np.stack([mxfp8.fake_quant_tensor(W1[e], m_w1[e]) for e in range(E)])
+    W2q = np.stack([mxfp8.fake_quant_tensor(W2[e], m_w2[e]) for e in range(E)])
+    GU = grouped_gemm(Xq, W1q, r["seg_off"])
+    G, U = GU[:, :F], GU[:, F:]
+    Z = silu(G) * U * p_row[:, None]
+    Zq = mxfp8.dequantize_tensor(mxfp8.e4m3_encode(Z * np.float64(m_z)), m_z)
+    Yp = grouped_gemm(Zq, W2q, r["seg_off"])
+    y = unpermute_sum(Yp, r["row_of_slot"])
+    saved = dict(route=r, Xq=Xq, p_row=p_row, G=G, U=U, Zq=Zq, W1q=W1q, W2q=W2q,
+                 z_amax=float(np.max(np.abs(Z[live]))) if live.any() else 0.0,
+                 m=dict(x=m_x, w1=m_w1, w2=m_w2, z=m_z))
+    return y, saved
+
+
+def mlp_bwd_fp8_tensor(dy, saved, dgu_amax_in):
+    """Backward of the per-tensor FP8 recipe (straight-through estimator). dY takes its
+    multiplier from its own largest magnitude; dGU, produced inside the fused backward
+    step, from ``dgu_amax_in`` (delayed scaling). A per-tensor quantiser has no block
+    direction, so every GEMM reuses the one quantised copy of each operand (x, W1, W2 and
+    Z from the forward, dY and dGU here). Returns dict dx, dW1, dW2, dprobs and dgu_amax
+    (the largest |dGU| over live rows, for the next step)."""
+    r = saved["route"]
+    G, U, p_row = saved["G"], saved["U"], saved["p_row"]
+    W1q, W2q = saved["W1q"], saved["W2q"]
+    F = G.shape[1]
+    live = r["token_of_row"] >= 0
+    dy = np.asarray(dy, dtype=np.float64)
+    m_dy = mxfp8.tensor_multiplier(np.max(np.abs(dy)))
+    dYq = permute_rows(mxfp8.fake_quant_tensor(dy, m_dy), r["token_of_row"])
+    dZ = grouped_gemm(dYq, np.transpose(W2q, (0, 2, 1)), r["seg_off"])      # contracts H
+    A = silu(G) * U
+    dprob_row = np.sum(dZ * A, axis=1)
+    dA = dZ * p_row[:, None]
+    dGU = np.concatenate([dA * U * dsilu(G), dA * silu(G)], axis=1)
+    m_g = mxfp8.tensor_multiplier(dgu_amax_in)
+    dGUq = mxfp8.dequantize_tensor(mxfp8.e4m3_encode(dGU * np.float64(m_g)), m_g)
+    dW2 = grouped_gemm_wgrad(dYq.T, saved["Zq"].T, r["seg_off"])
+    dXp = grouped_gemm(dGUq, np.transpose(W1q, (0, 2, 1)), r["seg_off"])    # contracts 2F
+    dW1 = grouped_gemm_wgrad(dGUq.T, saved["Xq"].T, r["seg_off"])
+    dx = unpermute_sum(dXp, r["row_of_slot"])
+    dprobs = dprob_row[r["row_of_slot"]]
+    del F
+    return dict(dx=dx, dW1=dW1, dW2=dW2, dprobs=dprobs,
+                dgu_amax=float(np.max(np.abs(dGU[live]))) if live.any() else 0.0, m_dy=m_dy, m_dgu=m_g)

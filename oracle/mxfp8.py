@@ -190,3 +190,44 @@ def fake_quant_colwise(a, fmt="e4m3", rule="ocp"):
     """Colwise quantise/dequantise, returned in the original [R, C] orientation."""
     c, s = quantize_colwise_t(a, fmt, rule)
     return dequantize_rowwise(c, s, fmt).T
+
+
+# ----------------------------------------------------------------------------- per-tensor FP8
+# The pages name FP8 beside MXFP8 ("MoE-Training für biologische Grundmodelle optimieren",
+# hyper.ai/de, precision passage) without fixing its scaling. Reading: one fp32 scale per
+# tensor (per expert for the expert weights), E4M3 elements. The scale is kept as the fp32
+# multiplier that maps the tensor's largest magnitude onto E4M3's largest value:
+#   m = fp32(448 / amax), rounded to nearest (m = 1 when amax == 0);
+#   code = E4M3(fp32(v * m)): the product is rounded to fp32 first, then to E4M3 (nearest,
+#   ties to even, saturating to +-448);
+#   value = decode(code) / m.
+# Rounding the product to fp32 before the E4M3 rounding makes the code a function of two
+# fp32 roundings that any fp32 implementation reproduces exactly.
+
+FP32_MAX = float(np.finfo(np.float32).max)
+
+
+def tensor_multiplier(amax):
+    """fp32 multiplier m = 448 / amax rounded to nearest fp32; 1 when amax == 0, and the
+    largest finite fp32 when the quotient overflows (amax below about 1.3e-36)."""
+    a = np.float32(amax)
+    if a == 0:
+        return np.float32(1.0)
+    with np.errstate(over="ignore"):
+        m = np.float32(np.float32(E4M3_MAX) / a)
+    return np.float32(min(float(m), FP32_MAX))
+
+
+def quantize_tensor(v, m):
+    """Per-tensor E4M3 codes of fp32-representable values v under the multiplier m."""
+    prod = np.asarray(v, dtype=np.float32) * np.float32(m)     # fp32 product, rounded to nearest
+    return e4m3_encode(prod.astype(np.float64))
+
+
+def dequantize_tensor(codes, m):
+    """decode(code) / m in fp64."""
+    return e4m3_decode(codes) / np.float64(m)
+
+
+def fake_quant_tensor(v, m):
+    return dequantize_tensor(quantize_tensor(v, m), m)
