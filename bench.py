@@ -60,6 +60,8 @@ def parse_args():
     p.add_argument("--cpu-fslice", type=int, default=2048, help="FFN columns in the CPU oracle sample")
     p.add_argument("--no-bf16-compare", action="store_true",
                    help="skip the comparison timings (the bf16 layer's step, the alternative recipes)")
+    p.add_argument("--no-workloads", action="store_true",
+                   help="skip the other workloads' steps (Mixtral with Zipf routing, genomics)")
     return p.parse_args()
 
 
@@ -278,8 +280,9 @@ def config_json(cfg, world):
 def time_recipes(cfg, layer, W1, W2, x, idx, probs, dy, y, dx, dW1, dW2, dprobs, stream, steps):
     """The same full step (weights quantised, forward, backward) under the layer's
     alternative recipes, beside the headline: E5M2 gradients (the backward's dY and dGU in
-    E5M2), G / U recomputed in the backward instead of saved, and the round-up scale rule. CUDA events over `steps`
-    steps after two warm-up steps; the saved-activation bytes of each recipe."""
+    E5M2), G / U recomputed in the backward instead of saved, the round-up scale rule, and
+    per-tensor FP8 in place of MXFP8. CUDA events over `steps` steps after two warm-up
+    steps; the saved-activation bytes of each recipe."""
     import torch
 
     import mxfp8_grouped_gemm_moe_b200 as mx
@@ -313,6 +316,35 @@ def time_recipes(cfg, layer, W1, W2, x, idx, probs, dy, y, dx, dW1, dW2, dprobs,
                      "saved_bytes": lib.grouped_mlp_saved_size_ex(*a, recipe),
                      "workspace_bytes": lib.grouped_mlp_workspace_size_ex(*a, recipe)}
         del saved, ws
+    torch.cuda.empty_cache()
+    # per-tensor FP8 (its own layer object: weights with per-expert amax, delayed scaling of
+    # Z / dGU rolled after every step, as a training loop would)
+    fl = mx.GroupedMLP(*a, device=x.device, precision="fp8")
+    fl.quantize_weights(W1, W2)
+    fl.forward(x, idx, probs, y)
+    fl.backward(dy, dx, dW1, dW2, dprobs)
+    fl.roll_amax()
+
+    def fstep():
+        fl.quantize_weights(W1, W2)
+        fl.forward(x, idx, probs, y)
+        fl.backward(dy, dx, dW1, dW2, dprobs)
+        fl.roll_amax()
+    for _ in range(2):
+        fstep()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        fstep()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    out["fp8_tensor"] = {"ms_per_step": ms, "tflops": cfg.fwdbwd_flops / (ms * 1e-3) / 1e12,
+                         "saved_bytes": lib.grouped_mlp_saved_size_ex(*a, mx.RECIPE_FP8_TENSOR),
+                         "workspace_bytes": lib.grouped_mlp_workspace_size_ex(*a, mx.RECIPE_FP8_TENSOR),
+                         "note": "per-tensor FP8 E4M3 (one fp32 multiplier per tensor, per expert for the weights; "
+                                 "delayed scaling of Z and dGU); includes the amax passes over x, dY and the weights"}
+    del fl
     torch.cuda.empty_cache()
     out["default_saved_bytes"] = lib.grouped_mlp_saved_size(*a)
     out["note"] = ("same step as the headline under each recipe; tflops counts the headline's algorithmic FLOPs "
@@ -377,6 +409,105 @@ def time_bf16_layer(cfg, W1, W2, x, idx, probs, dy, stream, dev, steps):
            "note": "bf16 layer (grouped_mlp_bf16_fwd/bwd), same step as the headline; quant_* stages are "
                    "bf16 row + transposed copies here"}
     del layer, y, dx, dW1, dW2, dprobs
+    torch.cuda.empty_cache()
+    return out
+
+
+def hbm_stage_bytes(cfg):
+    """Algorithmic HBM bytes of the bandwidth-bound stages (one read of the inputs, one
+    write of the outputs, scales included)."""
+    return {
+        "quant_x": cfg.T * cfg.H * 2 + 2 * (cfg.M * cfg.H + cfg.M * cfg.H / 32),
+        "quant_dy": cfg.T * cfg.H * 2 + 2 * (cfg.M * cfg.H + cfg.M * cfg.H / 32),
+        "combine": cfg.M * cfg.H * 2 + cfg.T * cfg.H * 2,
+        "combine_dx": cfg.M * cfg.H * 2 + cfg.T * cfg.H * 2,
+        "quant_w1": cfg.E * 2 * cfg.F * cfg.H * (2 + 2 * (1 + 1 / 32)),
+        "quant_w2": cfg.E * cfg.F * cfg.H * (2 + 2 * (1 + 1 / 32)),
+    }
+
+
+def stage_table(cfg, stages, peaks):
+    """Per-stage mean time over the timed steps, with TFLOP/s (GEMMs) or GB/s (HBM-bound
+    stages) and the fraction of the measured peak."""
+    MHF = float(cfg.M) * cfg.H * cfg.F
+    fp8_peak = peaks["bf16_tflops_sustained"] * FP8_OVER_BF16
+    hbm_bytes = hbm_stage_bytes(cfg)
+    per = {}
+    for name, t in stages:
+        per.setdefault(name, []).append(t)
+    out = {}
+    for name, ts in per.items():
+        a = sum(ts) / len(ts)
+        ent = {"ms": a, "launches": len(ts)}
+        if name in GEMM_FLOP_FACTOR:
+            tf = GEMM_FLOP_FACTOR[name] * MHF / (a * 1e-3) / 1e12
+            ent.update(tflops=tf, frac_of_measured=tf / fp8_peak, frac_of_spec=tf / SPEC_FP8_TFLOPS)
+        elif name in hbm_bytes:
+            gbs = hbm_bytes[name] / (a * 1e-3) / 1e9
+            ent.update(gbs=gbs, frac_of_measured=gbs / peaks["hbm_gbs"])
+        out[name] = ent
+    return out
+
+
+def time_workload(name, dev, steps, warmup, peaks):
+    """One more workload's full step (weights quantised, forward, backward), timed on its
+    own with CUDA events: ms, TFLOP/s, tokens/s, per-stage fractions and the clocks seen.
+    Inputs as for the headline (routing from the CPU recipe, dense tensors from a seeded
+    CUDA generator), already resident in HBM."""
+    import torch
+
+    import moe_workloads as wl
+    import mxfp8_grouped_gemm_moe_b200 as mx
+    cfg = wl.CONFIGS[name]
+    idx_h, probs_h = wl.make_routing(cfg)
+    g = torch.Generator(device=dev)
+    g.manual_seed(cfg.seed)
+    W1 = (torch.randn((cfg.E, 2 * cfg.F, cfg.H), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    W2 = (torch.randn((cfg.E, cfg.H, cfg.F), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    x = torch.randn((cfg.T, cfg.H), generator=g, device=dev).to(torch.bfloat16)
+    dy = torch.randn((cfg.T, cfg.H), generator=g, device=dev).to(torch.bfloat16)
+    idx, probs = idx_h.to(dev), probs_h.to(dev)
+    layer = mx.GroupedMLP(cfg.T, cfg.k, cfg.E, cfg.H, cfg.F, device=dev)
+    y = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=dev)
+    dx = torch.empty_like(y)
+    dW1 = torch.empty((cfg.E, 2 * cfg.F, cfg.H), dtype=torch.float32, device=dev)
+    dW2 = torch.empty((cfg.E, cfg.H, cfg.F), dtype=torch.float32, device=dev)
+    dprobs = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        layer.quantize_weights(W1, W2)
+        layer.forward(x, idx, probs, y)
+        layer.backward(dy, dx, dW1, dW2, dprobs)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index or 0)
+    mx.mxmoe_profile_enable(64 * (steps + 1))
+    mx.mxmoe_profile_read()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    stages = mx.mxmoe_profile_read()
+    mx.mxmoe_profile_disable()
+    ms = e0.elapsed_time(e1) / steps
+    st = stage_table(cfg, stages, peaks)
+    gemm_ms = sum(v["ms"] for n, v in st.items() if n in GEMM_FLOP_FACTOR)
+    MHF = float(cfg.M) * cfg.H * cfg.F
+    m_splits = torch.bincount(idx_h.reshape(-1).long(), minlength=cfg.E)
+    out = {"config": config_json(cfg, 1), "ms_per_step": ms, "tflops": cfg.fwdbwd_flops / (ms * 1e-3) / 1e12,
+           "tokens_per_s": cfg.T / (ms * 1e-3), "gemm_tflops": 18.0 * MHF / (gemm_ms * 1e-3) / 1e12,
+           "gemm_frac_of_measured_fp8": 18.0 * MHF / (gemm_ms * 1e-3) / 1e12
+           / (peaks["bf16_tflops_sustained"] * FP8_OVER_BF16),
+           "m_splits_min_max": [int(m_splits.min()), int(m_splits.max())], "stages": st, "clocks": clk,
+           "steps": steps, "warmup": warmup}
+    del layer, W1, W2, x, dy, y, dx, dW1, dW2, dprobs
     torch.cuda.empty_cache()
     return out
 
@@ -449,6 +580,13 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
     bf16_layer = None
     if rank == 0 and world == 1 and not args.no_bf16_compare:
         bf16_layer = time_bf16_layer(cfg, W1, W2, x, idx, probs, dy, stream, dev, min(args.steps, 5))
+
+    # ---- the other workloads of the target (skewed Mixtral routing; genomics), each
+    # timed on its own after the headline
+    workloads = None
+    if rank == 0 and world == 1 and not args.no_workloads and cfg.name == "mixtral":
+        peaks0, _ = load_peaks()
+        workloads = {n: time_workload(n, dev, min(args.steps, 5), 2, peaks0) for n in ("mixtral_zipf", "genomics")}
 
     # ---- router (the step upstream of the layer; timed on its own, not part of `value`)
     router = None
@@ -565,29 +703,9 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
     # ---- per-stage times and rooflines
     peaks, peak_kind = load_peaks()
     MHF = float(cfg.M) * cfg.H * cfg.F
-    per = {}
-    for name, t in stages:
-        per.setdefault(name, []).append(t)
-    stage_json = {}
-    hbm_bytes = {
-        "quant_x": cfg.T * cfg.H * 2 + 2 * (cfg.M * cfg.H + cfg.M * cfg.H / 32),
-        "quant_dy": cfg.T * cfg.H * 2 + 2 * (cfg.M * cfg.H + cfg.M * cfg.H / 32),
-        "combine": cfg.M * cfg.H * 2 + cfg.T * cfg.H * 2,
-        "combine_dx": cfg.M * cfg.H * 2 + cfg.T * cfg.H * 2,
-        "quant_w1": cfg.E * 2 * cfg.F * cfg.H * (2 + 2 * (1 + 1 / 32)),
-        "quant_w2": cfg.E * cfg.F * cfg.H * (2 + 2 * (1 + 1 / 32)),
-    }
+    hbm_bytes = hbm_stage_bytes(cfg)
     fp8_peak = peaks["bf16_tflops_sustained"] * FP8_OVER_BF16
-    for name, ts in per.items():
-        a = sum(ts) / len(ts)
-        ent = {"ms": a, "launches": len(ts)}
-        if name in GEMM_FLOP_FACTOR:
-            tf = GEMM_FLOP_FACTOR[name] * MHF / (a * 1e-3) / 1e12
-            ent.update(tflops=tf, frac_of_measured=tf / fp8_peak, frac_of_spec=tf / SPEC_FP8_TFLOPS)
-        elif name in hbm_bytes:
-            gbs = hbm_bytes[name] / (a * 1e-3) / 1e9
-            ent.update(gbs=gbs, frac_of_measured=gbs / peaks["hbm_gbs"])
-        stage_json[name] = ent
+    stage_json = stage_table(cfg, stages, peaks)
     gemm_names = [n for n in stage_json if n in GEMM_FLOP_FACTOR]
     dom = max(gemm_names, key=lambda n: stage_json[n]["ms"])
     dom_units = GEMM_FLOP_FACTOR[dom] * MHF
@@ -614,6 +732,8 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
             "gemm_frac_of_measured_fp8": (18.0 * MHF) / (gemm_ms * 1e-3) / 1e12 / fp8_peak,
             "roofline": roofline, "roofline_hbm": roofline_hbm, "stages": stage_json,
             "gpu_launches": launches, "e2e": e2e, "clocks": clk, "router": router}
+    if workloads is not None:
+        line["workloads"] = workloads
     if recipes is not None:
         line["recipes"] = recipes
     if bf16_layer is not None:

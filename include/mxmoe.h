@@ -262,6 +262,20 @@ mxmoe_status grouped_gemm_mxfp8(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, cons
                                 void* stream);
 
 /*
+ * grouped_gemm_mxfp8_debug_timeout -- test hook for the device-timeout path (failure
+ * detection; no counterpart in the pages). The same call as grouped_gemm_mxfp8, except
+ * that the first CTA pair's MMA issuer withholds its first accumulator-ready signal: that
+ * pair's epilogue warps wait for it until the wait limit (1 s) runs out, record
+ * MXMOE_ERR_DEVICE_TIMEOUT in the device status word and stop; the pair's other roles stop
+ * at their own limits, wait for their issued copies and MMAs, release TMEM and return. The
+ * kernel ends (no hang, no trap) with C only partly written; the context stays usable.
+ * Arguments, checks and errors as grouped_gemm_mxfp8. Never use it for results.
+ */
+mxmoe_status grouped_gemm_mxfp8_debug_timeout(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B,
+                                              const int32_t* seg_off_dev, int32_t E, int64_t N, int64_t K,
+                                              void* C_dev, int32_t c_dtype, int64_t ldc, void* stream);
+
+/*
  * grouped_gemm_mxfp8_wgrad -- weight-gradient form, contracting over each expert's
  * (ragged) rows: C[e] = dequant(At)[:, seg_e] . dequant(Bt)[:, seg_e]^T, fp32, [E, N, K2].
  * An expert with no rows gets zeros.
@@ -338,6 +352,8 @@ mxmoe_status mxmoe_weights_view(void* wq_dev, int32_t E, int32_t H, int32_t F, i
 #define MXMOE_SAVED_GU 9           /* bf16 [cap, 2F] (gate | up); 0 bytes with MXMOE_RECIPE_RECOMPUTE_GU */
 #define MXMOE_SAVED_X_ROW 10       /* e4m3 [cap, H], only with MXMOE_RECIPE_RECOMPUTE_GU (else 0 bytes) */
 #define MXMOE_SAVED_X_ROW_SF 11    /* e8m0, MMA layout, likewise */
+#define MXMOE_SAVED_AMAX 12        /* float [2]: largest |x|, and the Z amax the forward encoded Z with;
+                                      only with MXMOE_RECIPE_FP8_TENSOR (else 0 bytes) */
 size_t grouped_mlp_saved_size(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F);
 int64_t grouped_mlp_saved_offset(int32_t field, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F);
 
@@ -395,11 +411,16 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
  *   MXMOE_RECIPE_SCALE_CEIL     every quantiser of the call (x, Z; dY, dGU) uses
  *                               MXMOE_SCALE_RULE_CEIL; quantise the weights with
  *                               mxmoe_weights_quantize_ex(..., MXMOE_SCALE_RULE_CEIL, ...).
+ *   MXMOE_RECIPE_FP8_TENSOR     per-tensor FP8 in place of MXFP8 (see grouped_mlp_fp8_fwd);
+ *                               it combines with no other bit, is run only through
+ *                               grouped_mlp_fp8_fwd / _bwd (the _ex calls refuse it) and is
+ *                               passed to the _ex size queries for that layer's sizes.
  * A recipe with any other bit set returns MXMOE_ERR_INVALID_ARG (sizes: 0 / -1).
  */
 #define MXMOE_RECIPE_GRAD_E5M2 1
 #define MXMOE_RECIPE_RECOMPUTE_GU 2
 #define MXMOE_RECIPE_SCALE_CEIL 4
+#define MXMOE_RECIPE_FP8_TENSOR 8
 size_t grouped_mlp_saved_size_ex(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F, int32_t recipe);
 int64_t grouped_mlp_saved_offset_ex(int32_t field, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
                                     int32_t recipe);
@@ -412,6 +433,49 @@ mxmoe_status grouped_mlp_bwd_ex(const void* dy_dev, const void* saved_dev, size_
                                 size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
                                 int32_t recipe, void* dx_dev, float* dW1_dev, float* dW2_dev, float* dprobs_dev,
                                 void* ws_dev, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ per-tensor FP8 grouped MLP */
+
+/*
+ * The same layer with per-tensor FP8 in place of MXFP8 -- the pages name "FP8" beside
+ * "MXFP8" ("MoE-Training für biologische Grundmodelle optimieren", precision passage) and
+ * fix nothing else; the rule below is this library's reading.
+ * Every operand is OCP E4M3 under one fp32 multiplier per tensor, m = 448 / amax rounded
+ * to nearest (1 when amax == 0; the largest finite fp32 if the quotient overflows); an
+ * element's code is E4M3(fp32(v * m)) (nearest, ties to even, saturating), its value
+ * code / m. The tensors: x and dY (all tokens), W1[e] and W2[e] (one multiplier per
+ * expert), Z and dGU (all routed rows). x, dY and the weights use their own amax (current
+ * scaling: an extra read pass each). Z and dGU are produced tile by tile inside the fused
+ * GEMM epilogues, so their multipliers come from an amax known before the call (delayed
+ * scaling): the caller-owned device array amax_state_dev, fp32 [4], 16-byte aligned:
+ *   [0] Z amax the forward encodes Z with (read);  [1] largest |Z| of this forward (written);
+ *   [2] dGU amax the backward encodes dGU with (read); [3] largest |dGU| of this backward
+ *   (written).
+ * Values beyond the given amax saturate to +-448. A training loop copies [1] -> [0] and
+ * [3] -> [2] between steps (the first step needs a starting value, e.g. from a forward /
+ * backward run for that purpose). The operands' MXFP8 scale bytes are all 127 (2^0), so
+ * the grouped GEMMs run the same block-scaled tensor-core instruction; each GEMM output is
+ * scaled by 1 / (m_a * m_b) in its epilogue.
+ *
+ * mxmoe_weights_quantize_fp8: the per-expert amax of W1 and W2 (kept in the weights
+ *   buffer) and the four copies of mxmoe_weights_quantize, per-tensor encoded. Same
+ *   arguments, buffer size and limits as mxmoe_weights_quantize.
+ * grouped_mlp_fp8_fwd / grouped_mlp_fp8_bwd: the steps, arguments, limits and outputs of
+ *   grouped_mlp_fwd / _bwd, with weights from mxmoe_weights_quantize_fp8, saved-buffer and
+ *   workspace sizes from the _ex queries with MXMOE_RECIPE_FP8_TENSOR, and amax_state_dev as
+ *   above (null or misaligned: MXMOE_ERR_INVALID_ARG). The backward takes the saved buffer
+ *   of a per-tensor forward.
+ */
+mxmoe_status mxmoe_weights_quantize_fp8(const void* W1_dev, const void* W2_dev, int32_t E, int32_t H, int32_t F,
+                                        void* wq_dev, size_t wq_bytes, void* stream);
+mxmoe_status grouped_mlp_fp8_fwd(const void* x_dev, const int32_t* topk_idx_dev, const float* probs_dev,
+                                 const void* wq_dev, size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H,
+                                 int32_t F, float* amax_state_dev, void* y_dev, void* saved_dev, size_t saved_bytes,
+                                 void* ws_dev, size_t ws_bytes, void* stream);
+mxmoe_status grouped_mlp_fp8_bwd(const void* dy_dev, const void* saved_dev, size_t saved_bytes, const void* wq_dev,
+                                 size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
+                                 float* amax_state_dev, void* dx_dev, float* dW1_dev, float* dW2_dev,
+                                 float* dprobs_dev, void* ws_dev, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------ bf16 grouped MLP */
 

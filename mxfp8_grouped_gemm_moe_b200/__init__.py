@@ -26,12 +26,12 @@ STATUS_NAMES = {
 DTYPE_BF16, DTYPE_F32 = 0, 1
 SCALE_PLAIN, SCALE_MMA = 0, 1
 FMT_E4M3, FMT_E5M2 = 0, 1
-RECIPE_GRAD_E5M2, RECIPE_RECOMPUTE_GU, RECIPE_SCALE_CEIL = 1, 2, 4
+RECIPE_GRAD_E5M2, RECIPE_RECOMPUTE_GU, RECIPE_SCALE_CEIL, RECIPE_FP8_TENSOR = 1, 2, 4, 8
 SCALE_RULE_OCP, SCALE_RULE_CEIL = 0, 1
 _RULE = {"ocp": SCALE_RULE_OCP, "ceil": SCALE_RULE_CEIL}
 _FMT = {"e4m3": FMT_E4M3, "e5m2": FMT_E5M2}
 SAVED_FIELDS = ["m_splits", "seg_off", "row_of_slot", "token_of_row", "prob_of_row",
-                "x_colT", "x_colT_sf", "z_colT", "z_colT_sf", "gu", "x_row", "x_row_sf"]
+                "x_colT", "x_colT_sf", "z_colT", "z_colT_sf", "gu", "x_row", "x_row_sf", "amax"]
 
 
 class MxmoeError(RuntimeError):
@@ -70,6 +70,7 @@ _SIGNATURES = {
     "mxfp8_quantize": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _I64, _PMX, _PMX, _P]),
     "mxfp8_quantize_ex": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _I64, _PMX, _PMX, _I32, _P]),
     "grouped_gemm_mxfp8": (_I32, [_PMX, _PMX, _P, _I32, _I64, _I64, _P, _I32, _I64, _P]),
+    "grouped_gemm_mxfp8_debug_timeout": (_I32, [_PMX, _PMX, _P, _I32, _I64, _I64, _P, _I32, _I64, _P]),
     "grouped_gemm_mxfp8_wgrad": (_I32, [_PMX, _PMX, _P, _I32, _P, _P]),
     "mxmoe_weights_size": (_SZ, [_I32, _I32, _I32]),
     "mxmoe_weights_quantize": (_I32, [_P, _P, _I32, _I32, _I32, _P, _SZ, _P]),
@@ -84,6 +85,10 @@ _SIGNATURES = {
     "grouped_mlp_saved_offset_ex": (_I64, [_I32, _I32, _I32, _I32, _I32, _I32, _I32]),
     "grouped_mlp_workspace_size_ex": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32]),
     "grouped_mlp_fwd_ex": (_I32, [_P, _P, _P, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P, _SZ, _P, _SZ, _P]),
+    "mxmoe_weights_quantize_fp8": (_I32, [_P, _P, _I32, _I32, _I32, _P, _SZ, _P]),
+    "grouped_mlp_fp8_fwd": (_I32, [_P, _P, _P, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _SZ, _P, _SZ, _P]),
+    "grouped_mlp_fp8_bwd": (_I32, [_P, _P, _SZ, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ,
+                                   _P]),
     "grouped_mlp_bwd_ex": (_I32, [_P, _P, _SZ, _P, _SZ, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ,
                                   _P]),
     "mxmoe_weights_bf16_size": (_SZ, [_I32, _I32, _I32]),
@@ -281,6 +286,17 @@ def grouped_gemm_mxfp8(A: MXFP8, B: MXFP8, seg_off, E, N, out_dtype=torch.bfloat
     return C
 
 
+def grouped_gemm_mxfp8_debug_timeout(A: MXFP8, B: MXFP8, seg_off, E, N, out):
+    """Test hook of the device-timeout path: grouped_gemm_mxfp8 with the first CTA pair's
+    accumulator-ready signal withheld. The kernel ends after about a second with the device
+    status set to MXMOE_ERR_DEVICE_TIMEOUT and `out` only partly written."""
+    dt = DTYPE_BF16 if out.dtype == torch.bfloat16 else DTYPE_F32
+    st = load().grouped_gemm_mxfp8_debug_timeout(ctypes.byref(A.as_struct()), ctypes.byref(B.as_struct()),
+                                                 _ptr(seg_off), E, N, A.cols, _ptr(out), dt, out.stride(0), _stream())
+    _check("grouped_gemm_mxfp8_debug_timeout", st)
+    return out
+
+
 def grouped_gemm_mxfp8_wgrad(At: MXFP8, Bt: MXFP8, seg_off, E, out=None):
     C = out if out is not None else torch.empty((E, At.rows, Bt.rows), dtype=torch.float32, device=At.data.device)
     st = load().grouped_gemm_mxfp8_wgrad(ctypes.byref(At.as_struct()), ctypes.byref(Bt.as_struct()), _ptr(seg_off),
@@ -325,6 +341,43 @@ def mxmoe_weights_quantize(W1, W2, out=None, scale_rule=SCALE_RULE_OCP):
     return wq
 
 
+def mxmoe_weights_quantize_fp8(W1, W2, out=None):
+    """Per-tensor FP8 weights buffer: per-expert amax of W1 / W2 and the four E4M3 copies
+    (scale bytes 127)."""
+    lib = load()
+    E, F2, H = W1.shape
+    F = F2 // 2
+    wq = out if out is not None else torch.empty(lib.mxmoe_weights_size(E, H, F), dtype=torch.uint8,
+                                                 device=W1.device)
+    _check("mxmoe_weights_quantize_fp8",
+           lib.mxmoe_weights_quantize_fp8(_ptr(W1), _ptr(W2), E, H, F, _ptr(wq), wq.numel(), _stream()))
+    return wq
+
+
+def grouped_mlp_fp8_fwd(x, topk_idx, probs, wq, E, F, amax_state, saved, ws, y=None):
+    T, H = x.shape
+    k = topk_idx.shape[1]
+    y = y if y is not None else torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    st = load().grouped_mlp_fp8_fwd(_ptr(x), _ptr(topk_idx), _ptr(probs), _ptr(wq), wq.numel(), T, k, E, H, F,
+                                    _ptr(amax_state), _ptr(y), _ptr(saved), saved.numel(), _ptr(ws), ws.numel(),
+                                    _stream())
+    _check("grouped_mlp_fp8_fwd", st)
+    return y
+
+
+def grouped_mlp_fp8_bwd(dy, saved, wq, T, k, E, H, F, amax_state, ws, dx=None, dW1=None, dW2=None, dprobs=None):
+    dev = dy.device
+    dx = dx if dx is not None else torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    dW1 = dW1 if dW1 is not None else torch.empty((E, 2 * F, H), dtype=torch.float32, device=dev)
+    dW2 = dW2 if dW2 is not None else torch.empty((E, H, F), dtype=torch.float32, device=dev)
+    dprobs = dprobs if dprobs is not None else torch.empty((T, k), dtype=torch.float32, device=dev)
+    st = load().grouped_mlp_fp8_bwd(_ptr(dy), _ptr(saved), saved.numel(), _ptr(wq), wq.numel(), T, k, E, H, F,
+                                    _ptr(amax_state), _ptr(dx), _ptr(dW1), _ptr(dW2), _ptr(dprobs), _ptr(ws),
+                                    ws.numel(), _stream())
+    _check("grouped_mlp_fp8_bwd", st)
+    return dx, dW1, dW2, dprobs
+
+
 def mxmoe_weights_view(wq, E, H, F, which):
     """MXFP8 view (0 W1 row, 1 W1 colT, 2 W2 row, 3 W2 colT) into a weights buffer."""
     m = _MX()
@@ -339,7 +392,10 @@ class GroupedMLP:
     """Buffers for one layer shape; forward/backward call the fused C entry points.
 
     precision "mxfp8" (default) runs the MXFP8 layer (grouped_mlp_fwd / _bwd); "bf16" runs
-    the same steps on bf16 operands (grouped_mlp_bf16_fwd / _bwd). For the MXFP8 layer,
+    the same steps on bf16 operands (grouped_mlp_bf16_fwd / _bwd); "fp8" runs per-tensor FP8
+    (grouped_mlp_fp8_fwd / _bwd) with its delayed-scaling state in ``amax_state`` (fp32 [4]
+    on the device: Z amax in / out, dGU amax in / out; ``roll_amax`` starts the next step
+    with this step's values, ``set_amax`` sets the values to encode with). For the MXFP8 layer,
     grad_format "e4m3" (default) or "e5m2" picks the element format of the gradients (dY,
     dGU), recompute_gu=True saves the rowwise MXFP8 input instead of the bf16 gate/up
     pre-activations and recomputes those in the backward, and scale_rule "ocp" (default) or
@@ -348,7 +404,7 @@ class GroupedMLP:
 
     def __init__(self, T, k, E, H, F, device="cuda", precision="mxfp8", grad_format="e4m3", recompute_gu=False,
                  scale_rule="ocp"):
-        if precision not in ("mxfp8", "bf16"):
+        if precision not in ("mxfp8", "bf16", "fp8"):
             raise ValueError(f"unknown precision {precision!r}")
         if grad_format not in _FMT:
             raise ValueError(f"unknown grad_format {grad_format!r}")
@@ -358,8 +414,11 @@ class GroupedMLP:
         self.recipe = ((RECIPE_GRAD_E5M2 if grad_format == "e5m2" else 0) |
                        (RECIPE_RECOMPUTE_GU if recompute_gu else 0) |
                        (RECIPE_SCALE_CEIL if scale_rule == "ceil" else 0))
-        if precision == "bf16" and self.recipe:
+        if precision != "mxfp8" and self.recipe:
             raise ValueError("grad_format / recompute_gu / scale_rule apply to the MXFP8 layer")
+        if precision == "fp8":
+            self.recipe = RECIPE_FP8_TENSOR
+            self.amax_state = torch.zeros(4, dtype=torch.float32, device=device)
         lib = load()
         self.T, self.k, self.E, self.H, self.F = T, k, E, H, F
         self.precision = precision
@@ -382,11 +441,26 @@ class GroupedMLP:
         """Prepares the weights buffer: MXFP8 copies, or bf16 row / transposed copies."""
         if self.precision == "bf16":
             return mxmoe_weights_bf16_prepare(W1, W2, out=self.wq)
+        if self.precision == "fp8":
+            return mxmoe_weights_quantize_fp8(W1, W2, out=self.wq)
         return mxmoe_weights_quantize(W1, W2, out=self.wq, scale_rule=self.scale_rule)
+
+    def set_amax(self, z_amax, dgu_amax):
+        """Per-tensor FP8: the Z and dGU amax the next forward / backward encode with."""
+        self.amax_state[0] = float(z_amax)
+        self.amax_state[2] = float(dgu_amax)
+
+    def roll_amax(self):
+        """Per-tensor FP8 delayed scaling: the next step encodes Z and dGU with this step's
+        largest magnitudes (device copies, no synchronisation)."""
+        self.amax_state[0:4:2].copy_(self.amax_state[1:4:2])
 
     def forward(self, x, topk_idx, probs, y=None):
         if self.precision == "bf16":
             return grouped_mlp_bf16_fwd(x, topk_idx, probs, self.wq, self.E, self.F, self.saved, self.ws, y)
+        if self.precision == "fp8":
+            return grouped_mlp_fp8_fwd(x, topk_idx, probs, self.wq, self.E, self.F, self.amax_state, self.saved,
+                                       self.ws, y)
         return grouped_mlp_fwd(x, topk_idx, probs, self.wq, self.E, self.F, self.saved, self.ws, y,
                                recipe=self.recipe)
 
@@ -394,13 +468,16 @@ class GroupedMLP:
         if self.precision == "bf16":
             return grouped_mlp_bf16_bwd(dy, self.saved, self.wq, self.T, self.k, self.E, self.H, self.F, self.ws,
                                         dx, dW1, dW2, dprobs)
+        if self.precision == "fp8":
+            return grouped_mlp_fp8_bwd(dy, self.saved, self.wq, self.T, self.k, self.E, self.H, self.F,
+                                       self.amax_state, self.ws, dx, dW1, dW2, dprobs)
         return grouped_mlp_bwd(dy, self.saved, self.wq, self.T, self.k, self.E, self.H, self.F, self.ws, dx, dW1,
                                dW2, dprobs, recipe=self.recipe)
 
     def saved_field(self, name, dtype=torch.uint8, count=None):
         """View of a named field of the saved buffer of the MXFP8 layer (inspection / tests)."""
-        if self.precision != "mxfp8":
-            raise ValueError("saved_field describes the MXFP8 layer's saved buffer")
+        if self.precision == "bf16":
+            raise ValueError("saved_field describes the MXFP8 / FP8 layers' saved buffer")
         lib = load()
         f = SAVED_FIELDS.index(name)
         off = lib.grouped_mlp_saved_offset_ex(f, self.T, self.k, self.E, self.H, self.F, self.recipe)

@@ -41,7 +41,7 @@ bool valid_mlp_shape(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F) {
 
 // ---------------------------------------------------------------- layouts
 struct WeightsLayout {
-  size_t d[4], s[4], total;
+  size_t d[4], s[4], amax, total;  // amax: per-tensor FP8 weights' largest magnitudes, W1 [E] then W2 [E]
   int64_t rows[4], cols[4];
 };
 WeightsLayout weights_layout(int64_t E, int64_t H, int64_t F) {
@@ -55,20 +55,23 @@ WeightsLayout weights_layout(int64_t E, int64_t H, int64_t F) {
     L.d[i] = cv.take((size_t)(r[i] * c[i]));
     L.s[i] = cv.take((size_t)(r[i] * c[i] / 32));
   }
+  L.amax = cv.take((size_t)(2 * E * 4));
   L.total = cv.off;
   return L;
 }
 
 bool valid_recipe(int32_t recipe) {
+  if (recipe == MXMOE_RECIPE_FP8_TENSOR) return true;  // per-tensor FP8 combines with no other bit
   return (recipe & ~(MXMOE_RECIPE_GRAD_E5M2 | MXMOE_RECIPE_RECOMPUTE_GU | MXMOE_RECIPE_SCALE_CEIL)) == 0;
 }
+bool fp8_tensor(int32_t recipe) { return recipe == MXMOE_RECIPE_FP8_TENSOR; }
 int32_t recipe_scale_rule(int32_t recipe) {
   return (recipe & MXMOE_RECIPE_SCALE_CEIL) ? MXMOE_SCALE_RULE_CEIL : MXMOE_SCALE_RULE_OCP;
 }
 bool recomputes_gu(int32_t recipe) { return (recipe & MXMOE_RECIPE_RECOMPUTE_GU) != 0; }
 
 struct SavedLayout {
-  size_t off[12];
+  size_t off[13];
   size_t total;
 };
 // With MXMOE_RECIPE_RECOMPUTE_GU the gate/up pre-activations are not saved (zero bytes)
@@ -90,6 +93,7 @@ SavedLayout saved_layout(int64_t T, int64_t k, int64_t E, int64_t H, int64_t F, 
   L.off[MXMOE_SAVED_GU] = cv.take(rc ? 0 : cap * 2 * F * 2);
   L.off[MXMOE_SAVED_X_ROW] = cv.take(rc ? cap * H : 0);
   L.off[MXMOE_SAVED_X_ROW_SF] = cv.take(rc ? cap * H / 32 : 0);
+  L.off[MXMOE_SAVED_AMAX] = cv.take(fp8_tensor(recipe) ? 2 * 4 : 0);  // largest |x|, Z's amax in use
   L.total = cv.off;
   return L;
 }
@@ -113,7 +117,7 @@ FwdWs fwd_ws(int64_t T, int64_t k, int64_t E, int64_t H, int64_t F) {
 
 struct BwdWs {
   size_t dy_row, dy_row_sf, dy_colT, dy_colT_sf, dgu_row, dgu_row_sf, dgu_colT, dgu_colT_sf, dprob_part, dx_perm, gu,
-      total;
+      amax, total;
 };
 BwdWs bwd_ws(int64_t T, int64_t k, int64_t E, int64_t H, int64_t F, int32_t recipe = 0) {
   const int64_t cap = rows_cap(T, k, E);
@@ -130,6 +134,7 @@ BwdWs bwd_ws(int64_t T, int64_t k, int64_t E, int64_t H, int64_t F, int32_t reci
   w.dprob_part = cv.take(cap * (F / 128) * 4);
   w.dx_perm = cv.take(cap * H * 2);
   w.gu = cv.take(recomputes_gu(recipe) ? cap * 2 * F * 2 : 0);  // recomputed G / U (bf16)
+  w.amax = cv.take(fp8_tensor(recipe) ? 2 * 4 : 0);               // largest |dY|, dGU's amax in use
   w.total = cv.off;
   return w;
 }
@@ -296,7 +301,8 @@ mxmoe_status moe_unpermute(const void* y_perm_dev, const int32_t* row_of_slot_de
 static mxmoe_status quantize_impl(const void* src_dev, int32_t src_dtype, int64_t batch, int64_t rows, int64_t cols,
                                   const int32_t* row_gather_dev, const int32_t* nrows_dev, int64_t out_rows,
                                   const mxmoe_mxfp8* out_row, const mxmoe_mxfp8* out_colT, int64_t row_ilv,
-                                  int32_t scale_rule, void* stream) {
+                                  int32_t scale_rule, void* stream, const float* tensor_amax = nullptr,
+                                  int32_t tensor_per_batch = 0) {
   if (src_dtype != MXMOE_DTYPE_BF16 && src_dtype != MXMOE_DTYPE_F32) return MXMOE_ERR_INVALID_ARG;
   if (scale_rule != MXMOE_SCALE_RULE_OCP && scale_rule != MXMOE_SCALE_RULE_CEIL) return MXMOE_ERR_INVALID_ARG;
   if (!src_dev || !aligned16(src_dev) || (!out_row && !out_colT)) return MXMOE_ERR_INVALID_ARG;
@@ -336,6 +342,9 @@ static mxmoe_status quantize_impl(const void* src_dev, int32_t src_dtype, int64_
   a.col_sf = out_colT ? out_colT->scale : nullptr;
   a.col_layout = out_colT ? out_colT->scale_layout : 0;
   a.row_ilv = row_ilv;
+  a.tensor_amax = tensor_amax;
+  a.tensor_per_batch = tensor_per_batch;
+  if (tensor_amax && a.fmt != MXMOE_FMT_E4M3) return MXMOE_ERR_INVALID_ARG;
   StageScope sc(MXMOE_STAGE_QUANT, S(stream));
   return cuda_status(launch_quantize(a, S(stream)));
 }
@@ -355,9 +364,10 @@ mxmoe_status mxfp8_quantize_ex(const void* src_dev, int32_t src_dtype, int64_t b
                        scale_rule, stream);
 }
 
-mxmoe_status grouped_gemm_mxfp8(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, const int32_t* seg_off_dev,
-                                int32_t E, int64_t N, int64_t K, void* C_dev, int32_t c_dtype, int64_t ldc,
-                                void* stream) {
+static mxmoe_status grouped_gemm_impl(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, const int32_t* seg_off_dev,
+                                      int32_t E, int64_t N, int64_t K, void* C_dev, int32_t c_dtype, int64_t ldc,
+                                      int32_t debug_drop_commit, void* stream, const float* a_amax = nullptr,
+                                      const float* b_amax = nullptr) {
   if (!A || !B || !seg_off_dev || !C_dev || !aligned16(C_dev)) return MXMOE_ERR_INVALID_ARG;
   if (c_dtype != MXMOE_DTYPE_BF16 && c_dtype != MXMOE_DTYPE_F32) return MXMOE_ERR_INVALID_ARG;
   if (!mma_ready(A) || !mma_ready(B)) return MXMOE_ERR_INVALID_ARG;
@@ -371,12 +381,36 @@ mxmoe_status grouped_gemm_mxfp8(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, cons
   g.c = C_dev;
   g.c_dtype = c_dtype;
   g.ldc = ldc;
+  g.debug_drop_commit = debug_drop_commit;
+  g.a_amax = a_amax;  // per-tensor FP8 operands (b: one value per expert)
+  g.b_amax = b_amax;
+  g.b_amax_per_expert = 1;
   StageScope sc(MXMOE_STAGE_GEMM, S(stream));
   return cuda_status(launch_gemm(g, S(stream)));
 }
 
+mxmoe_status grouped_gemm_mxfp8(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, const int32_t* seg_off_dev,
+                                int32_t E, int64_t N, int64_t K, void* C_dev, int32_t c_dtype, int64_t ldc,
+                                void* stream) {
+  return grouped_gemm_impl(A, B, seg_off_dev, E, N, K, C_dev, c_dtype, ldc, 0, stream);
+}
+
+mxmoe_status grouped_gemm_mxfp8_debug_timeout(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B,
+                                              const int32_t* seg_off_dev, int32_t E, int64_t N, int64_t K,
+                                              void* C_dev, int32_t c_dtype, int64_t ldc, void* stream) {
+  return grouped_gemm_impl(A, B, seg_off_dev, E, N, K, C_dev, c_dtype, ldc, 1, stream);
+}
+
+static mxmoe_status grouped_wgrad_impl(const mxmoe_mxfp8* At, const mxmoe_mxfp8* Bt, const int32_t* seg_off_dev,
+                                       int32_t E, float* C_dev, void* stream, const float* a_amax,
+                                       const float* b_amax);
 mxmoe_status grouped_gemm_mxfp8_wgrad(const mxmoe_mxfp8* At, const mxmoe_mxfp8* Bt, const int32_t* seg_off_dev,
                                       int32_t E, float* C_dev, void* stream) {
+  return grouped_wgrad_impl(At, Bt, seg_off_dev, E, C_dev, stream, nullptr, nullptr);
+}
+static mxmoe_status grouped_wgrad_impl(const mxmoe_mxfp8* At, const mxmoe_mxfp8* Bt, const int32_t* seg_off_dev,
+                                       int32_t E, float* C_dev, void* stream, const float* a_amax,
+                                       const float* b_amax) {
   if (!At || !Bt || !seg_off_dev || !C_dev || !aligned16(C_dev)) return MXMOE_ERR_INVALID_ARG;
   if (!mma_ready(At) || !mma_ready(Bt)) return MXMOE_ERR_INVALID_ARG;
   if (E < 1 || E > 256 || At->cols != Bt->cols || At->rows <= 0 || At->rows % 256 != 0 || Bt->rows % 256 != 0 ||
@@ -388,6 +422,8 @@ mxmoe_status grouped_gemm_mxfp8_wgrad(const mxmoe_mxfp8* At, const mxmoe_mxfp8* 
   g.c = C_dev;
   g.c_dtype = MXMOE_DTYPE_F32;
   g.ldc = Bt->rows;
+  g.a_amax = a_amax;  // per-tensor FP8 operands (one value each)
+  g.b_amax = b_amax;
   StageScope sc(MXMOE_STAGE_WGRAD, S(stream));
   return cuda_status(launch_gemm(g, S(stream)));
 }
@@ -488,6 +524,34 @@ mxmoe_status mxmoe_weights_quantize_ex(const void* W1_dev, const void* W2_dev, i
   return mxfp8_quantize_ex(W2_dev, MXMOE_DTYPE_BF16, E, H, F, nullptr, nullptr, H, &w2r, &w2c, scale_rule, stream);
 }
 
+mxmoe_status mxmoe_weights_quantize_fp8(const void* W1_dev, const void* W2_dev, int32_t E, int32_t H, int32_t F,
+                                        void* wq_dev, size_t wq_bytes, void* stream) {
+  if (E < 1 || E > 256 || H <= 0 || F <= 0 || H % 256 != 0 || F % 256 != 0) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if (!W1_dev || !W2_dev || !wq_dev || !aligned16(W1_dev) || !aligned16(W2_dev) || !aligned16(wq_dev))
+    return MXMOE_ERR_INVALID_ARG;
+  const WeightsLayout L = weights_layout(E, H, F);
+  if (wq_bytes < L.total) return MXMOE_ERR_WORKSPACE_TOO_SMALL;
+  uint8_t* b = reinterpret_cast<uint8_t*>(wq_dev);
+  mxmoe_mxfp8 w1r = mk(b, L.d[0], L.s[0], L.rows[0], L.cols[0]);
+  mxmoe_mxfp8 w1c = mk(b, L.d[1], L.s[1], L.rows[1], L.cols[1]);
+  mxmoe_mxfp8 w2r = mk(b, L.d[2], L.s[2], L.rows[2], L.cols[2]);
+  mxmoe_mxfp8 w2c = mk(b, L.d[3], L.s[3], L.rows[3], L.cols[3]);
+  float* am = reinterpret_cast<float*>(b + L.amax);  // W1[e] then W2[e]
+  cudaStream_t st = S(stream);
+  mxmoe_status s;
+  {
+    StageScope sc(MXMOE_STAGE_QUANT_W1, st);
+    if (launch_amax_bf16(W1_dev, 2 * (int64_t)F * H, E, am, st) != cudaSuccess) return MXMOE_ERR_CUDA;
+    s = quantize_impl(W1_dev, MXMOE_DTYPE_BF16, E, 2 * (int64_t)F, H, nullptr, nullptr, 2 * (int64_t)F, &w1r, &w1c,
+                      F, MXMOE_SCALE_RULE_OCP, stream, am, 1);
+  }
+  if (s != MXMOE_OK) return s;
+  StageScope sc(MXMOE_STAGE_QUANT_W2, st);
+  if (launch_amax_bf16(W2_dev, (int64_t)H * F, E, am + E, st) != cudaSuccess) return MXMOE_ERR_CUDA;
+  return quantize_impl(W2_dev, MXMOE_DTYPE_BF16, E, H, F, nullptr, nullptr, H, &w2r, &w2c, 0, MXMOE_SCALE_RULE_OCP,
+                       stream, am + E, 1);
+}
+
 size_t grouped_mlp_saved_size(int32_t T, int32_t k, int32_t E, int32_t H, int32_t F) {
   return grouped_mlp_saved_size_ex(T, k, E, H, F, 0);
 }
@@ -501,7 +565,7 @@ int64_t grouped_mlp_saved_offset(int32_t field, int32_t T, int32_t k, int32_t E,
 }
 int64_t grouped_mlp_saved_offset_ex(int32_t field, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
                                     int32_t recipe) {
-  if (field < 0 || field > 11 || !valid_recipe(recipe)) return -1;
+  if (field < 0 || field > 12 || !valid_recipe(recipe)) return -1;
   return (int64_t)saved_layout(T, k, E, H, F, recipe).off[field];
 }
 
@@ -521,10 +585,33 @@ mxmoe_status grouped_mlp_fwd(const void* x_dev, const int32_t* topk_idx_dev, con
                             saved_bytes, ws_dev, ws_bytes, stream);
 }
 
+static mxmoe_status fwd_impl(const void* x_dev, const int32_t* topk_idx_dev, const float* probs_dev,
+                             const void* wq_dev, size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H,
+                             int32_t F, int32_t recipe, float* amax_state, void* y_dev, void* saved_dev,
+                             size_t saved_bytes, void* ws_dev, size_t ws_bytes, void* stream);
+
 mxmoe_status grouped_mlp_fwd_ex(const void* x_dev, const int32_t* topk_idx_dev, const float* probs_dev,
                                 const void* wq_dev, size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H,
                                 int32_t F, int32_t recipe, void* y_dev, void* saved_dev, size_t saved_bytes,
                                 void* ws_dev, size_t ws_bytes, void* stream) {
+  if (fp8_tensor(recipe)) return MXMOE_ERR_INVALID_ARG;  // per-tensor FP8: grouped_mlp_fp8_fwd
+  return fwd_impl(x_dev, topk_idx_dev, probs_dev, wq_dev, wq_bytes, T, k, E, H, F, recipe, nullptr, y_dev, saved_dev,
+                  saved_bytes, ws_dev, ws_bytes, stream);
+}
+
+mxmoe_status grouped_mlp_fp8_fwd(const void* x_dev, const int32_t* topk_idx_dev, const float* probs_dev,
+                                 const void* wq_dev, size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H,
+                                 int32_t F, float* amax_state_dev, void* y_dev, void* saved_dev, size_t saved_bytes,
+                                 void* ws_dev, size_t ws_bytes, void* stream) {
+  if (!amax_state_dev || !aligned16(amax_state_dev)) return MXMOE_ERR_INVALID_ARG;
+  return fwd_impl(x_dev, topk_idx_dev, probs_dev, wq_dev, wq_bytes, T, k, E, H, F, MXMOE_RECIPE_FP8_TENSOR,
+                  amax_state_dev, y_dev, saved_dev, saved_bytes, ws_dev, ws_bytes, stream);
+}
+
+static mxmoe_status fwd_impl(const void* x_dev, const int32_t* topk_idx_dev, const float* probs_dev,
+                             const void* wq_dev, size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H,
+                             int32_t F, int32_t recipe, float* amax_state, void* y_dev, void* saved_dev,
+                             size_t saved_bytes, void* ws_dev, size_t ws_bytes, void* stream) {
   if (!valid_recipe(recipe)) return MXMOE_ERR_INVALID_ARG;
   if (!valid_mlp_shape(T, k, E, H, F)) return MXMOE_ERR_UNSUPPORTED_SHAPE;
   if (!wq_dev || !saved_dev || !ws_dev || !aligned16(wq_dev) || !aligned16(saved_dev) || !aligned16(ws_dev))
@@ -556,6 +643,16 @@ mxmoe_status grouped_mlp_fwd_ex(const void* x_dev, const int32_t* topk_idx_dev, 
     e = launch_route(topk_idx_dev, probs_dev, T, k, E, m_splits, seg_off, ros, tor, por, ws + W.route, st);
   }
   if (e != cudaSuccess) return MXMOE_ERR_CUDA;
+  // per-tensor FP8: largest |x| and the Z amax this forward encodes with (both kept in the
+  // saved buffer for the backward); this step's largest |Z| is recorded into amax_state[1]
+  const bool pt = fp8_tensor(recipe);
+  float* x_amax = pt ? reinterpret_cast<float*>(sv + SL.off[MXMOE_SAVED_AMAX]) : nullptr;
+  float* z_used = pt ? x_amax + 1 : nullptr;
+  const float* w1_amax = pt ? reinterpret_cast<const float*>(wq + WL.amax) : nullptr;
+  const float* w2_amax = pt ? w1_amax + E : nullptr;
+  if (pt && (cudaMemcpyAsync(z_used, amax_state, 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+             cudaMemsetAsync(amax_state + 1, 0, 4, st) != cudaSuccess))
+    return MXMOE_ERR_CUDA;
   if (T == 0) return MXMOE_OK;
   // 2. permute + quantise x (rowwise for fc1 -- saved when the backward recomputes G / U --
   // and colwise, saved for fc1 wgrad)
@@ -565,8 +662,9 @@ mxmoe_status grouped_mlp_fwd_ex(const void* x_dev, const int32_t* topk_idx_dev, 
   mxmoe_status s;
   {
     StageScope sc(MXMOE_STAGE_QUANT_X, st);
-    s = mxfp8_quantize_ex(x_dev, MXMOE_DTYPE_BF16, 1, T, H, tor, seg_off + E, cap, &x_row, &x_col,
-                          recipe_scale_rule(recipe), stream);
+    if (pt && launch_amax_bf16(x_dev, (int64_t)T * H, 1, x_amax, st) != cudaSuccess) return MXMOE_ERR_CUDA;
+    s = quantize_impl(x_dev, MXMOE_DTYPE_BF16, 1, T, H, tor, seg_off + E, cap, &x_row, &x_col, 0,
+                      recipe_scale_rule(recipe), stream, x_amax, 0);
   }
   if (s != MXMOE_OK) return s;
   // 3. fc1 + SwiGLU x prob -> Z (MXFP8 row + colT), G/U saved unless recomputed
@@ -583,6 +681,11 @@ mxmoe_status grouped_mlp_fwd_ex(const void* x_dev, const int32_t* topk_idx_dev, 
   g.z_colT_sf = sv + SL.off[MXMOE_SAVED_Z_COLT_SF];
   g.scale_rule = recipe_scale_rule(recipe);
   g.gu = rc ? nullptr : reinterpret_cast<uint16_t*>(sv + SL.off[MXMOE_SAVED_GU]);
+  g.a_amax = x_amax;
+  g.b_amax = w1_amax;
+  g.b_amax_per_expert = 1;
+  g.out_amax_in = z_used;
+  g.out_amax_rec = pt ? amax_state + 1 : nullptr;
   {
     StageScope sc(MXMOE_STAGE_FC1_SWIGLU, st);
     e = launch_gemm(g, st);
@@ -593,7 +696,8 @@ mxmoe_status grouped_mlp_fwd_ex(const void* x_dev, const int32_t* topk_idx_dev, 
   mxmoe_mxfp8 w2r = mk(wq, WL.d[2], WL.s[2], WL.rows[2], WL.cols[2]);
   {
     StageScope sc(MXMOE_STAGE_FC2, st);
-    s = grouped_gemm_mxfp8(&z_row, &w2r, seg_off, E, H, F, ws + W.y_perm, MXMOE_DTYPE_BF16, H, stream);
+    s = grouped_gemm_impl(&z_row, &w2r, seg_off, E, H, F, ws + W.y_perm, MXMOE_DTYPE_BF16, H, 0, stream, z_used,
+                          w2_amax);
   }
   if (s != MXMOE_OK) return s;
   // 5. combine
@@ -609,10 +713,33 @@ mxmoe_status grouped_mlp_bwd(const void* dy_dev, const void* saved_dev, size_t s
                             dW2_dev, dprobs_dev, ws_dev, ws_bytes, stream);
 }
 
+static mxmoe_status bwd_impl(const void* dy_dev, const void* saved_dev, size_t saved_bytes, const void* wq_dev,
+                             size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F, int32_t recipe,
+                             float* amax_state, void* dx_dev, float* dW1_dev, float* dW2_dev, float* dprobs_dev,
+                             void* ws_dev, size_t ws_bytes, void* stream);
+
 mxmoe_status grouped_mlp_bwd_ex(const void* dy_dev, const void* saved_dev, size_t saved_bytes, const void* wq_dev,
                                 size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
                                 int32_t recipe, void* dx_dev, float* dW1_dev, float* dW2_dev, float* dprobs_dev,
                                 void* ws_dev, size_t ws_bytes, void* stream) {
+  if (fp8_tensor(recipe)) return MXMOE_ERR_INVALID_ARG;  // per-tensor FP8: grouped_mlp_fp8_bwd
+  return bwd_impl(dy_dev, saved_dev, saved_bytes, wq_dev, wq_bytes, T, k, E, H, F, recipe, nullptr, dx_dev, dW1_dev,
+                  dW2_dev, dprobs_dev, ws_dev, ws_bytes, stream);
+}
+
+mxmoe_status grouped_mlp_fp8_bwd(const void* dy_dev, const void* saved_dev, size_t saved_bytes, const void* wq_dev,
+                                 size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F,
+                                 float* amax_state_dev, void* dx_dev, float* dW1_dev, float* dW2_dev,
+                                 float* dprobs_dev, void* ws_dev, size_t ws_bytes, void* stream) {
+  if (!amax_state_dev || !aligned16(amax_state_dev)) return MXMOE_ERR_INVALID_ARG;
+  return bwd_impl(dy_dev, saved_dev, saved_bytes, wq_dev, wq_bytes, T, k, E, H, F, MXMOE_RECIPE_FP8_TENSOR,
+                  amax_state_dev, dx_dev, dW1_dev, dW2_dev, dprobs_dev, ws_dev, ws_bytes, stream);
+}
+
+static mxmoe_status bwd_impl(const void* dy_dev, const void* saved_dev, size_t saved_bytes, const void* wq_dev,
+                             size_t wq_bytes, int32_t T, int32_t k, int32_t E, int32_t H, int32_t F, int32_t recipe,
+                             float* amax_state, void* dx_dev, float* dW1_dev, float* dW2_dev, float* dprobs_dev,
+                             void* ws_dev, size_t ws_bytes, void* stream) {
   if (!valid_recipe(recipe)) return MXMOE_ERR_INVALID_ARG;
   const int32_t grad_format = (recipe & MXMOE_RECIPE_GRAD_E5M2) ? MXMOE_FMT_E5M2 : MXMOE_FMT_E4M3;
   if (!valid_mlp_shape(T, k, E, H, F)) return MXMOE_ERR_UNSUPPORTED_SHAPE;
@@ -638,14 +765,28 @@ mxmoe_status grouped_mlp_bwd_ex(const void* dy_dev, const void* saved_dev, size_
   const int32_t* tor = reinterpret_cast<const int32_t*>(sv + SL.off[MXMOE_SAVED_TOKEN_OF_ROW]);
   const float* por = reinterpret_cast<const float*>(sv + SL.off[MXMOE_SAVED_PROB_OF_ROW]);
 
+  // per-tensor FP8: the forward's largest |x| and Z amax (saved), largest |dY| and the dGU
+  // amax this backward encodes with (workspace); this step's largest |dGU| is recorded into
+  // amax_state[3]
+  const bool pt = fp8_tensor(recipe);
+  const float* x_amax = pt ? reinterpret_cast<const float*>(sv + SL.off[MXMOE_SAVED_AMAX]) : nullptr;
+  const float* z_used = pt ? x_amax + 1 : nullptr;
+  float* dy_amax = pt ? reinterpret_cast<float*>(ws + W.amax) : nullptr;
+  float* dgu_used = pt ? dy_amax + 1 : nullptr;
+  const float* w1_amax = pt ? reinterpret_cast<const float*>(wq + WL.amax) : nullptr;
+  const float* w2_amax = pt ? w1_amax + E : nullptr;
+  if (pt && (cudaMemcpyAsync(dgu_used, amax_state + 2, 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+             cudaMemsetAsync(amax_state + 3, 0, 4, st) != cudaSuccess))
+    return MXMOE_ERR_CUDA;
   // 1. permute + quantise dy: rowwise (fc2 dgrad) and colwise (fc2 wgrad)
   mxmoe_mxfp8 dy_row = mk(ws, W.dy_row, W.dy_row_sf, cap, H, grad_format);
   mxmoe_mxfp8 dy_col = mk(ws, W.dy_colT, W.dy_colT_sf, H, cap, grad_format);
   mxmoe_status s;
   if (T > 0) {
     StageScope sc(MXMOE_STAGE_QUANT_DY, st);
-    s = mxfp8_quantize_ex(dy_dev, MXMOE_DTYPE_BF16, 1, T, H, tor, seg_off + E, cap, &dy_row, &dy_col,
-                          recipe_scale_rule(recipe), stream);
+    if (pt && launch_amax_bf16(dy_dev, (int64_t)T * H, 1, dy_amax, st) != cudaSuccess) return MXMOE_ERR_CUDA;
+    s = quantize_impl(dy_dev, MXMOE_DTYPE_BF16, 1, T, H, tor, seg_off + E, cap, &dy_row, &dy_col, 0,
+                      recipe_scale_rule(recipe), stream, dy_amax, 0);
     if (s != MXMOE_OK) return s;
   }
   // 1b. G / U recomputed from the saved rowwise x (the fc1 GEMM again, epilogue writing
@@ -681,6 +822,11 @@ mxmoe_status grouped_mlp_bwd_ex(const void* dy_dev, const void* saved_dev, size_
     g.dprob_part = reinterpret_cast<float*>(ws + W.dprob_part);
     g.out_fmt = grad_format;
     g.scale_rule = recipe_scale_rule(recipe);
+    g.a_amax = dy_amax;
+    g.b_amax = w2_amax;
+    g.b_amax_per_expert = 1;
+    g.out_amax_in = dgu_used;
+    g.out_amax_rec = pt ? amax_state + 3 : nullptr;
     StageScope sc(MXMOE_STAGE_FC2_DGRAD, st);
     if (T > 0 && launch_gemm(g, st) != cudaSuccess) return MXMOE_ERR_CUDA;
   }
@@ -695,7 +841,7 @@ mxmoe_status grouped_mlp_bwd_ex(const void* dy_dev, const void* saved_dev, size_
   mxmoe_mxfp8 z_col = mk(sv, SL.off[MXMOE_SAVED_Z_COLT], SL.off[MXMOE_SAVED_Z_COLT_SF], F, cap);
   {
     StageScope sc(MXMOE_STAGE_FC2_WGRAD, st);
-    s = grouped_gemm_mxfp8_wgrad(&dy_col, &z_col, seg_off, E, dW2_dev, stream);
+    s = grouped_wgrad_impl(&dy_col, &z_col, seg_off, E, dW2_dev, stream, dy_amax, z_used);
   }
   if (s != MXMOE_OK) return s;
   // 5. fc1 dgrad: dXp = dGU . W1 (contract 2F)
@@ -703,8 +849,8 @@ mxmoe_status grouped_mlp_bwd_ex(const void* dy_dev, const void* saved_dev, size_
   mxmoe_mxfp8 w1c = mk(wq, WL.d[1], WL.s[1], WL.rows[1], WL.cols[1]);
   if (T > 0) {
     StageScope sc(MXMOE_STAGE_FC1_DGRAD, st);
-    s = grouped_gemm_mxfp8(&dgu_row, &w1c, seg_off, E, H, 2 * (int64_t)F, ws + W.dx_perm, MXMOE_DTYPE_BF16, H,
-                           stream);
+    s = grouped_gemm_impl(&dgu_row, &w1c, seg_off, E, H, 2 * (int64_t)F, ws + W.dx_perm, MXMOE_DTYPE_BF16, H, 0,
+                          stream, dgu_used, w1_amax);
     if (s != MXMOE_OK) return s;
   }
   // 6. fc1 wgrad: dW1[e] = dGU_e^T . Xp_e
@@ -712,7 +858,7 @@ mxmoe_status grouped_mlp_bwd_ex(const void* dy_dev, const void* saved_dev, size_
   mxmoe_mxfp8 x_col = mk(sv, SL.off[MXMOE_SAVED_X_COLT], SL.off[MXMOE_SAVED_X_COLT_SF], H, cap);
   {
     StageScope sc(MXMOE_STAGE_FC1_WGRAD, st);
-    s = grouped_gemm_mxfp8_wgrad(&dgu_col, &x_col, seg_off, E, dW1_dev, stream);
+    s = grouped_wgrad_impl(&dgu_col, &x_col, seg_off, E, dW1_dev, stream, dgu_used, x_amax);
   }
   if (s != MXMOE_OK) return s;
   // 7. combine dX

@@ -76,7 +76,7 @@ constexpr int kMaxE = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemSfa = 256;    // two buffers of 4 columns
 constexpr uint32_t kTmemSfb = 264;    // two buffers of 8 columns
-constexpr uint32_t kTmemStash = 384;  // epilogue scratch: 64 columns per (lane quadrant, half)
+constexpr uint32_t kTmemStash = 320;  // epilogue scratch: 96 columns per (lane quadrant, half)
 constexpr int kPrefetchSteps = 8;     // K steps of the next tile pulled into L2 at a tile start
 
 // Per-variant layout. Plain-store and weight-gradient modes: 5-stage operand ring, one
@@ -224,11 +224,20 @@ __device__ __forceinline__ uint32_t amax_bits32(const float (&v)[32]) {
 }
 
 // 32 fp32 -> 32 FP8 codes of format FMT (8 words) under the block's scale; returns the
-// E8M0 byte.
+// E8M0 byte. tm != 0: per-tensor FP8 under the multiplier tm (byte 127), and the block's
+// largest magnitude (fp32 bits) is folded into *amax_acc.
 template <int FMT = MXMOE_FMT_E4M3>
-__device__ __forceinline__ uint8_t quant32(const float (&v)[32], uint32_t (&q)[8], bool ceil_rule = false) {
-  const int32_t X = mx_scale_exp_from_amax_bits<FMT>(amax_bits32(v), ceil_rule);
-  const float sc = mx_inv_scale(X);
+__device__ __forceinline__ uint8_t quant32(const float (&v)[32], uint32_t (&q)[8], bool ceil_rule = false,
+                                           float tm = 0.f, uint32_t* amax_acc = nullptr) {
+  const uint32_t am = amax_bits32(v);
+  int32_t X = 0;
+  float sc = tm;
+  if (tm == 0.f) {
+    X = mx_scale_exp_from_amax_bits<FMT>(am, ceil_rule);
+    sc = mx_inv_scale(X);
+  } else if (amax_acc) {
+    *amax_acc = max(*amax_acc, am);
+  }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint32_t lo = fp8x2<FMT>(v[4 * i] * sc, v[4 * i + 1] * sc);
@@ -269,11 +278,20 @@ __device__ __forceinline__ void colwise_transpose2(const float (&v0)[32], const 
 template <int FMT = MXMOE_FMT_E4M3>
 __device__ __forceinline__ void colwise_codes2(const float (&v0)[32], const float (&v1)[32], float* stg, int lane,
                                                uint32_t (&q0)[8], uint32_t (&q1)[8], uint8_t& sb0, uint8_t& sb1,
-                                               bool ceil_rule = false) {
+                                               bool ceil_rule = false, float tm = 0.f) {
   float w0[32], w1[32];
   colwise_transpose2(v0, v1, stg, lane, w0, w1);
-  sb0 = quant32<FMT>(w0, q0, ceil_rule);
-  sb1 = quant32<FMT>(w1, q1, ceil_rule);
+  sb0 = quant32<FMT>(w0, q0, ceil_rule, tm);
+  sb1 = quant32<FMT>(w1, q1, ceil_rule, tm);
+}
+// Folds a warp's largest magnitude (fp32 bits, one per lane) into a launch-wide maximum.
+__device__ __forceinline__ void record_amax(float* dst, uint32_t am, int lane) {
+  am = __reduce_max_sync(0xffffffffu, am);
+  if (lane == 0 && am != 0) atomicMax(reinterpret_cast<unsigned int*>(dst), am);
+}
+// Per-tile output factor: 1 for MXFP8, 1 / (m_a * m_b) for per-tensor FP8 operands.
+__device__ __forceinline__ float tile_alpha(const GemmArgs& g, int32_t e) {
+  return g.a_amax ? tensor_alpha(*g.a_amax, g.b_amax[g.b_amax_per_expert ? e : 0]) : 1.f;
 }
 // bf16 output mode: lane r's 32 values as 64 bytes of bf16 at box + r * 64 (one row of a
 // 32 x 32 bf16 box).
@@ -353,12 +371,53 @@ __device__ __forceinline__ uint4 pack8_bf16(const uint32_t (&v)[N], int i0) {
   return o;
 }
 
+// Abort path of the GEMM kernel, called by every thread at teardown; it returns at once
+// unless a wait of this CTA ran out (s_abort). It is kept out of line and finds its state
+// in shared memory, so that the kernel's normal path keeps no extra values live.
+// The leader's producer thread waits (bounded) for the latest phase of every operand stage
+// it armed -- those phases also count the peer CTA's copies; the leader's MMA thread
+// commits once more and waits, so that every MMA it issued has completed; then one thread
+// per CTA lets 1 ms pass for copies that no barrier of its own tracks (a peer's, issued
+// ahead of the leader's producer). Nothing asynchronous is then in flight when TMEM is
+// released and the CTA retires.
+template <int PAIR, int STAGES, uint32_t kOffBars>
+__device__ __noinline__ void abort_drain() {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + kOffBars);
+  uint64_t* bar_drain = bar_full + 2 * STAGES + 2;
+  const volatile int32_t* s_abort = reinterpret_cast<const volatile int32_t*>(bar_drain + 1) + 1;
+  const uint32_t n_issued = *reinterpret_cast<const volatile uint32_t*>(s_abort + 2);
+  if (*s_abort == 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR == 2 ? ptx::cluster_rank() : 0u;
+  if (rank == 0 && lane == 0 && warp == 0) {
+    const uint32_t nlast = n_issued < (uint32_t)STAGES ? n_issued : (uint32_t)STAGES;
+    for (uint32_t j = 1; j <= nlast; ++j) {
+      const uint32_t i = n_issued - j;
+      ptx::mbar_wait(&bar_full[i % STAGES], (i / STAGES) & 1u, 5);
+    }
+  } else if (rank == 0 && lane == 0 && warp == 1) {
+    if (PAIR == 1) ptx::tc_commit(bar_drain);
+    else ptx::tc_commit_pair_mask(bar_drain, 0x1);
+    ptx::mbar_wait(bar_drain, 0, 6);
+  }
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = ptx::globaltimer();
+    while (ptx::globaltimer() - t0 < 1000000ull) {
+    }
+  }
+}
+
 // ESZ: operand element bytes -- 1: MXFP8 (E4M3 or E5M2 codes + E8M0 scales,
 // kind::mxf8f6f4.block_scale; the operand formats come from GemmArgs), 2: bf16 (kind::f16,
 // no scales; CTA pairs only).
 // OF: element format of the MXFP8 outputs of the backward fused epilogue (dGU): E4M3, or
 // E5M2 for the gradient variant.
-template <int MODE, int PAIR, int ESZ, int OF = MXMOE_FMT_E4M3>
+// PT: per-tensor FP8 operands and fused outputs (scale bytes 127; outputs scaled by
+// 1 / (m_a * m_b); Z / dGU encoded under a given multiplier, their largest magnitude
+// recorded). A separate instance, so the MXFP8 kernels carry none of it.
+template <int MODE, int PAIR, int ESZ, int OF = MXMOE_FMT_E4M3, bool PT = false>
 __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
     mxgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
@@ -376,9 +435,11 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
   uint64_t* bar_empty = bar_full + STAGES;
   uint64_t* bar_acc_full = bar_empty + STAGES;
   uint64_t* bar_acc_empty = bar_acc_full + 1;  // used in the leader CTA only
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_acc_empty + 1);
+  uint64_t* bar_drain = bar_acc_empty + 1;      // abort path: completion of the issued MMAs
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_drain + 1);
   volatile int32_t* s_abort = reinterpret_cast<volatile int32_t*>(s_tmem + 1);
   int32_t* s_bad = const_cast<int32_t*>(s_abort + 1);
+  uint32_t* s_issued = reinterpret_cast<uint32_t*>(s_bad + 1);  // operand stages the producer issued
   int32_t* s_seg = reinterpret_cast<int32_t*>(smem + C::kOffSeg);
   int32_t* s_order = reinterpret_cast<int32_t*>(smem + C::kOffOrder);
 
@@ -394,8 +455,10 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
     }
     ptx::mbar_init(bar_acc_full, 1);
     ptx::mbar_init(bar_acc_empty, kEpiWarps * PAIR);
+    ptx::mbar_init(bar_drain, 1);
     *s_abort = 0;
     *s_bad = 0;
+    *s_issued = 0;
     ptx::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -460,7 +523,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
     // ===================================================== TMA producer (every CTA)
     if (lane == 0) {
       int stage = 0;
-      uint32_t ph = 0;
+      uint32_t ph = 0, n_issued = 0;
       const int64_t a_kchunks = g.a_cols / 128, b_kchunks = g.b_cols / 128;
       for (int32_t tile = first; tile < ntiles && !*s_abort; tile += stride) {
         const TileInfo t = get_tile<MODE, PAIR, ESZ>(g, tile, s_seg, s_order, rank);
@@ -507,12 +570,14 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
               ptx::tma_load_2d_pair(s_sfa + kSfaBytes + 512, &tmSFB, 0, (int32_t)cb1, full_leader);
             }
           }
+          ++n_issued;
           if (++stage == STAGES) {
             stage = 0;
             ph ^= 1u;
           }
         }
       }
+      *s_issued = n_issued;
     }
    } else if (warp == 1) {
     // ===================================================== MMA issuer (leader CTA)
@@ -608,7 +673,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
     const uint64_t out_policy = ptx::make_policy_evict_first();
     uint32_t acc_ph = 0;
     const uint32_t t_lane = tmem_base + ((uint32_t)(32 * q) << 16);
-    const uint32_t t_stash = t_lane + kTmemStash + 64 * h;  // this warp's 64 spare TMEM columns
+    const uint32_t t_stash = t_lane + kTmemStash + 96 * h;  // this warp's 96 spare TMEM columns
     const uint32_t acc_empty_leader = PAIR == 2 ? ptx::map_to_rank(ptx::smem_u32(bar_acc_empty), 0) : 0u;
     for (int32_t tile = first; tile < ntiles; tile += stride) {
       // warp-uniform abort check (the TMEM loads below are warp-collective)
@@ -644,6 +709,11 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
             ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&acc[32 * c]));
           ptx::tmem_wait_ld();
           release_accumulator<PAIR>(bar_acc_empty, acc_empty_leader, lane);
+          const float alpha = PT ? tile_alpha(g, t.e) : 1.f;  // per-tensor FP8 operands: 1 / (m_a * m_b)
+          if (alpha != 1.f) {
+#pragma unroll
+            for (int i = 0; i < 128; ++i) acc[i] = __float_as_uint(__uint_as_float(acc[i]) * alpha);
+          }
         } else {
 #pragma unroll
           for (int i = 0; i < 128; ++i) acc[i] = 0u;
@@ -684,6 +754,16 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
         ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 96, *reinterpret_cast<uint32_t(*)[32]>(&ur[32]));
         ptx::tmem_wait_ld();
         release_accumulator<PAIR>(bar_acc_empty, acc_empty_leader, lane);
+        {
+          const float alpha = PT ? tile_alpha(g, t.e) : 1.f;  // per-tensor FP8 operands: 1 / (m_a * m_b)
+          if (alpha != 1.f) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+              gr[i] = __float_as_uint(__uint_as_float(gr[i]) * alpha);
+              ur[i] = __float_as_uint(__uint_as_float(ur[i]) * alpha);
+            }
+          }
+        }
         uint8_t* stg8 = reinterpret_cast<uint8_t*>(stg);
         // G and U as bf16 for the backward: two 32-row x 128-byte boxes (128-byte swizzle);
         // skipped when the forward does not save them (the backward recomputes them)
@@ -729,9 +809,14 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
         uint32_t r0[8], r1[8], c0[8], c1[8];
         uint8_t cs0, cs1;
         const bool cr = g.scale_rule != 0;
-        const uint32_t zsf = (uint32_t)quant32(z0, r0, cr) | ((uint32_t)quant32(z1, r1, cr) << 8);
+        // per-tensor FP8 Z: the multiplier from the given largest magnitude; this tile's
+        // largest |Z| joins the launch's record
+        const float tm = PT ? tensor_multiplier(*g.out_amax_in) : 0.f;
+        uint32_t zmax = 0;
+        const uint32_t zsf = (uint32_t)quant32(z0, r0, cr, tm, &zmax) | ((uint32_t)quant32(z1, r1, cr, tm, &zmax) << 8);
+        if (tm != 0.f) record_amax(g.out_amax_rec, zmax, lane);
         staging_acquire(lane);
-        colwise_codes2(z0, z1, stg, lane, c0, c1, cs0, cs1, cr);
+        colwise_codes2(z0, z1, stg, lane, c0, c1, cs0, cs1, cr, tm);
         put_codes32(stg8, lane, r0);
         put_codes32(stg8 + 1024, lane, r1);
         put_codes32(stg8 + 2048, lane, c0);
@@ -753,24 +838,22 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
         const int64_t F = g.F, F2 = 2 * g.F;
         const float p = g.prob_of_row[row];
         const int64_t f0 = (int64_t)t.n_tile * BN + 128 * h;  // this warp's 128 dZ columns
-        // phase 1: drain dZ into registers and hand the accumulator back at once, then park
-        // dZ in this warp's spare TMEM columns as packed bf16 pairs (the E4M3 rounding that
-        // follows is 2^5 coarser than that rounding)
+        // phase 1: drain dZ (fp32) into registers and hand the accumulator back at once;
+        // the first 32 columns stay in registers, the other 96 are parked, still fp32, in
+        // this warp's spare TMEM columns
+        uint32_t dz0[32];
         {
-          uint32_t dzr[128];
+          uint32_t dzr[96];
+          ptx::tmem_ld_32x32b_x32(t_lane + 128 * h, dz0);
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&dzr[32 * c]));
+          for (int c = 1; c < 4; ++c)
+            ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 32 * c,
+                                    *reinterpret_cast<uint32_t(*)[32]>(&dzr[32 * (c - 1)]));
           ptx::tmem_wait_ld();
           release_accumulator<PAIR>(bar_acc_empty, acc_empty_leader, lane);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = pack_bf16x2(__uint_as_float(dzr[32 * c + 2 * i]), __uint_as_float(dzr[32 * c + 2 * i + 1]));
-            ptx::tmem_st_32x32b_x16(t_stash + 16 * c, pk);
-          }
+          for (int c = 0; c < 3; ++c)
+            ptx::tmem_st_32x32b_x32(t_stash + 32 * c, *reinterpret_cast<const uint32_t(*)[32]>(&dzr[32 * c]));
           ptx::tmem_wait_st();
         }
         // phase 2: SwiGLU / probability backward, 32 columns at a time; G and U (pulled into
@@ -785,10 +868,13 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
         }
         float dprob = 0.f;
         uint32_t sfg = 0, sfu = 0;  // row scales of the four dG / dU blocks
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t dzw[16];
-          ptx::tmem_ld_32x32b_x16(t_stash + 16 * c, dzw);
+        const float alpha = PT ? tile_alpha(g, t.e) : 1.f;  // per-tensor FP8 operands: 1 / (m_a * m_b)
+        // per-tensor FP8 dGU: the multiplier from the given largest magnitude
+        const float tm = PT ? tensor_multiplier(*g.out_amax_in) : 0.f;
+        uint32_t gmax = 0;
+        // one 32-column chunk: dzw holds its dZ (fp32 bit patterns), possibly still in flight
+        // from TMEM until the wait below
+        auto chunk = [&](const int c, const uint32_t(&dzw)[32]) {
           const uint32_t gw[16] = {gq[0].x, gq[0].y, gq[0].z, gq[0].w, gq[1].x, gq[1].y, gq[1].z, gq[1].w,
                                    gq[2].x, gq[2].y, gq[2].z, gq[2].w, gq[3].x, gq[3].y, gq[3].z, gq[3].w};
           const uint32_t uw[16] = {uq[0].x, uq[0].y, uq[0].z, uq[0].w, uq[1].x, uq[1].y, uq[1].z, uq[1].w,
@@ -806,7 +892,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           for (int i = 0; i < 32; ++i) {
             const float gg = (i & 1) ? bf16_hi(gw[i >> 1]) : bf16_lo(gw[i >> 1]);
             const float uu = (i & 1) ? bf16_hi(uw[i >> 1]) : bf16_lo(uw[i >> 1]);
-            const float dz = (i & 1) ? bf16_hi(dzw[i >> 1]) : bf16_lo(dzw[i >> 1]);
+            const float dz = __uint_as_float(dzw[i]) * alpha;
             const float sg = sigmoid_f(gg);                  // sigmoid(G)
             const float sl = gg * sg;                        // silu(G)
             const float da = dz * p;                         // dA = dZ * p
@@ -832,15 +918,15 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
               ptx::tma_store_2d(&tmD, stg8 + 6144, (int32_t)mrow0, (int32_t)(F + fg));
               ptx::bulk_commit_group();
             }
-            continue;
+            return;
           }
           uint32_t rg[8], ru[8], cg[8], cu[8];
           uint8_t csg, csu;
           const bool cr = g.scale_rule != 0;
-          sfg |= (uint32_t)quant32<OF>(vg, rg, cr) << (8 * c);
-          sfu |= (uint32_t)quant32<OF>(vu, ru, cr) << (8 * c);
+          sfg |= (uint32_t)quant32<OF>(vg, rg, cr, tm, &gmax) << (8 * c);
+          sfu |= (uint32_t)quant32<OF>(vu, ru, cr, tm, &gmax) << (8 * c);
           staging_acquire(lane);
-          colwise_codes2<OF>(vg, vu, stg, lane, cg, cu, csg, csu, cr);
+          colwise_codes2<OF>(vg, vu, stg, lane, cg, cu, csg, csu, cr, tm);
           uint8_t* stg8 = reinterpret_cast<uint8_t*>(stg);
           put_codes32(stg8, lane, rg);
           put_codes32(stg8 + 1024, lane, ru);
@@ -856,7 +942,15 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           }
           g.dgu_colT_sf[sf_offset(MXMOE_SCALE_MMA, F2, g.rows_cap, fg + lane, mrow0 / 32)] = csg;
           g.dgu_colT_sf[sf_offset(MXMOE_SCALE_MMA, F2, g.rows_cap, F + fg + lane, mrow0 / 32)] = csu;
+        };
+        chunk(0, dz0);
+#pragma unroll 1
+        for (int c = 1; c < 4; ++c) {
+          uint32_t dzw[32];
+          ptx::tmem_ld_32x32b_x32(t_stash + 32 * (c - 1), dzw);
+          chunk(c, dzw);
         }
+        if (tm != 0.f) record_amax(g.out_amax_rec, gmax, lane);  // this tile's largest |dGU|
         // row scales: blocks f0/32 .. +3 (and their up-half twins) are one aligned word each
         if (ESZ == 1) {
           *reinterpret_cast<uint32_t*>(g.dgu_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F2, row, f0 / 32)) = sfg;
@@ -874,7 +968,11 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
   // accumulator, so every MMA has completed before TMEM is released. With CTA pairs the
   // cluster barrier also keeps each CTA (and the barriers its peer signals) alive until
   // the peer is done.
+  // After an abort (a wait that ran out) nothing asynchronous may still be in flight when
+  // TMEM is released or the CTA retires (abort_drain).
   ptx::tc_fence_before();
+  __syncthreads();
+  abort_drain<PAIR, STAGES, C::kOffBars>();
   __syncthreads();
   if (PAIR == 2) ptx::cluster_sync();
   if (warp == 1) {
@@ -976,21 +1074,22 @@ struct GemmMaps {
   CUtensorMap c, d, e;  // epilogue outputs (unused ones zeroed)
 };
 
-template <int MODE, int PAIR, int ESZ = 1, int OF = MXMOE_FMT_E4M3>
+template <int MODE, int PAIR, int ESZ = 1, int OF = MXMOE_FMT_E4M3, bool PT = false>
 static cudaError_t launch_mode(const GemmMaps& m, const GemmArgs& g, int64_t tiles_ub, cudaStream_t st) {
   constexpr uint32_t smem = Cfg<PAIR, MODE>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(mxgemm_kernel<MODE, PAIR, ESZ, OF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(mxgemm_kernel<MODE, PAIR, ESZ, OF, PT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // the warpgroup register split assumes the launch allocation it was sized for
   cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, mxgemm_kernel<MODE, PAIR, ESZ, OF>);
+  e = cudaFuncGetAttributes(&fa, mxgemm_kernel<MODE, PAIR, ESZ, OF, PT>);
   if (e != cudaSuccess) return e;
   if (Cfg<PAIR, MODE>::kSplitRegs && fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
   const int units = gemm_num_sms() / PAIR;  // SMs, or SM pairs
   const int n = (int)(tiles_ub < units ? (tiles_ub > 0 ? tiles_ub : 1) : units);
   if constexpr (PAIR == 1) {
-    mxgemm_kernel<MODE, 1, ESZ, OF><<<n, Cfg<PAIR, MODE>::kThreads, smem, st>>>(m.a, m.b, m.sfa, m.sfb, m.c, m.d, m.e, g);
+    mxgemm_kernel<MODE, 1, ESZ, OF, PT><<<n, Cfg<PAIR, MODE>::kThreads, smem, st>>>(m.a, m.b, m.sfa, m.sfb, m.c, m.d,
+                                                                                  m.e, g);
   } else {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * n, 1, 1);
@@ -1004,14 +1103,14 @@ static cudaError_t launch_mode(const GemmMaps& m, const GemmArgs& g, int64_t til
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, mxgemm_kernel<MODE, PAIR, ESZ, OF>, m.a, m.b, m.sfa, m.sfb, m.c, m.d, m.e, g);
+    e = cudaLaunchKernelEx(&cfg, mxgemm_kernel<MODE, PAIR, ESZ, OF, PT>, m.a, m.b, m.sfa, m.sfb, m.c, m.d, m.e, g);
     if (e != cudaSuccess) return e;
   }
   ++g_launch_count;
   return cudaGetLastError();
 }
 
-template <int PAIR>
+template <int PAIR, bool PT>
 static cudaError_t launch_variant(const GemmArgs& g, cudaStream_t st) {
   GemmMaps m;
   std::memset(&m.c, 0, sizeof(m.c));
@@ -1024,10 +1123,14 @@ static cudaError_t launch_variant(const GemmArgs& g, cudaStream_t st) {
   constexpr int TM = 128 * PAIR;
   if (g.out_fmt != MXMOE_FMT_E4M3 && (g.mode != kModeSwigluBwd || g.out_fmt != MXMOE_FMT_E5M2))
     return cudaErrorInvalidValue;  // Z stays E4M3; only the backward epilogue writes E5M2
+  if (PT && (g.out_fmt != MXMOE_FMT_E4M3 || g.a_fmt != MXMOE_FMT_E4M3 || g.b_fmt != MXMOE_FMT_E4M3 || !g.b_amax ||
+             ((g.mode == kModeSwigluFwd && g.z_row) || g.mode == kModeSwigluBwd) != (g.out_amax_in != nullptr) ||
+             (g.out_amax_in != nullptr) != (g.out_amax_rec != nullptr)))
+    return cudaErrorInvalidValue;  // per-tensor FP8 is E4M3 throughout; fused outputs need both amax words
   switch (g.mode) {
     case kModeStore:
       if (!make_out_map(&m.c, g.c, g.a_rows, g.N, g.ldc, g.c_dtype == MXMOE_DTYPE_F32)) return cudaErrorInvalidValue;
-      return launch_mode<kModeStore, PAIR>(m, g, (g.a_rows / TM) * (g.N / BN), st);
+      return launch_mode<kModeStore, PAIR, 1, MXMOE_FMT_E4M3, PT>(m, g, (g.a_rows / TM) * (g.N / BN), st);
     case kModeSwigluFwd:
       // Z (rows + colT) and the saved G / U are each optional, not both absent
       if ((g.z_row == nullptr) != (g.z_colT == nullptr) || (g.z_row == nullptr && g.gu == nullptr))
@@ -1036,17 +1139,17 @@ static cudaError_t launch_variant(const GemmArgs& g, cudaStream_t st) {
                       !make_codes32_map(&m.d, g.z_colT, g.F, g.rows_cap)))
         return cudaErrorInvalidValue;
       if (g.gu && !make_out_map(&m.e, g.gu, g.rows_cap, 2 * g.F, 2 * g.F, false)) return cudaErrorInvalidValue;
-      return launch_mode<kModeSwigluFwd, PAIR>(m, g, (g.a_rows / TM) * (g.F / 128), st);
+      return launch_mode<kModeSwigluFwd, PAIR, 1, MXMOE_FMT_E4M3, PT>(m, g, (g.a_rows / TM) * (g.F / 128), st);
     case kModeSwigluBwd:
       if (!make_codes32_map(&m.c, g.dgu_row, g.rows_cap, 2 * g.F) ||
           !make_codes32_map(&m.d, g.dgu_colT, 2 * g.F, g.rows_cap))
         return cudaErrorInvalidValue;
-      if (g.out_fmt == MXMOE_FMT_E5M2)
+      if (!PT && g.out_fmt == MXMOE_FMT_E5M2)
         return launch_mode<kModeSwigluBwd, PAIR, 1, MXMOE_FMT_E5M2>(m, g, (g.a_rows / TM) * (g.F / BN), st);
-      return launch_mode<kModeSwigluBwd, PAIR>(m, g, (g.a_rows / TM) * (g.F / BN), st);
+      return launch_mode<kModeSwigluBwd, PAIR, 1, MXMOE_FMT_E4M3, PT>(m, g, (g.a_rows / TM) * (g.F / BN), st);
     case kModeWgrad:
       if (!make_out_map(&m.c, g.c, (int64_t)g.E * g.N, g.K2, g.K2, true)) return cudaErrorInvalidValue;
-      return launch_mode<kModeWgrad, PAIR>(m, g, (int64_t)g.E * (g.N / TM) * (g.K2 / BN), st);
+      return launch_mode<kModeWgrad, PAIR, 1, MXMOE_FMT_E4M3, PT>(m, g, (int64_t)g.E * (g.N / TM) * (g.K2 / BN), st);
   }
   return cudaErrorInvalidValue;
 }
@@ -1081,7 +1184,9 @@ static cudaError_t launch_bf16(const GemmArgs& g, cudaStream_t st) {
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
   if (g.bf16_operands) return launch_bf16(g, st);
-  return gemm_tile_rows() == 128 ? launch_variant<1>(g, st) : launch_variant<2>(g, st);
+  if (g.a_amax)  // per-tensor FP8 operands
+    return gemm_tile_rows() == 128 ? launch_variant<1, true>(g, st) : launch_variant<2, true>(g, st);
+  return gemm_tile_rows() == 128 ? launch_variant<1, false>(g, st) : launch_variant<2, false>(g, st);
 }
 
 }  // namespace mxmoe

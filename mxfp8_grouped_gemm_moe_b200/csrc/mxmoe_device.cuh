@@ -55,15 +55,32 @@ __device__ __forceinline__ uint16_t fp8x2(float a, float b) {
 }
 __device__ __forceinline__ uint16_t e4m3x2(float a, float b) { return fp8x2<MXMOE_FMT_E4M3>(a, b); }
 
+// Per-tensor FP8: the fp32 multiplier m = 448 / amax, rounded to nearest (IEEE
+// division), 1 when amax == 0 and the largest finite fp32 when the quotient overflows. An
+// element's code is E4M3(fp32(v * m)).
+__device__ __forceinline__ float tensor_multiplier(float amax) {
+  if (!(amax > 0.f)) return 1.f;
+  return fminf(__fdiv_rn(448.f, amax), 3.40282346638528859812e38f);
+}
+// Dequantisation factor of a product of two per-tensor operands: 1 / (m_a * m_b).
+__device__ __forceinline__ float tensor_alpha(float amax_a, float amax_b) {
+  return __frcp_rn(tensor_multiplier(amax_a) * tensor_multiplier(amax_b));
+}
+
 // Quantise 32 fp32 values held by one thread -> 32 codes packed in 8 words; returns the
-// E8M0 scale byte.
+// E8M0 scale byte. tm != 0: per-tensor FP8 under the multiplier tm (scale byte 127).
 template <int FMT = MXMOE_FMT_E4M3>
-__device__ __forceinline__ uint8_t quant_block32(const float (&v)[32], uint32_t (&out)[8], bool ceil_rule = false) {
-  uint32_t amax = 0;
+__device__ __forceinline__ uint8_t quant_block32(const float (&v)[32], uint32_t (&out)[8], bool ceil_rule = false,
+                                                 float tm = 0.f) {
+  int32_t X = 0;
+  float s = tm;
+  if (tm == 0.f) {
+    uint32_t amax = 0;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) amax = max(amax, __float_as_uint(fabsf(v[i])));
-  const int32_t X = mx_scale_exp_from_amax_bits<FMT>(amax, ceil_rule);
-  const float s = mx_inv_scale(X);
+    for (int i = 0; i < 32; ++i) amax = max(amax, __float_as_uint(fabsf(v[i])));
+    X = mx_scale_exp_from_amax_bits<FMT>(amax, ceil_rule);
+    s = mx_inv_scale(X);
+  }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint32_t lo = fp8x2<FMT>(v[4 * i + 0] * s, v[4 * i + 1] * s);

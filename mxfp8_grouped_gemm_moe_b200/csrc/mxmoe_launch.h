@@ -47,8 +47,16 @@ struct QuantArgs {
   int64_t row_ilv;
   int32_t fmt;         // element format of both outputs: MXMOE_FMT_E4M3 or MXMOE_FMT_E5M2
   int32_t scale_rule;  // MXMOE_SCALE_RULE_OCP or MXMOE_SCALE_RULE_CEIL
+  // per-tensor FP8 (E4M3 only): when set, every element is encoded under the multiplier
+  // m = 448 / amax of its tensor (tensor_amax[batch index] when tensor_per_batch, else
+  // tensor_amax[0]) and every scale byte is 127 (2^0); null: MXFP8 block scales
+  const float* tensor_amax;
+  int32_t tensor_per_batch;
 };
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
+// Largest magnitude of each of `groups` consecutive bf16 arrays of n elements
+// (n % 8 == 0, 16-byte aligned) into out[groups] (fp32; cleared first).
+cudaError_t launch_amax_bf16(const void* src, int64_t n, int32_t groups, float* out, cudaStream_t st);
 // bf16 -> bf16 copies with the same row gather / valid-row count / gate-up interleave as
 // launch_quantize: row_data receives the (permuted) rows, col_data the transposed matrix
 // [batch*cols, out_rows]; the scale fields are ignored. bf16 sources only.
@@ -100,6 +108,16 @@ struct GemmArgs {
   float* dprob_part;  // [rows_cap, F/128]
   int32_t out_fmt;    // element format of the fused epilogues' MXFP8 outputs (Z / dGU)
   int32_t scale_rule; // scale rule of the fused epilogues' quantisers (MXMOE_SCALE_RULE_*)
+  // per-tensor FP8 (null for MXFP8): the operands' largest magnitudes (fp32); b_amax holds
+  // one value per expert when b_amax_per_expert. Every output is scaled by
+  // 1 / (m(a_amax) * m(b_amax)), m(amax) = 448 / amax (the operands' scale bytes are 127).
+  const float* a_amax;
+  const float* b_amax;
+  int32_t b_amax_per_expert;
+  // per-tensor FP8 outputs of the fused epilogues (Z, dGU): encoded under m(*out_amax_in);
+  // the largest |output| over the launch is recorded into *out_amax_rec (atomic max)
+  const float* out_amax_in;
+  float* out_amax_rec;
   // debug: if non-zero, the MMA warp withholds its first accumulator-ready signal so
   // that the epilogue's bounded wait expires (tests the timeout path; never set in
   // normal use)

@@ -87,15 +87,20 @@ __device__ __forceinline__ void load_pair(const float* p, float& a, float& b) {
 // 2k+1 in the high half). |bf16| bit patterns order like unsigned 16-bit integers, so
 // the block amax is a SIMD max over the masked words; the result equals the amax of the
 // values widened to fp32 (widening is exact), hence the same scale as quant_block32.
+// tm != 0: per-tensor FP8 under the multiplier tm (scale byte 127).
 template <int FMT = MXMOE_FMT_E4M3>
 __device__ __forceinline__ uint8_t quant_block32_bf16(const uint32_t (&w)[16], uint32_t (&out)[8],
-                                                      bool ceil_rule = false) {
-  uint32_t m = 0;
+                                                      bool ceil_rule = false, float tm = 0.f) {
+  int32_t X = 0;
+  float s = tm;
+  if (tm == 0.f) {
+    uint32_t m = 0;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
-  const uint32_t amax = max(m << 16, m & 0xFFFF0000u);
-  const int32_t X = mx_scale_exp_from_amax_bits<FMT>(amax, ceil_rule);
-  const float s = mx_inv_scale(X);
+    for (int i = 0; i < 16; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+    const uint32_t amax = max(m << 16, m & 0xFFFF0000u);
+    X = mx_scale_exp_from_amax_bits<FMT>(amax, ceil_rule);
+    s = mx_inv_scale(X);
+  }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint32_t lo = fp8x2<FMT>(bf16_lo(w[2 * i]) * s, bf16_hi(w[2 * i]) * s);
@@ -109,13 +114,19 @@ __device__ __forceinline__ uint8_t quant_block32_bf16(const uint32_t (&w)[16], u
 // its low half and (column c+1, row r) in its high half.
 template <int FMT = MXMOE_FMT_E4M3>
 __device__ __forceinline__ void quant_colpair_bf16(const uint32_t (&w)[32], uint32_t (&o0)[8], uint32_t (&o1)[8],
-                                                   uint8_t& sb0, uint8_t& sb1, bool ceil_rule = false) {
-  uint32_t m = 0;
+                                                   uint8_t& sb0, uint8_t& sb1, bool ceil_rule = false,
+                                                   float tm = 0.f) {
+  int32_t X0 = 0, X1 = 0;
+  float s0 = tm, s1 = tm;
+  if (tm == 0.f) {
+    uint32_t m = 0;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
-  const int32_t X0 = mx_scale_exp_from_amax_bits<FMT>(m << 16, ceil_rule);
-  const int32_t X1 = mx_scale_exp_from_amax_bits<FMT>(m & 0xFFFF0000u, ceil_rule);
-  const float s0 = mx_inv_scale(X0), s1 = mx_inv_scale(X1);
+    for (int i = 0; i < 32; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+    X0 = mx_scale_exp_from_amax_bits<FMT>(m << 16, ceil_rule);
+    X1 = mx_scale_exp_from_amax_bits<FMT>(m & 0xFFFF0000u, ceil_rule);
+    s0 = mx_inv_scale(X0);
+    s1 = mx_inv_scale(X1);
+  }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     o0[i] = (uint32_t)fp8x2<FMT>(bf16_lo(w[4 * i]) * s0, bf16_lo(w[4 * i + 1]) * s0) |
@@ -128,40 +139,41 @@ __device__ __forceinline__ void quant_colpair_bf16(const uint32_t (&w)[32], uint
 }
 
 template <int FMT>
-__device__ __forceinline__ uint8_t quant_row_block(const __nv_bfloat16* p, uint32_t (&q)[8], bool ceil_rule) {
+__device__ __forceinline__ uint8_t quant_row_block(const __nv_bfloat16* p, uint32_t (&q)[8], bool ceil_rule,
+                                                   float tm) {
   uint32_t w[16];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint4 v = reinterpret_cast<const uint4*>(p)[i];
     w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
   }
-  return quant_block32_bf16<FMT>(w, q, ceil_rule);
+  return quant_block32_bf16<FMT>(w, q, ceil_rule, tm);
 }
 template <int FMT>
-__device__ __forceinline__ uint8_t quant_row_block(const float* p, uint32_t (&q)[8], bool ceil_rule) {
+__device__ __forceinline__ uint8_t quant_row_block(const float* p, uint32_t (&q)[8], bool ceil_rule, float tm) {
   float v[32];
   load32_row(p, v);
-  return quant_block32<FMT>(v, q, ceil_rule);
+  return quant_block32<FMT>(v, q, ceil_rule, tm);
 }
 
 template <int FMT>
 __device__ __forceinline__ void quant_col_pair(const __nv_bfloat16* p, int ld, uint32_t (&q0)[8], uint32_t (&q1)[8],
-                                               uint8_t& s0, uint8_t& s1, bool ceil_rule) {
+                                               uint8_t& s0, uint8_t& s1, bool ceil_rule, float tm) {
   uint32_t w[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) w[i] = *reinterpret_cast<const uint32_t*>(p + i * ld);
-  quant_colpair_bf16<FMT>(w, q0, q1, s0, s1, ceil_rule);
+  quant_colpair_bf16<FMT>(w, q0, q1, s0, s1, ceil_rule, tm);
 }
 template <int FMT>
 __device__ __forceinline__ void quant_col_pair(const float* p, int ld, uint32_t (&q0)[8], uint32_t (&q1)[8],
-                                               uint8_t& s0, uint8_t& s1, bool ceil_rule) {
+                                               uint8_t& s0, uint8_t& s1, bool ceil_rule, float tm) {
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = p[i * ld];
-  s0 = quant_block32<FMT>(v, q0, ceil_rule);
+  s0 = quant_block32<FMT>(v, q0, ceil_rule, tm);
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = p[i * ld + 1];
-  s1 = quant_block32<FMT>(v, q1, ceil_rule);
+  s1 = quant_block32<FMT>(v, q1, ceil_rule, tm);
 }
 
 // One CTA per 128 x 128 tile (many resident per SM to overlap load latency).
@@ -181,6 +193,7 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
   }
   if (r0 >= nvalid) return;
   const T* src = reinterpret_cast<const T*>(a.src);
+  const float tm = a.tensor_amax ? tensor_multiplier(a.tensor_amax[a.tensor_per_batch ? b : 0]) : 0.f;
 
   // ---- load the tile (gathered rows, zero outside the matrix / for pad rows); all of a
   // thread's row indices, then all of its 16-byte loads, are issued before any use
@@ -218,7 +231,7 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
       const int64_t col = c0 + 32 * blk;
       if (orow >= nvalid || col >= a.cols) continue;
       uint32_t q[8];
-      const uint8_t sb = quant_row_block<FMT>(tile + tile_off<T>(row, 32 * blk), q, a.scale_rule != 0);
+      const uint8_t sb = quant_row_block<FMT>(tile + tile_off<T>(row, 32 * blk), q, a.scale_rule != 0, tm);
       int64_t drow = orow;
       if (a.row_ilv > 0) {  // gate / up interleave of the fc1 operand
         const int64_t hf = orow >= a.row_ilv, rr = orow - hf * a.row_ilv;
@@ -240,7 +253,8 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
     if (orow < nvalid && col < a.cols) {
       uint32_t q0[8], q1[8];
       uint8_t s0, s1;
-      quant_col_pair<FMT>(tile + tile_off<T>(32 * rb, 2 * pcol), 4 * Tr::kBS, q0, q1, s0, s1, a.scale_rule != 0);
+      quant_col_pair<FMT>(tile + tile_off<T>(32 * rb, 2 * pcol), 4 * Tr::kBS, q0, q1, s0, s1, a.scale_rule != 0,
+                          tm);
       const int64_t grow = b * a.cols + col;  // row of the transposed matrix
       uint4* d0 = reinterpret_cast<uint4*>(a.col_data + grow * a.out_rows + orow);
       uint4* d1 = reinterpret_cast<uint4*>(a.col_data + (grow + 1) * a.out_rows + orow);
@@ -330,6 +344,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
     const uint8_t* st = smem + (i % kQtStages) * kQtStageBytes;
     int64_t b, r0, c0;
     tile_of(i, b, r0, c0);
+    const float tm = a.tensor_amax ? tensor_multiplier(a.tensor_amax[a.tensor_per_batch ? b : 0]) : 0.f;
 
     // rowwise: 512 items (row, 32-column block), 2 per thread; a warp takes 8 rows and
     // lanes l, l + 8, l + 16, l + 24 share a row, so each 8-lane phase of a 16-byte shared
@@ -346,7 +361,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
         w[4 * t] = v.x; w[4 * t + 1] = v.y; w[4 * t + 2] = v.z; w[4 * t + 3] = v.w;
       }
       uint32_t q[8];
-      const uint8_t sb = quant_block32_bf16(w, q, a.scale_rule != 0);
+      const uint8_t sb = quant_block32_bf16(w, q, a.scale_rule != 0, tm);
       *reinterpret_cast<uint4*>(out_row + sw128(row, 2 * blk)) = make_uint4(q[0], q[1], q[2], q[3]);
       *reinterpret_cast<uint4*>(out_row + sw128(row, 2 * blk + 1)) = make_uint4(q[4], q[5], q[6], q[7]);
       const int64_t orow = r0 + row;
@@ -367,7 +382,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
       for (int r = 0; r < 32; ++r) w[r] = *reinterpret_cast<const uint32_t*>(st + qt_off(32 * rb + r, 2 * pcol));
       uint32_t q0[8], q1[8];
       uint8_t s0, s1;
-      quant_colpair_bf16(w, q0, q1, s0, s1, a.scale_rule != 0);
+      quant_colpair_bf16(w, q0, q1, s0, s1, a.scale_rule != 0, tm);
       *reinterpret_cast<uint4*>(out_col + sw128(2 * pcol, 2 * rb)) = make_uint4(q0[0], q0[1], q0[2], q0[3]);
       *reinterpret_cast<uint4*>(out_col + sw128(2 * pcol, 2 * rb + 1)) = make_uint4(q0[4], q0[5], q0[6], q0[7]);
       *reinterpret_cast<uint4*>(out_col + sw128(2 * pcol + 1, 2 * rb)) = make_uint4(q1[0], q1[1], q1[2], q1[3]);
@@ -563,8 +578,44 @@ static cudaError_t launch_q(const QuantArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// ----------------------------------------------------------------------------- per-tensor amax
+// Largest magnitude of each group (blockIdx.y) of a bf16 array: a grid-stride pass of
+// 16-byte loads per group, a SIMD max over the magnitude bits (|bf16| patterns order like
+// unsigned integers), a warp max, one atomic per warp on the group's fp32 word (non-negative
+// fp32 bit patterns also order like unsigned integers). HBM-bound: n * 2 bytes per group.
+__global__ void __launch_bounds__(256) amax_bf16_kernel(const uint4* __restrict__ src, int64_t nvec,
+                                                        float* __restrict__ out) {
+  const uint4* p = src + (int64_t)blockIdx.y * nvec;
+  uint32_t m = 0;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nvec; i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 v = __ldg(p + i);
+    m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
+  }
+  uint32_t am = max(m << 16, m & 0xFFFF0000u);
+  am = __reduce_max_sync(0xffffffffu, am);
+  if ((threadIdx.x & 31) == 0 && am != 0) atomicMax(reinterpret_cast<unsigned int*>(out + blockIdx.y), am);
+}
+
+cudaError_t launch_amax_bf16(const void* src, int64_t n, int32_t groups, float* out, cudaStream_t st) {
+  if (n <= 0 || n % 8 != 0 || groups < 1 || groups > 65535) return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * (size_t)groups, st);
+  if (e != cudaSuccess) return e;
+  const int64_t nvec = n / 8;
+  int64_t gx = (int64_t)gemm_num_sms() * 8 / groups;
+  const int64_t need = (nvec + 255) / 256;
+  gx = gx < 1 ? 1 : (gx > need ? need : gx);
+  amax_bf16_kernel<<<dim3((unsigned)gx, (unsigned)groups), 256, 0, st>>>(reinterpret_cast<const uint4*>(src), nvec,
+                                                                        out);
+  ++g_launch_count;
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st) {
   if (a.fmt != MXMOE_FMT_E4M3 && a.fmt != MXMOE_FMT_E5M2) return cudaErrorInvalidValue;
+  if (a.tensor_amax && a.fmt != MXMOE_FMT_E4M3) return cudaErrorInvalidValue;
   if (qt_applies(a)) return launch_qt(a, st);
   if (a.fmt == MXMOE_FMT_E5M2)
     return a.src_dtype == MXMOE_DTYPE_BF16 ? launch_q<__nv_bfloat16, MXMOE_FMT_E5M2>(a, st)

@@ -63,7 +63,18 @@ def test_sizes_are_host_only(lib):
     assert s >= cap * (4096 + 14336) * (1 + 1 / 32) + cap * 2 * 14336 * 2
     offs = [lib.grouped_mlp_saved_offset(f, 8192, 2, 8, 4096, 14336) for f in range(10)]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
-    assert lib.grouped_mlp_saved_offset(12, 1, 1, 1, 256, 256) == -1
+    assert lib.grouped_mlp_saved_offset(13, 1, 1, 1, 256, 256) == -1
+    # per-tensor FP8: the saved amax field takes room only under that recipe; the recipe
+    # combines with no other bit, and the MXFP8 _ex calls' sizes are unchanged by it
+    fp8 = 8
+    a = lib.grouped_mlp_saved_offset_ex(12, 8192, 2, 8, 4096, 14336, fp8)
+    assert a >= 0 and a % 256 == 0
+    assert lib.grouped_mlp_saved_size_ex(8192, 2, 8, 4096, 14336, fp8) == a + 256
+    assert lib.grouped_mlp_saved_size_ex(8192, 2, 8, 4096, 14336, 0) == lib.grouped_mlp_saved_size(8192, 2, 8, 4096,
+                                                                                                  14336)
+    assert lib.grouped_mlp_saved_size_ex(8192, 2, 8, 4096, 14336, fp8 | 1) == 0
+    assert lib.grouped_mlp_workspace_size_ex(8192, 2, 8, 4096, 14336, fp8) >= \
+        lib.grouped_mlp_workspace_size_ex(8192, 2, 8, 4096, 14336, 0)
 
 
 def test_host_argument_errors_enqueue_nothing(lib):
@@ -121,12 +132,22 @@ def test_host_argument_errors_enqueue_nothing(lib):
                                16, S) == 3
     assert lib.grouped_mlp_bwd(fake, fake, 1 << 40, fake, 1 << 40, 16, 2, 4, 256, 512, fake, bad, fake, fake,
                                fake, 1 << 40, S) == 1
-    # recipe flags: only MXMOE_RECIPE_GRAD_E5M2 | _RECOMPUTE_GU | _SCALE_CEIL (1 | 2 | 4)
+    # recipe flags: MXMOE_RECIPE_GRAD_E5M2 | _RECOMPUTE_GU | _SCALE_CEIL (1 | 2 | 4), or
+    # _FP8_TENSOR (8) alone, which the _ex calls refuse (it runs through grouped_mlp_fp8_*)
     assert lib.grouped_mlp_bwd_ex(fake, fake, 1 << 40, fake, 1 << 40, 16, 2, 4, 256, 512, 8, fake, fake, fake, fake,
                                   fake, 1 << 40, S) == 1
     assert lib.grouped_mlp_fwd_ex(fake, fake, fake, fake, 1 << 40, 16, 2, 4, 256, 512, 16, fake, fake, 1 << 40, fake,
                                   1 << 40, S) == 1
-    assert lib.grouped_mlp_saved_size_ex(16, 2, 4, 256, 512, 8) == 0
+    assert lib.grouped_mlp_fwd_ex(fake, fake, fake, fake, 1 << 40, 16, 2, 4, 256, 512, 8, fake, fake, 1 << 40, fake,
+                                  1 << 40, S) == 1
+    assert lib.grouped_mlp_saved_size_ex(16, 2, 4, 256, 512, 16) == 0
+    assert lib.grouped_mlp_saved_size_ex(16, 2, 4, 256, 512, 8 | 4) == 0
+    # per-tensor FP8: the delayed-scaling state must be given (16-byte aligned)
+    assert lib.grouped_mlp_fp8_fwd(fake, fake, fake, fake, 1 << 40, 16, 2, 4, 256, 512, None, fake, fake, 1 << 40,
+                                   fake, 1 << 40, S) == 1
+    assert lib.grouped_mlp_fp8_bwd(fake, fake, 1 << 40, fake, 1 << 40, 16, 2, 4, 256, 512, P((1 << 20) + 4), fake,
+                                   fake, fake, fake, fake, 1 << 40, S) == 1
+    assert lib.mxmoe_weights_quantize_fp8(fake, fake, 4, 256, 384, fake, 1 << 40, S) == 2
     assert lib.grouped_mlp_saved_size_ex(16, 2, 4, 256, 512, 7) > 0
     # scale rules: only OCP (0) and CEIL (1)
     m_ok = mx._MX(1 << 20, 1 << 20, 64, 64, 0, 0)

@@ -53,6 +53,11 @@ def test_fused_mlp_matches_oracle(gpu_lib, name):
         assert v <= TOL_E2E, (k, v)
     if name == "small":   # expert 7 has no tokens: zero weight gradients
         assert torch.all(dW1[cfg.E - 1] == 0) and torch.all(dW2[cfg.E - 1] == 0)
+    else:                 # and directly against the expert-by-expert restatement of the backward
+        ge = omoe.mlp_bwd_per_expert(f64(d["x"]), f64(d["dy"]), d["topk_idx"].numpy(), f64(d["probs"]),
+                                     f64(d["W1"]), f64(d["W2"]))
+        for k, got in (("dx", dx), ("dW1", dW1), ("dW2", dW2), ("dprobs", dprobs)):
+            assert rel_l2(f64(got), ge[k]) <= TOL_E2E, (k, "per expert")
 
 
 def test_fused_forward_tiny_config(gpu_lib):

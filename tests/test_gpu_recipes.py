@@ -247,10 +247,8 @@ def test_fused_layer_ceil_rule_matches_oracle(gpu_lib, grad_format):
     errs = dict(y=rel_l2(f64(y), yo), dx=rel_l2(f64(dx), go["dx"]), dW1=rel_l2(f64(dW1), go["dW1"]),
                 dW2=rel_l2(f64(dW2), go["dW2"]), dprobs=rel_l2(f64(dprobs), go["dprobs"]))
     print(grad_format, {k: f"{v:.2e}" for k, v in errs.items()})
-    # The GPU computes dGU in fp32 from a bf16 dZ, the oracle in fp64: near rounding
-    # midpoints the two pick neighbouring codes. Such flips are rarer and larger as the code
-    # step grows, so the relative L2 error grows as the square root of the step: E5M2
-    # gradients (one mantissa bit fewer) get sqrt(2) times the E4M3 bar.
-    tol = TOL_E2E * (np.sqrt(2.0) if grad_format == "e5m2" else 1.0)
+    # the stated end-to-end bar for every recipe; the GPU's remaining departures from the
+    # fp64 oracle (G / U saved as bf16, the approximate logistic function) move a few dGU
+    # codes by one step, which E5M2's wider step makes larger (about 1.6e-2 here)
     for k, v in errs.items():
-        assert v <= tol, (k, v)
+        assert v <= TOL_E2E, (k, v)
