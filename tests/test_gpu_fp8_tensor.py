@@ -5,8 +5,8 @@ Bars: the largest magnitudes the amax passes find and every E4M3 code of the wei
 of the permuted activations are bit-exact (both sides round fp32(v * m) to E4M3 with the
 same correctly rounded multiplier); the fused layer's outputs reach relative L2 <= 2e-2
 against the oracle run with the same delayed-scaling values for Z and dGU; the largest
-|Z| and |dGU| the fused epilogues record agree with the oracle's to 1e-3 (they come from
-fp32 values on the GPU, fp64 in the oracle)."""
+|Z| the forward records agrees with the oracle's to 1e-3 (fp32 values on the GPU, fp64 in
+the oracle), the largest |dGU| to 2^-7 (the backward reads G / U saved as bf16)."""
 import numpy as np
 import pytest
 import torch
@@ -94,7 +94,9 @@ def test_fp8_tensor_layer_matches_oracle(gpu_lib, name):
     # the largest |Z| and |dGU| recorded by the fused epilogues, then rolled into the inputs
     st = layer.amax_state.cpu().numpy()
     assert abs(st[1] - so["z_amax"]) <= 1e-3 * so["z_amax"], (st[1], so["z_amax"])
-    assert abs(st[3] - go["dgu_amax"]) <= 1e-3 * go["dgu_amax"], (st[3], go["dgu_amax"])
+    # dGU comes from G / U saved as bf16 (each rounded by at most 2^-9), so its largest
+    # magnitude may differ from the oracle's by up to about 2^-8 relative
+    assert abs(st[3] - go["dgu_amax"]) <= 2.0 ** -7 * go["dgu_amax"], (st[3], go["dgu_amax"])
     layer.roll_amax()
     st2 = layer.amax_state.cpu().numpy()
     assert st2[0] == st[1] and st2[2] == st[3]
