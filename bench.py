@@ -108,10 +108,13 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
+    _n = 0
+
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join("/tmp", f"mxmoe_clocks_{os.getpid()}.csv")
+        ClockSampler._n += 1   # one file per sampler: several run in one process
+        self.path = os.path.join("/tmp", f"mxmoe_clocks_{os.getpid()}_{ClockSampler._n}.csv")
 
     def start(self):
         try:
@@ -565,6 +568,7 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier(dist)
     launches = mx.mxmoe_launch_count() - n0
+    clk = clocks.stop()
     ms = ev0.elapsed_time(ev1) / args.steps
     stages = mx.mxmoe_profile_read()
     mx.mxmoe_profile_disable()
@@ -621,7 +625,9 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
     # step i+1's inputs travel while step i computes (a pipelined training loop); all of
     # them sit inside the timed region.
     e2e = None
+    clocks_e2e = ClockSampler(local_rank)
     if not args.no_e2e:
+        clocks_e2e.start()
         pin = lambda t: t.cpu().pin_memory()  # noqa: E731
         x_h, dy_h, idx_h2, probs_h2 = pin(x), pin(dy), pin(idx), pin(probs)
         y_h, dx_h, dp_h = pin(y), pin(dx), pin(dprobs)
@@ -694,7 +700,9 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
                "tokens_per_s": world * cfg.T / (ems * 1e-3),
                "note": "inputs copied host->device and results read back every step, on a side stream "
                        "overlapping the neighbouring steps' compute"}
-    clk = clocks.stop()
+    clk_e2e = clocks_e2e.stop()
+    if e2e is not None:
+        e2e["clocks"] = clk_e2e
 
     st, where = mx.mxmoe_get_device_status()
     if st != 0:
