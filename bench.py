@@ -568,56 +568,10 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier(dist)
     launches = mx.mxmoe_launch_count() - n0
-    clk = clocks.stop()
     ms = ev0.elapsed_time(ev1) / args.steps
     stages = mx.mxmoe_profile_read()
     mx.mxmoe_profile_disable()
     ms = max_over_ranks(dist, ms)
-
-    # ---- the same step under the alternative recipes (E5M2 gradients; G / U recomputed)
-    recipes = None
-    if rank == 0 and world == 1 and not args.no_bf16_compare:
-        recipes = time_recipes(cfg, layer, W1, W2, x, idx, probs, dy, y, dx, dW1, dW2, dprobs, stream,
-                               min(args.steps, 5))
-
-    # ---- the same step on the bf16 layer: the 16-bit comparison point, timed on its own
-    bf16_layer = None
-    if rank == 0 and world == 1 and not args.no_bf16_compare:
-        bf16_layer = time_bf16_layer(cfg, W1, W2, x, idx, probs, dy, stream, dev, min(args.steps, 5))
-
-    # ---- the other workloads of the target (skewed Mixtral routing; genomics), each
-    # timed on its own after the headline
-    workloads = None
-    if rank == 0 and world == 1 and not args.no_workloads and cfg.name == "mixtral":
-        peaks0, _ = load_peaks()
-        workloads = {n: time_workload(n, dev, min(args.steps, 5), 2, peaks0) for n in ("mixtral_zipf", "genomics")}
-
-    # ---- router (the step upstream of the layer; timed on its own, not part of `value`)
-    router = None
-    if rank == 0:
-        lg = torch.randn((cfg.T, cfg.E), generator=g, device=dev)
-        ridx, rp = mx.moe_router_topk(lg, cfg.k)
-        rdp = torch.randn_like(rp)
-        rdl = mx.moe_router_topk_bwd(lg, ridx, rdp)
-        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        times = []
-        for fn in (lambda: mx.moe_router_topk(lg, cfg.k), lambda: mx.moe_router_topk_bwd(lg, ridx, rdp)):
-            for _ in range(3):
-                fn()
-            torch.cuda.synchronize()
-            r0.record(stream)
-            for _ in range(20):
-                fn()
-            r1.record(stream)
-            torch.cuda.synchronize()
-            times.append(r0.elapsed_time(r1) / 20)
-        fb = cfg.T * cfg.E * 4 + cfg.T * cfg.k * 8
-        bb = 2 * cfg.T * cfg.E * 4 + cfg.T * cfg.k * 8
-        router = {"fwd_ms": times[0], "bwd_ms": times[1], "fwd_gbs": fb / (times[0] * 1e-3) / 1e9,
-                  "bwd_gbs": bb / (times[1] * 1e-3) / 1e9,
-                  "note": "softmax over all experts + top-k, and its backward, on [T, E] fp32 logits; "
-                          "timed separately (the layer's input routing is given)"}
-        del lg, ridx, rp, rdp, rdl
 
     # ---- end to end through the public API with host buffers: every step copies its
     # inputs (x, top-k ids, probabilities, dY) from pinned host memory and reads its
@@ -625,9 +579,7 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
     # step i+1's inputs travel while step i computes (a pipelined training loop); all of
     # them sit inside the timed region.
     e2e = None
-    clocks_e2e = ClockSampler(local_rank)
     if not args.no_e2e:
-        clocks_e2e.start()
         pin = lambda t: t.cpu().pin_memory()  # noqa: E731
         x_h, dy_h, idx_h2, probs_h2 = pin(x), pin(dy), pin(idx), pin(probs)
         y_h, dx_h, dp_h = pin(y), pin(dx), pin(dprobs)
@@ -700,9 +652,53 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
                "tokens_per_s": world * cfg.T / (ems * 1e-3),
                "note": "inputs copied host->device and results read back every step, on a side stream "
                        "overlapping the neighbouring steps' compute"}
-    clk_e2e = clocks_e2e.stop()
-    if e2e is not None:
-        e2e["clocks"] = clk_e2e
+    # clocks sampled over both timed runs of the step (device-resident, then end to end)
+    clk = clocks.stop()
+    # ---- the same step under the alternative recipes (E5M2 gradients; G / U recomputed)
+    recipes = None
+    if rank == 0 and world == 1 and not args.no_bf16_compare:
+        recipes = time_recipes(cfg, layer, W1, W2, x, idx, probs, dy, y, dx, dW1, dW2, dprobs, stream,
+                               min(args.steps, 5))
+
+    # ---- the same step on the bf16 layer: the 16-bit comparison point, timed on its own
+    bf16_layer = None
+    if rank == 0 and world == 1 and not args.no_bf16_compare:
+        bf16_layer = time_bf16_layer(cfg, W1, W2, x, idx, probs, dy, stream, dev, min(args.steps, 5))
+
+    # ---- the other workloads of the target (skewed Mixtral routing; genomics), each
+    # timed on its own after the headline
+    workloads = None
+    if rank == 0 and world == 1 and not args.no_workloads and cfg.name == "mixtral":
+        peaks0, _ = load_peaks()
+        workloads = {n: time_workload(n, dev, min(args.steps, 5), 2, peaks0) for n in ("mixtral_zipf", "genomics")}
+
+    # ---- router (the step upstream of the layer; timed on its own, not part of `value`)
+    router = None
+    if rank == 0:
+        lg = torch.randn((cfg.T, cfg.E), generator=g, device=dev)
+        ridx, rp = mx.moe_router_topk(lg, cfg.k)
+        rdp = torch.randn_like(rp)
+        rdl = mx.moe_router_topk_bwd(lg, ridx, rdp)
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        times = []
+        for fn in (lambda: mx.moe_router_topk(lg, cfg.k), lambda: mx.moe_router_topk_bwd(lg, ridx, rdp)):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            r0.record(stream)
+            for _ in range(20):
+                fn()
+            r1.record(stream)
+            torch.cuda.synchronize()
+            times.append(r0.elapsed_time(r1) / 20)
+        fb = cfg.T * cfg.E * 4 + cfg.T * cfg.k * 8
+        bb = 2 * cfg.T * cfg.E * 4 + cfg.T * cfg.k * 8
+        router = {"fwd_ms": times[0], "bwd_ms": times[1], "fwd_gbs": fb / (times[0] * 1e-3) / 1e9,
+                  "bwd_gbs": bb / (times[1] * 1e-3) / 1e9,
+                  "note": "softmax over all experts + top-k, and its backward, on [T, E] fp32 logits; "
+                          "timed separately (the layer's input routing is given)"}
+        del lg, ridx, rp, rdp, rdl
+
 
     st, where = mx.mxmoe_get_device_status()
     if st != 0:
