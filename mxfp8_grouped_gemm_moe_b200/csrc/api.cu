@@ -9,6 +9,8 @@
 #include <cstring>
 
 #include "../../include/mxmoe.h"
+#include <nvtx3/nvToolsExt.h>
+
 #include "mxmoe_launch.h"
 
 #include "mxmoe_device.cuh"
@@ -190,10 +192,22 @@ struct Profiler {
 };
 Profiler g_prof;
 
+// Stage names for NVTX ranges (index = MXMOE_STAGE_* tag).
+const char* const kStageNames[] = {"",           "route",       "quant_x",       "fc1_swiglu",    "fc2",
+                                   "combine",    "quant_w1",    "quant_w2",      "quant_dy",      "fc2_dgrad_swiglu_bwd",
+                                   "dprob",      "fc2_wgrad",   "fc1_dgrad",     "fc1_wgrad",     "combine_dx",
+                                   "gemm",       "wgrad",       "quant",         "router",        "router_bwd",
+                                   "fc1_recompute"};
+
+// One stage of the layer: an NVTX range on the host timeline (free unless a profiler
+// such as Nsight Systems is attached) and, while mxmoe_profile_enable is on, a pair of
+// CUDA events on the stage's stream (outermost stages only).
 struct StageScope {
   cudaStream_t st;
   bool rec = false;
   StageScope(int32_t tag, cudaStream_t s) : st(s) {
+    nvtxRangePushA(tag >= 0 && tag < (int32_t)(sizeof(kStageNames) / sizeof(kStageNames[0])) ? kStageNames[tag]
+                                                                                              : "mxmoe");
     if (g_prof.on && g_prof.depth == 0 && g_prof.n < g_prof.cap) {
       cudaEventRecord(g_prof.ev[2 * g_prof.n], st);
       g_prof.tags[g_prof.n] = tag;
@@ -207,6 +221,7 @@ struct StageScope {
       cudaEventRecord(g_prof.ev[2 * g_prof.n + 1], st);
       ++g_prof.n;
     }
+    nvtxRangePop();
   }
 };
 
