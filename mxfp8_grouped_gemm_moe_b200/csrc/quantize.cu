@@ -414,174 +414,6 @@ __global__ void __launch_bounds__(kQThreads, 2)
   if (threadIdx.x == 0) ptx::bulk_wait_group<0>();
 }
 
-// ----------------------------------------------------------------------------- gathered bf16 path
-// Persistent variant for the permutation fused with quantisation (x and dY: row r of the
-// output is source row gather[r], -1 = a zero pad row), bf16 sources, 128-multiple shapes.
-// Warp 0 loads: for every 128 x 128 tile it reads the 128 row indices and issues one
-// 256-byte bulk copy (cp.async.bulk) per live row into a 4-stage ring, zero-filling pad
-// rows, all completing on the stage's barrier; nothing is staged in registers, so a tile
-// or more of loads is in flight while the other warps quantise. Rows sit 272 bytes apart
-// (256 + 16), which makes the rowwise 16-byte and the colwise column-pair shared loads bank
-// conflict free. Warps 1..8 quantise as the dense TMA path does (same block arithmetic),
-// assemble both copies' codes in 128-byte-swizzled staging (two buffers) and write them by
-// TMA stores; scale bytes are stored directly.
-constexpr int kQgStages = 4;
-constexpr uint32_t kQgPitch = 272;                                 // bytes per tile row in the ring
-constexpr uint32_t kQgStageBytes = kQTile * kQgPitch;              // 34816
-constexpr uint32_t kQgOutBytes = 2 * kQTile * 128;                 // row + col codes of one tile
-constexpr uint32_t kQgOffOut = kQgStages * kQgStageBytes;
-constexpr uint32_t kQgOffBar = kQgOffOut + 2 * kQgOutBytes;
-constexpr uint32_t kQgSmem = kQgOffBar + 128 + 1024;
-constexpr int kQgThreads = 32 + kQThreads;                        // loader warp + 8 quantising warps
-
-template <int FMT>
-__global__ void __launch_bounds__(kQgThreads, 1)
-    mxfp8_quantize_gather_kernel(const __grid_constant__ CUtensorMap tm_row, const __grid_constant__ CUtensorMap tm_col,
-                                 const __grid_constant__ QuantArgs a, int32_t tiles_c) {
-  extern __shared__ uint8_t qg_smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qg_smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQgOffBar);
-  uint64_t* empty = full + kQgStages;
-  volatile int32_t* s_abort = reinterpret_cast<volatile int32_t*>(empty + kQgStages);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kQgStages; ++s) {
-      ptx::mbar_init(&full[s], 1);
-      ptx::mbar_init(&empty[s], kQThreads / 32);
-    }
-    *s_abort = 0;
-    ptx::fence_mbar_init();
-    ptx::prefetch_tensormap(&tm_row);
-    ptx::prefetch_tensormap(&tm_col);
-  }
-  __syncthreads();
-  int64_t nvalid = a.out_rows;
-  if (a.nrows) {
-    const int64_t nv = *a.nrows;
-    nvalid = nv < nvalid ? nv : nvalid;
-  }
-  const int32_t ntiles = (int32_t)((nvalid + kQTile - 1) / kQTile) * tiles_c;
-  const int32_t first = (int32_t)blockIdx.x, stride = (int32_t)gridDim.x;
-  const uint16_t* src = reinterpret_cast<const uint16_t*>(a.src);
-
-  if (warp == 0) {
-    // ============================== loader
-    int32_t i = 0;
-    for (int32_t t = first; t < ntiles && !*s_abort; t += stride, ++i) {
-      const int s = i % kQgStages;
-      if (!ptx::mbar_wait(&empty[s], ((uint32_t)(i / kQgStages) & 1u) ^ 1u, 31)) {
-        *s_abort = 1;
-        break;
-      }
-      const int64_t r0 = (int64_t)(t / tiles_c) * kQTile, c0 = (int64_t)(t % tiles_c) * kQTile;
-      uint8_t* st = smem + s * kQgStageBytes;
-      // this lane's rows j = lane + 32 m: source row, or -1 for a zero row
-      int64_t tok[kQTile / 32];
-      uint32_t live = 0;
-#pragma unroll
-      for (int m = 0; m < kQTile / 32; ++m) {
-        const int64_t r = r0 + lane + 32 * m;
-        tok[m] = r < nvalid ? (int64_t)__ldg(a.gather + r) : -1;
-        if (tok[m] >= a.rows) tok[m] = -1;
-        live += __popc(__ballot_sync(0xffffffffu, tok[m] >= 0));
-      }
-#pragma unroll
-      for (int m = 0; m < kQTile / 32; ++m) {
-        if (tok[m] < 0) {
-          uint4* z = reinterpret_cast<uint4*>(st + (lane + 32 * m) * kQgPitch);
-#pragma unroll
-          for (int q = 0; q < 16; ++q) z[q] = make_uint4(0, 0, 0, 0);
-        }
-      }
-      // the zero rows are written before the arrive (release) that publishes the stage; the
-      // barrier expects the live rows' bytes before any copy is issued
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive_expect_tx(&full[s], live * 256u);
-      __syncwarp();
-#pragma unroll
-      for (int m = 0; m < kQTile / 32; ++m)
-        if (tok[m] >= 0) ptx::bulk_load(st + (lane + 32 * m) * kQgPitch, src + (tok[m] * a.cols + c0), 256, &full[s]);
-    }
-  } else {
-    // ============================== quantising warps
-    const int tid = threadIdx.x - 32;
-    const float tm = a.tensor_amax ? tensor_multiplier(a.tensor_amax[0]) : 0.f;
-    const bool cr = a.scale_rule != 0;
-    int32_t i = 0;
-    for (int32_t t = first; t < ntiles; t += stride, ++i) {
-      const int s = i % kQgStages;
-      const bool ok = ptx::mbar_wait(&full[s], (uint32_t)(i / kQgStages) & 1u, 32);
-      if (!__all_sync(0xffffffffu, ok)) *s_abort = 1;
-      // this staging buffer was last used two tiles ago: its TMA stores have read it. Every
-      // quantising warp reaches this barrier (a wait that ran out only sets the flag), so the
-      // decision to stop below is the same in all of them.
-      if (tid == 0) ptx::bulk_wait_group_read<1>();
-      asm volatile("bar.sync 1, %0;" ::"n"(kQThreads) : "memory");
-      if (*s_abort) break;
-      const int64_t r0 = (int64_t)(t / tiles_c) * kQTile, c0 = (int64_t)(t % tiles_c) * kQTile;
-      const uint8_t* st = smem + s * kQgStageBytes;
-      uint8_t* out_row = smem + kQgOffOut + (i & 1) * kQgOutBytes;
-      uint8_t* out_col = out_row + kQTile * 128;
-      // rowwise: 512 items (row, 32-column block), 2 per thread; a warp takes 8 rows, lanes l,
-      // l + 8, l + 16, l + 24 share a row, so each 8-lane phase reads 8 rows 272 bytes apart
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int it = tid + k * kQThreads;
-        const int l = it & 31;
-        const int row = 8 * (it >> 5) + (l & 7), blk = l >> 3;
-        uint32_t w[16];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 v = *reinterpret_cast<const uint4*>(st + row * kQgPitch + blk * 64 + 16 * q);
-          w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
-        }
-        uint32_t qc[8];
-        const uint8_t sb = quant_block32_bf16<FMT>(w, qc, cr, tm);
-        *reinterpret_cast<uint4*>(out_row + sw128(row, 2 * blk)) = make_uint4(qc[0], qc[1], qc[2], qc[3]);
-        *reinterpret_cast<uint4*>(out_row + sw128(row, 2 * blk + 1)) = make_uint4(qc[4], qc[5], qc[6], qc[7]);
-        a.row_sf[sf_offset(a.row_layout, a.out_rows, a.cols, r0 + row, (c0 >> 5) + blk)] = sb;
-      }
-      // colwise: item = (pair of adjacent columns, 32-row block), one per thread; a warp reads
-      // 32 consecutive column pairs of a row per load
-      {
-        const int pcol = tid & 63, rb = tid >> 6;
-        uint32_t w[32];
-#pragma unroll
-        for (int r = 0; r < 32; ++r) w[r] = *reinterpret_cast<const uint32_t*>(st + (32 * rb + r) * kQgPitch + 4 * pcol);
-        uint32_t q0[8], q1[8];
-        uint8_t s0, s1;
-        quant_colpair_bf16<FMT>(w, q0, q1, s0, s1, cr, tm);
-        *reinterpret_cast<uint4*>(out_col + sw128(2 * pcol, 2 * rb)) = make_uint4(q0[0], q0[1], q0[2], q0[3]);
-        *reinterpret_cast<uint4*>(out_col + sw128(2 * pcol, 2 * rb + 1)) = make_uint4(q0[4], q0[5], q0[6], q0[7]);
-        *reinterpret_cast<uint4*>(out_col + sw128(2 * pcol + 1, 2 * rb)) = make_uint4(q1[0], q1[1], q1[2], q1[3]);
-        *reinterpret_cast<uint4*>(out_col + sw128(2 * pcol + 1, 2 * rb + 1)) = make_uint4(q1[4], q1[5], q1[6], q1[7]);
-        const int64_t grow = c0 + 2 * pcol;  // row of the transposed matrix
-        const int64_t kb = (r0 >> 5) + rb;
-        a.col_sf[sf_offset(a.col_layout, a.cols, a.out_rows, grow, kb)] = s0;
-        a.col_sf[sf_offset(a.col_layout, a.cols, a.out_rows, grow + 1, kb)] = s1;
-      }
-      // the stage has been read: hand it back to the loader
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&empty[s]);
-      ptx::fence_proxy_async_shared();  // this thread's staging writes before the TMA stores
-      asm volatile("bar.sync 1, %0;" ::"n"(kQThreads) : "memory");
-      if (tid == 0) {
-        ptx::tma_store_2d(&tm_row, out_row, (int32_t)c0, (int32_t)r0);
-        ptx::tma_store_2d(&tm_col, out_col, (int32_t)r0, (int32_t)c0);
-        ptx::bulk_commit_group();
-      }
-    }
-    if (tid == 0) ptx::bulk_wait_group<0>();
-  }
-  // after an abort let any copy still in flight land before the CTA retires
-  __syncthreads();
-  if (*s_abort && threadIdx.x == 0) {
-    const uint64_t t0 = ptx::globaltimer();
-    while (ptx::globaltimer() - t0 < 1000000ull) {
-    }
-  }
-}
-
 // ----------------------------------------------------------------------------- bf16 operand copies
 // Operands of the bf16 grouped MLP: the same tiles, gather and interleave as the
 // quantiser, but the outputs are plain bf16 -- the (permuted) rows and the transposed
@@ -781,36 +613,10 @@ cudaError_t launch_amax_bf16(const void* src, int64_t n, int32_t groups, float* 
   return cudaGetLastError();
 }
 
-static bool qg_applies(const QuantArgs& a) {
-  return a.src_dtype == MXMOE_DTYPE_BF16 && a.gather && a.batch == 1 && a.out_rows % kQTile == 0 &&
-         a.cols % kQTile == 0 && a.out_rows < (int64_t)1 << 31 && a.cols < (int64_t)1 << 31 && a.row_data &&
-         a.col_data && (reinterpret_cast<uintptr_t>(a.row_data) & 15) == 0 &&
-         (reinterpret_cast<uintptr_t>(a.col_data) & 15) == 0 && (reinterpret_cast<uintptr_t>(a.src) & 15) == 0;
-}
-template <int FMT>
-static cudaError_t launch_qg(const QuantArgs& a, cudaStream_t st) {
-  CUtensorMap tm_row, tm_col;
-  if (!make_code_map(&tm_row, a.row_data, a.out_rows, a.cols, 128) ||
-      !make_code_map(&tm_col, a.col_data, a.cols, a.out_rows, 128))
-    return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(mxfp8_quantize_gather_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kQgSmem);
-  if (e != cudaSuccess) return e;
-  const int32_t tiles_c = (int32_t)(a.cols / kQTile);
-  const int64_t tiles_ub = (a.out_rows / kQTile) * tiles_c;  // the device trims to seg_off[E]
-  if (tiles_ub == 0) return cudaSuccess;
-  const int grid = (int)std::min<int64_t>(tiles_ub, gemm_num_sms());
-  mxfp8_quantize_gather_kernel<FMT><<<grid, kQgThreads, kQgSmem, st>>>(tm_row, tm_col, a, tiles_c);
-  ++g_launch_count;
-  return cudaGetLastError();
-}
-
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st) {
   if (a.fmt != MXMOE_FMT_E4M3 && a.fmt != MXMOE_FMT_E5M2) return cudaErrorInvalidValue;
   if (a.tensor_amax && a.fmt != MXMOE_FMT_E4M3) return cudaErrorInvalidValue;
   if (qt_applies(a)) return launch_qt(a, st);
-  if (qg_applies(a))
-    return a.fmt == MXMOE_FMT_E5M2 ? launch_qg<MXMOE_FMT_E5M2>(a, st) : launch_qg<MXMOE_FMT_E4M3>(a, st);
   if (a.fmt == MXMOE_FMT_E5M2)
     return a.src_dtype == MXMOE_DTYPE_BF16 ? launch_q<__nv_bfloat16, MXMOE_FMT_E5M2>(a, st)
                                            : launch_q<float, MXMOE_FMT_E5M2>(a, st);
