@@ -200,27 +200,41 @@ __device__ __forceinline__ TileInfo get_tile(const GemmArgs& g, int32_t idx, con
 }
 
 // Logistic function from the hardware tanh: s(x) = (1 + tanh(x/2)) / 2 -- one special-
-// function-unit op and no division (the epilogues are bound by that unit). Its error
-// (about 2^-11 relative to 1) sits far below the E4M3 rounding that follows.
+// function-unit op and no division. Its error (about 2^-11 relative to 1) sits far below
+// the E4M3 rounding that follows.
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-__device__ __forceinline__ float sigmoid_f(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
-__device__ __forceinline__ float silu_f(float x) { return x * sigmoid_f(x); }
+// The epilogues' element-wise math runs on pairs of adjacent columns: sm_100 executes one
+// packed fp32x2 multiply / FMA per instruction, each lane rounded as its scalar op would
+// be, which halves the issue slots of the arithmetic (the epilogue warps are issue- and
+// latency-bound, not bound by a functional unit).
+__device__ __forceinline__ float2 sigmoid2(float2 x) {
+  const float2 half = make_float2(0.5f, 0.5f);
+  const float2 h = __fmul2_rn(x, half);
+  return __ffma2_rn(half, make_float2(tanh_approx(h.x), tanh_approx(h.y)), half);
+}
 
-// Largest |v[i]| as an fp32 bit pattern (integer max of the magnitude bits; a pairwise
-// tree so the 32 comparisons are 5 dependent steps deep).
+// Largest |v[i]| as an fp32 bit pattern: a pairwise tree of max-of-magnitudes (5
+// dependent steps deep), one instruction per comparison (the sign of each partial result
+// is meaningless and is cleared at the end). A NaN anywhere gives the canonical NaN, so
+// the block scale comes out of an all-ones exponent as for any NaN input.
+__device__ __forceinline__ float absmax2(float a, float b) {
+  float r;
+  asm("max.NaN.xorsign.abs.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
 __device__ __forceinline__ uint32_t amax_bits32(const float (&v)[32]) {
-  uint32_t m[16];
+  float m[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) m[i] = max(__float_as_uint(v[2 * i]) & 0x7FFFFFFFu, __float_as_uint(v[2 * i + 1]) & 0x7FFFFFFFu);
+  for (int i = 0; i < 16; ++i) m[i] = absmax2(v[2 * i], v[2 * i + 1]);
 #pragma unroll
   for (int w = 8; w >= 1; w >>= 1)
 #pragma unroll
-    for (int i = 0; i < w; ++i) m[i] = max(m[i], m[i + w]);
-  return m[0];
+    for (int i = 0; i < w; ++i) m[i] = absmax2(m[i], m[i + w]);
+  return __float_as_uint(m[0]) & 0x7FFFFFFFu;
 }
 
 // 32 fp32 -> 32 FP8 codes of format FMT (8 words) under the block's scale; returns the
@@ -238,11 +252,12 @@ __device__ __forceinline__ uint8_t quant32(const float (&v)[32], uint32_t (&q)[8
   } else if (amax_acc) {
     *amax_acc = max(*amax_acc, am);
   }
+  const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t lo = fp8x2<FMT>(v[4 * i] * sc, v[4 * i + 1] * sc);
-    const uint32_t hi = fp8x2<FMT>(v[4 * i + 2] * sc, v[4 * i + 3] * sc);
-    q[i] = lo | (hi << 16);
+    const float2 a = __fmul2_rn(make_float2(v[4 * i], v[4 * i + 1]), sc2);
+    const float2 b = __fmul2_rn(make_float2(v[4 * i + 2], v[4 * i + 3]), sc2);
+    q[i] = (uint32_t)fp8x2<FMT>(a.x, a.y) | ((uint32_t)fp8x2<FMT>(b.x, b.y) << 16);
   }
   return (uint8_t)(X + 127);
 }
@@ -784,7 +799,13 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
         if (g.z_row == nullptr) continue;  // recompute of G / U for the backward: no Z
         float zf[64];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) zf[i] = silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]) * p;
+        for (int i = 0; i < 32; ++i) {
+          const float2 gg = make_float2(__uint_as_float(gr[2 * i]), __uint_as_float(gr[2 * i + 1]));
+          const float2 uu = make_float2(__uint_as_float(ur[2 * i]), __uint_as_float(ur[2 * i + 1]));
+          const float2 z = __fmul2_rn(__fmul2_rn(__fmul2_rn(gg, sigmoid2(gg)), uu), make_float2(p, p));
+          zf[2 * i] = z.x;
+          zf[2 * i + 1] = z.y;
+        }
         // MXFP8 of Z, rowwise (fc2 operand) and colwise (fc2 weight-gradient operand)
         const float(&z0)[32] = *reinterpret_cast<const float(*)[32]>(&zf[0]);
         const float(&z1)[32] = *reinterpret_cast<const float(*)[32]>(&zf[32]);
@@ -841,10 +862,10 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
         // phase 1: drain dZ (fp32) into registers and hand the accumulator back at once;
         // the first 32 columns stay in registers, the other 96 are parked, still fp32, in
         // this warp's spare TMEM columns
-        uint32_t dz0[32];
+        uint32_t dz[32];
         {
           uint32_t dzr[96];
-          ptx::tmem_ld_32x32b_x32(t_lane + 128 * h, dz0);
+          ptx::tmem_ld_32x32b_x32(t_lane + 128 * h, dz);
 #pragma unroll
           for (int c = 1; c < 4; ++c)
             ptx::tmem_ld_32x32b_x32(t_lane + 128 * h + 32 * c,
@@ -866,15 +887,16 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           gq[i] = gsrc[i];
           uq[i] = usrc[i];
         }
-        float dprob = 0.f;
+        float2 dprob2 = make_float2(0.f, 0.f);
         uint32_t sfg = 0, sfu = 0;  // row scales of the four dG / dU blocks
         const float alpha = PT ? tile_alpha(g, t.e) : 1.f;  // per-tensor FP8 operands: 1 / (m_a * m_b)
         // per-tensor FP8 dGU: the multiplier from the given largest magnitude
         const float tm = PT ? tensor_multiplier(*g.out_amax_in) : 0.f;
         uint32_t gmax = 0;
         // one 32-column chunk: dzw holds its dZ (fp32 bit patterns), possibly still in flight
-        // from TMEM until the wait below
-        auto chunk = [&](const int c, const uint32_t(&dzw)[32]) {
+        // from TMEM until the wait below; once the chunk's math has read it, dzw receives
+        // the next chunk's dZ from the spare columns
+        auto chunk = [&](const int c, uint32_t(&dzw)[32]) {
           const uint32_t gw[16] = {gq[0].x, gq[0].y, gq[0].z, gq[0].w, gq[1].x, gq[1].y, gq[1].z, gq[1].w,
                                    gq[2].x, gq[2].y, gq[2].z, gq[2].w, gq[3].x, gq[3].y, gq[3].z, gq[3].w};
           const uint32_t uw[16] = {uq[0].x, uq[0].y, uq[0].z, uq[0].w, uq[1].x, uq[1].y, uq[1].z, uq[1].w,
@@ -888,18 +910,29 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           }
           ptx::tmem_wait_ld();
           float vg[32], vu[32];
+          const float2 one2 = make_float2(1.f, 1.f), p2 = make_float2(p, p);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float gg = (i & 1) ? bf16_hi(gw[i >> 1]) : bf16_lo(gw[i >> 1]);
-            const float uu = (i & 1) ? bf16_hi(uw[i >> 1]) : bf16_lo(uw[i >> 1]);
-            const float dz = __uint_as_float(dzw[i]) * alpha;
-            const float sg = sigmoid_f(gg);                  // sigmoid(G)
-            const float sl = gg * sg;                        // silu(G)
-            const float da = dz * p;                         // dA = dZ * p
-            dprob += dz * sl * uu;                           // dprob += dZ * A
-            vg[i] = da * uu * (sg * (1.0f + gg * (1.0f - sg)));
-            vu[i] = da * sl;
+          for (int i = 0; i < 16; ++i) {
+            const float2 gg = make_float2(bf16_lo(gw[i]), bf16_hi(gw[i]));
+            const float2 uu = make_float2(bf16_lo(uw[i]), bf16_hi(uw[i]));
+            float2 dz = make_float2(__uint_as_float(dzw[2 * i]), __uint_as_float(dzw[2 * i + 1]));
+            if (PT) dz = __fmul2_rn(dz, make_float2(alpha, alpha));
+            const float2 sg = sigmoid2(gg);                                  // sigmoid(G)
+            const float2 sl = __fmul2_rn(gg, sg);                            // silu(G)
+            const float2 da = __fmul2_rn(dz, p2);                            // dA = dZ * p
+            dprob2 = __ffma2_rn(__fmul2_rn(dz, sl), uu, dprob2);             // dprob += dZ * A
+            const float2 oms = __ffma2_rn(sg, make_float2(-1.f, -1.f), one2);  // 1 - s
+            const float2 dsl = __fmul2_rn(sg, __ffma2_rn(gg, oms, one2));     // silu'(G)
+            const float2 a = __fmul2_rn(__fmul2_rn(da, uu), dsl);
+            const float2 b = __fmul2_rn(da, sl);
+            vg[2 * i] = a.x;
+            vg[2 * i + 1] = a.y;
+            vu[2 * i] = b.x;
+            vu[2 * i + 1] = b.y;
           }
+          // dZ of the next chunk (spare columns 32 * c) comes out of TMEM while this one's
+          // quantisation and stores run
+          if (c < 3) ptx::tmem_ld_32x32b_x32(t_stash + 32 * c, dzw);
           const int64_t fg = f0 + 32 * c;
           if (ESZ == 2) {  // bf16 dG / dU: rows and transposed rows, no quantisation
             float wg[32], wu[32];
@@ -943,13 +976,8 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           g.dgu_colT_sf[sf_offset(MXMOE_SCALE_MMA, F2, g.rows_cap, fg + lane, mrow0 / 32)] = csg;
           g.dgu_colT_sf[sf_offset(MXMOE_SCALE_MMA, F2, g.rows_cap, F + fg + lane, mrow0 / 32)] = csu;
         };
-        chunk(0, dz0);
 #pragma unroll 1
-        for (int c = 1; c < 4; ++c) {
-          uint32_t dzw[32];
-          ptx::tmem_ld_32x32b_x32(t_stash + 32 * (c - 1), dzw);
-          chunk(c, dzw);
-        }
+        for (int c = 0; c < 4; ++c) chunk(c, dz);
         if (tm != 0.f) record_amax(g.out_amax_rec, gmax, lane);  // this tile's largest |dGU|
         // row scales: blocks f0/32 .. +3 (and their up-half twins) are one aligned word each
         if (ESZ == 1) {
@@ -957,7 +985,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           *reinterpret_cast<uint32_t*>(g.dgu_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F2, row, (F + f0) / 32)) =
               sfu;
         }
-        g.dprob_part[row * (F / 128) + t.n_tile * 2 + h] = dprob;
+        g.dprob_part[row * (F / 128) + t.n_tile * 2 + h] = dprob2.x + dprob2.y;
       }
     }
     // output boxes fully written before the CTA retires
