@@ -83,29 +83,48 @@ __device__ __forceinline__ void load_pair(const float* p, float& a, float& b) {
   b = w.y;
 }
 
+// Largest magnitudes of packed bf16 pairs: one bf16x2 max-of-magnitudes per pair of
+// words (the signs of partial results are meaningless and are cleared at the end); a
+// pairwise tree keeps the dependent chain short. A NaN gives the canonical NaN, whose
+// all-ones exponent yields the same block scale as any other NaN.
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+template <int N>
+__device__ __forceinline__ uint32_t bmax_tree(const uint32_t (&w)[N]) {
+  uint32_t t[N / 2];
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) t[i] = bmax2(w[2 * i], w[2 * i + 1]);
+#pragma unroll
+  for (int s = N / 4; s >= 1; s >>= 1)
+#pragma unroll
+    for (int i = 0; i < s; ++i) t[i] = bmax2(t[i], t[i + s]);
+  return t[0] & 0x7FFF7FFFu;
+}
 // MXFP8 of 32 bf16 values given as 16 packed words (element 2k in the low half of w[k],
-// 2k+1 in the high half). |bf16| bit patterns order like unsigned 16-bit integers, so
-// the block amax is a SIMD max over the masked words; the result equals the amax of the
-// values widened to fp32 (widening is exact), hence the same scale as quant_block32.
-// tm != 0: per-tensor FP8 under the multiplier tm (scale byte 127).
+// 2k+1 in the high half). The block amax of the bf16 values equals that of the values
+// widened to fp32 (widening is exact), hence the same scale as quant_block32; the scaled
+// values are formed two per instruction (packed fp32x2 multiply, each lane rounded as the
+// scalar multiply). tm != 0: per-tensor FP8 under the multiplier tm (scale byte 127).
 template <int FMT = MXMOE_FMT_E4M3>
 __device__ __forceinline__ uint8_t quant_block32_bf16(const uint32_t (&w)[16], uint32_t (&out)[8],
                                                       bool ceil_rule = false, float tm = 0.f) {
   int32_t X = 0;
   float s = tm;
   if (tm == 0.f) {
-    uint32_t m = 0;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+    const uint32_t m = bmax_tree(w);
     const uint32_t amax = max(m << 16, m & 0xFFFF0000u);
     X = mx_scale_exp_from_amax_bits<FMT>(amax, ceil_rule);
     s = mx_inv_scale(X);
   }
+  const float2 s2 = make_float2(s, s);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t lo = fp8x2<FMT>(bf16_lo(w[2 * i]) * s, bf16_hi(w[2 * i]) * s);
-    const uint32_t hi = fp8x2<FMT>(bf16_lo(w[2 * i + 1]) * s, bf16_hi(w[2 * i + 1]) * s);
-    out[i] = lo | (hi << 16);
+    const float2 a = __fmul2_rn(make_float2(bf16_lo(w[2 * i]), bf16_hi(w[2 * i])), s2);
+    const float2 c = __fmul2_rn(make_float2(bf16_lo(w[2 * i + 1]), bf16_hi(w[2 * i + 1])), s2);
+    out[i] = (uint32_t)fp8x2<FMT>(a.x, a.y) | ((uint32_t)fp8x2<FMT>(c.x, c.y) << 16);
   }
   return (uint8_t)(X + 127);
 }
@@ -119,20 +138,21 @@ __device__ __forceinline__ void quant_colpair_bf16(const uint32_t (&w)[32], uint
   int32_t X0 = 0, X1 = 0;
   float s0 = tm, s1 = tm;
   if (tm == 0.f) {
-    uint32_t m = 0;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+    const uint32_t m = bmax_tree(w);
     X0 = mx_scale_exp_from_amax_bits<FMT>(m << 16, ceil_rule);
     X1 = mx_scale_exp_from_amax_bits<FMT>(m & 0xFFFF0000u, ceil_rule);
     s0 = mx_inv_scale(X0);
     s1 = mx_inv_scale(X1);
   }
+  const float2 s02 = make_float2(s0, s0), s12 = make_float2(s1, s1);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    o0[i] = (uint32_t)fp8x2<FMT>(bf16_lo(w[4 * i]) * s0, bf16_lo(w[4 * i + 1]) * s0) |
-            ((uint32_t)fp8x2<FMT>(bf16_lo(w[4 * i + 2]) * s0, bf16_lo(w[4 * i + 3]) * s0) << 16);
-    o1[i] = (uint32_t)fp8x2<FMT>(bf16_hi(w[4 * i]) * s1, bf16_hi(w[4 * i + 1]) * s1) |
-            ((uint32_t)fp8x2<FMT>(bf16_hi(w[4 * i + 2]) * s1, bf16_hi(w[4 * i + 3]) * s1) << 16);
+    const float2 a0 = __fmul2_rn(make_float2(bf16_lo(w[4 * i]), bf16_lo(w[4 * i + 1])), s02);
+    const float2 b0 = __fmul2_rn(make_float2(bf16_lo(w[4 * i + 2]), bf16_lo(w[4 * i + 3])), s02);
+    const float2 a1 = __fmul2_rn(make_float2(bf16_hi(w[4 * i]), bf16_hi(w[4 * i + 1])), s12);
+    const float2 b1 = __fmul2_rn(make_float2(bf16_hi(w[4 * i + 2]), bf16_hi(w[4 * i + 3])), s12);
+    o0[i] = (uint32_t)fp8x2<FMT>(a0.x, a0.y) | ((uint32_t)fp8x2<FMT>(b0.x, b0.y) << 16);
+    o1[i] = (uint32_t)fp8x2<FMT>(a1.x, a1.y) | ((uint32_t)fp8x2<FMT>(b1.x, b1.y) << 16);
   }
   sb0 = (uint8_t)(X0 + 127);
   sb1 = (uint8_t)(X1 + 127);
