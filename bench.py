@@ -103,6 +103,17 @@ def load_traffic(kernel_key, paths, units):
 
 
 # ----------------------------------------------------------------------------- clocks
+def smi_id(dev_index):
+    """nvidia-smi's id of CUDA device `dev_index`: its UUID (nvidia-smi numbers every GPU of
+    the machine and ignores CUDA_VISIBLE_DEVICES, so an index could name another GPU)."""
+    try:
+        import torch
+        u = str(torch.cuda.get_device_properties(dev_index).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev_index)
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -111,7 +122,7 @@ class ClockSampler:
     _n = 0
 
     def __init__(self, gpu_index):
-        self.gpu = gpu_index
+        self.gpu = smi_id(gpu_index)
         self.proc = None
         ClockSampler._n += 1   # one file per sampler: several run in one process
         self.path = os.path.join("/tmp", f"mxmoe_clocks_{os.getpid()}_{ClockSampler._n}.csv")

@@ -266,8 +266,10 @@ mxmoe_status grouped_gemm_mxfp8(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, cons
  * detection; no counterpart in the pages). The same call as grouped_gemm_mxfp8, except
  * that the first CTA pair's MMA issuer withholds its first accumulator-ready signal: that
  * pair's epilogue warps wait for it until the wait limit (1 s) runs out, record
- * MXMOE_ERR_DEVICE_TIMEOUT in the device status word and stop; the pair's other roles stop
- * at their own limits, wait for their issued copies and MMAs, release TMEM and return. The
+ * MXMOE_ERR_DEVICE_TIMEOUT in the device status word and stop (the first wait of the pair
+ * to run out records its site: normally the epilogue's, possibly the scale-copy thread's,
+ * which stalls behind it); the pair's other roles stop at their own limits, wait for
+ * their issued copies, scale copies and MMAs, release TMEM and return. The
  * kernel ends (no hang, no trap) with C only partly written; the context stays usable.
  * Arguments, checks and errors as grouped_gemm_mxfp8. Never use it for results.
  */

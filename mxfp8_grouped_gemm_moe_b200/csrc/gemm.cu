@@ -29,7 +29,10 @@
 //    the tensor cores' scale order and are moved to TMEM with tcgen05.cp, and the MMA is
 //    kind::mxf8f6f4 with block-32 scales. bf16 operands (ESZ = 2, CTA pairs): kind::f16,
 //    no scales; the fused epilogues then write bf16 instead of MXFP8;
-//  * warp 0 issues the copies, warp 1 issues tcgen05.mma; the epilogue warps (2..9 for
+//  * warp 0 issues the operand copies, warp 1 issues tcgen05.mma, and for MXFP8 operands
+//    warp 2 moves each stage's scales into TMEM (tcgen05.cp issued by a thread other
+//    than the MMA issuer overlaps the MMAs in flight; from the MMA thread each stage's
+//    copies would wait behind the previous stage's MMAs); the epilogue warps (3..10 for
 //    plain stores and weight gradients, 4..11 for the fused modes, which run 12 warps
 //    with a register split) drain the accumulator from TMEM into registers (or spare
 //    TMEM columns), hand it back to the MMA warp at once, then run the epilogue math and
@@ -56,10 +59,10 @@ namespace mxmoe {
 
 constexpr int BN = 256;  // output tile columns (both variants)
 constexpr int BK = 128;  // K per pipeline stage
-// Warp roles: warp 0 TMA producer, warp 1 MMA issuer, then 8 epilogue warps.
-//  * plain-store / weight-gradient modes: 10 warps, epilogue warps 2..9, 168 registers
-//    per thread (the ptxas limit once three warps share a scheduler);
-//  * fused SwiGLU modes: 12 warps = 3 warpgroups, epilogue warps 4..11 (warps 2-3 idle).
+// Warp roles: warp 0 TMA producer, warp 1 MMA issuer, warp 2 scale copies (MXFP8
+// operands), then 8 epilogue warps.
+//  * plain-store / weight-gradient modes: 11 warps, epilogue warps 3..10;
+//  * fused SwiGLU modes: 12 warps = 3 warpgroups, epilogue warps 4..11 (warp 3 idle).
 //    The block launches with 168 registers per thread; warpgroup 0 then drops to
 //    kRegsCtl and the epilogue warpgroups rise to kRegsEpi, which together use exactly
 //    the launch allocation: 128 * kRegsCtl + 256 * kRegsEpi == 384 * kRegsLaunch.
@@ -74,8 +77,8 @@ constexpr uint32_t kSfaBytes = 512;     // 128 rows x 4 scale bytes
 constexpr uint32_t kSfbBytes = 1024;    // 256 rows x 4 scale bytes
 constexpr int kMaxE = 256;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemSfa = 256;    // two buffers of 4 columns
-constexpr uint32_t kTmemSfb = 264;    // two buffers of 8 columns
+constexpr uint32_t kTmemSfa = 256;    // one 4-column buffer per operand stage (up to 5)
+constexpr uint32_t kTmemSfb = 280;    // one 8-column buffer per operand stage (up to 5)
 constexpr uint32_t kTmemStash = 320;  // epilogue scratch: 96 columns per (lane quadrant, half)
 constexpr int kPrefetchSteps = 8;     // K steps of the next tile pulled into L2 at a tile start
 
@@ -88,8 +91,8 @@ template <int PAIR, int MODE>
 struct Cfg {
   static constexpr bool kTmaStore = MODE == kModeStore || MODE == kModeWgrad;
   static constexpr bool kSplitRegs = !kTmaStore;            // 12 warps with the register split
-  static constexpr int kThreads = kSplitRegs ? 384 : 320;
-  static constexpr int kEpiWarp0 = kSplitRegs ? 4 : 2;      // first epilogue warp
+  static constexpr int kThreads = kSplitRegs ? 384 : 352;
+  static constexpr int kEpiWarp0 = kSplitRegs ? 4 : 3;      // first epilogue warp
   static constexpr int TM = 128 * PAIR;                        // output tile rows
   static constexpr int STAGES = PAIR == 2 ? (kTmaStore ? 5 : 4) : 3;
   static constexpr uint32_t kBBytes = (BN / PAIR) * BK;        // this CTA's B rows per stage
@@ -104,6 +107,7 @@ struct Cfg {
   static constexpr int GROUP_M = 16 / PAIR;                    // M tiles per raster group (2048 rows)
   static constexpr int GROUP_W = 16 / PAIR;                    // wgrad N tiles per raster group
   static_assert(kStageBytes >= kTxBytes && kStageBytes % 1024 == 0, "stage layout");
+  static_assert(kTmemSfa + 4 * STAGES <= kTmemSfb && kTmemSfb + 8 * STAGES <= kTmemStash, "scale buffers in TMEM");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -390,19 +394,25 @@ __device__ __forceinline__ uint4 pack8_bf16(const uint32_t (&v)[N], int i0) {
 // unless a wait of this CTA ran out (s_abort). It is kept out of line and finds its state
 // in shared memory, so that the kernel's normal path keeps no extra values live.
 // The leader's producer thread waits (bounded) for the latest phase of every operand stage
-// it armed -- those phases also count the peer CTA's copies; the leader's MMA thread
-// commits once more and waits, so that every MMA it issued has completed; then one thread
+// it armed -- those phases also count the peer CTA's copies; the leader's MMA thread (and,
+// for MXFP8 operands, its scale-copy thread) commits once more and waits, so that every
+// MMA (and scale copy) it issued has completed; then one thread
 // per CTA lets 1 ms pass for copies that no barrier of its own tracks (a peer's, issued
 // ahead of the leader's producer). Nothing asynchronous is then in flight when TMEM is
 // released and the CTA retires.
-template <int PAIR, int STAGES, uint32_t kOffBars>
+template <int PAIR, int ESZ, int STAGES, uint32_t kOffBars>
 __device__ __noinline__ void abort_drain() {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + kOffBars);
   uint64_t* bar_drain = bar_full + 2 * STAGES + 2;
   const volatile int32_t* s_abort = reinterpret_cast<const volatile int32_t*>(bar_drain + 1) + 1;
-  const uint32_t n_issued = *reinterpret_cast<const volatile uint32_t*>(s_abort + 2);
+  const volatile uint32_t* s_issued = reinterpret_cast<const volatile uint32_t*>(s_abort + 2);
+  const uint32_t n_issued = *s_issued;
+  // the kernel's layout: full[S], empty[S], acc_full, acc_empty, drain, four 32-bit words, tma[S]
+  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(smem + kOffBars + 8 * (2 * STAGES + 3) + 16);
+  uint64_t* bar_sf_drain = bar_tma + STAGES;
+  uint64_t* bar_ld = ESZ == 1 ? bar_tma : bar_full;
   if (*s_abort == 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = PAIR == 2 ? ptx::cluster_rank() : 0u;
@@ -410,12 +420,16 @@ __device__ __noinline__ void abort_drain() {
     const uint32_t nlast = n_issued < (uint32_t)STAGES ? n_issued : (uint32_t)STAGES;
     for (uint32_t j = 1; j <= nlast; ++j) {
       const uint32_t i = n_issued - j;
-      ptx::mbar_wait(&bar_full[i % STAGES], (i / STAGES) & 1u, 5);
+      ptx::mbar_wait(&bar_ld[i % STAGES], (i / STAGES) & 1u, 5);
     }
   } else if (rank == 0 && lane == 0 && warp == 1) {
     if (PAIR == 1) ptx::tc_commit(bar_drain);
     else ptx::tc_commit_pair_mask(bar_drain, 0x1);
     ptx::mbar_wait(bar_drain, 0, 6);
+  } else if (ESZ == 1 && rank == 0 && lane == 0 && warp == 2) {
+    if (PAIR == 1) ptx::tc_commit(bar_sf_drain);
+    else ptx::tc_commit_pair_mask(bar_sf_drain, 0x1);
+    ptx::mbar_wait(bar_sf_drain, 0, 8);
   }
   if (threadIdx.x == 0) {
     const uint64_t t0 = ptx::globaltimer();
@@ -455,6 +469,12 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
   volatile int32_t* s_abort = reinterpret_cast<volatile int32_t*>(s_tmem + 1);
   int32_t* s_bad = const_cast<int32_t*>(s_abort + 1);
   uint32_t* s_issued = reinterpret_cast<uint32_t*>(s_bad + 1);  // operand stages the producer issued
+  // MXFP8 operands: the copies of a stage complete on bar_tma; the scale-copy thread then
+  // moves the stage's scales into TMEM and its commit completes bar_full for the MMAs
+  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(s_issued + 1);
+  uint64_t* bar_sf_drain = bar_tma + STAGES;  // abort path: completion of the issued scale copies
+  static_assert(8 * (3 * STAGES + 4) + 16 <= 256, "barrier block");
+  uint64_t* bar_ld = ESZ == 1 ? bar_tma : bar_full;  // where the operand copies complete
   int32_t* s_seg = reinterpret_cast<int32_t*>(smem + C::kOffSeg);
   int32_t* s_order = reinterpret_cast<int32_t*>(smem + C::kOffOrder);
 
@@ -467,10 +487,12 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
     for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(&bar_full[s], 1);
       ptx::mbar_init(&bar_empty[s], 1);
+      ptx::mbar_init(&bar_tma[s], 1);
     }
     ptx::mbar_init(bar_acc_full, 1);
     ptx::mbar_init(bar_acc_empty, kEpiWarps * PAIR);
     ptx::mbar_init(bar_drain, 1);
+    ptx::mbar_init(bar_sf_drain, 1);
     *s_abort = 0;
     *s_bad = 0;
     *s_issued = 0;
@@ -566,17 +588,17 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           const int64_t cb1 = cb0 + b_kchunks;
           uint8_t* s_sfa = sb + kABytes + kBBytes;
           if (PAIR == 1) {
-            ptx::mbar_arrive_expect_tx(&bar_full[stage], C::kTxBytes);
-            ptx::tma_load_2d(sb, &tmA, kx_a, t.a_y, &bar_full[stage]);
-            ptx::tma_load_2d(sb + kABytes, &tmB, kx_b, t.b_y0, &bar_full[stage]);
-            ptx::tma_load_2d(sb + kABytes + kBBytes / 2, &tmB, kx_b, t.b_y1, &bar_full[stage]);
-            ptx::bulk_load(s_sfa, g.a_sf + ca * 512, 512, &bar_full[stage]);
-            ptx::bulk_load(s_sfa + kSfaBytes, g.b_sf + cb0 * 512, 512, &bar_full[stage]);
-            ptx::bulk_load(s_sfa + kSfaBytes + 512, g.b_sf + cb1 * 512, 512, &bar_full[stage]);
+            ptx::mbar_arrive_expect_tx(&bar_ld[stage], C::kTxBytes);
+            ptx::tma_load_2d(sb, &tmA, kx_a, t.a_y, &bar_ld[stage]);
+            ptx::tma_load_2d(sb + kABytes, &tmB, kx_b, t.b_y0, &bar_ld[stage]);
+            ptx::tma_load_2d(sb + kABytes + kBBytes / 2, &tmB, kx_b, t.b_y1, &bar_ld[stage]);
+            ptx::bulk_load(s_sfa, g.a_sf + ca * 512, 512, &bar_ld[stage]);
+            ptx::bulk_load(s_sfa + kSfaBytes, g.b_sf + cb0 * 512, 512, &bar_ld[stage]);
+            ptx::bulk_load(s_sfa + kSfaBytes + 512, g.b_sf + cb1 * 512, 512, &bar_ld[stage]);
           } else {
             // both CTAs' copies complete on the leader's barrier, which expects the pair's bytes
-            const uint32_t full_leader = ptx::map_to_rank(ptx::smem_u32(&bar_full[stage]), 0);
-            if (rank == 0) ptx::mbar_arrive_expect_tx(&bar_full[stage], 2 * kTx);
+            const uint32_t full_leader = ptx::map_to_rank(ptx::smem_u32(&bar_ld[stage]), 0);
+            if (rank == 0) ptx::mbar_arrive_expect_tx(&bar_ld[stage], 2 * kTx);
             ptx::tma_load_2d_pair(sb, &tmA, kx_a, t.a_y, full_leader);
             ptx::tma_load_2d_pair(sb + kABytes, &tmB, kx_b, rank ? t.b_y1 : t.b_y0, full_leader);
             if (ESZ == 1) {
@@ -619,24 +641,9 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           }
           ptx::tc_fence_after();
           const uint32_t sbase = ptx::smem_u32(smem + stage * kStageBytes);
-          const uint32_t buf = (uint32_t)(stage & 1);
-          const uint32_t t_sfa = tmem_base + kTmemSfa + buf * 4;
-          const uint32_t t_sfb = tmem_base + kTmemSfb + buf * 8;
-          const uint32_t sfa_s = sbase + kABytes + kBBytes;
-          const uint64_t dsa = ptx::make_smem_desc(sfa_s, 0, 128, ptx::kLayoutSwizzleNone);
-          const uint64_t dsb0 = ptx::make_smem_desc(sfa_s + kSfaBytes, 0, 128, ptx::kLayoutSwizzleNone);
-          const uint64_t dsb1 = ptx::make_smem_desc(sfa_s + kSfaBytes + 512, 0, 128, ptx::kLayoutSwizzleNone);
-          if (ESZ == 1) {
-            if (PAIR == 1) {
-              ptx::tmem_cp_32x128b_warpx4(t_sfa, dsa);
-              ptx::tmem_cp_32x128b_warpx4(t_sfb, dsb0);
-              ptx::tmem_cp_32x128b_warpx4(t_sfb + 4, dsb1);
-            } else {
-              ptx::tmem_cp_pair_32x128b_warpx4(t_sfa, dsa);
-              ptx::tmem_cp_pair_32x128b_warpx4(t_sfb, dsb0);
-              ptx::tmem_cp_pair_32x128b_warpx4(t_sfb + 4, dsb1);
-            }
-          }
+          // this stage's scales, already in TMEM (the scale-copy thread's commit completed bar_full)
+          const uint32_t t_sfa = tmem_base + kTmemSfa + (uint32_t)stage * 4;
+          const uint32_t t_sfb = tmem_base + kTmemSfb + (uint32_t)stage * 8;
           const uint64_t adesc = ptx::make_smem_desc(sbase, 16, 1024, ptx::kLayoutSwizzle128B);
           const uint64_t bdesc = ptx::make_smem_desc(sbase + kABytes, 16, 1024, ptx::kLayoutSwizzle128B);
 #pragma unroll
@@ -674,6 +681,54 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           ptx::tc_commit_pair(bar_acc_full);
         }
         acc_ph ^= 1u;
+      }
+    }
+   } else if (warp == 2 && ESZ == 1) {
+    // ===================================================== scale copies (leader CTA)
+    // Moves each stage's E8M0 scales from shared memory into that stage's TMEM scale
+    // buffer once its operand copies have landed, and completes the stage for the MMA
+    // issuer with a commit. Issued from this thread, the copies overlap the MMAs already
+    // in flight; issued from the MMA thread, each stage's copies would sit between its
+    // MMAs and the previous stage's. A stage's buffer is rewritten only after its MMAs
+    // completed (the producer re-arms the stage once they have).
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      for (int32_t tile = first; tile < ntiles && !*s_abort; tile += stride) {
+        const TileInfo t = get_tile<MODE, PAIR, ESZ>(g, tile, s_seg, s_order, 0);
+        bool ok = true;
+        for (int kb = 0; kb < t.k_iters; ++kb) {
+          if (!ptx::mbar_wait(&bar_tma[stage], ph, 7)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sfa_s = ptx::smem_u32(smem + stage * kStageBytes) + kABytes + kBBytes;
+          const uint64_t dsa = ptx::make_smem_desc(sfa_s, 0, 128, ptx::kLayoutSwizzleNone);
+          const uint64_t dsb0 = ptx::make_smem_desc(sfa_s + kSfaBytes, 0, 128, ptx::kLayoutSwizzleNone);
+          const uint64_t dsb1 = ptx::make_smem_desc(sfa_s + kSfaBytes + 512, 0, 128, ptx::kLayoutSwizzleNone);
+          const uint32_t t_sfa = tmem_base + kTmemSfa + (uint32_t)stage * 4;
+          const uint32_t t_sfb = tmem_base + kTmemSfb + (uint32_t)stage * 8;
+          if (PAIR == 1) {
+            ptx::tmem_cp_32x128b_warpx4(t_sfa, dsa);
+            ptx::tmem_cp_32x128b_warpx4(t_sfb, dsb0);
+            ptx::tmem_cp_32x128b_warpx4(t_sfb + 4, dsb1);
+            ptx::tc_commit(&bar_full[stage]);
+          } else {
+            ptx::tmem_cp_pair_32x128b_warpx4(t_sfa, dsa);
+            ptx::tmem_cp_pair_32x128b_warpx4(t_sfb, dsb0);
+            ptx::tmem_cp_pair_32x128b_warpx4(t_sfb + 4, dsb1);
+            ptx::tc_commit_pair_mask(&bar_full[stage], 0x1);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) {
+          *s_abort = 1;
+          break;
+        }
       }
     }
    }
@@ -1000,7 +1055,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
   // TMEM is released or the CTA retires (abort_drain).
   ptx::tc_fence_before();
   __syncthreads();
-  abort_drain<PAIR, STAGES, C::kOffBars>();
+  abort_drain<PAIR, ESZ, STAGES, C::kOffBars>();
   __syncthreads();
   if (PAIR == 2) ptx::cluster_sync();
   if (warp == 1) {

@@ -19,7 +19,7 @@ from tests.util import f64, rel_l2
 
 pytestmark = pytest.mark.gpu
 TOL_GEMM = 5e-3
-WAIT_SITES = {1, 2, 3, 4}   # producer, MMA (accumulator / operands), epilogue
+WAIT_SITES = {1, 2, 3, 4, 7}   # producer, MMA (accumulator / operands), epilogue, scale copies
 
 
 @pytest.fixture(params=["pair", "single"])
