@@ -1,4 +1,6 @@
-"""Builds libmxmoe.so in-tree with nvcc for sm_100a (B200)."""
+"""Builds libmxmoe.so in-tree with nvcc for sm_100a (B200), and on request the checked
+build libmxmoe_checks.so (-DMXMOE_CHECKS=1: device-side bounds checks that record
+MXMOE_ERR_DEVICE_CHECK and skip the access; same API, slower, for tests)."""
 from __future__ import annotations
 
 import glob
@@ -9,6 +11,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmxmoe.so")
+LIB_CHECKS = os.path.join(HERE, "libmxmoe_checks.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 NVCC_FLAGS = [
@@ -24,10 +27,10 @@ def sources():
                   + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def needs_build():
-    if not os.path.exists(LIB):
+def needs_build(lib=LIB):
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(s) > t for s in sources())
 
 
@@ -38,22 +41,23 @@ def nvcc():
     return "nvcc"
 
 
-def build(force=False, verbose=False, ptxas_v=False):
-    if not force and not needs_build():
-        return LIB
-    cmd = [nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if ptxas_v else []) + [
-        "-o", LIB + ".tmp", os.path.join(CSRC, "mxmoe_unity.cu")]
+def build(force=False, verbose=False, ptxas_v=False, checks=False):
+    lib = LIB_CHECKS if checks else LIB
+    if not force and not needs_build(lib):
+        return lib
+    cmd = [nvcc()] + NVCC_FLAGS + (["-DMXMOE_CHECKS=1"] if checks else []) + (
+        ["-Xptxas", "-v"] if ptxas_v else []) + ["-o", lib + ".tmp", os.path.join(CSRC, "mxmoe_unity.cu")]
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("nvcc failed building libmxmoe.so")
+        raise RuntimeError(f"nvcc failed building {os.path.basename(lib)}")
     if verbose or ptxas_v:
         sys.stderr.write(r.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True, ptxas_v="--ptxas-v" in sys.argv)
+    build(force="--force" in sys.argv, verbose=True, ptxas_v="--ptxas-v" in sys.argv, checks="--checks" in sys.argv)

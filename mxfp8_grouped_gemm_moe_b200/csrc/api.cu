@@ -24,7 +24,6 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 inline mxmoe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MXMOE_OK : MXMOE_ERR_CUDA; }
 
-int64_t rows_cap(int64_t T, int64_t k, int64_t E) { return (T * k + 255 * E + 255) / 256 * 256; }
 
 // Sub-buffers of a caller-provided byte buffer, each 256-byte aligned.
 struct Carver {

@@ -752,9 +752,12 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
       const int64_t mrow0 = t.row0 + 32 * q;  // first row of this warp's 32-row block
       const int64_t row = mrow0 + lane;
       const bool have_acc = t.k_iters > 0;
+      // the row of G / U this lane reads in the backward epilogue (row 0 if the checked
+      // build finds it outside the buffer)
+      const int64_t gu_row = MODE == kModeSwigluBwd && !check_index(row, g.rows_cap, 63) ? 0 : row;
       if (MODE == kModeSwigluBwd) {
         // pull this row's G and U slices (2 x 256 B) into L2 while the MMAs run
-        const uint16_t* gp = g.gu_in + row * (2 * g.F) + (int64_t)t.n_tile * BN + 128 * h;
+        const uint16_t* gp = g.gu_in + gu_row * (2 * g.F) + (int64_t)t.n_tile * BN + 128 * h;
         ptx::prefetch_l2(gp);
         ptx::prefetch_l2(gp + 64);
         ptx::prefetch_l2(gp + g.F);
@@ -812,7 +815,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
         }
       } else if (MODE == kModeSwigluFwd) {
         const int64_t F = g.F;
-        const float p = g.prob_of_row[row];
+        const float p = check_index(row, g.rows_cap, 60) ? g.prob_of_row[row] : 0.f;
         const int64_t f0 = (int64_t)t.n_tile * 128 + 64 * h;  // this warp's 64 Z columns
         // drain gate / up (TMEM columns [128h, +64) and [128h + 64, +64), the interleaved
         // operand order) into registers and hand the accumulator back at once; then save G
@@ -905,14 +908,19 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           ptx::tma_store_2d(&tmD, stg8 + 3072, (int32_t)mrow0, (int32_t)(f0 + 32));
           ptx::bulk_commit_group();
         }
-        g.z_colT_sf[sf_offset(MXMOE_SCALE_MMA, F, g.rows_cap, f0 + lane, mrow0 / 32)] = cs0;
-        g.z_colT_sf[sf_offset(MXMOE_SCALE_MMA, F, g.rows_cap, f0 + 32 + lane, mrow0 / 32)] = cs1;
-        // row scales of the blocks [f0, f0 + 64): adjacent bytes (block index 2h, 2h + 1 mod 4)
-        *reinterpret_cast<uint16_t*>(g.z_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F, row, f0 / 32)) =
-            (uint16_t)zsf;
+        {
+          const int64_t n_sf = F * g.rows_cap / 32;  // bytes of each scale array of Z
+          const int64_t o0 = sf_offset(MXMOE_SCALE_MMA, F, g.rows_cap, f0 + lane, mrow0 / 32);
+          const int64_t o1 = sf_offset(MXMOE_SCALE_MMA, F, g.rows_cap, f0 + 32 + lane, mrow0 / 32);
+          if (check_index(o0, n_sf, 61)) g.z_colT_sf[o0] = cs0;
+          if (check_index(o1, n_sf, 61)) g.z_colT_sf[o1] = cs1;
+          // row scales of the blocks [f0, f0 + 64): adjacent bytes (block index 2h, 2h + 1 mod 4)
+          const int64_t orow = sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F, row, f0 / 32);
+          if (check_index(orow + 1, n_sf, 62)) *reinterpret_cast<uint16_t*>(g.z_row_sf + orow) = (uint16_t)zsf;
+        }
       } else if (MODE == kModeSwigluBwd) {
         const int64_t F = g.F, F2 = 2 * g.F;
-        const float p = g.prob_of_row[row];
+        const float p = check_index(row, g.rows_cap, 60) ? g.prob_of_row[row] : 0.f;
         const int64_t f0 = (int64_t)t.n_tile * BN + 128 * h;  // this warp's 128 dZ columns
         // phase 1: drain dZ (fp32) into registers and hand the accumulator back at once;
         // the first 32 columns stay in registers, the other 96 are parked, still fp32, in
@@ -934,8 +942,8 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
         }
         // phase 2: SwiGLU / probability backward, 32 columns at a time; G and U (pulled into
         // L2 when the tile started) of the next chunk are fetched while this one is processed
-        const uint4* gsrc = reinterpret_cast<const uint4*>(g.gu_in + row * F2 + f0);
-        const uint4* usrc = reinterpret_cast<const uint4*>(g.gu_in + row * F2 + F + f0);
+        const uint4* gsrc = reinterpret_cast<const uint4*>(g.gu_in + gu_row * F2 + f0);
+        const uint4* usrc = reinterpret_cast<const uint4*>(g.gu_in + gu_row * F2 + F + f0);
         uint4 gq[4], uq[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -1028,19 +1036,26 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
             ptx::tma_store_2d(&tmD, stg8 + 3072, (int32_t)mrow0, (int32_t)(F + fg));
             ptx::bulk_commit_group();
           }
-          g.dgu_colT_sf[sf_offset(MXMOE_SCALE_MMA, F2, g.rows_cap, fg + lane, mrow0 / 32)] = csg;
-          g.dgu_colT_sf[sf_offset(MXMOE_SCALE_MMA, F2, g.rows_cap, F + fg + lane, mrow0 / 32)] = csu;
+          const int64_t n_sf = F2 * g.rows_cap / 32;  // bytes of each scale array of dGU
+          const int64_t og = sf_offset(MXMOE_SCALE_MMA, F2, g.rows_cap, fg + lane, mrow0 / 32);
+          const int64_t ou = sf_offset(MXMOE_SCALE_MMA, F2, g.rows_cap, F + fg + lane, mrow0 / 32);
+          if (check_index(og, n_sf, 64)) g.dgu_colT_sf[og] = csg;
+          if (check_index(ou, n_sf, 64)) g.dgu_colT_sf[ou] = csu;
         };
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) chunk(c, dz);
         if (tm != 0.f) record_amax(g.out_amax_rec, gmax, lane);  // this tile's largest |dGU|
         // row scales: blocks f0/32 .. +3 (and their up-half twins) are one aligned word each
         if (ESZ == 1) {
-          *reinterpret_cast<uint32_t*>(g.dgu_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F2, row, f0 / 32)) = sfg;
-          *reinterpret_cast<uint32_t*>(g.dgu_row_sf + sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F2, row, (F + f0) / 32)) =
-              sfu;
+          const int64_t n_sf = F2 * g.rows_cap / 32;
+          const int64_t og = sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F2, row, f0 / 32);
+          const int64_t ou = sf_offset(MXMOE_SCALE_MMA, g.rows_cap, F2, row, (F + f0) / 32);
+          if (check_index(og + 3, n_sf, 65)) *reinterpret_cast<uint32_t*>(g.dgu_row_sf + og) = sfg;
+          if (check_index(ou + 3, n_sf, 65)) *reinterpret_cast<uint32_t*>(g.dgu_row_sf + ou) = sfu;
         }
-        g.dprob_part[row * (F / 128) + t.n_tile * 2 + h] = dprob2.x + dprob2.y;
+        const int64_t od = row * (F / 128) + t.n_tile * 2 + h;
+        if (check_index(od, (g.rows_cap * (F / 128)) >> (g.debug_check_shrink ? 1 : 0), 66))
+          g.dprob_part[od] = dprob2.x + dprob2.y;
       }
     }
     // output boxes fully written before the CTA retires
@@ -1265,7 +1280,14 @@ static cudaError_t launch_bf16(const GemmArgs& g, cudaStream_t st) {
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st) {
+cudaError_t launch_gemm(const GemmArgs& g0, cudaStream_t st) {
+  GemmArgs g = g0;
+#if MXMOE_CHECKS
+  // checked build: MXMOE_CHECKS_TRIP=1 makes the dprob bounds checks use half the real
+  // extent, so that valid writes are flagged and skipped (exercises the check path)
+  static const bool trip = std::getenv("MXMOE_CHECKS_TRIP") != nullptr;
+  g.debug_check_shrink = trip ? 1 : 0;
+#endif
   if (g.bf16_operands) return launch_bf16(g, st);
   if (g.a_amax)  // per-tensor FP8 operands
     return gemm_tile_rows() == 128 ? launch_variant<1, true>(g, st) : launch_variant<2, true>(g, st);

@@ -24,6 +24,28 @@ __device__ __forceinline__ void record_error(int32_t code, int32_t where) {
 }
 __device__ __forceinline__ void record_timeout(int32_t where) { record_error(MXMOE_ERR_DEVICE_TIMEOUT, where); }
 
+// Bounds checks of the checked build (compiled with -DMXMOE_CHECKS=1 into
+// libmxmoe_checks.so): an index computed from device data (segment offsets, gathers,
+// routing counts) that falls outside [0, n) records MXMOE_ERR_DEVICE_CHECK with the site's
+// tag (60..69) and the caller skips the access -- no trap, no out-of-bounds access. The
+// release build compiles every check to `true`.
+#ifndef MXMOE_CHECKS
+#define MXMOE_CHECKS 0
+#endif
+__device__ __forceinline__ bool check_index(int64_t i, int64_t n, int32_t site) {
+#if MXMOE_CHECKS
+  if (i < 0 || i >= n) {
+    record_error(MXMOE_ERR_DEVICE_CHECK, site);
+    return false;
+  }
+#else
+  (void)i;
+  (void)n;
+  (void)site;
+#endif
+  return true;
+}
+
 // ----------------------------------------------------------------------------- quantiser
 // Scale exponent X = clamp(floor(log2(amax)) - emax, -127, 127) from the bit pattern of a
 // non-negative fp32 amax (emax = 8 for E4M3 elements, 15 for E5M2); zero or subnormal

@@ -13,6 +13,10 @@ namespace mxmoe {
 // Kernels launched by this library since load (reported by mxmoe_launch_count).
 inline std::atomic<int64_t> g_launch_count{0};
 
+// Rows of the permuted buffers (live + pad) for T tokens, top-k, E experts:
+// roundup(T*k + 255*E, 256) -- every expert segment starts on a 256-row boundary.
+inline int64_t rows_cap(int64_t T, int64_t k, int64_t E) { return (T * k + 255 * E + 255) / 256 * 256; }
+
 // ---------------------------------------------------------------- routing / combine
 size_t route_workspace_bytes(int T, int k, int E);
 cudaError_t launch_route(const int32_t* idx, const float* probs, int T, int k, int E, int32_t* m_splits,
@@ -122,6 +126,9 @@ struct GemmArgs {
   // that the epilogue's bounded wait expires (tests the timeout path; never set in
   // normal use)
   int32_t debug_drop_commit;
+  // checked build only: if non-zero, the bounds checks of the dprob partials use half the
+  // real extent, so that valid writes are flagged and skipped (tests the check path)
+  int32_t debug_check_shrink;
 };
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t st);
 int gemm_num_sms();

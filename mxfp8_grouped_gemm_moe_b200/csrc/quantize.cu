@@ -229,6 +229,8 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
       const int64_t orow = r0 + row_t + k * RSTEP;
       srow[k] = -1;
       if (orow < nvalid && col < a.cols) srow[k] = a.gather ? (int64_t)__ldg(a.gather + orow) : b * a.rows + orow;
+      // checked build: a gathered row outside the source matrix reads as a zero row
+      if (a.gather && srow[k] >= 0 && !check_index(srow[k], a.rows, 67)) srow[k] = -1;
     }
     uint4 buf[NL];
 #pragma unroll

@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
 __global__ void __launch_bounds__(kRouteTokensPerBlock) route_scatter_kernel(
     const int32_t* __restrict__ idx, const float* __restrict__ probs, int T, int k, int E,
     const int32_t* __restrict__ block_base, int32_t* __restrict__ row_of_slot, int32_t* __restrict__ token_of_row,
-    float* __restrict__ prob_of_row) {
+    float* __restrict__ prob_of_row, int64_t cap) {
   constexpr int W = kRouteTokensPerBlock / 32;
   __shared__ uint32_t mask[kMaxExperts * W];
   for (int i = threadIdx.x; i < E * W; i += blockDim.x) mask[i] = 0u;
@@ -126,7 +126,9 @@ __global__ void __launch_bounds__(kRouteTokensPerBlock) route_scatter_kernel(
       int32_t rank = __popc(mask[e * W + w] & ((1u << lane) - 1u));
       for (int ww = 0; ww < w; ++ww) rank += __popc(mask[e * W + ww]);
       const int32_t row = block_base[(int64_t)blockIdx.x * E + e] + rank;
-      row_of_slot[(int64_t)t * k + j] = row;
+      const bool in = check_index(row, cap, 68);  // checked build: inside the row buffers
+      row_of_slot[(int64_t)t * k + j] = in ? row : -1;
+      if (!in) continue;
       token_of_row[row] = t;
       if (prob_of_row) prob_of_row[row] = probs[(int64_t)t * k + j];
     }
@@ -191,7 +193,7 @@ cudaError_t launch_route(const int32_t* idx, const float* probs, int T, int k, i
   route_scan_kernel<<<1, 1024, 0, st>>>(counts, nbl, E, base, m_splits, seg_off, token_of_row, prob_of_row);
   if (nb > 0)
     route_scatter_kernel<<<nb, kRouteTokensPerBlock, 0, st>>>(idx, probs, T, k, E, base, row_of_slot, token_of_row,
-                                                              prob_of_row);
+                                                              prob_of_row, rows_cap(T, k, E));
   g_launch_count += (nb > 0) ? 3 : 1;
   return cudaGetLastError();
 }

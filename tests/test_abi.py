@@ -40,6 +40,16 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n), n
 
 
+def test_checked_build_exports_the_same_symbols(lib):
+    """The bounds-checked build (libmxmoe_checks.so, built by __graft_entry__.build()) is
+    the same C ABI: every declared entry point is exported."""
+    from mxfp8_grouped_gemm_moe_b200 import build as b
+    assert os.path.exists(b.LIB_CHECKS)
+    checked = ctypes.CDLL(b.LIB_CHECKS)
+    for n in _declared_functions():
+        assert hasattr(checked, n), n
+
+
 def test_binding_signatures_cover_header(lib):
     import mxfp8_grouped_gemm_moe_b200 as mx
     assert set(_declared_functions()) == set(mx._SIGNATURES)
