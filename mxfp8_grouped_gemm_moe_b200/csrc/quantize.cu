@@ -206,9 +206,21 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
   const int64_t c0 = (int64_t)blockIdx.x * kQTile;
   const int64_t r0 = (int64_t)blockIdx.y * kQTile;
   const int64_t b = blockIdx.z;
+  constexpr int VPR = kQTile / Tr::kVec;        // vectors per tile row
+  constexpr int NL = kQTile * VPR / kQThreads;  // vectors per thread
+  constexpr int RSTEP = kQThreads / VPR;        // tile rows between a thread's vectors
+  const int row_t = threadIdx.x / VPR, cv = threadIdx.x % VPR;
+  // the valid-row count and this thread's gather indices are read together: the index
+  // array holds out_rows entries, so reading them before the count is known stays in bounds
+  int32_t gidx[NL];
+#pragma unroll
+  for (int k = 0; k < NL; ++k) {
+    const int64_t orow = r0 + row_t + k * RSTEP;
+    gidx[k] = (a.gather && orow < a.out_rows) ? __ldg(a.gather + orow) : -1;
+  }
   int64_t nvalid = a.out_rows;
   if (a.nrows) {
-    const int64_t nv = *a.nrows;
+    const int64_t nv = __ldg(a.nrows);
     nvalid = nv < nvalid ? nv : nvalid;
   }
   if (r0 >= nvalid) return;
@@ -216,11 +228,7 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
   const float tm = a.tensor_amax ? tensor_multiplier(a.tensor_amax[a.tensor_per_batch ? b : 0]) : 0.f;
 
   // ---- load the tile (gathered rows, zero outside the matrix / for pad rows); all of a
-  // thread's row indices, then all of its 16-byte loads, are issued before any use
-  constexpr int VPR = kQTile / Tr::kVec;        // vectors per tile row
-  constexpr int NL = kQTile * VPR / kQThreads;  // vectors per thread
-  constexpr int RSTEP = kQThreads / VPR;        // tile rows between a thread's vectors
-  const int row_t = threadIdx.x / VPR, cv = threadIdx.x % VPR;
+  // thread's 16-byte loads are issued before any use
   {
     const int64_t col = c0 + (int64_t)cv * Tr::kVec;
     int64_t srow[NL];
@@ -228,7 +236,7 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
     for (int k = 0; k < NL; ++k) {
       const int64_t orow = r0 + row_t + k * RSTEP;
       srow[k] = -1;
-      if (orow < nvalid && col < a.cols) srow[k] = a.gather ? (int64_t)__ldg(a.gather + orow) : b * a.rows + orow;
+      if (orow < nvalid && col < a.cols) srow[k] = a.gather ? (int64_t)gidx[k] : b * a.rows + orow;
       // checked build: a gathered row outside the source matrix reads as a zero row
       if (a.gather && srow[k] >= 0 && !check_index(srow[k], a.rows, 67)) srow[k] = -1;
     }
