@@ -228,6 +228,20 @@ mxmoe_status moe_unpermute(const void* y_perm_dev, const int32_t* row_of_slot_de
 mxmoe_status mxfp8_quantize(const void* src_dev, int32_t src_dtype, int64_t batch, int64_t rows, int64_t cols,
                             const int32_t* row_gather_dev, const int32_t* nrows_dev, int64_t out_rows,
                             const mxmoe_mxfp8* out_row, const mxmoe_mxfp8* out_colT, void* stream);
+/*
+ * mxfp8_dequantize -- the inverse of the rowwise quantisation, for MXFP8 rows that travel
+ * between devices (expert parallelism sends the routed rows as codes + scales): every
+ * element becomes element(code) * 2^(scale - 127), rounded once to bf16 (exact whenever
+ * the block's scale is at least 2^-124, i.e. for every block quantised from bf16 values
+ * of magnitude above about 2^-115).
+ *   src_row  rowwise MXFP8 [rows, cols], MXMOE_SCALE_PLAIN scales; cols % 32 == 0;
+ *            either element format.
+ *   dst_dev  bf16 [rows, cols], 16-byte aligned.
+ * Errors: MXMOE_ERR_INVALID_ARG for a null / unaligned pointer or an MMA scale layout,
+ * MXMOE_ERR_UNSUPPORTED_SHAPE for cols % 32 != 0.
+ */
+mxmoe_status mxfp8_dequantize(const mxmoe_mxfp8* src_row, void* dst_dev, void* stream);
+
 /* mxfp8_quantize with the scale rule chosen (MXMOE_SCALE_RULE_OCP, the rule above, or
  * MXMOE_SCALE_RULE_CEIL: the OCP exponent plus one for the blocks whose amax lies above
  * the format's largest value times the OCP scale, so that no element saturates). Any

@@ -69,6 +69,7 @@ _SIGNATURES = {
     "moe_router_topk_bwd": (_I32, [_P, _P, _P, _I32, _I32, _I32, _P, _P]),
     "mxfp8_quantize": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _I64, _PMX, _PMX, _P]),
     "mxfp8_quantize_ex": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _I64, _PMX, _PMX, _I32, _P]),
+    "mxfp8_dequantize": (_I32, [_PMX, _P, _P]),
     "grouped_gemm_mxfp8": (_I32, [_PMX, _PMX, _P, _I32, _I64, _I64, _P, _I32, _I64, _P]),
     "grouped_gemm_mxfp8_debug_timeout": (_I32, [_PMX, _PMX, _P, _I32, _I64, _I64, _P, _I32, _I64, _P]),
     "grouped_gemm_mxfp8_wgrad": (_I32, [_PMX, _PMX, _P, _I32, _P, _P]),
@@ -274,6 +275,14 @@ def mxfp8_quantize(src, rowwise=True, colwise=True, layout=SCALE_MMA, row_gather
                                    scale_rule, _stream())
         _check("mxfp8_quantize_ex", st)
     return r, c
+
+
+def mxfp8_dequantize(m: MXFP8, out=None):
+    """Rowwise MXFP8 with plain scales -> bf16 [rows, cols] (the library's kernel)."""
+    lib = load()
+    y = out if out is not None else torch.empty((m.rows, m.cols), dtype=torch.bfloat16, device=m.data.device)
+    _check("mxfp8_dequantize", lib.mxfp8_dequantize(ctypes.byref(m.as_struct()), _ptr(y), _stream()))
+    return y
 
 
 def grouped_gemm_mxfp8(A: MXFP8, B: MXFP8, seg_off, E, N, out_dtype=torch.bfloat16, out=None):

@@ -378,6 +378,15 @@ mxmoe_status mxfp8_quantize_ex(const void* src_dev, int32_t src_dtype, int64_t b
                        scale_rule, stream);
 }
 
+mxmoe_status mxfp8_dequantize(const mxmoe_mxfp8* src_row, void* dst_dev, void* stream) {
+  if (!src_row || !valid_mx(src_row) || !dst_dev || !aligned16(dst_dev)) return MXMOE_ERR_INVALID_ARG;
+  if (src_row->scale_layout != MXMOE_SCALE_PLAIN) return MXMOE_ERR_INVALID_ARG;
+  if (src_row->rows < 0 || src_row->cols <= 0 || src_row->cols % 32 != 0) return MXMOE_ERR_UNSUPPORTED_SHAPE;
+  if (src_row->rows == 0) return MXMOE_OK;
+  return cuda_status(launch_dequantize_rows(src_row->data, src_row->scale, src_row->rows, src_row->cols,
+                                            src_row->elem_format, dst_dev, S(stream)));
+}
+
 static mxmoe_status grouped_gemm_impl(const mxmoe_mxfp8* A, const mxmoe_mxfp8* B, const int32_t* seg_off_dev,
                                       int32_t E, int64_t N, int64_t K, void* C_dev, int32_t c_dtype, int64_t ldc,
                                       int32_t debug_drop_commit, void* stream, const float* a_amax = nullptr,

@@ -60,6 +60,9 @@ struct QuantArgs {
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
 // Largest magnitude of each of `groups` consecutive bf16 arrays of n elements
 // (n % 8 == 0, 16-byte aligned) into out[groups] (fp32; cleared first).
+// Rowwise MXFP8 with plain scales [rows, cols/32] -> bf16 [rows, cols] (cols % 32 == 0).
+cudaError_t launch_dequantize_rows(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols, int fmt,
+                                   void* out, cudaStream_t st);
 cudaError_t launch_amax_bf16(const void* src, int64_t n, int32_t groups, float* out, cudaStream_t st);
 // bf16 -> bf16 copies with the same row gather / valid-row count / gate-up interleave as
 // launch_quantize: row_data receives the (permuted) rows, col_data the transposed matrix

@@ -608,6 +608,50 @@ static cudaError_t launch_q(const QuantArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// ----------------------------------------------------------------------------- dequantisation
+// Rowwise MXFP8 (plain scale layout) -> bf16: value = element(code) * 2^(scale - 127). Each
+// thread turns 16 codes (one 16-byte load, within one 32-element block) into 16 bf16. The
+// codes decode exactly to fp16 (E4M3 and E5M2 are subsets of it), the power-of-two scaling
+// is exact in fp32, and the product rounds once to bf16 -- exact for every block whose
+// scale is at least 2^-124 (smaller scales can give values below bf16's subnormal step).
+template <int FMT>
+__global__ void __launch_bounds__(256) mxfp8_dequant_rows_kernel(const uint4* __restrict__ codes,
+                                                                 const uint8_t* __restrict__ scales, int64_t n16,
+                                                                 uint4* __restrict__ out) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n16) return;
+  const uint4 c = __ldg(codes + i);
+  const uint32_t sb = __ldg(scales + (i >> 1));
+  const float s = __uint_as_float(sb ? sb << 23 : 0x00400000u);  // 2^(byte - 127) (byte 0: the subnormal 2^-127)
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] >> (16 * hh)),
+                                                        FMT == MXMOE_FMT_E4M3 ? __NV_E4M3 : __NV_E5M2);
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+      o[2 * k + hh] = pack_bf16x2(f.x * s, f.y * s);
+    }
+  }
+  out[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+  out[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+cudaError_t launch_dequantize_rows(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols, int fmt,
+                                   void* out, cudaStream_t st) {
+  const int64_t n16 = rows * cols / 16;
+  if (n16 == 0) return cudaSuccess;
+  const int64_t blocks = (n16 + 255) / 256;
+  const uint4* c = reinterpret_cast<const uint4*>(codes);
+  uint4* o = reinterpret_cast<uint4*>(out);
+  if (fmt == MXMOE_FMT_E5M2) mxfp8_dequant_rows_kernel<MXMOE_FMT_E5M2><<<(unsigned)blocks, 256, 0, st>>>(c, scales, n16, o);
+  else mxfp8_dequant_rows_kernel<MXMOE_FMT_E4M3><<<(unsigned)blocks, 256, 0, st>>>(c, scales, n16, o);
+  ++g_launch_count;
+  return cudaGetLastError();
+}
+
 // ----------------------------------------------------------------------------- per-tensor amax
 // Largest magnitude of each group (blockIdx.y) of a bf16 array: a grid-stride pass of
 // 16-byte loads per group, a SIMD max over the magnitude bits (|bf16| patterns order like

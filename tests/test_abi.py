@@ -124,6 +124,12 @@ def test_host_argument_errors_enqueue_nothing(lib):
     assert lib.mxfp8_quantize(fake, 0, 1, 64, 64, None, None, 64, None, None, S) == 1
     m_bad_layout = mx._MX(1 << 20, 1 << 20, 64, 64, 1, 0)   # MMA layout needs multiples of 128
     assert lib.mxfp8_quantize(fake, 0, 1, 64, 64, None, None, 64, ctypes.byref(m_bad_layout), None, S) == 2
+    # dequantise: MMA scale layout, null destination, cols not a multiple of 32; 0 rows is a no-op
+    dq = mx._MX(1 << 20, 1 << 20, 64, 64, 0, 0)
+    assert lib.mxfp8_dequantize(ctypes.byref(mx._MX(1 << 20, 1 << 20, 128, 128, 1, 0)), fake, S) == 1
+    assert lib.mxfp8_dequantize(ctypes.byref(dq), None, S) == 1
+    assert lib.mxfp8_dequantize(ctypes.byref(mx._MX(1 << 20, 1 << 20, 64, 48, 0, 0)), fake, S) == 2
+    assert lib.mxfp8_dequantize(ctypes.byref(mx._MX(1 << 20, 1 << 20, 0, 64, 0, 0)), fake, S) == 0
     # grouped GEMM: N not a multiple of 128; A not in MMA layout
     A = mx._MX(1 << 20, 1 << 20, 256, 256, 1, 0)
     B = mx._MX(1 << 20, 1 << 20, 2 * 192, 256, 1, 0)

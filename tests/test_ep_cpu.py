@@ -65,6 +65,20 @@ class _OracleLocal:
                 torch.from_numpy(g["dprobs"]))
 
 
+class _OracleCodec:
+    """The MXFP8 wire through the oracle's rowwise quantiser and dequantiser."""
+
+    def encode(self, x, idx):
+        from oracle import mxfp8 as omx
+        q, sc = omx.quantize_rowwise(x[idx].double().numpy())
+        return torch.from_numpy(np.ascontiguousarray(q, dtype=np.uint8)), \
+            torch.from_numpy(np.ascontiguousarray(sc, dtype=np.uint8))
+
+    def decode(self, codes, scales):
+        from oracle import mxfp8 as omx
+        return torch.from_numpy(omx.dequantize_rowwise(codes.numpy(), scales.numpy()))
+
+
 def _combine(rows, pos, T, k):
     out = torch.zeros((T, rows.shape[1]), dtype=torch.float64)
     p = pos.view(T, k)
@@ -73,7 +87,7 @@ def _combine(rows, pos, T, k):
     return out
 
 
-def _worker(rank, world, port, out):
+def _worker(rank, world, port, out, wire="bf16"):
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
     from mxfp8_grouped_gemm_moe_b200.ep import ExpertParallelMLP
@@ -86,7 +100,8 @@ def _worker(rank, world, port, out):
         E_loc = cfg.E // world
         W1 = d["W1"].double().numpy()[rank * E_loc:(rank + 1) * E_loc]
         W2 = d["W2"].double().numpy()[rank * E_loc:(rank + 1) * E_loc]
-        layer = ExpertParallelMLP(Tl, cfg.k, cfg.E, cfg.H, cfg.F, local=_OracleLocal(W1, W2), combine=_combine)
+        layer = ExpertParallelMLP(Tl, cfg.k, cfg.E, cfg.H, cfg.F, local=_OracleLocal(W1, W2), combine=_combine,
+                                  wire=wire, codec=_OracleCodec() if wire == "mxfp8" else None)
         y = layer.forward(d["x"][sl], d["topk_idx"][sl], d["probs"][sl])
         dx, dW1, dW2, dprobs = layer.backward(d["dy"][sl])
         out[rank] = dict(y=y.numpy(), dx=dx.numpy(), dW1=dW1.numpy(), dW2=dW2.numpy(), dprobs=dprobs.numpy(),
@@ -104,6 +119,34 @@ def test_expert_parallel_exchange_equals_single_process_oracle():
     x, W1, W2, p = (d[n].double().numpy() for n in ("x", "W1", "W2", "probs"))
     y, s = moe.mlp_fwd(x, d["topk_idx"].numpy(), p, W1, W2)
     g = moe.mlp_bwd(d["dy"].double().numpy(), s, p, W1, W2)
+    Tl = cfg.T // world
+    for r in range(world):
+        o = out[r]
+        sl = slice(r * Tl, (r + 1) * Tl)
+        ex = o["experts"]
+        np.testing.assert_allclose(o["y"], y[sl], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(o["dx"], g["dx"][sl], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(o["dprobs"], g["dprobs"][sl], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(o["dW1"], g["dW1"][ex[0]:ex[-1] + 1], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(o["dW2"], g["dW2"][ex[0]:ex[-1] + 1], rtol=1e-10, atol=1e-12)
+
+
+def test_expert_parallel_mxfp8_wire_equals_oracle_on_rounded_inputs():
+    """With rows travelling as MXFP8 codes + scales, the layer computes what the single-process
+    oracle computes for x and dY rounded to their rowwise MXFP8 grid (the rowwise round trip
+    is lossless; the colwise copies come from the rounded rows)."""
+    from oracle import mxfp8 as omx
+    from oracle import moe
+    world, port = 2, _free_port()
+    out = mp.get_context("spawn").Manager().dict()
+    mp.start_processes(_worker, args=(world, port, out, "mxfp8"), nprocs=world, join=True, start_method="spawn")
+    cfg, d = _problem()
+    rnd = lambda a: omx.dequantize_rowwise(*omx.quantize_rowwise(a))  # noqa: E731
+    x, dy = rnd(d["x"].double().numpy()), rnd(d["dy"].double().numpy())
+    W1, W2, p = (d[n].double().numpy() for n in ("W1", "W2", "probs"))
+    assert not np.array_equal(x, d["x"].double().numpy())      # the wire does round
+    y, s = moe.mlp_fwd(x, d["topk_idx"].numpy(), p, W1, W2)
+    g = moe.mlp_bwd(dy, s, p, W1, W2)
     Tl = cfg.T // world
     for r in range(world):
         o = out[r]

@@ -157,3 +157,26 @@ def test_weights_buffer_layout(gpu_lib):
         qc2, sc2 = omx.quantize_colwise_t(f64(W2[e]))
         np.testing.assert_array_equal(u8(views[3].data)[e * F:(e + 1) * F], qc2)
         np.testing.assert_array_equal(u8(views[3].scale_plain())[e * F:(e + 1) * F], sc2)
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+def test_dequantize_rows_matches_oracle(gpu_lib, fmt):
+    """mxfp8_dequantize: every element equals the oracle's element(code) * 2^(scale - 127)
+    (exact in bf16 for these scales); re-quantising the dequantised rows gives back the same
+    codes and scales (the rowwise round trip is lossless, which expert parallelism relies on
+    when rows travel as MXFP8)."""
+    mx = gpu_lib
+    f = mx.FMT_E4M3 if fmt == "e4m3" else mx.FMT_E5M2
+    g = torch.Generator().manual_seed(91)
+    x = (torch.randn((300, 512), generator=g) * torch.exp2(torch.randint(-20, 20, (300, 1), generator=g).float()))
+    x = x.to(torch.bfloat16)
+    x[7] = 0                                    # an all-zero row (scale byte 0)
+    xr = torch.nn.functional.pad(x, (0, 0, 0, 20)).cuda()   # 320 rows (multiple of 32)
+    r, _ = mx.mxfp8_quantize(xr, colwise=False, layout=mx.SCALE_PLAIN, fmt=f)
+    y = mx.mxfp8_dequantize(r)
+    torch.cuda.synchronize()
+    want = omx.dequantize_rowwise(u8(r.data), u8(r.scale_plain()), fmt=fmt)
+    np.testing.assert_array_equal(f64(y.cpu()), want)
+    r2, _ = mx.mxfp8_quantize(y, colwise=False, layout=mx.SCALE_PLAIN, fmt=f)
+    np.testing.assert_array_equal(u8(r2.data), u8(r.data))
+    np.testing.assert_array_equal(u8(r2.scale_plain()), u8(r.scale_plain()))
