@@ -19,8 +19,8 @@
 //        a B tile crosses L2 -> SM once per pair instead of once per CTA; every TMA of
 //        both CTAs completes on the leader's stage barrier and the leader's commits
 //        release the stage in both CTAs (multicast commit; the loads themselves are
-//        never multicast). Ring of 34 KB stages: 5 for the plain-store and weight-
-//        gradient modes, 4 for the fused modes.
+//        never multicast). Ring of 34 KB stages: 5 for the plain-store, weight-gradient
+//        and fused-forward modes, 4 for the fused backward.
 //      PAIR = 1: one CTA per SM, tile 128 x 256, 3-stage ring of 50 KB.
 //    Each CTA ends a tile with the same 128 x 256 fp32 accumulator in its own TMEM, so
 //    the epilogues are shared by both variants;
@@ -84,21 +84,27 @@ constexpr int kPrefetchSteps = 8;     // K steps of the next tile pulled into L2
 
 // Per-variant layout. Plain-store and weight-gradient modes: 5-stage operand ring, one
 // 4 KB output box per epilogue warp for the TMA stores (the deeper ring measured faster
-// for the short-K weight-gradient tiles than a second box). Fused modes: 4 stages and
-// 8 KB per warp (two 4 KB transpose tiles, then the code blocks); 3 stages measured
-// clearly slower there.
-template <int PAIR, int MODE>
+// for the short-K weight-gradient tiles than a second box). Fused backward (and the bf16
+// and single-CTA fused kernels): 4 stages and 8 KB per warp (two 4 KB transpose tiles,
+// then the code blocks); 3 stages measured clearly slower there. Fused MXFP8 forward on
+// CTA pairs: 5 stages and 4 KB per warp (kDeep).
+template <int PAIR, int MODE, int ESZ = 1>
 struct Cfg {
   static constexpr bool kTmaStore = MODE == kModeStore || MODE == kModeWgrad;
+  // fused MXFP8 forward on CTA pairs: a 5th ring stage, paid for with 4 KB of staging per
+  // warp (the epilogue's G / U boxes and its two 32 x 32 transposes then go through it one
+  // after the other). Measured 1-5 % faster for the forward; the backward's epilogue, the
+  // busier one, was 2-4 % slower with sequential transposes, so it keeps 4 stages and 8 KB.
+  static constexpr bool kDeep = MODE == kModeSwigluFwd && PAIR == 2 && ESZ == 1;
   static constexpr bool kSplitRegs = !kTmaStore;            // 12 warps with the register split
   static constexpr int kThreads = kSplitRegs ? 384 : 352;
   static constexpr int kEpiWarp0 = kSplitRegs ? 4 : 3;      // first epilogue warp
   static constexpr int TM = 128 * PAIR;                        // output tile rows
-  static constexpr int STAGES = PAIR == 2 ? (kTmaStore ? 5 : 4) : 3;
+  static constexpr int STAGES = PAIR == 2 ? (kTmaStore || kDeep ? 5 : 4) : 3;
   static constexpr uint32_t kBBytes = (BN / PAIR) * BK;        // this CTA's B rows per stage
   static constexpr uint32_t kStageBytes = PAIR == 2 ? 34816 : 51200;
   static constexpr uint32_t kTxBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // per CTA
-  static constexpr uint32_t kStagingPerWarp = kTmaStore ? 4096 : 8192;
+  static constexpr uint32_t kStagingPerWarp = kTmaStore || kDeep ? 4096 : 8192;
   static constexpr uint32_t kOffStaging = STAGES * kStageBytes;
   static constexpr uint32_t kOffBars = kOffStaging + kEpiWarps * kStagingPerWarp;
   static constexpr uint32_t kOffSeg = kOffBars + 256;
@@ -276,6 +282,19 @@ __device__ __forceinline__ uint8_t quant32(const float (&v)[32], uint32_t (&q)[8
 // Two blocks go through the two 4 KB halves of the staging buffer together, with one
 // pair of warp syncs, so the two transposes and reductions interleave. Lane c gets the
 // 32 codes (and the scale byte) of column c of each block.
+// One 32 x 32 block into / out of a 4 KB staging buffer (same layout as above); the
+// caller places the warp syncs.
+__device__ __forceinline__ void colwise_put32(const float (&v)[32], float* stg, int lane) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int o = lane * 32 + ((j ^ (lane & 7)) << 2);
+    *reinterpret_cast<float4*>(stg + o) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  }
+}
+__device__ __forceinline__ void colwise_get32(const float* stg, int lane, float (&w)[32]) {
+#pragma unroll
+  for (int r = 0; r < 32; ++r) w[r] = stg[r * 32 + ((((lane >> 2) ^ (r & 7)) << 2) | (lane & 3))];
+}
 __device__ __forceinline__ void colwise_transpose2(const float (&v0)[32], const float (&v1)[32], float* stg, int lane,
                                                    float (&w0)[32], float (&w1)[32]) {
   float* stg1 = stg + 1024;
@@ -294,10 +313,30 @@ __device__ __forceinline__ void colwise_transpose2(const float (&v0)[32], const 
   }
   __syncwarp();  // the buffer may be refilled once every lane has read its columns
 }
-template <int FMT = MXMOE_FMT_E4M3>
+template <int FMT = MXMOE_FMT_E4M3, bool SEQ = false>
 __device__ __forceinline__ void colwise_codes2(const float (&v0)[32], const float (&v1)[32], float* stg, int lane,
                                                uint32_t (&q0)[8], uint32_t (&q1)[8], uint8_t& sb0, uint8_t& sb1,
                                                bool ceil_rule = false, float tm = 0.f) {
+  if (SEQ) {  // one 4 KB buffer: block 1 goes in as soon as block 0's columns are read out
+    float w[32];
+    colwise_put32(v0, stg, lane);
+    __syncwarp();
+    colwise_get32(stg, lane, w);
+    __syncwarp();
+    float* stg_a = stg;  // opaque copies of the buffer address (see below)
+    asm volatile("" : "+l"(stg_a));
+    colwise_put32(v1, stg_a, lane);  // v1 is dead from here on
+    sb0 = quant32<FMT>(w, q0, ceil_rule, tm);
+    __syncwarp();
+    // an opaque copy of the buffer address: the read addresses are recomputed rather than
+    // kept live through the first block's quantisation
+    float* stg_b = stg;
+    asm volatile("" : "+l"(stg_b));
+    colwise_get32(stg_b, lane, w);
+    __syncwarp();  // the buffer may be refilled once every lane has read its column
+    sb1 = quant32<FMT>(w, q1, ceil_rule, tm);
+    return;
+  }
   float w0[32], w1[32];
   colwise_transpose2(v0, v1, stg, lane, w0, w1);
   sb0 = quant32<FMT>(w0, q0, ceil_rule, tm);
@@ -452,7 +491,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
                   const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
                   const __grid_constant__ CUtensorMap tmE, const __grid_constant__ GemmArgs g) {
-  using C = Cfg<PAIR, MODE>;
+  using C = Cfg<PAIR, MODE, ESZ>;
   static_assert(ESZ == 1 || PAIR == 2, "bf16 operands run on CTA pairs");
   constexpr int STAGES = C::STAGES;
   constexpr uint32_t kTx = ESZ == 1 ? C::kTxBytes : kABytes + C::kBBytes;  // bytes per CTA per stage
@@ -840,7 +879,24 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
         uint8_t* stg8 = reinterpret_cast<uint8_t*>(stg);
         // G and U as bf16 for the backward: two 32-row x 128-byte boxes (128-byte swizzle);
         // skipped when the forward does not save them (the backward recomputes them)
-        if (g.gu != nullptr) {
+        if (g.gu != nullptr && C::kDeep) {  // 4 KB of staging: G, then U
+          staging_acquire(lane);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) out_box_put(stg8, lane, j, pack8_bf16(gr, 8 * j));
+          staging_publish();
+          if (lane == 0) {
+            ptx::tma_store_2d(&tmE, stg8, (int32_t)f0, (int32_t)mrow0);
+            ptx::bulk_commit_group();
+          }
+          staging_acquire(lane);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) out_box_put(stg8, lane, j, pack8_bf16(ur, 8 * j));
+          staging_publish();
+          if (lane == 0) {
+            ptx::tma_store_2d(&tmE, stg8, (int32_t)(F + f0), (int32_t)mrow0);
+            ptx::bulk_commit_group();
+          }
+        } else if (!C::kDeep && g.gu != nullptr) {
           staging_acquire(lane);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -895,7 +951,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
         const uint32_t zsf = (uint32_t)quant32(z0, r0, cr, tm, &zmax) | ((uint32_t)quant32(z1, r1, cr, tm, &zmax) << 8);
         if (tm != 0.f) record_amax(g.out_amax_rec, zmax, lane);
         staging_acquire(lane);
-        colwise_codes2(z0, z1, stg, lane, c0, c1, cs0, cs1, cr, tm);
+        colwise_codes2<MXMOE_FMT_E4M3, C::kDeep>(z0, z1, stg, lane, c0, c1, cs0, cs1, cr, tm);
         put_codes32(stg8, lane, r0);
         put_codes32(stg8 + 1024, lane, r1);
         put_codes32(stg8 + 2048, lane, c0);
@@ -1022,7 +1078,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, MODE>::kThreads, 1)
           sfg |= (uint32_t)quant32<OF>(vg, rg, cr, tm, &gmax) << (8 * c);
           sfu |= (uint32_t)quant32<OF>(vu, ru, cr, tm, &gmax) << (8 * c);
           staging_acquire(lane);
-          colwise_codes2<OF>(vg, vu, stg, lane, cg, cu, csg, csu, cr, tm);
+          colwise_codes2<OF, C::kDeep>(vg, vu, stg, lane, cg, cu, csg, csu, cr, tm);
           uint8_t* stg8 = reinterpret_cast<uint8_t*>(stg);
           put_codes32(stg8, lane, rg);
           put_codes32(stg8 + 1024, lane, ru);
@@ -1174,7 +1230,7 @@ struct GemmMaps {
 
 template <int MODE, int PAIR, int ESZ = 1, int OF = MXMOE_FMT_E4M3, bool PT = false>
 static cudaError_t launch_mode(const GemmMaps& m, const GemmArgs& g, int64_t tiles_ub, cudaStream_t st) {
-  constexpr uint32_t smem = Cfg<PAIR, MODE>::kSmemBytes;
+  constexpr uint32_t smem = Cfg<PAIR, MODE, ESZ>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(mxgemm_kernel<MODE, PAIR, ESZ, OF, PT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
