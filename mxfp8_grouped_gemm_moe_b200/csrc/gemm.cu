@@ -278,12 +278,9 @@ __device__ __forceinline__ uint8_t quant32(const float (&v)[32], uint32_t (&q)[8
 // transposed through 4 KB of the warp's staging buffer in one round: row r occupies words
 // [32r, 32r + 32) with its 16-byte chunk j stored at chunk j ^ (r % 8), so the row-wise
 // 16-byte writes and the column-wise 4-byte reads are both bank-conflict free; lane c
-// then holds column c whole.
-// Two blocks go through the two 4 KB halves of the staging buffer together, with one
-// pair of warp syncs, so the two transposes and reductions interleave. Lane c gets the
-// 32 codes (and the scale byte) of column c of each block.
-// One 32 x 32 block into / out of a 4 KB staging buffer (same layout as above); the
-// caller places the warp syncs.
+// then holds column c whole. Lane c gets the 32 codes (and the scale byte) of column c
+// of each block.
+// One 32 x 32 block into / out of a 4 KB staging buffer; the caller places the warp syncs.
 __device__ __forceinline__ void colwise_put32(const float (&v)[32], float* stg, int lane) {
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
@@ -295,6 +292,8 @@ __device__ __forceinline__ void colwise_get32(const float* stg, int lane, float 
 #pragma unroll
   for (int r = 0; r < 32; ++r) w[r] = stg[r * 32 + ((((lane >> 2) ^ (r & 7)) << 2) | (lane & 3))];
 }
+// Two blocks through the two 4 KB halves of an 8 KB staging buffer together, with one
+// pair of warp syncs, so the two transposes and reductions interleave.
 __device__ __forceinline__ void colwise_transpose2(const float (&v0)[32], const float (&v1)[32], float* stg, int lane,
                                                    float (&w0)[32], float (&w1)[32]) {
   float* stg1 = stg + 1024;
@@ -323,13 +322,13 @@ __device__ __forceinline__ void colwise_codes2(const float (&v0)[32], const floa
     __syncwarp();
     colwise_get32(stg, lane, w);
     __syncwarp();
-    float* stg_a = stg;  // opaque copies of the buffer address (see below)
+    // opaque copies of the buffer address: the second block's addresses are recomputed
+    // instead of being kept live (in registers) through the first block's quantisation
+    float* stg_a = stg;
     asm volatile("" : "+l"(stg_a));
     colwise_put32(v1, stg_a, lane);  // v1 is dead from here on
     sb0 = quant32<FMT>(w, q0, ceil_rule, tm);
     __syncwarp();
-    // an opaque copy of the buffer address: the read addresses are recomputed rather than
-    // kept live through the first block's quantisation
     float* stg_b = stg;
     asm volatile("" : "+l"(stg_b));
     colwise_get32(stg_b, lane, w);
