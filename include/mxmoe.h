@@ -230,7 +230,8 @@ mxmoe_status mxfp8_quantize(const void* src_dev, int32_t src_dtype, int64_t batc
                             const mxmoe_mxfp8* out_row, const mxmoe_mxfp8* out_colT, void* stream);
 /*
  * mxfp8_dequantize -- the inverse of the rowwise quantisation, for MXFP8 rows that travel
- * between devices (expert parallelism sends the routed rows as codes + scales): every
+ * between devices ("MoE-Training für biologische Grundmodelle optimieren", expert-parallel
+ * passage: the experts spread over GPUs; the routed rows can travel as codes + scales): every
  * element becomes element(code) * 2^(scale - 127), rounded once to bf16 (exact whenever
  * the block's scale is at least 2^-124, i.e. for every block quantised from bf16 values
  * of magnitude above about 2^-115).
