@@ -11,8 +11,10 @@
 //
 // One CTA quantises a 128 x 128 tile staged in shared memory: rowwise blocks (32
 // consecutive columns of a row) and colwise blocks (32 consecutive rows of a column,
-// written transposed) come from the same HBM read. Loads and stores are 16-byte
-// vectors; a warp's rowwise / colwise stores cover whole 32-byte sectors.
+// written transposed) come from the same HBM read. bf16 rows are read 32 bytes per load,
+// and the 32 codes of a block leave in one 256-bit store (a whole 32-byte sector) when the
+// destination is 32-byte aligned: half as many load and store requests as 16-byte vectors,
+// and no half-sector writes.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -27,6 +29,18 @@ namespace mxmoe {
 
 constexpr int kQTile = 128;
 constexpr int kQThreads = 256;
+// 32 code bytes at p: one 256-bit store when p is 32-byte aligned, else two 16-byte stores
+__device__ __forceinline__ void st_codes32(uint8_t* p, const uint32_t (&q)[8]) {
+  if ((reinterpret_cast<uintptr_t>(p) & 31) == 0) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(q[0]), "r"(q[1]),
+                 "r"(q[2]), "r"(q[3]), "r"(q[4]), "r"(q[5]), "r"(q[6]), "r"(q[7])
+                 : "memory");
+  } else {
+    uint4* d = reinterpret_cast<uint4*>(p);
+    d[0] = make_uint4(q[0], q[1], q[2], q[3]);
+    d[1] = make_uint4(q[4], q[5], q[6], q[7]);
+  }
+}
 
 template <typename T>
 struct SrcTraits;
@@ -202,11 +216,15 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
   using Tr = SrcTraits<T>;
   extern __shared__ __align__(16) uint8_t q_smem_raw[];
   T* tile = reinterpret_cast<T*>(q_smem_raw);
+  // the tile's scale bytes, four per row (rowwise) / per transposed row (colwise)
+  __shared__ uint32_t s_rsc[kQTile], s_csc[kQTile];
 
   const int64_t c0 = (int64_t)blockIdx.x * kQTile;
   const int64_t r0 = (int64_t)blockIdx.y * kQTile;
   const int64_t b = blockIdx.z;
-  constexpr int VPR = kQTile / Tr::kVec;        // vectors per tile row
+  // elements per load: 32 bytes for bf16 (one 256-bit load), 16 bytes for fp32
+  constexpr int LV = sizeof(T) == 2 ? 16 : Tr::kVec;
+  constexpr int VPR = kQTile / LV;              // vectors per tile row
   constexpr int NL = kQTile * VPR / kQThreads;  // vectors per thread
   constexpr int RSTEP = kQThreads / VPR;        // tile rows between a thread's vectors
   const int row_t = threadIdx.x / VPR, cv = threadIdx.x % VPR;
@@ -228,9 +246,9 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
   const float tm = a.tensor_amax ? tensor_multiplier(a.tensor_amax[a.tensor_per_batch ? b : 0]) : 0.f;
 
   // ---- load the tile (gathered rows, zero outside the matrix / for pad rows); all of a
-  // thread's 16-byte loads are issued before any use
+  // thread's loads (32 bytes per bf16 vector, 16 per fp32 vector) are issued before any use
   {
-    const int64_t col = c0 + (int64_t)cv * Tr::kVec;
+    const int64_t col = c0 + (int64_t)cv * LV;
     int64_t srow[NL];
 #pragma unroll
     for (int k = 0; k < NL; ++k) {
@@ -240,14 +258,36 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
       // checked build: a gathered row outside the source matrix reads as a zero row
       if (a.gather && srow[k] >= 0 && !check_index(srow[k], a.rows, 67)) srow[k] = -1;
     }
-    uint4 buf[NL];
+    constexpr int HV = LV / Tr::kVec;  // 16-byte halves per load
+    uint4 buf[NL][HV];
+    // a 256-bit load needs a 32-byte aligned address: rows are 64-byte multiples (cols % 32
+    // == 0) and vectors start at 32-byte offsets, so the base pointer decides
+    const bool v8 = (reinterpret_cast<uintptr_t>(src) & 31) == 0;
+#pragma unroll
+    for (int k = 0; k < NL; ++k) {
+      const uint4* p = reinterpret_cast<const uint4*>(src + srow[k] * a.cols + col);
+      if (srow[k] < 0) {
+#pragma unroll
+        for (int hv = 0; hv < HV; ++hv) buf[k][hv] = make_uint4(0, 0, 0, 0);
+      } else if constexpr (HV == 2) {
+        if (v8) {
+          asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                       : "=r"(buf[k][0].x), "=r"(buf[k][0].y), "=r"(buf[k][0].z), "=r"(buf[k][0].w),
+                         "=r"(buf[k][1].x), "=r"(buf[k][1].y), "=r"(buf[k][1].z), "=r"(buf[k][1].w)
+                       : "l"(p));
+        } else {
+          buf[k][0] = __ldg(p);
+          buf[k][1] = __ldg(p + 1);
+        }
+      } else {
+        buf[k][0] = __ldg(p);
+      }
+    }
 #pragma unroll
     for (int k = 0; k < NL; ++k)
-      buf[k] = srow[k] >= 0 ? __ldg(reinterpret_cast<const uint4*>(src + srow[k] * a.cols + col))
-                            : make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int k = 0; k < NL; ++k)
-      *reinterpret_cast<uint4*>(tile + tile_off<T>(row_t + k * RSTEP, cv * Tr::kVec)) = buf[k];
+      for (int hv = 0; hv < HV; ++hv)
+        *reinterpret_cast<uint4*>(tile + tile_off<T>(row_t + k * RSTEP, cv * LV + hv * Tr::kVec)) = buf[k][hv];
   }
   __syncthreads();
 
@@ -268,10 +308,8 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
         drow = (rr >> 6) * 128 + hf * 64 + (rr & 63);
       }
       const int64_t grow = b * a.out_rows + drow;
-      uint4* dst = reinterpret_cast<uint4*>(a.row_data + grow * a.cols + col);
-      dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
-      dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
-      a.row_sf[sf_offset(a.row_layout, a.batch * a.out_rows, a.cols, grow, col / 32)] = sb;
+      st_codes32(a.row_data + grow * a.cols + col, q);
+      reinterpret_cast<uint8_t*>(s_rsc)[row * 4 + blk] = sb;
     }
   }
   // ---- colwise: item = (pair of adjacent columns, 32-row block), one per thread; a warp
@@ -286,14 +324,56 @@ __global__ void __launch_bounds__(kQThreads, sizeof(T) == 2 ? 4 : 2) mxfp8_quant
       quant_col_pair<FMT>(tile + tile_off<T>(32 * rb, 2 * pcol), 4 * Tr::kBS, q0, q1, s0, s1, a.scale_rule != 0,
                           tm);
       const int64_t grow = b * a.cols + col;  // row of the transposed matrix
-      uint4* d0 = reinterpret_cast<uint4*>(a.col_data + grow * a.out_rows + orow);
-      uint4* d1 = reinterpret_cast<uint4*>(a.col_data + (grow + 1) * a.out_rows + orow);
-      d0[0] = make_uint4(q0[0], q0[1], q0[2], q0[3]);
-      d0[1] = make_uint4(q0[4], q0[5], q0[6], q0[7]);
-      d1[0] = make_uint4(q1[0], q1[1], q1[2], q1[3]);
-      d1[1] = make_uint4(q1[4], q1[5], q1[6], q1[7]);
-      a.col_sf[sf_offset(a.col_layout, a.batch * a.cols, a.out_rows, grow, orow / 32)] = s0;
-      a.col_sf[sf_offset(a.col_layout, a.batch * a.cols, a.out_rows, grow + 1, orow / 32)] = s1;
+      st_codes32(a.col_data + grow * a.out_rows + orow, q0);
+      st_codes32(a.col_data + (grow + 1) * a.out_rows + orow, q1);
+      reinterpret_cast<uint8_t*>(s_csc)[(2 * pcol) * 4 + rb] = s0;
+      reinterpret_cast<uint8_t*>(s_csc)[(2 * pcol + 1) * 4 + rb] = s1;
+    }
+  }
+  __syncthreads();
+  // ---- scale bytes: a row's four blocks of this tile are adjacent in both scale layouts
+  // (one 32-bit store); threads 0-127 store the rowwise scales, 128-255 the colwise ones.
+  // In the MMA layout the tile's 128 x 4 bytes of a copy form one 512-byte chunk, and
+  // thread t stores its word t (row (t % 4) * 32 + t / 4), so a warp writes 128
+  // consecutive bytes.
+  {
+    const bool rowwise = threadIdx.x < kQTile;
+    const int t = threadIdx.x & (kQTile - 1);
+    const int32_t layout = rowwise ? a.row_layout : a.col_layout;
+    const int r = layout == MXMOE_SCALE_MMA ? (t & 3) * 32 + (t >> 2) : t;
+    uint8_t* sf = rowwise ? a.row_sf : a.col_sf;
+    bool ok;
+    int64_t grow, kb0, srows, scols;
+    int nb;
+    if (rowwise) {
+      const int64_t orow = r0 + r;
+      int64_t drow = orow;
+      if (a.row_ilv > 0) {  // gate / up interleave of the fc1 operand
+        const int64_t hf = orow >= a.row_ilv, rr = orow - hf * a.row_ilv;
+        drow = (rr >> 6) * 128 + hf * 64 + (rr & 63);
+      }
+      ok = a.row_data != nullptr && orow < nvalid;
+      grow = b * a.out_rows + drow;
+      kb0 = c0 / 32;
+      nb = (int)((a.cols - c0) / 32 < 4 ? (a.cols - c0) / 32 : 4);
+      srows = a.batch * a.out_rows;
+      scols = a.cols;
+    } else {
+      ok = a.col_data != nullptr && c0 + r < a.cols;
+      grow = b * a.cols + c0 + r;
+      kb0 = r0 / 32;
+      nb = (int)((nvalid - r0 + 31) / 32 < 4 ? (nvalid - r0 + 31) / 32 : 4);
+      srows = a.batch * a.cols;
+      scols = a.out_rows;
+    }
+    if (ok) {
+      const uint32_t w = rowwise ? s_rsc[r] : s_csc[r];
+      uint8_t* p = sf + sf_offset(layout, srows, scols, grow, kb0);
+      if (nb == 4 && (reinterpret_cast<uintptr_t>(p) & 3) == 0) {
+        *reinterpret_cast<uint32_t*>(p) = w;
+      } else {
+        for (int j = 0; j < nb; ++j) sf[sf_offset(layout, srows, scols, grow, kb0 + j)] = (uint8_t)(w >> (8 * j));
+      }
     }
   }
 }
