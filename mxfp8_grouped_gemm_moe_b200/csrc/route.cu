@@ -136,29 +136,58 @@ __global__ void __launch_bounds__(kRouteTokensPerBlock) route_scatter_kernel(
 }
 
 // y[t] = sum_j y_perm[row_of_slot[t, j]] (fp32 in slot order, bf16 out). One block per
-// token, 16-byte vectors.
+// token; each thread issues the loads of all k routed rows of its vector before the first
+// sum (KMAX >= k slots, unrouted ones skipped), VW 16-byte words per vector: 2 (256-bit
+// loads and stores) when both buffers are 32-byte aligned, else 1.
+template <int KMAX, int VW>
 __global__ void __launch_bounds__(256) unpermute_kernel(const uint4* __restrict__ yp, const int32_t* __restrict__ ros,
                                                         int T, int k, int H, uint4* __restrict__ y) {
   const int t = blockIdx.x;
-  const int nvec = H / 8;
-  int32_t rows[kMaxTopK];
-  for (int j = 0; j < k; ++j) rows[j] = ros[(int64_t)t * k + j];
+  const int nvec = H / (8 * VW);
+  int32_t rows[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) rows[j] = j < k ? __ldg(ros + (int64_t)t * k + j) : -1;
   for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int j = 0; j < k; ++j) {
+    uint4 q[KMAX][VW];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
       if (rows[j] < 0) continue;
-      const uint4 q = __ldg(&yp[(int64_t)rows[j] * nvec + v]);
-      acc[0] += bf16_lo(q.x); acc[1] += bf16_hi(q.x);
-      acc[2] += bf16_lo(q.y); acc[3] += bf16_hi(q.y);
-      acc[4] += bf16_lo(q.z); acc[5] += bf16_hi(q.z);
-      acc[6] += bf16_lo(q.w); acc[7] += bf16_hi(q.w);
+      const uint4* p = yp + ((int64_t)rows[j] * nvec + v) * VW;
+      if constexpr (VW == 2) {
+        asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                     : "=r"(q[j][0].x), "=r"(q[j][0].y), "=r"(q[j][0].z), "=r"(q[j][0].w), "=r"(q[j][1].x),
+                       "=r"(q[j][1].y), "=r"(q[j][1].z), "=r"(q[j][1].w)
+                     : "l"(p));
+      } else {
+        q[j][0] = __ldg(p);
+      }
     }
-    uint4 o;
-    o.x = pack_bf16x2(acc[0], acc[1]);
-    o.y = pack_bf16x2(acc[2], acc[3]);
-    o.z = pack_bf16x2(acc[4], acc[5]);
-    o.w = pack_bf16x2(acc[6], acc[7]);
-    y[(int64_t)t * nvec + v] = o;
+    float acc[8 * VW];
+#pragma unroll
+    for (int i = 0; i < 8 * VW; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (rows[j] < 0) continue;
+#pragma unroll
+      for (int w = 0; w < VW; ++w) {
+        float* a = acc + 8 * w;
+        a[0] += bf16_lo(q[j][w].x); a[1] += bf16_hi(q[j][w].x);
+        a[2] += bf16_lo(q[j][w].y); a[3] += bf16_hi(q[j][w].y);
+        a[4] += bf16_lo(q[j][w].z); a[5] += bf16_hi(q[j][w].z);
+        a[6] += bf16_lo(q[j][w].w); a[7] += bf16_hi(q[j][w].w);
+      }
+    }
+    uint32_t o[4 * VW];
+#pragma unroll
+    for (int i = 0; i < 4 * VW; ++i) o[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
+    uint4* d = y + ((int64_t)t * nvec + v) * VW;
+    if constexpr (VW == 2) {
+      asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(d), "r"(o[0]), "r"(o[1]),
+                   "r"(o[2]), "r"(o[3]), "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
+                   : "memory");
+    } else {
+      *d = make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
 }
 
@@ -200,9 +229,21 @@ cudaError_t launch_route(const int32_t* idx, const float* probs, int T, int k, i
 
 cudaError_t launch_unpermute(const void* yp, const int32_t* ros, int T, int k, int H, void* y, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  const int threads = std::min(256, std::max(32, (H / 8 + 31) / 32 * 32));
-  unpermute_kernel<<<T, threads, 0, st>>>(reinterpret_cast<const uint4*>(yp), ros, T, k, H,
-                                          reinterpret_cast<uint4*>(y));
+  const bool v32 = H % 16 == 0 && (reinterpret_cast<uintptr_t>(yp) & 31) == 0 && (reinterpret_cast<uintptr_t>(y) & 31) == 0;
+  const int nvec = H / (v32 ? 16 : 8);
+  const int threads = std::min(256, std::max(32, (nvec + 31) / 32 * 32));
+  const uint4* src = reinterpret_cast<const uint4*>(yp);
+  uint4* dst = reinterpret_cast<uint4*>(y);
+#define MXMOE_UNPERMUTE(KM)                                                               \
+  do {                                                                                    \
+    if (v32) unpermute_kernel<KM, 2><<<T, threads, 0, st>>>(src, ros, T, k, H, dst);      \
+    else unpermute_kernel<KM, 1><<<T, threads, 0, st>>>(src, ros, T, k, H, dst);          \
+  } while (0)
+  if (k <= 1) MXMOE_UNPERMUTE(1);
+  else if (k <= 2) MXMOE_UNPERMUTE(2);
+  else if (k <= 4) MXMOE_UNPERMUTE(4);
+  else MXMOE_UNPERMUTE(kMaxTopK);
+#undef MXMOE_UNPERMUTE
   ++g_launch_count;
   return cudaGetLastError();
 }
