@@ -91,6 +91,43 @@ def test_quantize_untiled_shapes(gpu_lib, shape):
     np.testing.assert_array_equal(u8(c.scale_plain()), sc)
 
 
+def test_gathered_quantize_16_byte_aligned_buffers(gpu_lib):
+    """The per-tile kernel's 32-byte loads and stores need 32-byte aligned rows; a source
+    and outputs that are only 16-byte aligned take the 16-byte loads and the two-store
+    path, with the same bytes as the oracle (gathered rows, zero rows for index -1)."""
+    import ctypes
+    lib = gpu_lib.load()
+    R, C, OR = 200, 160, 224
+    x = wl.random_matrix(R, C, seed=77, dtype=torch.float32).to(torch.bfloat16)
+    g = torch.Generator().manual_seed(5)
+    gather = torch.randint(-1, R, (OR,), generator=g, dtype=torch.int32)
+    sbuf = torch.zeros(R * C + 8, dtype=torch.bfloat16, device="cuda")
+    src = sbuf[8:].view(R, C)                         # 16 bytes into the buffer
+    src.copy_(x.cuda())
+    rbuf = torch.zeros(OR * C + 16, dtype=torch.uint8, device="cuda")
+    cbuf = torch.zeros(C * OR + 16, dtype=torch.uint8, device="cuda")
+    r = gpu_lib.MXFP8(rbuf[16:].view(OR, C), torch.zeros(OR * C // 32, dtype=torch.uint8, device="cuda"),
+                      gpu_lib.SCALE_PLAIN)
+    c = gpu_lib.MXFP8(cbuf[16:].view(C, OR), torch.zeros(C * OR // 32, dtype=torch.uint8, device="cuda"),
+                      gpu_lib.SCALE_PLAIN)
+    assert src.data_ptr() % 32 == 16 and r.data.data_ptr() % 32 == 16 and c.data.data_ptr() % 32 == 16
+    gdev = gather.cuda()
+    rs, cs = r.as_struct(), c.as_struct()
+    st = lib.mxfp8_quantize(gpu_lib._ptr(src), gpu_lib.DTYPE_BF16, 1, R, C, gpu_lib._ptr(gdev), None, OR,
+                            ctypes.byref(rs), ctypes.byref(cs), gpu_lib._stream())
+    assert st == 0, gpu_lib.status_string(st)
+    torch.cuda.synchronize()
+    xp = np.zeros((OR, C))
+    live = gather.numpy() >= 0
+    xp[live] = f64(x)[gather.numpy()[live]]
+    qr, sr = omx.quantize_rowwise(xp)
+    qc, sc = omx.quantize_colwise_t(xp)
+    np.testing.assert_array_equal(u8(r.data), qr)
+    np.testing.assert_array_equal(u8(r.scale_plain()), sr)
+    np.testing.assert_array_equal(u8(c.data), qc)
+    np.testing.assert_array_equal(u8(c.scale_plain()), sc)
+
+
 def test_quantize_batched_weights(gpu_lib):
     E, N, K = 3, 256, 384
     W = wl.random_matrix(N, K, seed=9, std=0.02, batch=E)

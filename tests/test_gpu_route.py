@@ -81,8 +81,12 @@ def test_permute_invalid_ids_flagged(gpu_lib):
     assert gpu_lib.mxmoe_get_device_status()[0] == 0
 
 
-@pytest.mark.parametrize("k,H", [(2, 256), (8, 2048), (1, 1024)])
-def test_unpermute_matches_oracle(gpu_lib, k, H):
+@pytest.mark.parametrize("k,H,shift", [(2, 256, 0), (8, 2048, 0), (1, 1024, 0), (4, 264, 0), (3, 512, 8),
+                                         (2, 1024, 8)])
+def test_unpermute_matches_oracle(gpu_lib, k, H, shift):
+    """Combine of the routed rows. H % 16 != 0, or a source only 16-byte aligned (`shift`
+    bf16 elements into an aligned buffer), takes the 16-byte path; k = 3, 4 the four-slot
+    variant."""
     E = 8
     T = 500
     cfg = wl.custom(T=T, H=H, F=256, E=E, k=k, seed=40 + k)
@@ -90,7 +94,10 @@ def test_unpermute_matches_oracle(gpu_lib, k, H):
     out = gpu_lib.moe_permute(idx.cuda(), probs.cuda(), E)
     cap = gpu_lib.mxmoe_rows_capacity(T, k, E)
     yp = wl.random_matrix(cap, H, seed=3)
-    y = gpu_lib.moe_unpermute(yp.cuda(), out["row_of_slot"])
+    buf = torch.zeros(cap * H + shift, dtype=torch.bfloat16, device="cuda")
+    yp_dev = buf[shift:].view(cap, H)
+    yp_dev.copy_(yp.cuda())
+    y = gpu_lib.moe_unpermute(yp_dev, out["row_of_slot"])
     torch.cuda.synchronize()
     r = omoe.route(idx.numpy(), E, align=SEG_ALIGN)
     want = omoe.unpermute_sum(f64(yp), r["row_of_slot"])
