@@ -605,7 +605,9 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
                 for _ in range(2)]
 
         def run_e2e(nsteps):
-            loaded, consumed, read_done = [None, None], [None, None], [None, None]
+            # the forward's inputs (x, routing) and the backward's (dY) complete separately,
+            # so a step's forward starts while its dY is still on the way
+            loaded_fwd, loaded, consumed, read_done = [None, None], [None, None], [None, None], [None, None]
 
             def load(i):
                 b = bufs[i % 2]
@@ -615,6 +617,8 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
                     b["x"].copy_(x_h, non_blocking=True)
                     b["idx"].copy_(idx_h2, non_blocking=True)
                     b["probs"].copy_(probs_h2, non_blocking=True)
+                    loaded_fwd[i % 2] = ev()
+                    loaded_fwd[i % 2].record(cs)
                     b["dy"].copy_(dy_h, non_blocking=True)
                     loaded[i % 2] = ev()
                     loaded[i % 2].record(cs)
@@ -622,7 +626,7 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
             load(0)
             for i in range(nsteps):
                 b, o = bufs[i % 2], outs[i % 2]
-                stream.wait_event(loaded[i % 2])
+                stream.wait_event(loaded_fwd[i % 2])
                 if read_done[i % 2] is not None:
                     stream.wait_event(read_done[i % 2])
                 if i + 1 < nsteps:
@@ -631,6 +635,7 @@ def run_gpu(args, cfg, dist, rank, world, local_rank):
                 layer.forward(b["x"], b["idx"], b["probs"], o["y"])
                 fwd_done = ev()
                 fwd_done.record(stream)
+                stream.wait_event(loaded[i % 2])
                 layer.backward(b["dy"], o["dx"], dW1, dW2, o["dprobs"])
                 bwd_done = ev()
                 bwd_done.record(stream)
