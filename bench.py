@@ -62,6 +62,9 @@ def parse_args():
                    help="skip the comparison timings (the bf16 layer's step, the alternative recipes)")
     p.add_argument("--no-workloads", action="store_true",
                    help="skip the other workloads' steps (Mixtral with Zipf routing, genomics)")
+    p.add_argument("--stage", choices=["all", "permute_quantize"], default="all",
+                   help="permute_quantize: time only the routing and the gathered permute + quantise of x "
+                        "(a profiling case that holds well under 1 GB); prints its own JSON line")
     return p.parse_args()
 
 
@@ -526,6 +529,56 @@ def time_workload(name, dev, steps, warmup, peaks):
     return out
 
 
+def run_permute_quantize(args, cfg):
+    """Profiling mode: the routing, then --warmup untimed and --steps timed calls of the
+    gathered permute + quantise of x (rowwise and colwise MXFP8, MMA scale layout) into
+    preallocated outputs through the C ABI, each timed call after an L2 flush."""
+    import ctypes
+    import statistics
+
+    import torch
+
+    import moe_workloads as wl
+    import mxfp8_grouped_gemm_moe_b200 as mx
+
+    lib = mx.load()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    idx_h, probs_h = wl.make_routing(cfg)
+    g = torch.Generator(device=dev)
+    g.manual_seed(cfg.seed)
+    x = torch.randn((cfg.T, cfg.H), generator=g, device=dev).to(torch.bfloat16)
+    r = mx.moe_permute(idx_h.to(dev), probs_h.to(dev), cfg.E)
+    cap = r["token_of_row"].numel()
+    nrows = r["seg_off"][cfg.E:]
+    row = mx.MXFP8.empty(cap, cfg.H, mx.SCALE_MMA, dev)
+    col = mx.MXFP8.empty(cfg.H, cap, mx.SCALE_MMA, dev)
+    rs, cs = row.as_struct(), col.as_struct()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def call():
+        st = lib.mxfp8_quantize(mx._ptr(x), mx.DTYPE_BF16, 1, cfg.T, cfg.H, mx._ptr(r["token_of_row"]),
+                                mx._ptr(nrows), cap, ctypes.byref(rs), ctypes.byref(cs), mx._stream())
+        mx._check("mxfp8_quantize", st)
+
+    for _ in range(args.warmup):
+        call()
+    ev = []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        ev.append((e0, e1))
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    rows = int(nrows.item())
+    alg = cfg.T * cfg.H * 2 + 2 * rows * cfg.H * (1 + 1 / 32)
+    print(json.dumps({"stage": "permute_quantize", "workload": cfg.name, "steps": args.steps, "ms": ms,
+                      "gbs": alg / ms / 1e6, "algorithmic_bytes": alg, "rows": rows, "capacity": cap}), flush=True)
+
+
 def run_gpu(args, cfg, dist, rank, world, local_rank):
     import torch
 
@@ -777,6 +830,10 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, cfg, dist, rank, world)
+            return
+        if args.stage == "permute_quantize":
+            if rank == 0:
+                run_permute_quantize(args, cfg)
             return
         line = run_gpu(args, cfg, dist, rank, world, local_rank)
         if rank == 0:
