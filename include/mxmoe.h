@@ -199,7 +199,9 @@ mxmoe_status moe_permute_noalloc(const int32_t* topk_idx_dev, const float* probs
  * moe_unpermute -- returns routed rows to token order and sums the k copies of each
  * token: y[t] = sum_{j<k} y_perm[row_of_slot[t, j]], accumulated in fp32 in slot order
  * and rounded once to bf16 (the pages are silent on the combine; this is the plain
- * reading). y_perm_dev bf16 [rows, H]; y_dev bf16 [T, H]. H % 8 == 0.
+ * reading). y_perm_dev bf16 [rows, H]; y_dev bf16 [T, H]. H % 8 == 0; both pointers
+ * 16-byte aligned (MXMOE_ERR_INVALID_ARG otherwise). When both are 32-byte aligned and
+ * H % 16 == 0 the kernel moves 32 bytes per access (same results either way).
  */
 mxmoe_status moe_unpermute(const void* y_perm_dev, const int32_t* row_of_slot_dev, int32_t T, int32_t k,
                            int32_t H, void* y_dev, void* stream);
