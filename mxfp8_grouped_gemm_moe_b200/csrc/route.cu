@@ -191,16 +191,25 @@ __global__ void __launch_bounds__(256) unpermute_kernel(const uint4* __restrict_
   }
 }
 
-// dprobs[t, j] = sum over p of part[row, p] (fixed order: deterministic), row = row_of_slot[t, j].
-__global__ void dprob_reduce_kernel(const float* __restrict__ part, int nparts, const int32_t* __restrict__ ros,
-                                    int64_t n, float* __restrict__ dprobs) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  const int32_t row = ros[i];
+// dprobs[t, j] = sum over p of part[row, p], row = row_of_slot[t, j]. G lanes per (t, j):
+// lane l of the group adds partials l, l + G, ... in order (coalesced reads), then the G
+// lane sums are combined by a fixed butterfly, so the result is deterministic. Every lane
+// of a warp takes part in the shuffles; groups past n add nothing and store nothing.
+template <int G>
+__global__ void __launch_bounds__(256) dprob_reduce_kernel(const float* __restrict__ part, int nparts,
+                                                           const int32_t* __restrict__ ros, int64_t n,
+                                                           float* __restrict__ dprobs) {
+  const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
+  const int sub = threadIdx.x & (G - 1);
   float s = 0.f;
-  if (row >= 0)
-    for (int p = 0; p < nparts; ++p) s += part[(int64_t)row * nparts + p];
-  dprobs[i] = s;
+  if (i < n) {
+    const int32_t row = ros[i];
+    if (row >= 0)
+      for (int p = sub; p < nparts; p += G) s += part[(int64_t)row * nparts + p];
+  }
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (i < n && sub == 0) dprobs[i] = s;
 }
 
 // ----------------------------------------------------------------------------- launchers
@@ -251,7 +260,11 @@ cudaError_t launch_unpermute(const void* yp, const int32_t* ros, int T, int k, i
 cudaError_t launch_dprob_reduce(const float* part, int nparts, const int32_t* ros, int64_t n, float* dprobs,
                                 cudaStream_t st) {
   if (n == 0) return cudaSuccess;
-  dprob_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(part, nparts, ros, n, dprobs);
+  // a warp per output for long partial rows, a quarter warp for short ones
+  if (nparts >= 96)
+    dprob_reduce_kernel<32><<<(unsigned)((n * 32 + 255) / 256), 256, 0, st>>>(part, nparts, ros, n, dprobs);
+  else
+    dprob_reduce_kernel<8><<<(unsigned)((n * 8 + 255) / 256), 256, 0, st>>>(part, nparts, ros, n, dprobs);
   ++g_launch_count;
   return cudaGetLastError();
 }
